@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Benchmark: causal attention forward + backward (bf16) TFLOP/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one attn_fwd + one attn_bwd over the whole workload (default: the
+long-context window B=1, H=16, T=8192, D=128 with RoPE), inputs resident in
+HBM. Each timed step is bracketed by CUDA events on the launching stream; L2
+is flushed (a 256 MiB write) between steps, outside the events. FLOPs follow
+the nominal convention 4*B*H*T^2*D/2 forward and 2.5x that backward
+(7*B*H*T^2*D per step; for packed documents the within-document figure is
+reported beside it). With N > 1 (torchrun, one process per GPU) every rank
+runs its own replica of the workload (weak scaling: attention has no
+exchange step), the step time is the max over ranks, and value is the
+aggregate. Rank 0 prints one JSON line.
+
+--impl reference times the float64 CPU oracle on the host cores instead
+(rank 0 only), each step one (batch, head) slice of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "causal attention fwd+bwd TFLOP/s (bf16) and % of B200 dense BF16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# FP32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flop x 1.965 GHz.
+FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long_context_8k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# FLOP accounting
+# ---------------------------------------------------------------------------
+
+def causal_unit(w) -> float:
+    """One causal matmul over the workload: H*D*sum(L^2) flops (2 per MAC
+    over the L^2/2 allowed pairs of each document)."""
+    return w.algorithmic_flops() / 7.0
+
+
+def kernel_algorithmic(name: str, w, kinds_seen) -> tuple:
+    """(bound, algorithmic amount per launch, unit) for one kernel kind."""
+    U = causal_unit(w)
+    elem = 2 if w.dtype == "bf16" else 4
+    N = w.B * w.H * w.T * w.D
+    R = w.B * w.H * w.T
+    if name == "fwd":
+        return "tensor", 2 * U, "flop"
+    if name == "dkdv":
+        return "tensor", (4 if "dq" in kinds_seen else 5) * U, "flop"
+    if name == "dq":
+        return "tensor", 1 * U, "flop"
+    if name == "delta":
+        return "hbm", 2 * N * elem + 4 * R, "byte"
+    if name == "rope_prep":
+        return "hbm", 4 * N * elem, "byte"
+    if name == "dq_finalize":
+        return "hbm", N * 4 + N * elem, "byte"
+    return "hbm", 0, "byte"
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling (NVML, read-only) during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = [(0x4, "sw_power_cap"), (0x8, "hw_slowdown"), (0x20, "sw_thermal_slowdown"),
+               (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"),
+               (0x2, "applications_clocks_setting"), (0x1, "gpu_idle")]
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thr = None
+        self.error = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        except Exception as e:  # NVML missing: report no clocks rather than guess
+            self.error = repr(e)
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h) \
+                    if hasattr(nv, "nvmlDeviceGetCurrentClocksEventReasons") \
+                    else nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                for bit, name in self.REASONS:
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception as e:
+                self.error = repr(e)
+                break
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0, "error": self.error}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the baseline, and the reference arm)
+# ---------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 1) for p in threadpool_info() if p.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_slice_seconds(w, heads):
+    from oracle import attention_backward, attention_forward
+
+    t0 = time.perf_counter()
+    attention_forward(w.q, w.k, w.v, w.rope_cos, w.rope_sin, w.cu_seqlens, w.scale, heads=heads)
+    attention_backward(w.q, w.k, w.v, w.do, w.rope_cos, w.rope_sin, w.cu_seqlens, w.scale,
+                       heads=heads)
+    return time.perf_counter() - t0
+
+
+def slice_flops(w, heads) -> float:
+    """Nominal-convention flops of the given (b, h) slices (within-document for
+    packed rows): 7 * D * sum over their documents of L^2."""
+    import numpy as np
+    total = 0.0
+    for b, _h in heads:
+        if w.cu_seqlens is None:
+            total += 7.0 * w.D * w.T * w.T
+        else:
+            cu = w.cu_seqlens.astype(np.int64)
+            L = np.diff(cu)[(cu[:-1] >= b * w.T) & (cu[:-1] < (b + 1) * w.T)].astype(np.float64)
+            total += 7.0 * w.D * float((L * L).sum())
+    return total
+
+
+def sample_description(w, heads):
+    return (f"fwd+bwd of {len(heads)} (batch, head) slice(s) {heads} of {w.cfg.name} "
+            f"(T={w.T}, D={w.D}), float64 NumPy oracle")
+
+
+# ---------------------------------------------------------------------------
+# Arms
+# ---------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        if world == 1 and n_gpus > 1:
+            raise SystemExit("--gpus N > 1 needs torchrun with N processes")
+    return world, rank, local
+
+
+def run_reference(args):
+    import torch
+    from workloads import config_by_name, make_workload
+
+    world, rank, _ = dist_setup(args.gpus)
+    if rank != 0:
+        return 0
+    w = make_workload(config_by_name(args.workload))
+    heads = [(0, 0)]
+    for _ in range(args.warmup):
+        oracle_slice_seconds(w, heads)
+    secs = [oracle_slice_seconds(w, heads) for _ in range(args.steps)]
+    per_step = sum(secs) / len(secs)
+    value = slice_flops(w, heads) / per_step / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": workload_config(w, l2="n/a (host)"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample_description(w, heads)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    del torch
+    return 0
+
+
+def workload_config(w, l2):
+    c = {"workload": w.cfg.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D, "rope": w.rope_cos is not None,
+         "varlen": w.cu_seqlens is not None, "global_batch": w.B, "seq_len": w.T,
+         "parallelism": "replicas (one independent workload per GPU)", "l2": l2,
+         "flops_per_step_nominal": w.cfg.nominal_flops if (w.B, w.T, w.D) == (w.cfg.B, w.cfg.T, w.cfg.D)
+         else 7.0 * w.B * w.H * w.T * w.T * w.D,
+         "flops_per_step_within_documents": w.algorithmic_flops()}
+    if w.cu_seqlens is not None:
+        c["documents"] = int(len(w.cu_seqlens) - 1)
+    return c
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import bwd_causal_sdpa_b200 as A
+    from bwd_causal_sdpa_b200.runner import AttnRunner
+    from workloads import config_by_name, make_workload
+
+    world, rank, local = dist_setup(args.gpus)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    cfg = config_by_name(args.workload)
+    w = make_workload(cfg)
+    stream = torch.cuda.Stream(dev)
+    r = AttnRunner.from_workload(w, device=dev, stream=stream)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peaks, peak_src = load_peaks()
+    flops_step = 7.0 * w.B * w.H * w.T * w.T * w.D
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 0)):
+            r.forward()
+            r.backward()
+    st = r.status()
+    if st != A.ATTN_OK:
+        raise SystemExit(f"device status after warm-up: {A.error_string(st)}")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    n0 = A.attn_launch_count()
+    A.check(A.attn_profile_enable(1), "attn_profile_enable")
+    with ClockSampler(local) as clocks:
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                flush.zero_()
+                ev[i][0].record(stream)
+                r.forward()
+                r.backward()
+                ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    A.attn_profile_enable(0)
+    launches = A.attn_launch_count() - n0
+    prof = A.profile_summary()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms_local = sum(step_ms) / len(step_ms)
+    ms = max_over_ranks(ms_local)
+    value = flops_step * world / (ms / 1e3) / 1e12
+    st = r.status()
+    if st != A.ATTN_OK:
+        raise SystemExit(f"device status after timing: {A.error_string(st)}")
+
+    # Dominant kernel: the kind with the largest summed event time.
+    kinds = set(prof)
+    dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
+    roofline = None
+    kernels = {}
+    for name, (n, tot) in prof.items():
+        bound, amount, u = kernel_algorithmic(name, w, kinds)
+        kernels[name] = {"launches": n, "avg_ms": tot / n, "share": None, "bound": bound,
+                         "algorithmic": amount, "algorithmic_unit": u}
+    total_k = sum(tot for _, tot in prof.values())
+    for name in kernels:
+        kernels[name]["share"] = prof[name][1] / total_k if total_k else None
+    if dom is not None:
+        kd = kernels[dom]
+        simt = True  # the kernels below are the CUDA-core kernels until the tensor-core path lands
+        if kd["bound"] == "tensor":
+            achieved = kd["algorithmic"] / (kd["avg_ms"] / 1e3) / 1e12
+            if simt:
+                peak, unit, bound = FP32_SIMT_PEAK_TFLOPS, "TFLOP/s", "alu"
+                peak_note = "fp32 FMA peak of the CUDA cores (148 SMs x 128 x 2 x 1.965 GHz)"
+            else:
+                peak, unit, bound = peaks["bf16_tflops"], "TFLOP/s", "tensor"
+                peak_note = f"bf16_tflops burst ({peak_src})"
+        else:
+            achieved = kd["algorithmic"] / (kd["avg_ms"] / 1e3) / 1e9
+            peak, unit, bound = peaks["hbm_gbs"], "GB/s", "hbm"
+            peak_note = f"hbm_gbs ({peak_src})"
+        roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
+                    "unit": unit, "frac": achieved / peak, "traffic": None,
+                    "peak_source": peak_note}
+
+    # End to end through the public API with host buffers.
+    e2e = None
+    if not args.no_e2e:
+        td = r.q.dtype
+        host_in = [x.detach().to("cpu").pin_memory() for x in (r.q, r.k, r.v, r.do)]
+        host_out = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+                    for x in (r.o, r.lse, r.dq, r.dk, r.dv)]
+        h2d = sum(x.numel() * x.element_size() for x in host_in)
+        d2h = sum(x.numel() * x.element_size() for x in host_out)
+        e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+        torch.cuda.synchronize(dev)
+        barrier()
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                flush.zero_()
+                e_ev[i][0].record(stream)
+                for dst, src in zip((r.q, r.k, r.v, r.do), host_in):
+                    dst.copy_(src, non_blocking=True)
+                r.forward()
+                r.backward()
+                for dst, src in zip(host_out, (r.o, r.lse, r.dq, r.dk, r.dv)):
+                    dst.copy_(src, non_blocking=True)
+                e_ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev) / args.steps)
+        e2e = {"value": flops_step * world / (e_ms / 1e3) / 1e12, "unit": UNIT,
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del td
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        heads = [(0, 0)]
+        secs = oracle_slice_seconds(w, heads)
+        cpu = {"value": slice_flops(w, heads) / secs / 1e12, "unit": UNIT,
+               "cores": blas_threads(), "kind": "oracle", "seconds": secs,
+               "sample": sample_description(w, heads)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic (seeded)",
+            "config": workload_config(w, l2="flushed between steps (256 MiB write outside the step events)"),
+            "pct_of_bf16_peak": value / world / peaks["bf16_tflops"],
+            "pct_of_bf16_peak_sustained": value / world / peaks["bf16_tflops_sustained"],
+            "peaks_source": peak_src,
+            "value_within_documents": w.algorithmic_flops() * world / (ms / 1e3) / 1e12,
+            "roofline": roofline, "kernels": kernels,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

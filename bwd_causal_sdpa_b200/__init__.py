@@ -1,0 +1,159 @@
+"""Python binding of libattn.so: causal SDPA forward/backward on B200.
+
+Argument marshalling only. Every function here has the name and the argument
+order of the C entry point it calls (include/attn.h); tensors may be passed as
+torch tensors (their data_ptr() is used), plain integers (device addresses) or
+None (NULL). All computation happens in the library's CUDA kernels; there is
+no Python or CPU fallback, and importing this package fails if the library has
+not been built (``python bwd_causal_sdpa_b200/build.py``).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn.so")
+
+ATTN_BF16 = 0
+ATTN_F32 = 1
+
+ATTN_OK = 0
+ATTN_EINVAL = -1
+ATTN_EUNSUPPORTED = -2
+ATTN_EALIGN = -3
+ATTN_EWORKSPACE = -4
+ATTN_ECUDA = -5
+ATTN_EDEVICE_INPUT = -6
+ATTN_ETIMEOUT = -7
+
+# Every symbol include/attn.h declares, with its ctypes signature.
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SIGNATURES = {
+    "attn_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float, _I, _P,
+                      ctypes.c_size_t, _P]),
+    "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float, _I,
+                      _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "attn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
+    "attn_get_status": (_I, [_P]),
+    "attn_error_string": (ctypes.c_char_p, [_I]),
+    "attn_launch_count": (ctypes.c_ulonglong, []),
+    "attn_profile_enable": (_I, [_I]),
+    "attn_profile_kinds": (_I, []),
+    "attn_profile_read": (_I, [_I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_I),
+                               ctypes.POINTER(ctypes.c_double)]),
+}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {error_string(code)} (code {code})")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python bwd_causal_sdpa_b200/build.py` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream  # torch.cuda.Stream
+
+
+def error_string(code: int) -> str:
+    return _lib.attn_error_string(int(code)).decode()
+
+
+def attn_workspace_bytes(B, H, T, D, dtype, is_bwd) -> int:
+    return int(_lib.attn_workspace_bytes(B, H, T, D, dtype, int(is_bwd)))
+
+
+def attn_fwd(q, k, v, rope_cos, rope_sin, cu_seqlens, o, lse, B, H, T, D, scale, dtype,
+             workspace, ws_bytes, stream=None) -> int:
+    return int(_lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin),
+                             _ptr(cu_seqlens), _ptr(o), _ptr(lse), B, H, T, D, float(scale),
+                             dtype, _ptr(workspace), int(ws_bytes), _stream(stream)))
+
+
+def attn_bwd(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, T, D, scale, dtype,
+             dq, dk, dv, workspace, ws_bytes, stream=None) -> int:
+    return int(_lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse),
+                             _ptr(rope_cos), _ptr(rope_sin), _ptr(cu_seqlens), B, H, T, D,
+                             float(scale), dtype, _ptr(dq), _ptr(dk), _ptr(dv),
+                             _ptr(workspace), int(ws_bytes), _stream(stream)))
+
+
+def attn_get_status(stream=None) -> int:
+    return int(_lib.attn_get_status(_stream(stream)))
+
+
+def attn_error_string(code: int) -> str:
+    return error_string(code)
+
+
+def attn_launch_count() -> int:
+    return int(_lib.attn_launch_count())
+
+
+def attn_profile_enable(on) -> int:
+    return int(_lib.attn_profile_enable(int(bool(on))))
+
+
+def attn_profile_kinds() -> int:
+    return int(_lib.attn_profile_kinds())
+
+
+def attn_profile_read(kind: int):
+    """Returns (code, name, launches, total_ms) for one kernel kind."""
+    name = ctypes.c_char_p()
+    n = ctypes.c_int()
+    ms = ctypes.c_double()
+    code = int(_lib.attn_profile_read(int(kind), ctypes.byref(name), ctypes.byref(n),
+                                      ctypes.byref(ms)))
+    return code, (name.value or b"").decode(), int(n.value), float(ms.value)
+
+
+def profile_summary() -> dict:
+    """{kernel name: (timed launches, total ms)} for every kind with launches."""
+    out = {}
+    for kind in range(attn_profile_kinds()):
+        code, name, n, ms = attn_profile_read(kind)
+        check(code, "attn_profile_read")
+        if n:
+            out[name] = (n, ms)
+    return out
+
+
+def check(code: int, where: str = "attn") -> None:
+    """Raise AttnError for a non-zero return code."""
+    if code != ATTN_OK:
+        raise AttnError(code, where)
+
+
+__all__ = [name for name in list(globals()) if name.startswith(("attn_", "ATTN_"))] + [
+    "AttnError", "check", "error_string", "profile_summary", "LIB_PATH"]

@@ -1,0 +1,216 @@
+// attn_api.cu -- the C ABI of libattn.so (declared in include/attn.h):
+// host-side validation, the workspace plan, kernel launches and the device
+// status word. No function here allocates or frees device memory.
+#include <math.h>
+#include <stdint.h>
+
+#include "attn.h"
+#include "common.cuh"
+#include "prep.cuh"
+#include "simt.cuh"
+#include "trace.cuh"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Workspace layout (byte offsets from the caller's base pointer).
+struct WsPlan {
+  size_t doc_start = 0, doc_end = 0;  // int32 [B*T] each
+  size_t delta = 0;                   // f32 [B*H*T] (backward)
+  size_t total = 0;
+};
+
+bool sizes_ok(int B, int H, int T, int D) {
+  if (B <= 0 || H <= 0 || T <= 0) return false;
+  if (D != 64 && D != 128) return false;
+  const int64_t bt = (int64_t)B * T;
+  const int64_t n = bt * H * D;
+  return bt < INT32_MAX && n < INT32_MAX;
+}
+
+WsPlan plan(int B, int H, int T, int D, int dtype, int is_bwd) {
+  (void)D;
+  (void)dtype;
+  WsPlan p;
+  size_t off = 0;
+  const size_t bt = (size_t)B * T, rows = bt * H;
+  p.doc_start = off; off += round_up(bt * sizeof(int32_t));
+  p.doc_end = off;   off += round_up(bt * sizeof(int32_t));
+  if (is_bwd) { p.delta = off; off += round_up(rows * sizeof(float)); }
+  p.total = off;
+  return p;
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int check_common(const void* q, const void* k, const void* v, const float* rc, const float* rs,
+                 const int32_t* cu, int B, int H, int T, int D, float scale, int dtype,
+                 void* ws, size_t ws_bytes, int is_bwd) {
+  if (!q || !k || !v) return ATTN_EINVAL;
+  if (dtype != ATTN_BF16 && dtype != ATTN_F32) return ATTN_EINVAL;
+  if (B <= 0 || H <= 0 || T <= 0) return ATTN_EINVAL;
+  if (!isfinite(scale)) return ATTN_EINVAL;
+  if ((rc == nullptr) != (rs == nullptr)) return ATTN_EINVAL;
+  if (!sizes_ok(B, H, T, D)) return ATTN_EUNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return ATTN_EALIGN;
+  if ((rc && !aligned(rc, 4)) || (rs && !aligned(rs, 4)) || (cu && !aligned(cu, 4))) return ATTN_EALIGN;
+  const WsPlan p = plan(B, H, T, D, dtype, is_bwd);
+  if (p.total > 0) {
+    if (!ws) return ATTN_EWORKSPACE;
+    if (!aligned(ws, 16)) return ATTN_EALIGN;
+    if (ws_bytes < p.total) return ATTN_EWORKSPACE;
+  }
+  return ATTN_OK;
+}
+
+int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
+
+template <typename TIO, int D>
+int fwd_simt(const void* q, const void* k, const void* v, const float* rc, const float* rs,
+             const int32_t* ds, void* o, float* lse, int B, int H, int T, float scale,
+             cudaStream_t st) {
+  dim3 grid(B * H, (T + 15) / 16);
+  ATTN_LAUNCH(KK_FWD, st,
+              simt_fwd_kernel<TIO, D><<<grid, 128, 0, st>>>((const TIO*)q, (const TIO*)k,
+                                                            (const TIO*)v, rc, rs, ds, (TIO*)o,
+                                                            lse, H, T, scale));
+  return launch_status();
+}
+
+template <typename TIO, int D>
+int bwd_simt(const void* q, const void* k, const void* v, const void* o, const void* dO,
+             const float* lse, const float* rc, const float* rs, const int32_t* ds,
+             const int32_t* de, float* delta, void* dq, void* dk, void* dv, int B, int H, int T,
+             float scale, cudaStream_t st) {
+  const long rows = (long)B * H * T;
+  ATTN_LAUNCH(KK_DELTA, st,
+              delta_kernel<TIO, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+                  (const TIO*)o, (const TIO*)dO, delta, rows));
+  if (launch_status()) return ATTN_ECUDA;
+  dim3 g1(B * H, (T + 31) / 32);
+  ATTN_LAUNCH(KK_DKDV, st,
+              simt_dkdv_kernel<TIO, D><<<g1, 128, 0, st>>>(
+                  (const TIO*)q, (const TIO*)k, (const TIO*)v, (const TIO*)dO, lse, delta, rc, rs,
+                  ds, de, (TIO*)dk, (TIO*)dv, H, T, scale));
+  if (launch_status()) return ATTN_ECUDA;
+  ATTN_LAUNCH(KK_DQ, st,
+              simt_dq_kernel<TIO, D><<<g1, 128, 0, st>>>(
+                  (const TIO*)q, (const TIO*)k, (const TIO*)v, (const TIO*)dO, lse, delta, rc, rs,
+                  ds, (TIO*)dq, H, T, scale));
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t attn_workspace_bytes(int B, int H, int T, int D, int dtype, int is_bwd) {
+  if (!sizes_ok(B, H, T, D) || (dtype != ATTN_BF16 && dtype != ATTN_F32)) return 0;
+  return plan(B, H, T, D, dtype, is_bwd).total;
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, const float* rope_cos,
+             const float* rope_sin, const int32_t* cu_seqlens, void* o, float* lse, int B, int H,
+             int T, int D, float scale, int dtype, void* workspace, size_t ws_bytes,
+             void* stream) {
+  int rc = check_common(q, k, v, rope_cos, rope_sin, cu_seqlens, B, H, T, D, scale, dtype,
+                        workspace, ws_bytes, 0);
+  if (rc) return rc;
+  if (!o || !lse) return ATTN_EINVAL;
+  if (!aligned(o, 16) || !aligned(lse, 4)) return ATTN_EALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  const WsPlan p = plan(B, H, T, D, dtype, 0);
+  char* ws = (char*)workspace;
+  int32_t* ds = nullptr;
+  if (cu_seqlens) {
+    ds = (int32_t*)(ws + p.doc_start);
+    ATTN_LAUNCH(KK_DOC_RANGES, st,
+                doc_ranges_kernel<<<1, 1024, 0, st>>>(cu_seqlens, B, T, ds,
+                                                      (int32_t*)(ws + p.doc_end)));
+    if (launch_status()) return ATTN_ECUDA;
+  }
+  if (dtype == ATTN_F32) {
+    return D == 64 ? fwd_simt<float, 64>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, T, scale, st)
+                   : fwd_simt<float, 128>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, T, scale, st);
+  }
+  return D == 64
+             ? fwd_simt<__nv_bfloat16, 64>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, T, scale, st)
+             : fwd_simt<__nv_bfloat16, 128>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, T, scale, st);
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+             const float* lse, const float* rope_cos, const float* rope_sin,
+             const int32_t* cu_seqlens, int B, int H, int T, int D, float scale, int dtype,
+             void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_common(q, k, v, rope_cos, rope_sin, cu_seqlens, B, H, T, D, scale, dtype,
+                        workspace, ws_bytes, 1);
+  if (rc) return rc;
+  if (!o || !dO || !lse || !dq || !dk || !dv) return ATTN_EINVAL;
+  if (!aligned(o, 16) || !aligned(dO, 16) || !aligned(dq, 16) || !aligned(dk, 16) ||
+      !aligned(dv, 16) || !aligned(lse, 4))
+    return ATTN_EALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  const WsPlan p = plan(B, H, T, D, dtype, 1);
+  char* ws = (char*)workspace;
+  int32_t *ds = nullptr, *de = nullptr;
+  if (cu_seqlens) {
+    ds = (int32_t*)(ws + p.doc_start);
+    de = (int32_t*)(ws + p.doc_end);
+    ATTN_LAUNCH(KK_DOC_RANGES, st, doc_ranges_kernel<<<1, 1024, 0, st>>>(cu_seqlens, B, T, ds, de));
+    if (launch_status()) return ATTN_ECUDA;
+  }
+  float* delta = (float*)(ws + p.delta);
+  if (dtype == ATTN_F32) {
+    return D == 64 ? bwd_simt<float, 64>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, delta,
+                                         dq, dk, dv, B, H, T, scale, st)
+                   : bwd_simt<float, 128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, delta,
+                                          dq, dk, dv, B, H, T, scale, st);
+  }
+  return D == 64 ? bwd_simt<__nv_bfloat16, 64>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de,
+                                               delta, dq, dk, dv, B, H, T, scale, st)
+                 : bwd_simt<__nv_bfloat16, 128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de,
+                                                delta, dq, dk, dv, B, H, T, scale, st);
+}
+
+int attn_get_status(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return ATTN_ECUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ECUDA;
+  if (v != 0) {
+    const int z = 0;
+    if (cudaMemcpyToSymbol(g_attn_status, &z, sizeof(int)) != cudaSuccess) return ATTN_ECUDA;
+  }
+  return v;
+}
+
+const char* attn_error_string(int code) {
+  switch (code) {
+    case ATTN_OK: return "ok";
+    case ATTN_EINVAL: return "invalid argument (null pointer, non-positive size, bad dtype or scale)";
+    case ATTN_EUNSUPPORTED: return "unsupported size (D must be 64 or 128; indices must fit int32)";
+    case ATTN_EALIGN: return "misaligned pointer (tensors and workspace need 16 bytes)";
+    case ATTN_EWORKSPACE: return "workspace missing or smaller than attn_workspace_bytes()";
+    case ATTN_ECUDA: return "CUDA launch or runtime error";
+    case ATTN_EDEVICE_INPUT: return "malformed cu_seqlens detected on the device";
+    case ATTN_ETIMEOUT: return "a bounded device-side wait timed out";
+    default: return "unknown attn status code";
+  }
+}
+
+unsigned long long attn_launch_count(void) { return trace::launches(); }
+
+int attn_profile_enable(int on) { return trace::enable(on != 0) == 0 ? ATTN_OK : ATTN_ECUDA; }
+
+int attn_profile_kinds(void) { return KK_COUNT; }
+
+int attn_profile_read(int kind, const char** name, int* launches, double* total_ms) {
+  if (kind < 0 || kind >= KK_COUNT || !name || !launches || !total_ms) return ATTN_EINVAL;
+  *name = kKernelNames[kind];
+  return trace::read(kind, launches, total_ms) == 0 ? ATTN_OK : ATTN_ECUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,101 @@
+// common.cuh -- small device helpers shared by every kernel of libattn.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "attn.h"
+
+// Device status word (one per device context). Kernels record the first
+// device-detected problem here instead of trapping; attn_get_status() reads
+// and clears it.
+__device__ int g_attn_status;
+
+__device__ __forceinline__ void report_status(int code) {
+  atomicCAS(&g_attn_status, 0, code);
+}
+
+// ---- storage type conversions ---------------------------------------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Load / store NC consecutive elements (NC = 2 or 4) as fp32.
+template <int NC>
+__device__ __forceinline__ void load_vec(const float* p, float* out) {
+  if constexpr (NC == 4) {
+    float4 t = *reinterpret_cast<const float4*>(p);
+    out[0] = t.x; out[1] = t.y; out[2] = t.z; out[3] = t.w;
+  } else {
+    float2 t = *reinterpret_cast<const float2*>(p);
+    out[0] = t.x; out[1] = t.y;
+  }
+}
+template <int NC>
+__device__ __forceinline__ void load_vec(const __nv_bfloat16* p, float* out) {
+  if constexpr (NC == 4) {
+    uint2 t = *reinterpret_cast<const uint2*>(p);
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&t.x);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&t.y);
+    out[0] = __low2float(a); out[1] = __high2float(a);
+    out[2] = __low2float(b); out[3] = __high2float(b);
+  } else {
+    __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(p);
+    out[0] = __low2float(a); out[1] = __high2float(a);
+  }
+}
+template <int NC>
+__device__ __forceinline__ void store_vec(float* p, const float* v) {
+  if constexpr (NC == 4) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  } else {
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  }
+}
+template <int NC>
+__device__ __forceinline__ void store_vec(__nv_bfloat16* p, const float* v) {
+  if constexpr (NC == 4) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+    uint2 t;
+    t.x = *reinterpret_cast<uint32_t*>(&a);
+    t.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = t;
+  } else {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v[0], v[1]);
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+// Rotate (in place) NC consecutive elements starting at an even dimension d0
+// by the RoPE angles of position pos: pairs (x[2i], x[2i+1]) -> (x0 c - x1 s,
+// x0 s + x1 c). inverse = true applies the transpose rotation.
+template <int NC, int D>
+__device__ __forceinline__ void rope_pairs(float* x, const float* rc, const float* rs,
+                                           int pos, int d0, bool inverse) {
+#pragma unroll
+  for (int c = 0; c < NC; c += 2) {
+    const int pi = (d0 + c) >> 1;
+    const float cs = rc[(size_t)pos * (D / 2) + pi];
+    const float sn = inverse ? -rs[(size_t)pos * (D / 2) + pi] : rs[(size_t)pos * (D / 2) + pi];
+    const float x0 = x[c], x1 = x[c + 1];
+    x[c] = x0 * cs - x1 * sn;
+    x[c + 1] = x0 * sn + x1 * cs;
+  }
+}

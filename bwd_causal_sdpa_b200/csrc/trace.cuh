@@ -1,0 +1,101 @@
+// trace.cuh -- host-side launch counter and optional per-kernel CUDA-event
+// timing (a measurement aid; not thread safe, see include/attn.h).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <vector>
+
+enum KernelKind : int {
+  KK_DOC_RANGES = 0,
+  KK_ROPE_PREP,
+  KK_FWD,
+  KK_DELTA,
+  KK_DKDV,
+  KK_DQ,
+  KK_DQ_FINALIZE,
+  KK_COUNT
+};
+
+static const char* const kKernelNames[KK_COUNT] = {
+    "doc_ranges", "rope_prep", "fwd", "delta", "dkdv", "dq", "dq_finalize"};
+
+namespace trace {
+
+constexpr int kMaxTimed = 16384;
+
+struct Record {
+  cudaEvent_t a, b;
+  int kind;
+};
+
+inline unsigned long long& launches() {
+  static unsigned long long n = 0;
+  return n;
+}
+inline bool& enabled() {
+  static bool on = false;
+  return on;
+}
+inline std::vector<Record>& pool() {
+  static std::vector<Record> p;
+  return p;
+}
+inline int& used() {
+  static int u = 0;
+  return u;
+}
+
+// Call before a kernel launch: counts it and, when timing is on, records the
+// opening event on the launch stream. Returns the record index or -1.
+inline int begin(int kind, cudaStream_t st) {
+  ++launches();
+  if (!enabled() || used() >= (int)pool().size()) return -1;
+  Record& r = pool()[used()];
+  r.kind = kind;
+  if (cudaEventRecord(r.a, st) != cudaSuccess) return -1;
+  return used()++;
+}
+inline void end(int idx, cudaStream_t st) {
+  if (idx >= 0) cudaEventRecord(pool()[idx].b, st);
+}
+
+inline int enable(bool on) {
+  if (on && pool().empty()) {
+    pool().resize(kMaxTimed);
+    for (auto& r : pool()) {
+      if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess) {
+        pool().clear();
+        return -1;
+      }
+    }
+  }
+  if (on) used() = 0;
+  enabled() = on;
+  return 0;
+}
+
+inline int read(int kind, int* n, double* ms) {
+  *n = 0;
+  *ms = 0.0;
+  for (int i = 0; i < used(); ++i) {
+    const Record& r = pool()[i];
+    if (r.kind != kind) continue;
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return -1;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) return -1;
+    *ms += t;
+    ++*n;
+  }
+  return 0;
+}
+
+}  // namespace trace
+
+// Wrap one kernel launch: LAUNCH(kind, stream, kernel<<<grid, block, smem, stream>>>(...));
+#define ATTN_LAUNCH(kind, st, ...)            \
+  do {                                        \
+    const int _tr = trace::begin((kind), (st)); \
+    __VA_ARGS__;                              \
+    trace::end(_tr, (st));                    \
+  } while (0)

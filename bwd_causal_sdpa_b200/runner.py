@@ -1,0 +1,101 @@
+"""Device buffers for one attention problem, and the two C-ABI calls on them.
+
+PyTorch is used here only to own device memory and streams; every step of the
+attention runs in libattn.so through the ctypes binding.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import (ATTN_BF16, ATTN_F32, attn_bwd, attn_fwd, attn_get_status, attn_workspace_bytes,
+               check)
+
+
+def torch_dtype(dtype: int):
+    return torch.bfloat16 if dtype == ATTN_BF16 else torch.float32
+
+
+def to_device(x: np.ndarray, dtype: int, device) -> torch.Tensor:
+    """float32 numpy (already bf16-representable for bf16) -> device tensor."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(device=device, dtype=torch_dtype(dtype)).contiguous()
+
+
+@dataclass
+class Problem:
+    B: int
+    H: int
+    T: int
+    D: int
+    scale: float
+    dtype: int
+
+
+class AttnRunner:
+    """Holds q, k, v, dO (inputs), o, lse, dq, dk, dv (outputs), the RoPE
+    tables, cu_seqlens and one workspace sized for the larger of the two
+    calls, all on one device."""
+
+    def __init__(self, B, H, T, D, *, dtype=ATTN_BF16, scale=None, rope=None, cu_seqlens=None,
+                 device="cuda", stream: Optional[torch.cuda.Stream] = None):
+        self.p = Problem(B, H, T, D, 1.0 / math.sqrt(D) if scale is None else scale, dtype)
+        self.device = torch.device(device)
+        self.stream = stream
+        td = torch_dtype(dtype)
+        shape = (B, H, T, D)
+        mk = lambda: torch.empty(shape, dtype=td, device=self.device)
+        self.q, self.k, self.v, self.do = mk(), mk(), mk(), mk()
+        self.o, self.dq, self.dk, self.dv = mk(), mk(), mk(), mk()
+        self.lse = torch.empty((B, H, T), dtype=torch.float32, device=self.device)
+        self.rope_cos = self.rope_sin = None
+        if rope is not None:
+            c, s = rope
+            self.rope_cos = torch.from_numpy(np.ascontiguousarray(c, np.float32)).to(self.device)
+            self.rope_sin = torch.from_numpy(np.ascontiguousarray(s, np.float32)).to(self.device)
+        self.cu = None
+        if cu_seqlens is not None:
+            self.cu = torch.from_numpy(np.asarray(cu_seqlens, dtype=np.int32)).to(self.device)
+        self.ws_bytes = max(attn_workspace_bytes(B, H, T, D, dtype, 0),
+                            attn_workspace_bytes(B, H, T, D, dtype, 1))
+        self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=self.device)
+
+    @classmethod
+    def from_workload(cls, w, device="cuda", stream=None) -> "AttnRunner":
+        dtype = ATTN_BF16 if w.dtype == "bf16" else ATTN_F32
+        rope = None if w.rope_cos is None else (w.rope_cos, w.rope_sin)
+        r = cls(w.B, w.H, w.T, w.D, dtype=dtype, scale=w.scale, rope=rope,
+                cu_seqlens=w.cu_seqlens, device=device, stream=stream)
+        r.load_inputs(w.q, w.k, w.v, w.do)
+        return r
+
+    def load_inputs(self, q, k, v, do):
+        for dst, src in ((self.q, q), (self.k, k), (self.v, v), (self.do, do)):
+            dst.copy_(to_device(src, self.p.dtype, self.device))
+
+    def forward(self) -> None:
+        p = self.p
+        check(attn_fwd(self.q, self.k, self.v, self.rope_cos, self.rope_sin, self.cu, self.o,
+                       self.lse, p.B, p.H, p.T, p.D, p.scale, p.dtype, self.ws, self.ws_bytes,
+                       self.stream), "attn_fwd")
+
+    def backward(self) -> None:
+        p = self.p
+        check(attn_bwd(self.q, self.k, self.v, self.o, self.do, self.lse, self.rope_cos,
+                       self.rope_sin, self.cu, p.B, p.H, p.T, p.D, p.scale, p.dtype, self.dq,
+                       self.dk, self.dv, self.ws, self.ws_bytes, self.stream), "attn_bwd")
+
+    def status(self) -> int:
+        return attn_get_status(self.stream)
+
+    def results(self) -> dict:
+        """Outputs as float64 numpy arrays (synchronises)."""
+        torch.cuda.synchronize(self.device)
+        f = lambda t: t.detach().to(torch.float64).cpu().numpy()
+        return {"o": f(self.o), "lse": f(self.lse), "dq": f(self.dq), "dk": f(self.dk),
+                "dv": f(self.dv)}

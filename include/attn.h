@@ -1,0 +1,147 @@
+/*
+ * attn.h -- C ABI of libattn.so: causal multi-head scaled-dot-product
+ * attention (forward and backward) for NVIDIA B200 (sm_100a).
+ *
+ * What it computes. For every batch row b and head h, with q_r = R(pos) q and
+ * k_r = R(pos) k (RoPE, optional):
+ *     S   = scale * q_r k_r^T,  keeping S[i][j] only where j <= i and j is in
+ *           i's document; every other entry is -inf
+ *     P   = softmax over each row of S;   o = P v
+ *     lse = log(sum_j exp(S[i][j]))  (natural log)
+ * and the backward of L = sum(o * dO):
+ *     Delta_i = sum_d dO[i][d] * o[i][d];  dP = dO v^T;  dS = P * (dP - Delta)
+ *     dv = P^T dO;  dq = R(pos)^T (scale * dS k_r);  dk = R(pos)^T (scale * dS^T q_r)
+ * Sources, by page and section: ARK README, "Accelerated forward pass (GPU)"
+ * (multi-head SDPA with the causal mask fused in) and "Inference architecture
+ * (EKO)" (RoPE from precomputed sin/cos tables); ARK README, "Backward pass
+ * (AutoGrad)" (gradients of the attention inside training); Forge README,
+ * "What this is" (flash attention forward and backward) and "Architecture",
+ * Model line (RoPE on interleaved pairs); Cort33x, "Preserving context in the
+ * data" (short documents packed into one training window).
+ *
+ * Conventions shared by every call:
+ *   - Tensors q, k, v, o, dO, dq, dk, dv are [B, H, T, D], contiguous, D
+ *     fastest, in the storage type `dtype` (ATTN_BF16 or ATTN_F32). lse is
+ *     [B, H, T] float32. All are DEVICE pointers on the current CUDA device,
+ *     owned by the caller; the library never allocates or frees memory.
+ *   - q, k, v, o, dO, dq, dk, dv and the workspace must be 16-byte aligned
+ *     (the kernels move tiles with TMA); lse, rope tables and cu_seqlens must
+ *     be 4-byte aligned.
+ *   - D must be 64 or 128. B, H, T >= 1. B*T and B*H*T*D must fit in int32.
+ *   - RoPE: rope_cos and rope_sin are both NULL (no RoPE) or both [T, D/2]
+ *     float32 with row p holding cos/sin(p * theta_i) for position p. Pairs
+ *     (x[2i], x[2i+1]) of q and k are rotated by the angle of pair i; v is not
+ *     rotated. The position of token t is t minus the start of its document.
+ *   - Packed documents: cu_seqlens is NULL (each row is one document) or an
+ *     int32 device array over the flattened B*T token axis: strictly rising,
+ *     starting at 0, containing every row boundary r*T and ending with the
+ *     value B*T, which marks its end (the array holds at most B*T+1 entries;
+ *     the device reads it up to that end marker and no further). A malformed
+ *     array is detected on the device: the call then computes as if
+ *     cu_seqlens were NULL and the status word reports ATTN_EDEVICE_INPUT.
+ *   - Every call is asynchronous and stream ordered on `stream` (a
+ *     cudaStream_t; NULL = the legacy default stream). Host-side validation
+ *     errors return before anything is launched.
+ *   - The workspace is caller-owned device scratch of at least
+ *     attn_workspace_bytes(...) bytes; its contents on entry do not matter
+ *     and are undefined on return. Two calls that overlap in time must not
+ *     share one workspace.
+ *
+ * Return codes: ATTN_OK or one of the negative ATTN_E* values below.
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* storage types */
+#define ATTN_BF16 0
+#define ATTN_F32 1
+
+/* return / status codes */
+#define ATTN_OK 0
+#define ATTN_EINVAL (-1)        /* null pointer, B/H/T <= 0, non-finite scale, bad dtype */
+#define ATTN_EUNSUPPORTED (-2)  /* D not 64/128, or sizes beyond the int32 index range */
+#define ATTN_EALIGN (-3)        /* a pointer violates the alignment rules above */
+#define ATTN_EWORKSPACE (-4)    /* ws_bytes smaller than attn_workspace_bytes(...) */
+#define ATTN_ECUDA (-5)         /* a CUDA launch or runtime call failed */
+#define ATTN_EDEVICE_INPUT (-6) /* device-detected malformed cu_seqlens */
+#define ATTN_ETIMEOUT (-7)      /* a bounded device-side wait gave up */
+
+/*
+ * attn_fwd -- forward pass.
+ * In:  q, k, v [B,H,T,D] (dtype); rope_cos, rope_sin [T,D/2] f32 or NULL;
+ *      cu_seqlens (see above) or NULL; scale (usually 1/sqrt(D)).
+ * Out: o [B,H,T,D] (dtype); lse [B,H,T] f32, natural log, saved for attn_bwd.
+ * Workspace: attn_workspace_bytes(B,H,T,D,dtype,0) bytes.
+ */
+int attn_fwd(const void* q, const void* k, const void* v,
+             const float* rope_cos, const float* rope_sin,
+             const int32_t* cu_seqlens,
+             void* o, float* lse,
+             int B, int H, int T, int D, float scale,
+             int dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * attn_bwd -- backward pass of L = sum(o * dO).
+ * In:  q, k, v (the same un-rotated inputs given to attn_fwd), o and lse as
+ *      attn_fwd returned them, dO [B,H,T,D] (dtype), the same RoPE tables,
+ *      cu_seqlens and scale as the forward.
+ * Out: dq, dk, dv [B,H,T,D] (dtype): gradients with respect to the
+ *      un-rotated q and k, and v.
+ * Workspace: attn_workspace_bytes(B,H,T,D,dtype,1) bytes.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o,
+             const void* dO, const float* lse,
+             const float* rope_cos, const float* rope_sin,
+             const int32_t* cu_seqlens,
+             int B, int H, int T, int D, float scale, int dtype,
+             void* dq, void* dk, void* dv,
+             void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of workspace attn_fwd (is_bwd = 0) or attn_bwd (is_bwd = 1) needs for
+ * these sizes; 0 for invalid sizes. Pure host function, no CUDA call. */
+size_t attn_workspace_bytes(int B, int H, int T, int D, int dtype, int is_bwd);
+
+/* Synchronises `stream`, then returns and clears the current device's status
+ * word: ATTN_OK, ATTN_EDEVICE_INPUT or ATTN_ETIMEOUT (first error recorded
+ * since the last call), or ATTN_ECUDA if the synchronisation itself failed. */
+int attn_get_status(void* stream);
+
+/* Static, human-readable text for a return or status code. */
+const char* attn_error_string(int code);
+
+/*
+ * Tracing aids (the source pages define no counterpart; they support
+ * measurement only). Not thread safe: call them from the thread that
+ * launches the attention calls.
+ *
+ * attn_launch_count: number of kernels this library has launched in this
+ * process so far (all devices, all streams).
+ *
+ * attn_profile_enable(1) clears earlier records and starts recording a pair
+ * of CUDA events around every kernel the library launches (on the stream of
+ * that launch; up to 16384 launches, later ones are counted but not timed);
+ * attn_profile_enable(0) stops recording. Returns ATTN_OK or ATTN_ECUDA.
+ *
+ * attn_profile_read(kind, ...): for kernel kind 0 <= kind < attn_profile_kinds(),
+ * waits for the recorded events and stores the kind's name (static string),
+ * the number of timed launches and their summed duration in milliseconds.
+ * Returns ATTN_OK, ATTN_EINVAL (kind out of range or a null output pointer)
+ * or ATTN_ECUDA.
+ */
+unsigned long long attn_launch_count(void);
+int attn_profile_enable(int on);
+int attn_profile_kinds(void);
+int attn_profile_read(int kind, const char** name, int* launches, double* total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H_ */

@@ -1,0 +1,109 @@
+"""The C ABI surface, on the CPU: the library loads, exports every function
+include/attn.h declares, and rejects bad arguments on the host before any
+CUDA call (no kernel is launched by these tests)."""
+
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w \*]*?\b(attn_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    import ctypes
+
+    import bwd_causal_sdpa_b200 as A
+
+    names = _declared_functions()
+    assert {"attn_fwd", "attn_bwd", "attn_workspace_bytes", "attn_get_status",
+            "attn_error_string"} <= set(names)
+    lib = ctypes.CDLL(A.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+        assert hasattr(A, n), f"{n} has no Python binding of the same name"
+
+
+def test_error_strings_and_codes():
+    import bwd_causal_sdpa_b200 as A
+
+    for code in (A.ATTN_OK, A.ATTN_EINVAL, A.ATTN_EUNSUPPORTED, A.ATTN_EALIGN,
+                 A.ATTN_EWORKSPACE, A.ATTN_ECUDA, A.ATTN_EDEVICE_INPUT, A.ATTN_ETIMEOUT):
+        s = A.attn_error_string(code)
+        assert s and "unknown" not in s
+    assert "unknown" in A.attn_error_string(12345)
+
+
+def test_workspace_bytes():
+    import bwd_causal_sdpa_b200 as A
+
+    for dtype in (A.ATTN_BF16, A.ATTN_F32):
+        for D in (64, 128):
+            f = A.attn_workspace_bytes(2, 3, 200, D, dtype, 0)
+            b = A.attn_workspace_bytes(2, 3, 200, D, dtype, 1)
+            assert f > 0 and b > 0 and f % 256 == 0 and b % 256 == 0
+    assert A.attn_workspace_bytes(1, 1, 128, 96, A.ATTN_BF16, 1) == 0
+    assert A.attn_workspace_bytes(0, 1, 128, 64, A.ATTN_BF16, 1) == 0
+    assert A.attn_workspace_bytes(1, 1, 128, 64, 7, 1) == 0
+
+
+# Fake, aligned addresses: every call below fails validation on the host, so
+# nothing is dereferenced and no CUDA call is made.
+P = 1 << 20
+
+
+def _fwd(**kw):
+    import bwd_causal_sdpa_b200 as A
+
+    a = dict(q=P, k=P, v=P, rope_cos=None, rope_sin=None, cu_seqlens=None, o=P, lse=P, B=1, H=1,
+             T=128, D=64, scale=0.125, dtype=A.ATTN_BF16, workspace=P, ws_bytes=1 << 30)
+    a.update(kw)
+    return A.attn_fwd(**a)
+
+
+def _bwd(**kw):
+    import bwd_causal_sdpa_b200 as A
+
+    a = dict(q=P, k=P, v=P, o=P, dO=P, lse=P, rope_cos=None, rope_sin=None, cu_seqlens=None,
+             B=1, H=1, T=128, D=64, scale=0.125, dtype=A.ATTN_BF16, dq=P, dk=P, dv=P,
+             workspace=P, ws_bytes=1 << 30)
+    a.update(kw)
+    return A.attn_bwd(**a)
+
+
+@pytest.mark.parametrize("call", [_fwd, _bwd])
+def test_host_validation(call):
+    import bwd_causal_sdpa_b200 as A
+
+    assert call(q=None) == A.ATTN_EINVAL
+    assert call(B=0) == A.ATTN_EINVAL
+    assert call(T=-3) == A.ATTN_EINVAL
+    assert call(scale=float("nan")) == A.ATTN_EINVAL
+    assert call(dtype=5) == A.ATTN_EINVAL
+    assert call(rope_cos=P) == A.ATTN_EINVAL          # sin missing
+    assert call(D=96) == A.ATTN_EUNSUPPORTED
+    assert call(B=1 << 16, H=1 << 10, T=1 << 10) == A.ATTN_EUNSUPPORTED
+    assert call(k=P + 8) == A.ATTN_EALIGN
+    assert call(workspace=P + 4) == A.ATTN_EALIGN
+    assert call(cu_seqlens=P + 2) == A.ATTN_EALIGN
+    assert call(workspace=None) == A.ATTN_EWORKSPACE
+    assert call(ws_bytes=16) == A.ATTN_EWORKSPACE
+
+
+def test_bwd_specific_validation():
+    import bwd_causal_sdpa_b200 as A
+
+    assert _bwd(dO=None) == A.ATTN_EINVAL
+    assert _bwd(dv=P + 8) == A.ATTN_EALIGN
+    assert _fwd(lse=None) == A.ATTN_EINVAL
+    assert _fwd(o=P + 2) == A.ATTN_EALIGN
