@@ -27,6 +27,8 @@ ATTN_EWORKSPACE = -4
 ATTN_ECUDA = -5
 ATTN_EDEVICE_INPUT = -6
 ATTN_ETIMEOUT = -7
+ATTN_ESCRATCH = -8
+ATTN_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 # Every symbol include/attn.h declares, with its ctypes signature.
 _P = ctypes.c_void_p
@@ -36,6 +38,8 @@ _SIGNATURES = {
                       ctypes.c_size_t, _P]),
     "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float, _I,
                       _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float,
+                              _I, _P, _P, _P, _P]),
     "attn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
     "attn_get_status": (_I, [_P]),
     "attn_error_string": (ctypes.c_char_p, [_I]),
@@ -106,6 +110,16 @@ def attn_bwd(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, T, D, sc
                              _ptr(rope_cos), _ptr(rope_sin), _ptr(cu_seqlens), B, H, T, D,
                              float(scale), dtype, _ptr(dq), _ptr(dk), _ptr(dv),
                              _ptr(workspace), int(ws_bytes), _stream(stream)))
+
+
+def attn_bwd_noalloc(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, T, D, scale,
+                     dtype, dq, dk, dv, stream=None) -> int:
+    """attn_bwd without a workspace: the library's fixed device scratch array
+    is used instead (see include/attn.h for who needs this and its limits)."""
+    return int(_lib.attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse),
+                                     _ptr(rope_cos), _ptr(rope_sin), _ptr(cu_seqlens), B, H, T,
+                                     D, float(scale), dtype, _ptr(dq), _ptr(dk), _ptr(dv),
+                                     _stream(stream)))
 
 
 def attn_get_status(stream=None) -> int:

@@ -4,6 +4,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "attn.h"
 #include "common.cuh"
 #include "prep.cuh"
@@ -197,6 +199,9 @@ const char* attn_error_string(int code) {
     case ATTN_ECUDA: return "CUDA launch or runtime error";
     case ATTN_EDEVICE_INPUT: return "malformed cu_seqlens detected on the device";
     case ATTN_ETIMEOUT: return "a bounded device-side wait timed out";
+    case ATTN_ESCRATCH:
+      return "problem needs more scratch than attn_bwd_noalloc's fixed array "
+             "(ATTN_NOALLOC_SCRATCH_BYTES)";
     default: return "unknown attn status code";
   }
 }
@@ -214,3 +219,98 @@ int attn_profile_read(int kind, const char** name, int* launches, double* total_
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// attn_bwd_noalloc: the backward for callers that cannot allocate device
+// memory. Its scratch is this file-scope device array. In host code the name
+// g_noalloc_scratch is only a host-side stand-in for the symbol, never a
+// device address: the device address is looked up once per device with
+// cudaGetSymbolAddress and that pointer is what the kernels receive.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocBytes = ATTN_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_dev_ptr[kNoAllocMaxDevices] = {};
+
+// Scratch layout: document starts, document ends (int32 [B*T] each), then
+// Delta (f32 [B*H*T]); each part starts on a 256-byte boundary.
+struct NoAllocPlan {
+  size_t doc_start, doc_end, delta, total;
+};
+
+NoAllocPlan noalloc_plan(int B, int H, int T) {
+  NoAllocPlan p;
+  const size_t bt = (size_t)B * T;
+  p.doc_start = 0;
+  p.doc_end = round_up(bt * sizeof(int32_t));
+  p.delta = p.doc_end + round_up(bt * sizeof(int32_t));
+  p.total = p.delta + round_up(bt * (size_t)H * sizeof(float));
+  return p;
+}
+
+// Device address of the scratch array on the current device; the first call
+// per device does the lookup (with that device current).
+int noalloc_scratch(char** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
+    return ATTN_ECUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_dev_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return ATTN_ECUDA;
+    g_noalloc_dev_ptr[dev] = p;
+  }
+  *out = (char*)g_noalloc_dev_ptr[dev];
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                const void* dO, const float* lse, const float* rope_cos,
+                                const float* rope_sin, const int32_t* cu_seqlens, int B, int H,
+                                int T, int D, float scale, int dtype, void* dq, void* dk,
+                                void* dv, void* stream) {
+  // Host-side checks, as attn_bwd makes them (minus the workspace).
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return ATTN_EINVAL;
+  if (dtype != ATTN_BF16 && dtype != ATTN_F32) return ATTN_EINVAL;
+  if (B <= 0 || H <= 0 || T <= 0 || !isfinite(scale)) return ATTN_EINVAL;
+  if ((rope_cos == nullptr) != (rope_sin == nullptr)) return ATTN_EINVAL;
+  if (!sizes_ok(B, H, T, D)) return ATTN_EUNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dO, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4) || (rope_cos && !aligned(rope_cos, 4)) ||
+      (rope_sin && !aligned(rope_sin, 4)) || (cu_seqlens && !aligned(cu_seqlens, 4)))
+    return ATTN_EALIGN;
+  const NoAllocPlan p = noalloc_plan(B, H, T);
+  if (p.total > kNoAllocBytes) return ATTN_ESCRATCH;
+
+  char* ws = nullptr;
+  if (int rc = noalloc_scratch(&ws)) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  int32_t *ds = nullptr, *de = nullptr;
+  if (cu_seqlens) {
+    // doc_ranges_kernel writes every entry of both arrays.
+    ds = (int32_t*)(ws + p.doc_start);
+    de = (int32_t*)(ws + p.doc_end);
+    ATTN_LAUNCH(KK_DOC_RANGES, st, doc_ranges_kernel<<<1, 1024, 0, st>>>(cu_seqlens, B, T, ds, de));
+    if (launch_status()) return ATTN_ECUDA;
+  }
+  // delta_kernel writes every row of Delta before the two passes read it.
+  float* delta = (float*)(ws + p.delta);
+  if (dtype == ATTN_F32) {
+    return D == 64 ? bwd_simt<float, 64>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, delta,
+                                         dq, dk, dv, B, H, T, scale, st)
+                   : bwd_simt<float, 128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, delta,
+                                          dq, dk, dv, B, H, T, scale, st);
+  }
+  return D == 64 ? bwd_simt<__nv_bfloat16, 64>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de,
+                                               delta, dq, dk, dv, B, H, T, scale, st)
+                 : bwd_simt<__nv_bfloat16, 128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de,
+                                                delta, dq, dk, dv, B, H, T, scale, st);
+}

@@ -72,6 +72,7 @@ extern "C" {
 #define ATTN_ECUDA (-5)         /* a CUDA launch or runtime call failed */
 #define ATTN_EDEVICE_INPUT (-6) /* device-detected malformed cu_seqlens */
 #define ATTN_ETIMEOUT (-7)      /* a bounded device-side wait gave up */
+#define ATTN_ESCRATCH (-8)      /* too large for attn_bwd_noalloc's fixed scratch array */
 
 /*
  * attn_fwd -- forward pass.
@@ -115,6 +116,40 @@ int attn_get_status(void* stream);
 
 /* Static, human-readable text for a return or status code. */
 const char* attn_error_string(int code);
+
+/*
+ * attn_bwd_noalloc -- the backward pass for callers that cannot allocate
+ * device memory. (The source pages have no counterpart: this is an
+ * integration variant, not part of the method.)
+ *
+ * Some callers cannot hand the library a workspace: code embedded in a host
+ * runtime that has already reserved the whole device for its own memory pool
+ * (so a cudaMalloc would fail or fight that pool), or code on a hot path where
+ * a cudaMalloc/cudaFree is not allowed because it can synchronise the device
+ * and stall every other stream. This entry point takes the same arguments as
+ * attn_bwd minus the workspace and calls no allocating function at all: its
+ * scratch (the per-row Delta_i and the per-token document ranges) lives in one
+ * static device array of ATTN_NOALLOC_SCRATCH_BYTES, which every GPU that
+ * loads the library holds until the process exits.
+ *
+ * It runs the CUDA-core (fp32 arithmetic) backward kernels, for either dtype,
+ * and needs 4*B*H*T + 8*B*T bytes of scratch (each part rounded up to 256);
+ * larger problems are rejected with ATTN_ESCRATCH before anything is launched.
+ * The first call on each device looks up the array's device address with
+ * cudaGetSymbolAddress (no allocation); make that first call before any stream
+ * capture. All calls share the one array and it keeps the previous call's
+ * contents; every byte a call reads is written earlier in the same call, so
+ * nothing needs clearing, but two calls that overlap on the GPU (on different
+ * streams, or from different threads) race on it and must be serialised by the
+ * caller. Other arguments, rules and return codes are those of attn_bwd.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
+int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                     const void* dO, const float* lse,
+                     const float* rope_cos, const float* rope_sin,
+                     const int32_t* cu_seqlens,
+                     int B, int H, int T, int D, float scale, int dtype,
+                     void* dq, void* dk, void* dv, void* stream);
 
 /*
  * Tracing aids (the source pages define no counterpart; they support
