@@ -8,6 +8,7 @@
 
 #include "attn.h"
 #include "common.cuh"
+#include "fwd_sm100.cuh"
 #include "prep.cuh"
 #include "simt.cuh"
 #include "trace.cuh"
@@ -21,6 +22,8 @@ inline size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct WsPlan {
   size_t doc_start = 0, doc_end = 0;  // int32 [B*T] each
   size_t delta = 0;                   // f32 [B*H*T] (backward)
+  size_t q16 = 0, k16 = 0;            // rotated q, k as 16-bit [B*H*T*D] each (bf16 storage)
+  size_t qfac = 0, kfac = 0;          // f32 [B*H*ceil(T/128)] tile factors (bf16 forward)
   size_t total = 0;
 };
 
@@ -33,16 +36,71 @@ bool sizes_ok(int B, int H, int T, int D) {
 }
 
 WsPlan plan(int B, int H, int T, int D, int dtype, int is_bwd) {
-  (void)D;
-  (void)dtype;
   WsPlan p;
   size_t off = 0;
-  const size_t bt = (size_t)B * T, rows = bt * H;
+  const size_t bt = (size_t)B * T, rows = bt * H, n = rows * D;
+  const size_t tiles = (size_t)B * H * ((T + 127) / 128);
   p.doc_start = off; off += round_up(bt * sizeof(int32_t));
   p.doc_end = off;   off += round_up(bt * sizeof(int32_t));
   if (is_bwd) { p.delta = off; off += round_up(rows * sizeof(float)); }
+  if (dtype == ATTN_BF16 && !is_bwd) {
+    p.q16 = off;  off += round_up(n * 2);
+    p.k16 = off;  off += round_up(n * 2);
+    p.qfac = off; off += round_up(tiles * sizeof(float));
+    p.kfac = off; off += round_up(tiles * sizeof(float));
+  }
   p.total = off;
   return p;
+}
+
+// ---- TMA descriptors (driver entry point fetched through the runtime) ----
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)f;
+  }
+  return fn;
+}
+
+// A [B*H][T][D] 16-bit tensor seen in boxes of 128 rows x 64 columns with the
+// 128-byte swizzle; rows past T read as zeros.
+bool make_tile_map(CUtensorMap* m, const void* base, bool is_f16, int D, int T, int BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, is_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Opt a kernel into its dynamic shared memory once per device.
+template <typename K>
+bool ensure_smem(K kernel, int bytes, bool* done_per_device) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!done_per_device[dev]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+      return false;
+    done_per_device[dev] = true;
+  }
+  return true;
 }
 
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
@@ -106,6 +164,53 @@ int bwd_simt(const void* q, const void* k, const void* v, const void* o, const v
   return launch_status();
 }
 
+template <int D>
+int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const float* rs,
+           const int32_t* ds, void* o, float* lse, int B, int H, int T, float scale, char* ws,
+           const WsPlan& wp, cudaStream_t st) {
+  using L = fwd100::Layout<D>;
+  const int nt = (T + 127) / 128, BH = B * H;
+  const void* qs = q;
+  const void* ks = k;
+  bool f16 = false;
+  float *qf = nullptr, *kf = nullptr;
+  if (rc) {
+    __half* qh = (__half*)(ws + wp.q16);
+    __half* kh = (__half*)(ws + wp.k16);
+    qf = (float*)(ws + wp.qfac);
+    kf = (float*)(ws + wp.kfac);
+    ATTN_LAUNCH(KK_ROPE_PREP, st,
+                rope_prep_kernel<__half, D, true><<<dim3(nt, BH, 2), 256, 0, st>>>(
+                    (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qh, kh, qf, kf,
+                    H, T, nt));
+    if (launch_status()) return ATTN_ECUDA;
+    qs = qh;
+    ks = kh;
+    f16 = true;
+  }
+  CUtensorMap mq, mk, mv;
+  if (!make_tile_map(&mq, qs, f16, D, T, BH) || !make_tile_map(&mk, ks, f16, D, T, BH) ||
+      !make_tile_map(&mv, v, false, D, T, BH))
+    return ATTN_ECUDA;
+  static bool smem_set[64] = {};
+  if (!ensure_smem(fwd100::fwd_kernel<D>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
+  fwd100::Params prm;
+  prm.T = T;
+  prm.H = H;
+  prm.BH = BH;
+  prm.n_qtiles = nt;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.idesc_s = sm100::idesc_f16(128, 128, !f16, !f16, false, false);
+  prm.q_fac = qf;
+  prm.k_fac = kf;
+  prm.doc_start = ds;
+  prm.o = (__nv_bfloat16*)o;
+  prm.lse = lse;
+  ATTN_LAUNCH(KK_FWD, st,
+              fwd100::fwd_kernel<D><<<(unsigned)(nt * BH), 192, L::kSmemAlloc, st>>>(mq, mk, mv, prm));
+  return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -139,9 +244,8 @@ int attn_fwd(const void* q, const void* k, const void* v, const float* rope_cos,
     return D == 64 ? fwd_simt<float, 64>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, T, scale, st)
                    : fwd_simt<float, 128>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, T, scale, st);
   }
-  return D == 64
-             ? fwd_simt<__nv_bfloat16, 64>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, T, scale, st)
-             : fwd_simt<__nv_bfloat16, 128>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, T, scale, st);
+  return D == 64 ? fwd_tc<64>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, T, scale, ws, p, st)
+                 : fwd_tc<128>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, T, scale, ws, p, st);
 }
 
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,

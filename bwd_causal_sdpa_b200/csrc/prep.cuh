@@ -2,6 +2,8 @@
 // backward's row term Delta_i = sum_d dO[i][d] * o[i][d].
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 // From cu_seqlens (over the flattened B*T token axis, end marker B*T) build,
@@ -72,4 +74,77 @@ __global__ void __launch_bounds__(256) delta_kernel(const TIO* __restrict__ o, c
   for (int c = 0; c < NC; ++c) s = fmaf(a[c], g[c], s);
   s = warp_sum(s);
   if (lane == 0) delta[row] = s;
+}
+
+// RoPE pre-pass for the tensor-core kernels: rotate q and k once (fp32
+// arithmetic, interleaved pairs at the token's document position) and store
+// the rotated tiles in the 16-bit type the MMAs read. blockIdx = (128-row
+// tile, b*H + h, 0 for q / 1 for k).
+//
+// kTileScale (forward, fp16 output): fp16 keeps 3 more mantissa bits than
+// bf16, which the lse bound needs, but has a narrow range; a tile whose
+// largest magnitude reaches 2^14 is multiplied by a power of two that brings
+// it into [2^14, 2^15), and fac[] receives the inverse factor (exact), which
+// the forward folds into its score scale. Without kTileScale (bf16 output)
+// values are stored as they are.
+template <typename OutT, int D, bool kTileScale>
+__global__ void __launch_bounds__(256) rope_prep_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+    const float* __restrict__ rc, const float* __restrict__ rs,
+    const int32_t* __restrict__ doc_start, OutT* __restrict__ qo, OutT* __restrict__ ko,
+    float* __restrict__ qfac, float* __restrict__ kfac, int H, int T, int ntiles) {
+  constexpr int CH = D / 8;              // 16-byte chunks per row
+  constexpr int PER = 128 * CH / 256;    // chunks per thread
+  const int tile = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
+  const __nv_bfloat16* src = which ? k : q;
+  OutT* dst = which ? ko : qo;
+  const int b = bh / H, row0 = b * T, t0 = tile * 128;
+  float v[PER][8];
+  float amax = 0.f;
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int idx = threadIdx.x + u * 256, r = idx / CH, c8 = idx % CH, t = t0 + r;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[u][e] = 0.f;
+    if (t < T) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(src + ((size_t)bh * T + t) * D + c8 * 8);
+      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[u][e] = __bfloat162float(h[e]);
+      const int pos = t - (doc_start ? doc_start[row0 + t] - row0 : 0);
+      rope_pairs<8, D>(v[u], rc, rs, pos, c8 * 8, false);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[u][e]));
+    }
+  }
+  float f = 1.f;
+  if constexpr (kTileScale) {
+    __shared__ float red[8];
+    amax = warp_max(amax);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
+    if (amax >= 16384.f && amax <= 3.0e38f) f = ldexpf(1.f, 14 - ilogbf(amax));
+    if (threadIdx.x == 0) (which ? kfac : qfac)[bh * ntiles + tile] = 1.f / f;
+  }
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int idx = threadIdx.x + u * 256, r = idx / CH, c8 = idx % CH, t = t0 + r;
+    if (t >= T) continue;
+    uint4 out;
+    uint32_t* w = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if constexpr (sizeof(OutT) == 2 && std::is_same<OutT, __half>::value) {
+        __half2 hv = __floats2half2_rn(v[u][2 * e] * f, v[u][2 * e + 1] * f);
+        w[e] = *reinterpret_cast<uint32_t*>(&hv);
+      } else {
+        __nv_bfloat162 hv = __floats2bfloat162_rn(v[u][2 * e] * f, v[u][2 * e + 1] * f);
+        w[e] = *reinterpret_cast<uint32_t*>(&hv);
+      }
+    }
+    *reinterpret_cast<uint4*>(dst + ((size_t)bh * T + t) * D + c8 * 8) = out;
+  }
 }
