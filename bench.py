@@ -337,7 +337,7 @@ def run_ours(args):
         kernels[name]["share"] = prof[name][1] / total_k if total_k else None
     if dom is not None:
         kd = kernels[dom]
-        simt = True  # the kernels below are the CUDA-core kernels until the tensor-core path lands
+        simt = w.dtype != "bf16"  # bf16 runs on the tensor cores; f32 on the CUDA cores
         if kd["bound"] == "tensor":
             achieved = kd["algorithmic"] / (kd["avg_ms"] / 1e3) / 1e12
             if simt:

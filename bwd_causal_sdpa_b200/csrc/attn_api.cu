@@ -8,6 +8,7 @@
 
 #include "attn.h"
 #include "common.cuh"
+#include "bwd_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "prep.cuh"
 #include "simt.cuh"
@@ -21,7 +22,9 @@ inline size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // Workspace layout (byte offsets from the caller's base pointer).
 struct WsPlan {
   size_t doc_start = 0, doc_end = 0;  // int32 [B*T] each
-  size_t delta = 0;                   // f32 [B*H*T] (backward)
+  size_t delta = 0;                   // f32 [B*H*T] (f32 backward) or [B*H*Tpad] (bf16 backward)
+  size_t lse2 = 0;                    // f32 [B*H*Tpad] lse*log2(e) (bf16 backward)
+  size_t dq_acc = 0;                  // f32 [B*H*T*D] dq accumulator (bf16 backward)
   size_t q16 = 0, k16 = 0;            // rotated q, k as 16-bit [B*H*T*D] each (bf16 storage)
   size_t qfac = 0, kfac = 0;          // f32 [B*H*ceil(T/128)] tile factors (bf16 forward)
   size_t total = 0;
@@ -40,9 +43,17 @@ WsPlan plan(int B, int H, int T, int D, int dtype, int is_bwd) {
   size_t off = 0;
   const size_t bt = (size_t)B * T, rows = bt * H, n = rows * D;
   const size_t tiles = (size_t)B * H * ((T + 127) / 128);
+  const size_t rows_pad = tiles * 128;
   p.doc_start = off; off += round_up(bt * sizeof(int32_t));
   p.doc_end = off;   off += round_up(bt * sizeof(int32_t));
-  if (is_bwd) { p.delta = off; off += round_up(rows * sizeof(float)); }
+  if (is_bwd && dtype == ATTN_F32) { p.delta = off; off += round_up(rows * sizeof(float)); }
+  if (is_bwd && dtype == ATTN_BF16) {
+    p.delta = off;  off += round_up(rows_pad * sizeof(float));
+    p.lse2 = off;   off += round_up(rows_pad * sizeof(float));
+    p.dq_acc = off; off += round_up(n * sizeof(float));
+    p.q16 = off;    off += round_up(n * 2);
+    p.k16 = off;    off += round_up(n * 2);
+  }
   if (dtype == ATTN_BF16 && !is_bwd) {
     p.q16 = off;  off += round_up(n * 2);
     p.k16 = off;  off += round_up(n * 2);
@@ -211,6 +222,69 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
   return launch_status();
 }
 
+template <int D>
+int bwd_tc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+           const float* lse, const float* rc, const float* rs, const int32_t* ds,
+           const int32_t* de, void* dq, void* dk, void* dv, int B, int H, int T, float scale,
+           char* ws, const WsPlan& wp, cudaStream_t st) {
+  using L = bwd100::Layout<D>;
+  const int nt = (T + 127) / 128, BH = B * H, Tpad = nt * 128;
+  const void* qs = q;
+  const void* ks = k;
+  if (rc) {
+    __nv_bfloat16* qr = (__nv_bfloat16*)(ws + wp.q16);
+    __nv_bfloat16* kr = (__nv_bfloat16*)(ws + wp.k16);
+    ATTN_LAUNCH(KK_ROPE_PREP, st,
+                rope_prep_kernel<__nv_bfloat16, D, false><<<dim3(nt, BH, 2), 256, 0, st>>>(
+                    (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qr, kr, nullptr,
+                    nullptr, H, T, nt));
+    if (launch_status()) return ATTN_ECUDA;
+    qs = qr;
+    ks = kr;
+  }
+  float* delta = (float*)(ws + wp.delta);
+  float* lse2 = (float*)(ws + wp.lse2);
+  float* dq_acc = (float*)(ws + wp.dq_acc);
+  const long rows_pad = (long)BH * Tpad;
+  ATTN_LAUNCH(KK_DELTA, st,
+              bwd_prep_kernel<D><<<(unsigned)((rows_pad + 7) / 8), 256, 0, st>>>(
+                  (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse, delta, lse2, dq_acc, T,
+                  Tpad, rows_pad));
+  if (launch_status()) return ATTN_ECUDA;
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_tile_map(&mq, qs, false, D, T, BH) || !make_tile_map(&mk, ks, false, D, T, BH) ||
+      !make_tile_map(&mv, v, false, D, T, BH) || !make_tile_map(&mo, dO, false, D, T, BH))
+    return ATTN_ECUDA;
+  static bool smem_set[64] = {};
+  if (!ensure_smem(bwd100::dkdv_kernel<D>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
+  bwd100::Params prm;
+  prm.T = T;
+  prm.H = H;
+  prm.BH = BH;
+  prm.n_tiles = nt;
+  prm.Tpad = Tpad;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.scale = scale;
+  prm.lse2 = lse2;
+  prm.delta = delta;
+  prm.doc_start = ds;
+  prm.doc_end = de;
+  prm.rope_cos = rc;
+  prm.rope_sin = rs;
+  prm.dq_acc = dq_acc;
+  prm.dk = (__nv_bfloat16*)dk;
+  prm.dv = (__nv_bfloat16*)dv;
+  ATTN_LAUNCH(KK_DKDV, st,
+              bwd100::dkdv_kernel<D><<<(unsigned)(nt * BH), 192, L::kSmemAlloc, st>>>(mq, mk, mv,
+                                                                                       mo, prm));
+  if (launch_status()) return ATTN_ECUDA;
+  const long n8 = (long)BH * T * D / 8;
+  ATTN_LAUNCH(KK_DQ_FINALIZE, st,
+              dq_finalize_kernel<D><<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
+                  dq_acc, rc, rs, ds, (__nv_bfloat16*)dq, H, T, scale, n8));
+  return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -276,10 +350,10 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
                    : bwd_simt<float, 128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, delta,
                                           dq, dk, dv, B, H, T, scale, st);
   }
-  return D == 64 ? bwd_simt<__nv_bfloat16, 64>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de,
-                                               delta, dq, dk, dv, B, H, T, scale, st)
-                 : bwd_simt<__nv_bfloat16, 128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de,
-                                                delta, dq, dk, dv, B, H, T, scale, st);
+  return D == 64 ? bwd_tc<64>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, dq, dk, dv, B, H,
+                              T, scale, ws, p, st)
+                 : bwd_tc<128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, dq, dk, dv, B, H,
+                               T, scale, ws, p, st);
 }
 
 int attn_get_status(void* stream) {

@@ -1,0 +1,379 @@
+// bwd_sm100.cuh -- tensor-core (tcgen05) attention backward, key-tile
+// parallel, for bf16 storage.
+//
+// One CTA owns one 128-key tile of one (b, h) slice; K and V stay in shared
+// memory and the dK, dV accumulators stay in TMEM while the query tiles that
+// can see these keys stream through (from the diagonal tile to the end of the
+// last key's document). Per query tile i (keys are TMEM lanes, queries are
+// columns):
+//   S^T  = K Q^T           (TMEM)      dP^T = V dO^T        (TMEM)
+//   P^T  = exp2(S^T * scale*log2e - lse2_i), masked; written back to TMEM (bf16)
+//   dV  += P^T dO          (A = P^T from TMEM)
+//   dS^T = P^T (dP^T - Delta_i), written to shared memory (bf16, 128-B swizzle)
+//   dK  += dS^T Q          (A = dS^T read K-major from shared memory)
+//   dQ_i = dS K            (A = the same tile read MN-major), into the dP^T
+//                          columns, then added to the fp32 dq accumulator in
+//                          global memory with vector atomics.
+// Warps 0-3 do the elementwise work (thread t = key row t = TMEM lane t, and
+// thread t = query row t when reading dQ_i); warp 4 streams Q and dO with TMA
+// (two stages) after loading K and V once; warp 5 owns TMEM and issues MMAs.
+// dK is scaled and rotated back (R^T) in the epilogue; dq is finished by a
+// separate kernel once every key tile has added its part.
+//
+// Sources (page, section): ARK README, "Backward pass (AutoGrad)" (attention
+// gradients inside training); Forge README, finding 3 (key-tile-parallel dK/dV
+// kernels, the dK/dV split and register pressure) and "What this is" (fused
+// flash-attention backward). The dQ accumulation by atomics follows the
+// measurement contract's "atomic dQ" option. Tiling, TMEM plan and warp roles
+// are this library's own.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace bwd100 {
+
+using namespace sm100;
+
+template <int D>
+struct Layout {
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kBlockBytes = 128 * 128;
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kTileBytes;
+  static constexpr int kQ = kV + kTileBytes;          // 2 stages
+  static constexpr int kDO = kQ + 2 * kTileBytes;     // 2 stages
+  static constexpr int kDS = kDO + 2 * kTileBytes;    // 128 keys x 128 queries bf16
+  static constexpr int kBars = kDS + 128 * 128 * 2;
+  static constexpr int bKV = 0;
+  static constexpr int bQFull = 1, bQEmpty = 3, bDOFull = 5, bDOEmpty = 7;  // 2 each
+  static constexpr int bSFull = 9, bPFull = 10, bDPFull = 11, bDSFull = 12, bDVDone = 13,
+                       bDQFull = 14, bDQFree = 15, bFinal = 16;
+  static constexpr int kNumBars = 17;
+  static constexpr int kMisc = kBars + kNumBars * 8;
+  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kSmemAlloc = kBytes + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  // TMEM columns: S^T (P^T over its first half), dP^T (dQ_i after dS), dV, dK
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+};
+
+struct Params {
+  int T, H, BH, n_tiles, Tpad;
+  float scale_log2;  // scale * log2(e)
+  float scale;
+  const float* lse2;       // [BH][Tpad] lse * log2(e), zero-padded
+  const float* delta;      // [BH][Tpad], zero-padded
+  const int32_t* doc_start;
+  const int32_t* doc_end;  // flattened, or null
+  const float* rope_cos;   // [T][D/2] or null
+  const float* rope_sin;
+  float* dq_acc;           // [BH][T][D] fp32
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+};
+
+// Byte offset of 16-byte chunk `ch` (0..7 within a 64-column block) of row r
+// in a 128-byte-swizzled tile block.
+__device__ __forceinline__ uint32_t sw128(int r, int ch) {
+  return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4));
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                const Params p) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb0 = (raw + 1023u) & ~1023u;
+  uint8_t* sg = smem_raw + (sb0 - raw);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sg + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sg + L::kMisc + 4);
+  auto bar = [&](int i) -> uint32_t { return sb0 + L::kBars + 8u * i; };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = p.T;
+  // Flattened grid, heaviest key tiles (the earliest, which see the most
+  // query tiles) first.
+  const int bh = (int)blockIdx.x % p.BH, b = bh / p.H;
+  const int kt = (int)blockIdx.x / p.BH;
+  const int j0 = kt * 128;
+  const int row0 = b * T;
+  const int jlast = min(j0 + 127, T - 1);
+  const int q_end = p.doc_end ? p.doc_end[row0 + jlast] - row0 : T;  // exclusive
+  const int qt0 = kt;
+  const int n_q = (q_end + 127) / 128 - qt0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::bKV), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(L::bQFull + s), 1);
+      mbar_init(bar(L::bQEmpty + s), 1);
+      mbar_init(bar(L::bDOFull + s), 1);
+      mbar_init(bar(L::bDOEmpty + s), 1);
+    }
+    mbar_init(bar(L::bSFull), 1);
+    mbar_init(bar(L::bPFull), 128);
+    mbar_init(bar(L::bDPFull), 1);
+    mbar_init(bar(L::bDSFull), 128);
+    mbar_init(bar(L::bDVDone), 1);
+    mbar_init(bar(L::bDQFull), 1);
+    mbar_init(bar(L::bDQFree), 128);
+    mbar_init(bar(L::bFinal), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(sb0 + L::kMisc, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      prefetch_tensor_map(&tmQ);
+      prefetch_tensor_map(&tmK);
+      prefetch_tensor_map(&tmV);
+      prefetch_tensor_map(&tmDO);
+      mbar_arrive_expect_tx(bar(L::bKV), 2 * L::kTileBytes);
+      for (int cb = 0; cb < D / 64; ++cb) {
+        tma_load_3d(sb0 + L::kK + cb * L::kBlockBytes, &tmK, bar(L::bKV), cb * 64, j0, bh);
+        tma_load_3d(sb0 + L::kV + cb * L::kBlockBytes, &tmV, bar(L::bKV), cb * 64, j0, bh);
+      }
+      for (int it = 0; it < n_q; ++it) {
+        const int st = it & 1, round = it >> 1;
+        const int qrow = (qt0 + it) * 128;
+        if (it >= 2 && !mbar_wait(bar(L::bQEmpty + st), (round - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(L::bQFull + st), L::kTileBytes);
+        for (int cb = 0; cb < D / 64; ++cb)
+          tma_load_3d(sb0 + L::kQ + st * L::kTileBytes + cb * L::kBlockBytes, &tmQ,
+                      bar(L::bQFull + st), cb * 64, qrow, bh);
+        if (it >= 2 && !mbar_wait(bar(L::bDOEmpty + st), (round - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(L::bDOFull + st), L::kTileBytes);
+        for (int cb = 0; cb < D / 64; ++cb)
+          tma_load_3d(sb0 + L::kDO + st * L::kTileBytes + cb * L::kBlockBytes, &tmDO,
+                      bar(L::bDOFull + st), cb * 64, qrow, bh);
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_f16(128, 128, true, true, false, false);
+      constexpr uint32_t id_dv = idesc_f16(128, D, true, true, false, true);
+      constexpr uint32_t id_dk = idesc_f16(128, D, true, true, false, true);
+      constexpr uint32_t id_dq = idesc_f16(128, D, true, true, true, true);
+      const uint32_t tS = tmem + L::kColS, tDP = tmem + L::kColDP;
+      const uint32_t tDV = tmem + L::kColDV, tDK = tmem + L::kColDK;
+      bool ok = mbar_wait(bar(L::bKV), 0, abort_flag);
+      for (int it = 0; ok && it < n_q; ++it) {
+        const int st = it & 1, ph = it & 1, pph = (it - 1) & 1;
+        const uint32_t qb = sb0 + L::kQ + st * L::kTileBytes;
+        const uint32_t ob = sb0 + L::kDO + st * L::kTileBytes;
+        // S^T = K Q^T (the TMEM columns are free once dV of the previous tile ran)
+        if (!mbar_wait(bar(L::bQFull + st), (it >> 1) & 1, abort_flag)) break;
+        if (it > 0 && !mbar_wait(bar(L::bDVDone), pph, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
+          mma_ss(tS, smem_desc_sw128(sb0 + L::kK + off, 16, 1024),
+                 smem_desc_sw128(qb + off, 16, 1024), id_s, kk > 0);
+        }
+        mma_commit(bar(L::bSFull));
+        // dP^T = V dO^T (its columns held dQ of the previous tile until read out)
+        if (!mbar_wait(bar(L::bDOFull + st), (it >> 1) & 1, abort_flag)) break;
+        if (it > 0 && !mbar_wait(bar(L::bDQFree), pph, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
+          mma_ss(tDP, smem_desc_sw128(sb0 + L::kV + off, 16, 1024),
+                 smem_desc_sw128(ob + off, 16, 1024), id_s, kk > 0);
+        }
+        mma_commit(bar(L::bDPFull));
+        // dV += P^T dO
+        if (!mbar_wait(bar(L::bPFull), ph, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tDV, tS + kk * 8, smem_desc_sw128(ob + kk * 2048, L::kBlockBytes, 1024), id_dv,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar(L::bDVDone));
+        mma_commit(bar(L::bDOEmpty + st));
+        // dK += dS^T Q ; dQ_i = dS K
+        if (!mbar_wait(bar(L::bDSFull), ph, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t ds = sb0 + L::kDS;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tDK, smem_desc_sw128(ds + (kk >> 2) * L::kBlockBytes + (kk & 3) * 32, 16, 1024),
+                 smem_desc_sw128(qb + kk * 2048, L::kBlockBytes, 1024), id_dk,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tDP, smem_desc_sw128(ds + kk * 2048, L::kBlockBytes, 1024),
+                 smem_desc_sw128(sb0 + L::kK + kk * 2048, L::kBlockBytes, 1024), id_dq, kk > 0);
+        mma_commit(bar(L::bDQFull));
+        mma_commit(bar(L::bQEmpty + st));
+        if (it == n_q - 1) mma_commit(bar(L::bFinal));
+      }
+    }
+  } else {
+    // ---------------- elementwise warps 0-3 ----------------
+    const int r = threadIdx.x;  // TMEM lane: key row (S^T, dP^T, dK, dV) or query row (dQ_i)
+    const int j = j0 + r;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int de_j = (j < T) ? (p.doc_end ? p.doc_end[row0 + j] - row0 : T) : T;
+    const float* lse2_bh = p.lse2 + (size_t)bh * p.Tpad;
+    const float* delta_bh = p.delta + (size_t)bh * p.Tpad;
+    const uint32_t tS = tmem + lane_base + L::kColS;
+    const uint32_t tDP = tmem + lane_base + L::kColDP;
+    uint8_t* dsrow = sg + L::kDS;
+    bool ok = true;
+    for (int it = 0; it < n_q; ++it) {
+      const int ph = it & 1;
+      const int i0 = (qt0 + it) * 128;
+      const bool need_mask = (i0 < j) || (i0 + 127 >= de_j);
+      // ---- P^T ----
+      if (!mbar_wait(bar(L::bSFull), ph, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t s[32];
+        tmem_ld32(tS + 32 * c, s);
+        const float4* l4 = reinterpret_cast<const float4*>(lse2_bh + i0 + 32 * c);
+        float lv[32];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float4 t4 = l4[e];
+          lv[4 * e] = t4.x; lv[4 * e + 1] = t4.y; lv[4 * e + 2] = t4.z; lv[4 * e + 3] = t4.w;
+        }
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int i_a = i0 + 32 * c + 2 * e;
+          float p0 = ex2(fmaf(__uint_as_float(s[2 * e]), p.scale_log2, -lv[2 * e]));
+          float p1 = ex2(fmaf(__uint_as_float(s[2 * e + 1]), p.scale_log2, -lv[2 * e + 1]));
+          if (need_mask) {
+            if (i_a < j || i_a >= de_j) p0 = 0.f;
+            if (i_a + 1 < j || i_a + 1 >= de_j) p1 = 0.f;
+          }
+          pk[16 * c + e] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tS + 16 * c, pk + 16 * c);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(L::bPFull));
+      // ---- dS^T ----
+      if (!mbar_wait(bar(L::bDPFull), ph, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t dpv[32];
+        tmem_ld32(tDP + 32 * c, dpv);
+        const float4* d4 = reinterpret_cast<const float4*>(delta_bh + i0 + 32 * c);
+        float dl[32];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float4 t4 = d4[e];
+          dl[4 * e] = t4.x; dl[4 * e + 1] = t4.y; dl[4 * e + 2] = t4.z; dl[4 * e + 3] = t4.w;
+        }
+        tmem_wait_ld();
+        uint32_t dsk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          __nv_bfloat162 pp = *reinterpret_cast<const __nv_bfloat162*>(&pk[16 * c + e]);
+          const float a0 = __low2float(pp) * (__uint_as_float(dpv[2 * e]) - dl[2 * e]);
+          const float a1 = __high2float(pp) * (__uint_as_float(dpv[2 * e + 1]) - dl[2 * e + 1]);
+          dsk[e] = pack_bf16(a0, a1);
+        }
+        // row r of the dS^T tile, query columns [32c, 32c + 32): block c/2,
+        // 16-byte chunks 4*(c%2) .. 4*(c%2)+3
+        uint8_t* blk = dsrow + (c >> 1) * L::kBlockBytes;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          *reinterpret_cast<uint4*>(blk + sw128(r, 4 * (c & 1) + e)) =
+              make_uint4(dsk[4 * e], dsk[4 * e + 1], dsk[4 * e + 2], dsk[4 * e + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(L::bDSFull));
+      // ---- dQ_i: read out of TMEM (lane = query row) and accumulate ----
+      if (!mbar_wait(bar(L::bDQFull), ph, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const int iq = i0 + r;
+      float* dqrow = p.dq_acc + ((size_t)bh * T + min(iq, T - 1)) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tDP + 32 * c, v);
+        tmem_wait_ld();
+        if (iq < T) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            atomicAdd(reinterpret_cast<float4*>(dqrow + 32 * c + 4 * e),
+                      make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                  __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(L::bDQFree));
+    }
+    // ---- epilogue: dK = R^T (scale * dK_r), dV ----
+    if (ok && mbar_wait(bar(L::bFinal), 0, abort_flag)) {
+      tc_fence_after();
+      const int jj = min(j, T - 1);
+      const int pos = jj - (p.doc_start ? p.doc_start[row0 + jj] - row0 : 0);
+      __nv_bfloat16* dkrow = p.dk + ((size_t)bh * T + jj) * D;
+      __nv_bfloat16* dvrow = p.dv + ((size_t)bh * T + jj) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + L::kColDK + 32 * c, v);
+        tmem_wait_ld();
+        float f[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]) * p.scale;
+        if (p.rope_cos) rope_pairs<32, D>(f, p.rope_cos, p.rope_sin, pos, 32 * c, true);
+        if (j < T) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            reinterpret_cast<uint4*>(dkrow + 32 * c)[e] =
+                make_uint4(pack_bf16(f[8 * e], f[8 * e + 1]), pack_bf16(f[8 * e + 2], f[8 * e + 3]),
+                           pack_bf16(f[8 * e + 4], f[8 * e + 5]), pack_bf16(f[8 * e + 6], f[8 * e + 7]));
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + L::kColDV + 32 * c, v);
+        tmem_wait_ld();
+        if (j < T) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            reinterpret_cast<uint4*>(dvrow + 32 * c)[e] = make_uint4(
+                pack_bf16(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
+                pack_bf16(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
+                pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
+                pack_bf16(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace bwd100

@@ -148,3 +148,63 @@ __global__ void __launch_bounds__(256) rope_prep_kernel(
     *reinterpret_cast<uint4*>(dst + ((size_t)bh * T + t) * D + c8 * 8) = out;
   }
 }
+
+// Backward preprocessing for the tensor-core path, one warp per row of the
+// tile-padded [B*H][ntiles*128] view: Delta_i = sum_d dO[i][d] * o[i][d] and
+// lse2_i = lse_i * log2(e) (both 0 for padding rows t >= T, so the main
+// kernel's per-tile loads never leave the arrays), and the fp32 dq
+// accumulator row is zeroed.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(
+    const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+    const float* __restrict__ lse, float* __restrict__ delta_pad, float* __restrict__ lse2_pad,
+    float* __restrict__ dq_acc, int T, int Tpad, long rows_pad) {
+  constexpr int NC = D / 32;
+  const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows_pad) return;
+  const long bh = row / Tpad;
+  const int t = (int)(row - bh * Tpad);
+  float s = 0.f;
+  if (t < T) {
+    const long r = bh * T + t;
+    float a[NC], g[NC];
+    load_vec<NC>(o + r * D + lane * NC, a);
+    load_vec<NC>(dO + r * D + lane * NC, g);
+#pragma unroll
+    for (int c = 0; c < NC; ++c) s = fmaf(a[c], g[c], s);
+    s = warp_sum(s);
+    const float z[NC] = {};
+    store_vec<NC>(dq_acc + r * D + lane * NC, z);
+  }
+  if (lane == 0) {
+    delta_pad[row] = s;
+    lse2_pad[row] = t < T ? lse[bh * T + t] * 1.4426950408889634f : 0.f;
+  }
+}
+
+// dq = R(pos)^T (scale * dq_acc), stored as bf16; one thread per 8 values.
+template <int D>
+__global__ void __launch_bounds__(256) dq_finalize_kernel(
+    const float* __restrict__ dq_acc, const float* __restrict__ rc, const float* __restrict__ rs,
+    const int32_t* __restrict__ doc_start, __nv_bfloat16* __restrict__ dq, int H, int T,
+    float scale, long n8) {
+  const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n8) return;
+  const long e0 = idx * 8;
+  const long row = e0 / D;  // bh*T + t
+  const int d0 = (int)(e0 - row * D);
+  const int t = (int)(row % T);
+  const int b = (int)((row / T) / H);
+  float v[8];
+  load_vec<4>(dq_acc + e0, v);
+  load_vec<4>(dq_acc + e0 + 4, v + 4);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) v[e] *= scale;
+  if (rc) {
+    const int pos = t - (doc_start ? doc_start[b * T + t] - b * T : 0);
+    rope_pairs<8, D>(v, rc, rs, pos, d0, true);
+  }
+  store_vec<4>(dq + e0, v);
+  store_vec<4>(dq + e0 + 4, v + 4);
+}
