@@ -100,6 +100,20 @@ bool make_tile_map(CUtensorMap* m, const void* base, bool is_f16, int D, int T, 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The fp32 [B*H][T][D] dq accumulator seen in boxes of 32 rows x 32 columns
+// (128-byte swizzle) for tensor reduce-add; rows past T are clipped.
+bool make_acc_map(CUtensorMap* m, float* base, int D, int T, int BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)T * D * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Opt a kernel into its dynamic shared memory once per device.
 template <typename K>
 bool ensure_smem(K kernel, int bytes, bool* done_per_device) {
@@ -251,9 +265,10 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
                   (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse, delta, lse2, dq_acc, T,
                   Tpad, rows_pad));
   if (launch_status()) return ATTN_ECUDA;
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv, mo, mdq;
   if (!make_tile_map(&mq, qs, false, D, T, BH) || !make_tile_map(&mk, ks, false, D, T, BH) ||
-      !make_tile_map(&mv, v, false, D, T, BH) || !make_tile_map(&mo, dO, false, D, T, BH))
+      !make_tile_map(&mv, v, false, D, T, BH) || !make_tile_map(&mo, dO, false, D, T, BH) ||
+      !make_acc_map(&mdq, dq_acc, D, T, BH))
     return ATTN_ECUDA;
   static bool smem_set[64] = {};
   if (!ensure_smem(bwd100::dkdv_kernel<D>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
@@ -275,8 +290,8 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   prm.dk = (__nv_bfloat16*)dk;
   prm.dv = (__nv_bfloat16*)dv;
   ATTN_LAUNCH(KK_DKDV, st,
-              bwd100::dkdv_kernel<D><<<(unsigned)(nt * BH), 192, L::kSmemAlloc, st>>>(mq, mk, mv,
-                                                                                       mo, prm));
+              bwd100::dkdv_kernel<D><<<(unsigned)(nt * BH), L::kThreads, L::kSmemAlloc, st>>>(
+                  mq, mk, mv, mo, mdq, prm));
   if (launch_status()) return ATTN_ECUDA;
   const long n8 = (long)BH * T * D / 8;
   ATTN_LAUNCH(KK_DQ_FINALIZE, st,

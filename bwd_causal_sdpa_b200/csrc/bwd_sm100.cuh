@@ -12,20 +12,25 @@
 //   dS^T = P^T (dP^T - Delta_i), written to shared memory (bf16, 128-B swizzle)
 //   dK  += dS^T Q          (A = dS^T read K-major from shared memory)
 //   dQ_i = dS K            (A = the same tile read MN-major), into the dP^T
-//                          columns, then added to the fp32 dq accumulator in
-//                          global memory with vector atomics.
-// Warps 0-3 do the elementwise work (thread t = key row t = TMEM lane t, and
-// thread t = query row t when reading dQ_i); warp 4 streams Q and dO with TMA
-// (two stages) after loading K and V once; warp 5 owns TMEM and issues MMAs.
-// dK is scaled and rotated back (R^T) in the epilogue; dq is finished by a
-// separate kernel once every key tile has added its part.
+//                          columns; read out, staged in shared memory and
+//                          added to the fp32 dq accumulator in global memory by
+//                          bulk reduce-add operations of the TMA unit.
+// Warps 0-7 do the elementwise work in two warpgroups: warpgroup g takes query
+// columns [64g, 64g+64) of S^T and dP^T (its P^T goes to the first half of its
+// own S^T columns, so the two never touch each other's TMEM) and feature
+// columns [g*D/2, (g+1)*D/2) of dQ_i, dK and dV; thread t of a warpgroup owns
+// TMEM lane t (a key row, or a query row for dQ_i). Warp 8 streams Q (two
+// stages, with lse2 and Delta riding on the same barrier) and dO with TMA
+// after loading K and V once; warp 9 owns TMEM and issues the MMAs. dK is
+// scaled and rotated back (R^T) in the epilogue; dq is finished by a separate
+// kernel once every key tile has added its part.
 //
 // Sources (page, section): ARK README, "Backward pass (AutoGrad)" (attention
 // gradients inside training); Forge README, finding 3 (key-tile-parallel dK/dV
 // kernels, the dK/dV split and register pressure) and "What this is" (fused
-// flash-attention backward). The dQ accumulation by atomics follows the
-// measurement contract's "atomic dQ" option. Tiling, TMEM plan and warp roles
-// are this library's own.
+// flash-attention backward). The dQ accumulation follows the measurement
+// contract's "atomic dQ" option (reduce-add in L2). Tiling, TMEM plan and warp
+// roles are this library's own.
 #pragma once
 
 #include "sm100.cuh"
@@ -38,23 +43,28 @@ template <int D>
 struct Layout {
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr int kBlockBytes = 128 * 128;
+  static constexpr int kDOStages = (D == 128) ? 1 : 2;
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTileBytes;
-  static constexpr int kQ = kV + kTileBytes;          // 2 stages
-  static constexpr int kDO = kQ + 2 * kTileBytes;     // 2 stages
-  static constexpr int kDS = kDO + 2 * kTileBytes;    // 128 keys x 128 queries bf16
-  static constexpr int kBars = kDS + 128 * 128 * 2;
+  static constexpr int kQ = kV + kTileBytes;                  // 2 stages
+  static constexpr int kDO = kQ + 2 * kTileBytes;             // kDOStages stages
+  static constexpr int kDS = kDO + kDOStages * kTileBytes;    // 128 keys x 128 queries bf16
+  static constexpr int kLD = kDS + 128 * 128 * 2;             // 2 x {lse2[128], delta[128]} f32
+  static constexpr int kBars = kLD + 2 * 1024;
   static constexpr int bKV = 0;
   static constexpr int bQFull = 1, bQEmpty = 3, bDOFull = 5, bDOEmpty = 7;  // 2 each
   static constexpr int bSFull = 9, bPFull = 10, bDPFull = 11, bDSFull = 12, bDVDone = 13,
-                       bDQFull = 14, bDQFree = 15, bFinal = 16;
-  static constexpr int kNumBars = 17;
+                       bDQFull = 14, bDQFree = 15, bFinal = 16, bStageFree = 17;
+  static constexpr int kNumBars = 18;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kSmemAlloc = kBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
-  // TMEM columns: S^T (P^T over its first half), dP^T (dQ_i after dS), dV, dK
+  // TMEM columns: S^T (P^T over the first half of each warpgroup's 64), dP^T
+  // (dQ_i after dS), dV, dK
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+  static constexpr int kThreads = 320;
+  static constexpr int kEwThreads = 256;  // elementwise warps 0-7
 };
 
 struct Params {
@@ -79,10 +89,10 @@ __device__ __forceinline__ uint32_t sw128(int r, int ch) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                const Params p) {
+                const __grid_constant__ CUtensorMap tmDQ, const Params p) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -114,17 +124,18 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(bar(L::bDOEmpty + s), 1);
     }
     mbar_init(bar(L::bSFull), 1);
-    mbar_init(bar(L::bPFull), 128);
+    mbar_init(bar(L::bPFull), L::kEwThreads);
     mbar_init(bar(L::bDPFull), 1);
-    mbar_init(bar(L::bDSFull), 128);
+    mbar_init(bar(L::bDSFull), L::kEwThreads);
     mbar_init(bar(L::bDVDone), 1);
     mbar_init(bar(L::bDQFull), 1);
-    mbar_init(bar(L::bDQFree), 128);
+    mbar_init(bar(L::bDQFree), L::kEwThreads);
     mbar_init(bar(L::bFinal), 1);
+    mbar_init(bar(L::bStageFree), L::kEwThreads);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(sb0 + L::kMisc, L::kTmemCols);
     tmem_relinquish();
   }
@@ -133,7 +144,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       prefetch_tensor_map(&tmQ);
@@ -145,22 +156,29 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_3d(sb0 + L::kK + cb * L::kBlockBytes, &tmK, bar(L::bKV), cb * 64, j0, bh);
         tma_load_3d(sb0 + L::kV + cb * L::kBlockBytes, &tmV, bar(L::bKV), cb * 64, j0, bh);
       }
+      const float* lse2_bh = p.lse2 + (size_t)bh * p.Tpad;
+      const float* delta_bh = p.delta + (size_t)bh * p.Tpad;
       for (int it = 0; it < n_q; ++it) {
-        const int st = it & 1, round = it >> 1;
+        const int st = it & 1;
+        const int so = it % L::kDOStages;
         const int qrow = (qt0 + it) * 128;
-        if (it >= 2 && !mbar_wait(bar(L::bQEmpty + st), (round - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(L::bQFull + st), L::kTileBytes);
+        if (it >= 2 && !mbar_wait(bar(L::bQEmpty + st), ((it >> 1) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(L::bQFull + st), L::kTileBytes + 1024);
         for (int cb = 0; cb < D / 64; ++cb)
           tma_load_3d(sb0 + L::kQ + st * L::kTileBytes + cb * L::kBlockBytes, &tmQ,
                       bar(L::bQFull + st), cb * 64, qrow, bh);
-        if (it >= 2 && !mbar_wait(bar(L::bDOEmpty + st), (round - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(L::bDOFull + st), L::kTileBytes);
+        bulk_load(sb0 + L::kLD + st * 1024, lse2_bh + qrow, 512, bar(L::bQFull + st));
+        bulk_load(sb0 + L::kLD + st * 1024 + 512, delta_bh + qrow, 512, bar(L::bQFull + st));
+        if (it >= L::kDOStages &&
+            !mbar_wait(bar(L::bDOEmpty + so), ((it / L::kDOStages) - 1) & 1, abort_flag))
+          break;
+        mbar_arrive_expect_tx(bar(L::bDOFull + so), L::kTileBytes);
         for (int cb = 0; cb < D / 64; ++cb)
-          tma_load_3d(sb0 + L::kDO + st * L::kTileBytes + cb * L::kBlockBytes, &tmDO,
-                      bar(L::bDOFull + st), cb * 64, qrow, bh);
+          tma_load_3d(sb0 + L::kDO + so * L::kTileBytes + cb * L::kBlockBytes, &tmDO,
+                      bar(L::bDOFull + so), cb * 64, qrow, bh);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f16(128, 128, true, true, false, false);
@@ -171,9 +189,9 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t tDV = tmem + L::kColDV, tDK = tmem + L::kColDK;
       bool ok = mbar_wait(bar(L::bKV), 0, abort_flag);
       for (int it = 0; ok && it < n_q; ++it) {
-        const int st = it & 1, ph = it & 1, pph = (it - 1) & 1;
+        const int st = it & 1, so = it % L::kDOStages, ph = it & 1, pph = (it - 1) & 1;
         const uint32_t qb = sb0 + L::kQ + st * L::kTileBytes;
-        const uint32_t ob = sb0 + L::kDO + st * L::kTileBytes;
+        const uint32_t ob = sb0 + L::kDO + so * L::kTileBytes;
         // S^T = K Q^T (the TMEM columns are free once dV of the previous tile ran)
         if (!mbar_wait(bar(L::bQFull + st), (it >> 1) & 1, abort_flag)) break;
         if (it > 0 && !mbar_wait(bar(L::bDVDone), pph, abort_flag)) break;
@@ -186,7 +204,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         mma_commit(bar(L::bSFull));
         // dP^T = V dO^T (its columns held dQ of the previous tile until read out)
-        if (!mbar_wait(bar(L::bDOFull + st), (it >> 1) & 1, abort_flag)) break;
+        if (!mbar_wait(bar(L::bDOFull + so), (it / L::kDOStages) & 1, abort_flag)) break;
         if (it > 0 && !mbar_wait(bar(L::bDQFree), pph, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
@@ -196,15 +214,17 @@ __global__ void __launch_bounds__(192, 1)
                  smem_desc_sw128(ob + off, 16, 1024), id_s, kk > 0);
         }
         mma_commit(bar(L::bDPFull));
-        // dV += P^T dO
+        // dV += P^T dO; P^T of query columns [64g, 64g+64) sits in TMEM
+        // columns [64g, 64g+32)
         if (!mbar_wait(bar(L::bPFull), ph, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tDV, tS + kk * 8, smem_desc_sw128(ob + kk * 2048, L::kBlockBytes, 1024), id_dv,
+          mma_ts(tDV, tS + 64 * (kk >> 2) + 8 * (kk & 3),
+                 smem_desc_sw128(ob + kk * 2048, L::kBlockBytes, 1024), id_dv,
                  (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar(L::bDVDone));
-        mma_commit(bar(L::bDOEmpty + st));
+        mma_commit(bar(L::bDOEmpty + so));
         // dK += dS^T Q ; dQ_i = dS K
         if (!mbar_wait(bar(L::bDSFull), ph, abort_flag)) break;
         tc_fence_after();
@@ -224,40 +244,48 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    // ---------------- elementwise warps 0-3 ----------------
-    const int r = threadIdx.x;  // TMEM lane: key row (S^T, dP^T, dK, dV) or query row (dQ_i)
+    // ---------------- elementwise warps 0-7 ----------------
+    const int wg = warp >> 2, sub = warp & 3;
+    const int r = sub * 32 + lane;  // TMEM lane: key row (S^T, dP^T, dK, dV) or query row (dQ_i)
     const int j = j0 + r;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int qc0 = 64 * wg;        // query columns of S^T / dP^T handled here
+    const int dc0 = wg * (D / 2);   // feature columns of dQ_i / dK / dV handled here
+    const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
     const int de_j = (j < T) ? (p.doc_end ? p.doc_end[row0 + j] - row0 : T) : T;
-    const float* lse2_bh = p.lse2 + (size_t)bh * p.Tpad;
-    const float* delta_bh = p.delta + (size_t)bh * p.Tpad;
     const uint32_t tS = tmem + lane_base + L::kColS;
     const uint32_t tDP = tmem + lane_base + L::kColDP;
-    uint8_t* dsrow = sg + L::kDS;
+    uint8_t* dsb = sg + L::kDS;
+    uint8_t* stage = sg + L::kDS + warp * 4096;  // dQ staging box (reuses the dS tile)
     bool ok = true;
     for (int it = 0; it < n_q; ++it) {
-      const int ph = it & 1;
+      const int ph = it & 1, st = it & 1;
       const int i0 = (qt0 + it) * 128;
-      const bool need_mask = (i0 < j) || (i0 + 127 >= de_j);
+      const bool need_mask = (i0 + qc0 < j) || (i0 + qc0 + 63 >= de_j);
+      const float* sl = reinterpret_cast<const float*>(sg + L::kLD + st * 1024);
+      const float* sd = sl + 128;
       // ---- P^T ----
-      if (!mbar_wait(bar(L::bSFull), ph, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(L::bQFull + st), (it >> 1) & 1, abort_flag) ||
+          !mbar_wait(bar(L::bSFull), ph, abort_flag)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      uint32_t pk[64];
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
+        const int col = qc0 + 32 * c;
         uint32_t s[32];
-        tmem_ld32(tS + 32 * c, s);
-        const float4* l4 = reinterpret_cast<const float4*>(lse2_bh + i0 + 32 * c);
+        tmem_ld32(tS + col, s);
         float lv[32];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float4 t4 = l4[e];
+          const float4 t4 = reinterpret_cast<const float4*>(sl + col)[e];
           lv[4 * e] = t4.x; lv[4 * e + 1] = t4.y; lv[4 * e + 2] = t4.z; lv[4 * e + 3] = t4.w;
         }
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int i_a = i0 + 32 * c + 2 * e;
+          const int i_a = i0 + col + 2 * e;
           float p0 = ex2(fmaf(__uint_as_float(s[2 * e]), p.scale_log2, -lv[2 * e]));
           float p1 = ex2(fmaf(__uint_as_float(s[2 * e + 1]), p.scale_log2, -lv[2 * e + 1]));
           if (need_mask) {
@@ -266,23 +294,30 @@ __global__ void __launch_bounds__(192, 1)
           }
           pk[16 * c + e] = pack_bf16(p0, p1);
         }
-        tmem_st16(tS + 16 * c, pk + 16 * c);
+        tmem_st16(tS + qc0 + 16 * c, pk + 16 * c);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(L::bPFull));
-      // ---- dS^T ----
-      if (!mbar_wait(bar(L::bDPFull), ph, abort_flag)) { ok = false; break; }
+      // ---- dS^T (the dS tile doubled as dQ staging: every thread's bulk reads
+      // of it must be done; a bounded barrier over the elementwise warps) ----
+      bulk_wait_group_read0();
+      mbar_arrive(bar(L::bStageFree));
+      if (!mbar_wait(bar(L::bStageFree), ph, abort_flag) ||
+          !mbar_wait(bar(L::bDPFull), ph, abort_flag)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
+        const int col = qc0 + 32 * c;
         uint32_t dpv[32];
-        tmem_ld32(tDP + 32 * c, dpv);
-        const float4* d4 = reinterpret_cast<const float4*>(delta_bh + i0 + 32 * c);
+        tmem_ld32(tDP + col, dpv);
         float dl[32];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float4 t4 = d4[e];
+          const float4 t4 = reinterpret_cast<const float4*>(sd + col)[e];
           dl[4 * e] = t4.x; dl[4 * e + 1] = t4.y; dl[4 * e + 2] = t4.z; dl[4 * e + 3] = t4.w;
         }
         tmem_wait_ld();
@@ -294,38 +329,51 @@ __global__ void __launch_bounds__(192, 1)
           const float a1 = __high2float(pp) * (__uint_as_float(dpv[2 * e + 1]) - dl[2 * e + 1]);
           dsk[e] = pack_bf16(a0, a1);
         }
-        // row r of the dS^T tile, query columns [32c, 32c + 32): block c/2,
-        // 16-byte chunks 4*(c%2) .. 4*(c%2)+3
-        uint8_t* blk = dsrow + (c >> 1) * L::kBlockBytes;
+        // row r of the dS^T tile, query columns [col, col+32): block wg,
+        // 16-byte chunks 4c .. 4c+3
+        uint8_t* blk = dsb + wg * L::kBlockBytes;
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          *reinterpret_cast<uint4*>(blk + sw128(r, 4 * (c & 1) + e)) =
+          *reinterpret_cast<uint4*>(blk + sw128(r, 4 * c + e)) =
               make_uint4(dsk[4 * e], dsk[4 * e + 1], dsk[4 * e + 2], dsk[4 * e + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(L::bDSFull));
-      // ---- dQ_i: read out of TMEM (lane = query row) and accumulate ----
+      // ---- dQ_i (lane = query row): release TMEM first, then reduce into global ----
       if (!mbar_wait(bar(L::bDQFull), ph, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const int iq = i0 + r;
-      float* dqrow = p.dq_acc + ((size_t)bh * T + min(iq, T - 1)) * D;
+      constexpr int NQC = D / 64;  // 32-column chunks per warpgroup
+      uint32_t dqv[NQC][32];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tDP + 32 * c, v);
-        tmem_wait_ld();
-        if (iq < T) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            atomicAdd(reinterpret_cast<float4*>(dqrow + 32 * c + 4 * e),
-                      make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                  __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
-        }
-      }
+      for (int c = 0; c < NQC; ++c) tmem_ld32(tDP + dc0 + 32 * c, dqv[c]);
+      tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(L::bDQFree));
+      // Every thread has consumed the dS tile (dq_full implies the dK and dQ
+      // MMAs are done), so it now serves as staging: one 32x32 fp32 box per
+      // warp in the 128-byte-swizzled layout (conflict-free stores), added
+      // to the accumulator by one tensor reduce-add per box.
+      const uint32_t stage_s = smem_u32(stage);
+#pragma unroll
+      for (int c = 0; c < NQC; ++c) {
+        if (c > 0) {
+          if (lane == 0) bulk_wait_group_read0();
+          __syncwarp();
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          *reinterpret_cast<uint4*>(stage + sw128(lane, e)) =
+              make_uint4(dqv[c][4 * e], dqv[c][4 * e + 1], dqv[c][4 * e + 2], dqv[c][4 * e + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && i0 + 32 * sub < T) {  // rows past T are clipped by the map
+          tma_reduce_add_3d(&tmDQ, stage_s, dc0 + 32 * c, i0 + 32 * sub, bh);
+          bulk_commit_group();
+        }
+      }
     }
+    bulk_wait_group0();
     // ---- epilogue: dK = R^T (scale * dK_r), dV ----
     if (ok && mbar_wait(bar(L::bFinal), 0, abort_flag)) {
       tc_fence_after();
@@ -334,31 +382,33 @@ __global__ void __launch_bounds__(192, 1)
       __nv_bfloat16* dkrow = p.dk + ((size_t)bh * T + jj) * D;
       __nv_bfloat16* dvrow = p.dv + ((size_t)bh * T + jj) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
+        const int col = dc0 + 32 * c;
         uint32_t v[32];
-        tmem_ld32(tmem + lane_base + L::kColDK + 32 * c, v);
+        tmem_ld32(tmem + lane_base + L::kColDK + col, v);
         tmem_wait_ld();
         float f[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]) * p.scale;
-        if (p.rope_cos) rope_pairs<32, D>(f, p.rope_cos, p.rope_sin, pos, 32 * c, true);
+        if (p.rope_cos) rope_pairs<32, D>(f, p.rope_cos, p.rope_sin, pos, col, true);
         if (j < T) {
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            reinterpret_cast<uint4*>(dkrow + 32 * c)[e] =
+            reinterpret_cast<uint4*>(dkrow + col)[e] =
                 make_uint4(pack_bf16(f[8 * e], f[8 * e + 1]), pack_bf16(f[8 * e + 2], f[8 * e + 3]),
                            pack_bf16(f[8 * e + 4], f[8 * e + 5]), pack_bf16(f[8 * e + 6], f[8 * e + 7]));
         }
       }
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
+        const int col = dc0 + 32 * c;
         uint32_t v[32];
-        tmem_ld32(tmem + lane_base + L::kColDV + 32 * c, v);
+        tmem_ld32(tmem + lane_base + L::kColDV + col, v);
         tmem_wait_ld();
         if (j < T) {
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            reinterpret_cast<uint4*>(dvrow + 32 * c)[e] = make_uint4(
+            reinterpret_cast<uint4*>(dvrow + col)[e] = make_uint4(
                 pack_bf16(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
                 pack_bf16(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
                 pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
@@ -370,7 +420,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }
