@@ -43,6 +43,7 @@ _SIGNATURES = {
     "attn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
     "attn_get_status": (_I, [_P]),
     "attn_error_string": (ctypes.c_char_p, [_I]),
+    "attn_exp2_selftest": (_I, [_P, _P, _I, _P]),
     "attn_launch_count": (ctypes.c_ulonglong, []),
     "attn_profile_enable": (_I, [_I]),
     "attn_profile_kinds": (_I, []),
@@ -128,6 +129,10 @@ def attn_get_status(stream=None) -> int:
 
 def attn_error_string(code: int) -> str:
     return error_string(code)
+
+
+def attn_exp2_selftest(x, y, n, stream=None) -> int:
+    return int(_lib.attn_exp2_selftest(_ptr(x), _ptr(y), int(n), _stream(stream)))
 
 
 def attn_launch_count() -> int:

@@ -300,6 +300,11 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   return launch_status();
 }
 
+__global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = sm100::exp2_fma(x[i]);
+}
+
 }  // namespace
 
 extern "C" {
@@ -400,6 +405,13 @@ const char* attn_error_string(int code) {
 }
 
 unsigned long long attn_launch_count(void) { return trace::launches(); }
+
+int attn_exp2_selftest(const float* x, float* y, int n, void* stream) {
+  if (!x || !y || n < 0) return ATTN_EINVAL;
+  if (n == 0) return ATTN_OK;
+  exp2_selftest_kernel<<<(n + 255) / 256, 256, 0, (cudaStream_t)stream>>>(x, y, n);
+  return launch_status();
+}
 
 int attn_profile_enable(int on) { return trace::enable(on != 0) == 0 ? ATTN_OK : ATTN_ECUDA; }
 

@@ -15,13 +15,14 @@
 //                          columns; read out, staged in shared memory and
 //                          added to the fp32 dq accumulator in global memory by
 //                          bulk reduce-add operations of the TMA unit.
-// Warps 0-7 do the elementwise work in two warpgroups: warpgroup g takes query
-// columns [64g, 64g+64) of S^T and dP^T (its P^T goes to the first half of its
-// own S^T columns, so the two never touch each other's TMEM) and feature
-// columns [g*D/2, (g+1)*D/2) of dQ_i, dK and dV; thread t of a warpgroup owns
-// TMEM lane t (a key row, or a query row for dQ_i). Warp 8 streams Q (two
-// stages, with lse2 and Delta riding on the same barrier) and dO with TMA
-// after loading K and V once; warp 9 owns TMEM and issues the MMAs. dK is
+// The elementwise work runs in kNWG warpgroups (4 at D = 128, 2 at D = 64):
+// warpgroup g takes query columns [g*kQC, (g+1)*kQC) of S^T and dP^T (its P^T
+// goes to the first half of its own S^T columns, so warpgroups never touch
+// each other's TMEM) and feature columns [g*kDC, (g+1)*kDC) of dQ_i, dK and
+// dV; thread t of a warpgroup owns TMEM lane t (a key row, or a query row for
+// dQ_i). The next warp streams Q (two stages, with lse2 and Delta riding on
+// the same barrier) and dO with TMA after loading K and V once; the last warp
+// owns TMEM and issues the MMAs. dK is
 // scaled and rotated back (R^T) in the epilogue; dq is finished by a separate
 // kernel once every key tile has added its part.
 //
@@ -50,7 +51,10 @@ struct Layout {
   static constexpr int kDO = kQ + 2 * kTileBytes;             // kDOStages stages
   static constexpr int kDS = kDO + kDOStages * kTileBytes;    // 128 keys x 128 queries bf16
   static constexpr int kLD = kDS + 128 * 128 * 2;             // 2 x {lse2[128], delta[128]} f32
-  static constexpr int kBars = kLD + 2 * 1024;
+  // dQ_i staging: 32 x 32 fp32 boxes (4 KB), D/32 x 4 of them per tile: the
+  // first 8 in the (then free) dS tile, the rest (D = 128) in this area.
+  static constexpr int kXS = kLD + 2 * 1024;
+  static constexpr int kBars = kXS + (D == 128 ? 8 * 4096 : 0);
   static constexpr int bKV = 0;
   static constexpr int bQFull = 1, bQEmpty = 3, bDOFull = 5, bDOEmpty = 7;  // 2 each
   static constexpr int bSFull = 9, bPFull = 10, bDPFull = 11, bDSFull = 12, bDVDone = 13,
@@ -58,13 +62,22 @@ struct Layout {
   static constexpr int kNumBars = 18;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
-  static constexpr int kSmemAlloc = kBytes + 1024;
+  // The dynamic shared-memory window starts 1024-byte aligned on sm_100 (after
+  // the 1 KB the system reserves per block); the kernel checks this and
+  // reports an error instead of running misaligned.
+  static constexpr int kSmemAlloc = kBytes;
   static constexpr uint32_t kTmemCols = 512;
   // TMEM columns: S^T (P^T over the first half of each warpgroup's 64), dP^T
   // (dQ_i after dS), dV, dK
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
-  static constexpr int kThreads = 320;
-  static constexpr int kEwThreads = 256;  // elementwise warps 0-7
+  // Elementwise warpgroups: 4 at D = 128 (16 warps), 2 at D = 64; each owns
+  // kQC query columns of S^T / dP^T and kDC feature columns of dQ_i, dK, dV.
+  static constexpr int kNWG = (D == 128) ? 4 : 2;
+  static constexpr int kQC = 128 / kNWG;
+  static constexpr int kDC = D / kNWG;
+  static constexpr int kEwThreads = 128 * kNWG;
+  static constexpr int kProducerWarp = 4 * kNWG, kMmaWarp = 4 * kNWG + 1;
+  static constexpr int kThreads = kEwThreads + 64;
 };
 
 struct Params {
@@ -89,15 +102,18 @@ __device__ __forceinline__ uint32_t sw128(int r, int ch) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                 const __grid_constant__ CUtensorMap tmDQ, const Params p) {
   using L = Layout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t sb0 = (raw + 1023u) & ~1023u;
-  uint8_t* sg = smem_raw + (sb0 - raw);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t sb0 = smem_u32(smem_raw);
+  if (sb0 & 1023u) {  // uniform across the CTA: nothing has been issued yet
+    if (threadIdx.x == 0) report_status(ATTN_ECUDA_LAYOUT);
+    return;
+  }
+  uint8_t* sg = smem_raw;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sg + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sg + L::kMisc + 4);
   auto bar = [&](int i) -> uint32_t { return sb0 + L::kBars + 8u * i; };
@@ -135,7 +151,7 @@ __global__ void __launch_bounds__(320, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == L::kMmaWarp) {
     tmem_alloc(sb0 + L::kMisc, L::kTmemCols);
     tmem_relinquish();
   }
@@ -144,7 +160,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == L::kProducerWarp) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       prefetch_tensor_map(&tmQ);
@@ -178,8 +194,13 @@ __global__ void __launch_bounds__(320, 1)
                       bar(L::bDOFull + so), cb * 64, qrow, bh);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == L::kMmaWarp) {
     // ---------------- MMA issuer ----------------
+    // Issue order per query tile i: dV(i), S(i+1), dK(i), dQ(i), dP(i+1), so
+    // the tensor pipe has S(i+1) to run while the elementwise warps form dS(i),
+    // and dK/dQ(i) while they form P(i+1). TMEM reuse: S(i+1) waits for dV(i)
+    // (which reads P^T(i) from the S columns); dP(i+1) waits until dQ(i) has
+    // been read out of the dP columns.
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f16(128, 128, true, true, false, false);
       constexpr uint32_t id_dv = idesc_f16(128, D, true, true, false, true);
@@ -187,44 +208,55 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t id_dq = idesc_f16(128, D, true, true, true, true);
       const uint32_t tS = tmem + L::kColS, tDP = tmem + L::kColDP;
       const uint32_t tDV = tmem + L::kColDV, tDK = tmem + L::kColDK;
-      bool ok = mbar_wait(bar(L::bKV), 0, abort_flag);
-      for (int it = 0; ok && it < n_q; ++it) {
-        const int st = it & 1, so = it % L::kDOStages, ph = it & 1, pph = (it - 1) & 1;
-        const uint32_t qb = sb0 + L::kQ + st * L::kTileBytes;
-        const uint32_t ob = sb0 + L::kDO + so * L::kTileBytes;
-        // S^T = K Q^T (the TMEM columns are free once dV of the previous tile ran)
-        if (!mbar_wait(bar(L::bQFull + st), (it >> 1) & 1, abort_flag)) break;
-        if (it > 0 && !mbar_wait(bar(L::bDVDone), pph, abort_flag)) break;
+      auto qbuf = [&](int i) -> uint32_t { return sb0 + L::kQ + (i & 1) * L::kTileBytes; };
+      auto obuf = [&](int i) -> uint32_t {
+        return sb0 + L::kDO + (i % L::kDOStages) * L::kTileBytes;
+      };
+      // S^T(i) = K Q(i)^T
+      auto issue_S = [&](int i) -> bool {
+        if (!mbar_wait(bar(L::bQFull + (i & 1)), (i >> 1) & 1, abort_flag)) return false;
+        if (i > 0 && !mbar_wait(bar(L::bDVDone), (i - 1) & 1, abort_flag)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
           mma_ss(tS, smem_desc_sw128(sb0 + L::kK + off, 16, 1024),
-                 smem_desc_sw128(qb + off, 16, 1024), id_s, kk > 0);
+                 smem_desc_sw128(qbuf(i) + off, 16, 1024), id_s, kk > 0);
         }
         mma_commit(bar(L::bSFull));
-        // dP^T = V dO^T (its columns held dQ of the previous tile until read out)
-        if (!mbar_wait(bar(L::bDOFull + so), (it / L::kDOStages) & 1, abort_flag)) break;
-        if (it > 0 && !mbar_wait(bar(L::bDQFree), pph, abort_flag)) break;
+        return true;
+      };
+      // dP^T(i) = V dO(i)^T
+      auto issue_dP = [&](int i) -> bool {
+        if (!mbar_wait(bar(L::bDOFull + i % L::kDOStages), (i / L::kDOStages) & 1, abort_flag))
+          return false;
+        if (i > 0 && !mbar_wait(bar(L::bDQFree), (i - 1) & 1, abort_flag)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
           mma_ss(tDP, smem_desc_sw128(sb0 + L::kV + off, 16, 1024),
-                 smem_desc_sw128(ob + off, 16, 1024), id_s, kk > 0);
+                 smem_desc_sw128(obuf(i) + off, 16, 1024), id_s, kk > 0);
         }
         mma_commit(bar(L::bDPFull));
-        // dV += P^T dO; P^T of query columns [64g, 64g+64) sits in TMEM
-        // columns [64g, 64g+32)
+        return true;
+      };
+      bool ok = mbar_wait(bar(L::bKV), 0, abort_flag) && issue_S(0) && issue_dP(0);
+      for (int it = 0; ok && it < n_q; ++it) {
+        const int ph = it & 1;
+        // dV += P^T dO; P^T of warpgroup g's query columns [g*kQC, (g+1)*kQC)
+        // sits in TMEM columns [g*kQC, g*kQC + kQC/2), so the 16 queries of
+        // k-step kk start at column 8*kk + (kQC/2) * (16*kk / kQC)
         if (!mbar_wait(bar(L::bPFull), ph, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tDV, tS + 64 * (kk >> 2) + 8 * (kk & 3),
-                 smem_desc_sw128(ob + kk * 2048, L::kBlockBytes, 1024), id_dv,
+          mma_ts(tDV, tS + 8 * kk + (L::kQC / 2) * ((16 * kk) / L::kQC),
+                 smem_desc_sw128(obuf(it) + kk * 2048, L::kBlockBytes, 1024), id_dv,
                  (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar(L::bDVDone));
-        mma_commit(bar(L::bDOEmpty + so));
+        mma_commit(bar(L::bDOEmpty + it % L::kDOStages));
+        if (it + 1 < n_q && !issue_S(it + 1)) break;
         // dK += dS^T Q ; dQ_i = dS K
         if (!mbar_wait(bar(L::bDSFull), ph, abort_flag)) break;
         tc_fence_after();
@@ -232,118 +264,119 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ss(tDK, smem_desc_sw128(ds + (kk >> 2) * L::kBlockBytes + (kk & 3) * 32, 16, 1024),
-                 smem_desc_sw128(qb + kk * 2048, L::kBlockBytes, 1024), id_dk,
+                 smem_desc_sw128(qbuf(it) + kk * 2048, L::kBlockBytes, 1024), id_dk,
                  (it > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ss(tDP, smem_desc_sw128(ds + kk * 2048, L::kBlockBytes, 1024),
                  smem_desc_sw128(sb0 + L::kK + kk * 2048, L::kBlockBytes, 1024), id_dq, kk > 0);
         mma_commit(bar(L::bDQFull));
-        mma_commit(bar(L::bQEmpty + st));
+        mma_commit(bar(L::bQEmpty + (it & 1)));
         if (it == n_q - 1) mma_commit(bar(L::bFinal));
+        if (it + 1 < n_q && !issue_dP(it + 1)) break;
       }
     }
   } else {
-    // ---------------- elementwise warps 0-7 ----------------
+    // ---------------- elementwise warps ----------------
+    constexpr int QC = L::kQC, DC = L::kDC;
     const int wg = warp >> 2, sub = warp & 3;
     const int r = sub * 32 + lane;  // TMEM lane: key row (S^T, dP^T, dK, dV) or query row (dQ_i)
     const int j = j0 + r;
-    const int qc0 = 64 * wg;        // query columns of S^T / dP^T handled here
-    const int dc0 = wg * (D / 2);   // feature columns of dQ_i / dK / dV handled here
+    const int qc0 = QC * wg;        // query columns of S^T / dP^T handled here
+    const int dc0 = DC * wg;        // feature columns of dQ_i / dK / dV handled here
     const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
     const int de_j = (j < T) ? (p.doc_end ? p.doc_end[row0 + j] - row0 : T) : T;
     const uint32_t tS = tmem + lane_base + L::kColS;
     const uint32_t tDP = tmem + lane_base + L::kColDP;
     uint8_t* dsb = sg + L::kDS;
-    uint8_t* stage = sg + L::kDS + warp * 4096;  // dQ staging box (reuses the dS tile)
-    bool ok = true;
-    for (int it = 0; it < n_q; ++it) {
-      const int ph = it & 1, st = it & 1;
-      const int i0 = (qt0 + it) * 128;
-      const bool need_mask = (i0 + qc0 < j) || (i0 + qc0 + 63 >= de_j);
-      const float* sl = reinterpret_cast<const float*>(sg + L::kLD + st * 1024);
-      const float* sd = sl + 128;
-      // ---- P^T ----
-      if (!mbar_wait(bar(L::bQFull + st), (it >> 1) & 1, abort_flag) ||
-          !mbar_wait(bar(L::bSFull), ph, abort_flag)) {
-        ok = false;
-        break;
-      }
+    float pf[QC];  // P^T of this thread's key row, query columns [qc0, qc0 + QC)
+    // ---- P^T(i) = exp2(S^T scale log2e - lse2), masked; bf16 copy to TMEM ----
+    auto phase_P = [&](int i) -> bool {
+      const int i0 = (qt0 + i) * 128;
+      const bool need_mask = (i0 + qc0 < j) || (i0 + qc0 + QC - 1 >= de_j);
+      const float* sl = reinterpret_cast<const float*>(sg + L::kLD + (i & 1) * 1024);
+      if (!mbar_wait(bar(L::bQFull + (i & 1)), (i >> 1) & 1, abort_flag) ||
+          !mbar_wait(bar(L::bSFull), i & 1, abort_flag))
+        return false;
       tc_fence_after();
-      uint32_t pk[32];
+      uint32_t s[QC];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < QC / 32; ++c) tmem_ld32(tS + qc0 + 32 * c, s + 32 * c);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < QC / 32; ++c) {
         const int col = qc0 + 32 * c;
-        uint32_t s[32];
-        tmem_ld32(tS + col, s);
-        float lv[32];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float4 t4 = reinterpret_cast<const float4*>(sl + col)[e];
-          lv[4 * e] = t4.x; lv[4 * e + 1] = t4.y; lv[4 * e + 2] = t4.z; lv[4 * e + 3] = t4.w;
-        }
-        tmem_wait_ld();
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
+          const float2 lv = reinterpret_cast<const float2*>(sl + col)[e];
           const int i_a = i0 + col + 2 * e;
-          float p0 = ex2(fmaf(__uint_as_float(s[2 * e]), p.scale_log2, -lv[2 * e]));
-          float p1 = ex2(fmaf(__uint_as_float(s[2 * e + 1]), p.scale_log2, -lv[2 * e + 1]));
+          // about a third of the exponentials go to the FMA pipe
+          const float x0 = fmaf(__uint_as_float(s[32 * c + 2 * e]), p.scale_log2, -lv.x);
+          const float x1 = fmaf(__uint_as_float(s[32 * c + 2 * e + 1]), p.scale_log2, -lv.y);
+          float p0 = (e % 3 == 2) ? exp2_fma(x0) : ex2(x0);
+          float p1 = (e % 3 == 2) ? exp2_fma(x1) : ex2(x1);
           if (need_mask) {
             if (i_a < j || i_a >= de_j) p0 = 0.f;
             if (i_a + 1 < j || i_a + 1 >= de_j) p1 = 0.f;
           }
-          pk[16 * c + e] = pack_bf16(p0, p1);
+          pf[32 * c + 2 * e] = p0;
+          pf[32 * c + 2 * e + 1] = p1;
+          pk[e] = pack_bf16(p0, p1);
         }
-        tmem_st16(tS + qc0 + 16 * c, pk + 16 * c);
+        tmem_st16(tS + qc0 + 16 * c, pk);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(L::bPFull));
-      // ---- dS^T (the dS tile doubled as dQ staging: every thread's bulk reads
-      // of it must be done; a bounded barrier over the elementwise warps) ----
+      return true;
+    };
+    // ---- dS^T(i) = P^T (dP^T - Delta) into the shared dS tile ----
+    auto phase_dS = [&](int i) -> bool {
+      const float* sd = reinterpret_cast<const float*>(sg + L::kLD + (i & 1) * 1024) + 128;
+      // The dS tile doubled as dQ staging for tile i-1: every thread's bulk
+      // reads of it must be done (a bounded barrier over the elementwise warps).
       bulk_wait_group_read0();
       mbar_arrive(bar(L::bStageFree));
-      if (!mbar_wait(bar(L::bStageFree), ph, abort_flag) ||
-          !mbar_wait(bar(L::bDPFull), ph, abort_flag)) {
-        ok = false;
-        break;
-      }
+      if (!mbar_wait(bar(L::bStageFree), i & 1, abort_flag) ||
+          !mbar_wait(bar(L::bDPFull), i & 1, abort_flag))
+        return false;
       tc_fence_after();
+      uint32_t dpv[QC];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < QC / 32; ++c) tmem_ld32(tDP + qc0 + 32 * c, dpv + 32 * c);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < QC / 32; ++c) {
         const int col = qc0 + 32 * c;
-        uint32_t dpv[32];
-        tmem_ld32(tDP + col, dpv);
-        float dl[32];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float4 t4 = reinterpret_cast<const float4*>(sd + col)[e];
-          dl[4 * e] = t4.x; dl[4 * e + 1] = t4.y; dl[4 * e + 2] = t4.z; dl[4 * e + 3] = t4.w;
-        }
-        tmem_wait_ld();
         uint32_t dsk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          __nv_bfloat162 pp = *reinterpret_cast<const __nv_bfloat162*>(&pk[16 * c + e]);
-          const float a0 = __low2float(pp) * (__uint_as_float(dpv[2 * e]) - dl[2 * e]);
-          const float a1 = __high2float(pp) * (__uint_as_float(dpv[2 * e + 1]) - dl[2 * e + 1]);
+          const float2 dl = reinterpret_cast<const float2*>(sd + col)[e];
+          const float a0 = pf[32 * c + 2 * e] * (__uint_as_float(dpv[32 * c + 2 * e]) - dl.x);
+          const float a1 = pf[32 * c + 2 * e + 1] * (__uint_as_float(dpv[32 * c + 2 * e + 1]) - dl.y);
           dsk[e] = pack_bf16(a0, a1);
         }
-        // row r of the dS^T tile, query columns [col, col+32): block wg,
-        // 16-byte chunks 4c .. 4c+3
-        uint8_t* blk = dsb + wg * L::kBlockBytes;
+        // row r of the dS^T tile, query columns [col, col+32): block col/64,
+        // 16-byte chunks (col%64)/8 .. +3
+        uint8_t* blk = dsb + (col >> 6) * L::kBlockBytes;
+        const int ch0 = (col & 63) >> 3;
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          *reinterpret_cast<uint4*>(blk + sw128(r, 4 * c + e)) =
+          *reinterpret_cast<uint4*>(blk + sw128(r, ch0 + e)) =
               make_uint4(dsk[4 * e], dsk[4 * e + 1], dsk[4 * e + 2], dsk[4 * e + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(L::bDSFull));
-      // ---- dQ_i (lane = query row): release TMEM first, then reduce into global ----
-      if (!mbar_wait(bar(L::bDQFull), ph, abort_flag)) { ok = false; break; }
+      return true;
+    };
+    // ---- dQ_i (lane = query row): release TMEM first, then reduce into global ----
+    auto phase_dQ = [&](int i) -> bool {
+      const int i0 = (qt0 + i) * 128;
+      if (!mbar_wait(bar(L::bDQFull), i & 1, abort_flag)) return false;
       tc_fence_after();
-      constexpr int NQC = D / 64;  // 32-column chunks per warpgroup
+      constexpr int NQC = DC / 32;  // 32-column chunks per warpgroup
       uint32_t dqv[NQC][32];
 #pragma unroll
       for (int c = 0; c < NQC; ++c) tmem_ld32(tDP + dc0 + 32 * c, dqv[c]);
@@ -352,26 +385,34 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(bar(L::bDQFree));
       // Every thread has consumed the dS tile (dq_full implies the dK and dQ
       // MMAs are done), so it now serves as staging: one 32x32 fp32 box per
-      // warp in the 128-byte-swizzled layout (conflict-free stores), added
-      // to the accumulator by one tensor reduce-add per box.
-      const uint32_t stage_s = smem_u32(stage);
+      // warp and chunk in the 128-byte-swizzled layout (conflict-free stores),
+      // each added to the accumulator by one tensor reduce-add.
 #pragma unroll
       for (int c = 0; c < NQC; ++c) {
-        if (c > 0) {
-          if (lane == 0) bulk_wait_group_read0();
-          __syncwarp();
-        }
+        const int box = warp * NQC + c;
+        uint8_t* bx = (box < 8) ? sg + L::kDS + box * 4096 : sg + L::kXS + (box - 8) * 4096;
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          *reinterpret_cast<uint4*>(stage + sw128(lane, e)) =
+          *reinterpret_cast<uint4*>(bx + sw128(lane, e)) =
               make_uint4(dqv[c][4 * e], dqv[c][4 * e + 1], dqv[c][4 * e + 2], dqv[c][4 * e + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && i0 + 32 * sub < T) {  // rows past T are clipped by the map
-          tma_reduce_add_3d(&tmDQ, stage_s, dc0 + 32 * c, i0 + 32 * sub, bh);
-          bulk_commit_group();
-        }
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && i0 + 32 * sub < T) {  // rows past T are clipped by the map
+#pragma unroll
+        for (int c = 0; c < NQC; ++c) {
+          const int box = warp * NQC + c;
+          const uint32_t bx = (box < 8) ? sb0 + L::kDS + box * 4096 : sb0 + L::kXS + (box - 8) * 4096;
+          tma_reduce_add_3d(&tmDQ, bx, dc0 + 32 * c, i0 + 32 * sub, bh);
+        }
+        bulk_commit_group();
+      }
+      return true;
+    };
+    // Order: P(0); then per tile i: dS(i), P(i+1), dQ(i).
+    bool ok = phase_P(0);
+    for (int it = 0; ok && it < n_q; ++it) {
+      ok = phase_dS(it) && (it + 1 >= n_q || phase_P(it + 1)) && phase_dQ(it);
     }
     bulk_wait_group0();
     // ---- epilogue: dK = R^T (scale * dK_r), dV ----
@@ -382,7 +423,7 @@ __global__ void __launch_bounds__(320, 1)
       __nv_bfloat16* dkrow = p.dk + ((size_t)bh * T + jj) * D;
       __nv_bfloat16* dvrow = p.dv + ((size_t)bh * T + jj) * D;
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
+      for (int c = 0; c < DC / 32; ++c) {
         const int col = dc0 + 32 * c;
         uint32_t v[32];
         tmem_ld32(tmem + lane_base + L::kColDK + col, v);
@@ -400,7 +441,7 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
+      for (int c = 0; c < DC / 32; ++c) {
         const int col = dc0 + 32 * c;
         uint32_t v[32];
         tmem_ld32(tmem + lane_base + L::kColDV + col, v);
@@ -420,7 +461,7 @@ __global__ void __launch_bounds__(320, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == L::kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }

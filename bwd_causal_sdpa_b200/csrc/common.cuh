@@ -13,6 +13,10 @@
 // and clears it.
 __device__ int g_attn_status;
 
+// Internal status: a kernel found its shared-memory window misaligned for the
+// 128-byte swizzle and did nothing (reported to callers as ATTN_ECUDA).
+#define ATTN_ECUDA_LAYOUT ATTN_ECUDA
+
 __device__ __forceinline__ void report_status(int code) {
   atomicCAS(&g_attn_status, 0, code);
 }

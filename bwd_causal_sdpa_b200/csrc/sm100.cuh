@@ -259,6 +259,23 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^x on the FMA pipe (to take load off the MUFU unit): x = n + f with
+// n = round(x) from the 1.5*2^23 magic-add trick, 2^f from a degree-3
+// polynomial on [-1/2, 1/2] (coefficients from csrc/fit_exp2_poly.py, a
+// near-minimax fit of the relative error: max 1.0e-4 in float32), and n added
+// to the exponent field. Inputs below -126 give a value below 2^-125 (treated
+// as zero by every use here); x must not be NaN.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;   // 1.5 * 2^23
+  const float n = t - 12582912.f;   // round(x)
+  const float f = x - n;            // [-1/2, 1/2]
+  float p = fmaf(5.500892922e-02f, f, 2.422109693e-01f);
+  p = fmaf(p, f, 6.932829022e-01f);
+  p = fmaf(p, f, 1.0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

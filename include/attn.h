@@ -170,6 +170,12 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
  * Returns ATTN_OK, ATTN_EINVAL (kind out of range or a null output pointer)
  * or ATTN_ECUDA.
  */
+/* attn_exp2_selftest: y[i] = the forward/backward kernels' software 2^x
+ * (FMA-pipe polynomial) of x[i], for 0 <= i < n; x, y device f32 arrays,
+ * asynchronous on `stream`. A test hook for checking that routine against
+ * CUDA's exp2f. Returns ATTN_OK, ATTN_EINVAL or ATTN_ECUDA. */
+int attn_exp2_selftest(const float* x, float* y, int n, void* stream);
+
 unsigned long long attn_launch_count(void);
 int attn_profile_enable(int on);
 int attn_profile_kinds(void);
