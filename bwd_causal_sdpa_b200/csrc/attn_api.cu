@@ -220,9 +220,11 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
   static bool smem_set[64] = {};
   if (!ensure_smem(fwd100::fwd_kernel<D>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
   fwd100::Params prm;
+  const int n_pairs = (nt + 1) / 2;
   prm.T = T;
   prm.H = H;
   prm.BH = BH;
+  prm.n_pairs = n_pairs;
   prm.n_qtiles = nt;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.idesc_s = sm100::idesc_f16(128, 128, !f16, !f16, false, false);
@@ -232,7 +234,8 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
   prm.o = (__nv_bfloat16*)o;
   prm.lse = lse;
   ATTN_LAUNCH(KK_FWD, st,
-              fwd100::fwd_kernel<D><<<(unsigned)(nt * BH), 192, L::kSmemAlloc, st>>>(mq, mk, mv, prm));
+              fwd100::fwd_kernel<D><<<(unsigned)(n_pairs * BH), L::kThreads, L::kSmemAlloc, st>>>(
+                  mq, mk, mv, prm));
   return launch_status();
 }
 

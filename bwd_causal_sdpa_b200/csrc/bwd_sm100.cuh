@@ -50,7 +50,7 @@ struct Layout {
   static constexpr int kQ = kV + kTileBytes;                  // 2 stages
   static constexpr int kDO = kQ + 2 * kTileBytes;             // kDOStages stages
   static constexpr int kDS = kDO + kDOStages * kTileBytes;    // 128 keys x 128 queries bf16
-  static constexpr int kLD = kDS + 128 * 128 * 2;             // 2 x {lse2[128], delta[128]} f32
+  static constexpr int kLD = kDS + 128 * 128 * 2;             // 2 x {-lse2[128], -delta[128]} f32
   // dQ_i staging: 32 x 32 fp32 boxes (4 KB), D/32 x 4 of them per tile: the
   // first 8 in the (then free) dS tile, the rest (D = 128) in this area.
   static constexpr int kXS = kLD + 2 * 1024;
@@ -84,8 +84,8 @@ struct Params {
   int T, H, BH, n_tiles, Tpad;
   float scale_log2;  // scale * log2(e)
   float scale;
-  const float* lse2;       // [BH][Tpad] lse * log2(e), zero-padded
-  const float* delta;      // [BH][Tpad], zero-padded
+  const float* lse2;       // [BH][Tpad] -lse * log2(e), zero-padded
+  const float* delta;      // [BH][Tpad] -Delta, zero-padded
   const int32_t* doc_start;
   const int32_t* doc_end;  // flattened, or null
   const float* rope_cos;   // [T][D/2] or null
@@ -303,26 +303,27 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
 #pragma unroll
       for (int c = 0; c < QC / 32; ++c) tmem_ld32(tS + qc0 + 32 * c, s + 32 * c);
       tmem_wait_ld();
+      const float2 scl2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
       for (int c = 0; c < QC / 32; ++c) {
         const int col = qc0 + 32 * c;
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float2 lv = reinterpret_cast<const float2*>(sl + col)[e];
+          const float2 nl = reinterpret_cast<const float2*>(sl + col)[e];  // -lse2 pair
           const int i_a = i0 + col + 2 * e;
-          // about a third of the exponentials go to the FMA pipe
-          const float x0 = fmaf(__uint_as_float(s[32 * c + 2 * e]), p.scale_log2, -lv.x);
-          const float x1 = fmaf(__uint_as_float(s[32 * c + 2 * e + 1]), p.scale_log2, -lv.y);
-          float p0 = (e % 3 == 2) ? exp2_fma(x0) : ex2(x0);
-          float p1 = (e % 3 == 2) ? exp2_fma(x1) : ex2(x1);
+          const float2 sv = make_float2(__uint_as_float(s[32 * c + 2 * e]),
+                                        __uint_as_float(s[32 * c + 2 * e + 1]));
+          const float2 x = __ffma2_rn(sv, scl2, nl);
+          // about a third of the pairs go to the FMA pipe
+          float2 pv = (e % 3 == 2) ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
           if (need_mask) {
-            if (i_a < j || i_a >= de_j) p0 = 0.f;
-            if (i_a + 1 < j || i_a + 1 >= de_j) p1 = 0.f;
+            if (i_a < j || i_a >= de_j) pv.x = 0.f;
+            if (i_a + 1 < j || i_a + 1 >= de_j) pv.y = 0.f;
           }
-          pf[32 * c + 2 * e] = p0;
-          pf[32 * c + 2 * e + 1] = p1;
-          pk[e] = pack_bf16(p0, p1);
+          pf[32 * c + 2 * e] = pv.x;
+          pf[32 * c + 2 * e + 1] = pv.y;
+          pk[e] = pack_bf16(pv.x, pv.y);
         }
         tmem_st16(tS + qc0 + 16 * c, pk);
       }
@@ -352,10 +353,12 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         uint32_t dsk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float2 dl = reinterpret_cast<const float2*>(sd + col)[e];
-          const float a0 = pf[32 * c + 2 * e] * (__uint_as_float(dpv[32 * c + 2 * e]) - dl.x);
-          const float a1 = pf[32 * c + 2 * e + 1] * (__uint_as_float(dpv[32 * c + 2 * e + 1]) - dl.y);
-          dsk[e] = pack_bf16(a0, a1);
+          const float2 nd = reinterpret_cast<const float2*>(sd + col)[e];  // -Delta pair
+          const float2 dpp = make_float2(__uint_as_float(dpv[32 * c + 2 * e]),
+                                         __uint_as_float(dpv[32 * c + 2 * e + 1]));
+          const float2 a = __fmul2_rn(make_float2(pf[32 * c + 2 * e], pf[32 * c + 2 * e + 1]),
+                                      __fadd2_rn(dpp, nd));
+          dsk[e] = pack_bf16(a.x, a.y);
         }
         // row r of the dS^T tile, query columns [col, col+32): block col/64,
         // 16-byte chunks (col%64)/8 .. +3

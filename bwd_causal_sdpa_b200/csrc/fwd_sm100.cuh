@@ -1,30 +1,38 @@
 // fwd_sm100.cuh -- tensor-core (tcgen05) attention forward for bf16 storage.
 //
-// One CTA computes one 128-row query tile of one (b, h) slice:
-//   warps 0-3  softmax: thread t owns query row t (= TMEM lane t), so the row
-//              max and row sum are thread-local (no shuffles);
-//   warp 4     TMA producer: Q once, then K and V tiles through a ring of
-//              shared-memory stages;
-//   warp 5     TMEM owner and MMA issuer (one thread): S = Q K^T into one of
-//              two TMEM score buffers, O += P V with P read from TMEM.
-// Per key tile j the MMA warp issues S_j while the softmax warps still work
-// on S_{j-1}; the softmax writes P_j (bf16) back over the first half of S_j's
-// columns and the PV MMA reads it from there (A operand in TMEM).
+// One CTA computes two 128-row query tiles (A = rows [256t, 256t+128), B =
+// the next 128) of one (b, h) slice; both share every K and V tile it loads.
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread t owns
+//              query row t of its tile (= TMEM lane t), so the row max and row
+//              sum are thread-local (no shuffles);
+//   warp 8     TMA producer: both Q tiles once, then K and V tiles through a
+//              ring of shared-memory stages;
+//   warp 9     TMEM owner and MMA issuer (one thread).
+// TMEM (512 columns): per tile an S column block (P, bf16, is written back
+// over its first half) and an O accumulator. Per key tile j the MMA thread
+// issues S_A(j), S_B(j), then PV_A(j), PV_B(j) as each tile's P becomes ready,
+// so the tensor pipe works on one tile while the other tile's softmax runs.
+// S_t(j) is issued only after PV_t(j-1) completed (it overwrites the P that
+// PV_t(j-1) reads); since a tcgen05 commit covers every earlier MMA of the
+// issuing thread, a softmax warp that has seen S_t(j) may rescale O_t
+// without a further wait.
 //
-// Online softmax in log2 units with a lazy rescale: the running max is only
-// moved (and O, l rescaled) when a row's max grows by more than 8, so P stays
-// <= 2^8 and O is rarely touched; the final O / l and lse = (m + log2 l) ln 2
-// use the same reference, which makes the result exact up to rounding.
+// Online softmax in log2 units with a lazy rescale: a row's reference max
+// moves (and O, l are rescaled) only when the max grows by more than 8, so P
+// stays <= 2^8 and O is rarely touched; the final O / l and lse = (m +
+// log2 l) ln 2 use the same reference, so the result is exact up to rounding.
+// A quarter of the exponentials run on the FMA pipe (exp2_fma2) to relieve the
+// MUFU unit.
 //
 // Masking is per element only on tiles that cross the diagonal or the start
-// of a row's document; tiles wholly before the first row's document are never
-// loaded (block skipping), nor are tiles past the diagonal.
+// of a row's document; key tiles wholly before the first row's document are
+// never loaded (block skipping), nor are tiles past the diagonal.
 //
 // Sources (page, section): ARK README, "Accelerated forward pass (GPU)" (SDPA
 // with the causal mask fused in) and aten.metal entry (scores, softmax,
 // weighted sum, fused causal kernel); Forge README, "Acknowledgements"
-// (FlashAttention-2-style tiling) and finding 3 (keep the kernel's live state
-// small). The tiling, TMEM use and warp roles are this library's own design.
+// (FlashAttention-2-style tiling) and roadmap (attention tile sweep). The
+// tiling, TMEM plan and warp roles are this library's own design.
 #pragma once
 
 #include "sm100.cuh"
@@ -38,8 +46,8 @@ struct Layout {
   static constexpr int kTileBytes = 128 * D * 2;  // 128 rows x D 16-bit values
   static constexpr int kBlockBytes = 128 * 128;   // one 64-column block: 128 rows x 128 B
   static constexpr int kStages = (D == 128) ? 2 : 4;
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;
+  static constexpr int kQ = 0;                    // Q_A, Q_B
+  static constexpr int kK = kQ + 2 * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
   static constexpr int kBars = kV + kStages * kTileBytes;
   // barrier indices
@@ -48,21 +56,22 @@ struct Layout {
   static constexpr int bKEmpty = bKFull + kStages;
   static constexpr int bVFull = bKEmpty + kStages;
   static constexpr int bVEmpty = bVFull + kStages;
-  static constexpr int bSFull = bVEmpty + kStages;  // 2
-  static constexpr int bPFull = bSFull + 2;         // 2
-  static constexpr int bPVDone = bPFull + 2;        // 2
-  static constexpr int bOFinal = bPVDone + 2;       // 1
-  static constexpr int kNumBars = bOFinal + 1;
+  static constexpr int bSFull = bVEmpty + kStages;  // [tile]
+  static constexpr int bPFull = bSFull + 2;         // [tile], 128 arrivals
+  static constexpr int bPVDone = bPFull + 2;        // [tile]
+  static constexpr int bOFinal = bPVDone + 2;       // [tile]
+  static constexpr int kNumBars = bOFinal + 2;
   static constexpr int kMisc = kBars + kNumBars * 8;  // [0] TMEM base, [1] abort flag
   static constexpr int kBytes = kMisc + 16;
-  static constexpr int kSmemAlloc = kBytes + 1024;  // slack to align the base to 1024
-  // TMEM columns
+  static constexpr int kSmemAlloc = kBytes;  // the window is 1024-byte aligned (checked)
+  // TMEM columns: tile t uses [256t, 256t+128) for S/P and [256t+128, ...) for O
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+  static constexpr int kThreads = 320;
+  static constexpr int kProducerWarp = 8, kMmaWarp = 9;
 };
 
 struct Params {
-  int T, H, BH, n_qtiles;
+  int T, H, BH, n_pairs, n_qtiles;
   float scale_log2;          // scale * log2(e)
   uint32_t idesc_s;          // instruction descriptor of S = Q K^T
   const float* q_fac;        // per (bh, tile) power-of-two factor of the stored q tile, or null
@@ -73,29 +82,34 @@ struct Params {
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const Params p) {
   using L = Layout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t sb0 = (raw + 1023u) & ~1023u;
-  uint8_t* sg = smem_raw + (sb0 - raw);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t sb0 = smem_u32(smem_raw);
+  if (sb0 & 1023u) {  // uniform across the CTA: nothing has been issued yet
+    if (threadIdx.x == 0) report_status(ATTN_ECUDA_LAYOUT);
+    return;
+  }
+  uint8_t* sg = smem_raw;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sg + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sg + L::kMisc + 4);
   auto bar = [&](int i) -> uint32_t { return sb0 + L::kBars + 8u * i; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.T;
-  // Flattened grid, tile-major from the last query tile: the longest rows
-  // (most key tiles) are scheduled first.
+  // Flattened grid, tile-major from the last tile pair: the longest rows (most
+  // key tiles) are scheduled first.
   const int bh = (int)blockIdx.x % p.BH, b = bh / p.H;
-  const int qt = p.n_qtiles - 1 - (int)blockIdx.x / p.BH;
-  const int q0 = qt * 128;
+  const int pr = p.n_pairs - 1 - (int)blockIdx.x / p.BH;
+  const int qtA = 2 * pr, qtB = 2 * pr + 1;
+  const bool hasB = qtB * 128 < T;
   const int row0 = b * T;
-  const int ds0 = p.doc_start ? p.doc_start[row0 + q0] - row0 : 0;
+  const int ds0 = p.doc_start ? p.doc_start[row0 + qtA * 128] - row0 : 0;
   const int kv_t0 = ds0 >> 7;
-  const int n_kv = qt - kv_t0 + 1;
+  const int nA = qtA - kv_t0 + 1;           // key tiles tile A needs
+  const int n_kv = hasB ? nA + 1 : nA;      // tile B needs one more (its diagonal)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::bQFull), 1);
@@ -105,16 +119,16 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(bar(L::bVFull + s), 1);
       mbar_init(bar(L::bVEmpty + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(L::bSFull + s), 1);
-      mbar_init(bar(L::bPFull + s), 128);
-      mbar_init(bar(L::bPVDone + s), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(L::bSFull + t), 1);
+      mbar_init(bar(L::bPFull + t), 128);
+      mbar_init(bar(L::bPVDone + t), 1);
+      mbar_init(bar(L::bOFinal + t), 1);
     }
-    mbar_init(bar(L::bOFinal), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == L::kMmaWarp) {
     tmem_alloc(sb0 + L::kMisc, L::kTmemCols);
     tmem_relinquish();
   }
@@ -123,15 +137,17 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == L::kProducerWarp) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       prefetch_tensor_map(&tmQ);
       prefetch_tensor_map(&tmK);
       prefetch_tensor_map(&tmV);
-      mbar_arrive_expect_tx(bar(L::bQFull), L::kTileBytes);
-      for (int cb = 0; cb < D / 64; ++cb)
-        tma_load_3d(sb0 + L::kQ + cb * L::kBlockBytes, &tmQ, bar(L::bQFull), cb * 64, q0, bh);
+      mbar_arrive_expect_tx(bar(L::bQFull), (hasB ? 2 : 1) * L::kTileBytes);
+      for (int t = 0; t < (hasB ? 2 : 1); ++t)
+        for (int cb = 0; cb < D / 64; ++cb)
+          tma_load_3d(sb0 + L::kQ + t * L::kTileBytes + cb * L::kBlockBytes, &tmQ,
+                      bar(L::bQFull), cb * 64, (qtA + t) * 128, bh);
       for (int it = 0; it < n_kv; ++it) {
         const int st = it % L::kStages, round = it / L::kStages;
         const int kvrow = (kv_t0 + it) * 128;
@@ -147,130 +163,162 @@ __global__ void __launch_bounds__(192, 1)
                       bar(L::bVFull + st), cb * 64, kvrow, bh);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == L::kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_o = idesc_f16(128, D, true, true, false, true);
       bool ok = mbar_wait(bar(L::bQFull), 0, abort_flag);
-      for (int it = 0; ok && it <= n_kv; ++it) {
-        if (it < n_kv) {
-          const int sbuf = it & 1, st = it % L::kStages;
-          if (!mbar_wait(bar(L::bKFull + st), (it / L::kStages) & 1, abort_flag)) break;
-          if (it >= 2 && !mbar_wait(bar(L::bPVDone + sbuf), ((it - 2) >> 1) & 1, abort_flag)) break;
+      for (int it = 0; ok && it < n_kv; ++it) {
+        const int st = it % L::kStages;
+        const int t0 = (it < nA) ? 0 : 1;     // tile A runs only for it < nA
+        const int t1 = hasB ? 2 : 1;
+        if (!mbar_wait(bar(L::bKFull + st), (it / L::kStages) & 1, abort_flag)) break;
+        const uint32_t kbase = sb0 + L::kK + st * L::kTileBytes;
+        for (int t = t0; ok && t < t1; ++t) {
+          // S_t(it) overwrites P_t(it-1): wait until PV_t(it-1) is done
+          if (it > 0 && !mbar_wait(bar(L::bPVDone + t), (it - 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t dS = tmem + (sbuf ? L::kColS1 : L::kColS0);
-          const uint32_t kbase = sb0 + L::kK + st * L::kTileBytes;
+          const uint32_t qbase = sb0 + L::kQ + t * L::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
-            mma_ss(dS, smem_desc_sw128(sb0 + L::kQ + off, 16, 1024),
+            mma_ss(tmem + 256 * t, smem_desc_sw128(qbase + off, 16, 1024),
                    smem_desc_sw128(kbase + off, 16, 1024), p.idesc_s, kk > 0);
           }
-          mma_commit(bar(L::bSFull + sbuf));
-          mma_commit(bar(L::bKEmpty + st));
+          mma_commit(bar(L::bSFull + t));
         }
-        if (it >= 1) {
-          const int j = it - 1, pb = j & 1, vst = j % L::kStages;
-          if (!mbar_wait(bar(L::bPFull + pb), (j >> 1) & 1, abort_flag)) break;
-          if (!mbar_wait(bar(L::bVFull + vst), (j / L::kStages) & 1, abort_flag)) break;
+        if (!ok) break;
+        mma_commit(bar(L::bKEmpty + st));
+        if (!mbar_wait(bar(L::bVFull + st), (it / L::kStages) & 1, abort_flag)) break;
+        const uint32_t vbase = sb0 + L::kV + st * L::kTileBytes;
+        for (int t = t0; ok && t < t1; ++t) {
+          if (!mbar_wait(bar(L::bPFull + t), it & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t aP = tmem + (pb ? L::kColS1 : L::kColS0);
-          const uint32_t vbase = sb0 + L::kV + vst * L::kTileBytes;
+          const uint32_t aP = tmem + 256 * t;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            mma_ts(tmem + L::kColO, aP + kk * 8,
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + 256 * t + 128, aP + kk * 8,
                    smem_desc_sw128(vbase + kk * 2048, L::kBlockBytes, 1024), idesc_o,
-                   (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(bar(L::bPVDone + pb));
-          mma_commit(bar(L::bVEmpty + vst));
-          if (j == n_kv - 1) mma_commit(bar(L::bOFinal));
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(L::bPVDone + t));
         }
+        if (!ok) break;
+        mma_commit(bar(L::bVEmpty + st));
+      }
+      if (ok) {
+        mma_commit(bar(L::bOFinal + 0));
+        mma_commit(bar(L::bOFinal + 1));
       }
     }
   } else {
-    // ---------------- softmax warps 0-3 ----------------
-    const int r = threadIdx.x;  // row within the tile, TMEM lane
-    const int i = q0 + r;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // ---------------- softmax warpgroups (tile A: warps 0-3, B: 4-7) ----------------
+    const int t = warp >> 2;
+    const int r = threadIdx.x & 127;  // row within the tile = TMEM lane
+    const int qt = qtA + t;
+    const int i = qt * 128 + r;
+    const bool active = (t == 0) || hasB;
+    const int n_t = (t == 0) ? nA : n_kv;  // key tiles this tile processes
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + 256 * t;
+    const uint32_t tO = tS + 128;
     const int ds_i = p.doc_start ? p.doc_start[row0 + min(i, T - 1)] - row0 : 0;
-    const float fq = p.q_fac ? p.q_fac[bh * p.n_qtiles + qt] : 1.f;
+    const float fq = p.q_fac ? p.q_fac[bh * p.n_qtiles + min(qt, p.n_qtiles - 1)] : 1.f;
     float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int it = 0; it < n_kv; ++it) {
-      const int sbuf = it & 1;
+    bool ok = active;
+    for (int it = 0; ok && it < n_t; ++it) {
       const int kt = kv_t0 + it, j0 = kt * 128;
-      if (!mbar_wait(bar(L::bSFull + sbuf), (it >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(L::bSFull + t), it & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
+      // scale of this key tile's scores (q, k tiles may carry power-of-two factors)
       const float sc = p.scale_log2 * fq * (p.k_fac ? p.k_fac[bh * p.n_qtiles + kt] : 1.f);
-      const uint32_t tS = tmem + lane_base + (sbuf ? L::kColS1 : L::kColS0);
+      const bool pos_scale = sc > 0.f;
       uint32_t s[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s + 32 * c);
       tmem_wait_ld();
       const bool need_mask = (j0 + 127 > i) || (j0 < ds_i);
-      float mx = -INFINITY;
+      const float masked = pos_scale ? -INFINITY : INFINITY;
+      if (need_mask) {
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float x = __uint_as_float(s[c]) * sc;
-        if (need_mask && (j0 + c > i || j0 + c < ds_i)) x = -INFINITY;
-        s[c] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+        for (int c = 0; c < 128; ++c)
+          if (j0 + c > i || j0 + c < ds_i) s[c] = __float_as_uint(masked);
       }
+      // row extreme of the raw scores (max for a positive scale): four chains
+      // of three-input max / min
+      float e4[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) e4[q] = __uint_as_float(s[q]);
+      float ext;
+      if (pos_scale) {
+#pragma unroll
+        for (int c = 4; c < 128; c += 2)
+          e4[(c >> 1) & 3] = max3f(e4[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        ext = max3f(fmaxf(e4[0], e4[1]), e4[2], e4[3]);
+      } else {
+#pragma unroll
+        for (int c = 4; c < 128; c += 2)
+          e4[(c >> 1) & 3] = min3f(e4[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        ext = min3f(fminf(e4[0], e4[1]), e4[2], e4[3]);
+      }
+      const float mx = ext * sc;  // row max of the scaled scores (log2 units)
       // Move the reference max only when it grows by more than 8 (log2
       // units); the first key a row sees always moves it (m = -inf).
       const bool move = mx > m + 8.f;
       const float alpha = move ? ex2(m - mx) : 1.f;
-      // O needs rescaling only if it already holds a non-zero partial sum.
+      // O needs rescaling only if it already holds a non-zero partial sum;
+      // PV_t(it-1) is complete (it precedes S_t(it) in the commit order).
       const bool scale_o = move && m != -INFINITY && it > 0;
-      if (__any_sync(0xffffffffu, scale_o)) {
-        // Warp-collective: wait for PV_{it-1}, then scale each lane's row by
-        // its own factor (1 for lanes that keep their max).
-        if (!mbar_wait(bar(L::bPVDone + ((it - 1) & 1)), ((it - 1) >> 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const float f = scale_o ? alpha : 1.f;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tmem_ld32(tmem + lane_base + L::kColO + 32 * c, ov);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-          tmem_st32(tmem + lane_base + L::kColO + 32 * c, ov);
-        }
-      }
       if (move) {
         l *= alpha;
         m = mx;
       }
       const float mref = (m == -INFINITY) ? 0.f : m;
+      // p = 2^(s * sc - m) two at a time; a quarter of the pairs on the FMA pipe
+      const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-mref, -mref);
+      float2 l2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(__uint_as_float(s[32 * c + 2 * e]) - mref);
-          const float p1 = ex2(__uint_as_float(s[32 * c + 2 * e + 1]) - mref);
-          l += p0 + p1;
-          pk[e] = pack_bf16(p0, p1);
+          const float2 sv = make_float2(__uint_as_float(s[32 * c + 2 * e]),
+                                        __uint_as_float(s[32 * c + 2 * e + 1]));
+          const float2 x = __ffma2_rn(sv, sc2, nm2);
+          const float2 pv = (e % 4 == 3) ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
+          l2[e & 3] = __fadd2_rn(l2[e & 3], pv);
+          pk[e] = pack_bf16(pv.x, pv.y);
         }
         tmem_st16(tS + 16 * c, pk);
       }
+      const float2 la = __fadd2_rn(l2[0], l2[1]), lb = __fadd2_rn(l2[2], l2[3]);
+      l += (la.x + la.y) + (lb.x + lb.y);
+      // The scores are dead now; rescale O (warp-collective: each lane by its
+      // own factor, 1 for lanes that kept their max) before PV_t(it) runs.
+      if (__any_sync(0xffffffffu, scale_o)) {
+        const float f = scale_o ? alpha : 1.f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tO + 32 * c, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+          tmem_st32(tO + 32 * c, ov);
+        }
+      }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(L::bPFull + sbuf));
+      mbar_arrive(bar(L::bPFull + t));
     }
-    if (ok && mbar_wait(bar(L::bOFinal), 0, abort_flag)) {
+    if (ok && mbar_wait(bar(L::bOFinal + t), 0, abort_flag)) {
       tc_fence_after();
       const float inv = 1.f / l;
       __nv_bfloat16* orow = p.o + ((size_t)bh * T + min(i, T - 1)) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
-        tmem_ld32(tmem + lane_base + L::kColO + 32 * c, ov);  // warp-collective
+        tmem_ld32(tO + 32 * c, ov);  // warp-collective
         tmem_wait_ld();
         if (i < T) {
           uint32_t pk[16];
@@ -289,7 +337,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == L::kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }

@@ -150,10 +150,11 @@ __global__ void __launch_bounds__(256) rope_prep_kernel(
 }
 
 // Backward preprocessing for the tensor-core path, one warp per row of the
-// tile-padded [B*H][ntiles*128] view: Delta_i = sum_d dO[i][d] * o[i][d] and
-// lse2_i = lse_i * log2(e) (both 0 for padding rows t >= T, so the main
-// kernel's per-tile loads never leave the arrays), and the fp32 dq
-// accumulator row is zeroed.
+// tile-padded [B*H][ntiles*128] view: stores -Delta_i (Delta_i = sum_d
+// dO[i][d] * o[i][d]) and -lse_i * log2(e), negated so the main kernel folds
+// them in with one fused multiply-add (both 0 for padding rows t >= T, so its
+// per-tile loads never leave the arrays), and zeroes the fp32 dq accumulator
+// row.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(
     const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
@@ -178,8 +179,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
     store_vec<NC>(dq_acc + r * D + lane * NC, z);
   }
   if (lane == 0) {
-    delta_pad[row] = s;
-    lse2_pad[row] = t < T ? lse[bh * T + t] * 1.4426950408889634f : 0.f;
+    delta_pad[row] = -s;
+    lse2_pad[row] = t < T ? -lse[bh * T + t] * 1.4426950408889634f : 0.f;
   }
 }
 
