@@ -10,12 +10,11 @@
 //   warp 9     TMEM owner and MMA issuer (one thread).
 // TMEM (512 columns): per tile an S column block (P, bf16, is written back
 // over its first half) and an O accumulator. Per key tile j the MMA thread
-// issues S_A(j), S_B(j), then PV_A(j), PV_B(j) as each tile's P becomes ready,
-// so the tensor pipe works on one tile while the other tile's softmax runs.
-// S_t(j) is issued only after PV_t(j-1) completed (it overwrites the P that
-// PV_t(j-1) reads); since a tcgen05 commit covers every earlier MMA of the
-// issuing thread, a softmax warp that has seen S_t(j) may rescale O_t
-// without a further wait.
+// issues PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the tensor pipe works on one
+// tile while the other tile's softmax runs. S_t(j+1) is issued only after
+// PV_t(j) completed (it overwrites the P that PV_t(j) reads); since a tcgen05
+// commit covers every earlier MMA of the issuing thread, a softmax warp that
+// has seen S_t(j) may rescale O_t without a further wait.
 //
 // Online softmax in log2 units with a lazy rescale: a row's reference max
 // moves (and O, l are rescaled) only when the max grows by more than 8, so P
@@ -165,33 +164,40 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     }
   } else if (warp == L::kMmaWarp) {
     // ---------------- MMA issuer ----------------
+    // Issue order: S_A(0), S_B(0), then per key tile j: PV_A(j), S_A(j+1),
+    // PV_B(j), S_B(j+1). Each tile's S(j+1) follows its own PV(j) (it
+    // overwrites the P that PV(j) reads, so it waits for PV(j) to finish), and
+    // never waits for the other tile's softmax: the two chains
+    // S -> softmax -> PV run independently and fill each other's gaps.
     if (lane == 0) {
       constexpr uint32_t idesc_o = idesc_f16(128, D, true, true, false, true);
-      bool ok = mbar_wait(bar(L::bQFull), 0, abort_flag);
-      for (int it = 0; ok && it < n_kv; ++it) {
-        const int st = it % L::kStages;
-        const int t0 = (it < nA) ? 0 : 1;     // tile A runs only for it < nA
-        const int t1 = hasB ? 2 : 1;
-        if (!mbar_wait(bar(L::bKFull + st), (it / L::kStages) & 1, abort_flag)) break;
-        const uint32_t kbase = sb0 + L::kK + st * L::kTileBytes;
-        for (int t = t0; ok && t < t1; ++t) {
-          // S_t(it) overwrites P_t(it-1): wait until PV_t(it-1) is done
-          if (it > 0 && !mbar_wait(bar(L::bPVDone + t), (it - 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t qbase = sb0 + L::kQ + t * L::kTileBytes;
+      const int t1 = hasB ? 2 : 1;
+      auto active = [&](int t, int j) -> bool { return j < ((t == 0) ? nA : n_kv) && t < t1; };
+      auto issue_S = [&](int t, int j) {
+        const uint32_t kbase = sb0 + L::kK + (j % L::kStages) * L::kTileBytes;
+        const uint32_t qbase = sb0 + L::kQ + t * L::kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
-            mma_ss(tmem + 256 * t, smem_desc_sw128(qbase + off, 16, 1024),
-                   smem_desc_sw128(kbase + off, 16, 1024), p.idesc_s, kk > 0);
-          }
-          mma_commit(bar(L::bSFull + t));
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
+          mma_ss(tmem + 256 * t, smem_desc_sw128(qbase + off, 16, 1024),
+                 smem_desc_sw128(kbase + off, 16, 1024), p.idesc_s, kk > 0);
         }
-        if (!ok) break;
-        mma_commit(bar(L::bKEmpty + st));
+        mma_commit(bar(L::bSFull + t));
+      };
+      bool ok = mbar_wait(bar(L::bQFull), 0, abort_flag) && mbar_wait(bar(L::bKFull), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < t1; ++t)
+          if (active(t, 0)) issue_S(t, 0);
+        mma_commit(bar(L::bKEmpty));
+      }
+      for (int it = 0; ok && it < n_kv; ++it) {
+        const int st = it % L::kStages, nst = (it + 1) % L::kStages;
         if (!mbar_wait(bar(L::bVFull + st), (it / L::kStages) & 1, abort_flag)) break;
         const uint32_t vbase = sb0 + L::kV + st * L::kTileBytes;
-        for (int t = t0; ok && t < t1; ++t) {
+        bool issued_next = false;
+        for (int t = 0; ok && t < t1; ++t) {
+          if (!active(t, it)) continue;
           if (!mbar_wait(bar(L::bPFull + t), it & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t aP = tmem + 256 * t;
@@ -201,9 +207,20 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
                    smem_desc_sw128(vbase + kk * 2048, L::kBlockBytes, 1024), idesc_o,
                    (it > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(L::bPVDone + t));
+          if (active(t, it + 1)) {
+            if (!mbar_wait(bar(L::bKFull + nst), ((it + 1) / L::kStages) & 1, abort_flag) ||
+                !mbar_wait(bar(L::bPVDone + t), it & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_S(t, it + 1);
+            issued_next = true;
+          }
         }
         if (!ok) break;
         mma_commit(bar(L::bVEmpty + st));
+        if (issued_next) mma_commit(bar(L::bKEmpty + nst));
       }
       if (ok) {
         mma_commit(bar(L::bOFinal + 0));
