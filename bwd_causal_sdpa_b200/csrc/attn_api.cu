@@ -140,7 +140,7 @@ int check_common(const void* q, const void* k, const void* v, const float* rc, c
   if ((rc == nullptr) != (rs == nullptr)) return ATTN_EINVAL;
   if (!sizes_ok(B, H, T, D)) return ATTN_EUNSUPPORTED;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return ATTN_EALIGN;
-  if ((rc && !aligned(rc, 4)) || (rs && !aligned(rs, 4)) || (cu && !aligned(cu, 4))) return ATTN_EALIGN;
+  if ((rc && !aligned(rc, 16)) || (rs && !aligned(rs, 16)) || (cu && !aligned(cu, 4))) return ATTN_EALIGN;
   const WsPlan p = plan(B, H, T, D, dtype, is_bwd);
   if (p.total > 0) {
     if (!ws) return ATTN_EWORKSPACE;
@@ -246,26 +246,18 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
            char* ws, const WsPlan& wp, cudaStream_t st) {
   using L = bwd100::Layout<D>;
   const int nt = (T + 127) / 128, BH = B * H, Tpad = nt * 128;
-  const void* qs = q;
-  const void* ks = k;
-  if (rc) {
-    __nv_bfloat16* qr = (__nv_bfloat16*)(ws + wp.q16);
-    __nv_bfloat16* kr = (__nv_bfloat16*)(ws + wp.k16);
-    ATTN_LAUNCH(KK_ROPE_PREP, st,
-                rope_prep_kernel<__nv_bfloat16, D, false><<<dim3(nt, BH, 2), 256, 0, st>>>(
-                    (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qr, kr, nullptr,
-                    nullptr, H, T, nt));
-    if (launch_status()) return ATTN_ECUDA;
-    qs = qr;
-    ks = kr;
-  }
+  __nv_bfloat16* qr = (__nv_bfloat16*)(ws + wp.q16);
+  __nv_bfloat16* kr = (__nv_bfloat16*)(ws + wp.k16);
+  const void* qs = rc ? (const void*)qr : q;
+  const void* ks = rc ? (const void*)kr : k;
   float* delta = (float*)(ws + wp.delta);
   float* lse2 = (float*)(ws + wp.lse2);
   float* dq_acc = (float*)(ws + wp.dq_acc);
   const long rows_pad = (long)BH * Tpad;
   ATTN_LAUNCH(KK_DELTA, st,
               bwd_prep_kernel<D><<<(unsigned)((rows_pad + 7) / 8), 256, 0, st>>>(
-                  (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse, delta, lse2, dq_acc, T,
+                  (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse, delta, lse2, dq_acc,
+                  (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qr, kr, H, T,
                   Tpad, rows_pad));
   if (launch_status()) return ATTN_ECUDA;
   CUtensorMap mq, mk, mv, mo, mdq;
@@ -492,8 +484,8 @@ extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, con
   if (!sizes_ok(B, H, T, D)) return ATTN_EUNSUPPORTED;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(dO, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
-      !aligned(lse, 4) || (rope_cos && !aligned(rope_cos, 4)) ||
-      (rope_sin && !aligned(rope_sin, 4)) || (cu_seqlens && !aligned(cu_seqlens, 4)))
+      !aligned(lse, 4) || (rope_cos && !aligned(rope_cos, 16)) ||
+      (rope_sin && !aligned(rope_sin, 16)) || (cu_seqlens && !aligned(cu_seqlens, 4)))
     return ATTN_EALIGN;
   const NoAllocPlan p = noalloc_plan(B, H, T);
   if (p.total > kNoAllocBytes) return ATTN_ESCRATCH;

@@ -89,17 +89,37 @@ __device__ __forceinline__ float warp_max(float x) {
 
 // Rotate (in place) NC consecutive elements starting at an even dimension d0
 // by the RoPE angles of position pos: pairs (x[2i], x[2i+1]) -> (x0 c - x1 s,
-// x0 s + x1 c). inverse = true applies the transpose rotation.
+// x0 s + x1 c). inverse = true applies the transpose rotation. For NC a
+// multiple of 8, d0 must be a multiple of 8 and the tables 16-byte aligned:
+// four pairs' cos and sin then come in one 16-byte load each.
 template <int NC, int D>
 __device__ __forceinline__ void rope_pairs(float* x, const float* rc, const float* rs,
                                            int pos, int d0, bool inverse) {
+  if constexpr (NC % 8 == 0) {
+    const float4* c4 = reinterpret_cast<const float4*>(rc + (size_t)pos * (D / 2) + (d0 >> 1));
+    const float4* s4 = reinterpret_cast<const float4*>(rs + (size_t)pos * (D / 2) + (d0 >> 1));
 #pragma unroll
-  for (int c = 0; c < NC; c += 2) {
-    const int pi = (d0 + c) >> 1;
-    const float cs = rc[(size_t)pos * (D / 2) + pi];
-    const float sn = inverse ? -rs[(size_t)pos * (D / 2) + pi] : rs[(size_t)pos * (D / 2) + pi];
-    const float x0 = x[c], x1 = x[c + 1];
-    x[c] = x0 * cs - x1 * sn;
-    x[c + 1] = x0 * sn + x1 * cs;
+    for (int q = 0; q < NC / 8; ++q) {
+      const float4 cq = c4[q], sq0 = s4[q];
+      const float cs[4] = {cq.x, cq.y, cq.z, cq.w};
+      const float sn[4] = {inverse ? -sq0.x : sq0.x, inverse ? -sq0.y : sq0.y,
+                           inverse ? -sq0.z : sq0.z, inverse ? -sq0.w : sq0.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = x[8 * q + 2 * e], x1 = x[8 * q + 2 * e + 1];
+        x[8 * q + 2 * e] = x0 * cs[e] - x1 * sn[e];
+        x[8 * q + 2 * e + 1] = x0 * sn[e] + x1 * cs[e];
+      }
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < NC; c += 2) {
+      const int pi = (d0 + c) >> 1;
+      const float cs = rc[(size_t)pos * (D / 2) + pi];
+      const float sn = inverse ? -rs[(size_t)pos * (D / 2) + pi] : rs[(size_t)pos * (D / 2) + pi];
+      const float x0 = x[c], x1 = x[c + 1];
+      x[c] = x0 * cs - x1 * sn;
+      x[c + 1] = x0 * sn + x1 * cs;
+    }
   }
 }

@@ -153,13 +153,18 @@ __global__ void __launch_bounds__(256) rope_prep_kernel(
 // tile-padded [B*H][ntiles*128] view: stores -Delta_i (Delta_i = sum_d
 // dO[i][d] * o[i][d]) and -lse_i * log2(e), negated so the main kernel folds
 // them in with one fused multiply-add (both 0 for padding rows t >= T, so its
-// per-tile loads never leave the arrays), and zeroes the fp32 dq accumulator
-// row.
+// per-tile loads never leave the arrays), zeroes the fp32 dq accumulator row
+// and, with RoPE tables, writes the rotated q and k rows (bf16) the main
+// kernel reads.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(
     const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
     const float* __restrict__ lse, float* __restrict__ delta_pad, float* __restrict__ lse2_pad,
-    float* __restrict__ dq_acc, int T, int Tpad, long rows_pad) {
+    float* __restrict__ dq_acc, const __nv_bfloat16* __restrict__ q,
+    const __nv_bfloat16* __restrict__ k, const float* __restrict__ rc,
+    const float* __restrict__ rs, const int32_t* __restrict__ doc_start,
+    __nv_bfloat16* __restrict__ qr, __nv_bfloat16* __restrict__ kr, int H, int T, int Tpad,
+    long rows_pad) {
   constexpr int NC = D / 32;
   const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -177,6 +182,17 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
     s = warp_sum(s);
     const float z[NC] = {};
     store_vec<NC>(dq_acc + r * D + lane * NC, z);
+    if (rc) {
+      const int b = (int)(bh / H);
+      const int pos = t - (doc_start ? doc_start[b * T + t] - b * T : 0);
+      float x[NC];
+      load_vec<NC>(q + r * D + lane * NC, x);
+      rope_pairs<NC, D>(x, rc, rs, pos, lane * NC, false);
+      store_vec<NC>(qr + r * D + lane * NC, x);
+      load_vec<NC>(k + r * D + lane * NC, x);
+      rope_pairs<NC, D>(x, rc, rs, pos, lane * NC, false);
+      store_vec<NC>(kr + r * D + lane * NC, x);
+    }
   }
   if (lane == 0) {
     delta_pad[row] = -s;

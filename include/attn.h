@@ -24,9 +24,9 @@
  *     fastest, in the storage type `dtype` (ATTN_BF16 or ATTN_F32). lse is
  *     [B, H, T] float32. All are DEVICE pointers on the current CUDA device,
  *     owned by the caller; the library never allocates or frees memory.
- *   - q, k, v, o, dO, dq, dk, dv and the workspace must be 16-byte aligned
- *     (the kernels move tiles with TMA); lse, rope tables and cu_seqlens must
- *     be 4-byte aligned.
+ *   - q, k, v, o, dO, dq, dk, dv, the rope tables and the workspace must be
+ *     16-byte aligned (the kernels move tiles with TMA and read the tables in
+ *     16-byte groups); lse and cu_seqlens must be 4-byte aligned.
  *   - D must be 64 or 128. B, H, T >= 1. B*T and B*H*T*D must fit in int32.
  *   - RoPE: rope_cos and rope_sin are both NULL (no RoPE) or both [T, D/2]
  *     float32 with row p holding cos/sin(p * theta_i) for position p. Pairs

@@ -96,6 +96,7 @@ def test_host_validation(call):
     assert call(k=P + 8) == A.ATTN_EALIGN
     assert call(workspace=P + 4) == A.ATTN_EALIGN
     assert call(cu_seqlens=P + 2) == A.ATTN_EALIGN
+    assert call(rope_cos=P + 4, rope_sin=P) == A.ATTN_EALIGN
     assert call(workspace=None) == A.ATTN_EWORKSPACE
     assert call(ws_bytes=16) == A.ATTN_EWORKSPACE
 
