@@ -26,7 +26,11 @@ Conventions (the plainest reading where the pages are silent):
 - a token attends to itself (j <= i), so no row is empty;
 - cu_seqlens indexes the flattened B*T token axis, starts at 0, ends at B*T and
   contains every row boundary r*T (documents never cross rows);
-- the backward returns gradients with respect to the un-rotated q and k.
+- the backward returns gradients with respect to the un-rotated q and k;
+- grouped-query attention (Forge README, "Architecture": attention with GQA
+  and RoPE): k and v may have H_kv heads with H_kv dividing H; query head h
+  reads key/value head h // (H / H_kv), and the gradient of a shared key/value
+  head is the sum over the query heads that read it.
 """
 
 from __future__ import annotations
@@ -191,34 +195,53 @@ def _slices(B: int, H: int, heads: Optional[Iterable[Tuple[int, int]]]) -> Seque
     return list(heads)
 
 
+def _kv_head(h: int, H: int, H_kv: int) -> int:
+    if H % H_kv:
+        raise ValueError("the number of query heads must be a multiple of the key/value heads")
+    return h // (H // H_kv)
+
+
 def attention_forward(q, k, v, rope_cos, rope_sin, cu_seqlens, scale, heads=None):
     """o [B,H,T,D] and lse [B,H,T] in float64. Inputs are upcast exactly from
-    their float32/bf16 storage. ``heads`` optionally restricts the work to a
-    list of (b, h) slices (the other entries are left NaN)."""
+    their float32/bf16 storage; k, v may have fewer heads than q (grouped-query
+    attention). ``heads`` optionally restricts the work to a list of (b, h)
+    query slices (the other entries are left NaN)."""
     q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
     B, H, T, D = q.shape
+    H_kv = k.shape[1]
     cos, sin = _tables(rope_cos, rope_sin)
     pos, start = doc_layout(B, T, cu_seqlens)
     o = np.full((B, H, T, D), np.nan)
     lse = np.full((B, H, T), np.nan)
     for b, h in _slices(B, H, heads):
-        f = forward_head(q[b, h], k[b, h], v[b, h], cos, sin, pos[b], start[b], scale)
+        hk = _kv_head(h, H, H_kv)
+        f = forward_head(q[b, h], k[b, hk], v[b, hk], cos, sin, pos[b], start[b], scale)
         o[b, h] = f["o"]
         lse[b, h] = f["lse"]
     return o, lse
 
 
 def attention_backward(q, k, v, do, rope_cos, rope_sin, cu_seqlens, scale, heads=None):
-    """dq, dk, dv [B,H,T,D] in float64 for the loss L = sum(o * do), with o the
-    exact forward of the same inputs."""
+    """dq [B,H,T,D] and dk, dv [B,H_kv,T,D] in float64 for the loss
+    L = sum(o * do), with o the exact forward of the same inputs. With
+    ``heads`` (a list of (b, h) query slices) only those slices' contributions
+    are computed: dq for them, and dk, dv summed over them for the key/value
+    heads they read (entries no listed slice reads are left NaN)."""
     q, k, v, do = (np.asarray(a, dtype=np.float64) for a in (q, k, v, do))
     B, H, T, D = q.shape
+    H_kv = k.shape[1]
     cos, sin = _tables(rope_cos, rope_sin)
     pos, start = doc_layout(B, T, cu_seqlens)
     dq = np.full((B, H, T, D), np.nan)
-    dk = np.full((B, H, T, D), np.nan)
-    dv = np.full((B, H, T, D), np.nan)
+    dk = np.full((B, H_kv, T, D), np.nan)
+    dv = np.full((B, H_kv, T, D), np.nan)
     for b, h in _slices(B, H, heads):
-        g = backward_head(q[b, h], k[b, h], v[b, h], do[b, h], cos, sin, pos[b], start[b], scale)
-        dq[b, h], dk[b, h], dv[b, h] = g["dq"], g["dk"], g["dv"]
+        hk = _kv_head(h, H, H_kv)
+        g = backward_head(q[b, h], k[b, hk], v[b, hk], do[b, h], cos, sin, pos[b], start[b], scale)
+        dq[b, h] = g["dq"]
+        if np.isnan(dk[b, hk, 0, 0]):
+            dk[b, hk] = 0.0
+            dv[b, hk] = 0.0
+        dk[b, hk] += g["dk"]
+        dv[b, hk] += g["dv"]
     return dq, dk, dv

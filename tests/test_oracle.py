@@ -275,6 +275,42 @@ def test_gradient_identities():
     assert np.max(np.abs(g["dk"].sum(axis=0))) < 1e-12          # sum_j dk_j = 0 without RoPE
 
 
+def test_grouped_query_attention_gradients_match_central_differences():
+    rng = np.random.default_rng(30)
+    B, H, H_kv, T, D = 1, 4, 2, 6, 4
+    q, do = _rand(rng, B, H, T, D), _rand(rng, B, H, T, D)
+    k, v = _rand(rng, B, H_kv, T, D), _rand(rng, B, H_kv, T, D)
+    cos, sin = rope_angles_f64(T, D, 100.0)
+    dq, dk, dv = attention_backward(q, k, v, do, cos, sin, None, 0.6)
+    fq, fk, fv = _fd_grads(q, k, v, do, cos, sin, None, 0.6)
+    assert _rel(dq, fq) < 1e-7
+    assert _rel(dk, fk) < 1e-7
+    assert _rel(dv, fv) < 1e-7
+
+
+def test_grouped_query_attention_equals_repeated_heads():
+    # GQA is MHA on key/value heads repeated over each group; the shared
+    # heads' gradients are the sums over their group (chain rule).
+    rng = np.random.default_rng(31)
+    B, H, H_kv, T, D = 2, 6, 2, 9, 8
+    q, do = _rand(rng, B, H, T, D), _rand(rng, B, H, T, D)
+    k, v = _rand(rng, B, H_kv, T, D), _rand(rng, B, H_kv, T, D)
+    cu = np.asarray([0, 4, 9, 12, 18], dtype=np.int32)
+    cos, sin = rope_angles_f64(T, D)
+    kr, vr = np.repeat(k, H // H_kv, axis=1), np.repeat(v, H // H_kv, axis=1)
+    o, lse = attention_forward(q, k, v, cos, sin, cu, 0.4)
+    o2, lse2 = attention_forward(q, kr, vr, cos, sin, cu, 0.4)
+    assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+    dq, dk, dv = attention_backward(q, k, v, do, cos, sin, cu, 0.4)
+    dq2, dk2, dv2 = attention_backward(q, kr, vr, do, cos, sin, cu, 0.4)
+    np.testing.assert_allclose(dq, dq2, rtol=1e-13, atol=1e-14)
+    g = H // H_kv
+    np.testing.assert_allclose(dk, dk2.reshape(B, H_kv, g, T, D).sum(axis=2), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dv, dv2.reshape(B, H_kv, g, T, D).sum(axis=2), rtol=1e-12, atol=1e-13)
+    with pytest.raises(ValueError):
+        attention_forward(q, k[:, :1].repeat(4, axis=1), v[:, :1].repeat(4, axis=1), None, None, None, 1.0)
+
+
 def test_doc_layout_rejects_bad_boundaries():
     with pytest.raises(ValueError):
         doc_layout(2, 8, np.asarray([0, 5, 12, 16], dtype=np.int32))   # doc crosses row 0 -> 1
