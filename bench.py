@@ -68,6 +68,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="long_context_8k")
+    ap.add_argument("--kv-heads", type=int, default=None,
+                    help="grouped-query attention: key/value heads (dividing the workload's H)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -98,6 +100,7 @@ def kernel_algorithmic(name: str, w, kinds_seen) -> tuple:
     U = causal_unit(w)
     elem = 2 if w.dtype == "bf16" else 4
     N = w.B * w.H * w.T * w.D
+    Nkv = w.B * w.kv_heads * w.T * w.D
     R = w.B * w.H * w.T
     if name == "fwd":
         return "tensor", 2 * U, "flop"
@@ -106,9 +109,14 @@ def kernel_algorithmic(name: str, w, kinds_seen) -> tuple:
     if name == "dq":
         return "tensor", 1 * U, "flop"
     if name == "delta":
-        return "hbm", 2 * N * elem + 4 * R, "byte"
+        if w.dtype != "bf16":  # Delta only
+            return "hbm", 2 * N * elem + 4 * R, "byte"
+        # bf16 backward preparation: read o, dO, lse; write -Delta and -lse*log2e,
+        # zero the fp32 dq accumulator; with RoPE also rotate q and k
+        rope = 2 * (N + Nkv) * elem if w.rope_cos is not None else 0
+        return "hbm", 2 * N * elem + 12 * R + 4 * N + rope, "byte"
     if name == "rope_prep":
-        return "hbm", 4 * N * elem, "byte"
+        return "hbm", 2 * (N + Nkv) * elem, "byte"
     if name == "dq_finalize":
         return "hbm", N * 4 + N * elem, "byte"
     return "hbm", 0, "byte"
@@ -261,7 +269,8 @@ def run_reference(args):
 
 
 def workload_config(w, l2):
-    c = {"workload": w.cfg.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D, "rope": w.rope_cos is not None,
+    c = {"workload": w.cfg.name, "B": w.B, "H": w.H, "H_kv": w.kv_heads, "T": w.T, "D": w.D,
+         "rope": w.rope_cos is not None,
          "varlen": w.cu_seqlens is not None, "global_batch": w.B, "seq_len": w.T,
          "parallelism": "replicas (one independent workload per GPU)", "l2": l2,
          "flops_per_step_nominal": w.cfg.nominal_flops if (w.B, w.T, w.D) == (w.cfg.B, w.cfg.T, w.cfg.D)
@@ -303,7 +312,7 @@ def run_ours(args):
         return float(t.item())
 
     cfg = config_by_name(args.workload)
-    w = make_workload(cfg)
+    w = make_workload(cfg, H_kv=args.kv_heads)
     stream = torch.cuda.Stream(dev)
     r = AttnRunner.from_workload(w, device=dev, stream=stream)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -376,7 +385,8 @@ def run_ours(args):
             peak_note = f"hbm_gbs ({peak_src})"
         roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
                     "unit": unit, "frac": achieved / peak,
-                    "traffic": measured_traffic(dom, w.cfg.name) if (w.B, w.T) == (cfg.B, cfg.T) else None,
+                    "traffic": (measured_traffic(dom, w.cfg.name)
+                                if (w.B, w.T) == (cfg.B, cfg.T) and w.kv_heads == w.H else None),
                     "traffic_unit": "bytes per launch (ncu dram read + write)",
                     "algorithmic_per_launch": kd["algorithmic"],
                     "algorithmic_unit": kd["algorithmic_unit"],

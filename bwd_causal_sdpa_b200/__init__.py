@@ -38,6 +38,10 @@ _SIGNATURES = {
                       ctypes.c_size_t, _P]),
     "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float, _I,
                       _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "attn_fwd_gqa": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I,
+                          _P, ctypes.c_size_t, _P]),
+    "attn_bwd_gqa": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.c_float,
+                          _I, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float,
                               _I, _P, _P, _P, _P]),
     "attn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
@@ -111,6 +115,24 @@ def attn_bwd(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, T, D, sc
                              _ptr(rope_cos), _ptr(rope_sin), _ptr(cu_seqlens), B, H, T, D,
                              float(scale), dtype, _ptr(dq), _ptr(dk), _ptr(dv),
                              _ptr(workspace), int(ws_bytes), _stream(stream)))
+
+
+def attn_fwd_gqa(q, k, v, rope_cos, rope_sin, cu_seqlens, o, lse, B, H, H_kv, T, D, scale,
+                 dtype, workspace, ws_bytes, stream=None) -> int:
+    """attn_fwd with k, v of H_kv heads (grouped-query attention)."""
+    return int(_lib.attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin),
+                                 _ptr(cu_seqlens), _ptr(o), _ptr(lse), B, H, H_kv, T, D,
+                                 float(scale), dtype, _ptr(workspace), int(ws_bytes),
+                                 _stream(stream)))
+
+
+def attn_bwd_gqa(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, H_kv, T, D, scale,
+                 dtype, dq, dk, dv, workspace, ws_bytes, stream=None) -> int:
+    """attn_bwd with k, v, dk, dv of H_kv heads (grouped-query attention)."""
+    return int(_lib.attn_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse),
+                                 _ptr(rope_cos), _ptr(rope_sin), _ptr(cu_seqlens), B, H, H_kv,
+                                 T, D, float(scale), dtype, _ptr(dq), _ptr(dk), _ptr(dv),
+                                 _ptr(workspace), int(ws_bytes), _stream(stream)))
 
 
 def attn_bwd_noalloc(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, T, D, scale,

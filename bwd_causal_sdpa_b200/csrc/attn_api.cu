@@ -131,11 +131,12 @@ bool ensure_smem(K kernel, int bytes, bool* done_per_device) {
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 int check_common(const void* q, const void* k, const void* v, const float* rc, const float* rs,
-                 const int32_t* cu, int B, int H, int T, int D, float scale, int dtype,
+                 const int32_t* cu, int B, int H, int H_kv, int T, int D, float scale, int dtype,
                  void* ws, size_t ws_bytes, int is_bwd) {
   if (!q || !k || !v) return ATTN_EINVAL;
   if (dtype != ATTN_BF16 && dtype != ATTN_F32) return ATTN_EINVAL;
   if (B <= 0 || H <= 0 || T <= 0) return ATTN_EINVAL;
+  if (H_kv <= 0 || H % H_kv != 0) return ATTN_EINVAL;
   if (!isfinite(scale)) return ATTN_EINVAL;
   if ((rc == nullptr) != (rs == nullptr)) return ATTN_EINVAL;
   if (!sizes_ok(B, H, T, D)) return ATTN_EUNSUPPORTED;
@@ -156,45 +157,45 @@ int launch_status() {
 
 template <typename TIO, int D>
 int fwd_simt(const void* q, const void* k, const void* v, const float* rc, const float* rs,
-             const int32_t* ds, void* o, float* lse, int B, int H, int T, float scale,
+             const int32_t* ds, void* o, float* lse, int B, int H, int Hkv, int T, float scale,
              cudaStream_t st) {
   dim3 grid(B * H, (T + 15) / 16);
   ATTN_LAUNCH(KK_FWD, st,
               simt_fwd_kernel<TIO, D><<<grid, 128, 0, st>>>((const TIO*)q, (const TIO*)k,
                                                             (const TIO*)v, rc, rs, ds, (TIO*)o,
-                                                            lse, H, T, scale));
+                                                            lse, H, Hkv, T, scale));
   return launch_status();
 }
 
 template <typename TIO, int D>
 int bwd_simt(const void* q, const void* k, const void* v, const void* o, const void* dO,
              const float* lse, const float* rc, const float* rs, const int32_t* ds,
-             const int32_t* de, float* delta, void* dq, void* dk, void* dv, int B, int H, int T,
-             float scale, cudaStream_t st) {
+             const int32_t* de, float* delta, void* dq, void* dk, void* dv, int B, int H, int Hkv,
+             int T, float scale, cudaStream_t st) {
   const long rows = (long)B * H * T;
   ATTN_LAUNCH(KK_DELTA, st,
               delta_kernel<TIO, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
                   (const TIO*)o, (const TIO*)dO, delta, rows));
   if (launch_status()) return ATTN_ECUDA;
-  dim3 g1(B * H, (T + 31) / 32);
+  dim3 g1(B * Hkv, (T + 31) / 32), g2(B * H, (T + 31) / 32);
   ATTN_LAUNCH(KK_DKDV, st,
               simt_dkdv_kernel<TIO, D><<<g1, 128, 0, st>>>(
                   (const TIO*)q, (const TIO*)k, (const TIO*)v, (const TIO*)dO, lse, delta, rc, rs,
-                  ds, de, (TIO*)dk, (TIO*)dv, H, T, scale));
+                  ds, de, (TIO*)dk, (TIO*)dv, H, Hkv, T, scale));
   if (launch_status()) return ATTN_ECUDA;
   ATTN_LAUNCH(KK_DQ, st,
-              simt_dq_kernel<TIO, D><<<g1, 128, 0, st>>>(
+              simt_dq_kernel<TIO, D><<<g2, 128, 0, st>>>(
                   (const TIO*)q, (const TIO*)k, (const TIO*)v, (const TIO*)dO, lse, delta, rc, rs,
-                  ds, (TIO*)dq, H, T, scale));
+                  ds, (TIO*)dq, H, Hkv, T, scale));
   return launch_status();
 }
 
 template <int D>
 int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const float* rs,
-           const int32_t* ds, void* o, float* lse, int B, int H, int T, float scale, char* ws,
-           const WsPlan& wp, cudaStream_t st) {
+           const int32_t* ds, void* o, float* lse, int B, int H, int Hkv, int T, float scale,
+           char* ws, const WsPlan& wp, cudaStream_t st) {
   using L = fwd100::Layout<D>;
-  const int nt = (T + 127) / 128, BH = B * H;
+  const int nt = (T + 127) / 128, BH = B * H, BHkv = B * Hkv;
   const void* qs = q;
   const void* ks = k;
   bool f16 = false;
@@ -207,15 +208,15 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
     ATTN_LAUNCH(KK_ROPE_PREP, st,
                 rope_prep_kernel<__half, D, true><<<dim3(nt, BH, 2), 256, 0, st>>>(
                     (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qh, kh, qf, kf,
-                    H, T, nt));
+                    H, Hkv, T, nt));
     if (launch_status()) return ATTN_ECUDA;
     qs = qh;
     ks = kh;
     f16 = true;
   }
   CUtensorMap mq, mk, mv;
-  if (!make_tile_map(&mq, qs, f16, D, T, BH) || !make_tile_map(&mk, ks, f16, D, T, BH) ||
-      !make_tile_map(&mv, v, false, D, T, BH))
+  if (!make_tile_map(&mq, qs, f16, D, T, BH) || !make_tile_map(&mk, ks, f16, D, T, BHkv) ||
+      !make_tile_map(&mv, v, false, D, T, BHkv))
     return ATTN_ECUDA;
   static bool smem_set[64] = {};
   if (!ensure_smem(fwd100::fwd_kernel<D>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
@@ -223,6 +224,7 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
   const int n_pairs = (nt + 1) / 2;
   prm.T = T;
   prm.H = H;
+  prm.Hkv = Hkv;
   prm.BH = BH;
   prm.n_pairs = n_pairs;
   prm.n_qtiles = nt;
@@ -242,10 +244,10 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
 template <int D>
 int bwd_tc(const void* q, const void* k, const void* v, const void* o, const void* dO,
            const float* lse, const float* rc, const float* rs, const int32_t* ds,
-           const int32_t* de, void* dq, void* dk, void* dv, int B, int H, int T, float scale,
-           char* ws, const WsPlan& wp, cudaStream_t st) {
+           const int32_t* de, void* dq, void* dk, void* dv, int B, int H, int Hkv, int T,
+           float scale, char* ws, const WsPlan& wp, cudaStream_t st) {
   using L = bwd100::Layout<D>;
-  const int nt = (T + 127) / 128, BH = B * H, Tpad = nt * 128;
+  const int nt = (T + 127) / 128, BH = B * H, BHkv = B * Hkv, Tpad = nt * 128;
   __nv_bfloat16* qr = (__nv_bfloat16*)(ws + wp.q16);
   __nv_bfloat16* kr = (__nv_bfloat16*)(ws + wp.k16);
   const void* qs = rc ? (const void*)qr : q;
@@ -257,12 +259,12 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   ATTN_LAUNCH(KK_DELTA, st,
               bwd_prep_kernel<D><<<(unsigned)((rows_pad + 7) / 8), 256, 0, st>>>(
                   (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse, delta, lse2, dq_acc,
-                  (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qr, kr, H, T,
-                  Tpad, rows_pad));
+                  (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qr, kr, H, Hkv,
+                  T, Tpad, rows_pad));
   if (launch_status()) return ATTN_ECUDA;
   CUtensorMap mq, mk, mv, mo, mdq;
-  if (!make_tile_map(&mq, qs, false, D, T, BH) || !make_tile_map(&mk, ks, false, D, T, BH) ||
-      !make_tile_map(&mv, v, false, D, T, BH) || !make_tile_map(&mo, dO, false, D, T, BH) ||
+  if (!make_tile_map(&mq, qs, false, D, T, BH) || !make_tile_map(&mk, ks, false, D, T, BHkv) ||
+      !make_tile_map(&mv, v, false, D, T, BHkv) || !make_tile_map(&mo, dO, false, D, T, BH) ||
       !make_acc_map(&mdq, dq_acc, D, T, BH))
     return ATTN_ECUDA;
   static bool smem_set[64] = {};
@@ -270,7 +272,8 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   bwd100::Params prm;
   prm.T = T;
   prm.H = H;
-  prm.BH = BH;
+  prm.Hkv = Hkv;
+  prm.BHkv = BHkv;
   prm.n_tiles = nt;
   prm.Tpad = Tpad;
   prm.scale_log2 = scale * 1.4426950408889634f;
@@ -285,7 +288,7 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   prm.dk = (__nv_bfloat16*)dk;
   prm.dv = (__nv_bfloat16*)dv;
   ATTN_LAUNCH(KK_DKDV, st,
-              bwd100::dkdv_kernel<D><<<(unsigned)(nt * BH), L::kThreads, L::kSmemAlloc, st>>>(
+              bwd100::dkdv_kernel<D><<<(unsigned)(nt * BHkv), L::kThreads, L::kSmemAlloc, st>>>(
                   mq, mk, mv, mo, mdq, prm));
   if (launch_status()) return ATTN_ECUDA;
   const long n8 = (long)BH * T * D / 8;
@@ -309,11 +312,11 @@ size_t attn_workspace_bytes(int B, int H, int T, int D, int dtype, int is_bwd) {
   return plan(B, H, T, D, dtype, is_bwd).total;
 }
 
-int attn_fwd(const void* q, const void* k, const void* v, const float* rope_cos,
-             const float* rope_sin, const int32_t* cu_seqlens, void* o, float* lse, int B, int H,
-             int T, int D, float scale, int dtype, void* workspace, size_t ws_bytes,
-             void* stream) {
-  int rc = check_common(q, k, v, rope_cos, rope_sin, cu_seqlens, B, H, T, D, scale, dtype,
+int attn_fwd_gqa(const void* q, const void* k, const void* v, const float* rope_cos,
+                 const float* rope_sin, const int32_t* cu_seqlens, void* o, float* lse, int B,
+                 int H, int H_kv, int T, int D, float scale, int dtype, void* workspace,
+                 size_t ws_bytes, void* stream) {
+  int rc = check_common(q, k, v, rope_cos, rope_sin, cu_seqlens, B, H, H_kv, T, D, scale, dtype,
                         workspace, ws_bytes, 0);
   if (rc) return rc;
   if (!o || !lse) return ATTN_EINVAL;
@@ -330,18 +333,31 @@ int attn_fwd(const void* q, const void* k, const void* v, const float* rope_cos,
     if (launch_status()) return ATTN_ECUDA;
   }
   if (dtype == ATTN_F32) {
-    return D == 64 ? fwd_simt<float, 64>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, T, scale, st)
-                   : fwd_simt<float, 128>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, T, scale, st);
+    return D == 64 ? fwd_simt<float, 64>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, H_kv, T,
+                                         scale, st)
+                   : fwd_simt<float, 128>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, H_kv, T,
+                                          scale, st);
   }
-  return D == 64 ? fwd_tc<64>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, T, scale, ws, p, st)
-                 : fwd_tc<128>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, T, scale, ws, p, st);
+  return D == 64 ? fwd_tc<64>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, H_kv, T, scale, ws,
+                              p, st)
+                 : fwd_tc<128>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, H_kv, T, scale, ws,
+                               p, st);
 }
 
-int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
-             const float* lse, const float* rope_cos, const float* rope_sin,
-             const int32_t* cu_seqlens, int B, int H, int T, int D, float scale, int dtype,
-             void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream) {
-  int rc = check_common(q, k, v, rope_cos, rope_sin, cu_seqlens, B, H, T, D, scale, dtype,
+int attn_fwd(const void* q, const void* k, const void* v, const float* rope_cos,
+             const float* rope_sin, const int32_t* cu_seqlens, void* o, float* lse, int B, int H,
+             int T, int D, float scale, int dtype, void* workspace, size_t ws_bytes,
+             void* stream) {
+  return attn_fwd_gqa(q, k, v, rope_cos, rope_sin, cu_seqlens, o, lse, B, H, H, T, D, scale,
+                      dtype, workspace, ws_bytes, stream);
+}
+
+int attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, const float* rope_cos, const float* rope_sin,
+                 const int32_t* cu_seqlens, int B, int H, int H_kv, int T, int D, float scale,
+                 int dtype, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                 void* stream) {
+  int rc = check_common(q, k, v, rope_cos, rope_sin, cu_seqlens, B, H, H_kv, T, D, scale, dtype,
                         workspace, ws_bytes, 1);
   if (rc) return rc;
   if (!o || !dO || !lse || !dq || !dk || !dv) return ATTN_EINVAL;
@@ -361,14 +377,22 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
   float* delta = (float*)(ws + p.delta);
   if (dtype == ATTN_F32) {
     return D == 64 ? bwd_simt<float, 64>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, delta,
-                                         dq, dk, dv, B, H, T, scale, st)
+                                         dq, dk, dv, B, H, H_kv, T, scale, st)
                    : bwd_simt<float, 128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, delta,
-                                          dq, dk, dv, B, H, T, scale, st);
+                                          dq, dk, dv, B, H, H_kv, T, scale, st);
   }
   return D == 64 ? bwd_tc<64>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, dq, dk, dv, B, H,
-                              T, scale, ws, p, st)
+                              H_kv, T, scale, ws, p, st)
                  : bwd_tc<128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, dq, dk, dv, B, H,
-                               T, scale, ws, p, st);
+                               H_kv, T, scale, ws, p, st);
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+             const float* lse, const float* rope_cos, const float* rope_sin,
+             const int32_t* cu_seqlens, int B, int H, int T, int D, float scale, int dtype,
+             void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream) {
+  return attn_bwd_gqa(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, H, T, D, scale,
+                      dtype, dq, dk, dv, workspace, ws_bytes, stream);
 }
 
 int attn_get_status(void* stream) {
@@ -505,12 +529,12 @@ extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, con
   float* delta = (float*)(ws + p.delta);
   if (dtype == ATTN_F32) {
     return D == 64 ? bwd_simt<float, 64>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, delta,
-                                         dq, dk, dv, B, H, T, scale, st)
+                                         dq, dk, dv, B, H, H, T, scale, st)
                    : bwd_simt<float, 128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, delta,
-                                          dq, dk, dv, B, H, T, scale, st);
+                                          dq, dk, dv, B, H, H, T, scale, st);
   }
   return D == 64 ? bwd_simt<__nv_bfloat16, 64>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de,
-                                               delta, dq, dk, dv, B, H, T, scale, st)
+                                               delta, dq, dk, dv, B, H, H, T, scale, st)
                  : bwd_simt<__nv_bfloat16, 128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de,
-                                                delta, dq, dk, dv, B, H, T, scale, st);
+                                                delta, dq, dk, dv, B, H, H, T, scale, st);
 }

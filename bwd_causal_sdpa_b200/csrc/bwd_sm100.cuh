@@ -81,17 +81,17 @@ struct Layout {
 };
 
 struct Params {
-  int T, H, BH, n_tiles, Tpad;
+  int T, H, Hkv, BHkv, n_tiles, Tpad;  // H query heads read Hkv key/value heads
   float scale_log2;  // scale * log2(e)
   float scale;
-  const float* lse2;       // [BH][Tpad] -lse * log2(e), zero-padded
-  const float* delta;      // [BH][Tpad] -Delta, zero-padded
+  const float* lse2;       // [B*H][Tpad] -lse * log2(e), zero-padded
+  const float* delta;      // [B*H][Tpad] -Delta, zero-padded
   const int32_t* doc_start;
   const int32_t* doc_end;  // flattened, or null
   const float* rope_cos;   // [T][D/2] or null
   const float* rope_sin;
-  float* dq_acc;           // [BH][T][D] fp32
-  __nv_bfloat16* dk;
+  float* dq_acc;           // [B*H][T][D] fp32
+  __nv_bfloat16* dk;       // [B*Hkv][T][D]
   __nv_bfloat16* dv;
 };
 
@@ -121,15 +121,21 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.T;
   // Flattened grid, heaviest key tiles (the earliest, which see the most
-  // query tiles) first.
-  const int bh = (int)blockIdx.x % p.BH, b = bh / p.H;
-  const int kt = (int)blockIdx.x / p.BH;
+  // query tiles) first. One CTA per (key/value head, key tile); it walks the
+  // query tiles of every query head reading that key/value head (G of them),
+  // head by head: step `it` is query tile qt0 + it % n_q of the group's
+  // it / n_q-th head.
+  const int bhk = (int)blockIdx.x % p.BHkv, b = bhk / p.Hkv;
+  const int kt = (int)blockIdx.x / p.BHkv;
+  const int G = p.H / p.Hkv;
+  const int bhq0 = b * p.H + (bhk - b * p.Hkv) * G;  // first query head of the group
   const int j0 = kt * 128;
   const int row0 = b * T;
   const int jlast = min(j0 + 127, T - 1);
   const int q_end = p.doc_end ? p.doc_end[row0 + jlast] - row0 : T;  // exclusive
   const int qt0 = kt;
   const int n_q = (q_end + 127) / 128 - qt0;
+  const int n_it = G * n_q;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::bKV), 1);
@@ -169,15 +175,17 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       prefetch_tensor_map(&tmDO);
       mbar_arrive_expect_tx(bar(L::bKV), 2 * L::kTileBytes);
       for (int cb = 0; cb < D / 64; ++cb) {
-        tma_load_3d(sb0 + L::kK + cb * L::kBlockBytes, &tmK, bar(L::bKV), cb * 64, j0, bh);
-        tma_load_3d(sb0 + L::kV + cb * L::kBlockBytes, &tmV, bar(L::bKV), cb * 64, j0, bh);
+        tma_load_3d(sb0 + L::kK + cb * L::kBlockBytes, &tmK, bar(L::bKV), cb * 64, j0, bhk);
+        tma_load_3d(sb0 + L::kV + cb * L::kBlockBytes, &tmV, bar(L::bKV), cb * 64, j0, bhk);
       }
-      const float* lse2_bh = p.lse2 + (size_t)bh * p.Tpad;
-      const float* delta_bh = p.delta + (size_t)bh * p.Tpad;
-      for (int it = 0; it < n_q; ++it) {
+      for (int it = 0; it < n_it; ++it) {
         const int st = it & 1;
         const int so = it % L::kDOStages;
-        const int qrow = (qt0 + it) * 128;
+        const int gi = it / n_q;
+        const int bh = bhq0 + gi;
+        const int qrow = (qt0 + it - gi * n_q) * 128;
+        const float* lse2_bh = p.lse2 + (size_t)bh * p.Tpad;
+        const float* delta_bh = p.delta + (size_t)bh * p.Tpad;
         if (it >= 2 && !mbar_wait(bar(L::bQEmpty + st), ((it >> 1) - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar(L::bQFull + st), L::kTileBytes + 1024);
         for (int cb = 0; cb < D / 64; ++cb)
@@ -242,7 +250,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         return true;
       };
       bool ok = mbar_wait(bar(L::bKV), 0, abort_flag) && issue_S(0) && issue_dP(0);
-      for (int it = 0; ok && it < n_q; ++it) {
+      for (int it = 0; ok && it < n_it; ++it) {
         const int ph = it & 1;
         // dV += P^T dO; P^T of warpgroup g's query columns [g*kQC, (g+1)*kQC)
         // sits in TMEM columns [g*kQC, g*kQC + kQC/2), so the 16 queries of
@@ -256,7 +264,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
                  (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar(L::bDVDone));
         mma_commit(bar(L::bDOEmpty + it % L::kDOStages));
-        if (it + 1 < n_q && !issue_S(it + 1)) break;
+        if (it + 1 < n_it && !issue_S(it + 1)) break;
         // dK += dS^T Q ; dQ_i = dS K
         if (!mbar_wait(bar(L::bDSFull), ph, abort_flag)) break;
         tc_fence_after();
@@ -272,8 +280,8 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
                  smem_desc_sw128(sb0 + L::kK + kk * 2048, L::kBlockBytes, 1024), id_dq, kk > 0);
         mma_commit(bar(L::bDQFull));
         mma_commit(bar(L::bQEmpty + (it & 1)));
-        if (it == n_q - 1) mma_commit(bar(L::bFinal));
-        if (it + 1 < n_q && !issue_dP(it + 1)) break;
+        if (it == n_it - 1) mma_commit(bar(L::bFinal));
+        if (it + 1 < n_it && !issue_dP(it + 1)) break;
       }
     }
   } else {
@@ -292,7 +300,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     float pf[QC];  // P^T of this thread's key row, query columns [qc0, qc0 + QC)
     // ---- P^T(i) = exp2(S^T scale log2e - lse2), masked; bf16 copy to TMEM ----
     auto phase_P = [&](int i) -> bool {
-      const int i0 = (qt0 + i) * 128;
+      const int i0 = (qt0 + i % n_q) * 128;
       const bool need_mask = (i0 + qc0 < j) || (i0 + qc0 + QC - 1 >= de_j);
       const float* sl = reinterpret_cast<const float*>(sg + L::kLD + (i & 1) * 1024);
       if (!mbar_wait(bar(L::bQFull + (i & 1)), (i >> 1) & 1, abort_flag) ||
@@ -376,7 +384,8 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     };
     // ---- dQ_i (lane = query row): release TMEM first, then reduce into global ----
     auto phase_dQ = [&](int i) -> bool {
-      const int i0 = (qt0 + i) * 128;
+      const int gi = i / n_q;
+      const int i0 = (qt0 + i - gi * n_q) * 128;
       if (!mbar_wait(bar(L::bDQFull), i & 1, abort_flag)) return false;
       tc_fence_after();
       constexpr int NQC = DC / 32;  // 32-column chunks per warpgroup
@@ -406,7 +415,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         for (int c = 0; c < NQC; ++c) {
           const int box = warp * NQC + c;
           const uint32_t bx = (box < 8) ? sb0 + L::kDS + box * 4096 : sb0 + L::kXS + (box - 8) * 4096;
-          tma_reduce_add_3d(&tmDQ, bx, dc0 + 32 * c, i0 + 32 * sub, bh);
+          tma_reduce_add_3d(&tmDQ, bx, dc0 + 32 * c, i0 + 32 * sub, bhq0 + gi);
         }
         bulk_commit_group();
       }
@@ -414,8 +423,8 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     };
     // Order: P(0); then per tile i: dS(i), P(i+1), dQ(i).
     bool ok = phase_P(0);
-    for (int it = 0; ok && it < n_q; ++it) {
-      ok = phase_dS(it) && (it + 1 >= n_q || phase_P(it + 1)) && phase_dQ(it);
+    for (int it = 0; ok && it < n_it; ++it) {
+      ok = phase_dS(it) && (it + 1 >= n_it || phase_P(it + 1)) && phase_dQ(it);
     }
     bulk_wait_group0();
     // ---- epilogue: dK = R^T (scale * dK_r), dV ----
@@ -423,8 +432,8 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       tc_fence_after();
       const int jj = min(j, T - 1);
       const int pos = jj - (p.doc_start ? p.doc_start[row0 + jj] - row0 : 0);
-      __nv_bfloat16* dkrow = p.dk + ((size_t)bh * T + jj) * D;
-      __nv_bfloat16* dvrow = p.dv + ((size_t)bh * T + jj) * D;
+      __nv_bfloat16* dkrow = p.dk + ((size_t)bhk * T + jj) * D;
+      __nv_bfloat16* dvrow = p.dv + ((size_t)bhk * T + jj) * D;
 #pragma unroll
       for (int c = 0; c < DC / 32; ++c) {
         const int col = dc0 + 32 * c;

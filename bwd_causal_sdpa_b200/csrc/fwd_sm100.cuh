@@ -68,11 +68,11 @@ struct Layout {
 };
 
 struct Params {
-  int T, H, BH, n_pairs, n_qtiles;
+  int T, H, Hkv, BH, n_pairs, n_qtiles;  // H query heads read Hkv key/value heads
   float scale_log2;          // scale * log2(e)
   uint32_t idesc_s;          // instruction descriptor of S = Q K^T
   const float* q_fac;        // per (bh, tile) power-of-two factor of the stored q tile, or null
-  const float* k_fac;
+  const float* k_fac;        // indexed by (key/value head, tile)
   const int32_t* doc_start;  // flattened document starts, or null
   __nv_bfloat16* o;
   float* lse;
@@ -99,6 +99,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
   // Flattened grid, tile-major from the last tile pair: the longest rows (most
   // key tiles) are scheduled first.
   const int bh = (int)blockIdx.x % p.BH, b = bh / p.H;
+  const int bhk = b * p.Hkv + (bh - b * p.H) / (p.H / p.Hkv);  // its key/value head
   const int pr = p.n_pairs - 1 - (int)blockIdx.x / p.BH;
   const int qtA = 2 * pr, qtB = 2 * pr + 1;
   const bool hasB = qtB * 128 < T;
@@ -152,12 +153,12 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         mbar_arrive_expect_tx(bar(L::bKFull + st), L::kTileBytes);
         for (int cb = 0; cb < D / 64; ++cb)
           tma_load_3d(sb0 + L::kK + st * L::kTileBytes + cb * L::kBlockBytes, &tmK,
-                      bar(L::bKFull + st), cb * 64, kvrow, bh);
+                      bar(L::bKFull + st), cb * 64, kvrow, bhk);
         if (it >= L::kStages && !mbar_wait(bar(L::bVEmpty + st), (round - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar(L::bVFull + st), L::kTileBytes);
         for (int cb = 0; cb < D / 64; ++cb)
           tma_load_3d(sb0 + L::kV + st * L::kTileBytes + cb * L::kBlockBytes, &tmV,
-                      bar(L::bVFull + st), cb * 64, kvrow, bh);
+                      bar(L::bVFull + st), cb * 64, kvrow, bhk);
       }
     }
   } else if (warp == L::kMmaWarp) {
@@ -245,7 +246,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       if (!mbar_wait(bar(L::bSFull + t), it & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       // scale of this key tile's scores (q, k tiles may carry power-of-two factors)
-      const float sc = p.scale_log2 * fq * (p.k_fac ? p.k_fac[bh * p.n_qtiles + kt] : 1.f);
+      const float sc = p.scale_log2 * fq * (p.k_fac ? p.k_fac[bhk * p.n_qtiles + kt] : 1.f);
       const bool pos_scale = sc > 0.f;
       uint32_t s[128];
 #pragma unroll

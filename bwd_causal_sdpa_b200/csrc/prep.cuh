@@ -79,7 +79,8 @@ __global__ void __launch_bounds__(256) delta_kernel(const TIO* __restrict__ o, c
 // RoPE pre-pass for the tensor-core kernels: rotate q and k once (fp32
 // arithmetic, interleaved pairs at the token's document position) and store
 // the rotated tiles in the 16-bit type the MMAs read. blockIdx = (128-row
-// tile, b*H + h, 0 for q / 1 for k).
+// tile, head, 0 for q / 1 for k); the head is b*H + h for q and b*Hkv + h
+// for k (blocks past B*Hkv return at once).
 //
 // kTileScale (forward, fp16 output): fp16 keeps 3 more mantissa bits than
 // bf16, which the lse bound needs, but has a narrow range; a tile whose
@@ -92,13 +93,16 @@ __global__ void __launch_bounds__(256) rope_prep_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const float* __restrict__ rc, const float* __restrict__ rs,
     const int32_t* __restrict__ doc_start, OutT* __restrict__ qo, OutT* __restrict__ ko,
-    float* __restrict__ qfac, float* __restrict__ kfac, int H, int T, int ntiles) {
+    float* __restrict__ qfac, float* __restrict__ kfac, int H, int Hkv, int T, int ntiles) {
   constexpr int CH = D / 8;              // 16-byte chunks per row
   constexpr int PER = 128 * CH / 256;    // chunks per thread
+  // grid (ntiles, B*H, 2): z = 0 rotates q heads, z = 1 the B*Hkv k heads
   const int tile = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
+  const int heads = which ? Hkv : H;
+  const int b = bh / heads, row0 = b * T, t0 = tile * 128;
+  if (b >= (int)gridDim.y / H) return;  // k has fewer heads than q
   const __nv_bfloat16* src = which ? k : q;
   OutT* dst = which ? ko : qo;
-  const int b = bh / H, row0 = b * T, t0 = tile * 128;
   float v[PER][8];
   float amax = 0.f;
 #pragma unroll
@@ -163,8 +167,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
     float* __restrict__ dq_acc, const __nv_bfloat16* __restrict__ q,
     const __nv_bfloat16* __restrict__ k, const float* __restrict__ rc,
     const float* __restrict__ rs, const int32_t* __restrict__ doc_start,
-    __nv_bfloat16* __restrict__ qr, __nv_bfloat16* __restrict__ kr, int H, int T, int Tpad,
-    long rows_pad) {
+    __nv_bfloat16* __restrict__ qr, __nv_bfloat16* __restrict__ kr, int H, int Hkv, int T,
+    int Tpad, long rows_pad) {
   constexpr int NC = D / 32;
   const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -189,9 +193,15 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
       load_vec<NC>(q + r * D + lane * NC, x);
       rope_pairs<NC, D>(x, rc, rs, pos, lane * NC, false);
       store_vec<NC>(qr + r * D + lane * NC, x);
-      load_vec<NC>(k + r * D + lane * NC, x);
-      rope_pairs<NC, D>(x, rc, rs, pos, lane * NC, false);
-      store_vec<NC>(kr + r * D + lane * NC, x);
+      // row r of the [B*Hkv][T] k view exists for the first B*Hkv heads; its
+      // batch (hence document layout) is bh / Hkv
+      if (bh < (rows_pad / Tpad) / H * Hkv) {
+        const int bk = (int)(bh / Hkv);
+        const int posk = t - (doc_start ? doc_start[bk * T + t] - bk * T : 0);
+        load_vec<NC>(k + r * D + lane * NC, x);
+        rope_pairs<NC, D>(x, rc, rs, posk, lane * NC, false);
+        store_vec<NC>(kr + r * D + lane * NC, x);
+      }
     }
   }
   if (lane == 0) {

@@ -7,6 +7,8 @@
 //
 // Index conventions: bh = b*H + h; a row of one (b, h) slice is t in [0, T);
 // doc_start / doc_end (when non-null) hold flattened token indices b*T + t.
+// Grouped-query attention: k, v (and dk, dv) have Hkv heads; query head h
+// reads key/value head h / (H / Hkv).
 #pragma once
 
 #include "common.cuh"
@@ -30,7 +32,7 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(
     const TIO* __restrict__ q, const TIO* __restrict__ k, const TIO* __restrict__ v,
     const float* __restrict__ rc, const float* __restrict__ rs,
     const int32_t* __restrict__ doc_start, TIO* __restrict__ o, float* __restrict__ lse,
-    int H, int T, float scale) {
+    int H, int Hkv, int T, float scale) {
   constexpr int ROWS = 16, KC = 32, NC = D / 32, KP = D + 4;
   __shared__ __align__(16) float sQ[ROWS][D];
   __shared__ __align__(16) float sK[KC][KP];
@@ -39,6 +41,7 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(
   const int bh = blockIdx.x, b = bh / H;
   const int i0 = (gridDim.y - 1 - blockIdx.y) * ROWS;  // longest rows first
   const size_t base = (size_t)bh * T * D;
+  const size_t kvbase = ((size_t)b * Hkv + (bh % H) / (H / Hkv)) * T * D;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const DocView doc{doc_start, nullptr, b * T, T};
 
@@ -73,9 +76,9 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(
       const int r = idx / (D / 2), pi = idx % (D / 2), t = kb + r;
       float x[2] = {0.f, 0.f}, y[2] = {0.f, 0.f};
       if (t < iend) {
-        load_vec<2>(k + base + (size_t)t * D + 2 * pi, x);
+        load_vec<2>(k + kvbase + (size_t)t * D + 2 * pi, x);
         if (rc) rope_pairs<2, D>(x, rc, rs, t - doc.dstart(t), 2 * pi, false);
-        load_vec<2>(v + base + (size_t)t * D + 2 * pi, y);
+        load_vec<2>(v + kvbase + (size_t)t * D + 2 * pi, y);
       }
       sK[r][2 * pi] = x[0];
       sK[r][2 * pi + 1] = x[1];
@@ -146,15 +149,16 @@ __global__ void __launch_bounds__(128) simt_dkdv_kernel(
     const TIO* __restrict__ dO, const float* __restrict__ lse, const float* __restrict__ delta,
     const float* __restrict__ rc, const float* __restrict__ rs,
     const int32_t* __restrict__ doc_start, const int32_t* __restrict__ doc_end,
-    TIO* __restrict__ dk, TIO* __restrict__ dv, int H, int T, float scale) {
+    TIO* __restrict__ dk, TIO* __restrict__ dv, int H, int Hkv, int T, float scale) {
   constexpr int KC = 32, QC = 32, NC = D / 32, KW = 8;
   __shared__ __align__(16) float sQ[QC][D];
   __shared__ __align__(16) float sG[QC][D];
   __shared__ float sL[QC], sDl[QC];
 
-  const int bh = blockIdx.x, b = bh / H;
+  const int bhk = blockIdx.x, b = bhk / Hkv;  // key/value head of this block
+  const int G = H / Hkv;                       // query heads reading it
   const int j0 = (gridDim.y - 1 - blockIdx.y) * KC;
-  const size_t base = (size_t)bh * T * D;
+  const size_t base = (size_t)bhk * T * D;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const DocView doc{doc_start, doc_end, b * T, T};
 
@@ -176,15 +180,18 @@ __global__ void __launch_bounds__(128) simt_dkdv_kernel(
   const int jlast = min(j0 + KC, T) - 1;
   const int qhi = doc.dend(jlast);
 
+  for (int gi = 0; gi < G; ++gi) {
+  const int bhq = b * H + (bhk % Hkv) * G + gi;  // a query head of the group
+  const size_t qbase = (size_t)bhq * T * D;
   for (int ib = j0; ib < qhi; ib += QC) {
     __syncthreads();
     for (int idx = tid; idx < QC * (D / 2); idx += 128) {
       const int r = idx / (D / 2), pi = idx % (D / 2), t = ib + r;
       float x[2] = {0.f, 0.f}, g[2] = {0.f, 0.f};
       if (t < qhi) {
-        load_vec<2>(q + base + (size_t)t * D + 2 * pi, x);
+        load_vec<2>(q + qbase + (size_t)t * D + 2 * pi, x);
         if (rc) rope_pairs<2, D>(x, rc, rs, t - doc.dstart(t), 2 * pi, false);
-        load_vec<2>(dO + base + (size_t)t * D + 2 * pi, g);
+        load_vec<2>(dO + qbase + (size_t)t * D + 2 * pi, g);
       }
       sQ[r][2 * pi] = x[0];
       sQ[r][2 * pi + 1] = x[1];
@@ -193,8 +200,8 @@ __global__ void __launch_bounds__(128) simt_dkdv_kernel(
     }
     if (tid < QC) {
       const int t = ib + tid;
-      sL[tid] = t < qhi ? lse[(size_t)bh * T + t] : 0.f;
-      sDl[tid] = t < qhi ? delta[(size_t)bh * T + t] : 0.f;
+      sL[tid] = t < qhi ? lse[(size_t)bhq * T + t] : 0.f;
+      sDl[tid] = t < qhi ? delta[(size_t)bhq * T + t] : 0.f;
     }
     __syncthreads();
     const int iend = min(ib + QC, qhi);
@@ -226,6 +233,8 @@ __global__ void __launch_bounds__(128) simt_dkdv_kernel(
       }
     }
   }
+  __syncthreads();  // the next query head restages the shared tiles
+  }
 #pragma unroll
   for (int kk = 0; kk < KW; ++kk) {
     const int j = j0 + warp * KW + kk;
@@ -248,7 +257,8 @@ __global__ void __launch_bounds__(128) simt_dq_kernel(
     const TIO* __restrict__ q, const TIO* __restrict__ k, const TIO* __restrict__ v,
     const TIO* __restrict__ dO, const float* __restrict__ lse, const float* __restrict__ delta,
     const float* __restrict__ rc, const float* __restrict__ rs,
-    const int32_t* __restrict__ doc_start, TIO* __restrict__ dq, int H, int T, float scale) {
+    const int32_t* __restrict__ doc_start, TIO* __restrict__ dq, int H, int Hkv, int T,
+    float scale) {
   constexpr int QC = 32, KC = 32, NC = D / 32, QW = 8;
   __shared__ __align__(16) float sK[KC][D];
   __shared__ __align__(16) float sV[KC][D];
@@ -256,6 +266,7 @@ __global__ void __launch_bounds__(128) simt_dq_kernel(
   const int bh = blockIdx.x, b = bh / H;
   const int i0 = (gridDim.y - 1 - blockIdx.y) * QC;
   const size_t base = (size_t)bh * T * D;
+  const size_t kvbase = ((size_t)b * Hkv + (bh % H) / (H / Hkv)) * T * D;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const DocView doc{doc_start, nullptr, b * T, T};
 
@@ -288,9 +299,9 @@ __global__ void __launch_bounds__(128) simt_dq_kernel(
       const int r = idx / (D / 2), pi = idx % (D / 2), t = jb + r;
       float x[2] = {0.f, 0.f}, y[2] = {0.f, 0.f};
       if (t < kv_hi) {
-        load_vec<2>(k + base + (size_t)t * D + 2 * pi, x);
+        load_vec<2>(k + kvbase + (size_t)t * D + 2 * pi, x);
         if (rc) rope_pairs<2, D>(x, rc, rs, t - doc.dstart(t), 2 * pi, false);
-        load_vec<2>(v + base + (size_t)t * D + 2 * pi, y);
+        load_vec<2>(v + kvbase + (size_t)t * D + 2 * pi, y);
       }
       sK[r][2 * pi] = x[0];
       sK[r][2 * pi + 1] = x[1];

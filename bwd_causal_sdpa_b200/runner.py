@@ -13,8 +13,8 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (ATTN_BF16, ATTN_F32, attn_bwd, attn_fwd, attn_get_status, attn_workspace_bytes,
-               check)
+from . import (ATTN_BF16, ATTN_F32, attn_bwd, attn_bwd_gqa, attn_fwd, attn_fwd_gqa,
+               attn_get_status, attn_workspace_bytes, check)
 
 
 def torch_dtype(dtype: int):
@@ -35,23 +35,25 @@ class Problem:
     D: int
     scale: float
     dtype: int
+    H_kv: int
 
 
 class AttnRunner:
     """Holds q, k, v, dO (inputs), o, lse, dq, dk, dv (outputs), the RoPE
     tables, cu_seqlens and one workspace sized for the larger of the two
-    calls, all on one device."""
+    calls, all on one device. With H_kv < H (grouped-query attention) k, v,
+    dk, dv have H_kv heads and the *_gqa entry points are called."""
 
     def __init__(self, B, H, T, D, *, dtype=ATTN_BF16, scale=None, rope=None, cu_seqlens=None,
-                 device="cuda", stream: Optional[torch.cuda.Stream] = None):
-        self.p = Problem(B, H, T, D, 1.0 / math.sqrt(D) if scale is None else scale, dtype)
+                 device="cuda", stream: Optional[torch.cuda.Stream] = None, H_kv=None):
+        H_kv = H if H_kv is None else H_kv
+        self.p = Problem(B, H, T, D, 1.0 / math.sqrt(D) if scale is None else scale, dtype, H_kv)
         self.device = torch.device(device)
         self.stream = stream
         td = torch_dtype(dtype)
-        shape = (B, H, T, D)
-        mk = lambda: torch.empty(shape, dtype=td, device=self.device)
-        self.q, self.k, self.v, self.do = mk(), mk(), mk(), mk()
-        self.o, self.dq, self.dk, self.dv = mk(), mk(), mk(), mk()
+        mk = lambda h: torch.empty((B, h, T, D), dtype=td, device=self.device)
+        self.q, self.k, self.v, self.do = mk(H), mk(H_kv), mk(H_kv), mk(H)
+        self.o, self.dq, self.dk, self.dv = mk(H), mk(H), mk(H_kv), mk(H_kv)
         self.lse = torch.empty((B, H, T), dtype=torch.float32, device=self.device)
         self.rope_cos = self.rope_sin = None
         if rope is not None:
@@ -70,7 +72,7 @@ class AttnRunner:
         dtype = ATTN_BF16 if w.dtype == "bf16" else ATTN_F32
         rope = None if w.rope_cos is None else (w.rope_cos, w.rope_sin)
         r = cls(w.B, w.H, w.T, w.D, dtype=dtype, scale=w.scale, rope=rope,
-                cu_seqlens=w.cu_seqlens, device=device, stream=stream)
+                cu_seqlens=w.cu_seqlens, device=device, stream=stream, H_kv=w.kv_heads)
         r.load_inputs(w.q, w.k, w.v, w.do)
         return r
 
@@ -80,12 +82,23 @@ class AttnRunner:
 
     def forward(self) -> None:
         p = self.p
+        if p.H_kv != p.H:
+            check(attn_fwd_gqa(self.q, self.k, self.v, self.rope_cos, self.rope_sin, self.cu,
+                               self.o, self.lse, p.B, p.H, p.H_kv, p.T, p.D, p.scale, p.dtype,
+                               self.ws, self.ws_bytes, self.stream), "attn_fwd_gqa")
+            return
         check(attn_fwd(self.q, self.k, self.v, self.rope_cos, self.rope_sin, self.cu, self.o,
                        self.lse, p.B, p.H, p.T, p.D, p.scale, p.dtype, self.ws, self.ws_bytes,
                        self.stream), "attn_fwd")
 
     def backward(self) -> None:
         p = self.p
+        if p.H_kv != p.H:
+            check(attn_bwd_gqa(self.q, self.k, self.v, self.o, self.do, self.lse, self.rope_cos,
+                               self.rope_sin, self.cu, p.B, p.H, p.H_kv, p.T, p.D, p.scale,
+                               p.dtype, self.dq, self.dk, self.dv, self.ws, self.ws_bytes,
+                               self.stream), "attn_bwd_gqa")
+            return
         check(attn_bwd(self.q, self.k, self.v, self.o, self.do, self.lse, self.rope_cos,
                        self.rope_sin, self.cu, p.B, p.H, p.T, p.D, p.scale, p.dtype, self.dq,
                        self.dk, self.dv, self.ws, self.ws_bytes, self.stream), "attn_bwd")

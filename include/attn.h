@@ -105,6 +105,34 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o,
              void* dq, void* dk, void* dv,
              void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * Grouped-query attention (Forge README, "Architecture", Model line: the
+ * attention is GQA with RoPE). k and v have H_kv heads, H_kv dividing H; query
+ * head h reads key/value head h / (H / H_kv), and the gradient of a shared
+ * key/value head is the sum over the H / H_kv query heads that read it.
+ *
+ * attn_fwd_gqa / attn_bwd_gqa take the arguments of attn_fwd / attn_bwd plus
+ * H_kv (after H) and follow their rules, with these shapes:
+ *   q, o, dO, dq [B, H, T, D]; k, v, dk, dv [B, H_kv, T, D]; lse [B, H, T].
+ * Workspace: attn_workspace_bytes(B, H, T, D, dtype, is_bwd) bytes (sized by
+ * the query heads H). H_kv <= 0 or H not a multiple of H_kv: ATTN_EINVAL.
+ * attn_fwd and attn_bwd are these calls with H_kv = H.
+ */
+int attn_fwd_gqa(const void* q, const void* k, const void* v,
+                 const float* rope_cos, const float* rope_sin,
+                 const int32_t* cu_seqlens,
+                 void* o, float* lse,
+                 int B, int H, int H_kv, int T, int D, float scale,
+                 int dtype, void* workspace, size_t ws_bytes, void* stream);
+
+int attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                 const void* dO, const float* lse,
+                 const float* rope_cos, const float* rope_sin,
+                 const int32_t* cu_seqlens,
+                 int B, int H, int H_kv, int T, int D, float scale, int dtype,
+                 void* dq, void* dk, void* dv,
+                 void* workspace, size_t ws_bytes, void* stream);
+
 /* Bytes of workspace attn_fwd (is_bwd = 0) or attn_bwd (is_bwd = 1) needs for
  * these sizes; 0 for invalid sizes. Pure host function, no CUDA call. */
 size_t attn_workspace_bytes(int B, int H, int T, int D, int dtype, int is_bwd);

@@ -43,14 +43,23 @@ def gpu_outputs(w, *, runner_cls=None) -> dict:
 
 
 def compare(w, got: dict, ref: dict, heads=None) -> dict:
-    """Errors per tensor over the compared (b, h) slices; asserts the bounds."""
+    """Errors per tensor over the compared (b, h) query slices; asserts the
+    bounds. dk and dv are compared on the key/value heads those slices read,
+    which must come with every query head of their group (the oracle sums a
+    shared head's gradient over the listed query heads only)."""
     if heads is None:
         heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    G = w.H // w.kv_heads
+    kv_heads = sorted({(b, h // G) for b, h in heads})
+    listed = set(heads)
+    for b, hk in kv_heads:
+        assert all((b, hk * G + g) in listed for g in range(G)), "incomplete query-head group"
     tol = TOL[w.dtype]
     errs = {}
     for key in ("o", "lse", "dq", "dk", "dv"):
-        g = np.stack([got[key][b, h] for b, h in heads])
-        r = np.stack([ref[key][b, h] for b, h in heads])
+        pairs = kv_heads if key in ("dk", "dv") else heads
+        g = np.stack([got[key][b, h] for b, h in pairs])
+        r = np.stack([ref[key][b, h] for b, h in pairs])
         assert np.all(np.isfinite(g)), f"{key}: non-finite values"
         errs[key] = rel_fro(g, r)
     bad = {k: (e, tol[k]) for k, e in errs.items() if not e <= tol[k]}

@@ -108,3 +108,36 @@ def test_bwd_specific_validation():
     assert _bwd(dv=P + 8) == A.ATTN_EALIGN
     assert _fwd(lse=None) == A.ATTN_EINVAL
     assert _fwd(o=P + 2) == A.ATTN_EALIGN
+
+
+def _fwd_gqa(**kw):
+    import bwd_causal_sdpa_b200 as A
+
+    a = dict(q=P, k=P, v=P, rope_cos=None, rope_sin=None, cu_seqlens=None, o=P, lse=P, B=1, H=4,
+             H_kv=2, T=128, D=64, scale=0.125, dtype=A.ATTN_BF16, workspace=P, ws_bytes=1 << 30)
+    a.update(kw)
+    return A.attn_fwd_gqa(**a)
+
+
+def _bwd_gqa(**kw):
+    import bwd_causal_sdpa_b200 as A
+
+    a = dict(q=P, k=P, v=P, o=P, dO=P, lse=P, rope_cos=None, rope_sin=None, cu_seqlens=None,
+             B=1, H=4, H_kv=2, T=128, D=64, scale=0.125, dtype=A.ATTN_BF16, dq=P, dk=P, dv=P,
+             workspace=P, ws_bytes=1 << 30)
+    a.update(kw)
+    return A.attn_bwd_gqa(**a)
+
+
+@pytest.mark.parametrize("call", [_fwd_gqa, _bwd_gqa])
+def test_grouped_query_host_validation(call):
+    import bwd_causal_sdpa_b200 as A
+
+    assert call(H_kv=0) == A.ATTN_EINVAL
+    assert call(H_kv=-2) == A.ATTN_EINVAL
+    assert call(H_kv=3) == A.ATTN_EINVAL       # 4 query heads do not split into 3 groups
+    assert call(H_kv=8) == A.ATTN_EINVAL       # more key/value heads than query heads
+    assert call(q=None) == A.ATTN_EINVAL
+    assert call(D=96) == A.ATTN_EUNSUPPORTED
+    assert call(v=P + 8) == A.ATTN_EALIGN
+    assert call(ws_bytes=16) == A.ATTN_EWORKSPACE

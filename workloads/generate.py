@@ -80,6 +80,11 @@ class Workload:
     rope_cos: Optional[np.ndarray]
     rope_sin: Optional[np.ndarray]
     scale: float
+    H_kv: Optional[int] = None  # key/value heads (grouped-query attention); None = H
+
+    @property
+    def kv_heads(self) -> int:
+        return self.H if self.H_kv is None else self.H_kv
 
     @property
     def dtype(self) -> str:
@@ -101,9 +106,10 @@ def make_workload(cfg: Config, *, B: Optional[int] = None, H: Optional[int] = No
                   T: Optional[int] = None, D: Optional[int] = None,
                   seed: Optional[int] = None, varlen: Optional[bool] = None,
                   rope: Optional[bool] = None, doc_min: Optional[int] = None,
-                  doc_max: Optional[int] = None) -> Workload:
+                  doc_max: Optional[int] = None, H_kv: Optional[int] = None) -> Workload:
     """Draw one workload. Keyword overrides give smaller parity cases with the
-    same value distributions and structure as ``cfg``."""
+    same value distributions and structure as ``cfg``; ``H_kv`` (dividing H)
+    draws k and v with that many heads for grouped-query attention."""
     B = cfg.B if B is None else B
     H = cfg.H if H is None else H
     T = cfg.T if T is None else T
@@ -114,11 +120,14 @@ def make_workload(cfg: Config, *, B: Optional[int] = None, H: Optional[int] = No
     doc_min = cfg.doc_min if doc_min is None else doc_min
     doc_max = cfg.doc_max if doc_max is None else doc_max
 
+    if H_kv is not None and (H_kv <= 0 or H % H_kv):
+        raise ValueError("H_kv must divide H")
     rng = np.random.default_rng(seed)
     shape = (B, H, T, D)
+    kv_shape = shape if H_kv is None else (B, H_kv, T, D)
     q = rng.standard_normal(shape, dtype=np.float32) * np.float32(cfg.qk_std)
-    k = rng.standard_normal(shape, dtype=np.float32) * np.float32(cfg.qk_std)
-    v = rng.standard_normal(shape, dtype=np.float32) * np.float32(cfg.v_std)
+    k = rng.standard_normal(kv_shape, dtype=np.float32) * np.float32(cfg.qk_std)
+    v = rng.standard_normal(kv_shape, dtype=np.float32) * np.float32(cfg.v_std)
     do = rng.standard_normal(shape, dtype=np.float32) * np.float32(cfg.do_std)
     cu = draw_doc_lengths(rng, B, T, doc_min, doc_max) if varlen else None
     if cfg.dtype == "bf16":
@@ -127,4 +136,4 @@ def make_workload(cfg: Config, *, B: Optional[int] = None, H: Optional[int] = No
         rc, rs = rope_tables_f32(T, D, cfg.theta)
     else:
         rc = rs = None
-    return Workload(cfg, B, H, T, D, q, k, v, do, cu, rc, rs, 1.0 / float(np.sqrt(D)))
+    return Workload(cfg, B, H, T, D, q, k, v, do, cu, rc, rs, 1.0 / float(np.sqrt(D)), H_kv)
