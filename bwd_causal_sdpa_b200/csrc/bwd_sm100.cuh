@@ -1,30 +1,36 @@
 // bwd_sm100.cuh -- tensor-core (tcgen05) attention backward, key-tile
 // parallel, for bf16 storage.
 //
-// One CTA owns one 128-key tile of one (b, h) slice; K and V stay in shared
+// One CTA owns one 128-key tile of one key/value head; K and V stay in shared
 // memory and the dK, dV accumulators stay in TMEM while the query tiles that
 // can see these keys stream through (from the diagonal tile to the end of the
-// last key's document). Per query tile i (keys are TMEM lanes, queries are
-// columns):
+// last key's document, for every query head reading this key/value head).
+// Per query tile i (keys are TMEM lanes, queries are columns):
 //   S^T  = K Q^T           (TMEM)      dP^T = V dO^T        (TMEM)
-//   P^T  = exp2(S^T * scale*log2e - lse2_i), masked; written back to TMEM (bf16)
-//   dV  += P^T dO          (A = P^T from TMEM)
-//   dS^T = P^T (dP^T - Delta_i), written to shared memory (bf16, 128-B swizzle)
-//   dK  += dS^T Q          (A = dS^T read K-major from shared memory)
-//   dQ_i = dS K            (A = the same tile read MN-major), into the dP^T
-//                          columns; read out, staged in shared memory and
-//                          added to the fp32 dq accumulator in global memory by
-//                          bulk reduce-add operations of the TMA unit.
-// The elementwise work runs in kNWG warpgroups (4 at D = 128, 2 at D = 64):
-// warpgroup g takes query columns [g*kQC, (g+1)*kQC) of S^T and dP^T (its P^T
-// goes to the first half of its own S^T columns, so warpgroups never touch
-// each other's TMEM) and feature columns [g*kDC, (g+1)*kDC) of dQ_i, dK and
-// dV; thread t of a warpgroup owns TMEM lane t (a key row, or a query row for
-// dQ_i). The next warp streams Q (two stages, with lse2 and Delta riding on
-// the same barrier) and dO with TMA after loading K and V once; the last warp
-// owns TMEM and issues the MMAs. dK is
-// scaled and rotated back (R^T) in the epilogue; dq is finished by a separate
-// kernel once every key tile has added its part.
+//   P^T  = exp2(S^T * scale*log2e - lse2_i), masked; written to the shared
+//          P/dS tile (bf16, 128-byte swizzle)
+//   dV  += P^T dO          (A = P^T, K-major, from shared memory)
+//   dS^T = P^T (dP^T - Delta_i), written over P^T in the same tile once dV
+//          has read it
+//   dQ_i = dS K            (A = the tile read MN-major), into the S^T
+//                          columns once S^T of the next tile has been read
+//   dK  += dS^T Q          (A = the tile read K-major)
+// Because P^T lives in shared memory rather than in the S^T columns, S^T of
+// the next query tile is issued as soon as the elementwise warps have read
+// S^T of this one into registers, so the tensor pipe computes it while they
+// form P; the MMA warp issues each product as soon as its inputs are ready
+// rather than in a fixed order. dQ_i is drained by its own warpgroup: read out of TMEM in 32-column
+// chunks, staged through a two-buffer shared ring and added to the fp32 dq
+// accumulator in global memory by TMA bulk reduce-adds, off the elementwise
+// warps' path.
+//
+// Warp roles: four elementwise warpgroups; warpgroup g takes query columns [g*kQC, (g+1)*kQC) of S^T and dP^T and
+// feature columns [g*kDC, (g+1)*kDC) of dK and dV; thread t of a warpgroup
+// owns TMEM lane t (a key row). Then the dQ warpgroup (lane = query row),
+// one TMA warp (K and V once, then Q with lse2 and Delta on the same barrier,
+// and dO) and one MMA warp, which owns TMEM. dK is scaled and rotated back
+// (R^T) in the epilogue; dq is finished by a separate kernel once every key
+// tile has added its part.
 //
 // Sources (page, section): ARK README, "Backward pass (AutoGrad)" (attention
 // gradients inside training); Forge README, finding 3 (key-tile-parallel dK/dV
@@ -49,17 +55,18 @@ struct Layout {
   static constexpr int kV = kK + kTileBytes;
   static constexpr int kQ = kV + kTileBytes;                  // 2 stages
   static constexpr int kDO = kQ + 2 * kTileBytes;             // kDOStages stages
-  static constexpr int kDS = kDO + kDOStages * kTileBytes;    // 128 keys x 128 queries bf16
-  static constexpr int kLD = kDS + 128 * 128 * 2;             // 2 x {-lse2[128], -delta[128]} f32
-  // dQ_i staging: 32 x 32 fp32 boxes (4 KB), D/32 x 4 of them per tile: the
-  // first 8 in the (then free) dS tile, the rest (D = 128) in this area.
+  static constexpr int kPS = kDO + kDOStages * kTileBytes;    // P^T then dS^T: 128 keys x 128 queries bf16
+  static constexpr int kLD = kPS + 128 * 128 * 2;             // 2 x {-lse2[128], -delta[128]} f32
+  // dQ_i staging ring: two buffers of 128 query rows x 32 fp32 columns, each
+  // four 32 x 32 boxes (4 KB, 128-byte swizzle), one per dQ warp.
   static constexpr int kXS = kLD + 2 * 1024;
-  static constexpr int kBars = kXS + (D == 128 ? 8 * 4096 : 0);
+  static constexpr int kXSBuf = 128 * 32 * 4;
+  static constexpr int kBars = kXS + 2 * kXSBuf;
   static constexpr int bKV = 0;
   static constexpr int bQFull = 1, bQEmpty = 3, bDOFull = 5, bDOEmpty = 7;  // 2 each
-  static constexpr int bSFull = 9, bPFull = 10, bDPFull = 11, bDSFull = 12, bDVDone = 13,
-                       bDQFull = 14, bDQFree = 15, bFinal = 16, bStageFree = 17;
-  static constexpr int kNumBars = 18;
+  static constexpr int bSFull = 9, bSFree = 10, bPFull = 11, bDPFull = 12, bDSFull = 13,
+                       bDVDone = 14, bDQFull = 15, bDSFree = 16, bDQFree = 17, bFinal = 18;
+  static constexpr int kNumBars = 19;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
   // The dynamic shared-memory window starts 1024-byte aligned on sm_100 (after
@@ -67,17 +74,17 @@ struct Layout {
   // reports an error instead of running misaligned.
   static constexpr int kSmemAlloc = kBytes;
   static constexpr uint32_t kTmemCols = 512;
-  // TMEM columns: S^T (P^T over the first half of each warpgroup's 64), dP^T
-  // (dQ_i after dS), dV, dK
+  // TMEM columns: S^T (dQ_{i-1} once S^T(i) has been read), dP^T, dV, dK
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
-  // Elementwise warpgroups: 4 at D = 128 (16 warps), 2 at D = 64; each owns
-  // kQC query columns of S^T / dP^T and kDC feature columns of dQ_i, dK, dV.
-  static constexpr int kNWG = (D == 128) ? 4 : 2;
+  // Four elementwise warpgroups (16 warps); each owns kQC = 32 query columns
+  // of S^T / dP^T and kDC = D/4 feature columns of dK, dV.
+  static constexpr int kNWG = 4;
   static constexpr int kQC = 128 / kNWG;
   static constexpr int kDC = D / kNWG;
   static constexpr int kEwThreads = 128 * kNWG;
-  static constexpr int kProducerWarp = 4 * kNWG, kMmaWarp = 4 * kNWG + 1;
-  static constexpr int kThreads = kEwThreads + 64;
+  static constexpr int kDqWarp0 = 4 * kNWG;  // the dQ warpgroup: warps kDqWarp0 .. +3
+  static constexpr int kProducerWarp = 4 * kNWG + 4, kMmaWarp = 4 * kNWG + 5;
+  static constexpr int kThreads = kEwThreads + 128 + 64;
 };
 
 struct Params {
@@ -146,14 +153,15 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       mbar_init(bar(L::bDOEmpty + s), 1);
     }
     mbar_init(bar(L::bSFull), 1);
+    mbar_init(bar(L::bSFree), L::kEwThreads);
     mbar_init(bar(L::bPFull), L::kEwThreads);
     mbar_init(bar(L::bDPFull), 1);
     mbar_init(bar(L::bDSFull), L::kEwThreads);
     mbar_init(bar(L::bDVDone), 1);
     mbar_init(bar(L::bDQFull), 1);
-    mbar_init(bar(L::bDQFree), L::kEwThreads);
+    mbar_init(bar(L::bDSFree), 1);
+    mbar_init(bar(L::bDQFree), 128);
     mbar_init(bar(L::bFinal), 1);
-    mbar_init(bar(L::bStageFree), L::kEwThreads);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -178,37 +186,72 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         tma_load_3d(sb0 + L::kK + cb * L::kBlockBytes, &tmK, bar(L::bKV), cb * 64, j0, bhk);
         tma_load_3d(sb0 + L::kV + cb * L::kBlockBytes, &tmV, bar(L::bKV), cb * 64, j0, bhk);
       }
-      for (int it = 0; it < n_it; ++it) {
-        const int st = it & 1;
-        const int so = it % L::kDOStages;
-        const int gi = it / n_q;
-        const int bh = bhq0 + gi;
-        const int qrow = (qt0 + it - gi * n_q) * 128;
-        const float* lse2_bh = p.lse2 + (size_t)bh * p.Tpad;
-        const float* delta_bh = p.delta + (size_t)bh * p.Tpad;
-        if (it >= 2 && !mbar_wait(bar(L::bQEmpty + st), ((it >> 1) - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(L::bQFull + st), L::kTileBytes + 1024);
-        for (int cb = 0; cb < D / 64; ++cb)
-          tma_load_3d(sb0 + L::kQ + st * L::kTileBytes + cb * L::kBlockBytes, &tmQ,
-                      bar(L::bQFull + st), cb * 64, qrow, bh);
-        bulk_load(sb0 + L::kLD + st * 1024, lse2_bh + qrow, 512, bar(L::bQFull + st));
-        bulk_load(sb0 + L::kLD + st * 1024 + 512, delta_bh + qrow, 512, bar(L::bQFull + st));
-        if (it >= L::kDOStages &&
-            !mbar_wait(bar(L::bDOEmpty + so), ((it / L::kDOStages) - 1) & 1, abort_flag))
+      // Q (with its lse2 / Delta rows) and dO stream independently: each is
+      // loaded as soon as its buffer is free, in tile order.
+      int nq = 0, no = 0;
+      long long t_last = clock64();
+      while (nq < n_it || no < n_it) {
+        bool did = false;
+        if (nq < n_it && (nq < 2 || mbar_test(bar(L::bQEmpty + (nq & 1)), ((nq >> 1) - 1) & 1))) {
+          const int st = nq & 1;
+          const int gi = nq / n_q;
+          const int bh = bhq0 + gi;
+          const int qrow = (qt0 + nq - gi * n_q) * 128;
+          mbar_arrive_expect_tx(bar(L::bQFull + st), L::kTileBytes + 1024);
+          for (int cb = 0; cb < D / 64; ++cb)
+            tma_load_3d(sb0 + L::kQ + st * L::kTileBytes + cb * L::kBlockBytes, &tmQ,
+                        bar(L::bQFull + st), cb * 64, qrow, bh);
+          bulk_load(sb0 + L::kLD + st * 1024, p.lse2 + (size_t)bh * p.Tpad + qrow, 512,
+                    bar(L::bQFull + st));
+          bulk_load(sb0 + L::kLD + st * 1024 + 512, p.delta + (size_t)bh * p.Tpad + qrow, 512,
+                    bar(L::bQFull + st));
+          ++nq;
+          did = true;
+        }
+        if (no < n_it && (no < L::kDOStages ||
+                          mbar_test(bar(L::bDOEmpty + no % L::kDOStages),
+                                    ((no / L::kDOStages) - 1) & 1))) {
+          const int so = no % L::kDOStages;
+          const int gi = no / n_q;
+          const int qrow = (qt0 + no - gi * n_q) * 128;
+          mbar_arrive_expect_tx(bar(L::bDOFull + so), L::kTileBytes);
+          for (int cb = 0; cb < D / 64; ++cb)
+            tma_load_3d(sb0 + L::kDO + so * L::kTileBytes + cb * L::kBlockBytes, &tmDO,
+                        bar(L::bDOFull + so), cb * 64, qrow, bhq0 + gi);
+          ++no;
+          did = true;
+        }
+        if (did) {
+          t_last = clock64();
+          continue;
+        }
+        if (*abort_flag) break;
+        if (clock64() - t_last > kWaitLimitCycles) {
+          *abort_flag = 1;
+          report_status(ATTN_ETIMEOUT);
           break;
-        mbar_arrive_expect_tx(bar(L::bDOFull + so), L::kTileBytes);
-        for (int cb = 0; cb < D / 64; ++cb)
-          tma_load_3d(sb0 + L::kDO + so * L::kTileBytes + cb * L::kBlockBytes, &tmDO,
-                      bar(L::bDOFull + so), cb * 64, qrow, bh);
+        }
+        __nanosleep(32);
       }
     }
   } else if (warp == L::kMmaWarp) {
     // ---------------- MMA issuer ----------------
-    // Issue order per query tile i: dV(i), S(i+1), dK(i), dQ(i), dP(i+1), so
-    // the tensor pipe has S(i+1) to run while the elementwise warps form dS(i),
-    // and dK/dQ(i) while they form P(i+1). TMEM reuse: S(i+1) waits for dV(i)
-    // (which reads P^T(i) from the S columns); dP(i+1) waits until dQ(i) has
-    // been read out of the dP columns.
+    // Five groups per query tile i: S(i), dP(i), dV(i), dK(i), dQ(i). Each
+    // group is issued in tile order, but across groups the issuer takes
+    // whichever is ready (probing its barriers without blocking), in the
+    // priority dV, S, dK, dQ, dP. TMEM: S^T(i) and then dQ(i-1) share the S^T
+    // columns, dP^T has its own. Readiness:
+    //   S(i):  Q(i) loaded; the S^T columns free: S(0) always, S(1) once the
+    //          elementwise warps have read S(0), S(i >= 2) once dQ(i-2) has
+    //          been read out
+    //   dP(i): dO(i) loaded; dS^T(i-1) formed (so dP^T(i-1) has been read)
+    //   dV(i): P^T(i) in the P/dS tile; dP(i) issued (dO(i) is loaded and the
+    //          commit after dV(i) covers both readers of dO(i))
+    //   dK(i): dS^T(i) in the tile
+    //   dQ(i): dK(i) issued; the elementwise warps have read S(i+1) (or i is
+    //          the last tile). The tile is free again after dQ(i).
+    // Every barrier probed for phase k has been seen complete for phase k-1,
+    // so the parity probes are unambiguous.
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f16(128, 128, true, true, false, false);
       constexpr uint32_t id_dv = idesc_f16(128, D, true, true, false, true);
@@ -216,89 +259,165 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       constexpr uint32_t id_dq = idesc_f16(128, D, true, true, true, true);
       const uint32_t tS = tmem + L::kColS, tDP = tmem + L::kColDP;
       const uint32_t tDV = tmem + L::kColDV, tDK = tmem + L::kColDK;
+      const uint32_t ps = sb0 + L::kPS;
       auto qbuf = [&](int i) -> uint32_t { return sb0 + L::kQ + (i & 1) * L::kTileBytes; };
       auto obuf = [&](int i) -> uint32_t {
         return sb0 + L::kDO + (i % L::kDOStages) * L::kTileBytes;
       };
-      // S^T(i) = K Q(i)^T
-      auto issue_S = [&](int i) -> bool {
-        if (!mbar_wait(bar(L::bQFull + (i & 1)), (i >> 1) & 1, abort_flag)) return false;
-        if (i > 0 && !mbar_wait(bar(L::bDVDone), (i - 1) & 1, abort_flag)) return false;
-        tc_fence_after();
+      int nS = 0, nP = 0, nV = 0, nK = 0, nQ = 0;  // next tile of each group
+      bool ok = mbar_wait(bar(L::bKV), 0, abort_flag);
+      long long t_last = clock64();
+      while (ok && nQ < n_it) {
+        if (nV < nP && mbar_test(bar(L::bPFull), nV & 1)) {
+          // dV += P^T dO (P^T K-major in the P/dS tile, dO MN-major)
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
-          mma_ss(tS, smem_desc_sw128(sb0 + L::kK + off, 16, 1024),
-                 smem_desc_sw128(qbuf(i) + off, 16, 1024), id_s, kk > 0);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tDV, smem_desc_sw128(ps + (kk >> 2) * L::kBlockBytes + (kk & 3) * 32, 16, 1024),
+                   smem_desc_sw128(obuf(nV) + kk * 2048, L::kBlockBytes, 1024), id_dv,
+                   (nV > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(L::bDVDone));
+          mma_commit(bar(L::bDOEmpty + nV % L::kDOStages));
+          ++nV;
+        } else if (nS < n_it && mbar_test(bar(L::bQFull + (nS & 1)), (nS >> 1) & 1) &&
+                   (nS == 0 || (nS == 1 ? mbar_test(bar(L::bSFree), 0)
+                                        : (nQ > nS - 2 && mbar_test(bar(L::bDQFree), nS & 1))))) {
+          // S^T(i) = K Q(i)^T
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
+            mma_ss(tS, smem_desc_sw128(sb0 + L::kK + off, 16, 1024),
+                   smem_desc_sw128(qbuf(nS) + off, 16, 1024), id_s, kk > 0);
+          }
+          mma_commit(bar(L::bSFull));
+          ++nS;
+        } else if (nK < nV && mbar_test(bar(L::bDSFull), nK & 1)) {
+          // dK += dS^T Q (dS^T K-major)
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tDK, smem_desc_sw128(ps + (kk >> 2) * L::kBlockBytes + (kk & 3) * 32, 16, 1024),
+                   smem_desc_sw128(qbuf(nK) + kk * 2048, L::kBlockBytes, 1024), id_dk,
+                   (nK > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(L::bQEmpty + (nK & 1)));
+          if (nK == n_it - 1) mma_commit(bar(L::bFinal));
+          ++nK;
+        } else if (nQ < nK && (nQ == n_it - 1 ||
+                               (nS > nQ + 1 && mbar_test(bar(L::bSFree), (nQ + 1) & 1)))) {
+          // dQ_i = dS K (dS read MN-major), into the S^T columns
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tS, smem_desc_sw128(ps + kk * 2048, L::kBlockBytes, 1024),
+                   smem_desc_sw128(sb0 + L::kK + kk * 2048, L::kBlockBytes, 1024), id_dq, kk > 0);
+          mma_commit(bar(L::bDQFull));
+          mma_commit(bar(L::bDSFree));
+          ++nQ;
+        } else if (nP < n_it && nP <= nK &&
+                   mbar_test(bar(L::bDOFull + nP % L::kDOStages), (nP / L::kDOStages) & 1)) {
+          // dP^T(i) = V dO(i)^T
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
+            mma_ss(tDP, smem_desc_sw128(sb0 + L::kV + off, 16, 1024),
+                   smem_desc_sw128(obuf(nP) + off, 16, 1024), id_s, kk > 0);
+          }
+          mma_commit(bar(L::bDPFull));
+          ++nP;
+        } else {
+          // nothing ready: keep probing; give up like mbar_wait does
+          if (*abort_flag) break;
+          if (clock64() - t_last > kWaitLimitCycles) {
+            *abort_flag = 1;
+            report_status(ATTN_ETIMEOUT);
+            break;
+          }
+          continue;
         }
-        mma_commit(bar(L::bSFull));
-        return true;
-      };
-      // dP^T(i) = V dO(i)^T
-      auto issue_dP = [&](int i) -> bool {
-        if (!mbar_wait(bar(L::bDOFull + i % L::kDOStages), (i / L::kDOStages) & 1, abort_flag))
-          return false;
-        if (i > 0 && !mbar_wait(bar(L::bDQFree), (i - 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
-          mma_ss(tDP, smem_desc_sw128(sb0 + L::kV + off, 16, 1024),
-                 smem_desc_sw128(obuf(i) + off, 16, 1024), id_s, kk > 0);
-        }
-        mma_commit(bar(L::bDPFull));
-        return true;
-      };
-      bool ok = mbar_wait(bar(L::bKV), 0, abort_flag) && issue_S(0) && issue_dP(0);
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int ph = it & 1;
-        // dV += P^T dO; P^T of warpgroup g's query columns [g*kQC, (g+1)*kQC)
-        // sits in TMEM columns [g*kQC, g*kQC + kQC/2), so the 16 queries of
-        // k-step kk start at column 8*kk + (kQC/2) * (16*kk / kQC)
-        if (!mbar_wait(bar(L::bPFull), ph, abort_flag)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tDV, tS + 8 * kk + (L::kQC / 2) * ((16 * kk) / L::kQC),
-                 smem_desc_sw128(obuf(it) + kk * 2048, L::kBlockBytes, 1024), id_dv,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar(L::bDVDone));
-        mma_commit(bar(L::bDOEmpty + it % L::kDOStages));
-        if (it + 1 < n_it && !issue_S(it + 1)) break;
-        // dK += dS^T Q ; dQ_i = dS K
-        if (!mbar_wait(bar(L::bDSFull), ph, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t ds = sb0 + L::kDS;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tDK, smem_desc_sw128(ds + (kk >> 2) * L::kBlockBytes + (kk & 3) * 32, 16, 1024),
-                 smem_desc_sw128(qbuf(it) + kk * 2048, L::kBlockBytes, 1024), id_dk,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tDP, smem_desc_sw128(ds + kk * 2048, L::kBlockBytes, 1024),
-                 smem_desc_sw128(sb0 + L::kK + kk * 2048, L::kBlockBytes, 1024), id_dq, kk > 0);
-        mma_commit(bar(L::bDQFull));
-        mma_commit(bar(L::bQEmpty + (it & 1)));
-        if (it == n_it - 1) mma_commit(bar(L::bFinal));
-        if (it + 1 < n_it && !issue_dP(it + 1)) break;
+        t_last = clock64();
       }
     }
+  } else if (warp >= L::kDqWarp0) {
+    // ---------------- dQ warpgroup (lane = query row) ----------------
+    // Per query tile: read dQ_i out of the S^T columns in 32-column chunks
+    // (releasing the columns after the last read), stage each chunk as this
+    // warp's 32 x 32 box in the next ring buffer and reduce-add it into the
+    // accumulator. A buffer is rewritten only after the reduce that last used
+    // it (two chunks back) has read it.
+    const int sub = warp & 3;
+    const uint32_t tq = tmem + ((uint32_t)(sub * 32) << 16) + L::kColS;
+    constexpr int NCH = D / 32;
+    int chunk = 0;
+    bool prev_issued = false;  // did this warp reduce the previous chunk
+    for (int it = 0; it < n_it; ++it) {
+      const int gi = it / n_q;
+      const int i0 = (qt0 + it - gi * n_q) * 128;
+      const bool rows_in = i0 + 32 * sub < T;  // rows past T are clipped by the map
+      if (!mbar_wait(bar(L::bDQFull), it & 1, abort_flag)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < NCH; ++c, ++chunk) {
+        uint32_t v[32];
+        tmem_ld32(tq + 32 * c, v);
+        tmem_wait_ld();
+        if (c == NCH - 1) {
+          tc_fence_before();
+          mbar_arrive(bar(L::bDQFree));
+        }
+        const int buf = chunk & 1;
+        if (lane == 0) {
+          if (prev_issued) bulk_wait_group_read1();
+          else bulk_wait_group_read0();
+        }
+        __syncwarp();
+        uint8_t* bx = sg + L::kXS + buf * L::kXSBuf + sub * 4096;
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          *reinterpret_cast<uint4*>(bx + sw128(lane, e)) =
+              make_uint4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && rows_in) {
+          tma_reduce_add_3d(&tmDQ, sb0 + L::kXS + buf * L::kXSBuf + sub * 4096, 32 * c,
+                            i0 + 32 * sub, bhq0 + gi);
+          bulk_commit_group();
+        }
+        prev_issued = rows_in;
+      }
+    }
+    if (lane == 0) bulk_wait_group0();
   } else {
     // ---------------- elementwise warps ----------------
     constexpr int QC = L::kQC, DC = L::kDC;
     const int wg = warp >> 2, sub = warp & 3;
-    const int r = sub * 32 + lane;  // TMEM lane: key row (S^T, dP^T, dK, dV) or query row (dQ_i)
+    const int r = sub * 32 + lane;  // TMEM lane: key row of S^T, dP^T, dK, dV
     const int j = j0 + r;
     const int qc0 = QC * wg;        // query columns of S^T / dP^T handled here
-    const int dc0 = DC * wg;        // feature columns of dQ_i / dK / dV handled here
+    const int dc0 = DC * wg;        // feature columns of dK / dV handled here
     const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
     const int de_j = (j < T) ? (p.doc_end ? p.doc_end[row0 + j] - row0 : T) : T;
     const uint32_t tS = tmem + lane_base + L::kColS;
     const uint32_t tDP = tmem + lane_base + L::kColDP;
-    uint8_t* dsb = sg + L::kDS;
+    uint8_t* psb = sg + L::kPS;
     float pf[QC];  // P^T of this thread's key row, query columns [qc0, qc0 + QC)
-    // ---- P^T(i) = exp2(S^T scale log2e - lse2), masked; bf16 copy to TMEM ----
+    // Row r, query columns [qc0, qc0 + QC) of the P/dS tile (bf16 pairs in
+    // w[]): 64-column block col/64, 16-byte chunks (col%64)/8 onwards.
+    auto store_row = [&](const uint32_t* w) {
+#pragma unroll
+      for (int c = 0; c < QC / 32; ++c) {
+        const int col = qc0 + 32 * c;
+        uint8_t* blk = psb + (col >> 6) * L::kBlockBytes;
+        const int ch0 = (col & 63) >> 3;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          *reinterpret_cast<uint4*>(blk + sw128(r, ch0 + e)) =
+              make_uint4(w[16 * c + 4 * e], w[16 * c + 4 * e + 1], w[16 * c + 4 * e + 2],
+                         w[16 * c + 4 * e + 3]);
+      }
+    };
+    // ---- P^T(i) = exp2(S^T scale log2e - lse2), masked; bf16 into the tile ----
     auto phase_P = [&](int i) -> bool {
       const int i0 = (qt0 + i % n_q) * 128;
       const bool need_mask = (i0 + qc0 < j) || (i0 + qc0 + QC - 1 >= de_j);
@@ -311,122 +430,62 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
 #pragma unroll
       for (int c = 0; c < QC / 32; ++c) tmem_ld32(tS + qc0 + 32 * c, s + 32 * c);
       tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(L::bSFree));  // the S^T columns may take the next tile
       const float2 scl2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
-      for (int c = 0; c < QC / 32; ++c) {
-        const int col = qc0 + 32 * c;
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float2 nl = reinterpret_cast<const float2*>(sl + col)[e];  // -lse2 pair
-          const int i_a = i0 + col + 2 * e;
-          const float2 sv = make_float2(__uint_as_float(s[32 * c + 2 * e]),
-                                        __uint_as_float(s[32 * c + 2 * e + 1]));
-          const float2 x = __ffma2_rn(sv, scl2, nl);
-          // about a third of the pairs go to the FMA pipe
-          float2 pv = (e % 3 == 2) ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
-          if (need_mask) {
-            if (i_a < j || i_a >= de_j) pv.x = 0.f;
-            if (i_a + 1 < j || i_a + 1 >= de_j) pv.y = 0.f;
-          }
-          pf[32 * c + 2 * e] = pv.x;
-          pf[32 * c + 2 * e + 1] = pv.y;
-          pk[e] = pack_bf16(pv.x, pv.y);
+      for (int e = 0; e < QC / 2; ++e) {
+        const int col = qc0 + 2 * e;
+        const float2 nl = reinterpret_cast<const float2*>(sl + col)[0];  // -lse2 pair
+        const int i_a = i0 + col;
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]),
+                                                __uint_as_float(s[2 * e + 1])),
+                                    scl2, nl);
+        // about a third of the pairs go to the FMA pipe
+        float2 pv = (e % 3 == 2) ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
+        if (need_mask) {
+          if (i_a < j || i_a >= de_j) pv.x = 0.f;
+          if (i_a + 1 < j || i_a + 1 >= de_j) pv.y = 0.f;
         }
-        tmem_st16(tS + qc0 + 16 * c, pk);
+        pf[2 * e] = pv.x;
+        pf[2 * e + 1] = pv.y;
       }
-      tmem_wait_st();
-      tc_fence_before();
+      // dQ(i-1) and dK(i-1) must be done reading dS^T(i-1) from the tile
+      if (i > 0 && !mbar_wait(bar(L::bDSFree), (i - 1) & 1, abort_flag)) return false;
+      uint32_t w[QC / 2];
+#pragma unroll
+      for (int e = 0; e < QC / 2; ++e) w[e] = pack_bf16(pf[2 * e], pf[2 * e + 1]);
+      store_row(w);
+      fence_proxy_async_smem();
       mbar_arrive(bar(L::bPFull));
       return true;
     };
-    // ---- dS^T(i) = P^T (dP^T - Delta) into the shared dS tile ----
+    // ---- dS^T(i) = P^T (dP^T - Delta), over P^T in the tile once dV(i) ran ----
     auto phase_dS = [&](int i) -> bool {
       const float* sd = reinterpret_cast<const float*>(sg + L::kLD + (i & 1) * 1024) + 128;
-      // The dS tile doubled as dQ staging for tile i-1: every thread's bulk
-      // reads of it must be done (a bounded barrier over the elementwise warps).
-      bulk_wait_group_read0();
-      mbar_arrive(bar(L::bStageFree));
-      if (!mbar_wait(bar(L::bStageFree), i & 1, abort_flag) ||
-          !mbar_wait(bar(L::bDPFull), i & 1, abort_flag))
-        return false;
+      if (!mbar_wait(bar(L::bDPFull), i & 1, abort_flag)) return false;
       tc_fence_after();
       uint32_t dpv[QC];
 #pragma unroll
       for (int c = 0; c < QC / 32; ++c) tmem_ld32(tDP + qc0 + 32 * c, dpv + 32 * c);
       tmem_wait_ld();
+      uint32_t w[QC / 2];
 #pragma unroll
-      for (int c = 0; c < QC / 32; ++c) {
-        const int col = qc0 + 32 * c;
-        uint32_t dsk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float2 nd = reinterpret_cast<const float2*>(sd + col)[e];  // -Delta pair
-          const float2 dpp = make_float2(__uint_as_float(dpv[32 * c + 2 * e]),
-                                         __uint_as_float(dpv[32 * c + 2 * e + 1]));
-          const float2 a = __fmul2_rn(make_float2(pf[32 * c + 2 * e], pf[32 * c + 2 * e + 1]),
-                                      __fadd2_rn(dpp, nd));
-          dsk[e] = pack_bf16(a.x, a.y);
-        }
-        // row r of the dS^T tile, query columns [col, col+32): block col/64,
-        // 16-byte chunks (col%64)/8 .. +3
-        uint8_t* blk = dsb + (col >> 6) * L::kBlockBytes;
-        const int ch0 = (col & 63) >> 3;
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          *reinterpret_cast<uint4*>(blk + sw128(r, ch0 + e)) =
-              make_uint4(dsk[4 * e], dsk[4 * e + 1], dsk[4 * e + 2], dsk[4 * e + 3]);
+      for (int e = 0; e < QC / 2; ++e) {
+        const float2 nd = reinterpret_cast<const float2*>(sd + qc0)[e];  // -Delta pair
+        const float2 dpp = make_float2(__uint_as_float(dpv[2 * e]), __uint_as_float(dpv[2 * e + 1]));
+        const float2 a = __fmul2_rn(make_float2(pf[2 * e], pf[2 * e + 1]), __fadd2_rn(dpp, nd));
+        w[e] = pack_bf16(a.x, a.y);
       }
+      if (!mbar_wait(bar(L::bDVDone), i & 1, abort_flag)) return false;
+      store_row(w);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(L::bDSFull));
       return true;
     };
-    // ---- dQ_i (lane = query row): release TMEM first, then reduce into global ----
-    auto phase_dQ = [&](int i) -> bool {
-      const int gi = i / n_q;
-      const int i0 = (qt0 + i - gi * n_q) * 128;
-      if (!mbar_wait(bar(L::bDQFull), i & 1, abort_flag)) return false;
-      tc_fence_after();
-      constexpr int NQC = DC / 32;  // 32-column chunks per warpgroup
-      uint32_t dqv[NQC][32];
-#pragma unroll
-      for (int c = 0; c < NQC; ++c) tmem_ld32(tDP + dc0 + 32 * c, dqv[c]);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(L::bDQFree));
-      // Every thread has consumed the dS tile (dq_full implies the dK and dQ
-      // MMAs are done), so it now serves as staging: one 32x32 fp32 box per
-      // warp and chunk in the 128-byte-swizzled layout (conflict-free stores),
-      // each added to the accumulator by one tensor reduce-add.
-#pragma unroll
-      for (int c = 0; c < NQC; ++c) {
-        const int box = warp * NQC + c;
-        uint8_t* bx = (box < 8) ? sg + L::kDS + box * 4096 : sg + L::kXS + (box - 8) * 4096;
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          *reinterpret_cast<uint4*>(bx + sw128(lane, e)) =
-              make_uint4(dqv[c][4 * e], dqv[c][4 * e + 1], dqv[c][4 * e + 2], dqv[c][4 * e + 3]);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0 && i0 + 32 * sub < T) {  // rows past T are clipped by the map
-#pragma unroll
-        for (int c = 0; c < NQC; ++c) {
-          const int box = warp * NQC + c;
-          const uint32_t bx = (box < 8) ? sb0 + L::kDS + box * 4096 : sb0 + L::kXS + (box - 8) * 4096;
-          tma_reduce_add_3d(&tmDQ, bx, dc0 + 32 * c, i0 + 32 * sub, bhq0 + gi);
-        }
-        bulk_commit_group();
-      }
-      return true;
-    };
-    // Order: P(0); then per tile i: dS(i), P(i+1), dQ(i).
-    bool ok = phase_P(0);
-    for (int it = 0; ok && it < n_it; ++it) {
-      ok = phase_dS(it) && (it + 1 >= n_it || phase_P(it + 1)) && phase_dQ(it);
-    }
-    bulk_wait_group0();
+    bool ok = true;
+    for (int it = 0; ok && it < n_it; ++it) ok = phase_P(it) && phase_dS(it);
     // ---- epilogue: dK = R^T (scale * dK_r), dV ----
     if (ok && mbar_wait(bar(L::bFinal), 0, abort_flag)) {
       tc_fence_after();
@@ -434,33 +493,38 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       const int pos = jj - (p.doc_start ? p.doc_start[row0 + jj] - row0 : 0);
       __nv_bfloat16* dkrow = p.dk + ((size_t)bhk * T + jj) * D;
       __nv_bfloat16* dvrow = p.dv + ((size_t)bhk * T + jj) * D;
+      constexpr int CW = DC < 32 ? DC : 32;  // columns per TMEM load
+      auto ld = [&](uint32_t taddr, uint32_t* v) {
+        if constexpr (CW == 32) tmem_ld32(taddr, v);
+        else tmem_ld16(taddr, v);
+      };
 #pragma unroll
-      for (int c = 0; c < DC / 32; ++c) {
-        const int col = dc0 + 32 * c;
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + L::kColDK + col, v);
+      for (int c = 0; c < DC / CW; ++c) {
+        const int col = dc0 + CW * c;
+        uint32_t v[CW];
+        ld(tmem + lane_base + L::kColDK + col, v);
         tmem_wait_ld();
-        float f[32];
+        float f[CW];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]) * p.scale;
-        if (p.rope_cos) rope_pairs<32, D>(f, p.rope_cos, p.rope_sin, pos, col, true);
+        for (int e = 0; e < CW; ++e) f[e] = __uint_as_float(v[e]) * p.scale;
+        if (p.rope_cos) rope_pairs<CW, D>(f, p.rope_cos, p.rope_sin, pos, col, true);
         if (j < T) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
+          for (int e = 0; e < CW / 8; ++e)
             reinterpret_cast<uint4*>(dkrow + col)[e] =
                 make_uint4(pack_bf16(f[8 * e], f[8 * e + 1]), pack_bf16(f[8 * e + 2], f[8 * e + 3]),
                            pack_bf16(f[8 * e + 4], f[8 * e + 5]), pack_bf16(f[8 * e + 6], f[8 * e + 7]));
         }
       }
 #pragma unroll
-      for (int c = 0; c < DC / 32; ++c) {
-        const int col = dc0 + 32 * c;
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + L::kColDV + col, v);
+      for (int c = 0; c < DC / CW; ++c) {
+        const int col = dc0 + CW * c;
+        uint32_t v[CW];
+        ld(tmem + lane_base + L::kColDV + col, v);
         tmem_wait_ld();
         if (j < T) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
+          for (int e = 0; e < CW / 8; ++e)
             reinterpret_cast<uint4*>(dvrow + col)[e] = make_uint4(
                 pack_bf16(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
                 pack_bf16(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
