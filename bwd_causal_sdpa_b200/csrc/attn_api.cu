@@ -206,7 +206,7 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
     qf = (float*)(ws + wp.qfac);
     kf = (float*)(ws + wp.kfac);
     ATTN_LAUNCH(KK_ROPE_PREP, st,
-                rope_prep_kernel<__half, D, true><<<dim3(nt, BH, 2), 256, 0, st>>>(
+                rope_prep_kernel<__half, D, true><<<dim3(nt, BH, 2), kRopePrepThreads, 0, st>>>(
                     (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qh, kh, qf, kf,
                     H, Hkv, T, nt));
     if (launch_status()) return ATTN_ECUDA;
@@ -257,7 +257,7 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   float* dq_acc = (float*)(ws + wp.dq_acc);
   const long rows_pad = (long)BH * Tpad;
   ATTN_LAUNCH(KK_DELTA, st,
-              bwd_prep_kernel<D><<<(unsigned)((rows_pad + 7) / 8), 256, 0, st>>>(
+              bwd_prep_kernel<D><<<(unsigned)(rows_pad * (D / 8) / 256), 256, 0, st>>>(
                   (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse, delta, lse2, dq_acc,
                   (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qr, kr, H, Hkv,
                   T, Tpad, rows_pad));

@@ -88,14 +88,17 @@ __global__ void __launch_bounds__(256) delta_kernel(const TIO* __restrict__ o, c
 // it into [2^14, 2^15), and fac[] receives the inverse factor (exact), which
 // the forward folds into its score scale. Without kTileScale (bf16 output)
 // values are stored as they are.
+constexpr int kRopePrepThreads = 512;
+
 template <typename OutT, int D, bool kTileScale>
-__global__ void __launch_bounds__(256) rope_prep_kernel(
+__global__ void __launch_bounds__(kRopePrepThreads) rope_prep_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const float* __restrict__ rc, const float* __restrict__ rs,
     const int32_t* __restrict__ doc_start, OutT* __restrict__ qo, OutT* __restrict__ ko,
     float* __restrict__ qfac, float* __restrict__ kfac, int H, int Hkv, int T, int ntiles) {
   constexpr int CH = D / 8;              // 16-byte chunks per row
-  constexpr int PER = 128 * CH / 256;    // chunks per thread
+  constexpr int NT = kRopePrepThreads;
+  constexpr int PER = 128 * CH / NT;     // chunks per thread
   // grid (ntiles, B*H, 2): z = 0 rotates q heads, z = 1 the B*Hkv k heads
   const int tile = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const int heads = which ? Hkv : H;
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(256) rope_prep_kernel(
   float amax = 0.f;
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
-    const int idx = threadIdx.x + u * 256, r = idx / CH, c8 = idx % CH, t = t0 + r;
+    const int idx = threadIdx.x + u * NT, r = idx / CH, c8 = idx % CH, t = t0 + r;
 #pragma unroll
     for (int e = 0; e < 8; ++e) v[u][e] = 0.f;
     if (t < T) {
@@ -123,19 +126,19 @@ __global__ void __launch_bounds__(256) rope_prep_kernel(
   }
   float f = 1.f;
   if constexpr (kTileScale) {
-    __shared__ float red[8];
+    __shared__ float red[NT / 32];
     amax = warp_max(amax);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
     __syncthreads();
     amax = red[0];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
+    for (int w = 1; w < NT / 32; ++w) amax = fmaxf(amax, red[w]);
     if (amax >= 16384.f && amax <= 3.0e38f) f = ldexpf(1.f, 14 - ilogbf(amax));
     if (threadIdx.x == 0) (which ? kfac : qfac)[bh * ntiles + tile] = 1.f / f;
   }
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
-    const int idx = threadIdx.x + u * 256, r = idx / CH, c8 = idx % CH, t = t0 + r;
+    const int idx = threadIdx.x + u * NT, r = idx / CH, c8 = idx % CH, t = t0 + r;
     if (t >= T) continue;
     uint4 out;
     uint32_t* w = reinterpret_cast<uint32_t*>(&out);
@@ -153,13 +156,36 @@ __global__ void __launch_bounds__(256) rope_prep_kernel(
   }
 }
 
-// Backward preprocessing for the tensor-core path, one warp per row of the
-// tile-padded [B*H][ntiles*128] view: stores -Delta_i (Delta_i = sum_d
-// dO[i][d] * o[i][d]) and -lse_i * log2(e), negated so the main kernel folds
-// them in with one fused multiply-add (both 0 for padding rows t >= T, so its
-// per-tile loads never leave the arrays), zeroes the fp32 dq accumulator row
-// and, with RoPE tables, writes the rotated q and k rows (bf16) the main
-// kernel reads.
+// Eight bf16 values (16 bytes) as fp32, and back.
+__device__ __forceinline__ void load8_bf16(const __nv_bfloat16* p, float* v) {
+  const uint4 raw = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    v[2 * e] = __low2float(h[e]);
+    v[2 * e + 1] = __high2float(h[e]);
+  }
+}
+__device__ __forceinline__ void store8_bf16(__nv_bfloat16* p, const float* v) {
+  uint4 raw;
+  uint32_t* w = reinterpret_cast<uint32_t*>(&raw);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+    w[e] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  *reinterpret_cast<uint4*>(p) = raw;
+}
+
+// Backward preprocessing for the tensor-core path over the tile-padded
+// [B*H][ntiles*128] row view, D/8 threads per row (16 bytes of each bf16 row
+// per thread, so a warp covers 32*8/D whole rows): stores -Delta_i (Delta_i =
+// sum_d dO[i][d] * o[i][d]) and -lse_i * log2(e), negated so the main kernel
+// folds them in with one fused multiply-add (both 0 for padding rows t >= T,
+// so its per-tile loads never leave the arrays), zeroes the fp32 dq
+// accumulator row and, with RoPE tables, writes the rotated q and k rows
+// (bf16) the main kernel reads. The grid covers rows_pad * D/8 threads
+// exactly (rows_pad is a multiple of 128), so every warp is full.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(
     const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
@@ -169,42 +195,44 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
     const float* __restrict__ rs, const int32_t* __restrict__ doc_start,
     __nv_bfloat16* __restrict__ qr, __nv_bfloat16* __restrict__ kr, int H, int Hkv, int T,
     int Tpad, long rows_pad) {
-  constexpr int NC = D / 32;
-  const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows_pad) return;
+  constexpr int TPR = D / 8;  // threads per row
+  const long gt = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long row = gt / TPR;
+  const int c8 = (int)(gt - row * TPR) * 8;
   const long bh = row / Tpad;
   const int t = (int)(row - bh * Tpad);
   float s = 0.f;
-  if (t < T) {
+  if (row < rows_pad && t < T) {
     const long r = bh * T + t;
-    float a[NC], g[NC];
-    load_vec<NC>(o + r * D + lane * NC, a);
-    load_vec<NC>(dO + r * D + lane * NC, g);
+    float a[8], g[8];
+    load8_bf16(o + r * D + c8, a);
+    load8_bf16(dO + r * D + c8, g);
 #pragma unroll
-    for (int c = 0; c < NC; ++c) s = fmaf(a[c], g[c], s);
-    s = warp_sum(s);
-    const float z[NC] = {};
-    store_vec<NC>(dq_acc + r * D + lane * NC, z);
+    for (int e = 0; e < 8; ++e) s = fmaf(a[e], g[e], s);
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    reinterpret_cast<float4*>(dq_acc + r * D + c8)[0] = z;
+    reinterpret_cast<float4*>(dq_acc + r * D + c8)[1] = z;
     if (rc) {
       const int b = (int)(bh / H);
       const int pos = t - (doc_start ? doc_start[b * T + t] - b * T : 0);
-      float x[NC];
-      load_vec<NC>(q + r * D + lane * NC, x);
-      rope_pairs<NC, D>(x, rc, rs, pos, lane * NC, false);
-      store_vec<NC>(qr + r * D + lane * NC, x);
+      float x[8];
+      load8_bf16(q + r * D + c8, x);
+      rope_pairs<8, D>(x, rc, rs, pos, c8, false);
+      store8_bf16(qr + r * D + c8, x);
       // row r of the [B*Hkv][T] k view exists for the first B*Hkv heads; its
       // batch (hence document layout) is bh / Hkv
       if (bh < (rows_pad / Tpad) / H * Hkv) {
         const int bk = (int)(bh / Hkv);
         const int posk = t - (doc_start ? doc_start[bk * T + t] - bk * T : 0);
-        load_vec<NC>(k + r * D + lane * NC, x);
-        rope_pairs<NC, D>(x, rc, rs, posk, lane * NC, false);
-        store_vec<NC>(kr + r * D + lane * NC, x);
+        load8_bf16(k + r * D + c8, x);
+        rope_pairs<8, D>(x, rc, rs, posk, c8, false);
+        store8_bf16(kr + r * D + c8, x);
       }
     }
   }
-  if (lane == 0) {
+#pragma unroll
+  for (int off = TPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (c8 == 0 && row < rows_pad) {
     delta_pad[row] = -s;
     lse2_pad[row] = t < T ? -lse[bh * T + t] * 1.4426950408889634f : 0.f;
   }
