@@ -45,6 +45,7 @@ _SIGNATURES = {
     "attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float,
                               _I, _P, _P, _P, _P]),
     "attn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
+    "attn_workspace_bytes_gqa": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I]),
     "attn_get_status": (_I, [_P]),
     "attn_error_string": (ctypes.c_char_p, [_I]),
     "attn_exp2_selftest": (_I, [_P, _P, _I, _P]),
@@ -100,6 +101,10 @@ def error_string(code: int) -> str:
 
 def attn_workspace_bytes(B, H, T, D, dtype, is_bwd) -> int:
     return int(_lib.attn_workspace_bytes(B, H, T, D, dtype, int(is_bwd)))
+
+
+def attn_workspace_bytes_gqa(B, H, H_kv, T, D, dtype, is_bwd) -> int:
+    return int(_lib.attn_workspace_bytes_gqa(B, H, H_kv, T, D, dtype, int(is_bwd)))
 
 
 def attn_fwd(q, k, v, rope_cos, rope_sin, cu_seqlens, o, lse, B, H, T, D, scale, dtype,

@@ -27,8 +27,25 @@ struct WsPlan {
   size_t dq_acc = 0;                  // f32 [B*H*T*D] dq accumulator (bf16 backward)
   size_t q16 = 0, k16 = 0;            // rotated q, k as 16-bit [B*H*T*D] each (bf16 storage)
   size_t qfac = 0, kfac = 0;          // f32 [B*H*ceil(T/128)] tile factors (bf16 forward)
+  size_t dk_acc = 0, dv_acc = 0;      // f32 [B*Hkv*T*D] each when the backward splits groups
+  int split = 1;                      // query-head groups split over this many CTAs
   size_t total = 0;
 };
+
+// Grouped-query backward: one CTA per (key/value head, key tile) walks the G
+// query heads of its group. When that gives too few CTAs to fill the GPU, the
+// group is split over S CTAs (S the smallest divisor of G reaching about two
+// CTAs per SM of a B200), which then add their dK, dV parts into fp32
+// accumulators.
+constexpr long kSplitTargetCtas = 2 * 148;
+int choose_split(int B, int H, int Hkv, int T) {
+  const int G = H / Hkv;
+  const long base = (long)B * Hkv * ((T + 127) / 128);
+  if (G == 1 || base >= kSplitTargetCtas) return 1;
+  for (int S = 2; S < G; ++S)
+    if (G % S == 0 && base * S >= kSplitTargetCtas) return S;
+  return G;
+}
 
 bool sizes_ok(int B, int H, int T, int D) {
   if (B <= 0 || H <= 0 || T <= 0) return false;
@@ -38,8 +55,9 @@ bool sizes_ok(int B, int H, int T, int D) {
   return bt < INT32_MAX && n < INT32_MAX;
 }
 
-WsPlan plan(int B, int H, int T, int D, int dtype, int is_bwd) {
+WsPlan plan(int B, int H, int T, int D, int dtype, int is_bwd, int Hkv = 0) {
   WsPlan p;
+  if (Hkv <= 0) Hkv = H;
   size_t off = 0;
   const size_t bt = (size_t)B * T, rows = bt * H, n = rows * D;
   const size_t tiles = (size_t)B * H * ((T + 127) / 128);
@@ -53,6 +71,12 @@ WsPlan plan(int B, int H, int T, int D, int dtype, int is_bwd) {
     p.dq_acc = off; off += round_up(n * sizeof(float));
     p.q16 = off;    off += round_up(n * 2);
     p.k16 = off;    off += round_up(n * 2);
+    p.split = choose_split(B, H, Hkv, T);
+    if (p.split > 1) {
+      const size_t nkv = bt * Hkv * D;
+      p.dk_acc = off; off += round_up(nkv * sizeof(float));
+      p.dv_acc = off; off += round_up(nkv * sizeof(float));
+    }
   }
   if (dtype == ATTN_BF16 && !is_bwd) {
     p.q16 = off;  off += round_up(n * 2);
@@ -142,7 +166,7 @@ int check_common(const void* q, const void* k, const void* v, const float* rc, c
   if (!sizes_ok(B, H, T, D)) return ATTN_EUNSUPPORTED;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return ATTN_EALIGN;
   if ((rc && !aligned(rc, 16)) || (rs && !aligned(rs, 16)) || (cu && !aligned(cu, 4))) return ATTN_EALIGN;
-  const WsPlan p = plan(B, H, T, D, dtype, is_bwd);
+  const WsPlan p = plan(B, H, T, D, dtype, is_bwd, H_kv);
   if (p.total > 0) {
     if (!ws) return ATTN_EWORKSPACE;
     if (!aligned(ws, 16)) return ATTN_EALIGN;
@@ -256,11 +280,14 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   float* lse2 = (float*)(ws + wp.lse2);
   float* dq_acc = (float*)(ws + wp.dq_acc);
   const long rows_pad = (long)BH * Tpad;
+  const int split = wp.split;
+  float* dk_acc = split > 1 ? (float*)(ws + wp.dk_acc) : nullptr;
+  float* dv_acc = split > 1 ? (float*)(ws + wp.dv_acc) : nullptr;
   ATTN_LAUNCH(KK_DELTA, st,
               bwd_prep_kernel<D><<<(unsigned)(rows_pad * (D / 8) / 256), 256, 0, st>>>(
                   (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse, delta, lse2, dq_acc,
-                  (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qr, kr, H, Hkv,
-                  T, Tpad, rows_pad));
+                  (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qr, kr, dk_acc,
+                  dv_acc, H, Hkv, T, Tpad, rows_pad));
   if (launch_status()) return ATTN_ECUDA;
   CUtensorMap mq, mk, mv, mo, mdq;
   if (!make_tile_map(&mq, qs, false, D, T, BH) || !make_tile_map(&mk, ks, false, D, T, BHkv) ||
@@ -274,6 +301,7 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   prm.H = H;
   prm.Hkv = Hkv;
   prm.BHkv = BHkv;
+  prm.n_split = split;
   prm.n_tiles = nt;
   prm.Tpad = Tpad;
   prm.scale_log2 = scale * 1.4426950408889634f;
@@ -287,10 +315,24 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   prm.dq_acc = dq_acc;
   prm.dk = (__nv_bfloat16*)dk;
   prm.dv = (__nv_bfloat16*)dv;
+  prm.dk_acc = dk_acc;
+  prm.dv_acc = dv_acc;
   ATTN_LAUNCH(KK_DKDV, st,
-              bwd100::dkdv_kernel<D><<<(unsigned)(nt * BHkv), L::kThreads, L::kSmemAlloc, st>>>(
-                  mq, mk, mv, mo, mdq, prm));
+              bwd100::dkdv_kernel<D><<<(unsigned)(nt * BHkv * split), L::kThreads, L::kSmemAlloc,
+                                       st>>>(mq, mk, mv, mo, mdq, prm));
   if (launch_status()) return ATTN_ECUDA;
+  if (split > 1) {
+    // dk = R^T (scale * sum of the parts), dv = sum of the parts
+    const long n8kv = (long)BHkv * T * D / 8;
+    ATTN_LAUNCH(KK_DQ_FINALIZE, st,
+                dq_finalize_kernel<D><<<(unsigned)((n8kv + 255) / 256), 256, 0, st>>>(
+                    dk_acc, rc, rs, ds, (__nv_bfloat16*)dk, Hkv, T, scale, n8kv));
+    if (launch_status()) return ATTN_ECUDA;
+    ATTN_LAUNCH(KK_DQ_FINALIZE, st,
+                dq_finalize_kernel<D><<<(unsigned)((n8kv + 255) / 256), 256, 0, st>>>(
+                    dv_acc, nullptr, nullptr, nullptr, (__nv_bfloat16*)dv, Hkv, T, 1.0f, n8kv));
+    if (launch_status()) return ATTN_ECUDA;
+  }
   const long n8 = (long)BH * T * D / 8;
   ATTN_LAUNCH(KK_DQ_FINALIZE, st,
               dq_finalize_kernel<D><<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
@@ -310,6 +352,12 @@ extern "C" {
 size_t attn_workspace_bytes(int B, int H, int T, int D, int dtype, int is_bwd) {
   if (!sizes_ok(B, H, T, D) || (dtype != ATTN_BF16 && dtype != ATTN_F32)) return 0;
   return plan(B, H, T, D, dtype, is_bwd).total;
+}
+
+size_t attn_workspace_bytes_gqa(int B, int H, int H_kv, int T, int D, int dtype, int is_bwd) {
+  if (!sizes_ok(B, H, T, D) || (dtype != ATTN_BF16 && dtype != ATTN_F32)) return 0;
+  if (H_kv <= 0 || H % H_kv != 0) return 0;
+  return plan(B, H, T, D, dtype, is_bwd, H_kv).total;
 }
 
 int attn_fwd_gqa(const void* q, const void* k, const void* v, const float* rope_cos,
@@ -365,7 +413,7 @@ int attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, con
       !aligned(dv, 16) || !aligned(lse, 4))
     return ATTN_EALIGN;
   cudaStream_t st = (cudaStream_t)stream;
-  const WsPlan p = plan(B, H, T, D, dtype, 1);
+  const WsPlan p = plan(B, H, T, D, dtype, 1, H_kv);
   char* ws = (char*)workspace;
   int32_t *ds = nullptr, *de = nullptr;
   if (cu_seqlens) {

@@ -89,6 +89,7 @@ struct Layout {
 
 struct Params {
   int T, H, Hkv, BHkv, n_tiles, Tpad;  // H query heads read Hkv key/value heads
+  int n_split;  // CTAs sharing one (key/value head, key tile): each takes H/Hkv/n_split query heads
   float scale_log2;  // scale * log2(e)
   float scale;
   const float* lse2;       // [B*H][Tpad] -lse * log2(e), zero-padded
@@ -100,6 +101,8 @@ struct Params {
   float* dq_acc;           // [B*H][T][D] fp32
   __nv_bfloat16* dk;       // [B*Hkv][T][D]
   __nv_bfloat16* dv;
+  float* dk_acc;           // [B*Hkv][T][D] fp32 (n_split > 1: the parts are added here)
+  float* dv_acc;
 };
 
 // Byte offset of 16-byte chunk `ch` (0..7 within a 64-column block) of row r
@@ -128,14 +131,15 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.T;
   // Flattened grid, heaviest key tiles (the earliest, which see the most
-  // query tiles) first. One CTA per (key/value head, key tile); it walks the
-  // query tiles of every query head reading that key/value head (G of them),
-  // head by head: step `it` is query tile qt0 + it % n_q of the group's
-  // it / n_q-th head.
+  // query tiles) first. n_split CTAs per (key/value head, key tile); each
+  // walks the query tiles of G = H/Hkv/n_split query heads reading that
+  // key/value head, head by head: step `it` is query tile qt0 + it % n_q of
+  // its it / n_q-th head.
   const int bhk = (int)blockIdx.x % p.BHkv, b = bhk / p.Hkv;
-  const int kt = (int)blockIdx.x / p.BHkv;
-  const int G = p.H / p.Hkv;
-  const int bhq0 = b * p.H + (bhk - b * p.Hkv) * G;  // first query head of the group
+  const int kt = (int)blockIdx.x / (p.BHkv * p.n_split);
+  const int part = ((int)blockIdx.x / p.BHkv) % p.n_split;
+  const int G = p.H / p.Hkv / p.n_split;
+  const int bhq0 = b * p.H + (bhk - b * p.Hkv) * (p.H / p.Hkv) + part * G;  // first query head
   const int j0 = kt * 128;
   const int row0 = b * T;
   const int jlast = min(j0 + 127, T - 1);
@@ -498,6 +502,27 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         if constexpr (CW == 32) tmem_ld32(taddr, v);
         else tmem_ld16(taddr, v);
       };
+      if (p.n_split > 1) {
+        // this CTA's part of dK_r and dV: added into the fp32 accumulators
+        // (scale and R^T are applied by the finishing pass)
+        float* dka = p.dk_acc + ((size_t)bhk * T + jj) * D;
+        float* dva = p.dv_acc + ((size_t)bhk * T + jj) * D;
+#pragma unroll
+        for (int c = 0; c < DC / CW; ++c) {
+          const int col = dc0 + CW * c;
+          uint32_t v[CW], u[CW];
+          ld(tmem + lane_base + L::kColDK + col, v);
+          ld(tmem + lane_base + L::kColDV + col, u);
+          tmem_wait_ld();
+          if (j < T) {
+#pragma unroll
+            for (int e = 0; e < CW / 4; ++e) {
+              red_add_v4(dka + col + 4 * e, v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+              red_add_v4(dva + col + 4 * e, u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3]);
+            }
+          }
+        }
+      } else {
 #pragma unroll
       for (int c = 0; c < DC / CW; ++c) {
         const int col = dc0 + CW * c;
@@ -531,6 +556,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
                 pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
                 pack_bf16(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
         }
+      }
       }
     }
   }

@@ -184,8 +184,10 @@ __device__ __forceinline__ void store8_bf16(__nv_bfloat16* p, const float* v) {
 // folds them in with one fused multiply-add (both 0 for padding rows t >= T,
 // so its per-tile loads never leave the arrays), zeroes the fp32 dq
 // accumulator row and, with RoPE tables, writes the rotated q and k rows
-// (bf16) the main kernel reads. The grid covers rows_pad * D/8 threads
-// exactly (rows_pad is a multiple of 128), so every warp is full.
+// (bf16) the main kernel reads; when the grouped-query backward splits its
+// groups, it also zeroes the fp32 dk, dv accumulator rows. The grid covers
+// rows_pad * D/8 threads exactly (rows_pad is a multiple of 128), so every
+// warp is full.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(
     const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
@@ -193,8 +195,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
     float* __restrict__ dq_acc, const __nv_bfloat16* __restrict__ q,
     const __nv_bfloat16* __restrict__ k, const float* __restrict__ rc,
     const float* __restrict__ rs, const int32_t* __restrict__ doc_start,
-    __nv_bfloat16* __restrict__ qr, __nv_bfloat16* __restrict__ kr, int H, int Hkv, int T,
-    int Tpad, long rows_pad) {
+    __nv_bfloat16* __restrict__ qr, __nv_bfloat16* __restrict__ kr, float* __restrict__ dk_acc,
+    float* __restrict__ dv_acc, int H, int Hkv, int T, int Tpad, long rows_pad) {
   constexpr int TPR = D / 8;  // threads per row
   const long gt = (long)blockIdx.x * blockDim.x + threadIdx.x;
   const long row = gt / TPR;
@@ -212,6 +214,12 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
     reinterpret_cast<float4*>(dq_acc + r * D + c8)[0] = z;
     reinterpret_cast<float4*>(dq_acc + r * D + c8)[1] = z;
+    if (dk_acc && bh < (rows_pad / Tpad) / H * Hkv) {  // a row of the [B*Hkv][T] view
+      reinterpret_cast<float4*>(dk_acc + r * D + c8)[0] = z;
+      reinterpret_cast<float4*>(dk_acc + r * D + c8)[1] = z;
+      reinterpret_cast<float4*>(dv_acc + r * D + c8)[0] = z;
+      reinterpret_cast<float4*>(dv_acc + r * D + c8)[1] = z;
+    }
     if (rc) {
       const int b = (int)(bh / H);
       const int pos = t - (doc_start ? doc_start[b * T + t] - b * T : 0);

@@ -14,7 +14,7 @@ import numpy as np
 import torch
 
 from . import (ATTN_BF16, ATTN_F32, attn_bwd, attn_bwd_gqa, attn_fwd, attn_fwd_gqa,
-               attn_get_status, attn_workspace_bytes, check)
+               attn_get_status, attn_workspace_bytes, attn_workspace_bytes_gqa, check)
 
 
 def torch_dtype(dtype: int):
@@ -63,8 +63,12 @@ class AttnRunner:
         self.cu = None
         if cu_seqlens is not None:
             self.cu = torch.from_numpy(np.asarray(cu_seqlens, dtype=np.int32)).to(self.device)
-        self.ws_bytes = max(attn_workspace_bytes(B, H, T, D, dtype, 0),
-                            attn_workspace_bytes(B, H, T, D, dtype, 1))
+        if H_kv == H:
+            self.ws_bytes = max(attn_workspace_bytes(B, H, T, D, dtype, 0),
+                                attn_workspace_bytes(B, H, T, D, dtype, 1))
+        else:
+            self.ws_bytes = max(attn_workspace_bytes_gqa(B, H, H_kv, T, D, dtype, 0),
+                                attn_workspace_bytes_gqa(B, H, H_kv, T, D, dtype, 1))
         self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=self.device)
 
     @classmethod

@@ -114,9 +114,12 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o,
  * attn_fwd_gqa / attn_bwd_gqa take the arguments of attn_fwd / attn_bwd plus
  * H_kv (after H) and follow their rules, with these shapes:
  *   q, o, dO, dq [B, H, T, D]; k, v, dk, dv [B, H_kv, T, D]; lse [B, H, T].
- * Workspace: attn_workspace_bytes(B, H, T, D, dtype, is_bwd) bytes (sized by
- * the query heads H). H_kv <= 0 or H not a multiple of H_kv: ATTN_EINVAL.
- * attn_fwd and attn_bwd are these calls with H_kv = H.
+ * Workspace: attn_workspace_bytes_gqa(B, H, H_kv, T, D, dtype, is_bwd) bytes.
+ * (When the key/value heads times the 128-key tiles are too few to fill the
+ * GPU, the bf16 backward splits each group of query heads over several CTAs
+ * and needs room for fp32 dk, dv accumulators; the size includes it.)
+ * H_kv <= 0 or H not a multiple of H_kv: ATTN_EINVAL. attn_fwd and attn_bwd
+ * are these calls with H_kv = H.
  */
 int attn_fwd_gqa(const void* q, const void* k, const void* v,
                  const float* rope_cos, const float* rope_sin,
@@ -136,6 +139,10 @@ int attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
 /* Bytes of workspace attn_fwd (is_bwd = 0) or attn_bwd (is_bwd = 1) needs for
  * these sizes; 0 for invalid sizes. Pure host function, no CUDA call. */
 size_t attn_workspace_bytes(int B, int H, int T, int D, int dtype, int is_bwd);
+
+/* The same for attn_fwd_gqa / attn_bwd_gqa (H_kv key/value heads); 0 for
+ * invalid sizes, including H_kv not dividing H. Pure host function. */
+size_t attn_workspace_bytes_gqa(int B, int H, int H_kv, int T, int D, int dtype, int is_bwd);
 
 /* Synchronises `stream`, then returns and clears the current device's status
  * word: ATTN_OK, ATTN_EDEVICE_INPUT or ATTN_ETIMEOUT (first error recorded

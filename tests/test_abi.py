@@ -141,3 +141,21 @@ def test_grouped_query_host_validation(call):
     assert call(D=96) == A.ATTN_EUNSUPPORTED
     assert call(v=P + 8) == A.ATTN_EALIGN
     assert call(ws_bytes=16) == A.ATTN_EWORKSPACE
+
+
+def test_grouped_query_workspace_bytes():
+    import bwd_causal_sdpa_b200 as A
+
+    # G = 1 is the plain call's plan
+    for is_bwd in (0, 1):
+        assert (A.attn_workspace_bytes_gqa(2, 4, 4, 300, 128, A.ATTN_BF16, is_bwd)
+                == A.attn_workspace_bytes(2, 4, 300, 128, A.ATTN_BF16, is_bwd))
+    # a small grid splits the bf16 backward's groups: two fp32 [B*H_kv*T*D] accumulators more
+    base = A.attn_workspace_bytes(1, 16, 4096, 128, A.ATTN_BF16, 1)
+    split = A.attn_workspace_bytes_gqa(1, 16, 1, 4096, 128, A.ATTN_BF16, 1)
+    assert split >= base + 2 * 4096 * 128 * 4
+    # enough key/value heads x key tiles: no split, no extra room
+    assert (A.attn_workspace_bytes_gqa(4, 16, 8, 1280, 128, A.ATTN_BF16, 1)
+            <= A.attn_workspace_bytes(4, 16, 1280, 128, A.ATTN_BF16, 1))
+    assert A.attn_workspace_bytes_gqa(1, 4, 3, 128, 64, A.ATTN_BF16, 1) == 0
+    assert A.attn_workspace_bytes_gqa(1, 4, 0, 128, 64, A.ATTN_BF16, 1) == 0

@@ -56,6 +56,21 @@ def test_grouped_query_full_8k_sampled_group_matches_oracle():
     print(errs)
 
 
+@pytest.mark.parametrize("name,over,heads", [
+    # 16 query heads on one key/value head at T = 4096: each group is split
+    # over CTAs whose dk, dv parts are added in fp32 (the whole group compared)
+    ("long_context_8k", dict(H=16, H_kv=1, T=4096, seed=61), [(0, h) for h in range(16)]),
+    # enough key/value heads x key tiles to fill the GPU: no split (two groups compared)
+    ("packed_docs", dict(B=4, H=16, H_kv=8, T=1280, seed=62),
+     [(0, 0), (0, 1), (3, 14), (3, 15)]),
+], ids=["split_groups", "whole_groups"])
+def test_grouped_query_group_split_and_whole(name, over, heads):
+    _cuda()
+    w = make_workload(config_by_name(name), **over)
+    errs = compare(w, gpu_outputs(w), oracle_outputs(w, heads=heads), heads=heads)
+    print(name, over, errs)
+
+
 @pytest.mark.parametrize("name,over", [
     ("packed_docs", dict(B=2, H=4, H_kv=2, T=1000, seed=51)),
     ("tiny_fp32", dict(H=4, H_kv=1, T=260, seed=52)),
