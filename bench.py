@@ -41,10 +41,10 @@ FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # one ncu capture of the kernel on the workload, valid only while the kernel
 # sources still hash to what was captured (sha256, first 16 hex digits).
 MEASURED_TRAFFIC = {
-    ("dkdv", "long_context_8k"): (693.9e6, {"bwd_sm100.cuh": "0640f045771bd29b",
-                                            "sm100.cuh": "789bfda255dd1463"}),
-    ("fwd", "long_context_8k"): (156.4e6, {"fwd_sm100.cuh": "99e0fc780a6f5b58",
-                                           "sm100.cuh": "789bfda255dd1463"}),
+    ("dkdv", "long_context_8k"): (706.5e6, {"bwd_sm100.cuh": "a4e087a6ca38c64f",
+                                            "sm100.cuh": "1a2b026d7dc3ce22"}),
+    ("fwd", "long_context_8k"): (158.3e6, {"fwd_sm100.cuh": "2e9f5f7955c71a01",
+                                           "sm100.cuh": "1a2b026d7dc3ce22"}),
 }
 
 

@@ -12,10 +12,13 @@ something other than itself: central finite differences, closed forms, hand
 derived worked examples (``tests/golden``), invariants (softmax rows sum to 1,
 causality, RoPE norm preservation and relative-position dependence,
 packed-equals-separate documents) and the float64 PyTorch reference
-``scaled_dot_product_attention`` on the cases it covers. No function here is
+``scaled_dot_product_attention`` on the cases it covers. ``oracle.decode``
+(one new token against a key/value cache) is pinned against the last row of
+the training forward, a closed form and invariants. No function here is
 "parity unpinned".
 """
 
+from .decode import decode_forward
 from .attention import (
     attention_backward,
     attention_forward,
@@ -28,6 +31,7 @@ from .attention import (
 )
 
 __all__ = [
+    "decode_forward",
     "attention_backward",
     "attention_forward",
     "backward_head",
