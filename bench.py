@@ -70,6 +70,8 @@ def parse_args():
     ap.add_argument("--workload", default="long_context_8k")
     ap.add_argument("--kv-heads", type=int, default=None,
                     help="grouped-query attention: key/value heads (dividing the workload's H)")
+    ap.add_argument("--decode", default=None,
+                    help="time decode attention on this decode workload instead of the training step")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -452,8 +454,74 @@ def run_ours(args):
     return 0
 
 
+def run_decode(args):
+    """Decode attention (one new token per sequence against a key/value
+    cache): bytes of cache read per second, against the measured HBM copy
+    bandwidth; L2 is flushed between steps as in the training bench."""
+    import torch
+
+    import bwd_causal_sdpa_b200 as A
+    from bwd_causal_sdpa_b200.runner import DecodeRunner
+    from workloads import decode_config_by_name, make_decode_workload
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = make_decode_workload(decode_config_by_name(args.decode))
+    stream = torch.cuda.Stream(dev)
+    r = DecodeRunner(w, device=dev, stream=stream)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peaks, peak_src = load_peaks()
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 0)):
+            r.run()
+    if r.status() != A.ATTN_OK:
+        raise SystemExit("device status after warm-up is not OK")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    n0 = A.attn_launch_count()
+    A.check(A.attn_profile_enable(1), "attn_profile_enable")
+    with ClockSampler(0) as clocks:
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                flush.zero_()
+                ev[i][0].record(stream)
+                r.run()
+                ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    A.attn_profile_enable(0)
+    launches = A.attn_launch_count() - n0
+    prof = A.profile_summary()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    nbytes = w.cache_bytes_read()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    kd = prof.get("decode")
+    achieved = nbytes / (kd[1] / kd[0] / 1e3) / 1e9 if kd else None
+    line = {
+        "metric": "decode attention: key/value cache bytes read per second", "value": gbs,
+        "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded)",
+        "config": {"workload": w.cfg.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "T_max": w.T_max,
+                   "D": w.D, "cache_tokens": int(w.cache_lens.sum()), "cache_bytes": nbytes,
+                   "l2": "flushed between steps (256 MiB write outside the step events)"},
+        "roofline": None if achieved is None else {
+            "bound": "hbm", "kernel": "decode", "achieved": achieved, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+            "peak_source": f"hbm_gbs ({peak_src})"},
+        "kernels": {k: {"launches": n, "avg_ms": t / n} for k, (n, t) in prof.items()},
+        "gpu_launches": launches, "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.decode:
+        return run_decode(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -42,6 +42,9 @@ _SIGNATURES = {
                           _P, ctypes.c_size_t, _P]),
     "attn_bwd_gqa": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.c_float,
                           _I, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I,
+                         _P, ctypes.c_size_t, _P]),
+    "attn_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
     "attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float,
                               _I, _P, _P, _P, _P]),
     "attn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
@@ -138,6 +141,19 @@ def attn_bwd_gqa(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, H_kv
                                  _ptr(rope_cos), _ptr(rope_sin), _ptr(cu_seqlens), B, H, H_kv,
                                  T, D, float(scale), dtype, _ptr(dq), _ptr(dk), _ptr(dv),
                                  _ptr(workspace), int(ws_bytes), _stream(stream)))
+
+
+def attn_decode(q, k_cache, v_cache, cache_lens, rope_cos, rope_sin, o, lse, B, H, H_kv, T_max,
+                D, scale, dtype, workspace, ws_bytes, stream=None) -> int:
+    """One new token per sequence against a key/value cache (see include/attn.h)."""
+    return int(_lib.attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens),
+                                _ptr(rope_cos), _ptr(rope_sin), _ptr(o), _ptr(lse), B, H, H_kv,
+                                T_max, D, float(scale), dtype, _ptr(workspace), int(ws_bytes),
+                                _stream(stream)))
+
+
+def attn_decode_workspace_bytes(B, H, H_kv, T_max, D, dtype) -> int:
+    return int(_lib.attn_decode_workspace_bytes(B, H, H_kv, T_max, D, dtype))
 
 
 def attn_bwd_noalloc(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, T, D, scale,

@@ -9,6 +9,7 @@
 #include "attn.h"
 #include "common.cuh"
 #include "bwd_sm100.cuh"
+#include "decode.cuh"
 #include "fwd_sm100.cuh"
 #include "prep.cuh"
 #include "simt.cuh"
@@ -491,6 +492,107 @@ int attn_profile_read(int kind, const char** name, int* launches, double* total_
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// attn_decode: one new token per sequence against a key/value cache
+// ---------------------------------------------------------------------------
+namespace {
+
+// Workspace: per (query head, key chunk) the unnormalised partial sum
+// (f32 [B*H][n_chunks][D]), then its max and sum of exponentials
+// (f32 [B*H][n_chunks] each).
+struct DecodePlan {
+  size_t o_part = 0, m_part = 0, l_part = 0, total = 0;
+  int n_chunks = 0;
+};
+
+DecodePlan decode_plan(int B, int H, int T_max, int D) {
+  DecodePlan p;
+  p.n_chunks = (T_max + kDecodeChunk - 1) / kDecodeChunk;
+  const size_t slots = (size_t)B * H * p.n_chunks;
+  p.o_part = 0;
+  p.m_part = round_up(slots * D * sizeof(float));
+  p.l_part = p.m_part + round_up(slots * sizeof(float));
+  p.total = p.l_part + round_up(slots * sizeof(float));
+  return p;
+}
+
+bool decode_sizes_ok(int B, int H, int H_kv, int T_max, int D) {
+  if (B <= 0 || H <= 0 || H_kv <= 0 || T_max <= 0 || H % H_kv) return false;
+  if (D != 64 && D != 128) return false;
+  if (H / H_kv > kDecodeMaxGroup) return false;
+  if ((int64_t)B * H_kv > 65535) return false;  // grid y
+  return (int64_t)B * H_kv * T_max * D < ((int64_t)1 << 40);
+}
+
+template <typename TIO, int D>
+int decode_launch(const void* q, const void* k, const void* v, const int32_t* lens,
+                  const float* rc, const float* rs, void* o, float* lse, int B, int H, int H_kv,
+                  int T_max, float scale, char* ws, const DecodePlan& dp, cudaStream_t st) {
+  using L = DecodeLayout<TIO, D>;
+  static bool smem_set[64] = {};
+  if (!ensure_smem(decode_chunk_kernel<TIO, D>, L::bytes(kDecodeMaxGroup), smem_set))
+    return ATTN_ECUDA;
+  float* op = (float*)(ws + dp.o_part);
+  float* mp = (float*)(ws + dp.m_part);
+  float* lp = (float*)(ws + dp.l_part);
+  const int G = H / H_kv;
+  ATTN_LAUNCH(KK_DECODE, st,
+              decode_chunk_kernel<TIO, D><<<dim3(dp.n_chunks, B * H_kv), kDecodeThreads,
+                                            L::bytes(G), st>>>(
+                  (const TIO*)q, (const TIO*)k, (const TIO*)v, lens, rc, rs, op, mp, lp, H, H_kv,
+                  T_max, dp.n_chunks, scale * 1.4426950408889634f));
+  if (launch_status()) return ATTN_ECUDA;
+  const int BH = B * H;
+  ATTN_LAUNCH(KK_DECODE_COMBINE, st,
+              decode_combine_kernel<TIO, D><<<(BH + 7) / 8, 256, 0, st>>>(
+                  op, mp, lp, lens, (TIO*)o, lse, H, T_max, dp.n_chunks, BH));
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" size_t attn_decode_workspace_bytes(int B, int H, int H_kv, int T_max, int D,
+                                              int dtype) {
+  if (!decode_sizes_ok(B, H, H_kv, T_max, D) || (dtype != ATTN_BF16 && dtype != ATTN_F32))
+    return 0;
+  return decode_plan(B, H, T_max, D).total;
+}
+
+extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* cache_lens, const float* rope_cos,
+                           const float* rope_sin, void* o, float* lse, int B, int H, int H_kv,
+                           int T_max, int D, float scale, int dtype, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  if (!q || !k_cache || !v_cache || !cache_lens || !o || !lse) return ATTN_EINVAL;
+  if (dtype != ATTN_BF16 && dtype != ATTN_F32) return ATTN_EINVAL;
+  if (B <= 0 || H <= 0 || T_max <= 0 || !isfinite(scale)) return ATTN_EINVAL;
+  if (H_kv <= 0 || H % H_kv) return ATTN_EINVAL;
+  if ((rope_cos == nullptr) != (rope_sin == nullptr)) return ATTN_EINVAL;
+  if (!decode_sizes_ok(B, H, H_kv, T_max, D)) return ATTN_EUNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || !aligned(cache_lens, 4) || (rope_cos && !aligned(rope_cos, 16)) ||
+      (rope_sin && !aligned(rope_sin, 16)))
+    return ATTN_EALIGN;
+  const DecodePlan dp = decode_plan(B, H, T_max, D);
+  if (!workspace) return ATTN_EWORKSPACE;
+  if (!aligned(workspace, 16)) return ATTN_EALIGN;
+  if (ws_bytes < dp.total) return ATTN_EWORKSPACE;
+  char* ws = (char*)workspace;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (dtype == ATTN_F32)
+    return D == 64 ? decode_launch<float, 64>(q, k_cache, v_cache, cache_lens, rope_cos, rope_sin,
+                                              o, lse, B, H, H_kv, T_max, scale, ws, dp, st)
+                   : decode_launch<float, 128>(q, k_cache, v_cache, cache_lens, rope_cos,
+                                               rope_sin, o, lse, B, H, H_kv, T_max, scale, ws, dp,
+                                               st);
+  return D == 64 ? decode_launch<__nv_bfloat16, 64>(q, k_cache, v_cache, cache_lens, rope_cos,
+                                                    rope_sin, o, lse, B, H, H_kv, T_max, scale, ws,
+                                                    dp, st)
+                 : decode_launch<__nv_bfloat16, 128>(q, k_cache, v_cache, cache_lens, rope_cos,
+                                                     rope_sin, o, lse, B, H, H_kv, T_max, scale,
+                                                     ws, dp, st);
+}
 
 // ---------------------------------------------------------------------------
 // attn_bwd_noalloc: the backward for callers that cannot allocate device

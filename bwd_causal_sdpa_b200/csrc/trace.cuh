@@ -14,11 +14,14 @@ enum KernelKind : int {
   KK_DKDV,
   KK_DQ,
   KK_DQ_FINALIZE,
+  KK_DECODE,
+  KK_DECODE_COMBINE,
   KK_COUNT
 };
 
 static const char* const kKernelNames[KK_COUNT] = {
-    "doc_ranges", "rope_prep", "fwd", "delta", "dkdv", "dq", "dq_finalize"};
+    "doc_ranges", "rope_prep", "fwd", "delta", "dkdv", "dq", "dq_finalize", "decode",
+    "decode_combine"};
 
 namespace trace {
 

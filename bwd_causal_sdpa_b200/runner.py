@@ -116,3 +116,45 @@ class AttnRunner:
         f = lambda t: t.detach().to(torch.float64).cpu().numpy()
         return {"o": f(self.o), "lse": f(self.lse), "dq": f(self.dq), "dk": f(self.dk),
                 "dv": f(self.dv)}
+
+
+class DecodeRunner:
+    """Device buffers for one decode step (q, the key/value cache, the cache
+    lengths, o, lse, the RoPE tables and the workspace) and the attn_decode
+    call on them."""
+
+    def __init__(self, w, device="cuda", stream: Optional[torch.cuda.Stream] = None):
+        from . import attn_decode_workspace_bytes
+
+        self.w = w
+        self.device = torch.device(device)
+        self.stream = stream
+        self.dtype = ATTN_BF16 if w.dtype == "bf16" else ATTN_F32
+        self.q = to_device(w.q, self.dtype, self.device)
+        self.k = to_device(w.k_cache, self.dtype, self.device)
+        self.v = to_device(w.v_cache, self.dtype, self.device)
+        self.lens = torch.from_numpy(np.asarray(w.cache_lens, np.int32)).to(self.device)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((w.B, w.H), dtype=torch.float32, device=self.device)
+        self.rope_cos = self.rope_sin = None
+        if w.rope_cos is not None:
+            self.rope_cos = torch.from_numpy(np.ascontiguousarray(w.rope_cos, np.float32)).to(self.device)
+            self.rope_sin = torch.from_numpy(np.ascontiguousarray(w.rope_sin, np.float32)).to(self.device)
+        self.ws_bytes = attn_decode_workspace_bytes(w.B, w.H, w.H_kv, w.T_max, w.D, self.dtype)
+        self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=self.device)
+
+    def run(self) -> None:
+        from . import attn_decode
+
+        w = self.w
+        check(attn_decode(self.q, self.k, self.v, self.lens, self.rope_cos, self.rope_sin, self.o,
+                          self.lse, w.B, w.H, w.H_kv, w.T_max, w.D, w.scale, self.dtype, self.ws,
+                          self.ws_bytes, self.stream), "attn_decode")
+
+    def status(self) -> int:
+        return attn_get_status(self.stream)
+
+    def results(self) -> dict:
+        torch.cuda.synchronize(self.device)
+        f = lambda t: t.detach().to(torch.float64).cpu().numpy()
+        return {"o": f(self.o), "lse": f(self.lse)}

@@ -144,6 +144,38 @@ size_t attn_workspace_bytes(int B, int H, int T, int D, int dtype, int is_bwd);
  * invalid sizes, including H_kv not dividing H. Pure host function. */
 size_t attn_workspace_bytes_gqa(int B, int H, int H_kv, int T, int D, int dtype, int is_bwd);
 
+/*
+ * attn_decode -- decode attention: one new token per sequence against a
+ * key/value cache (Forge README, "Roadmap": a KV cache for generation on the
+ * training attention module; ARK README, "Inference architecture (EKO)":
+ * RoPE from precomputed tables).
+ * In:  q [B, H, D] (dtype): the new token's queries, un-rotated;
+ *      k_cache, v_cache [B, H_kv, T_max, D] (dtype): row b holds
+ *      cache_lens[b] tokens at positions 0 .. cache_lens[b]-1, the new
+ *      token's own key and value included; keys are stored already rotated
+ *      by their positions (as attn_fwd rotates k); rows past cache_lens[b]
+ *      are never read;
+ *      cache_lens [B] int32 device array, each in [1, T_max] (a value out of
+ *      range is clamped into it and the status word reports
+ *      ATTN_EDEVICE_INPUT);
+ *      rope_cos, rope_sin [T_max, D/2] f32 or NULL: the query is rotated at
+ *      position cache_lens[b]-1;
+ *      H_kv divides H (query head h reads cache head h / (H / H_kv)), at
+ *      most 64 query heads per key/value head; B * H_kv <= 65535.
+ * Out: o [B, H, D] (dtype) = softmax_j(scale * q_r . k_j) v_j over the
+ *      cached tokens; lse [B, H] f32, natural log.
+ * Workspace: attn_decode_workspace_bytes(B, H, H_kv, T_max, D, dtype) bytes.
+ * Alignment, ownership, asynchrony and return codes as for attn_fwd.
+ */
+int attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                const int32_t* cache_lens, const float* rope_cos, const float* rope_sin,
+                void* o, float* lse, int B, int H, int H_kv, int T_max, int D, float scale,
+                int dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of workspace attn_decode needs; 0 for invalid or unsupported sizes.
+ * Pure host function, no CUDA call. */
+size_t attn_decode_workspace_bytes(int B, int H, int H_kv, int T_max, int D, int dtype);
+
 /* Synchronises `stream`, then returns and clears the current device's status
  * word: ATTN_OK, ATTN_EDEVICE_INPUT or ATTN_ETIMEOUT (first error recorded
  * since the last call), or ATTN_ECUDA if the synchronisation itself failed. */

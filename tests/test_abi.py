@@ -159,3 +159,35 @@ def test_grouped_query_workspace_bytes():
             <= A.attn_workspace_bytes(4, 16, 1280, 128, A.ATTN_BF16, 1))
     assert A.attn_workspace_bytes_gqa(1, 4, 3, 128, 64, A.ATTN_BF16, 1) == 0
     assert A.attn_workspace_bytes_gqa(1, 4, 0, 128, 64, A.ATTN_BF16, 1) == 0
+
+
+def _decode(**kw):
+    import bwd_causal_sdpa_b200 as A
+
+    a = dict(q=P, k_cache=P, v_cache=P, cache_lens=P, rope_cos=None, rope_sin=None, o=P, lse=P,
+             B=2, H=8, H_kv=2, T_max=1000, D=128, scale=0.088, dtype=A.ATTN_BF16, workspace=P,
+             ws_bytes=1 << 30)
+    a.update(kw)
+    return A.attn_decode(**a)
+
+
+def test_decode_host_validation_and_workspace():
+    import bwd_causal_sdpa_b200 as A
+
+    assert _decode(q=None) == A.ATTN_EINVAL
+    assert _decode(cache_lens=None) == A.ATTN_EINVAL
+    assert _decode(H_kv=3) == A.ATTN_EINVAL
+    assert _decode(T_max=0) == A.ATTN_EINVAL
+    assert _decode(dtype=9) == A.ATTN_EINVAL
+    assert _decode(rope_sin=P) == A.ATTN_EINVAL
+    assert _decode(D=96) == A.ATTN_EUNSUPPORTED
+    assert _decode(H=130, H_kv=2) == A.ATTN_EUNSUPPORTED   # 65 query heads per cached head
+    assert _decode(v_cache=P + 8) == A.ATTN_EALIGN
+    assert _decode(cache_lens=P + 2) == A.ATTN_EALIGN
+    assert _decode(workspace=None) == A.ATTN_EWORKSPACE
+    assert _decode(ws_bytes=64) == A.ATTN_EWORKSPACE
+    # partial sums f32 [B*H][chunks][D] plus two f32 [B*H][chunks], chunks of 128 tokens
+    nb = A.attn_decode_workspace_bytes(2, 8, 2, 1000, 128, A.ATTN_BF16)
+    assert nb >= 2 * 8 * 8 * (128 + 2) * 4
+    assert A.attn_decode_workspace_bytes(2, 8, 3, 1000, 128, A.ATTN_BF16) == 0
+    assert A.attn_decode_workspace_bytes(2, 8, 2, 1000, 80, A.ATTN_BF16) == 0

@@ -7,6 +7,13 @@ sharing any of the method's code.
 """
 
 from .configs import CONFIGS, Config, config_by_name
+from .decode import (
+    DECODE_CONFIGS,
+    DecodeConfig,
+    DecodeWorkload,
+    decode_config_by_name,
+    make_decode_workload,
+)
 from .generate import (
     Workload,
     draw_doc_lengths,
@@ -17,6 +24,11 @@ from .generate import (
 
 __all__ = [
     "CONFIGS",
+    "DECODE_CONFIGS",
+    "DecodeConfig",
+    "DecodeWorkload",
+    "decode_config_by_name",
+    "make_decode_workload",
     "Config",
     "Workload",
     "config_by_name",
