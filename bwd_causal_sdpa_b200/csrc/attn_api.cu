@@ -498,18 +498,20 @@ int attn_profile_read(int kind, const char** name, int* launches, double* total_
 // ---------------------------------------------------------------------------
 namespace {
 
-// Workspace: per (query head, key chunk) the unnormalised partial sum
-// (f32 [B*H][n_chunks][D]), then its max and sum of exponentials
-// (f32 [B*H][n_chunks] each).
+// Workspace: per (query head, cache chunk of kDecodeChunk tokens) the
+// unnormalised partial sum (f32 [B*H][n_split][D]), then its max and sum of
+// exponentials (f32 [B*H][n_split] each).
 struct DecodePlan {
   size_t o_part = 0, m_part = 0, l_part = 0, total = 0;
-  int n_chunks = 0;
+  int n_split = 0, per_split = 0;
 };
 
-DecodePlan decode_plan(int B, int H, int T_max, int D) {
+DecodePlan decode_plan(int B, int H, int H_kv, int T_max, int D) {
   DecodePlan p;
-  p.n_chunks = (T_max + kDecodeChunk - 1) / kDecodeChunk;
-  const size_t slots = (size_t)B * H * p.n_chunks;
+  (void)H_kv;
+  p.per_split = kDecodeChunk;
+  p.n_split = (T_max + kDecodeChunk - 1) / kDecodeChunk;
+  const size_t slots = (size_t)B * H * p.n_split;
   p.o_part = 0;
   p.m_part = round_up(slots * D * sizeof(float));
   p.l_part = p.m_part + round_up(slots * sizeof(float));
@@ -531,22 +533,21 @@ int decode_launch(const void* q, const void* k, const void* v, const int32_t* le
                   int T_max, float scale, char* ws, const DecodePlan& dp, cudaStream_t st) {
   using L = DecodeLayout<TIO, D>;
   static bool smem_set[64] = {};
-  if (!ensure_smem(decode_chunk_kernel<TIO, D>, L::bytes(kDecodeMaxGroup), smem_set))
+  if (!ensure_smem(decode_split_kernel<TIO, D>, L::bytes(kDecodeMaxGroup), smem_set))
     return ATTN_ECUDA;
   float* op = (float*)(ws + dp.o_part);
   float* mp = (float*)(ws + dp.m_part);
   float* lp = (float*)(ws + dp.l_part);
   const int G = H / H_kv;
   ATTN_LAUNCH(KK_DECODE, st,
-              decode_chunk_kernel<TIO, D><<<dim3(dp.n_chunks, B * H_kv), kDecodeThreads,
+              decode_split_kernel<TIO, D><<<dim3(dp.n_split, B * H_kv), kDecodeThreads,
                                             L::bytes(G), st>>>(
                   (const TIO*)q, (const TIO*)k, (const TIO*)v, lens, rc, rs, op, mp, lp, H, H_kv,
-                  T_max, dp.n_chunks, scale * 1.4426950408889634f));
+                  T_max, dp.n_split, dp.per_split, scale * 1.4426950408889634f));
   if (launch_status()) return ATTN_ECUDA;
-  const int BH = B * H;
   ATTN_LAUNCH(KK_DECODE_COMBINE, st,
-              decode_combine_kernel<TIO, D><<<(BH + 7) / 8, 256, 0, st>>>(
-                  op, mp, lp, lens, (TIO*)o, lse, H, T_max, dp.n_chunks, BH));
+              decode_combine_kernel<TIO, D><<<B * H, D, 0, st>>>(
+                  op, mp, lp, lens, (TIO*)o, lse, H, T_max, dp.n_split, dp.per_split));
   return launch_status();
 }
 
@@ -556,7 +557,7 @@ extern "C" size_t attn_decode_workspace_bytes(int B, int H, int H_kv, int T_max,
                                               int dtype) {
   if (!decode_sizes_ok(B, H, H_kv, T_max, D) || (dtype != ATTN_BF16 && dtype != ATTN_F32))
     return 0;
-  return decode_plan(B, H, T_max, D).total;
+  return decode_plan(B, H, H_kv, T_max, D).total;
 }
 
 extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cache,
@@ -574,7 +575,7 @@ extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cac
       !aligned(lse, 4) || !aligned(cache_lens, 4) || (rope_cos && !aligned(rope_cos, 16)) ||
       (rope_sin && !aligned(rope_sin, 16)))
     return ATTN_EALIGN;
-  const DecodePlan dp = decode_plan(B, H, T_max, D);
+  const DecodePlan dp = decode_plan(B, H, H_kv, T_max, D);
   if (!workspace) return ATTN_EWORKSPACE;
   if (!aligned(workspace, 16)) return ATTN_EALIGN;
   if (ws_bytes < dp.total) return ATTN_EWORKSPACE;
