@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "attn.h"
 #include "common.cuh"
@@ -524,6 +525,7 @@ bool decode_sizes_ok(int B, int H, int H_kv, int T_max, int D) {
   if (D != 64 && D != 128) return false;
   if (H / H_kv > kDecodeMaxGroup) return false;
   if ((int64_t)B * H_kv > 65535) return false;  // grid y
+  if ((T_max + kDecodeChunk - 1) / kDecodeChunk > 8192) return false;  // combine weights in shared memory
   return (int64_t)B * H_kv * T_max * D < ((int64_t)1 << 40);
 }
 
@@ -539,14 +541,25 @@ int decode_launch(const void* q, const void* k, const void* v, const int32_t* le
   float* mp = (float*)(ws + dp.m_part);
   float* lp = (float*)(ws + dp.l_part);
   const int G = H / H_kv;
-  ATTN_LAUNCH(KK_DECODE, st,
-              decode_split_kernel<TIO, D><<<dim3(dp.n_split, B * H_kv), kDecodeThreads,
-                                            L::bytes(G), st>>>(
-                  (const TIO*)q, (const TIO*)k, (const TIO*)v, lens, rc, rs, op, mp, lp, H, H_kv,
-                  T_max, dp.n_split, dp.per_split, scale * 1.4426950408889634f));
+  if (std::is_same<TIO, __nv_bfloat16>::value && G <= 16) {
+    // tensor-core variant (up to 16 query heads per cached head)
+    ATTN_LAUNCH(KK_DECODE, st,
+                decode_mma_kernel<D><<<dim3(dp.n_split, B * H_kv), kDecodeMmaThreads,
+                                       DecodeMmaLayout<D>::kBytes, st>>>(
+                    (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+                    lens, rc, rs, op, mp, lp, H, H_kv, T_max, dp.n_split,
+                    scale * 1.4426950408889634f));
+  } else {
+    ATTN_LAUNCH(KK_DECODE, st,
+                decode_split_kernel<TIO, D><<<dim3(dp.n_split, B * H_kv), kDecodeThreads,
+                                              L::bytes(G), st>>>(
+                    (const TIO*)q, (const TIO*)k, (const TIO*)v, lens, rc, rs, op, mp, lp, H,
+                    H_kv, T_max, dp.n_split, dp.per_split, scale * 1.4426950408889634f));
+  }
   if (launch_status()) return ATTN_ECUDA;
   ATTN_LAUNCH(KK_DECODE_COMBINE, st,
-              decode_combine_kernel<TIO, D><<<B * H, D, 0, st>>>(
+              decode_combine_kernel<TIO, D><<<B * H, kDecodeCombineThreads,
+                                              dp.n_split * sizeof(float), st>>>(
                   op, mp, lp, lens, (TIO*)o, lse, H, T_max, dp.n_split, dp.per_split));
   return launch_status();
 }

@@ -234,30 +234,295 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core variant (bf16 cache, G <= 16): warp-level mma.sync with the G
+// query heads as the rows of a 16-row tile (zero rows past G). Same chunking,
+// same partial format. Scores S[16 x 64] = (Q_hi + Q_lo) K^T: the scaled,
+// rotated fp32 query is split into two bf16 parts (hi = bf16(q), lo =
+// bf16(q - hi)), so the scores keep ~16 more bits than a single bf16 query
+// (the lse bound needs them); K fragments come straight from the padded K
+// rows. Each of the 4 warps scores 16 keys (two n8 tiles over D/16 k-steps),
+// the row max and sum are combined across warps through shared memory, P is
+// written as bf16 [16][64] and O[16 x D] = P V is formed with each warp
+// taking D/4 columns (V fragments by transposing loads).
+// ---------------------------------------------------------------------------
+constexpr int kDecodeMmaThreads = 128;
+
+template <int D>
+struct DecodeMmaLayout {
+  static constexpr int kRowBytes = D * 2 + 16;   // padded bf16 rows (K, V, Q)
+  static constexpr int kPRowBytes = kDecodeChunk * 2 + 16;
+  static constexpr int kK = 0;
+  static constexpr int kV = kDecodeChunk * kRowBytes;
+  static constexpr int kQhi = 2 * kDecodeChunk * kRowBytes;
+  static constexpr int kQlo = kQhi + 16 * kRowBytes;
+  static constexpr int kP = kQlo + 16 * kRowBytes;
+  static constexpr int kRed = kP + 16 * kPRowBytes;    // f32 [2][4 warps][16]
+  static constexpr int kBytes = kRed + 2 * 4 * 16 * 4;
+};
+static_assert(DecodeMmaLayout<128>::kP % 16 == 0 && DecodeMmaLayout<64>::kRed % 16 == 0,
+              "ldmatrix rows need 16-byte alignment");
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+// D[16x8] += A[16x16] B[16x8], bf16 inputs, fp32 accumulators
+__device__ __forceinline__ void mma_bf16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecodeMmaThreads) decode_mma_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_cache,
+    const __nv_bfloat16* __restrict__ v_cache, const int32_t* __restrict__ cache_lens,
+    const float* __restrict__ rc, const float* __restrict__ rs, float* __restrict__ o_part,
+    float* __restrict__ m_part, float* __restrict__ l_part, int H, int Hkv, int T_max,
+    int n_split, float scale_log2) {
+  using L = DecodeMmaLayout<D>;
+  constexpr int C = kDecodeChunk;
+  constexpr int NT = D / 32;  // n8 tiles of the weighted sum per warp
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int G = H / Hkv;
+  const int bhk = blockIdx.y, b = bhk / Hkv, hk = bhk - b * Hkv;
+  const int split = blockIdx.x;
+  int len = cache_lens[b];
+  if (len < 1 || len > T_max) {
+    if (threadIdx.x == 0 && split == 0 && hk == 0) report_status(ATTN_EDEVICE_INPUT);
+    len = len < 1 ? 1 : T_max;
+  }
+  const int j0 = split * C;
+  if (j0 >= len) return;  // uniform: this chunk is past the cache
+  const int nk = min(C, len - j0);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sb = (uint32_t)__cvta_generic_to_shared(sm);
+
+  // K and V rows of the chunk (rows past the cache zero-filled)
+  {
+    const __nv_bfloat16* kb = k_cache + ((size_t)bhk * T_max + j0) * D;
+    const __nv_bfloat16* vb = v_cache + ((size_t)bhk * T_max + j0) * D;
+    for (int i = tid; i < C * D / 8; i += kDecodeMmaThreads) {
+      const int r = i / (D / 8), p = i - r * (D / 8);
+      const uint32_t nb = r < nk ? 16u : 0u;
+      const size_t src = (size_t)(r < nk ? r : 0) * D + p * 8;  // in bounds
+      cp_async16(sb + L::kK + r * L::kRowBytes + p * 16, kb + src, nb);
+      cp_async16(sb + L::kV + r * L::kRowBytes + p * 16, vb + src, nb);
+    }
+  }
+  // the queries: rotated to position len-1, scaled by scale*log2(e), split
+  // into bf16 hi + lo; rows G..15 zero
+  for (int i = tid; i < 16 * (D / 2); i += kDecodeMmaThreads) {
+    const int g = i / (D / 2), pi = i - g * (D / 2);
+    float x[2] = {0.f, 0.f};
+    if (g < G) {
+      load_vec<2>(q + ((size_t)b * H + hk * G + g) * D + 2 * pi, x);
+      if (rc) rope_pairs<2, D>(x, rc, rs, len - 1, 2 * pi, false);
+      x[0] *= scale_log2;
+      x[1] *= scale_log2;
+    }
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(x[0], x[1]);
+    const __nv_bfloat162 lo =
+        __floats2bfloat162_rn(x[0] - __low2float(hi), x[1] - __high2float(hi));
+    *reinterpret_cast<__nv_bfloat162*>(sm + L::kQhi + g * L::kRowBytes + pi * 4) = hi;
+    *reinterpret_cast<__nv_bfloat162*>(sm + L::kQlo + g * L::kRowBytes + pi * 4) = lo;
+  }
+  cp_async_wait_all();
+  __syncthreads();
+
+  // scores of this warp's 16 keys: two n8 tiles, D/16 k-steps, hi and lo
+  float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  {
+    const int arow = lane & 15, acol = (lane >> 4) * 8;        // x4 A addressing
+    const int brow = lane & 7, bcol = ((lane >> 3) & 1) * 8;    // x2 B addressing
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+      ldsm_x4(sb + L::kQhi + arow * L::kRowBytes + (ks * 16 + acol) * 2, h0, h1, h2, h3);
+      ldsm_x4(sb + L::kQlo + arow * L::kRowBytes + (ks * 16 + acol) * 2, l0, l1, l2, l3);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        uint32_t b0, b1;
+        const int key = warp * 16 + t * 8 + brow;
+        ldsm_x2(sb + L::kK + key * L::kRowBytes + (ks * 16 + bcol) * 2, b0, b1);
+        mma_bf16_16816(sc[t], h0, h1, h2, h3, b0, b1);
+        mma_bf16_16816(sc[t], l0, l1, l2, l3, b0, b1);
+      }
+    }
+  }
+  // fragment: sc[t][0..1] row lane/4, keys warp*16 + 8t + 2(lane%4) + {0,1};
+  // sc[t][2..3] row lane/4 + 8, same keys
+  const int r0 = lane >> 2, r1 = r0 + 8;
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int key = warp * 16 + t * 8 + 2 * (lane & 3) + (e & 1);
+      if (key >= nk) sc[t][e] = -INFINITY;
+    }
+  float* red = reinterpret_cast<float*>(sm + L::kRed);  // [2][4][16]
+  float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+  float mx1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
+#pragma unroll
+  for (int o = 1; o <= 2; o <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+  }
+  if ((lane & 3) == 0) {
+    red[warp * 16 + r0] = mx0;
+    red[warp * 16 + r1] = mx1;
+  }
+  __syncthreads();
+  const float m0 = fmaxf(fmaxf(red[r0], red[16 + r0]), fmaxf(red[32 + r0], red[48 + r0]));
+  const float m1 = fmaxf(fmaxf(red[r1], red[16 + r1]), fmaxf(red[32 + r1], red[48 + r1]));
+  float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    sc[t][0] = exp2f(sc[t][0] - m0);  // masked keys: exp2(-inf) = 0
+    sc[t][1] = exp2f(sc[t][1] - m0);
+    sc[t][2] = exp2f(sc[t][2] - m1);
+    sc[t][3] = exp2f(sc[t][3] - m1);
+    ls0 += sc[t][0] + sc[t][1];
+    ls1 += sc[t][2] + sc[t][3];
+    // P as bf16 [16 rows][64 keys]
+    const int key = warp * 16 + t * 8 + 2 * (lane & 3);
+    *reinterpret_cast<__nv_bfloat162*>(sm + L::kP + r0 * L::kPRowBytes + key * 2) =
+        __floats2bfloat162_rn(sc[t][0], sc[t][1]);
+    *reinterpret_cast<__nv_bfloat162*>(sm + L::kP + r1 * L::kPRowBytes + key * 2) =
+        __floats2bfloat162_rn(sc[t][2], sc[t][3]);
+  }
+#pragma unroll
+  for (int o = 1; o <= 2; o <<= 1) {
+    ls0 += __shfl_xor_sync(0xffffffffu, ls0, o);
+    ls1 += __shfl_xor_sync(0xffffffffu, ls1, o);
+  }
+  if ((lane & 3) == 0) {
+    red[64 + warp * 16 + r0] = ls0;
+    red[64 + warp * 16 + r1] = ls1;
+  }
+  __syncthreads();
+
+  // O[16 x D] = P V: warp w takes columns [w*D/4, (w+1)*D/4), NT n8 tiles
+  float oc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) oc[t][0] = oc[t][1] = oc[t][2] = oc[t][3] = 0.f;
+  {
+    const int arow = lane & 15, acol = (lane >> 4) * 8;
+    const int vrow = lane & 15;  // x2.trans: lanes 0-7 keys 0-7, lanes 8-15 keys 8-15
+#pragma unroll
+    for (int ks = 0; ks < C / 16; ++ks) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(sb + L::kP + arow * L::kPRowBytes + (ks * 16 + acol) * 2, a0, a1, a2, a3);
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        uint32_t b0, b1;
+        const int col = warp * (D / 4) + t * 8;
+        ldsm_x2_trans(sb + L::kV + (ks * 16 + vrow) * L::kRowBytes + col * 2, b0, b1);
+        mma_bf16_16816(oc[t], a0, a1, a2, a3, b0, b1);
+      }
+    }
+  }
+  // store rows < G: o (unnormalised), max (log2 units), sum
+  const float l0 = red[64 + r0] + red[80 + r0] + red[96 + r0] + red[112 + r0];
+  const float l1 = red[64 + r1] + red[80 + r1] + red[96 + r1] + red[112 + r1];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int col = warp * (D / 4) + t * 8 + 2 * (lane & 3);
+    if (r0 < G) {
+      const size_t slot = ((size_t)b * H + hk * G + r0) * n_split + split;
+      *reinterpret_cast<float2*>(o_part + slot * D + col) = make_float2(oc[t][0], oc[t][1]);
+    }
+    if (r1 < G) {
+      const size_t slot = ((size_t)b * H + hk * G + r1) * n_split + split;
+      *reinterpret_cast<float2*>(o_part + slot * D + col) = make_float2(oc[t][2], oc[t][3]);
+    }
+  }
+  if (warp == 0 && (lane & 3) == 0) {
+    if (r0 < G) {
+      const size_t slot = ((size_t)b * H + hk * G + r0) * n_split + split;
+      m_part[slot] = m0;
+      l_part[slot] = l0;
+    }
+    if (r1 < G) {
+      const size_t slot = ((size_t)b * H + hk * G + r1) * n_split + split;
+      m_part[slot] = m1;
+      l_part[slot] = l1;
+    }
+  }
+}
+
 // Merge the chunk partials of one (b, h): M = max m_s, l = sum l_s 2^(m_s-M),
-// o = sum o_s 2^(m_s-M) / l, lse = (M + log2 l) ln 2. One block of D threads
-// per query head.
+// o = sum o_s 2^(m_s-M) / l, lse = (M + log2 l) ln 2. One block of
+// kDecodeCombineThreads threads per query head: the chunks are spread over
+// the threads (block reductions through shared memory), then each of the
+// kDecodeCombineThreads / D thread groups sums a share of the chunks for
+// every column. Dynamic shared memory: n_split weights.
+constexpr int kDecodeCombineThreads = 256;
+
 template <typename TIO, int D>
-__global__ void __launch_bounds__(D) decode_combine_kernel(
+__global__ void __launch_bounds__(kDecodeCombineThreads) decode_combine_kernel(
     const float* __restrict__ o_part, const float* __restrict__ m_part,
     const float* __restrict__ l_part, const int32_t* __restrict__ cache_lens, TIO* __restrict__ o,
     float* __restrict__ lse, int H, int T_max, int n_split, int per_split) {
-  const int bh = blockIdx.x, d = threadIdx.x;
+  constexpr int NT = kDecodeCombineThreads, NG = NT / D;
+  extern __shared__ float wsh[];  // [n_split]
+  __shared__ float red[NT / 32];
+  __shared__ float part[NG][D];
+  const int bh = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int len = cache_lens[bh / H];
   len = len < 1 ? 1 : (len > T_max ? T_max : len);
   const int ns = (len + per_split - 1) / per_split;
   const size_t base = (size_t)bh * n_split;
-  // eight independent loads in flight per thread in both passes
+  // M
   float M = -INFINITY;
-#pragma unroll 8
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, m_part[base + s]);
-  float l = 0.f, acc = 0.f;
-#pragma unroll 8
-  for (int s = 0; s < ns; ++s) {
+  for (int s = tid; s < ns; s += NT) M = fmaxf(M, m_part[base + s]);
+  M = warp_max(M);
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  M = red[0];
+#pragma unroll
+  for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, red[w]);
+  __syncthreads();
+  // weights and l
+  float l = 0.f;
+  for (int s = tid; s < ns; s += NT) {
     const float w = exp2f(m_part[base + s] - M);
+    wsh[s] = w;
     l = fmaf(l_part[base + s], w, l);
-    acc = fmaf(o_part[(base + s) * D + d], w, acc);
   }
-  o[(size_t)bh * D + d] = from_f32<TIO>(acc / l);
-  if (d == 0) lse[bh] = (M + log2f(l)) * 0.69314718055994531f;
+  l = warp_sum(l);
+  if (lane == 0) red[warp] = l;
+  __syncthreads();
+  l = 0.f;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) l += red[w];
+  // o: group gi of the threads sums chunks gi, gi + NG, ... for column d
+  const int d = tid % D, gi = tid / D;
+  float acc = 0.f;
+#pragma unroll 4
+  for (int s = gi; s < ns; s += NG) acc = fmaf(o_part[(base + s) * D + d], wsh[s], acc);
+  part[gi][d] = acc;
+  __syncthreads();
+  if (gi == 0) {
+#pragma unroll
+    for (int g = 1; g < NG; ++g) acc += part[g][d];
+    o[(size_t)bh * D + d] = from_f32<TIO>(acc / l);
+    if (d == 0) lse[bh] = (M + log2f(l)) * 0.69314718055994531f;
+  }
 }

@@ -1,6 +1,6 @@
 """GPU parity for decode attention (one new token against a key/value cache)
 through the C ABI, against the float64 decode oracle: small cases element by
-element (both storage types and head sizes, group sizes 1 to 8, cache
+element (both storage types and head sizes, group sizes 1 to 32, cache
 lengths 1, ragged, a multiple of the 128-token chunk and the full capacity),
 the two named decode workloads on sampled heads, cache rows past the length
 never read, and out-of-range lengths reported and clamped."""
@@ -54,6 +54,8 @@ SMALL = [
     ("decode_8k_gqa", dict(B=2, H=4, H_kv=4, T_max=257, len_min=1, seed=35, rope=False)),
     ("decode_8k_gqa", dict(B=2, H=16, H_kv=2, T_max=384, len_min=100, seed=36, dtype="f32")),
     ("decode_237m", dict(B=2, H=2, H_kv=1, T_max=200, len_min=1, seed=37, dtype="f32")),
+    # 32 query heads per cached head: bf16 beyond the tensor-core variant's 16 rows
+    ("decode_8k_gqa", dict(B=2, H=32, H_kv=1, T_max=300, len_min=1, seed=41)),
 ]
 
 
