@@ -507,11 +507,26 @@ struct DecodePlan {
   int n_split = 0, per_split = 0;
 };
 
-DecodePlan decode_plan(int B, int H, int H_kv, int T_max, int D) {
+// bf16 caches with up to 16 query heads per cached head take the streaming
+// tensor-core kernel (cache ranges sized for about sixteen CTAs per SM over
+// the whole grid, measured best with a two-deep pipeline); the rest
+// take one 64-token chunk per CTA.
+bool decode_streams(int H, int H_kv, int dtype) { return dtype == ATTN_BF16 && H / H_kv <= 16; }
+constexpr long kDecodeStreamCtas = 16 * 148;
+
+DecodePlan decode_plan(int B, int H, int H_kv, int T_max, int D, int dtype) {
   DecodePlan p;
-  (void)H_kv;
-  p.per_split = kDecodeChunk;
-  p.n_split = (T_max + kDecodeChunk - 1) / kDecodeChunk;
+  if (decode_streams(H, H_kv, dtype)) {
+    const long stages = (T_max + kDecodePipeKeys - 1) / kDecodePipeKeys;
+    long want = (kDecodeStreamCtas + (long)B * H_kv - 1) / ((long)B * H_kv);
+    want = want < 1 ? 1 : (want > stages ? stages : want);
+    const long per = (stages + want - 1) / want;  // stages per range
+    p.per_split = (int)(per * kDecodePipeKeys);
+    p.n_split = (int)((stages + per - 1) / per);
+  } else {
+    p.per_split = kDecodeChunk;
+    p.n_split = (T_max + kDecodeChunk - 1) / kDecodeChunk;
+  }
   const size_t slots = (size_t)B * H * p.n_split;
   p.o_part = 0;
   p.m_part = round_up(slots * D * sizeof(float));
@@ -542,12 +557,15 @@ int decode_launch(const void* q, const void* k, const void* v, const int32_t* le
   float* lp = (float*)(ws + dp.l_part);
   const int G = H / H_kv;
   if (std::is_same<TIO, __nv_bfloat16>::value && G <= 16) {
-    // tensor-core variant (up to 16 query heads per cached head)
+    // streaming tensor-core variant (up to 16 query heads per cached head)
+    static bool pipe_smem_set[64] = {};
+    if (!ensure_smem(decode_pipe_kernel<D>, DecodePipeLayout<D>::kBytes, pipe_smem_set))
+      return ATTN_ECUDA;
     ATTN_LAUNCH(KK_DECODE, st,
-                decode_mma_kernel<D><<<dim3(dp.n_split, B * H_kv), kDecodeMmaThreads,
-                                       DecodeMmaLayout<D>::kBytes, st>>>(
+                decode_pipe_kernel<D><<<dim3(dp.n_split, B * H_kv), kDecodeMmaThreads,
+                                        DecodePipeLayout<D>::kBytes, st>>>(
                     (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-                    lens, rc, rs, op, mp, lp, H, H_kv, T_max, dp.n_split,
+                    lens, rc, rs, op, mp, lp, H, H_kv, T_max, dp.n_split, dp.per_split,
                     scale * 1.4426950408889634f));
   } else {
     ATTN_LAUNCH(KK_DECODE, st,
@@ -570,7 +588,7 @@ extern "C" size_t attn_decode_workspace_bytes(int B, int H, int H_kv, int T_max,
                                               int dtype) {
   if (!decode_sizes_ok(B, H, H_kv, T_max, D) || (dtype != ATTN_BF16 && dtype != ATTN_F32))
     return 0;
-  return decode_plan(B, H, H_kv, T_max, D).total;
+  return decode_plan(B, H, H_kv, T_max, D, dtype).total;
 }
 
 extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cache,
@@ -588,7 +606,7 @@ extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cac
       !aligned(lse, 4) || !aligned(cache_lens, 4) || (rope_cos && !aligned(rope_cos, 16)) ||
       (rope_sin && !aligned(rope_sin, 16)))
     return ATTN_EALIGN;
-  const DecodePlan dp = decode_plan(B, H, H_kv, T_max, D);
+  const DecodePlan dp = decode_plan(B, H, H_kv, T_max, D, dtype);
   if (!workspace) return ATTN_EWORKSPACE;
   if (!aligned(workspace, 16)) return ATTN_EALIGN;
   if (ws_bytes < dp.total) return ATTN_EWORKSPACE;
