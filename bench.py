@@ -335,7 +335,6 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize(dev)
     n0 = A.attn_launch_count()
-    A.check(A.attn_profile_enable(1), "attn_profile_enable")
     with ClockSampler(local) as clocks:
         with torch.cuda.stream(stream):
             for i in range(args.steps):
@@ -347,10 +346,20 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
     barrier()
     torch.cuda.synchronize(dev)
-    A.attn_profile_enable(0)
     launches = A.attn_launch_count() - n0
-    prof = A.profile_summary()
     step_ms = [a.elapsed_time(b) for a, b in ev]
+    # Per-kernel times for the roofline come from a second pass over the same
+    # number of steps with an event pair around every launch (kept out of the
+    # timed steps above: events between launches would stop them overlapping).
+    A.check(A.attn_profile_enable(1), "attn_profile_enable")
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.zero_()
+            r.forward()
+            r.backward()
+    torch.cuda.synchronize(dev)
+    A.attn_profile_enable(0)
+    prof = A.profile_summary()
     ms_local = sum(step_ms) / len(step_ms)
     ms = max_over_ranks(ms_local)
     value = flops_step * world / (ms / 1e3) / 1e12
@@ -482,7 +491,6 @@ def run_decode(args):
           for _ in range(args.steps)]
     torch.cuda.synchronize(dev)
     n0 = A.attn_launch_count()
-    A.check(A.attn_profile_enable(1), "attn_profile_enable")
     with ClockSampler(0) as clocks:
         with torch.cuda.stream(stream):
             for i in range(args.steps):
@@ -491,8 +499,15 @@ def run_decode(args):
                 r.run()
                 ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
-    A.attn_profile_enable(0)
     launches = A.attn_launch_count() - n0
+    # per-kernel times from a separate pass (events around every launch)
+    A.check(A.attn_profile_enable(1), "attn_profile_enable")
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.zero_()
+            r.run()
+    torch.cuda.synchronize(dev)
+    A.attn_profile_enable(0)
     prof = A.profile_summary()
     ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     nbytes = w.cache_bytes_read()

@@ -178,7 +178,9 @@ int check_common(const void* q, const void* k, const void* v, const float* rc, c
 }
 
 int launch_status() {
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+  const cudaError_t pe = pdl_launch_error();
+  pdl_launch_error() = cudaSuccess;
+  return (cudaGetLastError() == cudaSuccess && pe == cudaSuccess) ? ATTN_OK : ATTN_ECUDA;
 }
 
 template <typename TIO, int D>
@@ -186,8 +188,7 @@ int fwd_simt(const void* q, const void* k, const void* v, const float* rc, const
              const int32_t* ds, void* o, float* lse, int B, int H, int Hkv, int T, float scale,
              cudaStream_t st) {
   dim3 grid(B * H, (T + 15) / 16);
-  ATTN_LAUNCH(KK_FWD, st,
-              simt_fwd_kernel<TIO, D><<<grid, 128, 0, st>>>((const TIO*)q, (const TIO*)k,
+  ATTN_LAUNCH(KK_FWD, st, pdl_launch(simt_fwd_kernel<TIO, D>, grid, 128, 0, st, (const TIO*)q, (const TIO*)k,
                                                             (const TIO*)v, rc, rs, ds, (TIO*)o,
                                                             lse, H, Hkv, T, scale));
   return launch_status();
@@ -199,19 +200,13 @@ int bwd_simt(const void* q, const void* k, const void* v, const void* o, const v
              const int32_t* de, float* delta, void* dq, void* dk, void* dv, int B, int H, int Hkv,
              int T, float scale, cudaStream_t st) {
   const long rows = (long)B * H * T;
-  ATTN_LAUNCH(KK_DELTA, st,
-              delta_kernel<TIO, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
-                  (const TIO*)o, (const TIO*)dO, delta, rows));
+  ATTN_LAUNCH(KK_DELTA, st, pdl_launch(delta_kernel<TIO, D>, (unsigned)((rows + 7) / 8), 256, 0, st, (const TIO*)o, (const TIO*)dO, delta, rows));
   if (launch_status()) return ATTN_ECUDA;
   dim3 g1(B * Hkv, (T + 31) / 32), g2(B * H, (T + 31) / 32);
-  ATTN_LAUNCH(KK_DKDV, st,
-              simt_dkdv_kernel<TIO, D><<<g1, 128, 0, st>>>(
-                  (const TIO*)q, (const TIO*)k, (const TIO*)v, (const TIO*)dO, lse, delta, rc, rs,
+  ATTN_LAUNCH(KK_DKDV, st, pdl_launch(simt_dkdv_kernel<TIO, D>, g1, 128, 0, st, (const TIO*)q, (const TIO*)k, (const TIO*)v, (const TIO*)dO, lse, delta, rc, rs,
                   ds, de, (TIO*)dk, (TIO*)dv, H, Hkv, T, scale));
   if (launch_status()) return ATTN_ECUDA;
-  ATTN_LAUNCH(KK_DQ, st,
-              simt_dq_kernel<TIO, D><<<g2, 128, 0, st>>>(
-                  (const TIO*)q, (const TIO*)k, (const TIO*)v, (const TIO*)dO, lse, delta, rc, rs,
+  ATTN_LAUNCH(KK_DQ, st, pdl_launch(simt_dq_kernel<TIO, D>, g2, 128, 0, st, (const TIO*)q, (const TIO*)k, (const TIO*)v, (const TIO*)dO, lse, delta, rc, rs,
                   ds, (TIO*)dq, H, Hkv, T, scale));
   return launch_status();
 }
@@ -231,9 +226,7 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
     __half* kh = (__half*)(ws + wp.k16);
     qf = (float*)(ws + wp.qfac);
     kf = (float*)(ws + wp.kfac);
-    ATTN_LAUNCH(KK_ROPE_PREP, st,
-                rope_prep_kernel<__half, D, true><<<dim3(nt, BH, 2), kRopePrepThreads, 0, st>>>(
-                    (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qh, kh, qf, kf,
+    ATTN_LAUNCH(KK_ROPE_PREP, st, pdl_launch(rope_prep_kernel<__half, D, true>, dim3(nt, BH, 2), kRopePrepThreads, 0, st, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qh, kh, qf, kf,
                     H, Hkv, T, nt));
     if (launch_status()) return ATTN_ECUDA;
     qs = qh;
@@ -261,9 +254,7 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
   prm.doc_start = ds;
   prm.o = (__nv_bfloat16*)o;
   prm.lse = lse;
-  ATTN_LAUNCH(KK_FWD, st,
-              fwd100::fwd_kernel<D><<<(unsigned)(n_pairs * BH), L::kThreads, L::kSmemAlloc, st>>>(
-                  mq, mk, mv, prm));
+  ATTN_LAUNCH(KK_FWD, st, pdl_launch(fwd100::fwd_kernel<D>, (unsigned)(n_pairs * BH), L::kThreads, L::kSmemAlloc, st, mq, mk, mv, prm));
   return launch_status();
 }
 
@@ -285,9 +276,7 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   const int split = wp.split;
   float* dk_acc = split > 1 ? (float*)(ws + wp.dk_acc) : nullptr;
   float* dv_acc = split > 1 ? (float*)(ws + wp.dv_acc) : nullptr;
-  ATTN_LAUNCH(KK_DELTA, st,
-              bwd_prep_kernel<D><<<(unsigned)(rows_pad * (D / 8) / 256), 256, 0, st>>>(
-                  (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse, delta, lse2, dq_acc,
+  ATTN_LAUNCH(KK_DELTA, st, pdl_launch(bwd_prep_kernel<D>, (unsigned)(rows_pad * (D / 8) / 256), 256, 0, st, (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse, delta, lse2, dq_acc,
                   (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qr, kr, dk_acc,
                   dv_acc, H, Hkv, T, Tpad, rows_pad));
   if (launch_status()) return ATTN_ECUDA;
@@ -319,26 +308,19 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   prm.dv = (__nv_bfloat16*)dv;
   prm.dk_acc = dk_acc;
   prm.dv_acc = dv_acc;
-  ATTN_LAUNCH(KK_DKDV, st,
-              bwd100::dkdv_kernel<D><<<(unsigned)(nt * BHkv * split), L::kThreads, L::kSmemAlloc,
-                                       st>>>(mq, mk, mv, mo, mdq, prm));
+  ATTN_LAUNCH(KK_DKDV, st, pdl_launch(bwd100::dkdv_kernel<D>, (unsigned)(nt * BHkv * split), L::kThreads, L::kSmemAlloc,
+                                       st, mq, mk, mv, mo, mdq, prm));
   if (launch_status()) return ATTN_ECUDA;
   if (split > 1) {
     // dk = R^T (scale * sum of the parts), dv = sum of the parts
     const long n8kv = (long)BHkv * T * D / 8;
-    ATTN_LAUNCH(KK_DQ_FINALIZE, st,
-                dq_finalize_kernel<D><<<(unsigned)((n8kv + 255) / 256), 256, 0, st>>>(
-                    dk_acc, rc, rs, ds, (__nv_bfloat16*)dk, Hkv, T, scale, n8kv));
+    ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)((n8kv + 255) / 256), 256, 0, st, dk_acc, rc, rs, ds, (__nv_bfloat16*)dk, Hkv, T, scale, n8kv));
     if (launch_status()) return ATTN_ECUDA;
-    ATTN_LAUNCH(KK_DQ_FINALIZE, st,
-                dq_finalize_kernel<D><<<(unsigned)((n8kv + 255) / 256), 256, 0, st>>>(
-                    dv_acc, nullptr, nullptr, nullptr, (__nv_bfloat16*)dv, Hkv, T, 1.0f, n8kv));
+    ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)((n8kv + 255) / 256), 256, 0, st, dv_acc, nullptr, nullptr, nullptr, (__nv_bfloat16*)dv, Hkv, T, 1.0f, n8kv));
     if (launch_status()) return ATTN_ECUDA;
   }
   const long n8 = (long)BH * T * D / 8;
-  ATTN_LAUNCH(KK_DQ_FINALIZE, st,
-              dq_finalize_kernel<D><<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
-                  dq_acc, rc, rs, ds, (__nv_bfloat16*)dq, H, T, scale, n8));
+  ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)((n8 + 255) / 256), 256, 0, st, dq_acc, rc, rs, ds, (__nv_bfloat16*)dq, H, T, scale, n8));
   return launch_status();
 }
 
@@ -377,8 +359,7 @@ int attn_fwd_gqa(const void* q, const void* k, const void* v, const float* rope_
   int32_t* ds = nullptr;
   if (cu_seqlens) {
     ds = (int32_t*)(ws + p.doc_start);
-    ATTN_LAUNCH(KK_DOC_RANGES, st,
-                doc_ranges_kernel<<<1, 1024, 0, st>>>(cu_seqlens, B, T, ds,
+    ATTN_LAUNCH(KK_DOC_RANGES, st, pdl_launch(doc_ranges_kernel, 1, 1024, 0, st, cu_seqlens, B, T, ds,
                                                       (int32_t*)(ws + p.doc_end)));
     if (launch_status()) return ATTN_ECUDA;
   }
@@ -421,7 +402,7 @@ int attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, con
   if (cu_seqlens) {
     ds = (int32_t*)(ws + p.doc_start);
     de = (int32_t*)(ws + p.doc_end);
-    ATTN_LAUNCH(KK_DOC_RANGES, st, doc_ranges_kernel<<<1, 1024, 0, st>>>(cu_seqlens, B, T, ds, de));
+    ATTN_LAUNCH(KK_DOC_RANGES, st, pdl_launch(doc_ranges_kernel, 1, 1024, 0, st, cu_seqlens, B, T, ds, de));
     if (launch_status()) return ATTN_ECUDA;
   }
   float* delta = (float*)(ws + p.delta);
@@ -561,24 +542,18 @@ int decode_launch(const void* q, const void* k, const void* v, const int32_t* le
     static bool pipe_smem_set[64] = {};
     if (!ensure_smem(decode_pipe_kernel<D>, DecodePipeLayout<D>::kBytes, pipe_smem_set))
       return ATTN_ECUDA;
-    ATTN_LAUNCH(KK_DECODE, st,
-                decode_pipe_kernel<D><<<dim3(dp.n_split, B * H_kv), kDecodeMmaThreads,
-                                        DecodePipeLayout<D>::kBytes, st>>>(
-                    (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+    ATTN_LAUNCH(KK_DECODE, st, pdl_launch(decode_pipe_kernel<D>, dim3(dp.n_split, B * H_kv), kDecodeMmaThreads,
+                                        DecodePipeLayout<D>::kBytes, st, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
                     lens, rc, rs, op, mp, lp, H, H_kv, T_max, dp.n_split, dp.per_split,
                     scale * 1.4426950408889634f));
   } else {
-    ATTN_LAUNCH(KK_DECODE, st,
-                decode_split_kernel<TIO, D><<<dim3(dp.n_split, B * H_kv), kDecodeThreads,
-                                              L::bytes(G), st>>>(
-                    (const TIO*)q, (const TIO*)k, (const TIO*)v, lens, rc, rs, op, mp, lp, H,
+    ATTN_LAUNCH(KK_DECODE, st, pdl_launch(decode_split_kernel<TIO, D>, dim3(dp.n_split, B * H_kv), kDecodeThreads,
+                                              L::bytes(G), st, (const TIO*)q, (const TIO*)k, (const TIO*)v, lens, rc, rs, op, mp, lp, H,
                     H_kv, T_max, dp.n_split, dp.per_split, scale * 1.4426950408889634f));
   }
   if (launch_status()) return ATTN_ECUDA;
-  ATTN_LAUNCH(KK_DECODE_COMBINE, st,
-              decode_combine_kernel<TIO, D><<<B * H, kDecodeCombineThreads,
-                                              dp.n_split * sizeof(float), st>>>(
-                  op, mp, lp, lens, (TIO*)o, lse, H, T_max, dp.n_split, dp.per_split));
+  ATTN_LAUNCH(KK_DECODE_COMBINE, st, pdl_launch(decode_combine_kernel<TIO, D>, B * H, kDecodeCombineThreads,
+                                              dp.n_split * sizeof(float), st, op, mp, lp, lens, (TIO*)o, lse, H, T_max, dp.n_split, dp.per_split));
   return launch_status();
 }
 
@@ -704,7 +679,7 @@ extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, con
     // doc_ranges_kernel writes every entry of both arrays.
     ds = (int32_t*)(ws + p.doc_start);
     de = (int32_t*)(ws + p.doc_end);
-    ATTN_LAUNCH(KK_DOC_RANGES, st, doc_ranges_kernel<<<1, 1024, 0, st>>>(cu_seqlens, B, T, ds, de));
+    ATTN_LAUNCH(KK_DOC_RANGES, st, pdl_launch(doc_ranges_kernel, 1, 1024, 0, st, cu_seqlens, B, T, ds, de));
     if (launch_status()) return ATTN_ECUDA;
   }
   // delta_kernel writes every row of Delta before the two passes read it.

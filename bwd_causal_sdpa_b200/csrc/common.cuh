@@ -21,6 +21,17 @@ __device__ __forceinline__ void report_status(int code) {
   atomicCAS(&g_attn_status, 0, code);
 }
 
+// Programmatic dependent launch. Every kernel of this library runs this first:
+// wait until the kernel before it in the stream has completed and its memory
+// operations are visible (a no-op when launched without the attribute), so no
+// global access of this kernel, read or write, can overlap its predecessor;
+// then let the next kernel be scheduled (it will wait the same way), which
+// hides launch latency behind this kernel's tail.
+__device__ __forceinline__ void pdl_wait_and_trigger() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- storage type conversions ---------------------------------------------
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }

@@ -78,6 +78,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(
     const float* __restrict__ rs, float* __restrict__ o_part, float* __restrict__ m_part,
     float* __restrict__ l_part, int H, int Hkv, int T_max, int n_split, int per_split,
     float scale_log2) {
+  pdl_wait_and_trigger();
   using L = DecodeLayout<TIO, D>;
   constexpr int C = kDecodeChunk;
   constexpr int VEC = 16 / (int)sizeof(TIO);  // elements per 16-byte piece
@@ -313,6 +314,7 @@ __global__ void __launch_bounds__(kDecodeMmaThreads) decode_pipe_kernel(
     const float* __restrict__ rc, const float* __restrict__ rs, float* __restrict__ o_part,
     float* __restrict__ m_part, float* __restrict__ l_part, int H, int Hkv, int T_max,
     int n_split, int per_split, float scale_log2) {
+  pdl_wait_and_trigger();
   using L = DecodePipeLayout<D>;
   constexpr int C = kDecodePipeKeys;
   constexpr int NS = kDecodePipeStages;
@@ -517,6 +519,7 @@ __global__ void __launch_bounds__(kDecodeCombineThreads) decode_combine_kernel(
     const float* __restrict__ o_part, const float* __restrict__ m_part,
     const float* __restrict__ l_part, const int32_t* __restrict__ cache_lens, TIO* __restrict__ o,
     float* __restrict__ lse, int H, int T_max, int n_split, int per_split) {
+  pdl_wait_and_trigger();
   constexpr int NT = kDecodeCombineThreads, NG = NT / D;
   extern __shared__ float wsh[];  // [n_split]
   __shared__ float red[NT / 32];

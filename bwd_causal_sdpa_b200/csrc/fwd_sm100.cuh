@@ -82,6 +82,7 @@ template <int D>
 __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const Params p) {
+  pdl_wait_and_trigger();
   using L = Layout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sb0 = smem_u32(smem_raw);

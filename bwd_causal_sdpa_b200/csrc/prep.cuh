@@ -17,6 +17,7 @@
 __global__ void __launch_bounds__(1024) doc_ranges_kernel(const int32_t* __restrict__ cu, int B, int T,
                                                           int32_t* __restrict__ doc_start,
                                                           int32_t* __restrict__ doc_end) {
+  pdl_wait_and_trigger();
   __shared__ int s_ok, s_n;
   const int BT = B * T;
   if (threadIdx.x == 0) {
@@ -62,6 +63,7 @@ __global__ void __launch_bounds__(1024) doc_ranges_kernel(const int32_t* __restr
 template <typename TIO, int D>
 __global__ void __launch_bounds__(256) delta_kernel(const TIO* __restrict__ o, const TIO* __restrict__ dO,
                                                    float* __restrict__ delta, long rows) {
+  pdl_wait_and_trigger();
   constexpr int NC = D / 32;
   const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -96,6 +98,7 @@ __global__ void __launch_bounds__(kRopePrepThreads) rope_prep_kernel(
     const float* __restrict__ rc, const float* __restrict__ rs,
     const int32_t* __restrict__ doc_start, OutT* __restrict__ qo, OutT* __restrict__ ko,
     float* __restrict__ qfac, float* __restrict__ kfac, int H, int Hkv, int T, int ntiles) {
+  pdl_wait_and_trigger();
   constexpr int CH = D / 8;              // 16-byte chunks per row
   constexpr int NT = kRopePrepThreads;
   constexpr int PER = 128 * CH / NT;     // chunks per thread
@@ -197,6 +200,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
     const float* __restrict__ rs, const int32_t* __restrict__ doc_start,
     __nv_bfloat16* __restrict__ qr, __nv_bfloat16* __restrict__ kr, float* __restrict__ dk_acc,
     float* __restrict__ dv_acc, int H, int Hkv, int T, int Tpad, long rows_pad) {
+  pdl_wait_and_trigger();
   constexpr int TPR = D / 8;  // threads per row
   const long gt = (long)blockIdx.x * blockDim.x + threadIdx.x;
   const long row = gt / TPR;
@@ -252,6 +256,7 @@ __global__ void __launch_bounds__(256) dq_finalize_kernel(
     const float* __restrict__ dq_acc, const float* __restrict__ rc, const float* __restrict__ rs,
     const int32_t* __restrict__ doc_start, __nv_bfloat16* __restrict__ dq, int H, int T,
     float scale, long n8) {
+  pdl_wait_and_trigger();
   const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= n8) return;
   const long e0 = idx * 8;

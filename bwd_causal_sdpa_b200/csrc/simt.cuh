@@ -33,6 +33,7 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(
     const float* __restrict__ rc, const float* __restrict__ rs,
     const int32_t* __restrict__ doc_start, TIO* __restrict__ o, float* __restrict__ lse,
     int H, int Hkv, int T, float scale) {
+  pdl_wait_and_trigger();
   constexpr int ROWS = 16, KC = 32, NC = D / 32, KP = D + 4;
   __shared__ __align__(16) float sQ[ROWS][D];
   __shared__ __align__(16) float sK[KC][KP];
@@ -150,6 +151,7 @@ __global__ void __launch_bounds__(128) simt_dkdv_kernel(
     const float* __restrict__ rc, const float* __restrict__ rs,
     const int32_t* __restrict__ doc_start, const int32_t* __restrict__ doc_end,
     TIO* __restrict__ dk, TIO* __restrict__ dv, int H, int Hkv, int T, float scale) {
+  pdl_wait_and_trigger();
   constexpr int KC = 32, QC = 32, NC = D / 32, KW = 8;
   __shared__ __align__(16) float sQ[QC][D];
   __shared__ __align__(16) float sG[QC][D];
@@ -259,6 +261,7 @@ __global__ void __launch_bounds__(128) simt_dq_kernel(
     const float* __restrict__ rc, const float* __restrict__ rs,
     const int32_t* __restrict__ doc_start, TIO* __restrict__ dq, int H, int Hkv, int T,
     float scale) {
+  pdl_wait_and_trigger();
   constexpr int QC = 32, KC = 32, NC = D / 32, QW = 8;
   __shared__ __align__(16) float sK[KC][D];
   __shared__ __align__(16) float sV[KC][D];

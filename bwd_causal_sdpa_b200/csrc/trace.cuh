@@ -4,6 +4,7 @@
 
 #include <cuda_runtime.h>
 
+#include <utility>
 #include <vector>
 
 enum KernelKind : int {
@@ -95,7 +96,32 @@ inline int read(int kind, int* n, double* ms) {
 
 }  // namespace trace
 
-// Wrap one kernel launch: LAUNCH(kind, stream, kernel<<<grid, block, smem, stream>>>(...));
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while its predecessor in the stream is finishing (each kernel waits for its
+// predecessor's completion before touching memory, see pdl_wait_and_trigger).
+// A launch error is kept for launch_status().
+inline cudaError_t& pdl_launch_error() {
+  static cudaError_t e = cudaSuccess;
+  return e;
+}
+template <typename... KArgs, typename... Args>
+inline void pdl_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) pdl_launch_error() = e;
+}
+
+// Wrap one kernel launch: ATTN_LAUNCH(kind, stream, pdl_launch(kernel, grid, block, smem, stream, ...));
 #define ATTN_LAUNCH(kind, st, ...)            \
   do {                                        \
     const int _tr = trace::begin((kind), (st)); \
