@@ -41,10 +41,14 @@ FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # one ncu capture of the kernel on the workload, valid only while the kernel
 # sources still hash to what was captured (sha256, first 16 hex digits).
 MEASURED_TRAFFIC = {
-    ("dkdv", "long_context_8k"): (706.5e6, {"bwd_sm100.cuh": "a4e087a6ca38c64f",
-                                            "sm100.cuh": "1a2b026d7dc3ce22"}),
-    ("fwd", "long_context_8k"): (158.3e6, {"fwd_sm100.cuh": "2e9f5f7955c71a01",
-                                           "sm100.cuh": "1a2b026d7dc3ce22"}),
+    ("dkdv", "long_context_8k"): (699.8e6, {"bwd_sm100.cuh": "692670dd347a4156",
+                                            "sm100.cuh": "1a2b026d7dc3ce22",
+                                            "common.cuh": "10442a1674e61c67"}),
+    ("fwd", "long_context_8k"): (158.0e6, {"fwd_sm100.cuh": "dd2684a7407f7617",
+                                           "sm100.cuh": "1a2b026d7dc3ce22",
+                                           "common.cuh": "10442a1674e61c67"}),
+    ("decode", "decode_8k_gqa"): (201.9e6, {"decode.cuh": "a673449f05d438a0",
+                                            "common.cuh": "10442a1674e61c67"}),
 }
 
 
@@ -524,7 +528,8 @@ def run_decode(args):
                    "l2": "flushed between steps (256 MiB write outside the step events)"},
         "roofline": None if achieved is None else {
             "bound": "hbm", "kernel": "decode", "achieved": achieved, "peak": peaks["hbm_gbs"],
-            "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+            "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+            "traffic": measured_traffic("decode", w.cfg.name),
             "peak_source": f"hbm_gbs ({peak_src})"},
         "kernels": {k: {"launches": n, "avg_ms": t / n} for k, (n, t) in prof.items()},
         "gpu_launches": launches, "clocks": clocks.summary(),
