@@ -233,13 +233,34 @@ def sample_description(w, heads):
 # Arms
 # ---------------------------------------------------------------------------
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of every rank's value (the job's time is its slowest
+    rank's); one all-reduce on a one-element tensor on ``device`` (the GPU
+    under NCCL, the CPU under gloo)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank_step: float, world: int, ms: float) -> float:
+    """Weak scaling: every rank runs its own workload; the job's throughput is
+    all ranks' flops over the slowest rank's step time."""
+    return flops_per_rank_step * world / (ms / 1e3) / 1e12
+
+
 def dist_setup(n_gpus):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world != n_gpus:
-        if world == 1 and n_gpus > 1:
+        if world == 1:
             raise SystemExit("--gpus N > 1 needs torchrun with N processes")
+        raise SystemExit(f"--gpus {n_gpus} does not match the {world} launched processes")
     return world, rank, local
 
 
@@ -310,12 +331,6 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     cfg = config_by_name(args.workload)
     w = make_workload(cfg, H_kv=args.kv_heads)
@@ -365,8 +380,8 @@ def run_ours(args):
     A.attn_profile_enable(0)
     prof = A.profile_summary()
     ms_local = sum(step_ms) / len(step_ms)
-    ms = max_over_ranks(ms_local)
-    value = flops_step * world / (ms / 1e3) / 1e12
+    ms = max_over_ranks(ms_local, world, dev)
+    value = whole_job_tflops(flops_step, world, ms)
     st = r.status()
     if st != A.ATTN_OK:
         raise SystemExit(f"device status after timing: {A.error_string(st)}")
@@ -433,8 +448,8 @@ def run_ours(args):
                 e_ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev) / args.steps)
-        e2e = {"value": flops_step * world / (e_ms / 1e3) / 1e12, "unit": UNIT,
+        e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev) / args.steps, world, dev)
+        e2e = {"value": whole_job_tflops(flops_step, world, e_ms), "unit": UNIT,
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
         del td
 
