@@ -2,12 +2,15 @@
 //
 // One CTA computes two 128-row query tiles (A = rows [256t, 256t+128), B =
 // the next 128) of one (b, h) slice; both share every K and V tile it loads.
-//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread t owns
-//              query row t of its tile (= TMEM lane t), so the row max and row
-//              sum are thread-local (no shuffles);
-//   warp 8     TMA producer: both Q tiles once, then K and V tiles through a
+//   warps 0-15 softmax: warpgroup g takes tile g & 1 and key columns
+//              [64 (g >> 1), +64) of its S; thread t of a warpgroup owns query
+//              row t (= TMEM lane t), so each row is shared by two threads,
+//              which agree on the row's reference max through a small
+//              shared-memory exchange (double-buffered by key-tile parity,
+//              bounded mbarrier) and add their row sums at the end;
+//   warp 16    TMA producer: both Q tiles once, then K and V tiles through a
 //              ring of shared-memory stages;
-//   warp 9     TMEM owner and MMA issuer (one thread).
+//   warp 17    TMEM owner and MMA issuer (one thread).
 // TMEM (512 columns): per tile an S column block (P, bf16, is written back
 // over its first half) and an O accumulator. Per key tile j the MMA thread
 // issues PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the tensor pipe works on one
@@ -57,14 +60,20 @@ struct Layout {
   static constexpr int bPFull = bSFull + 2;         // [tile], 128 arrivals
   static constexpr int bPVDone = bPFull + 2;        // [tile]
   static constexpr int bOFinal = bPVDone + 2;       // [tile]
-  static constexpr int kNumBars = bOFinal + 2;
-  static constexpr int kMisc = kBars + kNumBars * 8;  // [0] TMEM base, [1] abort flag
+  static constexpr int bXch = bOFinal + 2;          // [tile], 256 arrivals: row maxima exchanged
+  static constexpr int kNumBars = bXch + 2;
+  // row-max exchange between the two halves of a row: f32 [2 parities][2 tiles][2 halves][128]
+  static constexpr int kXch = kBars + kNumBars * 8;
+  static constexpr int kMisc = (kXch + 2 * 2 * 2 * 128 * 4 + 15) / 16 * 16;  // [0] TMEM base, [1] abort flag
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kSmemAlloc = kBytes;  // the window is 1024-byte aligned (checked)
   // TMEM columns: tile t uses [256t, 256t+128) for S/P and [256t+128, ...) for O
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int kThreads = 320;
-  static constexpr int kProducerWarp = 8, kMmaWarp = 9;
+  // softmax warps 0-15 (warpgroup g: tile g & 1, key columns [64 (g >> 1), +64)),
+  // then the TMA producer and the MMA issuer
+  static constexpr int kSoftmaxThreads = 512;
+  static constexpr int kThreads = kSoftmaxThreads + 64;
+  static constexpr int kProducerWarp = 16, kMmaWarp = 17;
 };
 
 struct Params {
@@ -120,7 +129,8 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(L::bSFull + t), 1);
-      mbar_init(bar(L::bPFull + t), 128);
+      mbar_init(bar(L::bPFull + t), 256);
+      mbar_init(bar(L::bXch + t), 256);
       mbar_init(bar(L::bPVDone + t), 1);
       mbar_init(bar(L::bOFinal + t), 1);
     }
@@ -228,9 +238,10 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       }
     }
   } else {
-    // ---------------- softmax warpgroups (tile A: warps 0-3, B: 4-7) ----------------
-    const int t = warp >> 2;
-    const int r = threadIdx.x & 127;  // row within the tile = TMEM lane
+    // ---------------- softmax warpgroups ----------------
+    const int t = (warp >> 2) & 1;   // tile
+    const int hf = warp >> 3;        // key columns [64 hf, 64 hf + 64) of the tile's S
+    const int r = (warp & 3) * 32 + lane;  // row within the tile = TMEM lane
     const int qt = qtA + t;
     const int i = qt * 128 + r;
     const bool active = (t == 0) || hasB;
@@ -238,48 +249,55 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + 256 * t;
     const uint32_t tO = tS + 128;
+    float* xch = reinterpret_cast<float*>(sg + L::kXch);  // [parity][tile][half][row]
     const int ds_i = p.doc_start ? p.doc_start[row0 + min(i, T - 1)] - row0 : 0;
     const float fq = p.q_fac ? p.q_fac[bh * p.n_qtiles + min(qt, p.n_qtiles - 1)] : 1.f;
     float m = -INFINITY, l = 0.f;
     bool ok = active;
     for (int it = 0; ok && it < n_t; ++it) {
-      const int kt = kv_t0 + it, j0 = kt * 128;
+      const int kt = kv_t0 + it, j0 = kt * 128 + 64 * hf;  // first key of this half
       if (!mbar_wait(bar(L::bSFull + t), it & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       // scale of this key tile's scores (q, k tiles may carry power-of-two factors)
       const float sc = p.scale_log2 * fq * (p.k_fac ? p.k_fac[bhk * p.n_qtiles + kt] : 1.f);
       const bool pos_scale = sc > 0.f;
-      uint32_t s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s + 32 * c);
+      uint32_t s[64];
+      tmem_ld32(tS + 64 * hf, s);
+      tmem_ld32(tS + 64 * hf + 32, s + 32);
       tmem_wait_ld();
-      const bool need_mask = (j0 + 127 > i) || (j0 < ds_i);
+      const bool need_mask = (j0 + 63 > i) || (j0 < ds_i);
       const float masked = pos_scale ? -INFINITY : INFINITY;
       if (need_mask) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < 64; ++c)
           if (j0 + c > i || j0 + c < ds_i) s[c] = __float_as_uint(masked);
       }
-      // row extreme of the raw scores (max for a positive scale): four chains
-      // of three-input max / min
+      // extreme of this half's raw scores (max for a positive scale)
       float e4[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) e4[q] = __uint_as_float(s[q]);
       float ext;
       if (pos_scale) {
 #pragma unroll
-        for (int c = 4; c < 128; c += 2)
+        for (int c = 4; c < 64; c += 2)
           e4[(c >> 1) & 3] = max3f(e4[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
         ext = max3f(fmaxf(e4[0], e4[1]), e4[2], e4[3]);
       } else {
 #pragma unroll
-        for (int c = 4; c < 128; c += 2)
+        for (int c = 4; c < 64; c += 2)
           e4[(c >> 1) & 3] = min3f(e4[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
         ext = min3f(fminf(e4[0], e4[1]), e4[2], e4[3]);
       }
-      const float mx = ext * sc;  // row max of the scaled scores (log2 units)
+      // the row max of the scaled scores: this half's and the other half's
+      // (-inf for a half that is all masked, so both halves see the same value)
+      float* xs = xch + ((it & 1) * 4 + t * 2) * 128;
+      xs[hf * 128 + r] = ext * sc;
+      mbar_arrive(bar(L::bXch + t));
+      if (!mbar_wait(bar(L::bXch + t), it & 1, abort_flag)) { ok = false; break; }
+      const float mx = fmaxf(xs[r], xs[128 + r]);
       // Move the reference max only when it grows by more than 8 (log2
-      // units); the first key a row sees always moves it (m = -inf).
+      // units); the first key a row sees always moves it (m = -inf). Both
+      // halves compute the same m from the same inputs.
       const bool move = mx > m + 8.f;
       const float alpha = move ? ex2(m - mx) : 1.f;
       // O needs rescaling only if it already holds a non-zero partial sum;
@@ -290,13 +308,14 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         m = mx;
       }
       const float mref = (m == -INFINITY) ? 0.f : m;
-      // p = 2^(s * sc - m) two at a time (MUFU ex2; measured faster here than
-      // moving part of the work to the FMA pipe)
+      // p = 2^(s * sc - m) two at a time; P (bf16) goes over the first half
+      // of the S columns: this half's keys at columns [32 hf, 32 hf + 32),
+      // which both halves have read by now (they passed the exchange)
       const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-mref, -mref);
       float2 l2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                       make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -307,36 +326,46 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
           l2[e & 3] = __fadd2_rn(l2[e & 3], pv);
           pk[e] = pack_bf16(pv.x, pv.y);
         }
-        tmem_st16(tS + 16 * c, pk);
+        tmem_st16(tS + 32 * hf + 16 * c, pk);
       }
       const float2 la = __fadd2_rn(l2[0], l2[1]), lb = __fadd2_rn(l2[2], l2[3]);
       l += (la.x + la.y) + (lb.x + lb.y);
-      // The scores are dead now; rescale O (warp-collective: each lane by its
-      // own factor, 1 for lanes that kept their max) before PV_t(it) runs.
+      // rescale this half's O columns (warp-collective: each lane by its own
+      // factor, 1 for lanes that kept their max) before PV_t(it) runs
       if (__any_sync(0xffffffffu, scale_o)) {
         const float f = scale_o ? alpha : 1.f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t ov[32];
-          tmem_ld32(tO + 32 * c, ov);
+          tmem_ld32(tO + (D / 2) * hf + 32 * c, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-          tmem_st32(tO + 32 * c, ov);
+          tmem_st32(tO + (D / 2) * hf + 32 * c, ov);
         }
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(L::bPFull + t));
     }
+    // row sum: this half's plus the other half's (through the exchange area,
+    // parity n_t; both halves ran the same number of key tiles)
+    float lt = l;
+    if (ok) {
+      float* xs = xch + ((n_t & 1) * 4 + t * 2) * 128;
+      xs[hf * 128 + r] = l;
+      mbar_arrive(bar(L::bXch + t));
+      if (!mbar_wait(bar(L::bXch + t), n_t & 1, abort_flag)) ok = false;
+      else lt = xs[r] + xs[128 + r];
+    }
     if (ok && mbar_wait(bar(L::bOFinal + t), 0, abort_flag)) {
       tc_fence_after();
-      const float inv = 1.f / l;
-      __nv_bfloat16* orow = p.o + ((size_t)bh * T + min(i, T - 1)) * D;
+      const float inv = 1.f / lt;
+      __nv_bfloat16* orow = p.o + ((size_t)bh * T + min(i, T - 1)) * D + (D / 2) * hf;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t ov[32];
-        tmem_ld32(tO + 32 * c, ov);  // warp-collective
+        tmem_ld32(tO + (D / 2) * hf + 32 * c, ov);  // warp-collective
         tmem_wait_ld();
         if (i < T) {
           uint32_t pk[16];
@@ -349,7 +378,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
             dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
       }
-      if (i < T) p.lse[(size_t)bh * T + i] = (m + __log2f(l)) * 0.69314718055994531f;
+      if (i < T && hf == 0) p.lse[(size_t)bh * T + i] = (m + __log2f(lt)) * 0.69314718055994531f;
     }
   }
 
