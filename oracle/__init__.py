@@ -15,10 +15,20 @@ packed-equals-separate documents) and the float64 PyTorch reference
 ``scaled_dot_product_attention`` on the cases it covers. ``oracle.decode``
 (one new token against a key/value cache) is pinned against the last row of
 the training forward, a closed form and invariants. No function here is
-"parity unpinned".
+"parity unpinned". ``oracle.projection`` (the QKV projection with its RoPE
+and head layout, the output projection, and their backward products) is
+pinned against brute-force sums, finite differences and the attention
+oracle's own RoPE (rotating in the projection equals rotating in the
+attention).
 """
 
 from .decode import decode_forward
+from .projection import (
+    out_projection,
+    out_projection_backward,
+    qkv_projection,
+    qkv_projection_backward,
+)
 from .attention import (
     attention_backward,
     attention_forward,
@@ -32,6 +42,10 @@ from .attention import (
 
 __all__ = [
     "decode_forward",
+    "out_projection",
+    "out_projection_backward",
+    "qkv_projection",
+    "qkv_projection_backward",
     "attention_backward",
     "attention_forward",
     "backward_head",
