@@ -76,6 +76,8 @@ def parse_args():
                     help="grouped-query attention: key/value heads (dividing the workload's H)")
     ap.add_argument("--decode", default=None,
                     help="time decode attention on this decode workload instead of the training step")
+    ap.add_argument("--proj", default=None,
+                    help="time the projections around the attention on this projection workload")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -553,10 +555,93 @@ def run_decode(args):
     return 0
 
 
+def run_proj(args):
+    """The projections around one attention layer, forward and backward: the
+    QKV projection (head layout and RoPE in its epilogue), the output
+    projection and their four backward products (dx, dW for each), as
+    TFLOP/s of GEMM work against the measured bf16 tensor peak; L2 is flushed
+    between steps as in the training bench."""
+    import torch
+
+    import bwd_causal_sdpa_b200 as A
+    from bwd_causal_sdpa_b200.runner import ProjRunner
+    from workloads import make_proj_workload, proj_config_by_name
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = make_proj_workload(proj_config_by_name(args.proj))
+    stream = torch.cuda.Stream(dev)
+    r = ProjRunner(w, device=dev, stream=stream)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peaks, peak_src = load_peaks()
+
+    def step():
+        r.qkv()
+        r.out()
+        r.out_bwd()
+        r.qkv_bwd()
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 0)):
+            step()
+    if r.status() != A.ATTN_OK:
+        raise SystemExit("device status after warm-up is not OK")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    n0 = A.attn_launch_count()
+    with ClockSampler(0) as clocks:
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                flush.zero_()
+                ev[i][0].record(stream)
+                step()
+                ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    launches = A.attn_launch_count() - n0
+    A.check(A.attn_profile_enable(1), "attn_profile_enable")
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.zero_()
+            step()
+    torch.cuda.synchronize(dev)
+    A.attn_profile_enable(0)
+    prof = A.profile_summary()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    fl = w.flops()
+    flops = sum(fl.values())
+    tflops = flops / (ms / 1e3) / 1e12
+    kg = prof.get("gemm")
+    achieved = flops / (kg[1] / args.steps / 1e3) / 1e12 if kg else None
+    c = w.cfg
+    line = {
+        "metric": "attention-layer projections fwd+bwd TFLOP/s (bf16 GEMMs)", "value": tflops,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded)",
+        "config": {"workload": c.name, "B": c.B, "T": c.T, "C": c.C, "H": c.H, "H_kv": c.H_kv,
+                   "D": c.D, "rope": c.rope, "flops_per_step": flops, "flops_by_call": fl,
+                   "l2": "flushed between steps (256 MiB write outside the step events)"},
+        "roofline": None if achieved is None else {
+            "bound": "tensor", "kernel": "gemm (all six products of a step)",
+            "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+            "peak_source": f"bf16_tflops burst ({peak_src})"},
+        "kernels": {k: {"launches": n, "avg_ms": t / n} for k, (n, t) in prof.items()},
+        "gpu_launches": launches, "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.decode:
         return run_decode(args)
+    if args.proj:
+        return run_proj(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -48,6 +48,13 @@ _SIGNATURES = {
     "attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float,
                               _I, _P, _P, _P, _P]),
     "attn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
+    "attn_proj_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "attn_qkv_proj": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P,
+                           ctypes.c_size_t, _P]),
+    "attn_qkv_proj_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                               _P, ctypes.c_size_t, _P]),
+    "attn_out_proj": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "attn_out_proj_bwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "attn_workspace_bytes_gqa": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I]),
     "attn_get_status": (_I, [_P]),
     "attn_error_string": (ctypes.c_char_p, [_I]),
@@ -164,6 +171,38 @@ def attn_bwd_noalloc(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, 
                                      _ptr(rope_cos), _ptr(rope_sin), _ptr(cu_seqlens), B, H, T,
                                      D, float(scale), dtype, _ptr(dq), _ptr(dk), _ptr(dv),
                                      _stream(stream)))
+
+
+def attn_proj_workspace_bytes(B, T, H, H_kv, D) -> int:
+    return int(_lib.attn_proj_workspace_bytes(B, T, H, H_kv, D))
+
+
+def attn_qkv_proj(x, w_qkv, rope_cos, rope_sin, cu_seqlens, q, k, v, B, T, C, H, H_kv, D,
+                  workspace, ws_bytes, stream=None) -> int:
+    """q, k, v = heads of x W_qkv^T, q and k rotated when tables are given."""
+    return int(_lib.attn_qkv_proj(_ptr(x), _ptr(w_qkv), _ptr(rope_cos), _ptr(rope_sin),
+                                  _ptr(cu_seqlens), _ptr(q), _ptr(k), _ptr(v), B, T, C, H, H_kv,
+                                  D, _ptr(workspace), int(ws_bytes), _stream(stream)))
+
+
+def attn_qkv_proj_bwd(dq, dk, dv, x, w_qkv, rope_cos, rope_sin, cu_seqlens, dx, dw_qkv, B, T, C,
+                      H, H_kv, D, workspace, ws_bytes, stream=None) -> int:
+    """dx and dw_qkv (float32) from the gradients of attn_qkv_proj's outputs."""
+    return int(_lib.attn_qkv_proj_bwd(_ptr(dq), _ptr(dk), _ptr(dv), _ptr(x), _ptr(w_qkv),
+                                      _ptr(rope_cos), _ptr(rope_sin), _ptr(cu_seqlens), _ptr(dx),
+                                      _ptr(dw_qkv), B, T, C, H, H_kv, D, _ptr(workspace),
+                                      int(ws_bytes), _stream(stream)))
+
+
+def attn_out_proj(o, w_o, y, B, T, C, H, D, stream=None) -> int:
+    """y = o W_o^T, o in the attention's [B, H, T, D] layout."""
+    return int(_lib.attn_out_proj(_ptr(o), _ptr(w_o), _ptr(y), B, T, C, H, D, _stream(stream)))
+
+
+def attn_out_proj_bwd(dy, o, w_o, d_o, dw_o, B, T, C, H, D, stream=None) -> int:
+    """d_o = dy W_o ([B, H, T, D]) and dw_o = dy^T o (float32)."""
+    return int(_lib.attn_out_proj_bwd(_ptr(dy), _ptr(o), _ptr(w_o), _ptr(d_o), _ptr(dw_o), B, T,
+                                      C, H, D, _stream(stream)))
 
 
 def attn_get_status(stream=None) -> int:

@@ -695,3 +695,6 @@ extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, con
                  : bwd_simt<__nv_bfloat16, 128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de,
                                                 delta, dq, dk, dv, B, H, H, T, scale, st);
 }
+
+// The projections around the attention (tensor-core GEMMs).
+#include "proj_api.cuh"

@@ -1,0 +1,319 @@
+// proj_sm100.cuh -- tensor-core (tcgen05) GEMM for the projections around the
+// attention: C[M][N] = sum_k A[m][k] B[n][k], bf16 operands, fp32 accumulate.
+//
+// The three products of a linear layer (Forge README, "Benchmarks": forward
+// X W^T, backward dX = dY W and dW = dY^T X) and the layer around the
+// attention (ARK README, "Inference architecture (EKO)" and "Backward pass
+// (AutoGrad)": q, k, v and output projections with the weight gradients dwq,
+// dwk, dwv, dwo; Forge README, "Architecture": attention with GQA and RoPE on
+// interleaved pairs) all map onto this one kernel:
+//   * an operand is read either from a plain row-major matrix or from up to
+//     three [B*heads][T][D] head-major tensors (q, k, v: a feature index
+//     runs over q's heads, then k's, then v's, D features each), and either
+//     K-major (K contiguous) or MN-major (M or N contiguous); TMA moves it
+//     into 128-byte-swizzled shared tiles, so no transpose is ever written;
+//   * the epilogue writes bf16 rows, fp32 rows (added with reductions when K
+//     is split over several CTAs), or scatters the columns into the
+//     head-major q, k, v tensors, rotating q and k by RoPE on the way.
+// One CTA computes one 128 x BN tile (BN = 128 or 256, all of it in TMEM)
+// over its share of K in 64-wide blocks through a four-stage ring: a TMA
+// warp, an MMA warp (one elected thread issues tcgen05.mma) and four
+// epilogue warps (thread = TMEM lane = output row).
+#pragma once
+
+#include "common.cuh"
+#include "prep.cuh"
+#include "sm100.cuh"
+
+namespace proj100 {
+
+using namespace sm100;
+
+constexpr int kBM = 128, kBK = 64, kStages = 4;
+
+template <int BN>
+struct Layout {
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kA = 0;
+  static constexpr int kB = kStages * kABytes;
+  static constexpr int kBars = kB + kStages * kBBytes;
+  static constexpr int bFull = 0, bEmpty = kStages, bAcc = 2 * kStages;
+  static constexpr int kNumBars = 2 * kStages + 1;
+  static constexpr int kMisc = kBars + kNumBars * 8;
+  static constexpr int kSmemAlloc = kMisc + 16;
+  static constexpr int kProducerWarp = 0, kMmaWarp = 1;
+  static constexpr int kThreads = 192;  // + four epilogue warps
+  static constexpr uint32_t kTmemCols = BN;
+};
+
+enum Src : int { SRC_ROWS = 0, SRC_HEADS = 1 };
+enum Epi : int { EPI_ROWS_BF16 = 0, EPI_ROWS_F32 = 1, EPI_HEADS = 2 };
+
+// One operand. SRC_ROWS: a row-major matrix, [MN][K] when K-major, [K][MN]
+// when MN-major. SRC_HEADS: tensors [B*heads[s]][T][D]; the token index
+// b*T + t runs along MN when K-major, along K when MN-major, and the feature
+// index along the other.
+struct Operand {
+  int src;
+  int mn_major;
+  int heads[3];
+};
+
+struct Params {
+  int M, N, K;
+  int kb_per_split;     // 64-wide K blocks per CTA along blockIdx.z
+  int T, D;             // token rows per batch row; head dimension
+  Operand a, b;
+  int epi;
+  int out_heads[3];     // EPI_HEADS: head counts of the output tensors
+  void* out[3];         // EPI_HEADS: q, k, v (absent ones null); else out[0]
+  int reduce;           // EPI_ROWS_F32: add into out[0] instead of storing
+  int rope_segs;        // EPI_HEADS: rotate the first rope_segs tensors
+  const float* rope_cos;
+  const float* rope_sin;
+  const int32_t* doc_start;  // flattened document starts, or null
+};
+
+// Feature index f of a head-major operand -> (tensor, head, d).
+__device__ __forceinline__ void split_feature(const int* heads, int D, int f, int& seg, int& h,
+                                              int& d) {
+  seg = 0;
+  while (seg < 2 && f >= heads[seg] * D) {
+    f -= heads[seg] * D;
+    ++seg;
+  }
+  h = f / D;
+  d = f - h * D;
+}
+
+// Issue (or, with issue = false, only count the bytes of) the TMA boxes of
+// one operand tile: MN rows [mn0, mn0 + BMN) and K block kb, into dst.
+template <int BMN>
+__device__ __forceinline__ uint32_t operand_boxes(bool issue, const Operand& o,
+                                                  const CUtensorMap* m0, const CUtensorMap* m1,
+                                                  const CUtensorMap* m2, int mn_total, int T,
+                                                  int D, int mn0, int kb, uint32_t dst,
+                                                  uint32_t bar) {
+  const int k0 = kb * kBK;
+  if (!o.mn_major) {
+    // one box: BMN rows x 64 K values
+    if (issue) {
+      if (o.src == SRC_ROWS) {
+        tma_load_2d(dst, m0, bar, k0, mn0);
+      } else {
+        int seg, h, d;
+        split_feature(o.heads, D, k0, seg, h, d);
+        const int b = mn0 / T, t = mn0 - b * T;
+        tma_load_3d(dst, seg == 0 ? m0 : (seg == 1 ? m1 : m2), bar, d, t,
+                    b * o.heads[seg] + h);
+      }
+    }
+    return BMN * kBK * 2;
+  }
+  // MN-major: BMN / 64 boxes of 64 MN values x 64 K rows, 8 KB apart
+  uint32_t bytes = 0;
+#pragma unroll
+  for (int j = 0; j < BMN / 64; ++j) {
+    const int f = mn0 + 64 * j;
+    if (f >= mn_total) break;
+    if (issue) {
+      if (o.src == SRC_ROWS) {
+        tma_load_2d(dst + j * 8192, m0, bar, f, k0);
+      } else {
+        int seg, h, d;
+        split_feature(o.heads, D, f, seg, h, d);
+        const int b = k0 / T, t = k0 - b * T;
+        tma_load_3d(dst + j * 8192, seg == 0 ? m0 : (seg == 1 ? m1 : m2), bar, d, t,
+                    b * o.heads[seg] + h);
+      }
+    }
+    bytes += 64 * kBK * 2;
+  }
+  return bytes;
+}
+
+// K step kk (16 K values) of a 64-wide operand tile at base.
+__device__ __forceinline__ uint64_t operand_desc(bool mn_major, uint32_t base, int kk) {
+  return mn_major ? smem_desc_sw128(base + kk * 2048, 8192, 1024)
+                  : smem_desc_sw128(base + kk * 32, 16, 1024);
+}
+
+template <int BN>
+__global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB,
+                const Params p) {
+  pdl_wait_and_trigger();
+  using L = Layout<BN>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t sb0 = smem_u32(smem_raw);
+  if (sb0 & 1023u) {  // uniform across the CTA: nothing has been issued yet
+    if (threadIdx.x == 0) report_status(ATTN_ECUDA_LAYOUT);
+    return;
+  }
+  uint8_t* sg = smem_raw;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sg + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sg + L::kMisc + 4);
+  auto bar = [&](int i) -> uint32_t { return sb0 + L::kBars + 8u * i; };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = (int)blockIdx.x * kBM, n0 = (int)blockIdx.y * BN;
+  const int nkb_total = (p.K + kBK - 1) / kBK;
+  const int kb0 = (int)blockIdx.z * p.kb_per_split;
+  const int kb1 = min(nkb_total, kb0 + p.kb_per_split);
+  const int nkb = kb1 - kb0;  // >= 1: the host sizes the split so
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(L::bFull + s), 1);
+      mbar_init(bar(L::bEmpty + s), 1);
+    }
+    mbar_init(bar(L::bAcc), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == L::kMmaWarp) {
+    tmem_alloc(sb0 + L::kMisc, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == L::kProducerWarp) {
+    if (lane == 0) {
+      prefetch_tensor_map(&tmA0);
+      prefetch_tensor_map(&tmB);
+      for (int it = 0; it < nkb; ++it) {
+        const int s = it % kStages, round = it / kStages;
+        if (it >= kStages && !mbar_wait(bar(L::bEmpty + s), (round - 1) & 1, abort_flag)) break;
+        const uint32_t sa = sb0 + L::kA + s * L::kABytes, sbb = sb0 + L::kB + s * L::kBBytes;
+        const uint32_t bytes =
+            operand_boxes<kBM>(false, p.a, &tmA0, &tmA1, &tmA2, p.M, p.T, p.D, m0, kb0 + it, sa,
+                               0) +
+            operand_boxes<BN>(false, p.b, &tmB, &tmB, &tmB, p.N, p.T, p.D, n0, kb0 + it, sbb, 0);
+        mbar_arrive_expect_tx(bar(L::bFull + s), bytes);
+        operand_boxes<kBM>(true, p.a, &tmA0, &tmA1, &tmA2, p.M, p.T, p.D, m0, kb0 + it, sa,
+                           bar(L::bFull + s));
+        operand_boxes<BN>(true, p.b, &tmB, &tmB, &tmB, p.N, p.T, p.D, n0, kb0 + it, sbb,
+                          bar(L::bFull + s));
+      }
+    }
+  } else if (warp == L::kMmaWarp) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16(kBM, BN, true, true, p.a.mn_major != 0, p.b.mn_major != 0);
+      bool ok = true;
+      for (int it = 0; it < nkb; ++it) {
+        const int s = it % kStages;
+        if (!mbar_wait(bar(L::bFull + s), (it / kStages) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = sb0 + L::kA + s * L::kABytes, sbb = sb0 + L::kB + s * L::kBBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk)
+          mma_ss(tmem, operand_desc(p.a.mn_major, sa, kk), operand_desc(p.b.mn_major, sbb, kk),
+                 idesc, (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar(L::bEmpty + s));
+      }
+      if (ok) mma_commit(bar(L::bAcc));
+    }
+  } else {
+    // ---------------- epilogue: thread = TMEM lane = output row ----------------
+    const int sub = warp & 3;
+    const int r = sub * 32 + lane;
+    const int m = m0 + r;
+    const uint32_t tl = tmem + ((uint32_t)(sub * 32) << 16);
+    if (mbar_wait(bar(L::bAcc), 0, abort_flag)) {
+      tc_fence_after();
+      const int T = p.T, D = p.D;
+      const int b = m / T, t = m - b * T;
+      int pos = t;
+      if (p.epi == EPI_HEADS && p.rope_segs > 0 && m < p.M && p.doc_start)
+        pos = m - p.doc_start[m];
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int n = n0 + 32 * c;
+        if (n >= p.N) break;  // uniform across the warp
+        uint32_t v[32];
+        tmem_ld32(tl + 32 * c, v);
+        tmem_wait_ld();
+        if (m >= p.M) continue;
+        float f[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
+        if (p.epi == EPI_HEADS) {
+          int seg, h, d;
+          split_feature(p.out_heads, D, n, seg, h, d);  // 32 | D: the chunk stays in one head
+          if (seg < p.rope_segs) {
+            if (D == 64) rope_pairs<32, 64>(f, p.rope_cos, p.rope_sin, pos, d, false);
+            else rope_pairs<32, 128>(f, p.rope_cos, p.rope_sin, pos, d, false);
+          }
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out[seg]) +
+                               ((size_t)(b * p.out_heads[seg] + h) * T + t) * D + d;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            reinterpret_cast<uint4*>(dst)[e] =
+                make_uint4(pack_bf16(f[8 * e], f[8 * e + 1]), pack_bf16(f[8 * e + 2], f[8 * e + 3]),
+                           pack_bf16(f[8 * e + 4], f[8 * e + 5]),
+                           pack_bf16(f[8 * e + 6], f[8 * e + 7]));
+        } else if (p.epi == EPI_ROWS_BF16) {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out[0]) + (size_t)m * p.N + n;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (n + 8 * e < p.N)  // N % 8 == 0
+              reinterpret_cast<uint4*>(dst)[e] = make_uint4(
+                  pack_bf16(f[8 * e], f[8 * e + 1]), pack_bf16(f[8 * e + 2], f[8 * e + 3]),
+                  pack_bf16(f[8 * e + 4], f[8 * e + 5]), pack_bf16(f[8 * e + 6], f[8 * e + 7]));
+        } else {
+          float* dst = reinterpret_cast<float*>(p.out[0]) + (size_t)m * p.N + n;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (n + 4 * e >= p.N) break;  // N % 4 == 0
+            if (p.reduce)
+              red_add_v4(dst + 4 * e, v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+            else
+              reinterpret_cast<float4*>(dst)[e] =
+                  make_float4(f[4 * e], f[4 * e + 1], f[4 * e + 2], f[4 * e + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == L::kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// R(pos)^T applied to a [B*heads][T][D] bf16 gradient (taken with respect to
+// rotated vectors), written to dst: 8 values per thread.
+template <int D>
+__global__ void __launch_bounds__(256) rope_grad_kernel(const __nv_bfloat16* __restrict__ g,
+                                                        const float* __restrict__ rc,
+                                                        const float* __restrict__ rs,
+                                                        const int32_t* __restrict__ doc_start,
+                                                        __nv_bfloat16* __restrict__ dst, int heads,
+                                                        int T, long n8) {
+  pdl_wait_and_trigger();
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const long e0 = i * 8;
+  const int d0 = (int)(e0 % D);
+  const long row = e0 / D;  // (b * heads + h) * T + t
+  const int t = (int)(row % T);
+  const int b = (int)(row / T / heads);
+  const int m = b * T + t;
+  const int pos = doc_start ? m - doc_start[m] : t;
+  float v[8];
+  load8_bf16(g + e0, v);
+  rope_pairs<8, D>(v, rc, rs, pos, d0, true);
+  store8_bf16(dst + e0, v);
+}
+
+}  // namespace proj100

@@ -17,12 +17,15 @@ enum KernelKind : int {
   KK_DQ_FINALIZE,
   KK_DECODE,
   KK_DECODE_COMBINE,
+  KK_GEMM,
+  KK_ROPE_GRAD,
+  KK_FILL,
   KK_COUNT
 };
 
 static const char* const kKernelNames[KK_COUNT] = {
     "doc_ranges", "rope_prep", "fwd", "delta", "dkdv", "dq", "dq_finalize", "decode",
-    "decode_combine"};
+    "decode_combine", "gemm", "rope_grad", "fill"};
 
 namespace trace {
 

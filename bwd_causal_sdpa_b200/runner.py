@@ -158,3 +158,79 @@ class DecodeRunner:
         torch.cuda.synchronize(self.device)
         f = lambda t: t.detach().to(torch.float64).cpu().numpy()
         return {"o": f(self.o), "lse": f(self.lse)}
+
+
+class ProjRunner:
+    """Device buffers for the projections around one attention layer (x, the
+    weights, q, k, v, o, the output and the gradients) and the four
+    projection calls on them."""
+
+    def __init__(self, w, device="cuda", stream: Optional[torch.cuda.Stream] = None,
+                 rope: bool = True):
+        from . import attn_proj_workspace_bytes
+
+        c = w.cfg
+        self.w = w
+        self.device = torch.device(device)
+        self.stream = stream
+        dev = lambda a: to_device(a, ATTN_BF16, self.device)
+        self.x, self.w_qkv, self.w_o, self.o = dev(w.x), dev(w.w_qkv), dev(w.w_o), dev(w.o)
+        self.gq, self.gk, self.gv, self.dy = dev(w.dq), dev(w.dk), dev(w.dv), dev(w.dy)
+        bf = dict(dtype=torch.bfloat16, device=self.device)
+        self.q = torch.empty((c.B, c.H, c.T, c.D), **bf)
+        self.k = torch.empty((c.B, c.H_kv, c.T, c.D), **bf)
+        self.v = torch.empty((c.B, c.H_kv, c.T, c.D), **bf)
+        self.y = torch.empty((c.B, c.T, c.C), **bf)
+        self.dx = torch.empty((c.B, c.T, c.C), **bf)
+        self.d_o = torch.empty((c.B, c.H, c.T, c.D), **bf)
+        self.dw_qkv = torch.empty(tuple(w.w_qkv.shape), dtype=torch.float32, device=self.device)
+        self.dw_o = torch.empty(tuple(w.w_o.shape), dtype=torch.float32, device=self.device)
+        self.rope_cos = self.rope_sin = None
+        if rope and w.rope_cos is not None:
+            self.rope_cos = torch.from_numpy(np.ascontiguousarray(w.rope_cos, np.float32)).to(self.device)
+            self.rope_sin = torch.from_numpy(np.ascontiguousarray(w.rope_sin, np.float32)).to(self.device)
+        self.cu = None
+        if w.cu_seqlens is not None:
+            self.cu = torch.from_numpy(np.asarray(w.cu_seqlens, dtype=np.int32)).to(self.device)
+        self.ws_bytes = attn_proj_workspace_bytes(c.B, c.T, c.H, c.H_kv, c.D)
+        self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=self.device)
+
+    def qkv(self) -> None:
+        from . import attn_qkv_proj
+
+        c = self.w.cfg
+        check(attn_qkv_proj(self.x, self.w_qkv, self.rope_cos, self.rope_sin, self.cu, self.q,
+                            self.k, self.v, c.B, c.T, c.C, c.H, c.H_kv, c.D, self.ws,
+                            self.ws_bytes, self.stream), "attn_qkv_proj")
+
+    def qkv_bwd(self) -> None:
+        from . import attn_qkv_proj_bwd
+
+        c = self.w.cfg
+        check(attn_qkv_proj_bwd(self.gq, self.gk, self.gv, self.x, self.w_qkv, self.rope_cos,
+                                self.rope_sin, self.cu, self.dx, self.dw_qkv, c.B, c.T, c.C, c.H,
+                                c.H_kv, c.D, self.ws, self.ws_bytes, self.stream),
+              "attn_qkv_proj_bwd")
+
+    def out(self) -> None:
+        from . import attn_out_proj
+
+        c = self.w.cfg
+        check(attn_out_proj(self.o, self.w_o, self.y, c.B, c.T, c.C, c.H, c.D, self.stream),
+              "attn_out_proj")
+
+    def out_bwd(self) -> None:
+        from . import attn_out_proj_bwd
+
+        c = self.w.cfg
+        check(attn_out_proj_bwd(self.dy, self.o, self.w_o, self.d_o, self.dw_o, c.B, c.T, c.C,
+                                c.H, c.D, self.stream), "attn_out_proj_bwd")
+
+    def status(self) -> int:
+        return attn_get_status(self.stream)
+
+    def results(self) -> dict:
+        torch.cuda.synchronize(self.device)
+        f = lambda t: t.detach().to(torch.float64).cpu().numpy()
+        return {n: f(getattr(self, n)) for n in
+                ("q", "k", "v", "y", "dx", "d_o", "dw_qkv", "dw_o")}

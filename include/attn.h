@@ -219,6 +219,61 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                      void* dq, void* dk, void* dv, void* stream);
 
 /*
+ * ---- Projections around the attention (tensor-core GEMMs) ----
+ *
+ * The linear layers on either side of the attention in the pages' training
+ * layer: q, k, v = heads of x W_qkv^T (RoPE optionally applied to q and k in
+ * the same kernel) and y = o W_o^T, with their backward products dX = dY W and
+ * dW = dY^T X (ARK README, "Inference architecture (EKO)" and "Backward pass
+ * (AutoGrad)", whose per-layer gradients include dwq, dwk, dwv, dwo; Forge
+ * README, "Benchmarks" (the forward X W^T and the two backward products of a
+ * linear layer) and "Architecture" (Linear layers, attention with GQA and
+ * RoPE on interleaved pairs)). All operands and activations are bf16;
+ * accumulation is fp32; weight gradients are written in fp32.
+ *
+ * Layouts (row-major, contiguous, device pointers owned by the caller, each
+ * 16-byte aligned):
+ *   x, dx:        [B, T, C] bf16          y, dy:      [B, T, C] bf16
+ *   w_qkv:        [(H + 2 H_kv) D, C] bf16: rows of the H query heads, then
+ *                 the H_kv key heads, then the H_kv value heads, D per head
+ *   dw_qkv:       [(H + 2 H_kv) D, C] float32
+ *   q, dq:        [B, H, T, D] bf16       k, v, dk, dv: [B, H_kv, T, D] bf16
+ *   o, d_o:       [B, H, T, D] bf16 (feature index h D + d for W_o)
+ *   w_o:          [C, H D] bf16           dw_o:       [C, H D] float32
+ * Sizes: D is 64 or 128; T a multiple of 128; C a multiple of 8; B, T, C,
+ * H, H_kv >= 1; B*T < 2^31. Otherwise ATTN_EUNSUPPORTED (ATTN_EINVAL for a
+ * null pointer or H_kv <= 0, ATTN_EALIGN for a misaligned pointer).
+ * Every output is overwritten (weight gradients are not accumulated into).
+ * Asynchronous on `stream`, like the attention calls.
+ *
+ * attn_qkv_proj: with rope_cos/rope_sin NULL, q, k, v are the projection;
+ * with tables ([T, D/2] float32, as for attn_fwd) q and k are rotated at each
+ * token's position in its document (cu_seqlens as for attn_fwd, or NULL), so
+ * that attn_fwd is then called without tables. Workspace: needed only when
+ * both tables and cu_seqlens are given, attn_proj_workspace_bytes(...) bytes.
+ *
+ * attn_qkv_proj_bwd: dq, dk, dv are the gradients with respect to the
+ * outputs of attn_qkv_proj (with tables: with respect to the rotated q, k;
+ * they are rotated back first, in the workspace, which is then required).
+ * Writes dx and dw_qkv.
+ *
+ * attn_out_proj / attn_out_proj_bwd: y = o W_o^T; d_o = dy W_o (written in
+ * the attention's layout) and dw_o = dy^T o. No workspace.
+ */
+size_t attn_proj_workspace_bytes(int B, int T, int H, int H_kv, int D);
+int attn_qkv_proj(const void* x, const void* w_qkv, const float* rope_cos, const float* rope_sin,
+                  const int32_t* cu_seqlens, void* q, void* k, void* v, int B, int T, int C,
+                  int H, int H_kv, int D, void* workspace, size_t ws_bytes, void* stream);
+int attn_qkv_proj_bwd(const void* dq, const void* dk, const void* dv, const void* x,
+                      const void* w_qkv, const float* rope_cos, const float* rope_sin,
+                      const int32_t* cu_seqlens, void* dx, float* dw_qkv, int B, int T, int C,
+                      int H, int H_kv, int D, void* workspace, size_t ws_bytes, void* stream);
+int attn_out_proj(const void* o, const void* w_o, void* y, int B, int T, int C, int H, int D,
+                  void* stream);
+int attn_out_proj_bwd(const void* dy, const void* o, const void* w_o, void* d_o, float* dw_o,
+                      int B, int T, int C, int H, int D, void* stream);
+
+/*
  * Tracing aids (the source pages define no counterpart; they support
  * measurement only). Not thread safe: call them from the thread that
  * launches the attention calls.

@@ -191,3 +191,53 @@ def test_decode_host_validation_and_workspace():
     assert nb >= 2 * 8 * 8 * (128 + 2) * 4
     assert A.attn_decode_workspace_bytes(2, 8, 3, 1000, 128, A.ATTN_BF16) == 0
     assert A.attn_decode_workspace_bytes(2, 8, 2, 1000, 80, A.ATTN_BF16) == 0
+
+
+def test_projection_validation_on_host():
+    import bwd_causal_sdpa_b200 as A
+
+    def qkv(**kw):
+        a = dict(x=P, w_qkv=P, rope_cos=None, rope_sin=None, cu_seqlens=None, q=P, k=P, v=P, B=1,
+                 T=128, C=64, H=2, H_kv=1, D=64, workspace=None, ws_bytes=0)
+        a.update(kw)
+        return A.attn_qkv_proj(**a)
+
+    def qkv_bwd(**kw):
+        a = dict(dq=P, dk=P, dv=P, x=P, w_qkv=P, rope_cos=None, rope_sin=None, cu_seqlens=None,
+                 dx=P, dw_qkv=P, B=1, T=128, C=64, H=2, H_kv=1, D=64, workspace=None, ws_bytes=0)
+        a.update(kw)
+        return A.attn_qkv_proj_bwd(**a)
+
+    def out(**kw):
+        a = dict(o=P, w_o=P, y=P, B=1, T=128, C=64, H=2, D=64)
+        a.update(kw)
+        return A.attn_out_proj(**a)
+
+    def out_bwd(**kw):
+        a = dict(dy=P, o=P, w_o=P, d_o=P, dw_o=P, B=1, T=128, C=64, H=2, D=64)
+        a.update(kw)
+        return A.attn_out_proj_bwd(**a)
+
+    for call in (qkv, qkv_bwd):
+        assert call(x=None) == A.ATTN_EINVAL
+        assert call(H_kv=0) == A.ATTN_EINVAL
+        assert call(rope_cos=P) == A.ATTN_EINVAL  # one table without the other
+        assert call(D=96) == A.ATTN_EUNSUPPORTED
+        assert call(T=200) == A.ATTN_EUNSUPPORTED  # not a multiple of 128
+        assert call(C=60) == A.ATTN_EUNSUPPORTED   # rows not 16-byte strided
+        assert call(B=0) == A.ATTN_EUNSUPPORTED
+        assert call(x=P + 8) == A.ATTN_EALIGN
+    # RoPE with packed documents needs the workspace (document positions);
+    # the backward with RoPE needs it for the rotated-back gradients
+    assert qkv(rope_cos=P, rope_sin=P, cu_seqlens=P) == A.ATTN_EWORKSPACE
+    assert qkv_bwd(rope_cos=P, rope_sin=P) == A.ATTN_EWORKSPACE
+    for call in (out, out_bwd):
+        assert call(o=None) == A.ATTN_EINVAL
+        assert call(D=32) == A.ATTN_EUNSUPPORTED
+        assert call(T=64) == A.ATTN_EUNSUPPORTED
+        assert call(o=P + 4) == A.ATTN_EALIGN
+    assert out(y=None) == A.ATTN_EINVAL
+    assert out_bwd(dw_o=None) == A.ATTN_EINVAL
+    ws = A.attn_proj_workspace_bytes(2, 256, 3, 1, 64)
+    assert ws >= 2 * 256 * 4 * 2 + 2 * 256 * 4 * 64 * 2 and ws % 256 == 0
+    assert A.attn_proj_workspace_bytes(2, 200, 3, 1, 64) == 0

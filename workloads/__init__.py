@@ -14,6 +14,13 @@ from .decode import (
     decode_config_by_name,
     make_decode_workload,
 )
+from .projection import (
+    PROJ_CONFIGS,
+    ProjConfig,
+    ProjWorkload,
+    make_proj_workload,
+    proj_config_by_name,
+)
 from .generate import (
     Workload,
     draw_doc_lengths,
@@ -29,6 +36,11 @@ __all__ = [
     "DecodeWorkload",
     "decode_config_by_name",
     "make_decode_workload",
+    "PROJ_CONFIGS",
+    "ProjConfig",
+    "ProjWorkload",
+    "make_proj_workload",
+    "proj_config_by_name",
     "Config",
     "Workload",
     "config_by_name",
