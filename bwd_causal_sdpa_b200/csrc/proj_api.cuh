@@ -44,8 +44,9 @@ __global__ void __launch_bounds__(256) fill_zero_kernel(float4* __restrict__ p, 
 
 constexpr int kProjSms = 148;
 
-// One GEMM launch: the operands' maps are built by the caller. out_f32 marks
-// an fp32 row output, which may split K over CTAs (adding into a zeroed out).
+// One GEMM launch: the operands' maps are built by the caller. An fp32 row
+// output may split K over work units when the tiles alone fill less than one
+// wave (the parts are added into the zeroed output).
 int gemm_launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2,
                 const CUtensorMap& b, proj100::Params p, cudaStream_t st) {
   using namespace proj100;
@@ -62,13 +63,17 @@ int gemm_launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap&
   p.kb_per_split = (nkb + split - 1) / split;
   split = (nkb + p.kb_per_split - 1) / p.kb_per_split;  // every split gets >= 1 block
   p.reduce = split > 1;
-  if (tn > 65535 || split > 65535) return ATTN_EUNSUPPORTED;
+  p.tiles_m = tm;
+  p.tiles_n = tn;
+  p.splits = split;
+  const long units = (long)tm * tn * split;
+  if (units >= (1L << 31)) return ATTN_EUNSUPPORTED;
   if (p.reduce) {
     const long n4 = (long)p.M * p.N / 4;
     ATTN_LAUNCH(KK_FILL, st, pdl_launch(fill_zero_kernel, (unsigned)std::min<long>((n4 + 255) / 256, 4L * kProjSms),
                                         256, 0, st, (float4*)p.out[0], n4));
   }
-  const dim3 grid((unsigned)tm, (unsigned)tn, (unsigned)split);
+  const dim3 grid((unsigned)std::min<long>(units, kProjSms));  // persistent: one CTA per SM
   if (wide) {
     if (!ensure_smem(gemm_kernel<256>, Layout<256>::kSmemAlloc, smem_done256)) return ATTN_ECUDA;
     ATTN_LAUNCH(KK_GEMM, st, pdl_launch(gemm_kernel<256>, grid, Layout<256>::kThreads,

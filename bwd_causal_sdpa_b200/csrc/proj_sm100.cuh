@@ -15,10 +15,13 @@
 //   * the epilogue writes bf16 rows, fp32 rows (added with reductions when K
 //     is split over several CTAs), or scatters the columns into the
 //     head-major q, k, v tensors, rotating q and k by RoPE on the way.
-// One CTA computes one 128 x BN tile (BN = 128 or 256, all of it in TMEM)
-// over its share of K in 64-wide blocks through a four-stage ring: a TMA
-// warp, an MMA warp (one elected thread issues tcgen05.mma) and four
-// epilogue warps (thread = TMEM lane = output row).
+// Persistent: each CTA (at most one per SM) walks a strided list of work
+// units, a unit being one 128 x BN output tile (BN = 128 or 256) over one
+// share of K. K moves in 64-wide blocks through a four-stage ring that runs
+// across units; the accumulator alternates between two TMEM buffers, so the
+// epilogue of one unit overlaps the main loop of the next. Warps: TMA, MMA
+// (one elected thread issues tcgen05.mma) and four epilogue warps (thread =
+// TMEM lane = output row).
 #pragma once
 
 #include "common.cuh"
@@ -38,13 +41,14 @@ struct Layout {
   static constexpr int kA = 0;
   static constexpr int kB = kStages * kABytes;
   static constexpr int kBars = kB + kStages * kBBytes;
-  static constexpr int bFull = 0, bEmpty = kStages, bAcc = 2 * kStages;
-  static constexpr int kNumBars = 2 * kStages + 1;
+  static constexpr int bFull = 0, bEmpty = kStages, bAccFull = 2 * kStages,
+                       bAccEmpty = 2 * kStages + 2;
+  static constexpr int kNumBars = 2 * kStages + 4;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kSmemAlloc = kMisc + 16;
   static constexpr int kProducerWarp = 0, kMmaWarp = 1;
   static constexpr int kThreads = 192;  // + four epilogue warps
-  static constexpr uint32_t kTmemCols = BN;
+  static constexpr uint32_t kTmemCols = 2 * BN;  // two accumulators
 };
 
 enum Src : int { SRC_ROWS = 0, SRC_HEADS = 1 };
@@ -62,7 +66,8 @@ struct Operand {
 
 struct Params {
   int M, N, K;
-  int kb_per_split;     // 64-wide K blocks per CTA along blockIdx.z
+  int tiles_m, tiles_n, splits;  // work units: tiles_m * tiles_n * splits
+  int kb_per_split;     // 64-wide K blocks per unit
   int T, D;             // token rows per batch row; head dimension
   Operand a, b;
   int epi;
@@ -157,18 +162,30 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sg + L::kMisc + 4);
   auto bar = [&](int i) -> uint32_t { return sb0 + L::kBars + 8u * i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = (int)blockIdx.x * kBM, n0 = (int)blockIdx.y * BN;
   const int nkb_total = (p.K + kBK - 1) / kBK;
-  const int kb0 = (int)blockIdx.z * p.kb_per_split;
-  const int kb1 = min(nkb_total, kb0 + p.kb_per_split);
-  const int nkb = kb1 - kb0;  // >= 1: the host sizes the split so
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int n_units = tiles * p.splits;
+  // Work unit u (this CTA takes u = blockIdx.x, + gridDim.x, ...): split
+  // u / tiles, then the tile, M fastest so that CTAs running at the same time
+  // share the B tile (the weights) in L2.
+  auto unit = [&](int u, int& m0, int& n0, int& kb0, int& nkb) {
+    const int z = u / tiles, r = u - z * tiles;
+    const int tn = r / p.tiles_m;
+    m0 = (r - tn * p.tiles_m) * kBM;
+    n0 = tn * BN;
+    kb0 = z * p.kb_per_split;
+    nkb = min(nkb_total, kb0 + p.kb_per_split) - kb0;  // >= 1: the host sizes the split so
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(L::bFull + s), 1);
       mbar_init(bar(L::bEmpty + s), 1);
     }
-    mbar_init(bar(L::bAcc), 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar(L::bAccFull + a), 1);
+      mbar_init(bar(L::bAccEmpty + a), 128);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -185,68 +202,97 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
     if (lane == 0) {
       prefetch_tensor_map(&tmA0);
       prefetch_tensor_map(&tmB);
-      for (int it = 0; it < nkb; ++it) {
-        const int s = it % kStages, round = it / kStages;
-        if (it >= kStages && !mbar_wait(bar(L::bEmpty + s), (round - 1) & 1, abort_flag)) break;
-        const uint32_t sa = sb0 + L::kA + s * L::kABytes, sbb = sb0 + L::kB + s * L::kBBytes;
-        const uint32_t bytes =
-            operand_boxes<kBM>(false, p.a, &tmA0, &tmA1, &tmA2, p.M, p.T, p.D, m0, kb0 + it, sa,
-                               0) +
-            operand_boxes<BN>(false, p.b, &tmB, &tmB, &tmB, p.N, p.T, p.D, n0, kb0 + it, sbb, 0);
-        mbar_arrive_expect_tx(bar(L::bFull + s), bytes);
-        operand_boxes<kBM>(true, p.a, &tmA0, &tmA1, &tmA2, p.M, p.T, p.D, m0, kb0 + it, sa,
-                           bar(L::bFull + s));
-        operand_boxes<BN>(true, p.b, &tmB, &tmB, &tmB, p.N, p.T, p.D, n0, kb0 + it, sbb,
-                          bar(L::bFull + s));
+      int it = 0;  // K blocks loaded so far by this CTA, over all its units
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        int m0, n0, kb0, nkb;
+        unit(u, m0, n0, kb0, nkb);
+        for (int j = 0; j < nkb; ++j, ++it) {
+          const int s = it % kStages, round = it / kStages;
+          if (it >= kStages && !mbar_wait(bar(L::bEmpty + s), (round - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = sb0 + L::kA + s * L::kABytes, sbb = sb0 + L::kB + s * L::kBBytes;
+          const uint32_t bytes =
+              operand_boxes<kBM>(false, p.a, &tmA0, &tmA1, &tmA2, p.M, p.T, p.D, m0, kb0 + j, sa,
+                                 0) +
+              operand_boxes<BN>(false, p.b, &tmB, &tmB, &tmB, p.N, p.T, p.D, n0, kb0 + j, sbb, 0);
+          mbar_arrive_expect_tx(bar(L::bFull + s), bytes);
+          operand_boxes<kBM>(true, p.a, &tmA0, &tmA1, &tmA2, p.M, p.T, p.D, m0, kb0 + j, sa,
+                             bar(L::bFull + s));
+          operand_boxes<BN>(true, p.b, &tmB, &tmB, &tmB, p.N, p.T, p.D, n0, kb0 + j, sbb,
+                            bar(L::bFull + s));
+        }
       }
     }
   } else if (warp == L::kMmaWarp) {
     if (lane == 0) {
       const uint32_t idesc = idesc_f16(kBM, BN, true, true, p.a.mn_major != 0, p.b.mn_major != 0);
+      int it = 0, n = 0;  // K blocks consumed, units finished by this CTA
       bool ok = true;
-      for (int it = 0; it < nkb; ++it) {
-        const int s = it % kStages;
-        if (!mbar_wait(bar(L::bFull + s), (it / kStages) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++n) {
+        int m0, n0, kb0, nkb;
+        unit(u, m0, n0, kb0, nkb);
+        const int a = n & 1;
+        // the epilogue must have read this accumulator's previous unit out
+        if (n >= 2 && !mbar_wait(bar(L::bAccEmpty + a), ((n >> 1) - 1) & 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t sa = sb0 + L::kA + s * L::kABytes, sbb = sb0 + L::kB + s * L::kBBytes;
+        const uint32_t acc = tmem + a * BN;
+        for (int j = 0; j < nkb; ++j, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(bar(L::bFull + s), (it / kStages) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = sb0 + L::kA + s * L::kABytes, sbb = sb0 + L::kB + s * L::kBBytes;
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk)
-          mma_ss(tmem, operand_desc(p.a.mn_major, sa, kk), operand_desc(p.b.mn_major, sbb, kk),
-                 idesc, (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar(L::bEmpty + s));
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            mma_ss(acc, operand_desc(p.a.mn_major, sa, kk), operand_desc(p.b.mn_major, sbb, kk),
+                   idesc, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(L::bEmpty + s));
+        }
+        if (ok) mma_commit(bar(L::bAccFull + a));
       }
-      if (ok) mma_commit(bar(L::bAcc));
     }
   } else {
     // ---------------- epilogue: thread = TMEM lane = output row ----------------
     const int sub = warp & 3;
     const int r = sub * 32 + lane;
-    const int m = m0 + r;
     const uint32_t tl = tmem + ((uint32_t)(sub * 32) << 16);
-    if (mbar_wait(bar(L::bAcc), 0, abort_flag)) {
+    const int T = p.T, D = p.D;
+    int n = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++n) {
+      int m0, n0, kb0, nkb;
+      unit(u, m0, n0, kb0, nkb);
+      const int a = n & 1;
+      if (!mbar_wait(bar(L::bAccFull + a), (n >> 1) & 1, abort_flag)) break;
       tc_fence_after();
-      const int T = p.T, D = p.D;
+      const int m = m0 + r;
       const int b = m / T, t = m - b * T;
       int pos = t;
       if (p.epi == EPI_HEADS && p.rope_segs > 0 && m < p.M && p.doc_start)
         pos = m - p.doc_start[m];
+      const int nch = min(BN, p.N - n0 + 31) / 32;  // chunks holding columns < N
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        const int n = n0 + 32 * c;
-        if (n >= p.N) break;  // uniform across the warp
+      for (int c = 0; c < nch; ++c) {
+        const int nc = n0 + 32 * c;
         uint32_t v[32];
-        tmem_ld32(tl + 32 * c, v);
+        tmem_ld32(tl + a * BN + 32 * c, v);
         tmem_wait_ld();
+        if (c == nch - 1) {
+          // every column of this accumulator that is used has been read
+          tc_fence_before();
+          mbar_arrive(bar(L::bAccEmpty + a));
+        }
         if (m >= p.M) continue;
         float f[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
         if (p.epi == EPI_HEADS) {
           int seg, h, d;
-          split_feature(p.out_heads, D, n, seg, h, d);  // 32 | D: the chunk stays in one head
+          split_feature(p.out_heads, D, nc, seg, h, d);  // 32 | D: the chunk stays in one head
           if (seg < p.rope_segs) {
             if (D == 64) rope_pairs<32, 64>(f, p.rope_cos, p.rope_sin, pos, d, false);
             else rope_pairs<32, 128>(f, p.rope_cos, p.rope_sin, pos, d, false);
@@ -260,18 +306,18 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
                            pack_bf16(f[8 * e + 4], f[8 * e + 5]),
                            pack_bf16(f[8 * e + 6], f[8 * e + 7]));
         } else if (p.epi == EPI_ROWS_BF16) {
-          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out[0]) + (size_t)m * p.N + n;
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out[0]) + (size_t)m * p.N + nc;
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            if (n + 8 * e < p.N)  // N % 8 == 0
+            if (nc + 8 * e < p.N)  // N % 8 == 0
               reinterpret_cast<uint4*>(dst)[e] = make_uint4(
                   pack_bf16(f[8 * e], f[8 * e + 1]), pack_bf16(f[8 * e + 2], f[8 * e + 3]),
                   pack_bf16(f[8 * e + 4], f[8 * e + 5]), pack_bf16(f[8 * e + 6], f[8 * e + 7]));
         } else {
-          float* dst = reinterpret_cast<float*>(p.out[0]) + (size_t)m * p.N + n;
+          float* dst = reinterpret_cast<float*>(p.out[0]) + (size_t)m * p.N + nc;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            if (n + 4 * e >= p.N) break;  // N % 4 == 0
+            if (nc + 4 * e >= p.N) break;  // N % 4 == 0
             if (p.reduce)
               red_add_v4(dst + 4 * e, v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
             else
