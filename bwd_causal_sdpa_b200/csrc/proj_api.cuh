@@ -55,13 +55,39 @@ int gemm_launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap&
   const int BN = wide ? 256 : 128;
   const int tm = (p.M + kBM - 1) / kBM, tn = (p.N + BN - 1) / BN;
   const int nkb = (p.K + kBK - 1) / kBK;
+  // fp32 outputs may split K over work units. The split is chosen by a small
+  // cost model in microseconds: rounds of persistent CTAs times the K blocks
+  // of one unit (at the per-SM share of the measured bf16 tensor rate, about
+  // 11 TFLOP/s) plus a pipeline fill per round, plus, for a split, zeroing
+  // the output and one more fp32 reduce of it per part (at ~2.5 TB/s of L2
+  // reductions, half of which overlaps the main loops).
+  auto rounded = [&](int s) {
+    const int per = (nkb + s - 1) / s;
+    return (nkb + per - 1) / per;  // every split gets >= 1 block
+  };
+  auto cost_us = [&](int s) {
+    const int sr = rounded(s), per = (nkb + sr - 1) / sr;
+    const long units = (long)tm * tn * sr;
+    const long rounds = (units + kProjSms - 1) / kProjSms;
+    const double kb_us = 2.0 * kBM * BN * kBK / 11.2e6;
+    const double out_mb = (double)p.M * p.N * 4 / 1e6;
+    double t = rounds * (per * kb_us + 1.0);
+    if (sr > 1) t += out_mb / 6.0 + 0.5 * sr * out_mb / 2.5;  // MB at MB/us
+    return t;
+  };
   int split = 1;
-  if (p.epi == EPI_ROWS_F32 && (long)tm * tn < kProjSms) {
-    split = (int)(kProjSms / ((long)tm * tn));
-    split = std::max(1, std::min(split, nkb / 4));
+  if (p.epi == EPI_ROWS_F32) {
+    double best = cost_us(1);
+    for (int s = 2; s <= 32 && nkb / s >= 4; ++s) {
+      const double c = cost_us(s);
+      if (c < best) {
+        best = c;
+        split = s;
+      }
+    }
   }
+  split = rounded(split);
   p.kb_per_split = (nkb + split - 1) / split;
-  split = (nkb + p.kb_per_split - 1) / p.kb_per_split;  // every split gets >= 1 block
   p.reduce = split > 1;
   p.tiles_m = tm;
   p.tiles_n = tn;
