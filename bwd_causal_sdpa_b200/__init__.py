@@ -59,6 +59,7 @@ _SIGNATURES = {
     "attn_get_status": (_I, [_P]),
     "attn_error_string": (ctypes.c_char_p, [_I]),
     "attn_exp2_selftest": (_I, [_P, _P, _I, _P]),
+    "attn_debug_withhold": (_I, [_I]),
     "attn_launch_count": (ctypes.c_ulonglong, []),
     "attn_profile_enable": (_I, [_I]),
     "attn_profile_kinds": (_I, []),
@@ -215,6 +216,11 @@ def attn_error_string(code: int) -> str:
 
 def attn_exp2_selftest(x, y, n, stream=None) -> int:
     return int(_lib.attn_exp2_selftest(_ptr(x), _ptr(y), int(n), _stream(stream)))
+
+
+def attn_debug_withhold(what) -> int:
+    """Watchdog test hook; ATTN_EUNSUPPORTED in this (hook-free) library."""
+    return int(_lib.attn_debug_withhold(int(what)))
 
 
 def attn_launch_count() -> int:

@@ -463,6 +463,17 @@ int attn_exp2_selftest(const float* x, float* y, int n, void* stream) {
   return launch_status();
 }
 
+int attn_debug_withhold(int what) {
+#ifdef ATTN_DEBUG_HOOKS
+  if (what < 0 || what > 1) return ATTN_EINVAL;
+  return cudaMemcpyToSymbol(g_attn_withhold, &what, sizeof(int)) == cudaSuccess ? ATTN_OK
+                                                                              : ATTN_ECUDA;
+#else
+  (void)what;
+  return ATTN_EUNSUPPORTED;
+#endif
+}
+
 int attn_profile_enable(int on) { return trace::enable(on != 0) == 0 ? ATTN_OK : ATTN_ECUDA; }
 
 int attn_profile_kinds(void) { return KK_COUNT; }

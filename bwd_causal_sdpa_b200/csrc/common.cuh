@@ -21,6 +21,12 @@ __device__ __forceinline__ void report_status(int code) {
   atomicCAS(&g_attn_status, 0, code);
 }
 
+#ifdef ATTN_DEBUG_HOOKS
+// Watchdog test build only: a load the forward's TMA warp withholds (0 = none,
+// 1 = the first V tile), so that a consumer's bounded wait runs out.
+__device__ int g_attn_withhold;
+#endif
+
 // Programmatic dependent launch. Every kernel of this library runs this first:
 // wait until the kernel before it in the stream has completed and its memory
 // operations are visible (a no-op when launched without the attribute), so no

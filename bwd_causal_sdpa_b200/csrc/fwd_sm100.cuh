@@ -165,6 +165,9 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         for (int cb = 0; cb < D / 64; ++cb)
           tma_load_3d(sb0 + L::kK + st * L::kTileBytes + cb * L::kBlockBytes, &tmK,
                       bar(L::bKFull + st), cb * 64, kvrow, bhk);
+#ifdef ATTN_DEBUG_HOOKS
+        if (it == 0 && g_attn_withhold == 1) continue;  // V(0) never arrives
+#endif
         if (it >= L::kStages && !mbar_wait(bar(L::bVEmpty + st), (round - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar(L::bVFull + st), L::kTileBytes);
         for (int cb = 0; cb < D / 64; ++cb)

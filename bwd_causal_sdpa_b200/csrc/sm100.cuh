@@ -74,8 +74,12 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 // Give up after about two seconds at the top clock: a wait that long means a
 // lost arrival, never normal progress. On expiry the status word records
 // ATTN_ETIMEOUT, the CTA-wide abort flag is raised and false is returned; the
-// caller then unwinds (every role checks the flag) and frees its TMEM.
-constexpr long long kWaitLimitCycles = 4000000000LL;
+// caller then unwinds (every role checks the flag) and frees its TMEM. The
+// watchdog test build (debug hooks) shortens the limit to about 10 ms.
+#ifndef ATTN_WAIT_LIMIT_CYCLES
+#define ATTN_WAIT_LIMIT_CYCLES 4000000000LL
+#endif
+constexpr long long kWaitLimitCycles = ATTN_WAIT_LIMIT_CYCLES;
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;

@@ -298,6 +298,16 @@ int attn_out_proj_bwd(const void* dy, const void* o, const void* w_o, void* d_o,
  * CUDA's exp2f. Returns ATTN_OK, ATTN_EINVAL or ATTN_ECUDA. */
 int attn_exp2_selftest(const float* x, float* y, int n, void* stream);
 
+/* attn_debug_withhold: watchdog test hook. In a library built with the debug
+ * hooks (libattn_debug.so: bounded waits cut to about 10 ms), what = 1 makes
+ * every later attn_fwd / attn_fwd_gqa on the tensor-core path withhold the
+ * load of its first value tile, so the waits for it run out: the call
+ * completes, leaves o and lse undefined and the status word reports
+ * ATTN_ETIMEOUT; what = 0 restores normal loads. Synchronous (device-wide).
+ * Returns ATTN_OK, ATTN_EINVAL (what not 0 or 1), ATTN_ECUDA, or
+ * ATTN_EUNSUPPORTED in a library built without the hooks (libattn.so). */
+int attn_debug_withhold(int what);
+
 unsigned long long attn_launch_count(void);
 int attn_profile_enable(int on);
 int attn_profile_kinds(void);

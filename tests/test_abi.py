@@ -241,3 +241,17 @@ def test_projection_validation_on_host():
     ws = A.attn_proj_workspace_bytes(2, 256, 3, 1, 64)
     assert ws >= 2 * 256 * 4 * 2 + 2 * 256 * 4 * 64 * 2 and ws % 256 == 0
     assert A.attn_proj_workspace_bytes(2, 200, 3, 1, 64) == 0
+
+
+def test_debug_hook_is_absent_from_the_product_library():
+    import ctypes
+
+    import bwd_causal_sdpa_b200 as A
+
+    # the product library has no hooks compiled in; the call touches no CUDA
+    assert A.attn_debug_withhold(1) == A.ATTN_EUNSUPPORTED
+    debug = os.path.join(ROOT, "bwd_causal_sdpa_b200", "libattn_debug.so")
+    if os.path.exists(debug):
+        lib = ctypes.CDLL(debug)
+        for n in _declared_functions():
+            assert hasattr(lib, n), f"{n} missing from the watchdog build"
