@@ -201,14 +201,36 @@ def blas_threads() -> int:
         return 1
 
 
-def oracle_slice_seconds(w, heads):
+def oracle_slice_seconds(w, heads, outputs=None):
+    """Seconds the float64 oracle takes for the forward and backward of the
+    given (b, h) slices; its results go into ``outputs`` when a dict is given."""
     from oracle import attention_backward, attention_forward
 
     t0 = time.perf_counter()
-    attention_forward(w.q, w.k, w.v, w.rope_cos, w.rope_sin, w.cu_seqlens, w.scale, heads=heads)
-    attention_backward(w.q, w.k, w.v, w.do, w.rope_cos, w.rope_sin, w.cu_seqlens, w.scale,
-                       heads=heads)
-    return time.perf_counter() - t0
+    o, lse = attention_forward(w.q, w.k, w.v, w.rope_cos, w.rope_sin, w.cu_seqlens, w.scale,
+                               heads=heads)
+    dq, dk, dv = attention_backward(w.q, w.k, w.v, w.do, w.rope_cos, w.rope_sin, w.cu_seqlens,
+                                    w.scale, heads=heads)
+    secs = time.perf_counter() - t0
+    if outputs is not None:
+        outputs.update(o=o, lse=lse, dq=dq, dk=dk, dv=dv)
+    return secs
+
+
+def slice_errors(w, heads, ref, got):
+    """Relative Frobenius error of each output over the sampled slices (dk, dv
+    only when every query head has its own key/value head: with grouped heads
+    the oracle's partial sums over the sample are not the whole gradient)."""
+    import numpy as np
+
+    errs = {}
+    names = ["o", "lse", "dq"] + (["dk", "dv"] if w.kv_heads == w.H else [])
+    for n in names:
+        a = np.stack([got[n][b, h] for b, h in heads]).astype(np.float64)
+        r = np.stack([ref[n][b, h] for b, h in heads])
+        den = np.linalg.norm(r)
+        errs[n] = float(np.linalg.norm(a - r) / (den if den > 0 else 1.0))
+    return errs
 
 
 def slice_flops(w, heads) -> float:
@@ -508,12 +530,21 @@ def run_ours(args):
         del r2, sets
 
     cpu = None
+    parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         heads = [(0, 0)]
-        secs = oracle_slice_seconds(w, heads)
+        ref = {}
+        secs = oracle_slice_seconds(w, heads, ref)
         cpu = {"value": slice_flops(w, heads) / secs / 1e12, "unit": UNIT,
                "cores": blas_threads(), "kind": "oracle", "seconds": secs,
                "sample": sample_description(w, heads)}
+        # the timed path's own outputs (the inputs never change between
+        # steps) against the oracle on the same slice
+        parity = {"sample": [list(x) for x in heads],
+                  "rel_fro": slice_errors(w, heads, ref, r.results()),
+                  "tolerance": ({"o": 1e-2, "lse": 1e-4, "dq": 1e-2, "dk": 1e-2, "dv": 1e-2}
+                                if w.dtype == "bf16" else
+                                {"o": 1e-5, "lse": 1e-5, "dq": 1e-5, "dk": 1e-5, "dv": 1e-5})}
 
     if rank == 0:
         line = {
@@ -528,7 +559,7 @@ def run_ours(args):
             "value_within_documents": w.algorithmic_flops() * world / (ms / 1e3) / 1e12,
             "roofline": roofline, "kernels": kernels,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-            "clocks": clocks.summary(),
+            "clocks": clocks.summary(), "parity": parity,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
