@@ -126,3 +126,68 @@ def test_out_backward_matches_finite_differences():
         assert d_o[idx] == pytest.approx(_central(loss, o, idx), rel=1e-8, abs=1e-9)
     for idx in [(0, 0), (4, 7), (2, 5)]:
         assert dw[idx] == pytest.approx(_central(loss, w, idx), rel=1e-8, abs=1e-9)
+
+
+# --------------------------------------------------------------------------
+# Planted mistakes: every mutant of the projection oracle must fail a pin
+# --------------------------------------------------------------------------
+
+import oracle.projection as P  # noqa: E402
+
+
+def _pins_pass():
+    checks = [test_qkv_projection_matches_index_sums,
+              test_out_projection_matches_index_sums,
+              test_identity_weights_relabel_the_input,
+              lambda: test_rope_in_projection_equals_rope_in_attention(True),
+              lambda: test_qkv_backward_matches_finite_differences(True, True),
+              lambda: test_qkv_backward_matches_finite_differences(False, False),
+              test_out_backward_matches_finite_differences]
+    for c in checks:
+        try:
+            c()
+        except (AssertionError, ValueError, IndexError):
+            return False
+    return True
+
+
+_orig_split, _orig_merge = P._split_heads, P._merge_heads
+_orig_qkv, _orig_rot, _orig_inv = P.qkv_projection, P.rope_rotate, P.rope_rotate_inverse
+
+
+def _mut_split_d_major(y, B, T, heads, D):
+    # features read as d-major (d * heads + h) instead of head-major
+    return y.reshape(B, T, D, heads).transpose(0, 3, 1, 2)
+
+
+def _mut_merge_d_major(t):
+    B, heads, T, D = t.shape
+    return t.transpose(0, 2, 3, 1).reshape(B, T, heads * D)
+
+
+def _mut_k_v_swapped(x, w_qkv, H, H_kv, D, rope_cos=None, rope_sin=None, cu_seqlens=None):
+    q, k, v = _orig_qkv(x, w_qkv, H, H_kv, D, rope_cos, rope_sin, cu_seqlens)
+    return q, v, k
+
+
+def _mut_backward_no_inverse(g, cos, sin, pos):
+    return g  # the gradient of the rotated q, k used as if un-rotated
+
+
+MUTANTS = {
+    "heads_read_d_major": ("_split_heads", _mut_split_d_major),
+    "heads_merged_d_major": ("_merge_heads", _mut_merge_d_major),
+    "k_and_v_swapped": ("qkv_projection", _mut_k_v_swapped),
+    "backward_skips_inverse_rope": ("rope_rotate_inverse", _mut_backward_no_inverse),
+    "backward_rotates_forward": ("rope_rotate_inverse", lambda g, c, s, p: _orig_rot(g, c, s, p)),
+}
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_planted_mistake_is_caught(mutant, monkeypatch):
+    assert _pins_pass()
+    attr, fn = MUTANTS[mutant]
+    monkeypatch.setattr(P, attr, fn)
+    if attr == "qkv_projection":  # the pins call it through this module's own import
+        monkeypatch.setitem(globals(), "qkv_projection", fn)
+    assert not _pins_pass(), f"no pin caught the planted mistake {mutant}"
