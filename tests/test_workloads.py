@@ -60,3 +60,30 @@ def test_config_table():
                                          "long_context_8k", "packed_docs"]
     c = config_by_name("long_context_8k")
     assert c.nominal_flops == 7 * 1 * 16 * 8192 * 8192 * 128
+
+
+def test_projection_workloads_are_seeded_shaped_and_bf16():
+    from workloads import PROJ_CONFIGS, make_proj_workload, proj_config_by_name
+
+    for cfg in PROJ_CONFIGS:
+        w = make_proj_workload(cfg, B=1, T=256)
+        c = w.cfg
+        F = (c.H + 2 * c.H_kv) * c.D
+        assert w.x.shape == (1, 256, c.C) and w.w_qkv.shape == (F, c.C)
+        assert w.w_o.shape == (c.C, c.H * c.D) and w.o.shape == (1, c.H, 256, c.D)
+        assert w.dq.shape == (1, c.H, 256, c.D) and w.dk.shape == w.dv.shape == (1, c.H_kv, 256, c.D)
+        assert w.dy.shape == (1, 256, c.C)
+        for a in (w.x, w.w_qkv, w.w_o, w.o, w.dq, w.dk, w.dv, w.dy):
+            assert a.dtype == np.float32 and np.array_equal(round_to_bf16(a), a)
+        # fan-in scale of the weights, 0.01 for the output gradients
+        assert abs(w.w_qkv.std() * np.sqrt(c.C) - 1.0) < 0.05
+        assert abs(w.dy.std() / 0.01 - 1.0) < 0.05
+        if c.packed:
+            cu = w.cu_seqlens
+            assert cu[0] == 0 and cu[-1] == 256 and np.all(np.diff(cu) > 0)
+            assert np.all(np.diff(cu)[:-1] <= c.doc_hi)
+    a = make_proj_workload(proj_config_by_name("proj_small_d64"))
+    b = make_proj_workload(proj_config_by_name("proj_small_d64"))
+    assert np.array_equal(a.x, b.x) and np.array_equal(a.cu_seqlens, b.cu_seqlens)
+    c = make_proj_workload(proj_config_by_name("proj_small_d64"), seed=99)
+    assert not np.array_equal(a.x, c.x)
