@@ -49,6 +49,7 @@ _SIGNATURES = {
                               _I, _P, _P, _P, _P]),
     "attn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
     "attn_proj_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "attn_proj_gemm_plan": (_I, [_I, _I, _I, _I, ctypes.POINTER(_I)]),
     "attn_qkv_proj": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P,
                            ctypes.c_size_t, _P]),
     "attn_qkv_proj_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
@@ -176,6 +177,15 @@ def attn_bwd_noalloc(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, 
 
 def attn_proj_workspace_bytes(B, T, H, H_kv, D) -> int:
     return int(_lib.attn_proj_workspace_bytes(B, T, H, H_kv, D))
+
+
+def attn_proj_gemm_plan(M, N, K, f32_out):
+    """(code, {bn, tiles_m, tiles_n, splits, kb_per_split, ctas}) of one
+    projection GEMM; host arithmetic only."""
+    out = (ctypes.c_int * 6)()
+    code = int(_lib.attn_proj_gemm_plan(int(M), int(N), int(K), int(bool(f32_out)), out))
+    keys = ("bn", "tiles_m", "tiles_n", "splits", "kb_per_split", "ctas")
+    return code, dict(zip(keys, list(out)))
 
 
 def attn_qkv_proj(x, w_qkv, rope_cos, rope_sin, cu_seqlens, q, k, v, B, T, C, H, H_kv, D,

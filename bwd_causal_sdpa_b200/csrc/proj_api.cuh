@@ -44,39 +44,40 @@ __global__ void __launch_bounds__(256) fill_zero_kernel(float4* __restrict__ p, 
 
 constexpr int kProjSms = 148;
 
-// One GEMM launch: the operands' maps are built by the caller. An fp32 row
-// output may split K over work units when the tiles alone fill less than one
-// wave (the parts are added into the zeroed output).
-int gemm_launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2,
-                const CUtensorMap& b, proj100::Params p, cudaStream_t st) {
+// Tile width and K split of one GEMM. fp32 outputs may split K over work
+// units; the split is chosen by a small cost model in microseconds: rounds of
+// persistent CTAs times the K blocks of one unit (at the per-SM share of the
+// measured bf16 tensor rate, about 11 TFLOP/s) plus a pipeline fill per
+// round, plus, for a split, zeroing the output and one more fp32 reduce of it
+// per part (at ~2.5 TB/s of L2 reductions, half of which overlaps the main
+// loops).
+struct GemmPlan {
+  int bn, tiles_m, tiles_n, splits, kb_per_split;
+  long units, ctas;
+};
+GemmPlan plan_gemm(int M, int N, int K, bool f32_out) {
   using namespace proj100;
-  static bool smem_done128[64], smem_done256[64];
-  const bool wide = p.N >= 256;
-  const int BN = wide ? 256 : 128;
-  const int tm = (p.M + kBM - 1) / kBM, tn = (p.N + BN - 1) / BN;
-  const int nkb = (p.K + kBK - 1) / kBK;
-  // fp32 outputs may split K over work units. The split is chosen by a small
-  // cost model in microseconds: rounds of persistent CTAs times the K blocks
-  // of one unit (at the per-SM share of the measured bf16 tensor rate, about
-  // 11 TFLOP/s) plus a pipeline fill per round, plus, for a split, zeroing
-  // the output and one more fp32 reduce of it per part (at ~2.5 TB/s of L2
-  // reductions, half of which overlaps the main loops).
+  GemmPlan g;
+  g.bn = N >= 256 ? 256 : 128;
+  g.tiles_m = (M + kBM - 1) / kBM;
+  g.tiles_n = (N + g.bn - 1) / g.bn;
+  const int nkb = (K + kBK - 1) / kBK;
   auto rounded = [&](int s) {
     const int per = (nkb + s - 1) / s;
     return (nkb + per - 1) / per;  // every split gets >= 1 block
   };
   auto cost_us = [&](int s) {
     const int sr = rounded(s), per = (nkb + sr - 1) / sr;
-    const long units = (long)tm * tn * sr;
+    const long units = (long)g.tiles_m * g.tiles_n * sr;
     const long rounds = (units + kProjSms - 1) / kProjSms;
-    const double kb_us = 2.0 * kBM * BN * kBK / 11.2e6;
-    const double out_mb = (double)p.M * p.N * 4 / 1e6;
+    const double kb_us = 2.0 * kBM * g.bn * kBK / 11.2e6;
+    const double out_mb = (double)M * N * 4 / 1e6;
     double t = rounds * (per * kb_us + 1.0);
     if (sr > 1) t += out_mb / 6.0 + 0.5 * sr * out_mb / 2.5;  // MB at MB/us
     return t;
   };
   int split = 1;
-  if (p.epi == EPI_ROWS_F32) {
+  if (f32_out) {
     double best = cost_us(1);
     for (int s = 2; s <= 32 && nkb / s >= 4; ++s) {
       const double c = cost_us(s);
@@ -86,21 +87,33 @@ int gemm_launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap&
       }
     }
   }
-  split = rounded(split);
-  p.kb_per_split = (nkb + split - 1) / split;
-  p.reduce = split > 1;
-  p.tiles_m = tm;
-  p.tiles_n = tn;
-  p.splits = split;
-  const long units = (long)tm * tn * split;
-  if (units >= (1L << 31)) return ATTN_EUNSUPPORTED;
+  g.splits = rounded(split);
+  g.kb_per_split = (nkb + g.splits - 1) / g.splits;
+  g.units = (long)g.tiles_m * g.tiles_n * g.splits;
+  g.ctas = std::min<long>(g.units, kProjSms);  // persistent: at most one CTA per SM
+  return g;
+}
+
+// One GEMM launch: the operands' maps are built by the caller. With a K
+// split the fp32 output is zeroed first and the parts are added into it.
+int gemm_launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2,
+                const CUtensorMap& b, proj100::Params p, cudaStream_t st) {
+  using namespace proj100;
+  static bool smem_done128[64], smem_done256[64];
+  const GemmPlan g = plan_gemm(p.M, p.N, p.K, p.epi == EPI_ROWS_F32);
+  if (g.units >= (1L << 31)) return ATTN_EUNSUPPORTED;
+  p.tiles_m = g.tiles_m;
+  p.tiles_n = g.tiles_n;
+  p.splits = g.splits;
+  p.kb_per_split = g.kb_per_split;
+  p.reduce = g.splits > 1;
   if (p.reduce) {
     const long n4 = (long)p.M * p.N / 4;
     ATTN_LAUNCH(KK_FILL, st, pdl_launch(fill_zero_kernel, (unsigned)std::min<long>((n4 + 255) / 256, 4L * kProjSms),
                                         256, 0, st, (float4*)p.out[0], n4));
   }
-  const dim3 grid((unsigned)std::min<long>(units, kProjSms));  // persistent: one CTA per SM
-  if (wide) {
+  const dim3 grid((unsigned)g.ctas);
+  if (g.bn == 256) {
     if (!ensure_smem(gemm_kernel<256>, Layout<256>::kSmemAlloc, smem_done256)) return ATTN_ECUDA;
     ATTN_LAUNCH(KK_GEMM, st, pdl_launch(gemm_kernel<256>, grid, Layout<256>::kThreads,
                                         Layout<256>::kSmemAlloc, st, a0, a1, a2, b, p));
@@ -164,6 +177,19 @@ proj100::Params base_params(int M, int N, int K, int T, int D) {
 }  // namespace
 
 extern "C" {
+
+int attn_proj_gemm_plan(int M, int N, int K, int f32_out, int* out) {
+  if (!out || M <= 0 || N <= 0 || K <= 0) return ATTN_EINVAL;
+  const GemmPlan g = plan_gemm(M, N, K, f32_out != 0);
+  if (g.units >= (1L << 31)) return ATTN_EUNSUPPORTED;
+  out[0] = g.bn;
+  out[1] = g.tiles_m;
+  out[2] = g.tiles_n;
+  out[3] = g.splits;
+  out[4] = g.kb_per_split;
+  out[5] = (int)g.ctas;
+  return ATTN_OK;
+}
 
 size_t attn_proj_workspace_bytes(int B, int T, int H, int H_kv, int D) {
   if (!proj_sizes_ok(B, T, 8, H, H_kv, D)) return 0;

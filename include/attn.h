@@ -261,6 +261,13 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
  * the attention's layout) and dw_o = dy^T o. No workspace.
  */
 size_t attn_proj_workspace_bytes(int B, int T, int H, int H_kv, int D);
+/* attn_proj_gemm_plan: how the projection GEMM C[M][N] = sum over K runs
+ * (host arithmetic only, no CUDA call): out[0..5] = tile width BN (128 or
+ * 256), tiles along M and N, K parts (> 1 only for the fp32 weight gradients,
+ * f32_out != 0, whose parts are added into a zeroed output), 64-wide K blocks
+ * per part, and persistent CTAs launched (at most one per SM of a B200).
+ * Returns ATTN_OK, ATTN_EINVAL (null out, a size <= 0) or ATTN_EUNSUPPORTED. */
+int attn_proj_gemm_plan(int M, int N, int K, int f32_out, int* out);
 int attn_qkv_proj(const void* x, const void* w_qkv, const float* rope_cos, const float* rope_sin,
                   const int32_t* cu_seqlens, void* q, void* k, void* v, int B, int T, int C,
                   int H, int H_kv, int D, void* workspace, size_t ws_bytes, void* stream);

@@ -255,3 +255,36 @@ def test_debug_hook_is_absent_from_the_product_library():
         lib = ctypes.CDLL(debug)
         for n in _declared_functions():
             assert hasattr(lib, n), f"{n} missing from the watchdog build"
+
+
+def test_projection_gemm_plan():
+    """The tile width and K split of the projection GEMM (host arithmetic)."""
+    import bwd_causal_sdpa_b200 as A
+
+    def plan(M, N, K, f32):
+        code, p = A.attn_proj_gemm_plan(M, N, K, f32)
+        assert code == A.ATTN_OK
+        return p
+
+    # bf16 outputs never split K; a persistent grid of at most 148 CTAs
+    p = plan(8192, 3072, 2048, False)
+    assert (p["bn"], p["tiles_m"], p["tiles_n"], p["splits"], p["ctas"]) == (256, 64, 12, 1, 148)
+    assert p["kb_per_split"] == 32
+    assert plan(8192, 200, 768, False)["bn"] == 128
+    # fp32 weight gradients of the 8K layer: 192 tiles fill 1.3 rounds of 148
+    # SMs; three K parts make 576 units (97 % of four rounds)
+    p = plan(3072, 2048, 8192, True)
+    assert (p["splits"], p["kb_per_split"], p["ctas"]) == (3, 43, 148)
+    # 128 tiles: the extra reduce traffic of a split costs more than it saves
+    assert plan(2048, 2048, 8192, True)["splits"] == 1
+    # few tiles with a long K (the 237M layer's weights): split
+    assert plan(2304, 768, 8192, True)["splits"] == 2
+    p = plan(768, 768, 8192, True)
+    assert (p["splits"], p["kb_per_split"], p["ctas"]) == (8, 16, 144)
+    # every part gets at least one K block, and no more than K holds
+    for M, N, K in [(128, 8, 64), (320, 200, 512), (192, 8, 128), (100, 100, 100000)]:
+        p = plan(M, N, K, True)
+        nkb = -(-K // 64)
+        assert 1 <= p["splits"] <= nkb and (p["splits"] - 1) * p["kb_per_split"] < nkb
+        assert p["splits"] * p["kb_per_split"] >= nkb
+    assert A.attn_proj_gemm_plan(0, 8, 8, True)[0] == A.ATTN_EINVAL
