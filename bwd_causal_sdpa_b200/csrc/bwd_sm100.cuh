@@ -35,9 +35,9 @@
 // Sources (page, section): ARK README, "Backward pass (AutoGrad)" (attention
 // gradients inside training); Forge README, finding 3 (key-tile-parallel dK/dV
 // kernels, the dK/dV split and register pressure) and "What this is" (fused
-// flash-attention backward). The dQ accumulation follows the measurement
-// contract's "atomic dQ" option (reduce-add in L2). Tiling, TMEM plan and warp
-// roles are this library's own.
+// flash-attention backward). dQ is accumulated by reduce-adds in L2 rather
+// than by a separate query-tile pass, which would recompute S and dP (two more
+// products per tile). Tiling, TMEM plan and warp roles are this library's own.
 #pragma once
 
 #include "sm100.cuh"

@@ -3,8 +3,8 @@
 Shapes and distributions follow the training-layer shapes the source pages
 describe (a 12M GPT at context 512 in the Forge README, the 237M EKO decoder at
 seq 1024 in the ARK README, 2K-8K training windows and packed short documents in
-the Cort33x notes), with the head counts, seeds and value scales of the
-measurement contract this library is benchmarked on.
+the Cort33x notes); the head counts, seeds and value scales are fixed here, per
+workload, so that every run of the tests and the bench draws the same inputs.
 """
 
 from __future__ import annotations
