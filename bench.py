@@ -81,6 +81,9 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sustain", type=float, default=0.0,
+                    help="also time back-to-back steps for about this many seconds and report "
+                         "them against the sustained bf16 peak (clocks and power sampled)")
     return ap.parse_args()
 
 
@@ -130,6 +133,34 @@ def kernel_algorithmic(name: str, w, kinds_seen) -> tuple:
     return "hbm", 0, "byte"
 
 
+def ideal_tiles(w) -> dict:
+    """Tile products (128 queries x 128 keys, per query head) that hold at
+    least one allowed (query, key) pair, and the allowed pairs themselves in
+    tile units. A query tile's allowed keys form one range, from the start
+    of its first row's document to its last row (rows are causal and a
+    document is contiguous), so the tiles holding an allowed pair are exactly
+    the key tiles of that range; the same set, seen from a key tile, is the
+    query tiles from its own to the one holding its last key's document end.
+    This is the least work block skipping can do at this tile size."""
+    import numpy as np
+
+    T, B, H = w.T, w.B, w.H
+    nt = (T + 127) // 128
+    tiles = 0
+    for b in range(B):
+        ds = np.zeros(T, dtype=np.int64)
+        if w.cu_seqlens is not None:
+            cu = w.cu_seqlens.astype(np.int64)
+            row = cu[(cu >= b * T) & (cu <= (b + 1) * T)] - b * T
+            for a, e in zip(row[:-1], row[1:]):
+                ds[a:e] = a
+        first = np.arange(nt) * 128
+        tiles += int(np.sum(np.arange(nt) - ds[first] // 128 + 1))
+    L = np.asarray(w.doc_lengths(), dtype=np.float64)
+    allowed = float(np.sum(L * (L + 1) / 2))
+    return {"ideal": tiles * H, "allowed_pairs_in_tiles": allowed * H / (128 * 128)}
+
+
 # ---------------------------------------------------------------------------
 # Clock sampling (NVML, read-only) during the timed region
 # ---------------------------------------------------------------------------
@@ -142,6 +173,7 @@ class ClockSampler:
     def __init__(self, index: int, period_s: float = 0.02):
         self.index, self.period = index, period_s
         self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.power_w = []
         self._stop = threading.Event()
         self._thr = None
         self.error = None
@@ -164,6 +196,7 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.power_w.append(nv.nvmlDeviceGetPowerUsage(self._h) / 1000.0)
                 mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h) \
                     if hasattr(nv, "nvmlDeviceGetCurrentClocksEventReasons") \
                     else nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
@@ -185,7 +218,9 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
                     "samples": 0, "error": self.error}
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples),
+                "power_w_median": statistics.median(self.power_w) if self.power_w else None,
+                "power_w_max": max(self.power_w) if self.power_w else None}
 
 
 # ---------------------------------------------------------------------------
@@ -377,6 +412,7 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     barrier()
     torch.cuda.synchronize(dev)
+    A.check(A.attn_tile_counts()[0], "attn_tile_counts")  # reset the device counters
     n0 = A.attn_launch_count()
     with ClockSampler(local) as clocks:
         with torch.cuda.stream(stream):
@@ -390,6 +426,15 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize(dev)
     launches = A.attn_launch_count() - n0
+    code, fwd_tiles, bwd_tiles = A.attn_tile_counts()
+    A.check(code, "attn_tile_counts")
+    tiles = None
+    if w.dtype == "bf16":
+        tiles = ideal_tiles(w)
+        tiles.update(fwd_executed=fwd_tiles / args.steps, bwd_executed=bwd_tiles / args.steps)
+        tiles["fwd_over_ideal"] = tiles["fwd_executed"] / tiles["ideal"]
+        tiles["bwd_over_ideal"] = tiles["bwd_executed"] / tiles["ideal"]
+        tiles["unit"] = "128x128 tile products per step, all query heads (device counters)"
     step_ms = [a.elapsed_time(b) for a, b in ev]
     # Per-kernel times for the roofline come from a second pass over the same
     # number of steps with an event pair around every launch (kept out of the
@@ -529,6 +574,36 @@ def run_ours(args):
                "serial_ms_per_step": s_ms}
         del r2, sets
 
+    sustained = None
+    if args.sustain > 0:
+        # back-to-back steps for about args.sustain seconds (steps sized from
+        # the timed region), same step and flush as above, so the GPU reaches
+        # its power-limited clocks; reported against the sustained peak
+        n_sus = max(1, int(args.sustain * 1e3 / (ms_local + 0.05)))
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_sus)]
+        torch.cuda.synchronize(dev)
+        barrier()
+        with ClockSampler(local, period_s=0.05) as sclk:
+            with torch.cuda.stream(stream):
+                for i in range(n_sus):
+                    flush.zero_()
+                    evs[i][0].record(stream)
+                    r.forward()
+                    r.backward()
+                    evs[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+        barrier()
+        s_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / n_sus, world, dev)
+        s_val = whole_job_tflops(flops_step, world, s_ms)
+        sustained = {"value": s_val, "unit": UNIT, "steps": n_sus, "ms_per_step": s_ms,
+                     "timed_seconds": n_sus * s_ms / 1e3,
+                     "frac_of_bf16_sustained": s_val / world / peaks["bf16_tflops_sustained"],
+                     "frac_of_bf16_burst": s_val / world / peaks["bf16_tflops"],
+                     "clocks": sclk.summary()}
+        if r.status() != A.ATTN_OK:
+            raise SystemExit("device status after the sustained run is not OK")
+
     cpu = None
     parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -557,7 +632,7 @@ def run_ours(args):
             "pct_of_bf16_peak_sustained": value / world / peaks["bf16_tflops_sustained"],
             "peaks_source": peak_src,
             "value_within_documents": w.algorithmic_flops() * world / (ms / 1e3) / 1e12,
-            "roofline": roofline, "kernels": kernels,
+            "roofline": roofline, "kernels": kernels, "tiles": tiles, "sustained": sustained,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clocks.summary(), "parity": parity,
         }

@@ -62,6 +62,7 @@ _SIGNATURES = {
     "attn_exp2_selftest": (_I, [_P, _P, _I, _P]),
     "attn_debug_withhold": (_I, [_I]),
     "attn_launch_count": (ctypes.c_ulonglong, []),
+    "attn_tile_counts": (_I, [ctypes.POINTER(ctypes.c_ulonglong), ctypes.POINTER(ctypes.c_ulonglong)]),
     "attn_profile_enable": (_I, [_I]),
     "attn_profile_kinds": (_I, []),
     "attn_profile_read": (_I, [_I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_I),
@@ -235,6 +236,15 @@ def attn_debug_withhold(what) -> int:
 
 def attn_launch_count() -> int:
     return int(_lib.attn_launch_count())
+
+
+def attn_tile_counts():
+    """(code, fwd_tiles, bwd_tiles): tile products the tensor-core kernels
+    executed since the previous read (counted on the device; resets them)."""
+    f = ctypes.c_ulonglong()
+    b = ctypes.c_ulonglong()
+    code = int(_lib.attn_tile_counts(ctypes.byref(f), ctypes.byref(b)))
+    return code, int(f.value), int(b.value)
 
 
 def attn_profile_enable(on) -> int:

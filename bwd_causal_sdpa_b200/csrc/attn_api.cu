@@ -27,8 +27,11 @@ struct WsPlan {
   size_t delta = 0;                   // f32 [B*H*T] (f32 backward) or [B*H*Tpad] (bf16 backward)
   size_t lse2 = 0;                    // f32 [B*H*Tpad] lse*log2(e) (bf16 backward)
   size_t dq_acc = 0;                  // f32 [B*H*T*D] dq accumulator (bf16 backward)
-  size_t q16 = 0, k16 = 0;            // rotated q, k as 16-bit [B*H*T*D] each (bf16 storage)
-  size_t qfac = 0, kfac = 0;          // f32 [B*H*ceil(T/128)] tile factors (bf16 forward)
+  size_t q16 = 0, k16 = 0;            // rotated q, k as fp16 [B*H*T*D] each (bf16 storage)
+  size_t qfac = 0, kfac = 0;          // f32 [B*H*ceil(T/128)] inverse tile factors (bf16 forward)
+  size_t qinv = 0, kinv = 0;          // inverse q / k tile factors (bf16 backward): q as f32
+                                      // [B*H*ceil(T/128)][4] records, k as f32 [B*Hkv*ceil(T/128)]
+  size_t dmax = 0, deltamax = 0;      // f32 [B*H*ceil(T/128)] per-tile max |dO_i|, |Delta_i| (bf16 backward)
   size_t dk_acc = 0, dv_acc = 0;      // f32 [B*Hkv*T*D] each when the backward splits groups
   int split = 1;                      // query-head groups split over this many CTAs
   size_t total = 0;
@@ -73,6 +76,10 @@ WsPlan plan(int B, int H, int T, int D, int dtype, int is_bwd, int Hkv = 0) {
     p.dq_acc = off; off += round_up(n * sizeof(float));
     p.q16 = off;    off += round_up(n * 2);
     p.k16 = off;    off += round_up(n * 2);
+    p.qinv = off;     off += round_up(tiles * 4 * sizeof(float));
+    p.kinv = off;     off += round_up(tiles * sizeof(float));
+    p.dmax = off;     off += round_up(tiles * sizeof(float));
+    p.deltamax = off; off += round_up(tiles * sizeof(float));
     p.split = choose_split(B, H, Hkv, T);
     if (p.split > 1) {
       const size_t nkv = bt * Hkv * D;
@@ -217,22 +224,24 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
            char* ws, const WsPlan& wp, cudaStream_t st) {
   using L = fwd100::Layout<D>;
   const int nt = (T + 127) / 128, BH = B * H, BHkv = B * Hkv;
+  // With RoPE q and k are rotated once into fp16 tiles with power-of-two
+  // factors (rope_prep); without it the kernel reads them as given (bf16).
   const void* qs = q;
   const void* ks = k;
-  bool f16 = false;
   float *qf = nullptr, *kf = nullptr;
   if (rc) {
     __half* qh = (__half*)(ws + wp.q16);
     __half* kh = (__half*)(ws + wp.k16);
     qf = (float*)(ws + wp.qfac);
     kf = (float*)(ws + wp.kfac);
-    ATTN_LAUNCH(KK_ROPE_PREP, st, pdl_launch(rope_prep_kernel<__half, D, true>, dim3(nt, BH, 2), kRopePrepThreads, 0, st, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qh, kh, qf, kf,
-                    H, Hkv, T, nt));
+    ATTN_LAUNCH(KK_ROPE_PREP, st, pdl_launch(rope_prep_kernel<D>, dim3(nt, BH, 2), kRopePrepThreads, 0, st,
+                                             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds,
+                                             qh, kh, qf, kf, B, H, Hkv, T, nt));
     if (launch_status()) return ATTN_ECUDA;
     qs = qh;
     ks = kh;
-    f16 = true;
   }
+  const bool f16 = rc != nullptr;
   CUtensorMap mq, mk, mv;
   if (!make_tile_map(&mq, qs, f16, D, T, BH) || !make_tile_map(&mk, ks, f16, D, T, BHkv) ||
       !make_tile_map(&mv, v, false, D, T, BHkv))
@@ -258,35 +267,64 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
   return launch_status();
 }
 
+template <int D, bool kF16>
+int launch_dkdv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                const CUtensorMap& mo, const CUtensorMap& mdq, const bwd100::Params& prm,
+                unsigned grid, cudaStream_t st) {
+  using L = bwd100::Layout<D>;
+  static bool smem_set[64] = {};
+  if (!ensure_smem(bwd100::dkdv_kernel<D, kF16>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
+  ATTN_LAUNCH(KK_DKDV, st, pdl_launch(bwd100::dkdv_kernel<D, kF16>, grid, L::kThreads,
+                                       L::kSmemAlloc, st, mq, mk, mv, mo, mdq, prm));
+  return launch_status();
+}
+
 template <int D>
 int bwd_tc(const void* q, const void* k, const void* v, const void* o, const void* dO,
            const float* lse, const float* rc, const float* rs, const int32_t* ds,
            const int32_t* de, void* dq, void* dk, void* dv, int B, int H, int Hkv, int T,
            float scale, char* ws, const WsPlan& wp, cudaStream_t st) {
-  using L = bwd100::Layout<D>;
   const int nt = (T + 127) / 128, BH = B * H, BHkv = B * Hkv, Tpad = nt * 128;
-  __nv_bfloat16* qr = (__nv_bfloat16*)(ws + wp.q16);
-  __nv_bfloat16* kr = (__nv_bfloat16*)(ws + wp.k16);
-  const void* qs = rc ? (const void*)qr : q;
-  const void* ks = rc ? (const void*)kr : k;
+  // With RoPE the scores are recomputed from fp16 operands (the rotated q, k
+  // with per-tile factors, as the forward computed them); without it from q,
+  // k as given (bf16).
+  const bool f16 = rc != nullptr;
+  __half* q16 = (__half*)(ws + wp.q16);
+  __half* k16 = (__half*)(ws + wp.k16);
+  const void* qs = f16 ? (const void*)q16 : q;
+  const void* ks = f16 ? (const void*)k16 : k;
   float* delta = (float*)(ws + wp.delta);
   float* lse2 = (float*)(ws + wp.lse2);
   float* dq_acc = (float*)(ws + wp.dq_acc);
-  const long rows_pad = (long)BH * Tpad;
+  float* qinv = (float*)(ws + wp.qinv);
+  float* kinv = (float*)(ws + wp.kinv);
+  float* dmax = (float*)(ws + wp.dmax);
+  float* deltamax = (float*)(ws + wp.deltamax);
   const int split = wp.split;
   float* dk_acc = split > 1 ? (float*)(ws + wp.dk_acc) : nullptr;
   float* dv_acc = split > 1 ? (float*)(ws + wp.dv_acc) : nullptr;
-  ATTN_LAUNCH(KK_DELTA, st, pdl_launch(bwd_prep_kernel<D>, (unsigned)(rows_pad * (D / 8) / 256), 256, 0, st, (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse, delta, lse2, dq_acc,
-                  (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds, qr, kr, dk_acc,
-                  dv_acc, H, Hkv, T, Tpad, rows_pad));
+  const dim3 pgrid(nt, BH);
+  if (f16) {
+    ATTN_LAUNCH(KK_DELTA, st, pdl_launch(bwd_prep_kernel<D, true>, pgrid, kBwdPrepThreads, 0, st,
+                                         (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse,
+                                         delta, lse2, dq_acc, (const __nv_bfloat16*)q,
+                                         (const __nv_bfloat16*)k, rc, rs, ds, q16, k16, qinv,
+                                         kinv, dmax, deltamax, dk_acc, dv_acc, B, H, Hkv, T, Tpad,
+                                         nt));
+  } else {
+    ATTN_LAUNCH(KK_DELTA, st, pdl_launch(bwd_prep_kernel<D, false>, pgrid, kBwdPrepThreads, 0, st,
+                                         (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse,
+                                         delta, lse2, dq_acc, (const __nv_bfloat16*)q,
+                                         (const __nv_bfloat16*)k, rc, rs, ds, q16, k16, qinv,
+                                         kinv, dmax, deltamax, dk_acc, dv_acc, B, H, Hkv, T, Tpad,
+                                         nt));
+  }
   if (launch_status()) return ATTN_ECUDA;
   CUtensorMap mq, mk, mv, mo, mdq;
-  if (!make_tile_map(&mq, qs, false, D, T, BH) || !make_tile_map(&mk, ks, false, D, T, BHkv) ||
+  if (!make_tile_map(&mq, qs, f16, D, T, BH) || !make_tile_map(&mk, ks, f16, D, T, BHkv) ||
       !make_tile_map(&mv, v, false, D, T, BHkv) || !make_tile_map(&mo, dO, false, D, T, BH) ||
       !make_acc_map(&mdq, dq_acc, D, T, BH))
     return ATTN_ECUDA;
-  static bool smem_set[64] = {};
-  if (!ensure_smem(bwd100::dkdv_kernel<D>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
   bwd100::Params prm;
   prm.T = T;
   prm.H = H;
@@ -308,9 +346,14 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   prm.dv = (__nv_bfloat16*)dv;
   prm.dk_acc = dk_acc;
   prm.dv_acc = dv_acc;
-  ATTN_LAUNCH(KK_DKDV, st, pdl_launch(bwd100::dkdv_kernel<D>, (unsigned)(nt * BHkv * split), L::kThreads, L::kSmemAlloc,
-                                       st, mq, mk, mv, mo, mdq, prm));
-  if (launch_status()) return ATTN_ECUDA;
+  prm.qinv = qinv;
+  prm.kinv = kinv;
+  prm.dmax = dmax;
+  prm.deltamax = deltamax;
+  const unsigned grid = (unsigned)(nt * BHkv * split);
+  const int rc_k = f16 ? launch_dkdv<D, true>(mq, mk, mv, mo, mdq, prm, grid, st)
+                       : launch_dkdv<D, false>(mq, mk, mv, mo, mdq, prm, grid, st);
+  if (rc_k) return rc_k;
   if (split > 1) {
     // dk = R^T (scale * sum of the parts), dv = sum of the parts
     const long n8kv = (long)BHkv * T * D / 8;
@@ -455,6 +498,18 @@ const char* attn_error_string(int code) {
 }
 
 unsigned long long attn_launch_count(void) { return trace::launches(); }
+
+int attn_tile_counts(unsigned long long* fwd_tiles, unsigned long long* bwd_tiles) {
+  if (!fwd_tiles || !bwd_tiles) return ATTN_EINVAL;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ECUDA;
+  unsigned long long v[2] = {0, 0};
+  if (cudaMemcpyFromSymbol(v, g_attn_tiles, sizeof(v)) != cudaSuccess) return ATTN_ECUDA;
+  const unsigned long long z[2] = {0, 0};
+  if (cudaMemcpyToSymbol(g_attn_tiles, z, sizeof(z)) != cudaSuccess) return ATTN_ECUDA;
+  *fwd_tiles = v[0];
+  *bwd_tiles = v[1];
+  return ATTN_OK;
+}
 
 int attn_exp2_selftest(const float* x, float* y, int n, void* stream) {
   if (!x || !y || n < 0) return ATTN_EINVAL;
@@ -627,35 +682,65 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_dev_ptr[kNoAllocMaxDevices] = {};
+CUcontext g_noalloc_ctx[kNoAllocMaxDevices] = {};
 
-// Scratch layout: document starts, document ends (int32 [B*T] each), then
-// Delta (f32 [B*H*T]); each part starts on a 256-byte boundary.
+// Scratch layout: Delta (f32 [B*H*T]) at offset 0, then, only when documents
+// are packed (cu_seqlens given), the document starts and ends (int32 [B*T]
+// each); each part starts on a 256-byte boundary.
 struct NoAllocPlan {
-  size_t doc_start, doc_end, delta, total;
+  size_t delta, doc_start, doc_end, total;
 };
 
-NoAllocPlan noalloc_plan(int B, int H, int T) {
+NoAllocPlan noalloc_plan(int B, int H, int T, bool packed) {
   NoAllocPlan p;
   const size_t bt = (size_t)B * T;
-  p.doc_start = 0;
-  p.doc_end = round_up(bt * sizeof(int32_t));
-  p.delta = p.doc_end + round_up(bt * sizeof(int32_t));
-  p.total = p.delta + round_up(bt * (size_t)H * sizeof(float));
+  p.delta = 0;
+  p.total = round_up(bt * (size_t)H * sizeof(float));
+  p.doc_start = p.doc_end = 0;
+  if (packed) {
+    p.doc_start = p.total;
+    p.doc_end = p.doc_start + round_up(bt * sizeof(int32_t));
+    p.total = p.doc_end + round_up(bt * sizeof(int32_t));
+  }
   return p;
 }
 
-// Device address of the scratch array on the current device; the first call
-// per device does the lookup (with that device current).
+// The current context, through the driver entry point the runtime exposes
+// (the library links no driver library); null if it cannot be queried.
+CUcontext current_context() {
+  typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+  static CtxGetCurrentFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (CtxGetCurrentFn)f;
+  }
+  CUcontext c = nullptr;
+  if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+  return c;
+}
+
+// Device address of the scratch array on the current device. The lookup is
+// done once per device, with that device current, and again whenever the
+// device's context has changed since (after a cudaDeviceReset the module is
+// loaded anew and the array may sit at a new address).
 int noalloc_scratch(char** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
     return ATTN_ECUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_dev_ptr[dev] == nullptr) {
+  CUcontext ctx = current_context();
+  if (g_noalloc_dev_ptr[dev] == nullptr || ctx == nullptr || g_noalloc_ctx[dev] != ctx) {
+    // (also makes the device's primary context current if none is yet)
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return ATTN_ECUDA;
     g_noalloc_dev_ptr[dev] = p;
+    g_noalloc_ctx[dev] = current_context();
   }
   *out = (char*)g_noalloc_dev_ptr[dev];
   return ATTN_OK;
@@ -679,7 +764,7 @@ extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, con
       !aligned(lse, 4) || (rope_cos && !aligned(rope_cos, 16)) ||
       (rope_sin && !aligned(rope_sin, 16)) || (cu_seqlens && !aligned(cu_seqlens, 4)))
     return ATTN_EALIGN;
-  const NoAllocPlan p = noalloc_plan(B, H, T);
+  const NoAllocPlan p = noalloc_plan(B, H, T, cu_seqlens != nullptr);
   if (p.total > kNoAllocBytes) return ATTN_ESCRATCH;
 
   char* ws = nullptr;

@@ -32,6 +32,21 @@
 // (R^T) in the epilogue; dq is finished by a separate kernel once every key
 // tile has added its part.
 //
+// Operand types. Without RoPE every product reads bf16 (q, k as given, P^T
+// and dS^T rounded to bf16). With RoPE (kF16) the scores are recomputed from
+// the forward's own operands: the rotated q, k stored as fp16 times a
+// power-of-two factor per 128-row tile (the backward preprocessing writes the
+// same values the forward computed), so P matches the forward's lse. The
+// products that pair dS with those operands (dK = dS^T Q, dQ = dS K) then
+// need dS in fp16 as well, stored as dS * C * qinv_i: qinv_i (the inverse of
+// query tile i's factor) cancels that tile's factor in dK, which therefore
+// accumulates C dS^T Q for every tile, and C, a power of two per CTA, keeps
+// every stored value below 2^14 (from |dS_ij| <= |dO_i| max_j |v_j| +
+// |Delta_i|, the per-tile maxima the preprocessing recorded and this CTA's
+// own value rows). dK is divided by C in the epilogue and each dQ_i tile by
+// C qinv_i / kinv (kinv: this key tile's factor) before it is added. P^T and
+// dO stay bf16 for dV, and V, dO for dP.
+//
 // Sources (page, section): ARK README, "Backward pass (AutoGrad)" (attention
 // gradients inside training); Forge README, finding 3 (key-tile-parallel dK/dV
 // kernels, the dK/dV split and register pressure) and "What this is" (fused
@@ -59,14 +74,20 @@ struct Layout {
   static constexpr int kLD = kPS + 128 * 128 * 2;             // 2 x {-lse2[128], -delta[128]} f32
   // dQ_i staging ring: two buffers of 128 query rows x 32 fp32 columns, each
   // four 32 x 32 boxes (4 KB, 128-byte swizzle), one per dQ warp.
-  static constexpr int kXS = kLD + 2 * 1024;
+  static constexpr int kXS = kLD + 2 * 1024;  // 1024-byte aligned (128-byte swizzle)
   static constexpr int kXSBuf = 128 * 32 * 4;
-  static constexpr int kBars = kXS + 2 * kXSBuf;
+  // per elementwise warp: largest qinv, |dO_i|, |Delta_i| of this CTA's query
+  // tiles and of its key rows' value norms over its columns (f32 [16][4])
+  static constexpr int kStats = kXS + 2 * kXSBuf;
+  // per Q stage: the query tile's inverse factor record (16 bytes, qinv first)
+  static constexpr int kQInv = kStats + 16 * 4 * 4;
+  static constexpr int kBars = kQInv + 2 * 16;
   static constexpr int bKV = 0;
   static constexpr int bQFull = 1, bQEmpty = 3, bDOFull = 5, bDOEmpty = 7;  // 2 each
   static constexpr int bSFull = 9, bSFree = 10, bPFull = 11, bDPFull = 12, bDSFull = 13,
-                       bDVDone = 14, bDQFull = 15, bDSFree = 16, bDQFree = 17, bFinal = 18;
-  static constexpr int kNumBars = 19;
+                       bDVDone = 14, bDQFull = 15, bDSFree = 16, bDQFree = 17, bFinal = 18,
+                       bStats = 19;
+  static constexpr int kNumBars = 20;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
   // The dynamic shared-memory window starts 1024-byte aligned on sm_100 (after
@@ -85,6 +106,8 @@ struct Layout {
   static constexpr int kDqWarp0 = 4 * kNWG;  // the dQ warpgroup: warps kDqWarp0 .. +3
   static constexpr int kProducerWarp = 4 * kNWG + 4, kMmaWarp = 4 * kNWG + 5;
   static constexpr int kThreads = kEwThreads + 128 + 64;
+  static_assert(kXS % 1024 == 0, "the dQ staging boxes use the 128-byte swizzle");
+  static_assert(kBytes <= 232448, "more shared memory than a CTA may use");
 };
 
 struct Params {
@@ -103,7 +126,22 @@ struct Params {
   __nv_bfloat16* dv;
   float* dk_acc;           // [B*Hkv][T][D] fp32 (n_split > 1: the parts are added here)
   float* dv_acc;
+  // fp16 operands (RoPE): inverse tile factors of the stored q, one 16-byte
+  // record per tile ([B*H][n_tiles][4], value first), and of the stored k
+  // ([B*Hkv][n_tiles]), and per query tile the largest |dO_i| and |Delta_i|
+  const float* qinv;
+  const float* kinv;
+  const float* dmax;
+  const float* deltamax;
 };
+
+// The power of two C that keeps every stored dS * C * qinv_i below 2^14,
+// from X = max qinv_i * (max |dO_i| * max |v_j| + max |Delta_i|) >= max
+// |dS_ij| qinv_i; 1 when X is zero (dS is then zero too).
+__device__ __forceinline__ float ds_scale(float X) {
+  if (!(X > 0.f && X <= 3.0e38f)) return 1.f;
+  return ldexpf(1.f, max(-100, min(100, 13 - ilogbf(X))));
+}
 
 // Byte offset of 16-byte chunk `ch` (0..7 within a 64-column block) of row r
 // in a 128-byte-swizzled tile block.
@@ -111,7 +149,7 @@ __device__ __forceinline__ uint32_t sw128(int r, int ch) {
   return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4));
 }
 
-template <int D>
+template <int D, bool kF16>
 __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -167,8 +205,10 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     mbar_init(bar(L::bDSFree), 1);
     mbar_init(bar(L::bDQFree), 128);
     mbar_init(bar(L::bFinal), 1);
+    mbar_init(bar(L::bStats), L::kEwThreads);
     *abort_flag = 0;
     fence_barrier_init();
+    atomicAdd(&g_attn_tiles[1], (unsigned long long)n_it);
   }
   if (warp == L::kMmaWarp) {
     tmem_alloc(sb0 + L::kMisc, L::kTmemCols);
@@ -178,6 +218,27 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // fp16 operands: this key tile's inverse factor, and C from the posted
+  // statistics (every thread that needs it derives the same value)
+  const float kinv_cta = kF16 ? p.kinv[(size_t)bhk * p.n_tiles + kt] : 1.f;
+  float* stats = reinterpret_cast<float*>(sg + L::kStats);  // [warp][4]
+  auto cta_ds_scale = [&]() -> float {
+    float qm = 0.f, dm = 0.f, dl = 0.f, vb = 0.f;
+#pragma unroll
+    for (int g = 0; g < L::kNWG; ++g) {
+      float vg = 0.f;
+#pragma unroll
+      for (int w4 = 0; w4 < 4; ++w4) {
+        const float* e = stats + 4 * (4 * g + w4);
+        qm = fmaxf(qm, e[0]);
+        dm = fmaxf(dm, e[1]);
+        dl = fmaxf(dl, e[2]);
+        vg = fmaxf(vg, e[3]);
+      }
+      vb += vg;  // |v_j| <= sum over the column groups of their largest partial norms
+    }
+    return ds_scale(qm * fmaf(dm, vb, dl));
+  };
 
   if (warp == L::kProducerWarp) {
     // ---------------- TMA producer ----------------
@@ -202,14 +263,16 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
           const int gi = nq / n_q;
           const int bh = bhq0 + gi;
           const int qrow = (qt0 + nq - gi * n_q) * 128;
-          mbar_arrive_expect_tx(bar(L::bQFull + st), L::kTileBytes + 1024);
+          mbar_arrive_expect_tx(bar(L::bQFull + st), L::kTileBytes + 1024 + (kF16 ? 16 : 0));
           for (int cb = 0; cb < D / 64; ++cb)
             tma_load_3d(sb0 + L::kQ + st * L::kTileBytes + cb * L::kBlockBytes, &tmQ,
                         bar(L::bQFull + st), cb * 64, qrow, bh);
-          bulk_load(sb0 + L::kLD + st * 1024, p.lse2 + (size_t)bh * p.Tpad + qrow, 512,
-                    bar(L::bQFull + st));
-          bulk_load(sb0 + L::kLD + st * 1024 + 512, p.delta + (size_t)bh * p.Tpad + qrow, 512,
-                    bar(L::bQFull + st));
+          const uint32_t ld = sb0 + L::kLD + st * 1024;
+          bulk_load(ld, p.lse2 + (size_t)bh * p.Tpad + qrow, 512, bar(L::bQFull + st));
+          bulk_load(ld + 512, p.delta + (size_t)bh * p.Tpad + qrow, 512, bar(L::bQFull + st));
+          if (kF16)
+            bulk_load(sb0 + L::kQInv + st * 16, p.qinv + ((size_t)bh * p.n_tiles + (qrow >> 7)) * 4,
+                      16, bar(L::bQFull + st));
           ++nq;
           did = true;
         }
@@ -258,10 +321,11 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     // Every barrier probed for phase k has been seen complete for phase k-1,
     // so the parity probes are unambiguous.
     if (lane == 0) {
-      constexpr uint32_t id_s = idesc_f16(128, 128, true, true, false, false);
+      constexpr uint32_t id_s = idesc_f16(128, 128, !kF16, !kF16, false, false);
+      constexpr uint32_t id_dp = idesc_f16(128, 128, true, true, false, false);
       constexpr uint32_t id_dv = idesc_f16(128, D, true, true, false, true);
-      constexpr uint32_t id_dk = idesc_f16(128, D, true, true, false, true);
-      constexpr uint32_t id_dq = idesc_f16(128, D, true, true, true, true);
+      constexpr uint32_t id_dk = idesc_f16(128, D, !kF16, !kF16, false, true);
+      constexpr uint32_t id_dq = idesc_f16(128, D, !kF16, !kF16, true, true);
       const uint32_t tS = tmem + L::kColS, tDP = tmem + L::kColDP;
       const uint32_t tDV = tmem + L::kColDV, tDK = tmem + L::kColDK;
       const uint32_t ps = sb0 + L::kPS;
@@ -327,7 +391,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
             mma_ss(tDP, smem_desc_sw128(sb0 + L::kV + off, 16, 1024),
-                   smem_desc_sw128(obuf(nP) + off, 16, 1024), id_s, kk > 0);
+                   smem_desc_sw128(obuf(nP) + off, 16, 1024), id_dp, kk > 0);
           }
           mma_commit(bar(L::bDPFull));
           ++nP;
@@ -356,10 +420,20 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     constexpr int NCH = D / 32;
     int chunk = 0;
     bool prev_issued = false;  // did this warp reduce the previous chunk
-    for (int it = 0; it < n_it; ++it) {
+    float cscale = 1.f;
+    bool okq = true;
+    if constexpr (kF16) {
+      okq = mbar_wait(bar(L::bStats), 0, abort_flag);
+      if (okq) cscale = cta_ds_scale();
+    }
+    for (int it = 0; okq && it < n_it; ++it) {
       const int gi = it / n_q;
       const int i0 = (qt0 + it - gi * n_q) * 128;
       const bool rows_in = i0 + 32 * sub < T;  // rows past T are clipped by the map
+      // dQ_i as computed from the scaled operands, back to dS K
+      const float mulq =
+          kF16 ? kinv_cta / (cscale * p.qinv[((size_t)(bhq0 + gi) * p.n_tiles + (i0 >> 7)) * 4])
+               : 1.f;
       if (!mbar_wait(bar(L::bDQFull), it & 1, abort_flag)) break;
       tc_fence_after();
 #pragma unroll 1
@@ -378,6 +452,10 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         }
         __syncwarp();
         uint8_t* bx = sg + L::kXS + buf * L::kXSBuf + sub * 4096;
+        if constexpr (kF16) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * mulq);
+        }
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           *reinterpret_cast<uint4*>(bx + sw128(lane, e)) =
@@ -407,6 +485,52 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     const uint32_t tDP = tmem + lane_base + L::kColDP;
     uint8_t* psb = sg + L::kPS;
     float pf[QC];  // P^T of this thread's key row, query columns [qc0, qc0 + QC)
+    bool ok = true;
+    float cscale = 1.f;  // C (fp16 operands)
+    float qinv_i = 1.f;  // inverse factor of the current query tile (fp16 operands)
+    if constexpr (kF16) {
+      // Post this warp's share of the statistics C is made from: the largest
+      // qinv, |dO_i| and |Delta_i| over this CTA's query tiles, and the
+      // largest norm of this warpgroup's columns of the value rows.
+      float qm = 0.f, dm = 0.f, dl = 0.f;
+      for (int e = threadIdx.x; e < n_it; e += L::kEwThreads) {
+        const int gi = e / n_q;
+        const size_t ix = (size_t)(bhq0 + gi) * p.n_tiles + qt0 + (e - gi * n_q);
+        qm = fmaxf(qm, p.qinv[ix * 4]);
+        dm = fmaxf(dm, p.dmax[ix]);
+        dl = fmaxf(dl, p.deltamax[ix]);
+      }
+      float vn = 0.f;
+      ok = mbar_wait(bar(L::bKV), 0, abort_flag);
+      if (ok) {
+        const uint8_t* vb = sg + L::kV + (dc0 >> 6) * L::kBlockBytes;
+#pragma unroll
+        for (int e = 0; e < DC / 8; ++e) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(vb + sw128(r, ((dc0 & 63) >> 3) + e));
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+          for (int q2 = 0; q2 < 4; ++q2) {
+            const float a = __low2float(h[q2]), b2 = __high2float(h[q2]);
+            vn = fmaf(a, a, fmaf(b2, b2, vn));
+          }
+        }
+        vn = sqrtf(vn);
+      }
+      qm = warp_max(qm);
+      dm = warp_max(dm);
+      dl = warp_max(dl);
+      vn = warp_max(vn);
+      if (lane == 0) {
+        float* e = stats + 4 * warp;
+        e[0] = qm;
+        e[1] = dm;
+        e[2] = dl;
+        e[3] = vn;
+      }
+      mbar_arrive(bar(L::bStats));
+      ok = ok && mbar_wait(bar(L::bStats), 0, abort_flag);
+      if (ok) cscale = cta_ds_scale();
+    }
     // Row r, query columns [qc0, qc0 + QC) of the P/dS tile (bf16 pairs in
     // w[]): 64-column block col/64, 16-byte chunks (col%64)/8 onwards.
     auto store_row = [&](const uint32_t* w) {
@@ -437,7 +561,13 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(L::bSFree));  // the S^T columns may take the next tile
-      const float2 scl2 = make_float2(p.scale_log2, p.scale_log2);
+      float scl = p.scale_log2;
+      if constexpr (kF16) {
+        // loaded with this tile's lse2 and Delta rows
+        qinv_i = *reinterpret_cast<const float*>(sg + L::kQInv + (i & 1) * 16);
+        scl *= kinv_cta * qinv_i;  // the stored operands carry the tile factors
+      }
+      const float2 scl2 = make_float2(scl, scl);
 #pragma unroll
       for (int e = 0; e < QC / 2; ++e) {
         const int col = qc0 + 2 * e;
@@ -475,12 +605,20 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       for (int c = 0; c < QC / 32; ++c) tmem_ld32(tDP + qc0 + 32 * c, dpv + 32 * c);
       tmem_wait_ld();
       uint32_t w[QC / 2];
+      const float dsm = cscale * qinv_i;  // 1 for bf16 operands
+      const float2 dsm2 = make_float2(dsm, dsm);
 #pragma unroll
       for (int e = 0; e < QC / 2; ++e) {
         const float2 nd = reinterpret_cast<const float2*>(sd + qc0)[e];  // -Delta pair
         const float2 dpp = make_float2(__uint_as_float(dpv[2 * e]), __uint_as_float(dpv[2 * e + 1]));
-        const float2 a = __fmul2_rn(make_float2(pf[2 * e], pf[2 * e + 1]), __fadd2_rn(dpp, nd));
-        w[e] = pack_bf16(a.x, a.y);
+        if constexpr (kF16) {
+          const float2 a = __fmul2_rn(make_float2(pf[2 * e], pf[2 * e + 1]),
+                                      __fmul2_rn(__fadd2_rn(dpp, nd), dsm2));
+          w[e] = pack_half(a.x, a.y);
+        } else {
+          const float2 a = __fmul2_rn(make_float2(pf[2 * e], pf[2 * e + 1]), __fadd2_rn(dpp, nd));
+          w[e] = pack_bf16(a.x, a.y);
+        }
       }
       if (!mbar_wait(bar(L::bDVDone), i & 1, abort_flag)) return false;
       store_row(w);
@@ -489,7 +627,6 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       mbar_arrive(bar(L::bDSFull));
       return true;
     };
-    bool ok = true;
     for (int it = 0; ok && it < n_it; ++it) ok = phase_P(it) && phase_dS(it);
     // ---- epilogue: dK = R^T (scale * dK_r), dV ----
     if (ok && mbar_wait(bar(L::bFinal), 0, abort_flag)) {
@@ -503,6 +640,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         if constexpr (CW == 32) tmem_ld32(taddr, v);
         else tmem_ld16(taddr, v);
       };
+      const float inv_c = 1.f / cscale;  // dK accumulated C dS^T Q (exact power of two)
       if (p.n_split > 1) {
         // this CTA's part of dK_r and dV: added into the fp32 accumulators
         // (scale and R^T are applied by the finishing pass)
@@ -515,6 +653,10 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
           ld(tmem + lane_base + L::kColDK + col, v);
           ld(tmem + lane_base + L::kColDV + col, u);
           tmem_wait_ld();
+          if constexpr (kF16) {
+#pragma unroll
+            for (int e = 0; e < CW; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * inv_c);
+          }
           if (j < T) {
 #pragma unroll
             for (int e = 0; e < CW / 4; ++e) {
@@ -532,7 +674,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         tmem_wait_ld();
         float f[CW];
 #pragma unroll
-        for (int e = 0; e < CW; ++e) f[e] = __uint_as_float(v[e]) * p.scale;
+        for (int e = 0; e < CW; ++e) f[e] = __uint_as_float(v[e]) * (p.scale * inv_c);
         if (p.rope_cos) rope_pairs<CW, D>(f, p.rope_cos, p.rope_sin, pos, col, true);
         if (j < T) {
 #pragma unroll

@@ -21,6 +21,12 @@ __device__ __forceinline__ void report_status(int code) {
   atomicCAS(&g_attn_status, 0, code);
 }
 
+// Executed tile products of the tensor-core kernels since the last read by
+// attn_tile_counts(): [0] forward (128-query x 128-key tiles a forward CTA
+// computes), [1] backward (the same unit in the key-tile kernel). One atomic
+// add per CTA.
+__device__ unsigned long long g_attn_tiles[2];
+
 #ifdef ATTN_DEBUG_HOOKS
 // Watchdog test build only: a load the forward's TMA warp withholds (0 = none,
 // 1 = the first V tile), so that a consumer's bounded wait runs out.
@@ -104,11 +110,50 @@ __device__ __forceinline__ float warp_max(float x) {
   return x;
 }
 
+// fp16 storage of rotated q / k tiles: fp16 keeps 3 more mantissa bits than
+// bf16 (which the lse bound needs) but has a narrow range (overflow above
+// 65504, subnormals below 2^-14). A 128-row tile is therefore stored times
+// the power of two that brings a bound amax on its magnitudes (its largest
+// pair norm) into [2^14, 2^15): large tiles cannot overflow and small ones
+// keep all 11 bits down to 2^-28 of their maximum. The exponent is clamped so
+// that the factor and its inverse stay normal floats; an all-zero tile keeps
+// factor 1.
+__device__ __forceinline__ float fp16_tile_factor(float amax) {
+  if (!(amax > 0.f && amax <= 3.0e38f)) return 1.f;
+  return ldexpf(1.f, max(-100, min(100, 14 - ilogbf(amax))));
+}
+// The largest squared Euclidean norm of the four pairs (x[2i], x[2i+1]) of
+// eight values. A rotation keeps each pair's norm, so its values never exceed
+// it: the largest pair norm of a tile, taken before rotating, bounds the
+// rotated tile and fixes its factor (every kernel that stores a rotated tile
+// derives the factor this way, from the same bf16 inputs).
+__device__ __forceinline__ float pair_norm2_max8(const float* x) {
+  float m = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) m = fmaxf(m, fmaf(x[2 * e], x[2 * e], __fmul_rn(x[2 * e + 1], x[2 * e + 1])));
+  return m;
+}
+
+// Eight floats times f as eight fp16 values (round to nearest even).
+__device__ __forceinline__ uint4 pack8_half(const float* v, float f) {
+  uint4 out;
+  uint32_t* w = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __half2 hv = __floats2half2_rn(v[2 * e] * f, v[2 * e + 1] * f);
+    w[e] = *reinterpret_cast<uint32_t*>(&hv);
+  }
+  return out;
+}
+
 // Rotate (in place) NC consecutive elements starting at an even dimension d0
 // by the RoPE angles of position pos: pairs (x[2i], x[2i+1]) -> (x0 c - x1 s,
 // x0 s + x1 c). inverse = true applies the transpose rotation. For NC a
 // multiple of 8, d0 must be a multiple of 8 and the tables 16-byte aligned:
-// four pairs' cos and sin then come in one 16-byte load each.
+// four pairs' cos and sin then come in one 16-byte load each. The rounding is
+// spelled out (one product, then one fused multiply-add), so every kernel
+// that rotates the same value gets the same bits: the backward recomputes
+// the forward's scores from its own rotated copies.
 template <int NC, int D>
 __device__ __forceinline__ void rope_pairs(float* x, const float* rc, const float* rs,
                                            int pos, int d0, bool inverse) {
@@ -124,8 +169,8 @@ __device__ __forceinline__ void rope_pairs(float* x, const float* rc, const floa
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float x0 = x[8 * q + 2 * e], x1 = x[8 * q + 2 * e + 1];
-        x[8 * q + 2 * e] = x0 * cs[e] - x1 * sn[e];
-        x[8 * q + 2 * e + 1] = x0 * sn[e] + x1 * cs[e];
+        x[8 * q + 2 * e] = fmaf(x0, cs[e], -__fmul_rn(x1, sn[e]));
+        x[8 * q + 2 * e + 1] = fmaf(x0, sn[e], __fmul_rn(x1, cs[e]));
       }
     }
   } else {
@@ -135,8 +180,8 @@ __device__ __forceinline__ void rope_pairs(float* x, const float* rc, const floa
       const float cs = rc[(size_t)pos * (D / 2) + pi];
       const float sn = inverse ? -rs[(size_t)pos * (D / 2) + pi] : rs[(size_t)pos * (D / 2) + pi];
       const float x0 = x[c], x1 = x[c + 1];
-      x[c] = x0 * cs - x1 * sn;
-      x[c + 1] = x0 * sn + x1 * cs;
+      x[c] = fmaf(x0, cs, -__fmul_rn(x1, sn));
+      x[c + 1] = fmaf(x0, sn, __fmul_rn(x1, cs));
     }
   }
 }

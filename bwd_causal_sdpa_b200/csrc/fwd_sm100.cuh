@@ -80,8 +80,9 @@ struct Params {
   int T, H, Hkv, BH, n_pairs, n_qtiles;  // H query heads read Hkv key/value heads
   float scale_log2;          // scale * log2(e)
   uint32_t idesc_s;          // instruction descriptor of S = Q K^T
-  const float* q_fac;        // per (bh, tile) power-of-two factor of the stored q tile, or null
-  const float* k_fac;        // indexed by (key/value head, tile)
+  const float* q_fac;        // inverse power-of-two factor per (query head, tile) of the
+                             // stored rotated q, or null (q as given)
+  const float* k_fac;        // the same per (key/value head, tile) for k
   const int32_t* doc_start;  // flattened document starts, or null
   __nv_bfloat16* o;
   float* lse;
@@ -114,10 +115,18 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
   const int qtA = 2 * pr, qtB = 2 * pr + 1;
   const bool hasB = qtB * 128 < T;
   const int row0 = b * T;
+  // Key tiles are numbered from kv_t0, the tile holding the start of tile A's
+  // first row's document; tile A takes key tiles [0, nA) of that range, tile
+  // B [jB0, n_kv): from the tile holding its own first row's document start
+  // to its diagonal. Every key tile of a range holds a key some row of the
+  // query tile may see (a query tile's allowed keys form one interval).
   const int ds0 = p.doc_start ? p.doc_start[row0 + qtA * 128] - row0 : 0;
   const int kv_t0 = ds0 >> 7;
   const int nA = qtA - kv_t0 + 1;           // key tiles tile A needs
   const int n_kv = hasB ? nA + 1 : nA;      // tile B needs one more (its diagonal)
+  const int jB0 = (hasB && p.doc_start) ? ((p.doc_start[row0 + qtB * 128] - row0) >> 7) - kv_t0 : 0;
+  auto t_lo = [&](int t) -> int { return t == 0 ? 0 : jB0; };
+  auto t_hi = [&](int t) -> int { return t == 0 ? nA : (hasB ? n_kv : 0); };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::bQFull), 1);
@@ -136,6 +145,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     }
     *abort_flag = 0;
     fence_barrier_init();
+    atomicAdd(&g_attn_tiles[0], (unsigned long long)(nA + (hasB ? n_kv - jB0 : 0)));
   }
   if (warp == L::kMmaWarp) {
     tmem_alloc(sb0 + L::kMisc, L::kTmemCols);
@@ -177,15 +187,18 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     }
   } else if (warp == L::kMmaWarp) {
     // ---------------- MMA issuer ----------------
-    // Issue order: S_A(0), S_B(0), then per key tile j: PV_A(j), S_A(j+1),
-    // PV_B(j), S_B(j+1). Each tile's S(j+1) follows its own PV(j) (it
-    // overwrites the P that PV(j) reads, so it waits for PV(j) to finish), and
-    // never waits for the other tile's softmax: the two chains
-    // S -> softmax -> PV run independently and fill each other's gaps.
+    // Issue order: S of each tile whose range starts at key tile 0, then per
+    // key tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), each only where tile
+    // t's range holds j (a tile whose range starts at j+1 gets its first S
+    // there). Each tile's S(j+1) follows its own PV(j) (it overwrites the P
+    // that PV(j) reads, so it waits for PV(j) to finish), and never waits for
+    // the other tile's softmax: the two chains S -> softmax -> PV run
+    // independently and fill each other's gaps. Barrier phases of tile t count
+    // its own key tiles (j - t_lo(t)).
     if (lane == 0) {
       constexpr uint32_t idesc_o = idesc_f16(128, D, true, true, false, true);
       const int t1 = hasB ? 2 : 1;
-      auto active = [&](int t, int j) -> bool { return j < ((t == 0) ? nA : n_kv) && t < t1; };
+      auto active = [&](int t, int j) -> bool { return t < t1 && j >= t_lo(t) && j < t_hi(t); };
       auto issue_S = [&](int t, int j) {
         const uint32_t kbase = sb0 + L::kK + (j % L::kStages) * L::kTileBytes;
         const uint32_t qbase = sb0 + L::kQ + t * L::kTileBytes;
@@ -210,19 +223,31 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         const uint32_t vbase = sb0 + L::kV + st * L::kTileBytes;
         bool issued_next = false;
         for (int t = 0; ok && t < t1; ++t) {
-          if (!active(t, it)) continue;
-          if (!mbar_wait(bar(L::bPFull + t), it & 1, abort_flag)) { ok = false; break; }
+          if (!active(t, it)) {
+            if (active(t, it + 1)) {  // tile t's range starts at it + 1
+              if (!mbar_wait(bar(L::bKFull + nst), ((it + 1) / L::kStages) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              issue_S(t, it + 1);
+              issued_next = true;
+            }
+            continue;
+          }
+          const int li = it - t_lo(t);  // this tile's own key-tile count
+          if (!mbar_wait(bar(L::bPFull + t), li & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t aP = tmem + 256 * t;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tmem + 256 * t + 128, aP + kk * 8,
                    smem_desc_sw128(vbase + kk * 2048, L::kBlockBytes, 1024), idesc_o,
-                   (it > 0 || kk > 0) ? 1u : 0u);
+                   (li > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(L::bPVDone + t));
           if (active(t, it + 1)) {
             if (!mbar_wait(bar(L::bKFull + nst), ((it + 1) / L::kStages) & 1, abort_flag) ||
-                !mbar_wait(bar(L::bPVDone + t), it & 1, abort_flag)) {
+                !mbar_wait(bar(L::bPVDone + t), li & 1, abort_flag)) {
               ok = false;
               break;
             }
@@ -248,7 +273,8 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     const int qt = qtA + t;
     const int i = qt * 128 + r;
     const bool active = (t == 0) || hasB;
-    const int n_t = (t == 0) ? nA : n_kv;  // key tiles this tile processes
+    const int n_t = t_hi(t) - t_lo(t);  // key tiles this tile processes
+    const int kt_first = kv_t0 + t_lo(t);
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + 256 * t;
     const uint32_t tO = tS + 128;
@@ -258,11 +284,17 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = active;
     for (int it = 0; ok && it < n_t; ++it) {
-      const int kt = kv_t0 + it, j0 = kt * 128 + 64 * hf;  // first key of this half
+      const int kt = kt_first + it, j0 = kt * 128 + 64 * hf;  // first key of this half
       if (!mbar_wait(bar(L::bSFull + t), it & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      // scale of this key tile's scores (q, k tiles may carry power-of-two factors)
-      const float sc = p.scale_log2 * fq * (p.k_fac ? p.k_fac[bhk * p.n_qtiles + kt] : 1.f);
+      // scale of this key tile's scores (q, k tiles may carry power-of-two
+      // factors). A zero scale (uniform attention) is evaluated with the
+      // smallest normal scale instead: a score below 2^100 in magnitude then
+      // scales to below 2^-26, so each kept probability rounds to exactly 1
+      // as it should, while a masked score still becomes -inf rather than
+      // inf * 0 = NaN.
+      float sc = p.scale_log2 * fq * (p.k_fac ? p.k_fac[bhk * p.n_qtiles + kt] : 1.f);
+      if (sc == 0.f) sc = 1.17549435e-38f;
       const bool pos_scale = sc > 0.f;
       uint32_t s[64];
       tmem_ld32(tS + 64 * hf, s);

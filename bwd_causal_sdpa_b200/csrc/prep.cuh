@@ -2,28 +2,32 @@
 // backward's row term Delta_i = sum_d dO[i][d] * o[i][d].
 #pragma once
 
-#include <type_traits>
-
 #include "common.cuh"
 
 // From cu_seqlens (over the flattened B*T token axis, end marker B*T) build,
 // for every token, the flattened index where its document starts and where it
 // ends (exclusive). One block: thread 0 walks the array up to the end marker
-// (never past it) and validates it; then all threads fill the per-token
-// arrays by binary search. A malformed array sets ATTN_EDEVICE_INPUT and the
-// arrays fall back to "each row is one document", so later kernels stay in
-// bounds. (Cort33x, "Preserving context in the data": documents packed into
-// one window; attention stays within a document.)
+// (never past it), validates it and copies up to kDocRangesSmem + 1
+// boundaries into shared memory; then all threads fill the per-token arrays
+// by binary search over that copy (over the global array when it has more
+// documents). A malformed array sets ATTN_EDEVICE_INPUT and the arrays fall
+// back to "each row is one document", so later kernels stay in bounds.
+// (Cort33x, "Preserving context in the data": documents packed into one
+// window; attention stays within a document.)
+constexpr int kDocRangesSmem = 4096;
+
 __global__ void __launch_bounds__(1024) doc_ranges_kernel(const int32_t* __restrict__ cu, int B, int T,
                                                           int32_t* __restrict__ doc_start,
                                                           int32_t* __restrict__ doc_end) {
   pdl_wait_and_trigger();
+  __shared__ int s_cu[kDocRangesSmem + 1];
   __shared__ int s_ok, s_n;
   const int BT = B * T;
   if (threadIdx.x == 0) {
     int ok = 1, n = 0;
     int prev = cu[0];
     if (prev != 0) ok = 0;
+    s_cu[0] = prev;
     // Strictly rising values bounded by BT: at most BT steps.
     while (ok && prev < BT) {
       const int nxt = cu[n + 1];  // exists: prev < BT is not the end marker
@@ -33,6 +37,7 @@ __global__ void __launch_bounds__(1024) doc_ranges_kernel(const int32_t* __restr
       }
       prev = nxt;
       ++n;
+      if (n <= kDocRangesSmem) s_cu[n] = nxt;
     }
     s_ok = ok;
     s_n = n;
@@ -40,14 +45,15 @@ __global__ void __launch_bounds__(1024) doc_ranges_kernel(const int32_t* __restr
   __syncthreads();
   if (s_ok) {
     const int n = s_n;
+    const int32_t* bounds = n <= kDocRangesSmem ? s_cu : cu;
     for (int t = threadIdx.x; t < BT; t += blockDim.x) {
-      int lo = 0, hi = n;  // cu[lo] <= t < cu[hi]
+      int lo = 0, hi = n;  // bounds[lo] <= t < bounds[hi]
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (cu[mid] <= t) lo = mid; else hi = mid;
+        if (bounds[mid] <= t) lo = mid; else hi = mid;
       }
-      doc_start[t] = cu[lo];
-      doc_end[t] = cu[hi];
+      doc_start[t] = bounds[lo];
+      doc_end[t] = bounds[hi];
     }
   } else {
     if (threadIdx.x == 0) report_status(ATTN_EDEVICE_INPUT);
@@ -78,39 +84,34 @@ __global__ void __launch_bounds__(256) delta_kernel(const TIO* __restrict__ o, c
   if (lane == 0) delta[row] = s;
 }
 
-// RoPE pre-pass for the tensor-core kernels: rotate q and k once (fp32
-// arithmetic, interleaved pairs at the token's document position) and store
-// the rotated tiles in the 16-bit type the MMAs read. blockIdx = (128-row
-// tile, head, 0 for q / 1 for k); the head is b*H + h for q and b*Hkv + h
-// for k (blocks past B*Hkv return at once).
-//
-// kTileScale (forward, fp16 output): fp16 keeps 3 more mantissa bits than
-// bf16, which the lse bound needs, but has a narrow range; a tile whose
-// largest magnitude reaches 2^14 is multiplied by a power of two that brings
-// it into [2^14, 2^15), and fac[] receives the inverse factor (exact), which
-// the forward folds into its score scale. Without kTileScale (bf16 output)
-// values are stored as they are.
+// RoPE pre-pass for the forward: rotate q and k once (fp32 arithmetic,
+// interleaved pairs at the token's document position) and store every
+// 128-row tile as fp16 times its power-of-two factor (fp16_tile_factor of the
+// tile's largest pair norm); fac[] receives the inverse factor (exact), which
+// the forward folds into its score scale. blockIdx = (128-row tile, head,
+// 0 for q / 1 for k); the head is b*H + h for q and b*Hkv + h for k (blocks
+// past B*Hkv return at once).
 constexpr int kRopePrepThreads = 512;
 
-template <typename OutT, int D, bool kTileScale>
+template <int D>
 __global__ void __launch_bounds__(kRopePrepThreads) rope_prep_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const float* __restrict__ rc, const float* __restrict__ rs,
-    const int32_t* __restrict__ doc_start, OutT* __restrict__ qo, OutT* __restrict__ ko,
-    float* __restrict__ qfac, float* __restrict__ kfac, int H, int Hkv, int T, int ntiles) {
+    const int32_t* __restrict__ doc_start, __half* __restrict__ qo, __half* __restrict__ ko,
+    float* __restrict__ qfac, float* __restrict__ kfac, int B, int H, int Hkv, int T,
+    int ntiles) {
   pdl_wait_and_trigger();
   constexpr int CH = D / 8;              // 16-byte chunks per row
   constexpr int NT = kRopePrepThreads;
   constexpr int PER = 128 * CH / NT;     // chunks per thread
-  // grid (ntiles, B*H, 2): z = 0 rotates q heads, z = 1 the B*Hkv k heads
   const int tile = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const int heads = which ? Hkv : H;
+  if (bh >= B * heads) return;  // k has fewer heads than q
   const int b = bh / heads, row0 = b * T, t0 = tile * 128;
-  if (b >= (int)gridDim.y / H) return;  // k has fewer heads than q
   const __nv_bfloat16* src = which ? k : q;
-  OutT* dst = which ? ko : qo;
+  __half* dst = which ? ko : qo;
   float v[PER][8];
-  float amax = 0.f;
+  float n2 = 0.f;
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
     const int idx = threadIdx.x + u * NT, r = idx / CH, c8 = idx % CH, t = t0 + r;
@@ -121,41 +122,24 @@ __global__ void __launch_bounds__(kRopePrepThreads) rope_prep_kernel(
       const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[u][e] = __bfloat162float(h[e]);
-      const int pos = t - (doc_start ? doc_start[row0 + t] - row0 : 0);
-      rope_pairs<8, D>(v[u], rc, rs, pos, c8 * 8, false);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[u][e]));
+      n2 = fmaxf(n2, pair_norm2_max8(v[u]));
     }
   }
-  float f = 1.f;
-  if constexpr (kTileScale) {
-    __shared__ float red[NT / 32];
-    amax = warp_max(amax);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
-    __syncthreads();
-    amax = red[0];
+  __shared__ float red[NT / 32];
+  n2 = warp_max(n2);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = n2;
+  __syncthreads();
+  n2 = red[0];
 #pragma unroll
-    for (int w = 1; w < NT / 32; ++w) amax = fmaxf(amax, red[w]);
-    if (amax >= 16384.f && amax <= 3.0e38f) f = ldexpf(1.f, 14 - ilogbf(amax));
-    if (threadIdx.x == 0) (which ? kfac : qfac)[bh * ntiles + tile] = 1.f / f;
-  }
+  for (int w = 1; w < NT / 32; ++w) n2 = fmaxf(n2, red[w]);
+  const float f = fp16_tile_factor(sqrtf(n2));
+  if (threadIdx.x == 0) (which ? kfac : qfac)[(size_t)bh * ntiles + tile] = 1.f / f;
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
     const int idx = threadIdx.x + u * NT, r = idx / CH, c8 = idx % CH, t = t0 + r;
     if (t >= T) continue;
-    uint4 out;
-    uint32_t* w = reinterpret_cast<uint32_t*>(&out);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if constexpr (sizeof(OutT) == 2 && std::is_same<OutT, __half>::value) {
-        __half2 hv = __floats2half2_rn(v[u][2 * e] * f, v[u][2 * e + 1] * f);
-        w[e] = *reinterpret_cast<uint32_t*>(&hv);
-      } else {
-        __nv_bfloat162 hv = __floats2bfloat162_rn(v[u][2 * e] * f, v[u][2 * e + 1] * f);
-        w[e] = *reinterpret_cast<uint32_t*>(&hv);
-      }
-    }
-    *reinterpret_cast<uint4*>(dst + ((size_t)bh * T + t) * D + c8 * 8) = out;
+    rope_pairs<8, D>(v[u], rc, rs, t - (doc_start ? doc_start[row0 + t] - row0 : 0), c8 * 8, false);
+    *reinterpret_cast<uint4*>(dst + ((size_t)bh * T + t) * D + c8 * 8) = pack8_half(v[u], f);
   }
 }
 
@@ -180,73 +164,140 @@ __device__ __forceinline__ void store8_bf16(__nv_bfloat16* p, const float* v) {
   *reinterpret_cast<uint4*>(p) = raw;
 }
 
-// Backward preprocessing for the tensor-core path over the tile-padded
-// [B*H][ntiles*128] row view, D/8 threads per row (16 bytes of each bf16 row
-// per thread, so a warp covers 32*8/D whole rows): stores -Delta_i (Delta_i =
-// sum_d dO[i][d] * o[i][d]) and -lse_i * log2(e), negated so the main kernel
-// folds them in with one fused multiply-add (both 0 for padding rows t >= T,
-// so its per-tile loads never leave the arrays), zeroes the fp32 dq
-// accumulator row and, with RoPE tables, writes the rotated q and k rows
-// (bf16) the main kernel reads; when the grouped-query backward splits its
-// groups, it also zeroes the fp32 dk, dv accumulator rows. The grid covers
-// rows_pad * D/8 threads exactly (rows_pad is a multiple of 128), so every
-// warp is full.
-template <int D>
-__global__ void __launch_bounds__(256) bwd_prep_kernel(
+// Backward preprocessing for the tensor-core path, one block per (128-row
+// tile, query head bh). Per row it stores -Delta_i (Delta_i = sum_d dO[i][d]
+// * o[i][d]) and -lse_i * log2(e) in the tile-padded [B*H][Tpad] arrays,
+// negated so the main kernel folds them in with one fused multiply-add (both
+// 0 for rows t >= T, so its per-tile loads never leave the arrays), and
+// zeroes the row of the fp32 dq accumulator (when the grouped-query backward
+// splits its groups, also of the dk, dv accumulators: blocks with bh below
+// B*Hkv take those rows of key/value head bh). Per tile it records the
+// largest |dO_i| (Euclidean norm) and |Delta_i|, which bound dS for the main
+// kernel's fp16 scaling.
+//
+// kRope: the tile's q rows (and, for bh below B*Hkv, the same rows of key/value
+// head bh's k) are rotated and stored as fp16 times the tile's power-of-two
+// factor (fp16_tile_factor of the largest pair norm, found in the first read
+// of the rows), with the inverse factors in qinv (a 16-byte record per tile,
+// value first, so the main kernel can bulk-load it) and kinv: the same values the
+// forward's scores were computed from, so the main kernel recomputes exactly
+// those scores. The rows are read again (from cache) to be rotated.
+constexpr int kBwdPrepThreads = 256;
+
+template <int D, bool kRope>
+__global__ void __launch_bounds__(kBwdPrepThreads) bwd_prep_kernel(
     const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
     const float* __restrict__ lse, float* __restrict__ delta_pad, float* __restrict__ lse2_pad,
     float* __restrict__ dq_acc, const __nv_bfloat16* __restrict__ q,
     const __nv_bfloat16* __restrict__ k, const float* __restrict__ rc,
     const float* __restrict__ rs, const int32_t* __restrict__ doc_start,
-    __nv_bfloat16* __restrict__ qr, __nv_bfloat16* __restrict__ kr, float* __restrict__ dk_acc,
-    float* __restrict__ dv_acc, int H, int Hkv, int T, int Tpad, long rows_pad) {
+    __half* __restrict__ q16, __half* __restrict__ k16, float* __restrict__ qinv,
+    float* __restrict__ kinv, float* __restrict__ dmax, float* __restrict__ deltamax,
+    float* __restrict__ dk_acc, float* __restrict__ dv_acc, int B, int H, int Hkv, int T,
+    int Tpad, int ntiles) {
   pdl_wait_and_trigger();
-  constexpr int TPR = D / 8;  // threads per row
-  const long gt = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long row = gt / TPR;
-  const int c8 = (int)(gt - row * TPR) * 8;
-  const long bh = row / Tpad;
-  const int t = (int)(row - bh * Tpad);
-  float s = 0.f;
-  if (row < rows_pad && t < T) {
-    const long r = bh * T + t;
-    float a[8], g[8];
-    load8_bf16(o + r * D + c8, a);
-    load8_bf16(dO + r * D + c8, g);
+  constexpr int CPR = D / 8;                    // 16-byte chunks per row
+  constexpr int RPP = kBwdPrepThreads / CPR;    // rows per pass
+  constexpr int NP = 128 / RPP;                 // passes over the tile
+  const int tile = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / H;
+  const bool kv = bh < B * Hkv;  // also a key/value head index
+  const int bk = kv ? bh / Hkv : 0;
+  const int c = threadIdx.x % CPR, rsub = threadIdx.x / CPR;
+  float dmx = 0.f, dlx = 0.f, aq = 0.f, ak = 0.f;
+  for (int u = 0; u < NP; ++u) {
+    const int t = tile * 128 + u * RPP + rsub;
+    const bool valid = t < T;
+    const size_t off = ((size_t)bh * T + (valid ? t : 0)) * D + 8 * c;
+    float s = 0.f, n2 = 0.f;
+    if (valid) {
+      float a[8], g[8];
+      load8_bf16(o + off, a);
+      load8_bf16(dO + off, g);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) s = fmaf(a[e], g[e], s);
-    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    reinterpret_cast<float4*>(dq_acc + r * D + c8)[0] = z;
-    reinterpret_cast<float4*>(dq_acc + r * D + c8)[1] = z;
-    if (dk_acc && bh < (rows_pad / Tpad) / H * Hkv) {  // a row of the [B*Hkv][T] view
-      reinterpret_cast<float4*>(dk_acc + r * D + c8)[0] = z;
-      reinterpret_cast<float4*>(dk_acc + r * D + c8)[1] = z;
-      reinterpret_cast<float4*>(dv_acc + r * D + c8)[0] = z;
-      reinterpret_cast<float4*>(dv_acc + r * D + c8)[1] = z;
-    }
-    if (rc) {
-      const int b = (int)(bh / H);
-      const int pos = t - (doc_start ? doc_start[b * T + t] - b * T : 0);
-      float x[8];
-      load8_bf16(q + r * D + c8, x);
-      rope_pairs<8, D>(x, rc, rs, pos, c8, false);
-      store8_bf16(qr + r * D + c8, x);
-      // row r of the [B*Hkv][T] k view exists for the first B*Hkv heads; its
-      // batch (hence document layout) is bh / Hkv
-      if (bh < (rows_pad / Tpad) / H * Hkv) {
-        const int bk = (int)(bh / Hkv);
-        const int posk = t - (doc_start ? doc_start[bk * T + t] - bk * T : 0);
-        load8_bf16(k + r * D + c8, x);
-        rope_pairs<8, D>(x, rc, rs, posk, c8, false);
-        store8_bf16(kr + r * D + c8, x);
+      for (int e = 0; e < 8; ++e) {
+        s = fmaf(a[e], g[e], s);
+        n2 = fmaf(g[e], g[e], n2);
+      }
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      reinterpret_cast<float4*>(dq_acc + off)[0] = z;
+      reinterpret_cast<float4*>(dq_acc + off)[1] = z;
+      if (dk_acc && kv) {
+        reinterpret_cast<float4*>(dk_acc + off)[0] = z;
+        reinterpret_cast<float4*>(dk_acc + off)[1] = z;
+        reinterpret_cast<float4*>(dv_acc + off)[0] = z;
+        reinterpret_cast<float4*>(dv_acc + off)[1] = z;
+      }
+      if constexpr (kRope) {  // the tiles' largest pair norms (squared), before rotating
+        float x[8];
+        load8_bf16(q + off, x);
+        aq = fmaxf(aq, pair_norm2_max8(x));
+        if (kv) {
+          load8_bf16(k + off, x);
+          ak = fmaxf(ak, pair_norm2_max8(x));
+        }
       }
     }
-  }
+    // a row's CPR chunks sit in consecutive lanes of one warp
 #pragma unroll
-  for (int off = TPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (c8 == 0 && row < rows_pad) {
-    delta_pad[row] = -s;
-    lse2_pad[row] = t < T ? -lse[bh * T + t] * 1.4426950408889634f : 0.f;
+    for (int sh = CPR / 2; sh > 0; sh >>= 1) {
+      s += __shfl_xor_sync(0xffffffffu, s, sh);
+      n2 += __shfl_xor_sync(0xffffffffu, n2, sh);
+    }
+    if (c == 0) {
+      delta_pad[(size_t)bh * Tpad + t] = valid ? -s : 0.f;
+      lse2_pad[(size_t)bh * Tpad + t] = valid ? -lse[(size_t)bh * T + t] * 1.4426950408889634f : 0.f;
+    }
+    if (valid) {
+      dmx = fmaxf(dmx, sqrtf(n2));
+      dlx = fmaxf(dlx, fabsf(s));
+    }
+  }
+  __shared__ float red[4][kBwdPrepThreads / 32];
+  dmx = warp_max(dmx);
+  dlx = warp_max(dlx);
+  aq = warp_max(aq);
+  ak = warp_max(ak);
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    red[0][w] = dmx;
+    red[1][w] = dlx;
+    red[2][w] = aq;
+    red[3][w] = ak;
+  }
+  __syncthreads();
+  float m[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    m[j] = red[j][0];
+#pragma unroll
+    for (int i = 1; i < kBwdPrepThreads / 32; ++i) m[j] = fmaxf(m[j], red[j][i]);
+  }
+  const float fq = fp16_tile_factor(sqrtf(m[2])), fk = fp16_tile_factor(sqrtf(m[3]));
+  if (threadIdx.x == 0) {
+    dmax[(size_t)bh * ntiles + tile] = m[0];
+    deltamax[(size_t)bh * ntiles + tile] = m[1];
+    if (kRope) {
+      reinterpret_cast<float4*>(qinv)[(size_t)bh * ntiles + tile] = make_float4(1.f / fq, 0.f, 0.f, 0.f);
+      if (kv) kinv[(size_t)bh * ntiles + tile] = 1.f / fk;
+    }
+  }
+  if constexpr (kRope) {
+    for (int u = 0; u < NP; ++u) {
+      const int t = tile * 128 + u * RPP + rsub;
+      if (t >= T) continue;
+      const size_t off = ((size_t)bh * T + t) * D + 8 * c;
+      float x[8];
+      load8_bf16(q + off, x);
+      rope_pairs<8, D>(x, rc, rs, t - (doc_start ? doc_start[b * T + t] - b * T : 0), 8 * c, false);
+      *reinterpret_cast<uint4*>(q16 + off) = pack8_half(x, fq);
+      if (kv) {
+        load8_bf16(k + off, x);
+        rope_pairs<8, D>(x, rc, rs, t - (doc_start ? doc_start[bk * T + t] - bk * T : 0), 8 * c,
+                         false);
+        *reinterpret_cast<uint4*>(k16 + off) = pack8_half(x, fk);
+      }
+    }
   }
 }
 

@@ -200,11 +200,12 @@ const char* attn_error_string(int code);
  * loads the library holds until the process exits.
  *
  * It runs the CUDA-core (fp32 arithmetic) backward kernels, for either dtype,
- * and needs 4*B*H*T + 8*B*T bytes of scratch (each part rounded up to 256);
- * larger problems are rejected with ATTN_ESCRATCH before anything is launched.
- * The first call on each device looks up the array's device address with
- * cudaGetSymbolAddress (no allocation); make that first call before any stream
- * capture. All calls share the one array and it keeps the previous call's
+ * and needs 4*B*H*T bytes of scratch, plus 8*B*T more when cu_seqlens is
+ * given (each part rounded up to 256); larger problems are rejected with
+ * ATTN_ESCRATCH before anything is launched. The first call on each device
+ * looks up the array's device address with cudaGetSymbolAddress (no
+ * allocation), and so does the first call after that device's context was
+ * reset (cudaDeviceReset); make those calls before any stream capture. All calls share the one array and it keeps the previous call's
  * contents; every byte a call reads is written earlier in the same call, so
  * nothing needs clearing, but two calls that overlap on the GPU (on different
  * streams, or from different threads) race on it and must be serialised by the
@@ -298,6 +299,14 @@ int attn_out_proj_bwd(const void* dy, const void* o, const void* w_o, void* d_o,
  * the number of timed launches and their summed duration in milliseconds.
  * Returns ATTN_OK, ATTN_EINVAL (kind out of range or a null output pointer)
  * or ATTN_ECUDA.
+ *
+ * attn_tile_counts: the 128-query x 128-key tile products the tensor-core
+ * forward (fwd_tiles) and key-tile backward (bwd_tiles) kernels executed on
+ * the current device since the previous read, counted on the device (one
+ * atomic add per CTA; the CUDA-core float32 path is not counted); resets both
+ * counters. Block skipping makes these close to the tiles that hold at least
+ * one allowed (query, key) pair. Synchronises the device. Returns ATTN_OK,
+ * ATTN_EINVAL (a null pointer) or ATTN_ECUDA.
  */
 /* attn_exp2_selftest: y[i] = the forward/backward kernels' software 2^x
  * (FMA-pipe polynomial) of x[i], for 0 <= i < n; x, y device f32 arrays,
@@ -316,6 +325,7 @@ int attn_exp2_selftest(const float* x, float* y, int n, void* stream);
 int attn_debug_withhold(int what);
 
 unsigned long long attn_launch_count(void);
+int attn_tile_counts(unsigned long long* fwd_tiles, unsigned long long* bwd_tiles);
 int attn_profile_enable(int on);
 int attn_profile_kinds(void);
 int attn_profile_read(int kind, const char** name, int* launches, double* total_ms);

@@ -14,12 +14,46 @@ TOL = {
     "f32": {"o": 1e-5, "lse": 1e-5, "dq": 1e-5, "dk": 1e-5, "dv": 1e-5},
 }
 
+# Per-tile check: every 128-row tile of every compared slice must also meet
+# TILE_FACTOR x the tensor's bound, its error taken relative to the larger of
+# its own reference norm and TILE_FLOOR x the slice's RMS row norm scaled to
+# the tile's row count. A tile's error has the expectation of the whole
+# tensor's (the same roundings, on 128*D instead of T*D values); the factor
+# leaves room for the tiles whose rows see few keys (the first rows of a
+# causal head, short documents), and the floor keeps tiles whose reference
+# is near zero (late keys' dk, dv) from dividing by almost nothing. A tile
+# that is wrong as a whole fails by orders of magnitude; on an 8K head it
+# would move the whole-tensor norm by only 1/8 of its own error.
+TILE = 128
+TILE_FACTOR = 2.0
+TILE_FLOOR = 0.1
+
 
 def rel_fro(got, ref) -> float:
     ref = np.asarray(ref, dtype=np.float64)
     got = np.asarray(got, dtype=np.float64)
     den = np.linalg.norm(ref)
     return float(np.linalg.norm(got - ref) / (den if den > 0 else 1.0))
+
+
+def tile_errors(got, ref) -> np.ndarray:
+    """Relative error of every 128-row tile of every slice; got and ref are
+    [n_slices, T] or [n_slices, T, D]."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    n, T = ref.shape[0], ref.shape[1]
+    out = []
+    for s in range(n):
+        r_all = ref[s].reshape(T, -1)
+        g_all = got[s].reshape(T, -1)
+        rms_row = np.linalg.norm(r_all) / np.sqrt(T)
+        for t0 in range(0, T, TILE):
+            r = r_all[t0:t0 + TILE]
+            g = g_all[t0:t0 + TILE]
+            floor = TILE_FLOOR * rms_row * np.sqrt(r.shape[0])
+            den = max(np.linalg.norm(r), floor)
+            out.append(np.linalg.norm(g - r) / (den if den > 0 else 1.0))
+    return np.asarray(out)
 
 
 def oracle_outputs(w, heads=None) -> dict:
@@ -42,6 +76,27 @@ def gpu_outputs(w, *, runner_cls=None) -> dict:
     return r.results()
 
 
+def compare_arrays(got: dict, ref: dict, tol: dict, keys=None) -> dict:
+    """Whole-tensor and per-tile errors of stacked slices ([n, T(, D)] per
+    key); asserts both bounds and returns {key: error, key + "_tile": worst
+    tile error}."""
+    errs = {}
+    bad = {}
+    for key in (keys or list(ref)):
+        g, r = got[key], ref[key]
+        assert np.all(np.isfinite(g)), f"{key}: non-finite values"
+        e = rel_fro(g, r)
+        et = float(tile_errors(g, r).max())
+        errs[key] = e
+        errs[key + "_tile"] = et
+        if not e <= tol[key]:
+            bad[key] = (e, tol[key])
+        if not et <= TILE_FACTOR * tol[key]:
+            bad[key + "_tile"] = (et, TILE_FACTOR * tol[key])
+    assert not bad, f"parity failed (error, bound): {bad}; all errors {errs}"
+    return errs
+
+
 def compare(w, got: dict, ref: dict, heads=None) -> dict:
     """Errors per tensor over the compared (b, h) query slices; asserts the
     bounds. dk and dv are compared on the key/value heads those slices read,
@@ -54,14 +109,9 @@ def compare(w, got: dict, ref: dict, heads=None) -> dict:
     listed = set(heads)
     for b, hk in kv_heads:
         assert all((b, hk * G + g) in listed for g in range(G)), "incomplete query-head group"
-    tol = TOL[w.dtype]
-    errs = {}
+    g_st, r_st = {}, {}
     for key in ("o", "lse", "dq", "dk", "dv"):
         pairs = kv_heads if key in ("dk", "dv") else heads
-        g = np.stack([got[key][b, h] for b, h in pairs])
-        r = np.stack([ref[key][b, h] for b, h in pairs])
-        assert np.all(np.isfinite(g)), f"{key}: non-finite values"
-        errs[key] = rel_fro(g, r)
-    bad = {k: (e, tol[k]) for k, e in errs.items() if not e <= tol[k]}
-    assert not bad, f"parity failed (error, bound): {bad}; all errors {errs}"
-    return errs
+        g_st[key] = np.stack([got[key][b, h] for b, h in pairs])
+        r_st[key] = np.stack([ref[key][b, h] for b, h in pairs])
+    return compare_arrays(g_st, r_st, TOL[w.dtype], keys=("o", "lse", "dq", "dk", "dv"))

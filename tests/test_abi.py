@@ -288,3 +288,22 @@ def test_projection_gemm_plan():
         assert 1 <= p["splits"] <= nkb and (p["splits"] - 1) * p["kb_per_split"] < nkb
         assert p["splits"] * p["kb_per_split"] >= nkb
     assert A.attn_proj_gemm_plan(0, 8, 8, True)[0] == A.ATTN_EINVAL
+
+
+def test_noalloc_counts_document_ranges_only_when_packed():
+    """attn_bwd_noalloc's scratch holds Delta (4*B*H*T bytes) and, only when
+    documents are packed, the document ranges (8*B*T more): a problem whose
+    Delta alone fits the 8 MiB array is rejected with packing and passes the
+    size check without it (on a machine without a GPU the call then stops at
+    the device query, before any launch)."""
+    import bwd_causal_sdpa_b200 as A
+
+    P = 1 << 20  # fake aligned addresses, never dereferenced
+    B, H, T = 1, 1, (1 << 21) - 256  # 4*T bytes: just under 8 MiB
+    args = (P, P, P, P, P, P, None, None)
+    tail = (B, H, T, 64, 0.125, A.ATTN_BF16, P, P, P, None)
+    assert A.attn_bwd_noalloc(*args, P, *tail) == A.ATTN_ESCRATCH
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("the unpacked call would launch kernels on fake addresses")
+    assert A.attn_bwd_noalloc(*args, None, *tail) == A.ATTN_ECUDA

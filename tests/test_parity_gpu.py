@@ -99,3 +99,68 @@ def test_malformed_cu_seqlens_reports_status_and_falls_back():
     assert r.status() == ATTN_OK  # cleared by the read
     w.cu_seqlens = None
     compare(w, r.results(), ref)
+
+
+# ---------------------------------------------------------------------------
+# Magnitudes and signs of the score scale. With RoPE the forward stores the
+# rotated q and k as fp16 with one power-of-two factor per 128-row tile (each
+# tile's largest magnitude brought into [2^14, 2^15)) and folds the factors
+# into the score scale; these cases drive tiles far outside fp16's own range
+# in both directions, tiles of different magnitudes in one head, and negative
+# and zero scales, against the oracle through the C ABI.
+# ---------------------------------------------------------------------------
+
+def _scaled(w, q_tiles=(1.0,), k_tiles=(1.0,), scale=None):
+    """Multiply q and k by a factor per 128-row tile (cycling through the
+    given factors), round back to bf16 and set the score scale."""
+    from workloads import round_to_bf16
+
+    def apply(x, facs):
+        f = np.array([facs[(t // 128) % len(facs)] for t in range(x.shape[2])], np.float32)
+        return round_to_bf16(x * f[None, None, :, None])
+
+    w.q = apply(w.q, q_tiles)
+    w.k = apply(w.k, k_tiles)
+    if scale is not None:
+        w.scale = float(scale)
+    return w
+
+
+MAGNITUDES = [
+    # name, q factors per tile, k factors per tile, scale multiplier
+    ("large_q_k", (2e4,), (2e4,), 1 / 4e8),        # every tile scaled down, max |x| ~ 1e5 > 65504
+    ("tiny_q_k", (1e-5,), (1e-5,), 1e10),         # fp16 subnormal range without the factors
+    ("large_q_tiny_k", (3e4,), (3e-5,), 1.0),
+    ("mixed_tiles", (1.0, 4.0, 0.5), (1.0, 0.25, 3.0), 1.0),
+    ("mixed_extreme", (2e4, 1.0), (1.0, 1e-4), 1 / 2e4),
+]
+
+
+@pytest.mark.parametrize("name,fq,fk,smul", MAGNITUDES, ids=[m[0] for m in MAGNITUDES])
+@pytest.mark.parametrize("D", [64, 128])
+def test_tile_factor_magnitudes_match_oracle(name, fq, fk, smul, D):
+    _cuda()
+    w = make_workload(config_by_name("packed_docs"), B=2, H=2, T=600, D=D, doc_min=40,
+                      doc_max=400, seed=51)
+    w = _scaled(w, fq, fk, w.scale * smul)
+    errs = compare(w, gpu_outputs(w), oracle_outputs(w))
+    print(name, D, errs)
+
+
+@pytest.mark.parametrize("sign", ["negative", "zero"])
+@pytest.mark.parametrize("rope", [True, False])
+def test_negative_and_zero_scale_match_oracle(sign, rope):
+    _cuda()
+    w = make_workload(config_by_name("packed_docs"), B=2, H=2, T=400, D=128, rope=rope,
+                      doc_min=30, doc_max=300, seed=52)
+    w = _scaled(w, (1.0, 3.0), (2.0, 0.5), -w.scale if sign == "negative" else 0.0)
+    errs = compare(w, gpu_outputs(w), oracle_outputs(w))
+    print(sign, rope, errs)
+
+
+def test_tile_factors_on_grouped_heads_match_oracle():
+    _cuda()
+    w = make_workload(config_by_name("long_context_8k"), B=1, H=4, H_kv=2, T=520, seed=53)
+    w = _scaled(w, (5e3, 1.0, 0.01), (1.0, 7e-3), w.scale / 5e3)
+    errs = compare(w, gpu_outputs(w), oracle_outputs(w))
+    print(errs)
