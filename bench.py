@@ -122,10 +122,9 @@ def kernel_algorithmic(name: str, w, kinds_seen) -> tuple:
     if name == "delta":
         if w.dtype != "bf16":  # Delta only
             return "hbm", 2 * N * elem + 4 * R, "byte"
-        # bf16 backward preparation: read o, dO, lse; write -Delta and -lse*log2e,
-        # zero the fp32 dq accumulator; with RoPE also rotate q and k
-        rope = 2 * (N + Nkv) * elem if w.rope_cos is not None else 0
-        return "hbm", 2 * N * elem + 12 * R + 4 * N + rope, "byte"
+        # bf16 backward row pass: read o, dO, lse; write -Delta and -lse*log2e,
+        # zero the fp32 dq accumulator
+        return "hbm", 2 * N * elem + 12 * R + 4 * N, "byte"
     if name == "rope_prep":
         return "hbm", 2 * (N + Nkv) * elem, "byte"
     if name == "dq_finalize":
@@ -426,12 +425,13 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize(dev)
     launches = A.attn_launch_count() - n0
-    code, fwd_tiles, bwd_tiles = A.attn_tile_counts()
+    code, fwd_tiles, bwd_tiles, dq_tiles = A.attn_tile_counts()
     A.check(code, "attn_tile_counts")
     tiles = None
     if w.dtype == "bf16":
         tiles = ideal_tiles(w)
-        tiles.update(fwd_executed=fwd_tiles / args.steps, bwd_executed=bwd_tiles / args.steps)
+        tiles.update(fwd_executed=fwd_tiles / args.steps, bwd_executed=bwd_tiles / args.steps,
+                     dq_pass_executed=dq_tiles / args.steps)
         tiles["fwd_over_ideal"] = tiles["fwd_executed"] / tiles["ideal"]
         tiles["bwd_over_ideal"] = tiles["bwd_executed"] / tiles["ideal"]
         tiles["unit"] = "128x128 tile products per step, all query heads (device counters)"

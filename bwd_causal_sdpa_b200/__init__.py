@@ -62,7 +62,7 @@ _SIGNATURES = {
     "attn_exp2_selftest": (_I, [_P, _P, _I, _P]),
     "attn_debug_withhold": (_I, [_I]),
     "attn_launch_count": (ctypes.c_ulonglong, []),
-    "attn_tile_counts": (_I, [ctypes.POINTER(ctypes.c_ulonglong), ctypes.POINTER(ctypes.c_ulonglong)]),
+    "attn_tile_counts": (_I, [ctypes.POINTER(ctypes.c_ulonglong)] * 3),
     "attn_profile_enable": (_I, [_I]),
     "attn_profile_kinds": (_I, []),
     "attn_profile_read": (_I, [_I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_I),
@@ -239,12 +239,12 @@ def attn_launch_count() -> int:
 
 
 def attn_tile_counts():
-    """(code, fwd_tiles, bwd_tiles): tile products the tensor-core kernels
-    executed since the previous read (counted on the device; resets them)."""
-    f = ctypes.c_ulonglong()
-    b = ctypes.c_ulonglong()
-    code = int(_lib.attn_tile_counts(ctypes.byref(f), ctypes.byref(b)))
-    return code, int(f.value), int(b.value)
+    """(code, fwd_tiles, bwd_tiles, dq_tiles): tile products the tensor-core
+    kernels executed since the previous read (counted on the device; resets
+    them)."""
+    f, b, q = ctypes.c_ulonglong(), ctypes.c_ulonglong(), ctypes.c_ulonglong()
+    code = int(_lib.attn_tile_counts(ctypes.byref(f), ctypes.byref(b), ctypes.byref(q)))
+    return code, int(f.value), int(b.value), int(q.value)
 
 
 def attn_profile_enable(on) -> int:

@@ -71,10 +71,12 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
     return _compile(LIB, list(extra_flags or []), verbose)
 
 
-# The watchdog test library: the same sources with the debug hooks compiled in
-# (attn_debug_withhold works) and the bounded waits cut to 2e7 cycles (~10 ms).
+# The test library: the same sources with the debug hooks compiled in
+# (attn_debug_withhold works), the bounded waits cut to 2e7 cycles (~10 ms),
+# and the backward's dQ formed by the other of its two routes than the
+# product library's, so that the GPU tests cover both.
 LIB_DEBUG = os.path.join(PKG, "libattn_debug.so")
-DEBUG_FLAGS = ["-DATTN_DEBUG_HOOKS", "-DATTN_WAIT_LIMIT_CYCLES=20000000LL"]
+DEBUG_FLAGS = ["-DATTN_DEBUG_HOOKS", "-DATTN_WAIT_LIMIT_CYCLES=20000000LL", "-DATTN_DQ_ROUTE_SWAPPED"]
 
 
 def build_debug(force: bool = False, verbose: bool = False) -> str:

@@ -10,6 +10,7 @@
 #include "attn.h"
 #include "common.cuh"
 #include "bwd_sm100.cuh"
+#include "dq_sm100.cuh"
 #include "decode.cuh"
 #include "fwd_sm100.cuh"
 #include "prep.cuh"
@@ -28,10 +29,9 @@ struct WsPlan {
   size_t lse2 = 0;                    // f32 [B*H*Tpad] lse*log2(e) (bf16 backward)
   size_t dq_acc = 0;                  // f32 [B*H*T*D] dq accumulator (bf16 backward)
   size_t q16 = 0, k16 = 0;            // rotated q, k as fp16 [B*H*T*D] each (bf16 storage)
-  size_t qfac = 0, kfac = 0;          // f32 [B*H*ceil(T/128)] inverse tile factors (bf16 forward)
-  size_t qinv = 0, kinv = 0;          // inverse q / k tile factors (bf16 backward): q as f32
-                                      // [B*H*ceil(T/128)][4] records, k as f32 [B*Hkv*ceil(T/128)]
-  size_t dmax = 0, deltamax = 0;      // f32 [B*H*ceil(T/128)] per-tile max |dO_i|, |Delta_i| (bf16 backward)
+  size_t qfac = 0, kfac = 0;          // inverse tile factors (bf16, both passes): q as f32
+                                      // [B*H*ceil(T/128)][4] records, k as f32 [B*H*ceil(T/128)]
+  size_t hstat = 0;                   // f32 [B*H][4] per-head max |dO_i|, |Delta_i|, |v_j| (bf16 backward)
   size_t dk_acc = 0, dv_acc = 0;      // f32 [B*Hkv*T*D] each when the backward splits groups
   int split = 1;                      // query-head groups split over this many CTAs
   size_t total = 0;
@@ -76,10 +76,9 @@ WsPlan plan(int B, int H, int T, int D, int dtype, int is_bwd, int Hkv = 0) {
     p.dq_acc = off; off += round_up(n * sizeof(float));
     p.q16 = off;    off += round_up(n * 2);
     p.k16 = off;    off += round_up(n * 2);
-    p.qinv = off;     off += round_up(tiles * 4 * sizeof(float));
-    p.kinv = off;     off += round_up(tiles * sizeof(float));
-    p.dmax = off;     off += round_up(tiles * sizeof(float));
-    p.deltamax = off; off += round_up(tiles * sizeof(float));
+    p.qfac = off;   off += round_up(tiles * 4 * sizeof(float));
+    p.kfac = off;   off += round_up(tiles * sizeof(float));
+    p.hstat = off;  off += round_up((size_t)B * H * 4 * sizeof(float));
     p.split = choose_split(B, H, Hkv, T);
     if (p.split > 1) {
       const size_t nkv = bt * Hkv * D;
@@ -90,7 +89,7 @@ WsPlan plan(int B, int H, int T, int D, int dtype, int is_bwd, int Hkv = 0) {
   if (dtype == ATTN_BF16 && !is_bwd) {
     p.q16 = off;  off += round_up(n * 2);
     p.k16 = off;  off += round_up(n * 2);
-    p.qfac = off; off += round_up(tiles * sizeof(float));
+    p.qfac = off; off += round_up(tiles * 4 * sizeof(float));
     p.kfac = off; off += round_up(tiles * sizeof(float));
   }
   p.total = off;
@@ -236,7 +235,7 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
     kf = (float*)(ws + wp.kfac);
     ATTN_LAUNCH(KK_ROPE_PREP, st, pdl_launch(rope_prep_kernel<D>, dim3(nt, BH, 2), kRopePrepThreads, 0, st,
                                              (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds,
-                                             qh, kh, qf, kf, B, H, Hkv, T, nt));
+                                             qh, kh, qf, kf, (float*)nullptr, B, H, Hkv, T, nt));
     if (launch_status()) return ATTN_ECUDA;
     qs = qh;
     ks = kh;
@@ -267,16 +266,49 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
   return launch_status();
 }
 
-template <int D, bool kF16>
+template <int D, bool kF16, bool kDQ>
 int launch_dkdv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                 const CUtensorMap& mo, const CUtensorMap& mdq, const bwd100::Params& prm,
                 unsigned grid, cudaStream_t st) {
-  using L = bwd100::Layout<D>;
+  using L = bwd100::Layout<D, kDQ>;
   static bool smem_set[64] = {};
-  if (!ensure_smem(bwd100::dkdv_kernel<D, kF16>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
-  ATTN_LAUNCH(KK_DKDV, st, pdl_launch(bwd100::dkdv_kernel<D, kF16>, grid, L::kThreads,
+  if (!ensure_smem(bwd100::dkdv_kernel<D, kF16, kDQ>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
+  ATTN_LAUNCH(KK_DKDV, st, pdl_launch(bwd100::dkdv_kernel<D, kF16, kDQ>, grid, L::kThreads,
                                        L::kSmemAlloc, st, mq, mk, mv, mo, mdq, prm));
   return launch_status();
+}
+
+template <int D, bool kF16>
+int launch_dq(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+              const CUtensorMap& mo, const dq100::Params& prm, unsigned grid, cudaStream_t st) {
+  using L = dq100::Layout<D>;
+  static bool smem_set[64] = {};
+  if (!ensure_smem(dq100::dq_kernel<D, kF16>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
+  ATTN_LAUNCH(KK_DQ, st, pdl_launch(dq100::dq_kernel<D, kF16>, grid, L::kThreads, L::kSmemAlloc,
+                                     st, mq, mk, mv, mo, prm));
+  return launch_status();
+}
+
+// dQ by the query-tile pass (dq_sm100.cuh: two more products per tile pair,
+// no fp32 accumulator, no atomics, no zeroing or finishing pass) or by
+// reduce-adds from the key-tile kernel: a per-head-size choice, set by
+// measuring both on the B200 (the measurement is recorded with the library's
+// design notes).
+// The test build (build.py --debug) takes the other route, so the GPU tests
+// cover both.
+#ifndef ATTN_DQ_PASS_D64
+#define ATTN_DQ_PASS_D64 0
+#endif
+#ifndef ATTN_DQ_PASS_D128
+#define ATTN_DQ_PASS_D128 0
+#endif
+#ifdef ATTN_DQ_ROUTE_SWAPPED
+constexpr bool kDqRouteSwapped = true;
+#else
+constexpr bool kDqRouteSwapped = false;
+#endif
+constexpr bool use_dq_pass(int D) {
+  return (D == 64 ? ATTN_DQ_PASS_D64 : ATTN_DQ_PASS_D128) != kDqRouteSwapped;
 }
 
 template <int D>
@@ -296,29 +328,25 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   float* delta = (float*)(ws + wp.delta);
   float* lse2 = (float*)(ws + wp.lse2);
   float* dq_acc = (float*)(ws + wp.dq_acc);
-  float* qinv = (float*)(ws + wp.qinv);
-  float* kinv = (float*)(ws + wp.kinv);
-  float* dmax = (float*)(ws + wp.dmax);
-  float* deltamax = (float*)(ws + wp.deltamax);
+  float* qinv = (float*)(ws + wp.qfac);
+  float* kinv = (float*)(ws + wp.kfac);
+  float* hstat = f16 ? (float*)(ws + wp.hstat) : nullptr;
   const int split = wp.split;
   float* dk_acc = split > 1 ? (float*)(ws + wp.dk_acc) : nullptr;
   float* dv_acc = split > 1 ? (float*)(ws + wp.dv_acc) : nullptr;
-  const dim3 pgrid(nt, BH);
   if (f16) {
-    ATTN_LAUNCH(KK_DELTA, st, pdl_launch(bwd_prep_kernel<D, true>, pgrid, kBwdPrepThreads, 0, st,
-                                         (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse,
-                                         delta, lse2, dq_acc, (const __nv_bfloat16*)q,
-                                         (const __nv_bfloat16*)k, rc, rs, ds, q16, k16, qinv,
-                                         kinv, dmax, deltamax, dk_acc, dv_acc, B, H, Hkv, T, Tpad,
-                                         nt));
-  } else {
-    ATTN_LAUNCH(KK_DELTA, st, pdl_launch(bwd_prep_kernel<D, false>, pgrid, kBwdPrepThreads, 0, st,
-                                         (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse,
-                                         delta, lse2, dq_acc, (const __nv_bfloat16*)q,
-                                         (const __nv_bfloat16*)k, rc, rs, ds, q16, k16, qinv,
-                                         kinv, dmax, deltamax, dk_acc, dv_acc, B, H, Hkv, T, Tpad,
-                                         nt));
+    // the forward's rotation, factors included (same kernel, same values)
+    ATTN_LAUNCH(KK_ROPE_PREP, st, pdl_launch(rope_prep_kernel<D>, dim3(nt, BH, 2), kRopePrepThreads, 0, st,
+                                             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds,
+                                             q16, k16, qinv, kinv, hstat, B, H, Hkv, T, nt));
+    if (launch_status()) return ATTN_ECUDA;
   }
+  const bool dq_pass = use_dq_pass(D);
+  const long rows_pad = (long)BH * Tpad;
+  ATTN_LAUNCH(KK_DELTA, st, pdl_launch(bwd_prep_kernel<D>, (unsigned)(rows_pad * (D / 8) / 256), 256, 0, st,
+                                       (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse, delta, lse2,
+                                       dq_pass ? nullptr : dq_acc, dk_acc, dv_acc,
+                                       (const __nv_bfloat16*)v, hstat, H, Hkv, T, Tpad, rows_pad));
   if (launch_status()) return ATTN_ECUDA;
   CUtensorMap mq, mk, mv, mo, mdq;
   if (!make_tile_map(&mq, qs, f16, D, T, BH) || !make_tile_map(&mk, ks, f16, D, T, BHkv) ||
@@ -348,22 +376,49 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   prm.dv_acc = dv_acc;
   prm.qinv = qinv;
   prm.kinv = kinv;
-  prm.dmax = dmax;
-  prm.deltamax = deltamax;
+  prm.hstat = hstat;
   const unsigned grid = (unsigned)(nt * BHkv * split);
-  const int rc_k = f16 ? launch_dkdv<D, true>(mq, mk, mv, mo, mdq, prm, grid, st)
-                       : launch_dkdv<D, false>(mq, mk, mv, mo, mdq, prm, grid, st);
+  int rc_k;
+  if (dq_pass)
+    rc_k = f16 ? launch_dkdv<D, true, false>(mq, mk, mv, mo, mdq, prm, grid, st)
+               : launch_dkdv<D, false, false>(mq, mk, mv, mo, mdq, prm, grid, st);
+  else
+    rc_k = f16 ? launch_dkdv<D, true, true>(mq, mk, mv, mo, mdq, prm, grid, st)
+               : launch_dkdv<D, false, true>(mq, mk, mv, mo, mdq, prm, grid, st);
   if (rc_k) return rc_k;
   if (split > 1) {
     // dk = R^T (scale * sum of the parts), dv = sum of the parts
     const long n8kv = (long)BHkv * T * D / 8;
-    ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)((n8kv + 255) / 256), 256, 0, st, dk_acc, rc, rs, ds, (__nv_bfloat16*)dk, Hkv, T, scale, n8kv));
+    ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)((n8kv + 255) / 256), 256, 0, st, dk_acc, rc, rs, ds, (__nv_bfloat16*)dk, Hkv, T, scale, n8kv, (const float*)nullptr, (const float*)nullptr, Hkv, nt));
     if (launch_status()) return ATTN_ECUDA;
-    ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)((n8kv + 255) / 256), 256, 0, st, dv_acc, nullptr, nullptr, nullptr, (__nv_bfloat16*)dv, Hkv, T, 1.0f, n8kv));
+    ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)((n8kv + 255) / 256), 256, 0, st, dv_acc, nullptr, nullptr, nullptr, (__nv_bfloat16*)dv, Hkv, T, 1.0f, n8kv, (const float*)nullptr, (const float*)nullptr, Hkv, nt));
     if (launch_status()) return ATTN_ECUDA;
   }
+  if (dq_pass) {
+    dq100::Params qp;
+    qp.T = T;
+    qp.H = H;
+    qp.Hkv = Hkv;
+    qp.BH = BH;
+    qp.n_tiles = nt;
+    qp.Tpad = Tpad;
+    qp.scale_log2 = scale * 1.4426950408889634f;
+    qp.scale = scale;
+    qp.lse2 = lse2;
+    qp.delta = delta;
+    qp.doc_start = ds;
+    qp.rope_cos = rc;
+    qp.rope_sin = rs;
+    qp.qinv = qinv;
+    qp.kinv = kinv;
+    qp.hstat = hstat;
+    qp.dq = (__nv_bfloat16*)dq;
+    const unsigned qgrid = (unsigned)(nt * BH);
+    return f16 ? launch_dq<D, true>(mq, mk, mv, mo, qp, qgrid, st)
+               : launch_dq<D, false>(mq, mk, mv, mo, qp, qgrid, st);
+  }
   const long n8 = (long)BH * T * D / 8;
-  ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)((n8 + 255) / 256), 256, 0, st, dq_acc, rc, rs, ds, (__nv_bfloat16*)dq, H, T, scale, n8));
+  ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)((n8 + 255) / 256), 256, 0, st, dq_acc, rc, rs, ds, (__nv_bfloat16*)dq, H, T, scale, n8, f16 ? (const float*)qinv : nullptr, (const float*)hstat, Hkv, nt));
   return launch_status();
 }
 
@@ -499,15 +554,17 @@ const char* attn_error_string(int code) {
 
 unsigned long long attn_launch_count(void) { return trace::launches(); }
 
-int attn_tile_counts(unsigned long long* fwd_tiles, unsigned long long* bwd_tiles) {
-  if (!fwd_tiles || !bwd_tiles) return ATTN_EINVAL;
+int attn_tile_counts(unsigned long long* fwd_tiles, unsigned long long* bwd_tiles,
+                     unsigned long long* dq_tiles) {
+  if (!fwd_tiles || !bwd_tiles || !dq_tiles) return ATTN_EINVAL;
   if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ECUDA;
-  unsigned long long v[2] = {0, 0};
+  unsigned long long v[3] = {0, 0, 0};
   if (cudaMemcpyFromSymbol(v, g_attn_tiles, sizeof(v)) != cudaSuccess) return ATTN_ECUDA;
-  const unsigned long long z[2] = {0, 0};
+  const unsigned long long z[3] = {0, 0, 0};
   if (cudaMemcpyToSymbol(g_attn_tiles, z, sizeof(z)) != cudaSuccess) return ATTN_ECUDA;
   *fwd_tiles = v[0];
   *bwd_tiles = v[1];
+  *dq_tiles = v[2];
   return ATTN_OK;
 }
 

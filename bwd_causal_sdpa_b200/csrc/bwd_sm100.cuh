@@ -35,17 +35,18 @@
 // Operand types. Without RoPE every product reads bf16 (q, k as given, P^T
 // and dS^T rounded to bf16). With RoPE (kF16) the scores are recomputed from
 // the forward's own operands: the rotated q, k stored as fp16 times a
-// power-of-two factor per 128-row tile (the backward preprocessing writes the
-// same values the forward computed), so P matches the forward's lse. The
-// products that pair dS with those operands (dK = dS^T Q, dQ = dS K) then
-// need dS in fp16 as well, stored as dS * C * qinv_i: qinv_i (the inverse of
-// query tile i's factor) cancels that tile's factor in dK, which therefore
-// accumulates C dS^T Q for every tile, and C, a power of two per CTA, keeps
-// every stored value below 2^14 (from |dS_ij| <= |dO_i| max_j |v_j| +
-// |Delta_i|, the per-tile maxima the preprocessing recorded and this CTA's
-// own value rows). dK is divided by C in the epilogue and each dQ_i tile by
-// C qinv_i / kinv (kinv: this key tile's factor) before it is added. P^T and
-// dO stay bf16 for dV, and V, dO for dP.
+// power-of-two factor per 128-row tile (the preprocessing writes the same
+// values the forward computed), so P matches the forward's lse. The products
+// that pair dS with those operands (dK = dS^T Q, dQ = dS K) then need dS in
+// fp16 as well, stored as dS * C * qinv_i: qinv_i (the inverse of query tile
+// i's factor) cancels that tile's factor in dK, which therefore accumulates
+// C dS^T Q over all tiles, and C, a power of two per CTA, keeps every stored
+// value below 2^14 (from |dS_ij| <= |dO_i| max_j |v_j| + |Delta_i|). With the
+// dQ warpgroup, C = Cg * kinv (kinv: this key tile's inverse factor, Cg one
+// power of two per key/value head), so every key tile adds Cg qinv_i dS K to
+// query tile i's dQ and the finishing pass divides that out; without it
+// (dQ from the query-tile pass), C is this CTA's own. dK is divided by C in
+// the epilogue. P^T and dO stay bf16 for dV, and V, dO for dP.
 //
 // Sources (page, section): ARK README, "Backward pass (AutoGrad)" (attention
 // gradients inside training); Forge README, finding 3 (key-tile-parallel dK/dV
@@ -61,11 +62,15 @@ namespace bwd100 {
 
 using namespace sm100;
 
-template <int D>
+// kDQ: the kernel also forms dQ_i = dS K per query tile and adds it into the
+// fp32 accumulator (its own warpgroup and staging ring); without it dQ comes
+// from the query-tile pass (dq_sm100.cuh) and the freed shared memory holds a
+// second dO stage at D = 128.
+template <int D, bool kDQ = true>
 struct Layout {
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr int kBlockBytes = 128 * 128;
-  static constexpr int kDOStages = (D == 128) ? 1 : 2;
+  static constexpr int kDOStages = (D == 128 && kDQ) ? 1 : 2;
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTileBytes;
   static constexpr int kQ = kV + kTileBytes;                  // 2 stages
@@ -75,9 +80,10 @@ struct Layout {
   // dQ_i staging ring: two buffers of 128 query rows x 32 fp32 columns, each
   // four 32 x 32 boxes (4 KB, 128-byte swizzle), one per dQ warp.
   static constexpr int kXS = kLD + 2 * 1024;  // 1024-byte aligned (128-byte swizzle)
-  static constexpr int kXSBuf = 128 * 32 * 4;
-  // per elementwise warp: largest qinv, |dO_i|, |Delta_i| of this CTA's query
-  // tiles and of its key rows' value norms over its columns (f32 [16][4])
+  static constexpr int kXSBuf = kDQ ? 128 * 32 * 4 : 0;
+  // per warp that makes C: largest qinv, |dO_i|, |Delta_i| of this CTA's
+  // query tiles and of its key rows' value norms (f32 [16][4]); with the dQ
+  // warpgroup, C itself in the last slot
   static constexpr int kStats = kXS + 2 * kXSBuf;
   // per Q stage: the query tile's inverse factor record (16 bytes, qinv first)
   static constexpr int kQInv = kStats + 16 * 4 * 4;
@@ -103,10 +109,11 @@ struct Layout {
   static constexpr int kQC = 128 / kNWG;
   static constexpr int kDC = D / kNWG;
   static constexpr int kEwThreads = 128 * kNWG;
-  static constexpr int kDqWarp0 = 4 * kNWG;  // the dQ warpgroup: warps kDqWarp0 .. +3
-  static constexpr int kProducerWarp = 4 * kNWG + 4, kMmaWarp = 4 * kNWG + 5;
-  static constexpr int kThreads = kEwThreads + 128 + 64;
+  static constexpr int kDqWarp0 = 4 * kNWG;  // the dQ warpgroup: warps kDqWarp0 .. +3 (kDQ)
+  static constexpr int kProducerWarp = 4 * kNWG + (kDQ ? 4 : 0), kMmaWarp = kProducerWarp + 1;
+  static constexpr int kThreads = kEwThreads + (kDQ ? 128 : 0) + 64;
   static_assert(kXS % 1024 == 0, "the dQ staging boxes use the 128-byte swizzle");
+  static_assert(kDQ || kThreads == 576, "without dQ: 16 elementwise warps, TMA and MMA warps");
   static_assert(kBytes <= 232448, "more shared memory than a CTA may use");
 };
 
@@ -128,16 +135,17 @@ struct Params {
   float* dv_acc;
   // fp16 operands (RoPE): inverse tile factors of the stored q, one 16-byte
   // record per tile ([B*H][n_tiles][4], value first), and of the stored k
-  // ([B*Hkv][n_tiles]), and per query tile the largest |dO_i| and |Delta_i|
+  // ([B*Hkv][n_tiles]), and per query head the largest |dO_i| and |Delta_i|
+  // ([B*H][4]: dO, Delta, then v of the key/value head of that index)
   const float* qinv;
   const float* kinv;
-  const float* dmax;
-  const float* deltamax;
+  float* hstat;  // with the dQ warpgroup, slot 3 of each key/value head receives Cg
 };
 
 // The power of two C that keeps every stored dS * C * qinv_i below 2^14,
 // from X = max qinv_i * (max |dO_i| * max |v_j| + max |Delta_i|) >= max
-// |dS_ij| qinv_i; 1 when X is zero (dS is then zero too).
+// |dS_ij| qinv_i (maxima over this CTA's query tiles, its query heads and its
+// key rows); 1 when X is zero (dS is then zero too).
 __device__ __forceinline__ float ds_scale(float X) {
   if (!(X > 0.f && X <= 3.0e38f)) return 1.f;
   return ldexpf(1.f, max(-100, min(100, 13 - ilogbf(X))));
@@ -149,13 +157,13 @@ __device__ __forceinline__ uint32_t sw128(int r, int ch) {
   return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4));
 }
 
-template <int D, bool kF16>
-__global__ void __launch_bounds__(Layout<D>::kThreads, 1)
+template <int D, bool kF16, bool kDQ>
+__global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                 const __grid_constant__ CUtensorMap tmDQ, const Params p) {
   pdl_wait_and_trigger();
-  using L = Layout<D>;
+  using L = Layout<D, kDQ>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sb0 = smem_u32(smem_raw);
   if (sb0 & 1023u) {  // uniform across the CTA: nothing has been issued yet
@@ -205,7 +213,9 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     mbar_init(bar(L::bDSFree), 1);
     mbar_init(bar(L::bDQFree), 128);
     mbar_init(bar(L::bFinal), 1);
-    mbar_init(bar(L::bStats), L::kEwThreads);
+    // C is made by the dQ warpgroup when there is one (it is idle until the
+    // first dQ), else by the elementwise warps
+    mbar_init(bar(L::bStats), kDQ ? 128 : L::kEwThreads);
     *abort_flag = 0;
     fence_barrier_init();
     atomicAdd(&g_attn_tiles[1], (unsigned long long)n_it);
@@ -336,7 +346,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       int nS = 0, nP = 0, nV = 0, nK = 0, nQ = 0;  // next tile of each group
       bool ok = mbar_wait(bar(L::bKV), 0, abort_flag);
       long long t_last = clock64();
-      while (ok && nQ < n_it) {
+      while (ok && (kDQ ? nQ : nK) < n_it) {
         if (nV < nP && mbar_test(bar(L::bPFull), nV & 1)) {
           // dV += P^T dO (P^T K-major in the P/dS tile, dO MN-major)
           tc_fence_after();
@@ -349,8 +359,10 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
           mma_commit(bar(L::bDOEmpty + nV % L::kDOStages));
           ++nV;
         } else if (nS < n_it && mbar_test(bar(L::bQFull + (nS & 1)), (nS >> 1) & 1) &&
-                   (nS == 0 || (nS == 1 ? mbar_test(bar(L::bSFree), 0)
-                                        : (nQ > nS - 2 && mbar_test(bar(L::bDQFree), nS & 1))))) {
+                   (nS == 0 ||
+                    (kDQ ? (nS == 1 ? mbar_test(bar(L::bSFree), 0)
+                                    : (nQ > nS - 2 && mbar_test(bar(L::bDQFree), nS & 1)))
+                         : mbar_test(bar(L::bSFree), (nS - 1) & 1)))) {
           // S^T(i) = K Q(i)^T
           tc_fence_after();
 #pragma unroll
@@ -370,9 +382,10 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
                    smem_desc_sw128(qbuf(nK) + kk * 2048, L::kBlockBytes, 1024), id_dk,
                    (nK > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(L::bQEmpty + (nK & 1)));
+          if (!kDQ) mma_commit(bar(L::bDSFree));  // the P/dS tile is free again
           if (nK == n_it - 1) mma_commit(bar(L::bFinal));
           ++nK;
-        } else if (nQ < nK && (nQ == n_it - 1 ||
+        } else if (kDQ && nQ < nK && (nQ == n_it - 1 ||
                                (nS > nQ + 1 && mbar_test(bar(L::bSFree), (nQ + 1) & 1)))) {
           // dQ_i = dS K (dS read MN-major), into the S^T columns
           tc_fence_after();
@@ -408,7 +421,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         t_last = clock64();
       }
     }
-  } else if (warp >= L::kDqWarp0) {
+  } else if (kDQ && warp >= L::kDqWarp0) {
     // ---------------- dQ warpgroup (lane = query row) ----------------
     // Per query tile: read dQ_i out of the S^T columns in 32-column chunks
     // (releasing the columns after the last read), stage each chunk as this
@@ -423,17 +436,58 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     float cscale = 1.f;
     bool okq = true;
     if constexpr (kF16) {
-      okq = mbar_wait(bar(L::bStats), 0, abort_flag);
-      if (okq) cscale = cta_ds_scale();
+      // C for this CTA, made here. Every CTA that adds into a query head's
+      // dQ accumulator must carry the same factor per query tile, so C is
+      // Cg * kinv (this key tile's inverse factor, which then cancels in dQ),
+      // with Cg one power of two per key/value head: from the largest qinv
+      // and kinv over all of that head's tiles, |dO_i| and |Delta_i| over its
+      // query heads and |v_j| over its keys (the preprocessing's per-head
+      // maxima). dQ then accumulates Cg qinv_i dS K for query tile i, which
+      // the finishing pass divides out; Cg is left in the head's fourth
+      // statistics slot for it. Published to the elementwise warps in the
+      // last statistics slot.
+      const int tq = threadIdx.x - 32 * L::kDqWarp0;  // 0..127
+      const int Gf = p.H / p.Hkv;
+      const int bhq_first = b * p.H + (bhk - b * p.Hkv) * Gf;  // the group's query heads follow
+      float qm = 0.f, km = 0.f, dm = 0.f, dl = 0.f;
+      for (int e = tq; e < Gf * p.n_tiles; e += 128)
+        qm = fmaxf(qm, p.qinv[((size_t)bhq_first * p.n_tiles + e) * 4]);
+      for (int e = tq; e < p.n_tiles; e += 128) km = fmaxf(km, p.kinv[(size_t)bhk * p.n_tiles + e]);
+      for (int g = tq; g < Gf; g += 128) {
+        dm = fmaxf(dm, p.hstat[4 * (bhq_first + g)]);
+        dl = fmaxf(dl, p.hstat[4 * (bhq_first + g) + 1]);
+      }
+      qm = warp_max(qm);
+      km = warp_max(km);
+      dm = warp_max(dm);
+      dl = warp_max(dl);
+      if (lane == 0) {
+        float* e = stats + 4 * sub;
+        e[0] = qm;
+        e[1] = km;
+        e[2] = dm;
+        e[3] = dl;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // the four dQ warps, none exits early
+#pragma unroll
+      for (int w4 = 0; w4 < 4; ++w4) {
+        qm = fmaxf(qm, stats[4 * w4]);
+        km = fmaxf(km, stats[4 * w4 + 1]);
+        dm = fmaxf(dm, stats[4 * w4 + 2]);
+        dl = fmaxf(dl, stats[4 * w4 + 3]);
+      }
+      const float cg = ds_scale(qm * km * fmaf(dm, p.hstat[4 * bhk + 2], dl));
+      cscale = cg * kinv_cta;
+      if (tq == 0) {
+        stats[63] = cscale;
+        if (kt == 0 && part == 0) p.hstat[4 * bhk + 3] = cg;
+      }
+      mbar_arrive(bar(L::bStats));
     }
     for (int it = 0; okq && it < n_it; ++it) {
       const int gi = it / n_q;
       const int i0 = (qt0 + it - gi * n_q) * 128;
       const bool rows_in = i0 + 32 * sub < T;  // rows past T are clipped by the map
-      // dQ_i as computed from the scaled operands, back to dS K
-      const float mulq =
-          kF16 ? kinv_cta / (cscale * p.qinv[((size_t)(bhq0 + gi) * p.n_tiles + (i0 >> 7)) * 4])
-               : 1.f;
       if (!mbar_wait(bar(L::bDQFull), it & 1, abort_flag)) break;
       tc_fence_after();
 #pragma unroll 1
@@ -452,10 +506,6 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         }
         __syncwarp();
         uint8_t* bx = sg + L::kXS + buf * L::kXSBuf + sub * 4096;
-        if constexpr (kF16) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * mulq);
-        }
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           *reinterpret_cast<uint4*>(bx + sw128(lane, e)) =
@@ -488,21 +538,29 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     bool ok = true;
     float cscale = 1.f;  // C (fp16 operands)
     float qinv_i = 1.f;  // inverse factor of the current query tile (fp16 operands)
-    if constexpr (kF16) {
-      // Post this warp's share of the statistics C is made from: the largest
-      // qinv, |dO_i| and |Delta_i| over this CTA's query tiles, and the
-      // largest norm of this warpgroup's columns of the value rows.
+    // fp16 operands: this warp's share of the statistics C is made from (the
+    // largest qinv over this CTA's query tiles, |dO_i| and |Delta_i| over its
+    // query heads, and the largest norm of this warpgroup's columns of the
+    // value rows) is posted after the first P tile (C is needed from the
+    // first dS tile on); the per-tile values are prefetched into L1 here.
+    auto stat_index = [&](int e) -> size_t {
+      const int gi = e / n_q;
+      return (size_t)(bhq0 + gi) * p.n_tiles + qt0 + (e - gi * n_q);
+    };
+    if constexpr (kF16 && !kDQ) {
+      for (int e = threadIdx.x; e < n_it; e += L::kEwThreads)
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(p.qinv + stat_index(e) * 4));
+    }
+    auto post_stats = [&]() -> bool {
       float qm = 0.f, dm = 0.f, dl = 0.f;
-      for (int e = threadIdx.x; e < n_it; e += L::kEwThreads) {
-        const int gi = e / n_q;
-        const size_t ix = (size_t)(bhq0 + gi) * p.n_tiles + qt0 + (e - gi * n_q);
-        qm = fmaxf(qm, p.qinv[ix * 4]);
-        dm = fmaxf(dm, p.dmax[ix]);
-        dl = fmaxf(dl, p.deltamax[ix]);
+      for (int e = threadIdx.x; e < n_it; e += L::kEwThreads) qm = fmaxf(qm, p.qinv[stat_index(e) * 4]);
+      for (int g = threadIdx.x; g < G; g += L::kEwThreads) {
+        dm = fmaxf(dm, p.hstat[4 * (bhq0 + g)]);
+        dl = fmaxf(dl, p.hstat[4 * (bhq0 + g) + 1]);
       }
       float vn = 0.f;
-      ok = mbar_wait(bar(L::bKV), 0, abort_flag);
-      if (ok) {
+      bool okv = mbar_wait(bar(L::bKV), 0, abort_flag);
+      if (okv) {
         const uint8_t* vb = sg + L::kV + (dc0 >> 6) * L::kBlockBytes;
 #pragma unroll
         for (int e = 0; e < DC / 8; ++e) {
@@ -528,9 +586,10 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         e[3] = vn;
       }
       mbar_arrive(bar(L::bStats));
-      ok = ok && mbar_wait(bar(L::bStats), 0, abort_flag);
-      if (ok) cscale = cta_ds_scale();
-    }
+      okv = okv && mbar_wait(bar(L::bStats), 0, abort_flag);
+      if (okv) cscale = cta_ds_scale();
+      return okv;
+    };
     // Row r, query columns [qc0, qc0 + QC) of the P/dS tile (bf16 pairs in
     // w[]): 64-column block col/64, 16-byte chunks (col%64)/8 onwards.
     auto store_row = [&](const uint32_t* w) {
@@ -627,7 +686,19 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       mbar_arrive(bar(L::bDSFull));
       return true;
     };
-    for (int it = 0; ok && it < n_it; ++it) ok = phase_P(it) && phase_dS(it);
+    // the first tile is peeled: C is made (without the dQ warpgroup) or picked
+    // up (with it) between its P and dS
+    ok = phase_P(0);
+    if constexpr (kF16) {
+      if constexpr (kDQ) {
+        ok = ok && mbar_wait(bar(L::bStats), 0, abort_flag);
+        if (ok) cscale = stats[63];
+      } else {
+        ok = post_stats() && ok;  // every thread arrives, even after a failed wait
+      }
+    }
+    ok = ok && phase_dS(0);
+    for (int it = 1; ok && it < n_it; ++it) ok = phase_P(it) && phase_dS(it);
     // ---- epilogue: dK = R^T (scale * dK_r), dV ----
     if (ok && mbar_wait(bar(L::bFinal), 0, abort_flag)) {
       tc_fence_after();

@@ -23,9 +23,9 @@ __device__ __forceinline__ void report_status(int code) {
 
 // Executed tile products of the tensor-core kernels since the last read by
 // attn_tile_counts(): [0] forward (128-query x 128-key tiles a forward CTA
-// computes), [1] backward (the same unit in the key-tile kernel). One atomic
-// add per CTA.
-__device__ unsigned long long g_attn_tiles[2];
+// computes), [1] backward key-tile kernel, [2] backward query-tile (dQ) pass,
+// in the same unit. One atomic add per CTA.
+__device__ unsigned long long g_attn_tiles[3];
 
 #ifdef ATTN_DEBUG_HOOKS
 // Watchdog test build only: a load the forward's TMA warp withholds (0 = none,
@@ -113,25 +113,37 @@ __device__ __forceinline__ float warp_max(float x) {
 // fp16 storage of rotated q / k tiles: fp16 keeps 3 more mantissa bits than
 // bf16 (which the lse bound needs) but has a narrow range (overflow above
 // 65504, subnormals below 2^-14). A 128-row tile is therefore stored times
-// the power of two that brings a bound amax on its magnitudes (its largest
-// pair norm) into [2^14, 2^15): large tiles cannot overflow and small ones
-// keep all 11 bits down to 2^-28 of their maximum. The exponent is clamped so
+// the power of two that brings its largest magnitude amax into [2^14, 2^15):
+// large tiles cannot overflow and small ones keep all 11 bits down to 2^-28
+// of their maximum. The exponent is clamped so
 // that the factor and its inverse stay normal floats; an all-zero tile keeps
 // factor 1.
 __device__ __forceinline__ float fp16_tile_factor(float amax) {
   if (!(amax > 0.f && amax <= 3.0e38f)) return 1.f;
   return ldexpf(1.f, max(-100, min(100, 14 - ilogbf(amax))));
 }
-// The largest squared Euclidean norm of the four pairs (x[2i], x[2i+1]) of
-// eight values. A rotation keeps each pair's norm, so its values never exceed
-// it: the largest pair norm of a tile, taken before rotating, bounds the
-// rotated tile and fixes its factor (every kernel that stores a rotated tile
-// derives the factor this way, from the same bf16 inputs).
-__device__ __forceinline__ float pair_norm2_max8(const float* x) {
-  float m = 0.f;
+// RoPE table entries for eight consecutive dimensions d0.. (d0 a multiple of
+// 8) at position pos: four pairs' cos and sin, one 16-byte load each (the
+// tables must be 16-byte aligned); rotate8 applies them with the same
+// roundings as rope_pairs.
+struct Rope8 {
+  float4 c, s;
+};
+template <int D>
+__device__ __forceinline__ Rope8 rope8_load(const float* rc, const float* rs, int pos, int d0) {
+  Rope8 t;
+  t.c = *reinterpret_cast<const float4*>(rc + (size_t)pos * (D / 2) + (d0 >> 1));
+  t.s = *reinterpret_cast<const float4*>(rs + (size_t)pos * (D / 2) + (d0 >> 1));
+  return t;
+}
+__device__ __forceinline__ void rotate8(float* x, const Rope8& t) {
+  const float cs[4] = {t.c.x, t.c.y, t.c.z, t.c.w}, sn[4] = {t.s.x, t.s.y, t.s.z, t.s.w};
 #pragma unroll
-  for (int e = 0; e < 4; ++e) m = fmaxf(m, fmaf(x[2 * e], x[2 * e], __fmul_rn(x[2 * e + 1], x[2 * e + 1])));
-  return m;
+  for (int e = 0; e < 4; ++e) {
+    const float x0 = x[2 * e], x1 = x[2 * e + 1];
+    x[2 * e] = fmaf(x0, cs[e], -__fmul_rn(x1, sn[e]));
+    x[2 * e + 1] = fmaf(x0, sn[e], __fmul_rn(x1, cs[e]));
+  }
 }
 
 // Eight floats times f as eight fp16 values (round to nearest even).

@@ -81,7 +81,8 @@ struct Params {
   float scale_log2;          // scale * log2(e)
   uint32_t idesc_s;          // instruction descriptor of S = Q K^T
   const float* q_fac;        // inverse power-of-two factor per (query head, tile) of the
-                             // stored rotated q, or null (q as given)
+                             // stored rotated q, one 16-byte record each (value first),
+                             // or null (q as given)
   const float* k_fac;        // the same per (key/value head, tile) for k
   const int32_t* doc_start;  // flattened document starts, or null
   __nv_bfloat16* o;
@@ -280,7 +281,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     const uint32_t tO = tS + 128;
     float* xch = reinterpret_cast<float*>(sg + L::kXch);  // [parity][tile][half][row]
     const int ds_i = p.doc_start ? p.doc_start[row0 + min(i, T - 1)] - row0 : 0;
-    const float fq = p.q_fac ? p.q_fac[bh * p.n_qtiles + min(qt, p.n_qtiles - 1)] : 1.f;
+    const float fq = p.q_fac ? p.q_fac[((size_t)bh * p.n_qtiles + min(qt, p.n_qtiles - 1)) * 4] : 1.f;
     float m = -INFINITY, l = 0.f;
     bool ok = active;
     for (int it = 0; ok && it < n_t; ++it) {

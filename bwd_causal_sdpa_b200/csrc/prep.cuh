@@ -84,13 +84,19 @@ __global__ void __launch_bounds__(256) delta_kernel(const TIO* __restrict__ o, c
   if (lane == 0) delta[row] = s;
 }
 
-// RoPE pre-pass for the forward: rotate q and k once (fp32 arithmetic,
+// RoPE pre-pass of both passes: rotate q and k once (fp32 arithmetic,
 // interleaved pairs at the token's document position) and store every
-// 128-row tile as fp16 times its power-of-two factor (fp16_tile_factor of the
-// tile's largest pair norm); fac[] receives the inverse factor (exact), which
-// the forward folds into its score scale. blockIdx = (128-row tile, head,
-// 0 for q / 1 for k); the head is b*H + h for q and b*Hkv + h for k (blocks
-// past B*Hkv return at once).
+// 128-row tile as fp16 times its power-of-two factor (fp16_tile_factor of
+// the tile's largest rotated magnitude). qfac receives the inverse factor of
+// each q tile as a 16-byte record (value first, so the backward's main kernel
+// can bulk-load it with the tile), kfac that of each k tile; the forward
+// folds them into its score scale and the backward's main kernel into its
+// own, which therefore recomputes the forward's scores exactly (same kernel,
+// same inputs, same values). blockIdx = (128-row tile, head, 0 for q / 1 for
+// k); the head is b*H + h for q and b*Hkv + h for k (blocks past B*Hkv
+// return at once). hstat (backward only, else null): the first block of each
+// head zeroes that head's four statistics slots, which the row pass that
+// follows fills.
 constexpr int kRopePrepThreads = 512;
 
 template <int D>
@@ -98,8 +104,8 @@ __global__ void __launch_bounds__(kRopePrepThreads) rope_prep_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const float* __restrict__ rc, const float* __restrict__ rs,
     const int32_t* __restrict__ doc_start, __half* __restrict__ qo, __half* __restrict__ ko,
-    float* __restrict__ qfac, float* __restrict__ kfac, int B, int H, int Hkv, int T,
-    int ntiles) {
+    float* __restrict__ qfac, float* __restrict__ kfac, float* __restrict__ hstat, int B, int H,
+    int Hkv, int T, int ntiles) {
   pdl_wait_and_trigger();
   constexpr int CH = D / 8;              // 16-byte chunks per row
   constexpr int NT = kRopePrepThreads;
@@ -107,11 +113,12 @@ __global__ void __launch_bounds__(kRopePrepThreads) rope_prep_kernel(
   const int tile = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const int heads = which ? Hkv : H;
   if (bh >= B * heads) return;  // k has fewer heads than q
+  if (hstat && which == 0 && tile == 0 && threadIdx.x < 4) hstat[4 * bh + threadIdx.x] = 0.f;
   const int b = bh / heads, row0 = b * T, t0 = tile * 128;
   const __nv_bfloat16* src = which ? k : q;
   __half* dst = which ? ko : qo;
   float v[PER][8];
-  float n2 = 0.f;
+  float amax = 0.f;
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
     const int idx = threadIdx.x + u * NT, r = idx / CH, c8 = idx % CH, t = t0 + r;
@@ -122,23 +129,28 @@ __global__ void __launch_bounds__(kRopePrepThreads) rope_prep_kernel(
       const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[u][e] = __bfloat162float(h[e]);
-      n2 = fmaxf(n2, pair_norm2_max8(v[u]));
+      rotate8(v[u], rope8_load<D>(rc, rs, t - (doc_start ? doc_start[row0 + t] - row0 : 0), c8 * 8));
+#pragma unroll
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[u][e]));
     }
   }
   __shared__ float red[NT / 32];
-  n2 = warp_max(n2);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = n2;
+  amax = warp_max(amax);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
   __syncthreads();
-  n2 = red[0];
+  amax = red[0];
 #pragma unroll
-  for (int w = 1; w < NT / 32; ++w) n2 = fmaxf(n2, red[w]);
-  const float f = fp16_tile_factor(sqrtf(n2));
-  if (threadIdx.x == 0) (which ? kfac : qfac)[(size_t)bh * ntiles + tile] = 1.f / f;
+  for (int w = 1; w < NT / 32; ++w) amax = fmaxf(amax, red[w]);
+  const float f = fp16_tile_factor(amax);
+  if (threadIdx.x == 0) {
+    const size_t ti = (size_t)bh * ntiles + tile;
+    if (which) kfac[ti] = 1.f / f;
+    else reinterpret_cast<float4*>(qfac)[ti] = make_float4(1.f / f, 0.f, 0.f, 0.f);
+  }
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
     const int idx = threadIdx.x + u * NT, r = idx / CH, c8 = idx % CH, t = t0 + r;
     if (t >= T) continue;
-    rope_pairs<8, D>(v[u], rc, rs, t - (doc_start ? doc_start[row0 + t] - row0 : 0), c8 * 8, false);
     *reinterpret_cast<uint4*>(dst + ((size_t)bh * T + t) * D + c8 * 8) = pack8_half(v[u], f);
   }
 }
@@ -164,149 +176,113 @@ __device__ __forceinline__ void store8_bf16(__nv_bfloat16* p, const float* v) {
   *reinterpret_cast<uint4*>(p) = raw;
 }
 
-// Backward preprocessing for the tensor-core path, one block per (128-row
-// tile, query head bh). Per row it stores -Delta_i (Delta_i = sum_d dO[i][d]
-// * o[i][d]) and -lse_i * log2(e) in the tile-padded [B*H][Tpad] arrays,
-// negated so the main kernel folds them in with one fused multiply-add (both
-// 0 for rows t >= T, so its per-tile loads never leave the arrays), and
-// zeroes the row of the fp32 dq accumulator (when the grouped-query backward
-// splits its groups, also of the dk, dv accumulators: blocks with bh below
-// B*Hkv take those rows of key/value head bh). Per tile it records the
-// largest |dO_i| (Euclidean norm) and |Delta_i|, which bound dS for the main
-// kernel's fp16 scaling.
-//
-// kRope: the tile's q rows (and, for bh below B*Hkv, the same rows of key/value
-// head bh's k) are rotated and stored as fp16 times the tile's power-of-two
-// factor (fp16_tile_factor of the largest pair norm, found in the first read
-// of the rows), with the inverse factors in qinv (a 16-byte record per tile,
-// value first, so the main kernel can bulk-load it) and kinv: the same values the
-// forward's scores were computed from, so the main kernel recomputes exactly
-// those scores. The rows are read again (from cache) to be rotated.
-constexpr int kBwdPrepThreads = 256;
-
-template <int D, bool kRope>
-__global__ void __launch_bounds__(kBwdPrepThreads) bwd_prep_kernel(
+// Backward row pass for the tensor-core path over the tile-padded
+// [B*H][Tpad] row view, D/8 threads per row (16 bytes of each bf16 row per
+// thread, so a warp covers 32*8/D whole rows of one head): stores -Delta_i
+// (Delta_i = sum_d dO[i][d] * o[i][d]) and -lse_i * log2(e), negated so the
+// main kernel folds them in with one fused multiply-add (both 0 for padding
+// rows t >= T, so its per-tile loads never leave the arrays), and zeroes the
+// fp32 dq accumulator row; when the grouped-query backward splits its groups
+// it also zeroes the fp32 dk, dv accumulator rows (rows of the first B*Hkv
+// heads of the view). dq_acc null: dQ comes from the query-tile pass and no
+// accumulator is used. hstat (fp16 operands, else null; [B*H][4]): per query
+// head the largest |dO_i| (Euclidean norm) and |Delta_i|, per key/value head
+// the largest |v_j| (slots zeroed by rope_prep, filled here by atomic maxima
+// of non-negative floats), which bound dS for the main kernels' fp16 scaling.
+// The grid covers rows_pad * D/8 threads exactly (rows_pad is a multiple of
+// 128), so every warp is full.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(
     const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
     const float* __restrict__ lse, float* __restrict__ delta_pad, float* __restrict__ lse2_pad,
-    float* __restrict__ dq_acc, const __nv_bfloat16* __restrict__ q,
-    const __nv_bfloat16* __restrict__ k, const float* __restrict__ rc,
-    const float* __restrict__ rs, const int32_t* __restrict__ doc_start,
-    __half* __restrict__ q16, __half* __restrict__ k16, float* __restrict__ qinv,
-    float* __restrict__ kinv, float* __restrict__ dmax, float* __restrict__ deltamax,
-    float* __restrict__ dk_acc, float* __restrict__ dv_acc, int B, int H, int Hkv, int T,
-    int Tpad, int ntiles) {
+    float* __restrict__ dq_acc, float* __restrict__ dk_acc, float* __restrict__ dv_acc,
+    const __nv_bfloat16* __restrict__ v, float* __restrict__ hstat, int H, int Hkv, int T,
+    int Tpad, long rows_pad) {
   pdl_wait_and_trigger();
-  constexpr int CPR = D / 8;                    // 16-byte chunks per row
-  constexpr int RPP = kBwdPrepThreads / CPR;    // rows per pass
-  constexpr int NP = 128 / RPP;                 // passes over the tile
-  const int tile = blockIdx.x, bh = blockIdx.y;
-  const int b = bh / H;
-  const bool kv = bh < B * Hkv;  // also a key/value head index
-  const int bk = kv ? bh / Hkv : 0;
-  const int c = threadIdx.x % CPR, rsub = threadIdx.x / CPR;
-  float dmx = 0.f, dlx = 0.f, aq = 0.f, ak = 0.f;
-  for (int u = 0; u < NP; ++u) {
-    const int t = tile * 128 + u * RPP + rsub;
-    const bool valid = t < T;
-    const size_t off = ((size_t)bh * T + (valid ? t : 0)) * D + 8 * c;
-    float s = 0.f, n2 = 0.f;
-    if (valid) {
-      float a[8], g[8];
-      load8_bf16(o + off, a);
-      load8_bf16(dO + off, g);
+  constexpr int TPR = D / 8;  // threads per row
+  const long gt = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long row = gt / TPR;
+  const int c8 = (int)(gt - row * TPR) * 8;
+  const long bh = row / Tpad;
+  const int t = (int)(row - bh * Tpad);
+  float s = 0.f, g2 = 0.f, v2 = 0.f;
+  const bool kv_row = bh < (rows_pad / Tpad) / H * Hkv;  // a row of the [B*Hkv][T] view
+  if (row < rows_pad && t < T) {
+    const long r = bh * T + t;
+    float a[8], g[8];
+    load8_bf16(o + r * D + c8, a);
+    load8_bf16(dO + r * D + c8, g);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        s = fmaf(a[e], g[e], s);
-        n2 = fmaf(g[e], g[e], n2);
-      }
-      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-      reinterpret_cast<float4*>(dq_acc + off)[0] = z;
-      reinterpret_cast<float4*>(dq_acc + off)[1] = z;
-      if (dk_acc && kv) {
-        reinterpret_cast<float4*>(dk_acc + off)[0] = z;
-        reinterpret_cast<float4*>(dk_acc + off)[1] = z;
-        reinterpret_cast<float4*>(dv_acc + off)[0] = z;
-        reinterpret_cast<float4*>(dv_acc + off)[1] = z;
-      }
-      if constexpr (kRope) {  // the tiles' largest pair norms (squared), before rotating
-        float x[8];
-        load8_bf16(q + off, x);
-        aq = fmaxf(aq, pair_norm2_max8(x));
-        if (kv) {
-          load8_bf16(k + off, x);
-          ak = fmaxf(ak, pair_norm2_max8(x));
-        }
-      }
+    for (int e = 0; e < 8; ++e) {
+      s = fmaf(a[e], g[e], s);
+      g2 = fmaf(g[e], g[e], g2);
     }
-    // a row's CPR chunks sit in consecutive lanes of one warp
-#pragma unroll
-    for (int sh = CPR / 2; sh > 0; sh >>= 1) {
-      s += __shfl_xor_sync(0xffffffffu, s, sh);
-      n2 += __shfl_xor_sync(0xffffffffu, n2, sh);
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (dq_acc) {
+      reinterpret_cast<float4*>(dq_acc + r * D + c8)[0] = z;
+      reinterpret_cast<float4*>(dq_acc + r * D + c8)[1] = z;
     }
-    if (c == 0) {
-      delta_pad[(size_t)bh * Tpad + t] = valid ? -s : 0.f;
-      lse2_pad[(size_t)bh * Tpad + t] = valid ? -lse[(size_t)bh * T + t] * 1.4426950408889634f : 0.f;
-    }
-    if (valid) {
-      dmx = fmaxf(dmx, sqrtf(n2));
-      dlx = fmaxf(dlx, fabsf(s));
-    }
-  }
-  __shared__ float red[4][kBwdPrepThreads / 32];
-  dmx = warp_max(dmx);
-  dlx = warp_max(dlx);
-  aq = warp_max(aq);
-  ak = warp_max(ak);
-  const int w = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) {
-    red[0][w] = dmx;
-    red[1][w] = dlx;
-    red[2][w] = aq;
-    red[3][w] = ak;
-  }
-  __syncthreads();
-  float m[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    m[j] = red[j][0];
-#pragma unroll
-    for (int i = 1; i < kBwdPrepThreads / 32; ++i) m[j] = fmaxf(m[j], red[j][i]);
-  }
-  const float fq = fp16_tile_factor(sqrtf(m[2])), fk = fp16_tile_factor(sqrtf(m[3]));
-  if (threadIdx.x == 0) {
-    dmax[(size_t)bh * ntiles + tile] = m[0];
-    deltamax[(size_t)bh * ntiles + tile] = m[1];
-    if (kRope) {
-      reinterpret_cast<float4*>(qinv)[(size_t)bh * ntiles + tile] = make_float4(1.f / fq, 0.f, 0.f, 0.f);
-      if (kv) kinv[(size_t)bh * ntiles + tile] = 1.f / fk;
-    }
-  }
-  if constexpr (kRope) {
-    for (int u = 0; u < NP; ++u) {
-      const int t = tile * 128 + u * RPP + rsub;
-      if (t >= T) continue;
-      const size_t off = ((size_t)bh * T + t) * D + 8 * c;
+    if (hstat && kv_row) {
       float x[8];
-      load8_bf16(q + off, x);
-      rope_pairs<8, D>(x, rc, rs, t - (doc_start ? doc_start[b * T + t] - b * T : 0), 8 * c, false);
-      *reinterpret_cast<uint4*>(q16 + off) = pack8_half(x, fq);
-      if (kv) {
-        load8_bf16(k + off, x);
-        rope_pairs<8, D>(x, rc, rs, t - (doc_start ? doc_start[bk * T + t] - bk * T : 0), 8 * c,
-                         false);
-        *reinterpret_cast<uint4*>(k16 + off) = pack8_half(x, fk);
-      }
+      load8_bf16(v + r * D + c8, x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v2 = fmaf(x[e], x[e], v2);
+    }
+    if (dk_acc && kv_row) {
+      reinterpret_cast<float4*>(dk_acc + r * D + c8)[0] = z;
+      reinterpret_cast<float4*>(dk_acc + r * D + c8)[1] = z;
+      reinterpret_cast<float4*>(dv_acc + r * D + c8)[0] = z;
+      reinterpret_cast<float4*>(dv_acc + r * D + c8)[1] = z;
+    }
+  }
+#pragma unroll
+  for (int off = TPR / 2; off > 0; off >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, off);
+    g2 += __shfl_xor_sync(0xffffffffu, g2, off);
+    v2 += __shfl_xor_sync(0xffffffffu, v2, off);
+  }
+  if (c8 == 0 && row < rows_pad) {
+    delta_pad[row] = -s;
+    lse2_pad[row] = t < T ? -lse[bh * T + t] * 1.4426950408889634f : 0.f;
+  }
+  if (hstat) {
+    // The block's rows share one head (a block covers 256 * 8 / D rows and
+    // Tpad is a multiple of 128); padding rows contribute zeros. One atomic
+    // maximum per block and quantity: many same-address atomics from every
+    // warp would serialise in L2.
+    __shared__ float red[3][8];
+    const float dn = warp_max(sqrtf(g2)), dl = warp_max(fabsf(s)), vn = warp_max(sqrtf(v2));
+    const int w = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+      red[0][w] = dn;
+      red[1][w] = dl;
+      red[2][w] = vn;
+    }
+    __syncthreads();
+    if (threadIdx.x < 3) {
+      float m = red[threadIdx.x][0];
+#pragma unroll
+      for (int i = 1; i < 8; ++i) m = fmaxf(m, red[threadIdx.x][i]);
+      const long row_b = (long)blockIdx.x * (256 / TPR);  // the block's first row
+      const long bh_b = row_b / Tpad;
+      const bool kv_b = bh_b < (rows_pad / Tpad) / H * Hkv;
+      if (row_b < rows_pad && (threadIdx.x < 2 || kv_b))
+        atomicMax(reinterpret_cast<int*>(hstat) + 4 * bh_b + threadIdx.x, __float_as_int(m));
     }
   }
 }
 
 // dq = R(pos)^T (scale * dq_acc), stored as bf16; one thread per 8 values.
+// With fp16 operands (qinv non-null) the accumulator holds Cg qinv_i dS K for
+// query tile i (Cg per key/value head, in the fourth statistics slot of its
+// index), which is divided out here. The same pass finishes split dk, dv
+// accumulators (H the key/value heads, qinv null).
 template <int D>
 __global__ void __launch_bounds__(256) dq_finalize_kernel(
     const float* __restrict__ dq_acc, const float* __restrict__ rc, const float* __restrict__ rs,
     const int32_t* __restrict__ doc_start, __nv_bfloat16* __restrict__ dq, int H, int T,
-    float scale, long n8) {
+    float scale, long n8, const float* __restrict__ qinv, const float* __restrict__ hstat,
+    int Hkv, int ntiles) {
   pdl_wait_and_trigger();
   const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= n8) return;
@@ -314,12 +290,18 @@ __global__ void __launch_bounds__(256) dq_finalize_kernel(
   const long row = e0 / D;  // bh*T + t
   const int d0 = (int)(e0 - row * D);
   const int t = (int)(row % T);
-  const int b = (int)((row / T) / H);
+  const int bh = (int)(row / T);
+  const int b = bh / H;
+  float f = scale;
+  if (qinv) {
+    const int bhk = b * Hkv + (bh - b * H) / (H / Hkv);
+    f /= hstat[4 * bhk + 3] * qinv[((size_t)bh * ntiles + (t >> 7)) * 4];
+  }
   float v[8];
   load_vec<4>(dq_acc + e0, v);
   load_vec<4>(dq_acc + e0 + 4, v + 4);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) v[e] *= scale;
+  for (int e = 0; e < 8; ++e) v[e] *= f;
   if (rc) {
     const int pos = t - (doc_start ? doc_start[b * T + t] - b * T : 0);
     rope_pairs<8, D>(v, rc, rs, pos, d0, true);

@@ -301,10 +301,11 @@ int attn_out_proj_bwd(const void* dy, const void* o, const void* w_o, void* d_o,
  * or ATTN_ECUDA.
  *
  * attn_tile_counts: the 128-query x 128-key tile products the tensor-core
- * forward (fwd_tiles) and key-tile backward (bwd_tiles) kernels executed on
- * the current device since the previous read, counted on the device (one
- * atomic add per CTA; the CUDA-core float32 path is not counted); resets both
- * counters. Block skipping makes these close to the tiles that hold at least
+ * forward (fwd_tiles), key-tile backward (bwd_tiles) and query-tile dQ pass
+ * (dq_tiles; zero when dQ is formed in the key-tile kernel) executed on the
+ * current device since the previous read, counted on the device (one atomic
+ * add per CTA; the CUDA-core float32 path is not counted); resets the
+ * counters. Block skipping makes each equal to the tiles that hold at least
  * one allowed (query, key) pair. Synchronises the device. Returns ATTN_OK,
  * ATTN_EINVAL (a null pointer) or ATTN_ECUDA.
  */
@@ -325,7 +326,8 @@ int attn_exp2_selftest(const float* x, float* y, int n, void* stream);
 int attn_debug_withhold(int what);
 
 unsigned long long attn_launch_count(void);
-int attn_tile_counts(unsigned long long* fwd_tiles, unsigned long long* bwd_tiles);
+int attn_tile_counts(unsigned long long* fwd_tiles, unsigned long long* bwd_tiles,
+                     unsigned long long* dq_tiles);
 int attn_profile_enable(int on);
 int attn_profile_kinds(void);
 int attn_profile_read(int kind, const char** name, int* launches, double* total_ms);
