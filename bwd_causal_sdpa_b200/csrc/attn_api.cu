@@ -119,12 +119,13 @@ EncodeTiledFn encode_fn() {
 
 // A [B*H][T][D] 16-bit tensor seen in boxes of 128 rows x 64 columns with the
 // 128-byte swizzle; rows past T read as zeros.
-bool make_tile_map(CUtensorMap* m, const void* base, bool is_f16, int D, int T, int BH) {
+bool make_tile_map(CUtensorMap* m, const void* base, bool is_f16, int D, int T, int BH,
+                   int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, is_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -242,8 +243,8 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
   }
   const bool f16 = rc != nullptr;
   CUtensorMap mq, mk, mv;
-  if (!make_tile_map(&mq, qs, f16, D, T, BH) || !make_tile_map(&mk, ks, f16, D, T, BHkv) ||
-      !make_tile_map(&mv, v, false, D, T, BHkv))
+  if (!make_tile_map(&mq, qs, f16, D, T, BH) || !make_tile_map(&mk, ks, f16, D, T, BHkv, L::kKV) ||
+      !make_tile_map(&mv, v, false, D, T, BHkv, L::kKV))
     return ATTN_ECUDA;
   static bool smem_set[64] = {};
   if (!ensure_smem(fwd100::fwd_kernel<D>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
@@ -256,7 +257,7 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
   prm.n_pairs = n_pairs;
   prm.n_qtiles = nt;
   prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.idesc_s = sm100::idesc_f16(128, 128, !f16, !f16, false, false);
+  prm.idesc_s = sm100::idesc_f16(128, L::kKV, !f16, !f16, false, false);
   prm.q_fac = qf;
   prm.k_fac = kf;
   prm.doc_start = ds;

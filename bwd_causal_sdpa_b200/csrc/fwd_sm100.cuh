@@ -1,32 +1,42 @@
 // fwd_sm100.cuh -- tensor-core (tcgen05) attention forward for bf16 storage.
 //
 // One CTA computes two 128-row query tiles (A = rows [256t, 256t+128), B =
-// the next 128) of one (b, h) slice; both share every K and V tile it loads.
-//   warps 0-15 softmax: warpgroup g takes tile g & 1 and key columns
-//              [64 (g >> 1), +64) of its S; thread t of a warpgroup owns query
-//              row t (= TMEM lane t), so each row is shared by two threads,
-//              which agree on the row's reference max through a small
-//              shared-memory exchange (double-buffered by key-tile parity,
-//              bounded mbarrier) and add their row sums at the end;
-//   warp 16    TMA producer: both Q tiles once, then K and V tiles through a
-//              ring of shared-memory stages;
-//   warp 17    TMEM owner and MMA issuer (one thread).
-// TMEM (512 columns): per tile an S column block (P, bf16, is written back
-// over its first half) and an O accumulator. Per key tile j the MMA thread
-// issues PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the tensor pipe works on one
-// tile while the other tile's softmax runs. S_t(j+1) is issued only after
-// PV_t(j) completed (it overwrites the P that PV_t(j) reads); since a tcgen05
-// commit covers every earlier MMA of the issuing thread, a softmax warp that
-// has seen S_t(j) may rescale O_t without a further wait.
+// the next 128) of one (b, h) slice; both share every K and V block it loads.
+// Keys advance in blocks of 64, which keeps the scores of a block small
+// enough (64 TMEM columns per tile) that S, P and O of both tiles live in
+// TMEM side by side:
+//   columns [64 t, +64)            S_t   = Q_t K_j^T (fp32)
+//   columns [128 + 64 t + 32 b, +32) P_t, buffer b = j & 1 (bf16 pairs)
+//   columns [256 + 128 t, +D)      O_t   (fp32 accumulator)
+// so S_t(j+1) is computed while the softmax of block j still runs (it only
+// has to wait until that softmax has copied S_t(j) into registers), and the
+// softmax never waits for a PV product except to reuse a P buffer two blocks
+// later. Per query tile the work is one chain of softmax blocks kept fed by
+// the tensor pipe, and the two tiles' chains run side by side.
+//
+// Warp roles (352 threads):
+//   warps 0-7  softmax: warp w serves tile w >> 2, thread = query row
+//              32 (w & 3) + lane (= TMEM lane), all 64 columns of a block;
+//   warp 8     TMA producer: both Q tiles once, then K and V blocks through
+//              rings of shared-memory stages;
+//   warps 9,10 MMA issuers, one per tile (one elected thread each): S_t(0),
+//              then per block j: S_t(j+1) once the softmax released S_t(j),
+//              PV_t(j) once P_t(j) is in TMEM. A K or V stage is released by
+//              a commit (or, for a block the tile does not use, an arrive) of
+//              each issuer, so the ring cannot be overrun by either.
 //
 // Online softmax in log2 units with a lazy rescale: a row's reference max
 // moves (and O, l are rescaled) only when the max grows by more than 8, so P
 // stays <= 2^8 and O is rarely touched; the final O / l and lse = (m +
 // log2 l) ln 2 use the same reference, so the result is exact up to rounding.
+// A fixed share of the exponentials (kPolyPairs pairs of every 32) runs as a
+// polynomial on the FMA pipe, the rest on MUFU, so that neither unit alone
+// sets the pace of the softmax.
 //
-// Masking is per element only on tiles that cross the diagonal or the start
-// of a row's document; key tiles wholly before the first row's document are
-// never loaded (block skipping), nor are tiles past the diagonal.
+// Masking is per element only on blocks that cross the diagonal or the start
+// of a row's document; key blocks wholly before the document of a tile's
+// first row are never loaded (block skipping, per query tile), nor are
+// blocks past the diagonal or past the sequence end.
 //
 // Sources (page, section): ARK README, "Accelerated forward pass (GPU)" (SDPA
 // with the causal mask fused in) and aten.metal entry (scores, softmax,
@@ -37,53 +47,60 @@
 
 #include "sm100.cuh"
 
+#ifndef ATTN_FWD_POLY_PAIRS
+#define ATTN_FWD_POLY_PAIRS 8
+#endif
+
 namespace fwd100 {
 
 using namespace sm100;
 
 template <int D>
 struct Layout {
-  static constexpr int kTileBytes = 128 * D * 2;  // 128 rows x D 16-bit values
-  static constexpr int kBlockBytes = 128 * 128;   // one 64-column block: 128 rows x 128 B
-  static constexpr int kStages = (D == 128) ? 2 : 4;
-  static constexpr int kQ = 0;                    // Q_A, Q_B
-  static constexpr int kK = kQ + 2 * kTileBytes;
-  static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kBars = kV + kStages * kTileBytes;
+  static constexpr int kQTileBytes = 128 * D * 2;  // 128 rows x D 16-bit values
+  static constexpr int kQBlockBytes = 128 * 128;   // one 64-column block of a Q tile
+  static constexpr int kKV = 64;                   // keys per block
+  static constexpr int kKVBytes = kKV * D * 2;     // one K or V block
+  static constexpr int kKVBlockBytes = kKV * 128;  // one 64-column block of it
+  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kQ = 0;  // Q_A, Q_B
+  static constexpr int kK = kQ + 2 * kQTileBytes;
+  static constexpr int kV = kK + kStages * kKVBytes;
+  static constexpr int kBars = kV + kStages * kKVBytes;
   // barrier indices
   static constexpr int bQFull = 0;
   static constexpr int bKFull = 1;
   static constexpr int bKEmpty = bKFull + kStages;
   static constexpr int bVFull = bKEmpty + kStages;
   static constexpr int bVEmpty = bVFull + kStages;
-  static constexpr int bSFull = bVEmpty + kStages;  // [tile]
-  static constexpr int bPFull = bSFull + 2;         // [tile], 128 arrivals
-  static constexpr int bPVDone = bPFull + 2;        // [tile]
-  static constexpr int bOFinal = bPVDone + 2;       // [tile]
-  static constexpr int bXch = bOFinal + 2;          // [tile], 256 arrivals: row maxima exchanged
-  static constexpr int kNumBars = bXch + 2;
-  // row-max exchange between the two halves of a row: f32 [2 parities][2 tiles][2 halves][128]
-  static constexpr int kXch = kBars + kNumBars * 8;
-  static constexpr int kMisc = (kXch + 2 * 2 * 2 * 128 * 4 + 15) / 16 * 16;  // [0] TMEM base, [1] abort flag
+  static constexpr int bSFull = bVEmpty + kStages;  // [tile]: S_t(j) in TMEM
+  static constexpr int bSFree = bSFull + 2;         // [tile], 4 warps: S_t(j) copied out
+  static constexpr int bPFull = bSFree + 2;         // [tile][j & 1], 4 warps: P_t(j) stored
+  static constexpr int bPVDone = bPFull + 4;        // [tile][j & 1]: PV_t(j) complete
+  static constexpr int bOFinal = bPVDone + 4;       // [tile]
+  static constexpr int kNumBars = bOFinal + 2;
+  static constexpr int kMisc = (kBars + kNumBars * 8 + 15) / 16 * 16;  // [0] TMEM base, [1] abort flag
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kSmemAlloc = kBytes;  // the window is 1024-byte aligned (checked)
-  // TMEM columns: tile t uses [256t, 256t+128) for S/P and [256t+128, ...) for O
   static constexpr uint32_t kTmemCols = 512;
-  // softmax warps 0-15 (warpgroup g: tile g & 1, key columns [64 (g >> 1), +64)),
-  // then the TMA producer and the MMA issuer
-  static constexpr int kSoftmaxThreads = 512;
-  static constexpr int kThreads = kSoftmaxThreads + 64;
-  static constexpr int kProducerWarp = 16, kMmaWarp = 17;
+  static constexpr uint32_t kColS = 0, kColP = 128, kColO = 256;
+  static constexpr int kSoftmaxThreads = 256;
+  static constexpr int kThreads = kSoftmaxThreads + 96;
+  static constexpr int kProducerWarp = 8, kMmaWarp0 = 9;
+  static constexpr int kPolyPairs = ATTN_FWD_POLY_PAIRS;  // of the 32 pairs of a block row
+  static_assert(kBytes <= 232448, "shared memory");
+  static_assert(kQTileBytes % 1024 == 0 && kKVBytes % 1024 == 0, "swizzle atoms stay aligned");
+  static_assert(kPolyPairs >= 0 && kPolyPairs <= 32, "poly share");
 };
 
 struct Params {
   int T, H, Hkv, BH, n_pairs, n_qtiles;  // H query heads read Hkv key/value heads
   float scale_log2;          // scale * log2(e)
-  uint32_t idesc_s;          // instruction descriptor of S = Q K^T
+  uint32_t idesc_s;          // instruction descriptor of S = Q K^T (M = 128, N = 64)
   const float* q_fac;        // inverse power-of-two factor per (query head, tile) of the
                              // stored rotated q, one 16-byte record each (value first),
                              // or null (q as given)
-  const float* k_fac;        // the same per (key/value head, tile) for k
+  const float* k_fac;        // the same per (key/value head, 128-key tile) for k, plain floats
   const int32_t* doc_start;  // flattened document starts, or null
   __nv_bfloat16* o;
   float* lse;
@@ -109,46 +126,54 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.T;
   // Flattened grid, tile-major from the last tile pair: the longest rows (most
-  // key tiles) are scheduled first.
+  // key blocks) are scheduled first.
   const int bh = (int)blockIdx.x % p.BH, b = bh / p.H;
   const int bhk = b * p.Hkv + (bh - b * p.H) / (p.H / p.Hkv);  // its key/value head
   const int pr = p.n_pairs - 1 - (int)blockIdx.x / p.BH;
-  const int qtA = 2 * pr, qtB = 2 * pr + 1;
-  const bool hasB = qtB * 128 < T;
+  const int qtA = 2 * pr;
+  const bool hasB = (qtA + 1) * 128 < T;
   const int row0 = b * T;
-  // Key tiles are numbered from kv_t0, the tile holding the start of tile A's
-  // first row's document; tile A takes key tiles [0, nA) of that range, tile
-  // B [jB0, n_kv): from the tile holding its own first row's document start
-  // to its diagonal. Every key tile of a range holds a key some row of the
-  // query tile may see (a query tile's allowed keys form one interval).
-  const int ds0 = p.doc_start ? p.doc_start[row0 + qtA * 128] - row0 : 0;
-  const int kv_t0 = ds0 >> 7;
-  const int nA = qtA - kv_t0 + 1;           // key tiles tile A needs
-  const int n_kv = hasB ? nA + 1 : nA;      // tile B needs one more (its diagonal)
-  const int jB0 = (hasB && p.doc_start) ? ((p.doc_start[row0 + qtB * 128] - row0) >> 7) - kv_t0 : 0;
-  auto t_lo = [&](int t) -> int { return t == 0 ? 0 : jB0; };
-  auto t_hi = [&](int t) -> int { return t == 0 ? nA : (hasB ? n_kv : 0); };
+  const int n64 = (T + 63) >> 6;
+  // Key blocks of tile t: [lo(t), hi(t)), from the block holding the start of
+  // the document of the tile's first row to the block holding its last row's
+  // key (its diagonal), clipped to the sequence. Every block of the range
+  // holds a key some row of the tile may see (a query tile's allowed keys
+  // form one interval). The producer loads the union [lo(0), hi_u).
+  auto first_block = [&](int qt) -> int {
+    return p.doc_start ? ((p.doc_start[row0 + qt * 128] - row0) >> 6) : 0;
+  };
+  const int lo0 = first_block(qtA);
+  const int hi0 = min(2 * qtA + 2, n64);
+  const int lo1 = hasB ? first_block(qtA + 1) : hi0;
+  const int hi1 = hasB ? min(2 * qtA + 4, n64) : hi0;
+  const int hi_u = hasB ? hi1 : hi0;
+  auto lo_of = [&](int t) -> int { return t == 0 ? lo0 : lo1; };
+  auto hi_of = [&](int t) -> int { return t == 0 ? hi0 : hi1; };
 
   if (threadIdx.x == 0) {
+    const uint32_t users = hasB ? 2 : 1;  // issuers that release each K / V stage
     mbar_init(bar(L::bQFull), 1);
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(bar(L::bKFull + s), 1);
-      mbar_init(bar(L::bKEmpty + s), 1);
+      mbar_init(bar(L::bKEmpty + s), users);
       mbar_init(bar(L::bVFull + s), 1);
-      mbar_init(bar(L::bVEmpty + s), 1);
+      mbar_init(bar(L::bVEmpty + s), users);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(L::bSFull + t), 1);
-      mbar_init(bar(L::bPFull + t), 256);
-      mbar_init(bar(L::bXch + t), 256);
-      mbar_init(bar(L::bPVDone + t), 1);
+      mbar_init(bar(L::bSFree + t), 4);
       mbar_init(bar(L::bOFinal + t), 1);
+      for (int e = 0; e < 2; ++e) {
+        mbar_init(bar(L::bPFull + 2 * t + e), 4);
+        mbar_init(bar(L::bPVDone + 2 * t + e), 1);
+      }
     }
     *abort_flag = 0;
     fence_barrier_init();
-    atomicAdd(&g_attn_tiles[0], (unsigned long long)(nA + (hasB ? n_kv - jB0 : 0)));
+    // 64-key blocks x 128 query rows processed (the tile counter's unit)
+    atomicAdd(&g_attn_tiles[0], (unsigned long long)((hi0 - lo0) + (hasB ? hi1 - lo1 : 0)));
   }
-  if (warp == L::kMmaWarp) {
+  if (warp == L::kMmaWarp0) {
     tmem_alloc(sb0 + L::kMisc, L::kTmemCols);
     tmem_relinquish();
   }
@@ -163,144 +188,125 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       prefetch_tensor_map(&tmQ);
       prefetch_tensor_map(&tmK);
       prefetch_tensor_map(&tmV);
-      mbar_arrive_expect_tx(bar(L::bQFull), (hasB ? 2 : 1) * L::kTileBytes);
+      mbar_arrive_expect_tx(bar(L::bQFull), (hasB ? 2 : 1) * L::kQTileBytes);
       for (int t = 0; t < (hasB ? 2 : 1); ++t)
         for (int cb = 0; cb < D / 64; ++cb)
-          tma_load_3d(sb0 + L::kQ + t * L::kTileBytes + cb * L::kBlockBytes, &tmQ,
+          tma_load_3d(sb0 + L::kQ + t * L::kQTileBytes + cb * L::kQBlockBytes, &tmQ,
                       bar(L::bQFull), cb * 64, (qtA + t) * 128, bh);
-      for (int it = 0; it < n_kv; ++it) {
-        const int st = it % L::kStages, round = it / L::kStages;
-        const int kvrow = (kv_t0 + it) * 128;
+      for (int j = lo0; j < hi_u; ++j) {
+        const int it = j - lo0, st = it % L::kStages, round = it / L::kStages;
         if (it >= L::kStages && !mbar_wait(bar(L::bKEmpty + st), (round - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(L::bKFull + st), L::kTileBytes);
+        mbar_arrive_expect_tx(bar(L::bKFull + st), L::kKVBytes);
         for (int cb = 0; cb < D / 64; ++cb)
-          tma_load_3d(sb0 + L::kK + st * L::kTileBytes + cb * L::kBlockBytes, &tmK,
-                      bar(L::bKFull + st), cb * 64, kvrow, bhk);
+          tma_load_3d(sb0 + L::kK + st * L::kKVBytes + cb * L::kKVBlockBytes, &tmK,
+                      bar(L::bKFull + st), cb * 64, j * 64, bhk);
 #ifdef ATTN_DEBUG_HOOKS
-        if (it == 0 && g_attn_withhold == 1) continue;  // V(0) never arrives
+        if (it == 0 && g_attn_withhold == 1) continue;  // V(first block) never arrives
 #endif
         if (it >= L::kStages && !mbar_wait(bar(L::bVEmpty + st), (round - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(L::bVFull + st), L::kTileBytes);
+        mbar_arrive_expect_tx(bar(L::bVFull + st), L::kKVBytes);
         for (int cb = 0; cb < D / 64; ++cb)
-          tma_load_3d(sb0 + L::kV + st * L::kTileBytes + cb * L::kBlockBytes, &tmV,
-                      bar(L::bVFull + st), cb * 64, kvrow, bhk);
+          tma_load_3d(sb0 + L::kV + st * L::kKVBytes + cb * L::kKVBlockBytes, &tmV,
+                      bar(L::bVFull + st), cb * 64, j * 64, bhk);
       }
     }
-  } else if (warp == L::kMmaWarp) {
-    // ---------------- MMA issuer ----------------
-    // Issue order: S of each tile whose range starts at key tile 0, then per
-    // key tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), each only where tile
-    // t's range holds j (a tile whose range starts at j+1 gets its first S
-    // there). Each tile's S(j+1) follows its own PV(j) (it overwrites the P
-    // that PV(j) reads, so it waits for PV(j) to finish), and never waits for
-    // the other tile's softmax: the two chains S -> softmax -> PV run
-    // independently and fill each other's gaps. Barrier phases of tile t count
-    // its own key tiles (j - t_lo(t)).
-    if (lane == 0) {
+  } else if (warp == L::kMmaWarp0 || warp == L::kMmaWarp0 + 1) {
+    // ---------------- MMA issuers (one per tile) ----------------
+    const int t = warp - L::kMmaWarp0;
+    if (lane == 0 && (t == 0 || hasB)) {
       constexpr uint32_t idesc_o = idesc_f16(128, D, true, true, false, true);
-      const int t1 = hasB ? 2 : 1;
-      auto active = [&](int t, int j) -> bool { return t < t1 && j >= t_lo(t) && j < t_hi(t); };
-      auto issue_S = [&](int t, int j) {
-        const uint32_t kbase = sb0 + L::kK + (j % L::kStages) * L::kTileBytes;
-        const uint32_t qbase = sb0 + L::kQ + t * L::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
-          mma_ss(tmem + 256 * t, smem_desc_sw128(qbase + off, 16, 1024),
-                 smem_desc_sw128(kbase + off, 16, 1024), p.idesc_s, kk > 0);
-        }
-        mma_commit(bar(L::bSFull + t));
+      const int lo = lo_of(t), hi = hi_of(t), n = hi - lo;
+      const uint32_t tS = tmem + L::kColS + 64 * t;
+      const uint32_t tO = tmem + L::kColO + 128 * t;
+      const uint32_t qbase = sb0 + L::kQ + t * L::kQTileBytes;
+      auto stage = [&](int j) -> int { return (j - lo0) % L::kStages; };
+      auto phase = [&](int j) -> uint32_t { return (uint32_t)((j - lo0) / L::kStages) & 1u; };
+      // release a block this tile does not use (after it arrived, so that
+      // the arrival counts toward that block's use of the stage)
+      auto pass = [&](int j) -> bool {
+        if (!mbar_wait(bar(L::bKFull + stage(j)), phase(j), abort_flag)) return false;
+        mbar_arrive(bar(L::bKEmpty + stage(j)));
+        if (!mbar_wait(bar(L::bVFull + stage(j)), phase(j), abort_flag)) return false;
+        mbar_arrive(bar(L::bVEmpty + stage(j)));
+        return true;
       };
-      bool ok = mbar_wait(bar(L::bQFull), 0, abort_flag) && mbar_wait(bar(L::bKFull), 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        for (int t = 0; t < t1; ++t)
-          if (active(t, 0)) issue_S(t, 0);
-        mma_commit(bar(L::bKEmpty));
-      }
-      for (int it = 0; ok && it < n_kv; ++it) {
-        const int st = it % L::kStages, nst = (it + 1) % L::kStages;
-        if (!mbar_wait(bar(L::bVFull + st), (it / L::kStages) & 1, abort_flag)) break;
-        const uint32_t vbase = sb0 + L::kV + st * L::kTileBytes;
-        bool issued_next = false;
-        for (int t = 0; ok && t < t1; ++t) {
-          if (!active(t, it)) {
-            if (active(t, it + 1)) {  // tile t's range starts at it + 1
-              if (!mbar_wait(bar(L::bKFull + nst), ((it + 1) / L::kStages) & 1, abort_flag)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              issue_S(t, it + 1);
-              issued_next = true;
-            }
-            continue;
-          }
-          const int li = it - t_lo(t);  // this tile's own key-tile count
-          if (!mbar_wait(bar(L::bPFull + t), li & 1, abort_flag)) { ok = false; break; }
+      bool ok = true;
+      for (int j = lo0; ok && j < lo; ++j) ok = pass(j);
+      if (ok) ok = mbar_wait(bar(L::bQFull), 0, abort_flag);
+      for (int li = 0; ok && li <= n; ++li) {
+        if (li < n) {  // S_t(li) = Q_t K_j^T
+          const int j = lo + li;
+          if (!mbar_wait(bar(L::bKFull + stage(j)), phase(j), abort_flag)) { ok = false; break; }
+          if (li > 0 && !mbar_wait(bar(L::bSFree + t), (li - 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t aP = tmem + 256 * t;
+          const uint32_t kbase = sb0 + L::kK + stage(j) * L::kKVBytes;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + 256 * t + 128, aP + kk * 8,
-                   smem_desc_sw128(vbase + kk * 2048, L::kBlockBytes, 1024), idesc_o,
-                   (li > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(bar(L::bPVDone + t));
-          if (active(t, it + 1)) {
-            if (!mbar_wait(bar(L::bKFull + nst), ((it + 1) / L::kStages) & 1, abort_flag) ||
-                !mbar_wait(bar(L::bPVDone + t), li & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            issue_S(t, it + 1);
-            issued_next = true;
-          }
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tS,
+                   smem_desc_sw128(qbase + (kk >> 2) * L::kQBlockBytes + (kk & 3) * 32, 16, 1024),
+                   smem_desc_sw128(kbase + (kk >> 2) * L::kKVBlockBytes + (kk & 3) * 32, 16, 1024),
+                   p.idesc_s, kk > 0);
+          mma_commit(bar(L::bSFull + t));
+          mma_commit(bar(L::bKEmpty + stage(j)));
         }
-        if (!ok) break;
-        mma_commit(bar(L::bVEmpty + st));
-        if (issued_next) mma_commit(bar(L::bKEmpty + nst));
+        if (li > 0) {  // O_t += P_t(lj) V_j
+          const int lj = li - 1, j = lo + lj;
+          if (!mbar_wait(bar(L::bVFull + stage(j)), phase(j), abort_flag) ||
+              !mbar_wait(bar(L::bPFull + 2 * t + (lj & 1)), (lj >> 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t vbase = sb0 + L::kV + stage(j) * L::kKVBytes;
+          const uint32_t aP = tmem + L::kColP + 64 * t + 32 * (lj & 1);
+#pragma unroll
+          for (int kk = 0; kk < L::kKV / 16; ++kk)
+            mma_ts(tO, aP + kk * 8, smem_desc_sw128(vbase + kk * 2048, L::kKVBlockBytes, 1024),
+                   idesc_o, (lj > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(L::bPVDone + 2 * t + (lj & 1)));
+          mma_commit(bar(L::bVEmpty + stage(j)));
+        }
       }
-      if (ok) {
-        mma_commit(bar(L::bOFinal + 0));
-        mma_commit(bar(L::bOFinal + 1));
-      }
+      if (ok) mma_commit(bar(L::bOFinal + t));
+      for (int j = hi; ok && j < hi_u; ++j) ok = pass(j);
     }
   } else {
-    // ---------------- softmax warpgroups ----------------
-    const int t = (warp >> 2) & 1;   // tile
-    const int hf = warp >> 3;        // key columns [64 hf, 64 hf + 64) of the tile's S
+    // ---------------- softmax warps ----------------
+    const int t = warp >> 2;
     const int r = (warp & 3) * 32 + lane;  // row within the tile = TMEM lane
     const int qt = qtA + t;
     const int i = qt * 128 + r;
     const bool active = (t == 0) || hasB;
-    const int n_t = t_hi(t) - t_lo(t);  // key tiles this tile processes
-    const int kt_first = kv_t0 + t_lo(t);
+    const int lo = lo_of(t), n = hi_of(t) - lo;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base + 256 * t;
-    const uint32_t tO = tS + 128;
-    float* xch = reinterpret_cast<float*>(sg + L::kXch);  // [parity][tile][half][row]
+    const uint32_t tS = tmem + lane_base + L::kColS + 64 * t;
+    const uint32_t tP = tmem + lane_base + L::kColP + 64 * t;
+    const uint32_t tO = tmem + lane_base + L::kColO + 128 * t;
     const int ds_i = p.doc_start ? p.doc_start[row0 + min(i, T - 1)] - row0 : 0;
     const float fq = p.q_fac ? p.q_fac[((size_t)bh * p.n_qtiles + min(qt, p.n_qtiles - 1)) * 4] : 1.f;
     float m = -INFINITY, l = 0.f;
     bool ok = active;
-    for (int it = 0; ok && it < n_t; ++it) {
-      const int kt = kt_first + it, j0 = kt * 128 + 64 * hf;  // first key of this half
-      if (!mbar_wait(bar(L::bSFull + t), it & 1, abort_flag)) { ok = false; break; }
+    for (int li = 0; ok && li < n; ++li) {
+      const int j = lo + li, j0 = j * 64;  // first key of the block
+      if (!mbar_wait(bar(L::bSFull + t), li & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      // scale of this key tile's scores (q, k tiles may carry power-of-two
+      uint32_t s[64];
+      tmem_ld32(tS, s);
+      tmem_ld32(tS + 32, s + 32);
+      tmem_wait_ld();
+      // S_t(li) is in registers: the issuer may compute S_t(li+1) over it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::bSFree + t));
+      // scale of this block's scores (q, k tiles may carry power-of-two
       // factors). A zero scale (uniform attention) is evaluated with the
       // smallest normal scale instead: a score below 2^100 in magnitude then
       // scales to below 2^-26, so each kept probability rounds to exactly 1
       // as it should, while a masked score still becomes -inf rather than
       // inf * 0 = NaN.
-      float sc = p.scale_log2 * fq * (p.k_fac ? p.k_fac[bhk * p.n_qtiles + kt] : 1.f);
+      float sc = p.scale_log2 * fq * (p.k_fac ? p.k_fac[bhk * p.n_qtiles + (j >> 1)] : 1.f);
       if (sc == 0.f) sc = 1.17549435e-38f;
       const bool pos_scale = sc > 0.f;
-      uint32_t s[64];
-      tmem_ld32(tS + 64 * hf, s);
-      tmem_ld32(tS + 64 * hf + 32, s + 32);
-      tmem_wait_ld();
       const bool need_mask = (j0 + 63 > i) || (j0 < ds_i);
       const float masked = pos_scale ? -INFINITY : INFINITY;
       if (need_mask) {
@@ -308,7 +314,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         for (int c = 0; c < 64; ++c)
           if (j0 + c > i || j0 + c < ds_i) s[c] = __float_as_uint(masked);
       }
-      // extreme of this half's raw scores (max for a positive scale)
+      // extreme of the raw scores (max for a positive scale)
       float e4[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) e4[q] = __uint_as_float(s[q]);
@@ -324,84 +330,77 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
           e4[(c >> 1) & 3] = min3f(e4[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
         ext = min3f(fminf(e4[0], e4[1]), e4[2], e4[3]);
       }
-      // the row max of the scaled scores: this half's and the other half's
-      // (-inf for a half that is all masked, so both halves see the same value)
-      float* xs = xch + ((it & 1) * 4 + t * 2) * 128;
-      xs[hf * 128 + r] = ext * sc;
-      mbar_arrive(bar(L::bXch + t));
-      if (!mbar_wait(bar(L::bXch + t), it & 1, abort_flag)) { ok = false; break; }
-      const float mx = fmaxf(xs[r], xs[128 + r]);
+      const float mx = ext * sc;  // -inf for a block the row may not see at all
       // Move the reference max only when it grows by more than 8 (log2
-      // units); the first key a row sees always moves it (m = -inf). Both
-      // halves compute the same m from the same inputs.
+      // units); the first key a row sees always moves it (m = -inf).
       const bool move = mx > m + 8.f;
       const float alpha = move ? ex2(m - mx) : 1.f;
-      // O needs rescaling only if it already holds a non-zero partial sum;
-      // PV_t(it-1) is complete (it precedes S_t(it) in the commit order).
-      const bool scale_o = move && m != -INFINITY && it > 0;
+      // O needs rescaling only if it already holds a non-zero partial sum
+      const bool scale_o = move && m != -INFINITY && li > 0;
       if (move) {
         l *= alpha;
         m = mx;
       }
       const float mref = (m == -INFINITY) ? 0.f : m;
-      // p = 2^(s * sc - m) two at a time; P (bf16) goes over the first half
-      // of the S columns: this half's keys at columns [32 hf, 32 hf + 32),
-      // which both halves have read by now (they passed the exchange)
+      // p = 2^(s * sc - m) two at a time, kPolyPairs of the 32 pairs on the
+      // FMA pipe, the others on MUFU
       const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-mref, -mref);
       float2 l2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                       make_float2(0.f, 0.f)};
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float2 sv = make_float2(__uint_as_float(s[32 * c + 2 * e]),
-                                        __uint_as_float(s[32 * c + 2 * e + 1]));
-          const float2 x = __ffma2_rn(sv, sc2, nm2);
-          const float2 pv = make_float2(ex2(x.x), ex2(x.y));
-          l2[e & 3] = __fadd2_rn(l2[e & 3], pv);
-          pk[e] = pack_bf16(pv.x, pv.y);
-        }
-        tmem_st16(tS + 32 * hf + 16 * c, pk);
+      for (int e = 0; e < 32; ++e) {
+        const float2 sv = make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1]));
+        const float2 x = __ffma2_rn(sv, sc2, nm2);
+        // pair e is a polynomial one when the running count e * share / 32
+        // steps up at e (spreads kPolyPairs pairs evenly over the 32)
+        const bool poly = (e * L::kPolyPairs) / 32 != ((e + 1) * L::kPolyPairs) / 32;
+        const float2 pv = poly ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
+        l2[e & 3] = __fadd2_rn(l2[e & 3], pv);
+        pk[e] = pack_bf16(pv.x, pv.y);
       }
       const float2 la = __fadd2_rn(l2[0], l2[1]), lb = __fadd2_rn(l2[2], l2[3]);
       l += (la.x + la.y) + (lb.x + lb.y);
-      // rescale this half's O columns (warp-collective: each lane by its own
-      // factor, 1 for lanes that kept their max) before PV_t(it) runs
+      // P_t(li) goes to buffer li & 1, last read by PV_t(li - 2)
+      if (li >= 2 &&
+          !mbar_wait(bar(L::bPVDone + 2 * t + (li & 1)), ((li - 2) >> 1) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      // rescale O (warp-collective: each lane by its own factor, 1 for lanes
+      // that kept their max) once PV_t(li - 1), the last product into O, is done
       if (__any_sync(0xffffffffu, scale_o)) {
+        if (!mbar_wait(bar(L::bPVDone + 2 * t + ((li - 1) & 1)), ((li - 1) >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         const float f = scale_o ? alpha : 1.f;
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           uint32_t ov[32];
-          tmem_ld32(tO + (D / 2) * hf + 32 * c, ov);
+          tmem_ld32(tO + 32 * c, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-          tmem_st32(tO + (D / 2) * hf + 32 * c, ov);
+          tmem_st32(tO + 32 * c, ov);
         }
       }
+      tc_fence_after();
+      tmem_st32(tP + 32 * (li & 1), pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(L::bPFull + t));
-    }
-    // row sum: this half's plus the other half's (through the exchange area,
-    // parity n_t; both halves ran the same number of key tiles)
-    float lt = l;
-    if (ok) {
-      float* xs = xch + ((n_t & 1) * 4 + t * 2) * 128;
-      xs[hf * 128 + r] = l;
-      mbar_arrive(bar(L::bXch + t));
-      if (!mbar_wait(bar(L::bXch + t), n_t & 1, abort_flag)) ok = false;
-      else lt = xs[r] + xs[128 + r];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::bPFull + 2 * t + (li & 1)));
     }
     if (ok && mbar_wait(bar(L::bOFinal + t), 0, abort_flag)) {
       tc_fence_after();
-      const float inv = 1.f / lt;
-      __nv_bfloat16* orow = p.o + ((size_t)bh * T + min(i, T - 1)) * D + (D / 2) * hf;
+      const float inv = 1.f / l;
+      __nv_bfloat16* orow = p.o + ((size_t)bh * T + min(i, T - 1)) * D;
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
-        tmem_ld32(tO + (D / 2) * hf + 32 * c, ov);  // warp-collective
+        tmem_ld32(tO + 32 * c, ov);  // warp-collective
         tmem_wait_ld();
         if (i < T) {
           uint32_t pk[16];
@@ -414,13 +413,13 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
             dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
       }
-      if (i < T && hf == 0) p.lse[(size_t)bh * T + i] = (m + __log2f(lt)) * 0.69314718055994531f;
+      if (i < T) p.lse[(size_t)bh * T + i] = (m + __log2f(l)) * 0.69314718055994531f;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == L::kMmaWarp) {
+  if (warp == L::kMmaWarp0) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }

@@ -300,14 +300,15 @@ int attn_out_proj_bwd(const void* dy, const void* o, const void* w_o, void* d_o,
  * Returns ATTN_OK, ATTN_EINVAL (kind out of range or a null output pointer)
  * or ATTN_ECUDA.
  *
- * attn_tile_counts: the 128-query x 128-key tile products the tensor-core
- * forward (fwd_tiles), key-tile backward (bwd_tiles) and query-tile dQ pass
- * (dq_tiles; zero when dQ is formed in the key-tile kernel) executed on the
- * current device since the previous read, counted on the device (one atomic
- * add per CTA; the CUDA-core float32 path is not counted); resets the
- * counters. Block skipping makes each equal to the tiles that hold at least
- * one allowed (query, key) pair. Synchronises the device. Returns ATTN_OK,
- * ATTN_EINVAL (a null pointer) or ATTN_ECUDA.
+ * attn_tile_counts: the block products the tensor-core forward (fwd_tiles:
+ * 128 queries x 64 keys each), key-tile backward (bwd_tiles: 128 x 128) and
+ * query-tile dQ pass (dq_tiles: 128 x 128; zero when dQ is formed in the
+ * key-tile kernel) executed on the current device since the previous read,
+ * counted on the device (one atomic add per CTA; the CUDA-core float32 path
+ * is not counted); resets the counters. Block skipping makes each equal to
+ * the blocks of its size that hold at least one allowed (query, key) pair.
+ * Synchronises the device. Returns ATTN_OK, ATTN_EINVAL (a null pointer) or
+ * ATTN_ECUDA.
  */
 /* attn_exp2_selftest: y[i] = the forward/backward kernels' software 2^x
  * (FMA-pipe polynomial) of x[i], for 0 <= i < n; x, y device f32 arrays,
