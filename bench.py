@@ -3,9 +3,11 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-A step is one attn_fwd + one attn_bwd over the whole workload (default: the
+A step is one forward + one backward over the whole workload (default: the
 long-context window B=1, H=16, T=8192, D=128 with RoPE), inputs resident in
-HBM. Each timed step is bracketed by CUDA events on the launching stream; L2
+HBM: attn_fwd_save + attn_bwd_saved, the forward's rotated q, k kept for the
+backward as a training step keeps its activations (--no-save: the plain
+attn_fwd + attn_bwd, which rotate q, k in both calls). Each timed step is bracketed by CUDA events on the launching stream; L2
 is flushed (a 256 MiB write) between steps, outside the events. FLOPs follow
 the nominal convention 4*B*H*T^2*D/2 forward and 2.5x that backward
 (7*B*H*T^2*D per step; for packed documents the within-document figure is
@@ -84,6 +86,8 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-save", action="store_true",
+                    help="plain attn_fwd / attn_bwd (the backward rotates q, k again)")
     ap.add_argument("--sustain", type=float, default=0.0,
                     help="also time back-to-back steps for about this many seconds and report "
                          "them against the sustained bf16 peak (clocks and power sampled)")
@@ -401,7 +405,7 @@ def run_ours(args):
     cfg = config_by_name(args.workload)
     w = make_workload(cfg, H_kv=args.kv_heads)
     stream = torch.cuda.Stream(dev)
-    r = AttnRunner.from_workload(w, device=dev, stream=stream)
+    r = AttnRunner.from_workload(w, device=dev, stream=stream, save=not args.no_save)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     peaks, peak_src = load_peaks()
     flops_step = 7.0 * w.B * w.H * w.T * w.T * w.D
@@ -511,7 +515,7 @@ def run_ours(args):
     # beside it.
     e2e = None
     if not args.no_e2e:
-        r2 = AttnRunner.from_workload(w, device=dev, stream=stream)
+        r2 = AttnRunner.from_workload(w, device=dev, stream=stream, save=not args.no_save)
         sets = [r, r2]
         host_in = [x.detach().to("cpu").pin_memory() for x in (r.q, r.k, r.v, r.do)]
         host_out = [[torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
@@ -637,7 +641,9 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic (seeded)",
-            "config": workload_config(w, l2="flushed between steps (256 MiB write outside the step events)"),
+            "config": dict(workload_config(w, l2="flushed between steps (256 MiB write outside the step events)"),
+                           calls=("attn_fwd_gqa + attn_bwd_gqa" if args.no_save or r.saved is None
+                                  else "attn_fwd_save + attn_bwd_saved (rotated q, k kept between them)")),
             "pct_of_bf16_peak": value / world / peaks["bf16_tflops"],
             "pct_of_bf16_peak_sustained": value / world / peaks["bf16_tflops_sustained"],
             "peaks_source": peak_src,

@@ -42,6 +42,12 @@ _SIGNATURES = {
                           _P, ctypes.c_size_t, _P]),
     "attn_bwd_gqa": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.c_float,
                           _I, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "attn_saved_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I]),
+    "attn_fwd_save": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I,
+                           _P, ctypes.c_size_t, _P, ctypes.c_size_t, _P]),
+    "attn_bwd_saved": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
+                            ctypes.c_float, _I, _P, _P, _P, _P, ctypes.c_size_t, _P,
+                            ctypes.c_size_t, _P]),
     "attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I,
                          _P, ctypes.c_size_t, _P]),
     "attn_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
@@ -151,6 +157,30 @@ def attn_bwd_gqa(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, H_kv
                                  _ptr(rope_cos), _ptr(rope_sin), _ptr(cu_seqlens), B, H, H_kv,
                                  T, D, float(scale), dtype, _ptr(dq), _ptr(dk), _ptr(dv),
                                  _ptr(workspace), int(ws_bytes), _stream(stream)))
+
+
+def attn_saved_bytes(B, H, H_kv, T, D, dtype, has_rope) -> int:
+    """Bytes of the buffer attn_fwd_save keeps the rotated operands in (0: none)."""
+    return int(_lib.attn_saved_bytes(B, H, H_kv, T, D, dtype, int(bool(has_rope))))
+
+
+def attn_fwd_save(q, k, v, rope_cos, rope_sin, cu_seqlens, o, lse, B, H, H_kv, T, D, scale,
+                  dtype, workspace, ws_bytes, saved, saved_bytes, stream=None) -> int:
+    """attn_fwd_gqa that also leaves its rotated q, k in `saved` for attn_bwd_saved."""
+    return int(_lib.attn_fwd_save(_ptr(q), _ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin),
+                                  _ptr(cu_seqlens), _ptr(o), _ptr(lse), B, H, H_kv, T, D,
+                                  float(scale), dtype, _ptr(workspace), int(ws_bytes),
+                                  _ptr(saved), int(saved_bytes), _stream(stream)))
+
+
+def attn_bwd_saved(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, H_kv, T, D, scale,
+                   dtype, dq, dk, dv, workspace, ws_bytes, saved, saved_bytes, stream=None) -> int:
+    """attn_bwd_gqa reading the rotated q, k attn_fwd_save left in `saved`."""
+    return int(_lib.attn_bwd_saved(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse),
+                                   _ptr(rope_cos), _ptr(rope_sin), _ptr(cu_seqlens), B, H, H_kv,
+                                   T, D, float(scale), dtype, _ptr(dq), _ptr(dk), _ptr(dv),
+                                   _ptr(workspace), int(ws_bytes), _ptr(saved), int(saved_bytes),
+                                   _stream(stream)))
 
 
 def attn_decode(q, k_cache, v_cache, cache_lens, rope_cos, rope_sin, o, lse, B, H, H_kv, T_max,

@@ -96,6 +96,25 @@ WsPlan plan(int B, int H, int T, int D, int dtype, int is_bwd, int Hkv = 0) {
   return p;
 }
 
+// The forward's rotated operands kept for the backward (attn_fwd_save /
+// attn_bwd_saved): rotated q, k as fp16 and their inverse tile factors, in the
+// layout rope_prep writes them.
+struct SavedPlan {
+  size_t q16 = 0, k16 = 0, qfac = 0, kfac = 0, total = 0;
+};
+
+SavedPlan saved_plan(int B, int H, int Hkv, int T, int D) {
+  SavedPlan p;
+  const size_t nt = (size_t)((T + 127) / 128);
+  size_t off = 0;
+  p.q16 = off;  off += round_up((size_t)B * H * T * D * 2);
+  p.k16 = off;  off += round_up((size_t)B * Hkv * T * D * 2);
+  p.qfac = off; off += round_up((size_t)B * H * nt * 4 * sizeof(float));
+  p.kfac = off; off += round_up((size_t)B * Hkv * nt * sizeof(float));
+  p.total = off;
+  return p;
+}
+
 // ---- TMA descriptors (driver entry point fetched through the runtime) ----
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -221,7 +240,7 @@ int bwd_simt(const void* q, const void* k, const void* v, const void* o, const v
 template <int D>
 int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const float* rs,
            const int32_t* ds, void* o, float* lse, int B, int H, int Hkv, int T, float scale,
-           char* ws, const WsPlan& wp, cudaStream_t st) {
+           char* ws, const WsPlan& wp, char* saved, cudaStream_t st) {
   using L = fwd100::Layout<D>;
   const int nt = (T + 127) / 128, BH = B * H, BHkv = B * Hkv;
   // With RoPE q and k are rotated once into fp16 tiles with power-of-two
@@ -230,10 +249,12 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
   const void* ks = k;
   float *qf = nullptr, *kf = nullptr;
   if (rc) {
-    __half* qh = (__half*)(ws + wp.q16);
-    __half* kh = (__half*)(ws + wp.k16);
-    qf = (float*)(ws + wp.qfac);
-    kf = (float*)(ws + wp.kfac);
+    // into the caller's saved buffer when it keeps them for the backward
+    const SavedPlan sp = saved_plan(B, H, Hkv, T, D);
+    __half* qh = (__half*)(saved ? saved + sp.q16 : ws + wp.q16);
+    __half* kh = (__half*)(saved ? saved + sp.k16 : ws + wp.k16);
+    qf = (float*)(saved ? saved + sp.qfac : ws + wp.qfac);
+    kf = (float*)(saved ? saved + sp.kfac : ws + wp.kfac);
     ATTN_LAUNCH(KK_ROPE_PREP, st, pdl_launch(rope_prep_kernel<D>, dim3(nt, BH, 2), kRopePrepThreads, 0, st,
                                              (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds,
                                              qh, kh, qf, kf, (float*)nullptr, B, H, Hkv, T, nt));
@@ -316,26 +337,34 @@ template <int D>
 int bwd_tc(const void* q, const void* k, const void* v, const void* o, const void* dO,
            const float* lse, const float* rc, const float* rs, const int32_t* ds,
            const int32_t* de, void* dq, void* dk, void* dv, int B, int H, int Hkv, int T,
-           float scale, char* ws, const WsPlan& wp, cudaStream_t st) {
+           float scale, char* ws, const WsPlan& wp, const char* saved, cudaStream_t st) {
   const int nt = (T + 127) / 128, BH = B * H, BHkv = B * Hkv, Tpad = nt * 128;
   // With RoPE the scores are recomputed from fp16 operands (the rotated q, k
   // with per-tile factors, as the forward computed them); without it from q,
   // k as given (bf16).
   const bool f16 = rc != nullptr;
-  __half* q16 = (__half*)(ws + wp.q16);
-  __half* k16 = (__half*)(ws + wp.k16);
+  // the forward's rotated operands: from the caller's saved buffer when given
+  // (attn_bwd_saved), else made again here
+  const bool reuse = f16 && saved != nullptr;
+  const SavedPlan sp = saved_plan(B, H, Hkv, T, D);
+  __half* q16 = reuse ? (__half*)(saved + sp.q16) : (__half*)(ws + wp.q16);
+  __half* k16 = reuse ? (__half*)(saved + sp.k16) : (__half*)(ws + wp.k16);
   const void* qs = f16 ? (const void*)q16 : q;
   const void* ks = f16 ? (const void*)k16 : k;
   float* delta = (float*)(ws + wp.delta);
   float* lse2 = (float*)(ws + wp.lse2);
   float* dq_acc = (float*)(ws + wp.dq_acc);
-  float* qinv = (float*)(ws + wp.qfac);
-  float* kinv = (float*)(ws + wp.kfac);
+  float* qinv = reuse ? (float*)(saved + sp.qfac) : (float*)(ws + wp.qfac);
+  float* kinv = reuse ? (float*)(saved + sp.kfac) : (float*)(ws + wp.kfac);
   float* hstat = f16 ? (float*)(ws + wp.hstat) : nullptr;
   const int split = wp.split;
   float* dk_acc = split > 1 ? (float*)(ws + wp.dk_acc) : nullptr;
   float* dv_acc = split > 1 ? (float*)(ws + wp.dv_acc) : nullptr;
-  if (f16) {
+  if (reuse) {
+    // the statistics slots the row pass fills with atomic maxima start at 0
+    // (rope_prep zeroes them when it runs)
+    if (cudaMemsetAsync(hstat, 0, (size_t)BH * 4 * sizeof(float), st) != cudaSuccess) return ATTN_ECUDA;
+  } else if (f16) {
     // the forward's rotation, factors included (same kernel, same values)
     ATTN_LAUNCH(KK_ROPE_PREP, st, pdl_launch(rope_prep_kernel<D>, dim3(nt, BH, 2), kRopePrepThreads, 0, st,
                                              (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds,
@@ -443,10 +472,31 @@ size_t attn_workspace_bytes_gqa(int B, int H, int H_kv, int T, int D, int dtype,
   return plan(B, H, T, D, dtype, is_bwd, H_kv).total;
 }
 
-int attn_fwd_gqa(const void* q, const void* k, const void* v, const float* rope_cos,
-                 const float* rope_sin, const int32_t* cu_seqlens, void* o, float* lse, int B,
-                 int H, int H_kv, int T, int D, float scale, int dtype, void* workspace,
-                 size_t ws_bytes, void* stream) {
+size_t attn_saved_bytes(int B, int H, int H_kv, int T, int D, int dtype, int has_rope) {
+  if (!sizes_ok(B, H, T, D) || dtype != ATTN_BF16 || !has_rope) return 0;
+  if (H_kv <= 0 || H % H_kv != 0) return 0;
+  return saved_plan(B, H, H_kv, T, D).total;
+}
+
+}  // extern "C"
+
+namespace {
+
+// A saved buffer is used only where there is something to keep (bf16
+// storage with RoPE); elsewhere it may be null and is ignored.
+int check_saved(const void* saved, size_t saved_bytes, int B, int H, int H_kv, int T, int D,
+                int dtype, const float* rope_cos) {
+  const size_t need = attn_saved_bytes(B, H, H_kv, T, D, dtype, rope_cos != nullptr);
+  if (need == 0 || saved == nullptr) return ATTN_OK;  // nothing kept: the plain call
+  if (!aligned(saved, 16)) return ATTN_EALIGN;
+  if (saved_bytes < need) return ATTN_EWORKSPACE;
+  return ATTN_OK;
+}
+
+int fwd_impl(const void* q, const void* k, const void* v, const float* rope_cos,
+             const float* rope_sin, const int32_t* cu_seqlens, void* o, float* lse, int B, int H,
+             int H_kv, int T, int D, float scale, int dtype, void* workspace, size_t ws_bytes,
+             void* saved, void* stream) {
   int rc = check_common(q, k, v, rope_cos, rope_sin, cu_seqlens, B, H, H_kv, T, D, scale, dtype,
                         workspace, ws_bytes, 0);
   if (rc) return rc;
@@ -468,10 +518,39 @@ int attn_fwd_gqa(const void* q, const void* k, const void* v, const float* rope_
                    : fwd_simt<float, 128>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, H_kv, T,
                                           scale, st);
   }
+  char* sv = (rope_cos && saved) ? (char*)saved : nullptr;
   return D == 64 ? fwd_tc<64>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, H_kv, T, scale, ws,
-                              p, st)
+                              p, sv, st)
                  : fwd_tc<128>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, H_kv, T, scale, ws,
-                               p, st);
+                               p, sv, st);
+}
+
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dO,
+             const float* lse, const float* rope_cos, const float* rope_sin,
+             const int32_t* cu_seqlens, int B, int H, int H_kv, int T, int D, float scale,
+             int dtype, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+             const void* saved, void* stream);
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd_gqa(const void* q, const void* k, const void* v, const float* rope_cos,
+                 const float* rope_sin, const int32_t* cu_seqlens, void* o, float* lse, int B,
+                 int H, int H_kv, int T, int D, float scale, int dtype, void* workspace,
+                 size_t ws_bytes, void* stream) {
+  return fwd_impl(q, k, v, rope_cos, rope_sin, cu_seqlens, o, lse, B, H, H_kv, T, D, scale,
+                  dtype, workspace, ws_bytes, nullptr, stream);
+}
+
+int attn_fwd_save(const void* q, const void* k, const void* v, const float* rope_cos,
+                  const float* rope_sin, const int32_t* cu_seqlens, void* o, float* lse, int B,
+                  int H, int H_kv, int T, int D, float scale, int dtype, void* workspace,
+                  size_t ws_bytes, void* saved, size_t saved_bytes, void* stream) {
+  const int rc = check_saved(saved, saved_bytes, B, H, H_kv, T, D, dtype, rope_cos);
+  if (rc) return rc;
+  return fwd_impl(q, k, v, rope_cos, rope_sin, cu_seqlens, o, lse, B, H, H_kv, T, D, scale,
+                  dtype, workspace, ws_bytes, saved, stream);
 }
 
 int attn_fwd(const void* q, const void* k, const void* v, const float* rope_cos,
@@ -487,6 +566,30 @@ int attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, con
                  const int32_t* cu_seqlens, int B, int H, int H_kv, int T, int D, float scale,
                  int dtype, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
                  void* stream) {
+  return bwd_impl(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, H_kv, T, D, scale,
+                  dtype, dq, dk, dv, workspace, ws_bytes, nullptr, stream);
+}
+
+int attn_bwd_saved(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                   const float* lse, const float* rope_cos, const float* rope_sin,
+                   const int32_t* cu_seqlens, int B, int H, int H_kv, int T, int D, float scale,
+                   int dtype, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                   const void* saved, size_t saved_bytes, void* stream) {
+  const int rc = check_saved(saved, saved_bytes, B, H, H_kv, T, D, dtype, rope_cos);
+  if (rc) return rc;
+  return bwd_impl(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, H_kv, T, D, scale,
+                  dtype, dq, dk, dv, workspace, ws_bytes, saved, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dO,
+             const float* lse, const float* rope_cos, const float* rope_sin,
+             const int32_t* cu_seqlens, int B, int H, int H_kv, int T, int D, float scale,
+             int dtype, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+             const void* saved, void* stream) {
   int rc = check_common(q, k, v, rope_cos, rope_sin, cu_seqlens, B, H, H_kv, T, D, scale, dtype,
                         workspace, ws_bytes, 1);
   if (rc) return rc;
@@ -511,11 +614,16 @@ int attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, con
                    : bwd_simt<float, 128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, delta,
                                           dq, dk, dv, B, H, H_kv, T, scale, st);
   }
+  const char* sv = (rope_cos && saved) ? (const char*)saved : nullptr;
   return D == 64 ? bwd_tc<64>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, dq, dk, dv, B, H,
-                              H_kv, T, scale, ws, p, st)
+                              H_kv, T, scale, ws, p, sv, st)
                  : bwd_tc<128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, dq, dk, dv, B, H,
-                               H_kv, T, scale, ws, p, st);
+                               H_kv, T, scale, ws, p, sv, st);
 }
+
+}  // namespace
+
+extern "C" {
 
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
              const float* lse, const float* rope_cos, const float* rope_sin,

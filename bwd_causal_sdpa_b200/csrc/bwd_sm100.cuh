@@ -610,8 +610,7 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
       const int i0 = (qt0 + i % n_q) * 128;
       const bool need_mask = (i0 + qc0 < j) || (i0 + qc0 + QC - 1 >= de_j);
       const float* sl = reinterpret_cast<const float*>(sg + L::kLD + (i & 1) * 1024);
-      if (!mbar_wait(bar(L::bQFull + (i & 1)), (i >> 1) & 1, abort_flag) ||
-          !mbar_wait(bar(L::bSFull), i & 1, abort_flag))
+      if (!mbar_wait2(bar(L::bQFull + (i & 1)), (i >> 1) & 1, bar(L::bSFull), i & 1, abort_flag))
         return false;
       tc_fence_after();
       uint32_t s[QC];
@@ -620,6 +619,8 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(L::bSFree));  // the S^T columns may take the next tile
+      // asked now, answered by the time P is formed (see the wait below)
+      const bool ds_free = i == 0 || mbar_test(bar(L::bDSFree), (i - 1) & 1);
       float scl = p.scale_log2;
       if constexpr (kF16) {
         // loaded with this tile's lse2 and Delta rows
@@ -645,7 +646,7 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
         pf[2 * e + 1] = pv.y;
       }
       // dQ(i-1) and dK(i-1) must be done reading dS^T(i-1) from the tile
-      if (i > 0 && !mbar_wait(bar(L::bDSFree), (i - 1) & 1, abort_flag)) return false;
+      if (!ds_free && !mbar_wait(bar(L::bDSFree), (i - 1) & 1, abort_flag)) return false;
       uint32_t w[QC / 2];
 #pragma unroll
       for (int e = 0; e < QC / 2; ++e) w[e] = pack_bf16(pf[2 * e], pf[2 * e + 1]);
@@ -663,6 +664,7 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
 #pragma unroll
       for (int c = 0; c < QC / 32; ++c) tmem_ld32(tDP + qc0 + 32 * c, dpv + 32 * c);
       tmem_wait_ld();
+      const bool dv_done = mbar_test(bar(L::bDVDone), i & 1);  // answered by the store below
       uint32_t w[QC / 2];
       const float dsm = cscale * qinv_i;  // 1 for bf16 operands
       const float2 dsm2 = make_float2(dsm, dsm);
@@ -679,7 +681,7 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
           w[e] = pack_bf16(a.x, a.y);
         }
       }
-      if (!mbar_wait(bar(L::bDVDone), i & 1, abort_flag)) return false;
+      if (!dv_done && !mbar_wait(bar(L::bDVDone), i & 1, abort_flag)) return false;
       store_row(w);
       fence_proxy_async_smem();
       tc_fence_before();

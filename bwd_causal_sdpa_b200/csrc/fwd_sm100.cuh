@@ -236,8 +236,10 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       for (int li = 0; ok && li <= n; ++li) {
         if (li < n) {  // S_t(li) = Q_t K_j^T
           const int j = lo + li;
-          if (!mbar_wait(bar(L::bKFull + stage(j)), phase(j), abort_flag)) { ok = false; break; }
-          if (li > 0 && !mbar_wait(bar(L::bSFree + t), (li - 1) & 1, abort_flag)) { ok = false; break; }
+          const bool ready = li > 0 ? mbar_wait2(bar(L::bKFull + stage(j)), phase(j), bar(L::bSFree + t),
+                                                 (li - 1) & 1, abort_flag)
+                                    : mbar_wait(bar(L::bKFull + stage(j)), phase(j), abort_flag);
+          if (!ready) { ok = false; break; }
           tc_fence_after();
           const uint32_t kbase = sb0 + L::kK + stage(j) * L::kKVBytes;
 #pragma unroll
@@ -251,8 +253,8 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         }
         if (li > 0) {  // O_t += P_t(lj) V_j
           const int lj = li - 1, j = lo + lj;
-          if (!mbar_wait(bar(L::bVFull + stage(j)), phase(j), abort_flag) ||
-              !mbar_wait(bar(L::bPFull + 2 * t + (lj & 1)), (lj >> 1) & 1, abort_flag)) {
+          if (!mbar_wait2(bar(L::bVFull + stage(j)), phase(j), bar(L::bPFull + 2 * t + (lj & 1)),
+                          (lj >> 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -284,10 +286,13 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     const uint32_t tO = tmem + lane_base + L::kColO + 128 * t;
     const int ds_i = p.doc_start ? p.doc_start[row0 + min(i, T - 1)] - row0 : 0;
     const float fq = p.q_fac ? p.q_fac[((size_t)bh * p.n_qtiles + min(qt, p.n_qtiles - 1)) * 4] : 1.f;
+    const float* kfp = p.k_fac ? p.k_fac + (size_t)bhk * p.n_qtiles : nullptr;
+    float kf = (kfp && active) ? kfp[lo >> 1] : 1.f;  // this block's k factor (loaded a block ahead)
     float m = -INFINITY, l = 0.f;
     bool ok = active;
     for (int li = 0; ok && li < n; ++li) {
       const int j = lo + li, j0 = j * 64;  // first key of the block
+      const float kf_next = (kfp && li + 1 < n) ? kfp[(j + 1) >> 1] : 1.f;
       if (!mbar_wait(bar(L::bSFull + t), li & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       uint32_t s[64];
@@ -304,7 +309,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       // scales to below 2^-26, so each kept probability rounds to exactly 1
       // as it should, while a masked score still becomes -inf rather than
       // inf * 0 = NaN.
-      float sc = p.scale_log2 * fq * (p.k_fac ? p.k_fac[bhk * p.n_qtiles + (j >> 1)] : 1.f);
+      float sc = p.scale_log2 * fq * kf;
       if (sc == 0.f) sc = 1.17549435e-38f;
       const bool pos_scale = sc > 0.f;
       const bool need_mask = (j0 + 63 > i) || (j0 < ds_i);
@@ -342,6 +347,10 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
         m = mx;
       }
       const float mref = (m == -INFINITY) ? 0.f : m;
+      // P_t(li) goes to buffer li & 1, last read by PV_t(li - 2): asked now,
+      // answered by the time P is formed
+      const bool buf_free =
+          li < 2 || mbar_test(bar(L::bPVDone + 2 * t + (li & 1)), ((li - 2) >> 1) & 1);
       // p = 2^(s * sc - m) two at a time, kPolyPairs of the 32 pairs on the
       // FMA pipe, the others on MUFU
       const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-mref, -mref);
@@ -361,8 +370,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       }
       const float2 la = __fadd2_rn(l2[0], l2[1]), lb = __fadd2_rn(l2[2], l2[3]);
       l += (la.x + la.y) + (lb.x + lb.y);
-      // P_t(li) goes to buffer li & 1, last read by PV_t(li - 2)
-      if (li >= 2 &&
+      if (!buf_free &&
           !mbar_wait(bar(L::bPVDone + 2 * t + (li & 1)), ((li - 2) >> 1) & 1, abort_flag)) {
         ok = false;
         break;
@@ -392,6 +400,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::bPFull + 2 * t + (li & 1)));
+      kf = kf_next;
     }
     if (ok && mbar_wait(bar(L::bOFinal + t), 0, abort_flag)) {
       tc_fence_after();

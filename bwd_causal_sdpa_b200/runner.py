@@ -13,8 +13,9 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (ATTN_BF16, ATTN_F32, attn_bwd, attn_bwd_gqa, attn_fwd, attn_fwd_gqa,
-               attn_get_status, attn_workspace_bytes, attn_workspace_bytes_gqa, check)
+from . import (ATTN_BF16, ATTN_F32, attn_bwd, attn_bwd_gqa, attn_bwd_saved, attn_fwd,
+               attn_fwd_gqa, attn_fwd_save, attn_get_status, attn_saved_bytes,
+               attn_workspace_bytes, attn_workspace_bytes_gqa, check)
 
 
 def torch_dtype(dtype: int):
@@ -42,10 +43,16 @@ class AttnRunner:
     """Holds q, k, v, dO (inputs), o, lse, dq, dk, dv (outputs), the RoPE
     tables, cu_seqlens and one workspace sized for the larger of the two
     calls, all on one device. With H_kv < H (grouped-query attention) k, v,
-    dk, dv have H_kv heads and the *_gqa entry points are called."""
+    dk, dv have H_kv heads and the *_gqa entry points are called.
+
+    save=True (a training step's usual pattern) also holds the buffer in
+    which attn_fwd_save keeps the forward's rotated q, k, and runs the pair
+    attn_fwd_save / attn_bwd_saved; backward() then needs the forward() of
+    the same inputs before it. save=False runs the plain calls."""
 
     def __init__(self, B, H, T, D, *, dtype=ATTN_BF16, scale=None, rope=None, cu_seqlens=None,
-                 device="cuda", stream: Optional[torch.cuda.Stream] = None, H_kv=None):
+                 device="cuda", stream: Optional[torch.cuda.Stream] = None, H_kv=None,
+                 save: bool = False):
         H_kv = H if H_kv is None else H_kv
         self.p = Problem(B, H, T, D, 1.0 / math.sqrt(D) if scale is None else scale, dtype, H_kv)
         self.device = torch.device(device)
@@ -70,13 +77,16 @@ class AttnRunner:
             self.ws_bytes = max(attn_workspace_bytes_gqa(B, H, H_kv, T, D, dtype, 0),
                                 attn_workspace_bytes_gqa(B, H, H_kv, T, D, dtype, 1))
         self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=self.device)
+        self.saved_bytes = attn_saved_bytes(B, H, H_kv, T, D, dtype, rope is not None) if save else 0
+        self.saved = (torch.empty(self.saved_bytes, dtype=torch.uint8, device=self.device)
+                      if self.saved_bytes else None)
 
     @classmethod
-    def from_workload(cls, w, device="cuda", stream=None) -> "AttnRunner":
+    def from_workload(cls, w, device="cuda", stream=None, save: bool = False) -> "AttnRunner":
         dtype = ATTN_BF16 if w.dtype == "bf16" else ATTN_F32
         rope = None if w.rope_cos is None else (w.rope_cos, w.rope_sin)
         r = cls(w.B, w.H, w.T, w.D, dtype=dtype, scale=w.scale, rope=rope,
-                cu_seqlens=w.cu_seqlens, device=device, stream=stream, H_kv=w.kv_heads)
+                cu_seqlens=w.cu_seqlens, device=device, stream=stream, H_kv=w.kv_heads, save=save)
         r.load_inputs(w.q, w.k, w.v, w.do)
         return r
 
@@ -86,6 +96,12 @@ class AttnRunner:
 
     def forward(self) -> None:
         p = self.p
+        if self.saved is not None:
+            check(attn_fwd_save(self.q, self.k, self.v, self.rope_cos, self.rope_sin, self.cu,
+                                self.o, self.lse, p.B, p.H, p.H_kv, p.T, p.D, p.scale, p.dtype,
+                                self.ws, self.ws_bytes, self.saved, self.saved_bytes,
+                                self.stream), "attn_fwd_save")
+            return
         if p.H_kv != p.H:
             check(attn_fwd_gqa(self.q, self.k, self.v, self.rope_cos, self.rope_sin, self.cu,
                                self.o, self.lse, p.B, p.H, p.H_kv, p.T, p.D, p.scale, p.dtype,
@@ -97,6 +113,12 @@ class AttnRunner:
 
     def backward(self) -> None:
         p = self.p
+        if self.saved is not None:
+            check(attn_bwd_saved(self.q, self.k, self.v, self.o, self.do, self.lse, self.rope_cos,
+                                 self.rope_sin, self.cu, p.B, p.H, p.H_kv, p.T, p.D, p.scale,
+                                 p.dtype, self.dq, self.dk, self.dv, self.ws, self.ws_bytes,
+                                 self.saved, self.saved_bytes, self.stream), "attn_bwd_saved")
+            return
         if p.H_kv != p.H:
             check(attn_bwd_gqa(self.q, self.k, self.v, self.o, self.do, self.lse, self.rope_cos,
                                self.rope_sin, self.cu, p.B, p.H, p.H_kv, p.T, p.D, p.scale,

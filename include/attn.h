@@ -145,6 +145,48 @@ size_t attn_workspace_bytes(int B, int H, int T, int D, int dtype, int is_bwd);
 size_t attn_workspace_bytes_gqa(int B, int H, int H_kv, int T, int D, int dtype, int is_bwd);
 
 /*
+ * Keeping the forward's rotated operands for the backward (the saved
+ * activations of a training step). With bf16 storage and RoPE tables the
+ * forward rotates q and k once (interleaved pairs at document positions,
+ * ARK README, "Inference architecture (EKO)"; Forge README, "Architecture")
+ * into fp16 tiles with power-of-two tile factors, and the backward recomputes
+ * the scores from exactly those operands. attn_fwd_save leaves them in the
+ * caller's buffer `saved`; attn_bwd_saved reads them from there instead of
+ * rotating q and k again (one pass over q and k fewer per step).
+ *
+ * attn_saved_bytes: bytes of that buffer; 0 when there is nothing to keep
+ * (dtype ATTN_F32, has_rope = 0, or invalid sizes). Pure host function.
+ * attn_fwd_save: attn_fwd_gqa plus `saved` (device, 16-byte aligned,
+ * saved_bytes >= attn_saved_bytes(...), written by the call).
+ * attn_bwd_saved: attn_bwd_gqa plus `saved` (read only): it must hold what
+ * attn_fwd_save wrote for the same q, k, rope tables, cu_seqlens and sizes,
+ * unchanged since; results are then identical to attn_bwd_gqa's. That
+ * correspondence is the caller's contract and is not checked.
+ * For both: when attn_saved_bytes is 0, or saved is NULL, the call is the
+ * plain attn_fwd_gqa / attn_bwd_gqa and `saved` is not touched. Misaligned
+ * saved: ATTN_EALIGN; saved_bytes too small: ATTN_EWORKSPACE. The buffer
+ * stays owned by the caller; workspaces are sized as for the plain calls.
+ */
+size_t attn_saved_bytes(int B, int H, int H_kv, int T, int D, int dtype, int has_rope);
+
+int attn_fwd_save(const void* q, const void* k, const void* v,
+                  const float* rope_cos, const float* rope_sin,
+                  const int32_t* cu_seqlens,
+                  void* o, float* lse,
+                  int B, int H, int H_kv, int T, int D, float scale,
+                  int dtype, void* workspace, size_t ws_bytes,
+                  void* saved, size_t saved_bytes, void* stream);
+
+int attn_bwd_saved(const void* q, const void* k, const void* v, const void* o,
+                   const void* dO, const float* lse,
+                   const float* rope_cos, const float* rope_sin,
+                   const int32_t* cu_seqlens,
+                   int B, int H, int H_kv, int T, int D, float scale, int dtype,
+                   void* dq, void* dk, void* dv,
+                   void* workspace, size_t ws_bytes,
+                   const void* saved, size_t saved_bytes, void* stream);
+
+/*
  * attn_decode -- decode attention: one new token per sequence against a
  * key/value cache (Forge README, "Roadmap": a KV cache for generation on the
  * training attention module; ARK README, "Inference architecture (EKO)":

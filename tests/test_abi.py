@@ -307,3 +307,31 @@ def test_noalloc_counts_document_ranges_only_when_packed():
     if torch.cuda.is_available():
         pytest.skip("the unpacked call would launch kernels on fake addresses")
     assert A.attn_bwd_noalloc(*args, None, *tail) == A.ATTN_ECUDA
+
+
+def test_saved_operand_buffer_size_and_validation():
+    import bwd_causal_sdpa_b200 as A
+
+    up = lambda x: (x + 255) // 256 * 256
+    B, H, Hkv, T, D = 2, 8, 2, 300, 128
+    nt = (T + 127) // 128
+    want = (up(B * H * T * D * 2) + up(B * Hkv * T * D * 2) + up(B * H * nt * 16)
+            + up(B * Hkv * nt * 4))
+    assert A.attn_saved_bytes(B, H, Hkv, T, D, A.ATTN_BF16, 1) == want
+    # nothing to keep: float32 storage, no RoPE, invalid sizes
+    assert A.attn_saved_bytes(B, H, Hkv, T, D, A.ATTN_F32, 1) == 0
+    assert A.attn_saved_bytes(B, H, Hkv, T, D, A.ATTN_BF16, 0) == 0
+    assert A.attn_saved_bytes(B, H, 3, T, D, A.ATTN_BF16, 1) == 0
+    assert A.attn_saved_bytes(B, H, Hkv, T, 96, A.ATTN_BF16, 1) == 0
+
+    common = dict(q=P, k=P, v=P, rope_cos=P, rope_sin=P, cu_seqlens=None, B=B, H=H, H_kv=Hkv,
+                  T=T, D=D, scale=0.088, dtype=A.ATTN_BF16, workspace=P, ws_bytes=1 << 30)
+    fwd = lambda **kw: A.attn_fwd_save(**{**common, "o": P, "lse": P, "saved": P,
+                                          "saved_bytes": want, **kw})
+    bwd = lambda **kw: A.attn_bwd_saved(**{**common, "o": P, "dO": P, "lse": P, "dq": P,
+                                           "dk": P, "dv": P, "saved": P, "saved_bytes": want,
+                                           **kw})
+    for call in (fwd, bwd):
+        assert call(saved=P + 8) == A.ATTN_EALIGN
+        assert call(saved_bytes=want - 1) == A.ATTN_EWORKSPACE
+        assert call(q=None) == A.ATTN_EINVAL  # the plain call's checks still apply
