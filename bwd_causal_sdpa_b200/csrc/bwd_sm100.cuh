@@ -314,11 +314,17 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
     }
   } else if (warp == L::kMmaWarp) {
     // ---------------- MMA issuer ----------------
-    // Five groups per query tile i: S(i), dP(i), dV(i), dK(i), dQ(i). Each
-    // group is issued in tile order, but across groups the issuer takes
-    // whichever is ready (probing its barriers without blocking), in the
-    // priority dV, S, dK, dQ, dP. TMEM: S^T(i) and then dQ(i-1) share the S^T
-    // columns, dP^T has its own. Readiness:
+    // Five groups per query tile i: S(i), dP(i), dV(i), dK(i), dQ(i). TMEM:
+    // S^T(i) and then dQ(i-1) share the S^T columns, dP^T has its own.
+    // With dQ formed here the issuer follows one fixed order, S(0) dP(0),
+    // then per tile dV(i) S(i+1) dK(i) dQ(i) dP(i+1), each group after a
+    // blocking wait for what it needs. That wait is normally complete already
+    // and its answer then arrives while the previous group's products are
+    // still queued on the tensor pipe; probing several groups for readiness
+    // instead costs the probes' answer time before every issue, with the pipe
+    // draining meanwhile (measured at 8K: 767 against 886 us). Without dQ
+    // the issuer takes whichever group is ready, probing in the priority dV,
+    // S, dK, dP. Readiness:
     //   S(i):  Q(i) loaded; the S^T columns free: S(0) always, S(1) once the
     //          elementwise warps have read S(0), S(i >= 2) once dQ(i-2) has
     //          been read out
@@ -345,8 +351,83 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
       };
       int nS = 0, nP = 0, nV = 0, nK = 0, nQ = 0;  // next tile of each group
       bool ok = mbar_wait(bar(L::bKV), 0, abort_flag);
+      if constexpr (kDQ) {
+        // Every barrier is waited on for its phases in order, and its next
+        // phase needs a group issued after the wait, so the parity is exact.
+        auto wait1 = [&](int b1, int ph1) { return mbar_wait(bar(b1), ph1 & 1, abort_flag); };
+        auto wait2 = [&](int b1, int ph1, int b2, int ph2) {
+          return mbar_wait2(bar(b1), ph1 & 1, bar(b2), ph2 & 1, abort_flag);
+        };
+        auto group_S = [&](int i) -> bool {
+          const bool r = i == 0   ? wait1(L::bQFull, 0)
+                         : i == 1 ? wait2(L::bQFull + 1, 0, L::bSFree, 0)
+                                  : wait2(L::bQFull + (i & 1), i >> 1, L::bDQFree, i - 2);
+          if (!r) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
+            mma_ss(tS, smem_desc_sw128(sb0 + L::kK + off, 16, 1024),
+                   smem_desc_sw128(qbuf(i) + off, 16, 1024), id_s, kk > 0);
+          }
+          mma_commit(bar(L::bSFull));
+          return true;
+        };
+        auto group_dP = [&](int i) -> bool {
+          if (!wait1(L::bDOFull + i % L::kDOStages, i / L::kDOStages)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
+            mma_ss(tDP, smem_desc_sw128(sb0 + L::kV + off, 16, 1024),
+                   smem_desc_sw128(obuf(i) + off, 16, 1024), id_dp, kk > 0);
+          }
+          mma_commit(bar(L::bDPFull));
+          return true;
+        };
+        auto group_dV = [&](int i) -> bool {
+          if (!wait1(L::bPFull, i)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tDV, smem_desc_sw128(ps + (kk >> 2) * L::kBlockBytes + (kk & 3) * 32, 16, 1024),
+                   smem_desc_sw128(obuf(i) + kk * 2048, L::kBlockBytes, 1024), id_dv,
+                   (i > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(L::bDVDone));
+          mma_commit(bar(L::bDOEmpty + i % L::kDOStages));
+          return true;
+        };
+        auto group_dK = [&](int i) -> bool {
+          if (!wait1(L::bDSFull, i)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tDK, smem_desc_sw128(ps + (kk >> 2) * L::kBlockBytes + (kk & 3) * 32, 16, 1024),
+                   smem_desc_sw128(qbuf(i) + kk * 2048, L::kBlockBytes, 1024), id_dk,
+                   (i > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(L::bQEmpty + (i & 1)));
+          if (i == n_it - 1) mma_commit(bar(L::bFinal));
+          return true;
+        };
+        auto group_dQ = [&](int i) -> bool {
+          // into the S^T columns once the elementwise warps have read S(i+1)
+          if (i < n_it - 1 && !wait1(L::bSFree, i + 1)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tS, smem_desc_sw128(ps + kk * 2048, L::kBlockBytes, 1024),
+                   smem_desc_sw128(sb0 + L::kK + kk * 2048, L::kBlockBytes, 1024), id_dq, kk > 0);
+          mma_commit(bar(L::bDQFull));
+          mma_commit(bar(L::bDSFree));  // the P/dS tile is free again (dK(i) is covered too)
+          return true;
+        };
+        ok = ok && group_S(0) && group_dP(0);
+        for (int i = 0; ok && i < n_it; ++i)
+          ok = group_dV(i) && (i + 1 == n_it || group_S(i + 1)) && group_dK(i) && group_dQ(i) &&
+               (i + 1 == n_it || group_dP(i + 1));
+      }
       long long t_last = clock64();
-      while (ok && (kDQ ? nQ : nK) < n_it) {
+      while (!kDQ && ok && nK < n_it) {
         if (nV < nP && mbar_test(bar(L::bPFull), nV & 1)) {
           // dV += P^T dO (P^T K-major in the P/dS tile, dO MN-major)
           tc_fence_after();
