@@ -133,8 +133,10 @@ def kernel_algorithmic(name: str, w, kinds_seen) -> tuple:
         if w.dtype != "bf16":  # Delta only
             return "hbm", 2 * N * elem + 4 * R, "byte"
         # bf16 backward row pass: read o, dO, lse; write -Delta and -lse*log2e,
-        # zero the fp32 dq accumulator
-        return "hbm", 2 * N * elem + 12 * R + 4 * N, "byte"
+        # zero the fp32 dq accumulator; with RoPE (fp16 operands) also read v
+        # for the per-head norm statistics
+        v_read = Nkv * elem if w.rope_cos is not None else 0
+        return "hbm", 2 * N * elem + 12 * R + 4 * N + v_read, "byte"
     if name == "rope_prep":
         return "hbm", 2 * (N + Nkv) * elem, "byte"
     if name == "dq_finalize":
