@@ -237,6 +237,23 @@ int bwd_simt(const void* q, const void* k, const void* v, const void* o, const v
   return launch_status();
 }
 
+// The RoPE pre-pass over q and k (see prep.cuh): one block per tile, batch and
+// group of heads, the tile's table rows staged in dynamic shared memory.
+template <int D>
+int launch_rope_prep(const void* q, const void* k, const float* rc, const float* rs,
+                     const int32_t* ds, __half* qo, __half* ko, float* qf, float* kf, float* hstat,
+                     int B, int H, int Hkv, int T, int nt, cudaStream_t st) {
+  static bool smem_set[64] = {};
+  constexpr int smem = rope_prep_smem_bytes<D>();
+  if (!ensure_smem(rope_prep_kernel<D>, smem, smem_set)) return ATTN_ECUDA;
+  const int group = rope_prep_group(B, H, Hkv, nt);
+  const dim3 grid(nt, B, (H + Hkv + group - 1) / group);
+  ATTN_LAUNCH(KK_ROPE_PREP, st, pdl_launch(rope_prep_kernel<D>, grid, kRopePrepThreads, smem, st,
+                                           (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs,
+                                           ds, qo, ko, qf, kf, hstat, B, H, Hkv, T, nt, group));
+  return launch_status();
+}
+
 template <int D>
 int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const float* rs,
            const int32_t* ds, void* o, float* lse, int B, int H, int Hkv, int T, float scale,
@@ -255,10 +272,8 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
     __half* kh = (__half*)(saved ? saved + sp.k16 : ws + wp.k16);
     qf = (float*)(saved ? saved + sp.qfac : ws + wp.qfac);
     kf = (float*)(saved ? saved + sp.kfac : ws + wp.kfac);
-    ATTN_LAUNCH(KK_ROPE_PREP, st, pdl_launch(rope_prep_kernel<D>, dim3(nt, BH, 2), kRopePrepThreads, 0, st,
-                                             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds,
-                                             qh, kh, qf, kf, (float*)nullptr, B, H, Hkv, T, nt));
-    if (launch_status()) return ATTN_ECUDA;
+    if (launch_rope_prep<D>(q, k, rc, rs, ds, qh, kh, qf, kf, nullptr, B, H, Hkv, T, nt, st))
+      return ATTN_ECUDA;
     qs = qh;
     ks = kh;
   }
@@ -366,10 +381,8 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
     if (cudaMemsetAsync(hstat, 0, (size_t)BH * 4 * sizeof(float), st) != cudaSuccess) return ATTN_ECUDA;
   } else if (f16) {
     // the forward's rotation, factors included (same kernel, same values)
-    ATTN_LAUNCH(KK_ROPE_PREP, st, pdl_launch(rope_prep_kernel<D>, dim3(nt, BH, 2), kRopePrepThreads, 0, st,
-                                             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs, ds,
-                                             q16, k16, qinv, kinv, hstat, B, H, Hkv, T, nt));
-    if (launch_status()) return ATTN_ECUDA;
+    if (launch_rope_prep<D>(q, k, rc, rs, ds, q16, k16, qinv, kinv, hstat, B, H, Hkv, T, nt, st))
+      return ATTN_ECUDA;
   }
   const bool dq_pass = use_dq_pass(D);
   const long rows_pad = (long)BH * Tpad;

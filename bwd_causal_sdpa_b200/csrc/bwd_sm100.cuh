@@ -741,25 +741,30 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
       const float* sd = reinterpret_cast<const float*>(sg + L::kLD + (i & 1) * 1024) + 128;
       if (!mbar_wait(bar(L::bDPFull), i & 1, abort_flag)) return false;
       tc_fence_after();
-      uint32_t dpv[QC];
-#pragma unroll
-      for (int c = 0; c < QC / 32; ++c) tmem_ld32(tDP + qc0 + 32 * c, dpv + 32 * c);
-      tmem_wait_ld();
-      const bool dv_done = mbar_test(bar(L::bDVDone), i & 1);  // answered by the store below
+      // 16 columns of dP^T at a time: fewer registers live next to P
       uint32_t w[QC / 2];
+      bool dv_done = false;
       const float dsm = cscale * qinv_i;  // 1 for bf16 operands
       const float2 dsm2 = make_float2(dsm, dsm);
 #pragma unroll
-      for (int e = 0; e < QC / 2; ++e) {
-        const float2 nd = reinterpret_cast<const float2*>(sd + qc0)[e];  // -Delta pair
-        const float2 dpp = make_float2(__uint_as_float(dpv[2 * e]), __uint_as_float(dpv[2 * e + 1]));
-        if constexpr (kF16) {
-          const float2 a = __fmul2_rn(make_float2(pf[2 * e], pf[2 * e + 1]),
-                                      __fmul2_rn(__fadd2_rn(dpp, nd), dsm2));
-          w[e] = pack_half(a.x, a.y);
-        } else {
-          const float2 a = __fmul2_rn(make_float2(pf[2 * e], pf[2 * e + 1]), __fadd2_rn(dpp, nd));
-          w[e] = pack_bf16(a.x, a.y);
+      for (int h = 0; h < QC / 16; ++h) {
+        uint32_t dpv[16];
+        tmem_ld16(tDP + qc0 + 16 * h, dpv);
+        tmem_wait_ld();
+        if (h == 0) dv_done = mbar_test(bar(L::bDVDone), i & 1);  // answered by the store below
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) {
+          const int e = 8 * h + e2;
+          const float2 nd = reinterpret_cast<const float2*>(sd + qc0)[e];  // -Delta pair
+          const float2 dpp = make_float2(__uint_as_float(dpv[2 * e2]), __uint_as_float(dpv[2 * e2 + 1]));
+          if constexpr (kF16) {
+            const float2 a = __fmul2_rn(make_float2(pf[2 * e], pf[2 * e + 1]),
+                                        __fmul2_rn(__fadd2_rn(dpp, nd), dsm2));
+            w[e] = pack_half(a.x, a.y);
+          } else {
+            const float2 a = __fmul2_rn(make_float2(pf[2 * e], pf[2 * e + 1]), __fadd2_rn(dpp, nd));
+            w[e] = pack_bf16(a.x, a.y);
+          }
         }
       }
       if (!dv_done && !mbar_wait(bar(L::bDVDone), i & 1, abort_flag)) return false;
