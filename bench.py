@@ -89,6 +89,9 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--bwd-route", type=int, default=0,
+                    help="backward route (attn_set_backward_route): 0 default, 1 key-tile dK/dV + "
+                         "query-tile dQ pass, 2 CTA-pair dK/dV (D = 128) + query-tile dQ pass")
     ap.add_argument("--no-save", action="store_true",
                     help="plain attn_fwd / attn_bwd (the backward rotates q, k again)")
     ap.add_argument("--sustain", type=float, default=0.0,
@@ -410,6 +413,7 @@ def run_ours(args):
     cfg = config_by_name(args.workload)
     w = make_workload(cfg, H_kv=args.kv_heads)
     stream = torch.cuda.Stream(dev)
+    A.check(A.attn_set_backward_route(args.bwd_route), "attn_set_backward_route")
     r = AttnRunner.from_workload(w, device=dev, stream=stream, save=not args.no_save)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     peaks, peak_src = load_peaks()
@@ -648,7 +652,8 @@ def run_ours(args):
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic (seeded)",
             "config": dict(workload_config(w, l2="flushed between steps (256 MiB write outside the step events)"),
                            calls=("attn_fwd_gqa + attn_bwd_gqa" if args.no_save or r.saved is None
-                                  else "attn_fwd_save + attn_bwd_saved (rotated q, k kept between them)")),
+                                  else "attn_fwd_save + attn_bwd_saved (rotated q, k kept between them)"),
+                           backward_route=args.bwd_route),
             "pct_of_bf16_peak": value / world / peaks["bf16_tflops"],
             "pct_of_bf16_peak_sustained": value / world / peaks["bf16_tflops_sustained"],
             "peaks_source": peak_src,

@@ -67,6 +67,7 @@ _SIGNATURES = {
     "attn_error_string": (ctypes.c_char_p, [_I]),
     "attn_exp2_selftest": (_I, [_P, _P, _I, _P]),
     "attn_debug_withhold": (_I, [_I]),
+    "attn_set_backward_route": (_I, [_I]),
     "attn_launch_count": (ctypes.c_ulonglong, []),
     "attn_tile_counts": (_I, [ctypes.POINTER(ctypes.c_ulonglong)] * 3),
     "attn_profile_enable": (_I, [_I]),
@@ -266,6 +267,12 @@ def attn_debug_withhold(what) -> int:
 
 def attn_launch_count() -> int:
     return int(_lib.attn_launch_count())
+
+
+def attn_set_backward_route(route: int) -> int:
+    """0 default, 1 key-tile dK/dV + query-tile dQ pass, 2 CTA-pair dK/dV
+    (D = 128) + query-tile dQ pass (see include/attn.h)."""
+    return int(_lib.attn_set_backward_route(int(route)))
 
 
 def attn_tile_counts():

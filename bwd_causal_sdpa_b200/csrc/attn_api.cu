@@ -10,6 +10,7 @@
 #include "attn.h"
 #include "common.cuh"
 #include "bwd_sm100.cuh"
+#include "bwd_pair_sm100.cuh"
 #include "dq_sm100.cuh"
 #include "decode.cuh"
 #include "fwd_sm100.cuh"
@@ -348,6 +349,33 @@ constexpr bool use_dq_pass(int D) {
   return (D == 64 ? ATTN_DQ_PASS_D64 : ATTN_DQ_PASS_D128) != kDqRouteSwapped;
 }
 
+// The tensor-core backward's route, chosen at run time by
+// attn_set_backward_route: 0 = the default above, 1 = key-tile kernel without
+// dQ + query-tile dQ pass, 2 = the CTA-pair key-tile kernel (D = 128; D = 64
+// takes route 1) + query-tile dQ pass.
+int g_bwd_route = 0;
+int backward_route(int D) {
+  if (g_bwd_route == 2) return D == 128 ? 2 : 1;
+  if (g_bwd_route == 1) return 1;
+  return use_dq_pass(D) ? 1 : 0;
+}
+
+template <bool kF16>
+int launch_dkdv_pair(const void* qs, const void* dO, const CUtensorMap& mq, const CUtensorMap& mk,
+                     const CUtensorMap& mv, const CUtensorMap& mo, const bwd100::Params& prm,
+                     int T, int BH, cudaStream_t st) {
+  using L = bwd2::Layout<128>;
+  CUtensorMap mqr, mor;  // 64-row boxes: the row halves of q and dO
+  if (!make_tile_map(&mqr, qs, kF16, 128, T, BH, 64) || !make_tile_map(&mor, dO, false, 128, T, BH, 64))
+    return ATTN_ECUDA;
+  static bool smem_set[64] = {};
+  if (!ensure_smem(bwd2::dkdv_pair_kernel<128, kF16>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
+  const unsigned grid = 2u * (unsigned)(prm.BHkv * prm.n_split * ((prm.n_tiles + 1) / 2));
+  ATTN_LAUNCH(KK_DKDV, st, pdl_cluster_launch(bwd2::dkdv_pair_kernel<128, kF16>, grid, L::kThreads,
+                                              L::kSmemAlloc, st, 2u, mqr, mq, mk, mv, mor, mo, prm));
+  return launch_status();
+}
+
 template <int D>
 int bwd_tc(const void* q, const void* k, const void* v, const void* o, const void* dO,
            const float* lse, const float* rc, const float* rs, const int32_t* ds,
@@ -384,7 +412,8 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
     if (launch_rope_prep<D>(q, k, rc, rs, ds, q16, k16, qinv, kinv, hstat, B, H, Hkv, T, nt, st))
       return ATTN_ECUDA;
   }
-  const bool dq_pass = use_dq_pass(D);
+  const int route = backward_route(D);
+  const bool dq_pass = route != 0;
   const long rows_pad = (long)BH * Tpad;
   ATTN_LAUNCH(KK_DELTA, st, pdl_launch(bwd_prep_kernel<D>, (unsigned)(rows_pad * (D / 8) / 256), 256, 0, st,
                                        (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse, delta, lse2,
@@ -421,8 +450,12 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   prm.kinv = kinv;
   prm.hstat = hstat;
   const unsigned grid = (unsigned)(nt * BHkv * split);
-  int rc_k;
-  if (dq_pass)
+  int rc_k = ATTN_ECUDA;
+  if (route == 2) {  // backward_route gives 2 only at D = 128
+    if constexpr (D == 128)
+      rc_k = f16 ? launch_dkdv_pair<true>(qs, dO, mq, mk, mv, mo, prm, T, BH, st)
+                 : launch_dkdv_pair<false>(qs, dO, mq, mk, mv, mo, prm, T, BH, st);
+  } else if (dq_pass)
     rc_k = f16 ? launch_dkdv<D, true, false>(mq, mk, mv, mo, mdq, prm, grid, st)
                : launch_dkdv<D, false, false>(mq, mk, mv, mo, mdq, prm, grid, st);
   else
@@ -644,6 +677,12 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
              void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream) {
   return attn_bwd_gqa(q, k, v, o, dO, lse, rope_cos, rope_sin, cu_seqlens, B, H, H, T, D, scale,
                       dtype, dq, dk, dv, workspace, ws_bytes, stream);
+}
+
+int attn_set_backward_route(int route) {
+  if (route < 0 || route > 2) return ATTN_EINVAL;
+  g_bwd_route = route;
+  return ATTN_OK;
 }
 
 int attn_get_status(void* stream) {

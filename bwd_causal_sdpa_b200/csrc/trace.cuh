@@ -124,6 +124,28 @@ inline void pdl_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   if (e != cudaSuccess) pdl_launch_error() = e;
 }
 
+// pdl_launch for a kernel whose CTAs run as clusters of cluster_x along x.
+template <typename... KArgs, typename... Args>
+inline void pdl_cluster_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                               cudaStream_t st, unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) pdl_launch_error() = e;
+}
+
 // Wrap one kernel launch: ATTN_LAUNCH(kind, stream, pdl_launch(kernel, grid, block, smem, stream, ...));
 #define ATTN_LAUNCH(kind, st, ...)            \
   do {                                        \

@@ -368,6 +368,18 @@ int attn_exp2_selftest(const float* x, float* y, int n, void* stream);
  * ATTN_EUNSUPPORTED in a library built without the hooks (libattn.so). */
 int attn_debug_withhold(int what);
 
+/* attn_set_backward_route: which tensor-core backward the attn_bwd* calls
+ * of this process run (bf16 storage; float32 is unaffected). 0 = the
+ * library's default (the key-tile kernel forms dQ by reduce-adds into an fp32
+ * accumulator); 1 = the key-tile kernel for dK, dV and the query-tile pass
+ * for dQ; 2 = the key-tile kernel on CTA pairs (clusters of two CTAs,
+ * tcgen05 products of M = 256 keys issued for both SMs by one thread) for
+ * dK, dV at D = 128 (D = 64 takes route 1) and the query-tile pass for dQ.
+ * All routes compute the same gradients within the bf16 tolerance. A global
+ * setting for tuning and tests: calls already enqueued keep their route.
+ * Returns ATTN_OK or ATTN_EINVAL (route not 0, 1 or 2). Host only. */
+int attn_set_backward_route(int route);
+
 unsigned long long attn_launch_count(void);
 int attn_tile_counts(unsigned long long* fwd_tiles, unsigned long long* bwd_tiles,
                      unsigned long long* dq_tiles);

@@ -335,3 +335,11 @@ def test_saved_operand_buffer_size_and_validation():
         assert call(saved=P + 8) == A.ATTN_EALIGN
         assert call(saved_bytes=want - 1) == A.ATTN_EWORKSPACE
         assert call(q=None) == A.ATTN_EINVAL  # the plain call's checks still apply
+
+
+def test_backward_route_argument_checked():
+    import bwd_causal_sdpa_b200 as A
+
+    assert A.attn_set_backward_route(3) == A.ATTN_EINVAL
+    assert A.attn_set_backward_route(-1) == A.ATTN_EINVAL
+    assert A.attn_set_backward_route(0) == A.ATTN_OK
