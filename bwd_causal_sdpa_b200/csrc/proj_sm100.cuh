@@ -16,12 +16,15 @@
 //     is split over several CTAs), or scatters the columns into the
 //     head-major q, k, v tensors, rotating q and k by RoPE on the way.
 // Persistent: each CTA (at most one per SM) walks a strided list of work
-// units, a unit being one 128 x BN output tile (BN = 128 or 256) over one
-// share of K. K moves in 64-wide blocks through a four-stage ring that runs
-// across units; the accumulator alternates between two TMEM buffers, so the
-// epilogue of one unit overlaps the main loop of the next. Warps: TMA, MMA
-// (one elected thread issues tcgen05.mma) and four epilogue warps (thread =
-// TMEM lane = output row).
+// units, a unit being one 128 x 128 output tile over one share of K. 256-wide
+// tiles run on clusters of two CTAs instead: a unit is a 256 x 256 tile, each
+// CTA loads its 128 rows of A and half of the B tile, and CTA 0 issues
+// products of M = 256 (cta_group::2) that read both CTAs' tiles and write
+// both CTAs' accumulators. K moves in 64-wide blocks through a ring (four
+// stages, six for a pair) that runs across units; the accumulator alternates
+// between two TMEM buffers, so the epilogue of one unit overlaps the main
+// loop of the next. Warps: TMA, MMA (one elected thread issues tcgen05.mma)
+// and four epilogue warps (thread = TMEM lane = output row).
 #pragma once
 
 #include "common.cuh"
@@ -32,12 +35,17 @@ namespace proj100 {
 
 using namespace sm100;
 
-constexpr int kBM = 128, kBK = 64, kStages = 4;
+constexpr int kBM = 128, kBK = 64;
 
-template <int BN>
+// kPair: the CTA is one of a cluster of two that computes a 256 x BN tile
+// (this CTA's 128 rows), loading only its half of every B tile (BN / 2 rows)
+// while the pair's products (M = 256, issued by CTA 0) read both halves.
+template <int BN, bool kPair = false>
 struct Layout {
+  static constexpr int kStages = kPair ? 6 : 4;
+  static constexpr int kBLocal = kPair ? BN / 2 : BN;  // B rows this CTA loads
   static constexpr int kABytes = kBM * kBK * 2;
-  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kBBytes = kBLocal * kBK * 2;
   static constexpr int kA = 0;
   static constexpr int kB = kStages * kABytes;
   static constexpr int kBars = kB + kStages * kBBytes;
@@ -94,7 +102,7 @@ __device__ __forceinline__ void split_feature(const int* heads, int D, int f, in
 
 // Issue (or, with issue = false, only count the bytes of) the TMA boxes of
 // one operand tile: MN rows [mn0, mn0 + BMN) and K block kb, into dst.
-template <int BMN>
+template <int BMN, bool kPairLoad = false>
 __device__ __forceinline__ uint32_t operand_boxes(bool issue, const Operand& o,
                                                   const CUtensorMap* m0, const CUtensorMap* m1,
                                                   const CUtensorMap* m2, int mn_total, int T,
@@ -105,13 +113,15 @@ __device__ __forceinline__ uint32_t operand_boxes(bool issue, const Operand& o,
     // one box: BMN rows x 64 K values
     if (issue) {
       if (o.src == SRC_ROWS) {
-        tma_load_2d(dst, m0, bar, k0, mn0);
+        if (kPairLoad) tma_load_2d_pair(dst, m0, bar, k0, mn0);
+        else tma_load_2d(dst, m0, bar, k0, mn0);
       } else {
         int seg, h, d;
         split_feature(o.heads, D, k0, seg, h, d);
         const int b = mn0 / T, t = mn0 - b * T;
-        tma_load_3d(dst, seg == 0 ? m0 : (seg == 1 ? m1 : m2), bar, d, t,
-                    b * o.heads[seg] + h);
+        const CUtensorMap* mp = seg == 0 ? m0 : (seg == 1 ? m1 : m2);
+        if (kPairLoad) tma_load_3d_pair(dst, mp, bar, d, t, b * o.heads[seg] + h);
+        else tma_load_3d(dst, mp, bar, d, t, b * o.heads[seg] + h);
       }
     }
     return BMN * kBK * 2;
@@ -124,13 +134,15 @@ __device__ __forceinline__ uint32_t operand_boxes(bool issue, const Operand& o,
     if (f >= mn_total) break;
     if (issue) {
       if (o.src == SRC_ROWS) {
-        tma_load_2d(dst + j * 8192, m0, bar, f, k0);
+        if (kPairLoad) tma_load_2d_pair(dst + j * 8192, m0, bar, f, k0);
+        else tma_load_2d(dst + j * 8192, m0, bar, f, k0);
       } else {
         int seg, h, d;
         split_feature(o.heads, D, f, seg, h, d);
         const int b = k0 / T, t = k0 - b * T;
-        tma_load_3d(dst + j * 8192, seg == 0 ? m0 : (seg == 1 ? m1 : m2), bar, d, t,
-                    b * o.heads[seg] + h);
+        const CUtensorMap* mp = seg == 0 ? m0 : (seg == 1 ? m1 : m2);
+        if (kPairLoad) tma_load_3d_pair(dst + j * 8192, mp, bar, d, t, b * o.heads[seg] + h);
+        else tma_load_3d(dst + j * 8192, mp, bar, d, t, b * o.heads[seg] + h);
       }
     }
     bytes += 64 * kBK * 2;
@@ -144,13 +156,15 @@ __device__ __forceinline__ uint64_t operand_desc(bool mn_major, uint32_t base, i
                   : smem_desc_sw128(base + kk * 32, 16, 1024);
 }
 
-template <int BN>
-__global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
+// kPair: launched in clusters of two; p.tiles_m then counts 256-row tiles.
+template <int BN, bool kPair = false>
+__global__ void __launch_bounds__(Layout<BN, kPair>::kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                 const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB,
                 const Params p) {
   pdl_wait_and_trigger();
-  using L = Layout<BN>;
+  using L = Layout<BN, kPair>;
+  constexpr int kStages = L::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sb0 = smem_u32(smem_raw);
   if (sb0 & 1023u) {  // uniform across the CTA: nothing has been issued yet
@@ -162,16 +176,21 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sg + L::kMisc + 4);
   auto bar = [&](int i) -> uint32_t { return sb0 + L::kBars + 8u * i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = kPair ? (int)cluster_rank() : 0;
+  auto lead = [&](int i) -> uint32_t { return kPair ? map_rank(bar(i), 0) : bar(i); };
   const int nkb_total = (p.K + kBK - 1) / kBK;
   const int tiles = p.tiles_m * p.tiles_n;
   const int n_units = tiles * p.splits;
-  // Work unit u (this CTA takes u = blockIdx.x, + gridDim.x, ...): split
-  // u / tiles, then the tile, M fastest so that CTAs running at the same time
-  // share the B tile (the weights) in L2.
+  // Work unit u (this CTA, or this pair, takes u = its index, + the number
+  // of CTAs or pairs, ...): split u / tiles, then the tile, M fastest so that
+  // CTAs running at the same time share the B tile (the weights) in L2. A
+  // pair's CTA r takes rows [256 tm + 128 r, +128) of tile tm.
+  const int u_first = kPair ? (int)blockIdx.x >> 1 : (int)blockIdx.x;
+  const int u_step = kPair ? (int)gridDim.x >> 1 : (int)gridDim.x;
   auto unit = [&](int u, int& m0, int& n0, int& kb0, int& nkb) {
     const int z = u / tiles, r = u - z * tiles;
     const int tn = r / p.tiles_m;
-    m0 = (r - tn * p.tiles_m) * kBM;
+    m0 = kPair ? (r - tn * p.tiles_m) * 2 * kBM + rank * kBM : (r - tn * p.tiles_m) * kBM;
     n0 = tn * BN;
     kb0 = z * p.kb_per_split;
     nkb = min(nkb_total, kb0 + p.kb_per_split) - kb0;  // >= 1: the host sizes the split so
@@ -184,17 +203,25 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar(L::bAccFull + a), 1);
-      mbar_init(bar(L::bAccEmpty + a), 128);
+      // the epilogue threads that read the accumulator out (for a pair, one
+      // arrival per epilogue warp of either CTA, on CTA 0's barrier)
+      mbar_init(bar(L::bAccEmpty + a), kPair ? 8 : 128);
     }
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == L::kMmaWarp) {
-    tmem_alloc(sb0 + L::kMisc, L::kTmemCols);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(sb0 + L::kMisc, L::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(sb0 + L::kMisc, L::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync_all();  // both CTAs' barriers ready before cross-CTA signals
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -204,9 +231,11 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
       prefetch_tensor_map(&tmB);
       int it = 0;  // K blocks loaded so far by this CTA, over all its units
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      constexpr int BL = L::kBLocal;
+      for (int u = u_first; ok && u < n_units; u += u_step) {
         int m0, n0, kb0, nkb;
         unit(u, m0, n0, kb0, nkb);
+        const int nb = n0 + rank * BL;  // this CTA's B rows
         for (int j = 0; j < nkb; ++j, ++it) {
           const int s = it % kStages, round = it / kStages;
           if (it >= kStages && !mbar_wait(bar(L::bEmpty + s), (round - 1) & 1, abort_flag)) {
@@ -214,46 +243,65 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
             break;
           }
           const uint32_t sa = sb0 + L::kA + s * L::kABytes, sbb = sb0 + L::kB + s * L::kBBytes;
-          const uint32_t bytes =
-              operand_boxes<kBM>(false, p.a, &tmA0, &tmA1, &tmA2, p.M, p.T, p.D, m0, kb0 + j, sa,
-                                 0) +
-              operand_boxes<BN>(false, p.b, &tmB, &tmB, &tmB, p.N, p.T, p.D, n0, kb0 + j, sbb, 0);
-          mbar_arrive_expect_tx(bar(L::bFull + s), bytes);
-          operand_boxes<kBM>(true, p.a, &tmA0, &tmA1, &tmA2, p.M, p.T, p.D, m0, kb0 + j, sa,
-                             bar(L::bFull + s));
-          operand_boxes<BN>(true, p.b, &tmB, &tmB, &tmB, p.N, p.T, p.D, n0, kb0 + j, sbb,
-                            bar(L::bFull + s));
+          if (rank == 0) {
+            // CTA 0's barrier counts the bytes of both CTAs' boxes
+            uint32_t bytes = 0;
+            for (int q = 0; q < (kPair ? 2 : 1); ++q)
+              bytes += operand_boxes<kBM>(false, p.a, &tmA0, &tmA1, &tmA2, p.M, p.T, p.D,
+                                          m0 + q * kBM, kb0 + j, sa, 0) +
+                       operand_boxes<BL>(false, p.b, &tmB, &tmB, &tmB, p.N, p.T, p.D,
+                                         n0 + q * BL, kb0 + j, sbb, 0);
+            mbar_arrive_expect_tx(bar(L::bFull + s), bytes);
+          }
+          operand_boxes<kBM, kPair>(true, p.a, &tmA0, &tmA1, &tmA2, p.M, p.T, p.D, m0, kb0 + j,
+                                    sa, lead(L::bFull + s));
+          operand_boxes<BL, kPair>(true, p.b, &tmB, &tmB, &tmB, p.N, p.T, p.D, nb, kb0 + j, sbb,
+                                   lead(L::bFull + s));
         }
       }
     }
   } else if (warp == L::kMmaWarp) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_f16(kBM, BN, true, true, p.a.mn_major != 0, p.b.mn_major != 0);
+    // one instruction stream: this CTA's, or for a pair CTA 0's, whose
+    // products (M = 256) read both CTAs' tiles and write both accumulators
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc =
+          idesc_f16(kPair ? 2 * kBM : kBM, BN, true, true, p.a.mn_major != 0, p.b.mn_major != 0);
+      auto wait = [&](uint32_t b, uint32_t par) {
+        return kPair ? mbar_wait_cl(b, par, abort_flag) : mbar_wait(b, par, abort_flag);
+      };
+      auto commit = [&](uint32_t b) {
+        if constexpr (kPair) commit_pair(b);
+        else mma_commit(b);
+      };
       int it = 0, n = 0;  // K blocks consumed, units finished by this CTA
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++n) {
+      for (int u = u_first; ok && u < n_units; u += u_step, ++n) {
         int m0, n0, kb0, nkb;
         unit(u, m0, n0, kb0, nkb);
         const int a = n & 1;
         // the epilogue must have read this accumulator's previous unit out
-        if (n >= 2 && !mbar_wait(bar(L::bAccEmpty + a), ((n >> 1) - 1) & 1, abort_flag)) break;
+        if (n >= 2 && !wait(bar(L::bAccEmpty + a), ((n >> 1) - 1) & 1)) break;
         tc_fence_after();
         const uint32_t acc = tmem + a * BN;
         for (int j = 0; j < nkb; ++j, ++it) {
           const int s = it % kStages;
-          if (!mbar_wait(bar(L::bFull + s), (it / kStages) & 1, abort_flag)) {
+          if (!wait(bar(L::bFull + s), (it / kStages) & 1)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t sa = sb0 + L::kA + s * L::kABytes, sbb = sb0 + L::kB + s * L::kBBytes;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            mma_ss(acc, operand_desc(p.a.mn_major, sa, kk), operand_desc(p.b.mn_major, sbb, kk),
-                   idesc, (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(bar(L::bEmpty + s));
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t da = operand_desc(p.a.mn_major, sa, kk),
+                           db = operand_desc(p.b.mn_major, sbb, kk);
+            const uint32_t acc_on = (j > 0 || kk > 0) ? 1u : 0u;
+            if constexpr (kPair) mma_ss_pair(acc, da, db, idesc, acc_on);
+            else mma_ss(acc, da, db, idesc, acc_on);
+          }
+          commit(bar(L::bEmpty + s));
         }
-        if (ok) mma_commit(bar(L::bAccFull + a));
+        if (ok) commit(bar(L::bAccFull + a));
       }
     }
   } else {
@@ -263,7 +311,7 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)(sub * 32) << 16);
     const int T = p.T, D = p.D;
     int n = 0;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++n) {
+    for (int u = u_first; u < n_units; u += u_step, ++n) {
       int m0, n0, kb0, nkb;
       unit(u, m0, n0, kb0, nkb);
       const int a = n & 1;
@@ -284,7 +332,12 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
         if (c == nch - 1) {
           // every column of this accumulator that is used has been read
           tc_fence_before();
-          mbar_arrive(bar(L::bAccEmpty + a));
+          if constexpr (kPair) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(lead(L::bAccEmpty + a));
+          } else {
+            mbar_arrive(bar(L::bAccEmpty + a));
+          }
         }
         if (m >= p.M) continue;
         float f[32];
@@ -331,9 +384,12 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // a pair: no CTA leaves (or frees TMEM) while the other may still signal it
+  if constexpr (kPair) cluster_sync_all();
   if (warp == L::kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, L::kTmemCols);
+    if constexpr (kPair) tmem_dealloc_pair(tmem, L::kTmemCols);
+    else tmem_dealloc(tmem, L::kTmemCols);
   }
 }
 
