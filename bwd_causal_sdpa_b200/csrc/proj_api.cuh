@@ -55,19 +55,24 @@ struct GemmPlan {
   int bn, tiles_m, tiles_n, splits, kb_per_split;
   long units, ctas;
 };
-GemmPlan plan_gemm(int M, int N, int K, bool f32_out) {
+// even: the K blocks per split must be even (stages of two K blocks).
+GemmPlan plan_gemm(int M, int N, int K, bool f32_out, bool even = false) {
   using namespace proj100;
   GemmPlan g;
   g.bn = N >= 256 ? 256 : 128;
   g.tiles_m = (M + kBM - 1) / kBM;
   g.tiles_n = (N + g.bn - 1) / g.bn;
   const int nkb = (K + kBK - 1) / kBK;
-  auto rounded = [&](int s) {
+  auto per_of = [&](int s) {
     const int per = (nkb + s - 1) / s;
+    return even ? per + (per & 1) : per;
+  };
+  auto rounded = [&](int s) {
+    const int per = per_of(s);
     return (nkb + per - 1) / per;  // every split gets >= 1 block
   };
   auto cost_us = [&](int s) {
-    const int sr = rounded(s), per = (nkb + sr - 1) / sr;
+    const int sr = rounded(s), per = even ? per_of(s) : (nkb + sr - 1) / sr;
     const long units = (long)g.tiles_m * g.tiles_n * sr;
     const long rounds = (units + kProjSms - 1) / kProjSms;
     const double kb_us = 2.0 * kBM * g.bn * kBK / 11.2e6;
@@ -88,7 +93,7 @@ GemmPlan plan_gemm(int M, int N, int K, bool f32_out) {
     }
   }
   g.splits = rounded(split);
-  g.kb_per_split = (nkb + g.splits - 1) / g.splits;
+  g.kb_per_split = even ? per_of(split) : (nkb + g.splits - 1) / g.splits;
   g.units = (long)g.tiles_m * g.tiles_n * g.splits;
   g.ctas = std::min<long>(g.units, kProjSms);  // persistent: at most one CTA per SM
   return g;
@@ -99,13 +104,35 @@ GemmPlan plan_gemm(int M, int N, int K, bool f32_out) {
 // of the B tile, so every box is 128 rows high.
 int gemm_b_box_rows(int) { return 128; }
 
-// One GEMM launch: the operands' maps are built by the caller. With a K
-// split the fp32 output is zeroed first and the parts are added into it.
+// TMA box rows of an MN-major operand: its K extent per ring stage (GEMMs
+// with an MN-major operand run stages of 128 K values).
+constexpr int kMnBoxRows = 128;
+
+template <int BN, bool kPair, int KB>
+int gemm_kernel_launch(dim3 grid, const CUtensorMap& a0, const CUtensorMap& a1,
+                       const CUtensorMap& a2, const CUtensorMap& b, const proj100::Params& p,
+                       cudaStream_t st) {
+  using namespace proj100;
+  using L = Layout<BN, kPair, KB>;
+  static bool smem_done[64];
+  if (!ensure_smem(gemm_kernel<BN, kPair, KB>, L::kSmemAlloc, smem_done)) return ATTN_ECUDA;
+  if (kPair)
+    ATTN_LAUNCH(KK_GEMM, st, pdl_cluster_launch(gemm_kernel<BN, kPair, KB>, grid, L::kThreads,
+                                                L::kSmemAlloc, st, 2u, a0, a1, a2, b, p));
+  else
+    ATTN_LAUNCH(KK_GEMM, st, pdl_launch(gemm_kernel<BN, kPair, KB>, grid, L::kThreads,
+                                        L::kSmemAlloc, st, a0, a1, a2, b, p));
+  return launch_status();
+}
+
+// One GEMM launch: the operands' maps are built by the caller (an MN-major
+// operand's boxes kMnBoxRows high). With a K split the fp32 output is zeroed
+// first and the parts are added into it.
 int gemm_launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2,
                 const CUtensorMap& b, proj100::Params p, cudaStream_t st) {
   using namespace proj100;
-  static bool smem_done128[64];
-  const GemmPlan g = plan_gemm(p.M, p.N, p.K, p.epi == EPI_ROWS_F32);
+  const bool kb128 = p.a.mn_major || p.b.mn_major;
+  const GemmPlan g = plan_gemm(p.M, p.N, p.K, p.epi == EPI_ROWS_F32, kb128);
   if (g.units >= (1L << 31)) return ATTN_EUNSUPPORTED;
   p.tiles_m = g.tiles_m;
   p.tiles_n = g.tiles_n;
@@ -121,20 +148,14 @@ int gemm_launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap&
   if (g.bn == 256) {
     // measured on the two projection workloads: 15 % and 6 % faster than
     // one CTA per 128 x 256 tile (the per-SM tile loads halve for B)
-    static bool smem_done_pair[64];
-    using LP = Layout<256, true>;
     p.tiles_m = (p.M + 2 * kBM - 1) / (2 * kBM);  // 256-row tiles, one per pair
     const long units = (long)p.tiles_m * p.tiles_n * p.splits;
     const dim3 pgrid((unsigned)(2 * std::min<long>(units, kProjSms / 2)));
-    if (!ensure_smem(gemm_kernel<256, true>, LP::kSmemAlloc, smem_done_pair)) return ATTN_ECUDA;
-    ATTN_LAUNCH(KK_GEMM, st, pdl_cluster_launch(gemm_kernel<256, true>, pgrid, LP::kThreads,
-                                                LP::kSmemAlloc, st, 2u, a0, a1, a2, b, p));
-  } else {
-    if (!ensure_smem(gemm_kernel<128>, Layout<128>::kSmemAlloc, smem_done128)) return ATTN_ECUDA;
-    ATTN_LAUNCH(KK_GEMM, st, pdl_launch(gemm_kernel<128>, grid, Layout<128>::kThreads,
-                                        Layout<128>::kSmemAlloc, st, a0, a1, a2, b, p));
+    return kb128 ? gemm_kernel_launch<256, true, 128>(pgrid, a0, a1, a2, b, p, st)
+                 : gemm_kernel_launch<256, true, 64>(pgrid, a0, a1, a2, b, p, st);
   }
-  return launch_status();
+  return kb128 ? gemm_kernel_launch<128, false, 128>(grid, a0, a1, a2, b, p, st)
+               : gemm_kernel_launch<128, false, 64>(grid, a0, a1, a2, b, p, st);
 }
 
 struct ProjWs {
@@ -299,7 +320,8 @@ int attn_qkv_proj_bwd(const void* dq, const void* dk, const void* dv, const void
     CUtensorMap a0, a1, a2, mb;
     if (!make_heads_map(&a0, gq, D, T, (long)B * H, kBM) ||
         !make_heads_map(&a1, gk, D, T, (long)B * H_kv, kBM) ||
-        !make_heads_map(&a2, dv, D, T, (long)B * H_kv, kBM) || !make_rows_map(&mb, w_qkv, F, C, 64))
+        !make_heads_map(&a2, dv, D, T, (long)B * H_kv, kBM) ||
+        !make_rows_map(&mb, w_qkv, F, C, kMnBoxRows))
       return ATTN_ECUDA;
     Params p = base_params((int)BT, C, F, T, D);
     p.a = {SRC_HEADS, 0, {H, H_kv, H_kv}};
@@ -312,9 +334,10 @@ int attn_qkv_proj_bwd(const void* dq, const void* dk, const void* dv, const void
   // head, tokens along K), B = x read MN-major ([BT][C])
   {
     CUtensorMap a0, a1, a2, mb;
-    if (!make_heads_map(&a0, gq, D, T, (long)B * H, 64) ||
-        !make_heads_map(&a1, gk, D, T, (long)B * H_kv, 64) ||
-        !make_heads_map(&a2, dv, D, T, (long)B * H_kv, 64) || !make_rows_map(&mb, x, BT, C, 64))
+    if (!make_heads_map(&a0, gq, D, T, (long)B * H, kMnBoxRows) ||
+        !make_heads_map(&a1, gk, D, T, (long)B * H_kv, kMnBoxRows) ||
+        !make_heads_map(&a2, dv, D, T, (long)B * H_kv, kMnBoxRows) ||
+        !make_rows_map(&mb, x, BT, C, kMnBoxRows))
       return ATTN_ECUDA;
     Params p = base_params(F, C, (int)BT, T, D);
     p.a = {SRC_HEADS, 1, {H, H_kv, H_kv}};
@@ -359,7 +382,7 @@ int attn_out_proj_bwd(const void* dy, const void* o, const void* w_o, void* d_o,
   // d_o = dy W_o: A = dy K-major, B = W_o read MN-major ([C][HD]: HD contiguous)
   {
     CUtensorMap ma, mb;
-    if (!make_rows_map(&ma, dy, BT, C, kBM) || !make_rows_map(&mb, w_o, C, HD, 64))
+    if (!make_rows_map(&ma, dy, BT, C, kBM) || !make_rows_map(&mb, w_o, C, HD, kMnBoxRows))
       return ATTN_ECUDA;
     Params p = base_params((int)BT, HD, C, T, D);
     p.a = {SRC_ROWS, 0, {0, 0, 0}};
@@ -372,7 +395,8 @@ int attn_out_proj_bwd(const void* dy, const void* o, const void* w_o, void* d_o,
   // dW_o = dy^T o: A = dy read MN-major ([BT][C]), B = o read MN-major
   {
     CUtensorMap ma, mb;
-    if (!make_rows_map(&ma, dy, BT, C, 64) || !make_heads_map(&mb, o, D, T, (long)B * H, 64))
+    if (!make_rows_map(&ma, dy, BT, C, kMnBoxRows) ||
+        !make_heads_map(&mb, o, D, T, (long)B * H, kMnBoxRows))
       return ATTN_ECUDA;
     Params p = base_params(C, HD, (int)BT, T, D);
     p.a = {SRC_ROWS, 1, {0, 0, 0}};

@@ -35,17 +35,20 @@ namespace proj100 {
 
 using namespace sm100;
 
-constexpr int kBM = 128, kBK = 64;
+constexpr int kBM = 128, kBK = 64;  // kBK: the K block of the unit split
 
 // kPair: the CTA is one of a cluster of two that computes a 256 x BN tile
 // (this CTA's 128 rows), loading only its half of every B tile (BN / 2 rows)
 // while the pair's products (M = 256, issued by CTA 0) read both halves.
-template <int BN, bool kPair = false>
+// KB: K values per ring stage (64, or 128 = two K blocks, which lets an
+// MN-major operand arrive in boxes of 128 K rows: TMA moves 64-row boxes
+// markedly slower per byte).
+template <int BN, bool kPair = false, int KB = 64>
 struct Layout {
-  static constexpr int kStages = kPair ? 6 : 4;
   static constexpr int kBLocal = kPair ? BN / 2 : BN;  // B rows this CTA loads
-  static constexpr int kABytes = kBM * kBK * 2;
-  static constexpr int kBBytes = kBLocal * kBK * 2;
+  static constexpr int kABytes = kBM * KB * 2;
+  static constexpr int kBBytes = kBLocal * KB * 2;
+  static constexpr int kStages = 196608 / (kABytes + kBBytes) > 8 ? 8 : 196608 / (kABytes + kBBytes);
   static constexpr int kA = 0;
   static constexpr int kB = kStages * kABytes;
   static constexpr int kBars = kB + kStages * kBBytes;
@@ -100,33 +103,46 @@ __device__ __forceinline__ void split_feature(const int* heads, int D, int f, in
   d = f - h * D;
 }
 
+// One K-major box: BMN rows x the 64 K values from k0.
+template <int BMN, bool kPairLoad>
+__device__ __forceinline__ void operand_box_kmajor(bool issue, const Operand& o,
+                                                   const CUtensorMap* m0, const CUtensorMap* m1,
+                                                   const CUtensorMap* m2, int T, int D, int mn0,
+                                                   int k0, uint32_t dst, uint32_t bar) {
+  if (!issue) return;
+  if (o.src == SRC_ROWS) {
+    if (kPairLoad) tma_load_2d_pair(dst, m0, bar, k0, mn0);
+    else tma_load_2d(dst, m0, bar, k0, mn0);
+  } else {
+    int seg, h, d;
+    split_feature(o.heads, D, k0, seg, h, d);
+    const int b = mn0 / T, t = mn0 - b * T;
+    const CUtensorMap* mp = seg == 0 ? m0 : (seg == 1 ? m1 : m2);
+    if (kPairLoad) tma_load_3d_pair(dst, mp, bar, d, t, b * o.heads[seg] + h);
+    else tma_load_3d(dst, mp, bar, d, t, b * o.heads[seg] + h);
+  }
+}
+
 // Issue (or, with issue = false, only count the bytes of) the TMA boxes of
-// one operand tile: MN rows [mn0, mn0 + BMN) and K block kb, into dst.
-template <int BMN, bool kPairLoad = false>
+// one operand tile: MN rows [mn0, mn0 + BMN) and the nsub (1 or KB / 64)
+// K blocks from kb on, into dst.
+template <int BMN, int KB, bool kPairLoad = false>
 __device__ __forceinline__ uint32_t operand_boxes(bool issue, const Operand& o,
                                                   const CUtensorMap* m0, const CUtensorMap* m1,
                                                   const CUtensorMap* m2, int mn_total, int T,
-                                                  int D, int mn0, int kb, uint32_t dst,
+                                                  int D, int mn0, int kb, int nsub, uint32_t dst,
                                                   uint32_t bar) {
-  const int k0 = kb * kBK;
   if (!o.mn_major) {
-    // one box: BMN rows x 64 K values
-    if (issue) {
-      if (o.src == SRC_ROWS) {
-        if (kPairLoad) tma_load_2d_pair(dst, m0, bar, k0, mn0);
-        else tma_load_2d(dst, m0, bar, k0, mn0);
-      } else {
-        int seg, h, d;
-        split_feature(o.heads, D, k0, seg, h, d);
-        const int b = mn0 / T, t = mn0 - b * T;
-        const CUtensorMap* mp = seg == 0 ? m0 : (seg == 1 ? m1 : m2);
-        if (kPairLoad) tma_load_3d_pair(dst, mp, bar, d, t, b * o.heads[seg] + h);
-        else tma_load_3d(dst, mp, bar, d, t, b * o.heads[seg] + h);
-      }
-    }
-    return BMN * kBK * 2;
+    // per K block one box of BMN rows x 64 K values, BMN * 128 bytes apart
+    for (int sb = 0; sb < nsub; ++sb)
+      operand_box_kmajor<BMN, kPairLoad>(issue, o, m0, m1, m2, T, D, mn0, (kb + sb) * kBK,
+                                         dst + sb * BMN * 128, bar);
+    return nsub * BMN * kBK * 2;
   }
-  // MN-major: BMN / 64 boxes of 64 MN values x 64 K rows, 8 KB apart
+  // MN-major: BMN / 64 boxes of 64 MN values x KB K rows, KB * 128 bytes
+  // apart (a box reads all KB rows; those of a missing second block are
+  // never multiplied)
+  const int k0 = kb * kBK;
   uint32_t bytes = 0;
 #pragma unroll
   for (int j = 0; j < BMN / 64; ++j) {
@@ -134,37 +150,41 @@ __device__ __forceinline__ uint32_t operand_boxes(bool issue, const Operand& o,
     if (f >= mn_total) break;
     if (issue) {
       if (o.src == SRC_ROWS) {
-        if (kPairLoad) tma_load_2d_pair(dst + j * 8192, m0, bar, f, k0);
-        else tma_load_2d(dst + j * 8192, m0, bar, f, k0);
+        if (kPairLoad) tma_load_2d_pair(dst + j * KB * 128, m0, bar, f, k0);
+        else tma_load_2d(dst + j * KB * 128, m0, bar, f, k0);
       } else {
         int seg, h, d;
         split_feature(o.heads, D, f, seg, h, d);
         const int b = k0 / T, t = k0 - b * T;
         const CUtensorMap* mp = seg == 0 ? m0 : (seg == 1 ? m1 : m2);
-        if (kPairLoad) tma_load_3d_pair(dst + j * 8192, mp, bar, d, t, b * o.heads[seg] + h);
-        else tma_load_3d(dst + j * 8192, mp, bar, d, t, b * o.heads[seg] + h);
+        if (kPairLoad) tma_load_3d_pair(dst + j * KB * 128, mp, bar, d, t, b * o.heads[seg] + h);
+        else tma_load_3d(dst + j * KB * 128, mp, bar, d, t, b * o.heads[seg] + h);
       }
     }
-    bytes += 64 * kBK * 2;
+    bytes += KB * 128;
   }
   return bytes;
 }
 
-// K step kk (16 K values) of a 64-wide operand tile at base.
+// K step kk (16 K values) of an operand tile of BMN rows and KB K values.
+template <int BMN, int KB>
 __device__ __forceinline__ uint64_t operand_desc(bool mn_major, uint32_t base, int kk) {
-  return mn_major ? smem_desc_sw128(base + kk * 2048, 8192, 1024)
-                  : smem_desc_sw128(base + kk * 32, 16, 1024);
+  return mn_major ? smem_desc_sw128(base + kk * 2048, KB * 128, 1024)
+                  : smem_desc_sw128(base + (kk >> 2) * (BMN * 128) + (kk & 3) * 32, 16, 1024);
 }
 
 // kPair: launched in clusters of two; p.tiles_m then counts 256-row tiles.
-template <int BN, bool kPair = false>
-__global__ void __launch_bounds__(Layout<BN, kPair>::kThreads, 1)
+// KB = 128: p.kb_per_split is even (a stage never straddles two units' K
+// ranges); only the last stage of K may hold one K block.
+template <int BN, bool kPair = false, int KB = 64>
+__global__ void __launch_bounds__(Layout<BN, kPair, KB>::kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                 const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB,
                 const Params p) {
   pdl_wait_and_trigger();
-  using L = Layout<BN, kPair>;
+  using L = Layout<BN, kPair, KB>;
   constexpr int kStages = L::kStages;
+  constexpr int kSub = KB / kBK;  // K blocks per stage
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sb0 = smem_u32(smem_raw);
   if (sb0 & 1023u) {  // uniform across the CTA: nothing has been issued yet
@@ -229,14 +249,15 @@ __global__ void __launch_bounds__(Layout<BN, kPair>::kThreads, 1)
     if (lane == 0) {
       prefetch_tensor_map(&tmA0);
       prefetch_tensor_map(&tmB);
-      int it = 0;  // K blocks loaded so far by this CTA, over all its units
+      int it = 0;  // stages loaded so far by this CTA, over all its units
       bool ok = true;
       constexpr int BL = L::kBLocal;
       for (int u = u_first; ok && u < n_units; u += u_step) {
         int m0, n0, kb0, nkb;
         unit(u, m0, n0, kb0, nkb);
         const int nb = n0 + rank * BL;  // this CTA's B rows
-        for (int j = 0; j < nkb; ++j, ++it) {
+        for (int jb = 0; jb < nkb; jb += kSub, ++it) {
+          const int ns = min(kSub, nkb - jb);  // K blocks in this stage
           const int s = it % kStages, round = it / kStages;
           if (it >= kStages && !mbar_wait(bar(L::bEmpty + s), (round - 1) & 1, abort_flag)) {
             ok = false;
@@ -247,16 +268,16 @@ __global__ void __launch_bounds__(Layout<BN, kPair>::kThreads, 1)
             // CTA 0's barrier counts the bytes of both CTAs' boxes
             uint32_t bytes = 0;
             for (int q = 0; q < (kPair ? 2 : 1); ++q)
-              bytes += operand_boxes<kBM>(false, p.a, &tmA0, &tmA1, &tmA2, p.M, p.T, p.D,
-                                          m0 + q * kBM, kb0 + j, sa, 0) +
-                       operand_boxes<BL>(false, p.b, &tmB, &tmB, &tmB, p.N, p.T, p.D,
-                                         n0 + q * BL, kb0 + j, sbb, 0);
+              bytes += operand_boxes<kBM, KB>(false, p.a, &tmA0, &tmA1, &tmA2, p.M, p.T, p.D,
+                                              m0 + q * kBM, kb0 + jb, ns, sa, 0) +
+                       operand_boxes<BL, KB>(false, p.b, &tmB, &tmB, &tmB, p.N, p.T, p.D,
+                                             n0 + q * BL, kb0 + jb, ns, sbb, 0);
             mbar_arrive_expect_tx(bar(L::bFull + s), bytes);
           }
-          operand_boxes<kBM, kPair>(true, p.a, &tmA0, &tmA1, &tmA2, p.M, p.T, p.D, m0, kb0 + j,
-                                    sa, lead(L::bFull + s));
-          operand_boxes<BL, kPair>(true, p.b, &tmB, &tmB, &tmB, p.N, p.T, p.D, nb, kb0 + j, sbb,
-                                   lead(L::bFull + s));
+          operand_boxes<kBM, KB, kPair>(true, p.a, &tmA0, &tmA1, &tmA2, p.M, p.T, p.D, m0,
+                                        kb0 + jb, ns, sa, lead(L::bFull + s));
+          operand_boxes<BL, KB, kPair>(true, p.b, &tmB, &tmB, &tmB, p.N, p.T, p.D, nb, kb0 + jb,
+                                       ns, sbb, lead(L::bFull + s));
         }
       }
     }
@@ -273,7 +294,7 @@ __global__ void __launch_bounds__(Layout<BN, kPair>::kThreads, 1)
         if constexpr (kPair) commit_pair(b);
         else mma_commit(b);
       };
-      int it = 0, n = 0;  // K blocks consumed, units finished by this CTA
+      int it = 0, n = 0;  // stages consumed, units finished by this CTA
       bool ok = true;
       for (int u = u_first; ok && u < n_units; u += u_step, ++n) {
         int m0, n0, kb0, nkb;
@@ -283,7 +304,7 @@ __global__ void __launch_bounds__(Layout<BN, kPair>::kThreads, 1)
         if (n >= 2 && !wait(bar(L::bAccEmpty + a), ((n >> 1) - 1) & 1)) break;
         tc_fence_after();
         const uint32_t acc = tmem + a * BN;
-        for (int j = 0; j < nkb; ++j, ++it) {
+        for (int jb = 0; jb < nkb; jb += kSub, ++it) {
           const int s = it % kStages;
           if (!wait(bar(L::bFull + s), (it / kStages) & 1)) {
             ok = false;
@@ -291,11 +312,13 @@ __global__ void __launch_bounds__(Layout<BN, kPair>::kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sa = sb0 + L::kA + s * L::kABytes, sbb = sb0 + L::kB + s * L::kBBytes;
+          const int nk = (kSub == 1 || jb + kSub <= nkb) ? KB / 16 : (nkb - jb) * (kBK / 16);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t da = operand_desc(p.a.mn_major, sa, kk),
-                           db = operand_desc(p.b.mn_major, sbb, kk);
-            const uint32_t acc_on = (j > 0 || kk > 0) ? 1u : 0u;
+          for (int kk = 0; kk < KB / 16; ++kk) {
+            if (kk >= nk) break;
+            const uint64_t da = operand_desc<kBM, KB>(p.a.mn_major, sa, kk),
+                           db = operand_desc<L::kBLocal, KB>(p.b.mn_major, sbb, kk);
+            const uint32_t acc_on = (jb > 0 || kk > 0) ? 1u : 0u;
             if constexpr (kPair) mma_ss_pair(acc, da, db, idesc, acc_on);
             else mma_ss(acc, da, db, idesc, acc_on);
           }
