@@ -55,8 +55,8 @@ struct GemmPlan {
   int bn, tiles_m, tiles_n, splits, kb_per_split;
   long units, ctas;
 };
-// even: the K blocks per split must be even (stages of two K blocks).
-GemmPlan plan_gemm(int M, int N, int K, bool f32_out, bool even = false) {
+// The K blocks per split are even: the kernel's ring stages hold two.
+GemmPlan plan_gemm(int M, int N, int K, bool f32_out) {
   using namespace proj100;
   GemmPlan g;
   g.bn = N >= 256 ? 256 : 128;
@@ -65,14 +65,14 @@ GemmPlan plan_gemm(int M, int N, int K, bool f32_out, bool even = false) {
   const int nkb = (K + kBK - 1) / kBK;
   auto per_of = [&](int s) {
     const int per = (nkb + s - 1) / s;
-    return even ? per + (per & 1) : per;
+    return per + (per & 1);
   };
   auto rounded = [&](int s) {
     const int per = per_of(s);
     return (nkb + per - 1) / per;  // every split gets >= 1 block
   };
   auto cost_us = [&](int s) {
-    const int sr = rounded(s), per = even ? per_of(s) : (nkb + sr - 1) / sr;
+    const int sr = rounded(s), per = per_of(s);
     const long units = (long)g.tiles_m * g.tiles_n * sr;
     const long rounds = (units + kProjSms - 1) / kProjSms;
     const double kb_us = 2.0 * kBM * g.bn * kBK / 11.2e6;
@@ -93,7 +93,7 @@ GemmPlan plan_gemm(int M, int N, int K, bool f32_out, bool even = false) {
     }
   }
   g.splits = rounded(split);
-  g.kb_per_split = even ? per_of(split) : (nkb + g.splits - 1) / g.splits;
+  g.kb_per_split = per_of(split);
   g.units = (long)g.tiles_m * g.tiles_n * g.splits;
   g.ctas = std::min<long>(g.units, kProjSms);  // persistent: at most one CTA per SM
   return g;
@@ -104,8 +104,7 @@ GemmPlan plan_gemm(int M, int N, int K, bool f32_out, bool even = false) {
 // of the B tile, so every box is 128 rows high.
 int gemm_b_box_rows(int) { return 128; }
 
-// TMA box rows of an MN-major operand: its K extent per ring stage (GEMMs
-// with an MN-major operand run stages of 128 K values).
+// TMA box rows of an MN-major operand: its K extent per ring stage.
 constexpr int kMnBoxRows = 128;
 
 template <int BN, bool kPair, int KB>
@@ -131,8 +130,7 @@ int gemm_kernel_launch(dim3 grid, const CUtensorMap& a0, const CUtensorMap& a1,
 int gemm_launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2,
                 const CUtensorMap& b, proj100::Params p, cudaStream_t st) {
   using namespace proj100;
-  const bool kb128 = p.a.mn_major || p.b.mn_major;
-  const GemmPlan g = plan_gemm(p.M, p.N, p.K, p.epi == EPI_ROWS_F32, kb128);
+  const GemmPlan g = plan_gemm(p.M, p.N, p.K, p.epi == EPI_ROWS_F32);
   if (g.units >= (1L << 31)) return ATTN_EUNSUPPORTED;
   p.tiles_m = g.tiles_m;
   p.tiles_n = g.tiles_n;
@@ -151,11 +149,9 @@ int gemm_launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap&
     p.tiles_m = (p.M + 2 * kBM - 1) / (2 * kBM);  // 256-row tiles, one per pair
     const long units = (long)p.tiles_m * p.tiles_n * p.splits;
     const dim3 pgrid((unsigned)(2 * std::min<long>(units, kProjSms / 2)));
-    return kb128 ? gemm_kernel_launch<256, true, 128>(pgrid, a0, a1, a2, b, p, st)
-                 : gemm_kernel_launch<256, true, 64>(pgrid, a0, a1, a2, b, p, st);
+    return gemm_kernel_launch<256, true, 128>(pgrid, a0, a1, a2, b, p, st);
   }
-  return kb128 ? gemm_kernel_launch<128, false, 128>(grid, a0, a1, a2, b, p, st)
-               : gemm_kernel_launch<128, false, 64>(grid, a0, a1, a2, b, p, st);
+  return gemm_kernel_launch<128, false, 128>(grid, a0, a1, a2, b, p, st);
 }
 
 struct ProjWs {

@@ -20,8 +20,8 @@
 // tiles run on clusters of two CTAs instead: a unit is a 256 x 256 tile, each
 // CTA loads its 128 rows of A and half of the B tile, and CTA 0 issues
 // products of M = 256 (cta_group::2) that read both CTAs' tiles and write
-// both CTAs' accumulators. K moves in 64-wide blocks through a ring (four
-// stages, six for a pair) that runs across units; the accumulator alternates
+// both CTAs' accumulators. K moves through a three-stage ring of 128-wide
+// stages (two K blocks of 64) that runs across units; the accumulator alternates
 // between two TMEM buffers, so the epilogue of one unit overlaps the main
 // loop of the next. Warps: TMA, MMA (one elected thread issues tcgen05.mma)
 // and four epilogue warps (thread = TMEM lane = output row).
@@ -42,8 +42,8 @@ constexpr int kBM = 128, kBK = 64;  // kBK: the K block of the unit split
 // while the pair's products (M = 256, issued by CTA 0) read both halves.
 // KB: K values per ring stage (64, or 128 = two K blocks, which lets an
 // MN-major operand arrive in boxes of 128 K rows: TMA moves 64-row boxes
-// markedly slower per byte).
-template <int BN, bool kPair = false, int KB = 64>
+// markedly slower per byte; K-major GEMMs gain a few per cent too).
+template <int BN, bool kPair = false, int KB = 128>
 struct Layout {
   static constexpr int kBLocal = kPair ? BN / 2 : BN;  // B rows this CTA loads
   static constexpr int kABytes = kBM * KB * 2;
@@ -176,7 +176,7 @@ __device__ __forceinline__ uint64_t operand_desc(bool mn_major, uint32_t base, i
 // kPair: launched in clusters of two; p.tiles_m then counts 256-row tiles.
 // KB = 128: p.kb_per_split is even (a stage never straddles two units' K
 // ranges); only the last stage of K may hold one K block.
-template <int BN, bool kPair = false, int KB = 64>
+template <int BN, bool kPair = false, int KB = 128>
 __global__ void __launch_bounds__(Layout<BN, kPair, KB>::kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                 const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB,

@@ -272,9 +272,9 @@ def test_projection_gemm_plan():
     assert p["kb_per_split"] == 32
     assert plan(8192, 200, 768, False)["bn"] == 128
     # fp32 weight gradients of the 8K layer: 192 tiles fill 1.3 rounds of 148
-    # SMs; three K parts make 576 units (97 % of four rounds)
+    # SMs; two K parts of 64 blocks make 384 units
     p = plan(3072, 2048, 8192, True)
-    assert (p["splits"], p["kb_per_split"], p["ctas"]) == (3, 43, 148)
+    assert (p["splits"], p["kb_per_split"], p["ctas"]) == (2, 64, 148)
     # 128 tiles: the extra reduce traffic of a split costs more than it saves
     assert plan(2048, 2048, 8192, True)["splits"] == 1
     # few tiles with a long K (the 237M layer's weights): split
@@ -287,6 +287,7 @@ def test_projection_gemm_plan():
         nkb = -(-K // 64)
         assert 1 <= p["splits"] <= nkb and (p["splits"] - 1) * p["kb_per_split"] < nkb
         assert p["splits"] * p["kb_per_split"] >= nkb
+        assert p["kb_per_split"] % 2 == 0  # the kernel's stages hold two K blocks
     assert A.attn_proj_gemm_plan(0, 8, 8, True)[0] == A.ATTN_EINVAL
 
 
