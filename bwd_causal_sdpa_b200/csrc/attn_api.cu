@@ -764,34 +764,34 @@ int attn_profile_read(int kind, const char** name, int* launches, double* total_
 // ---------------------------------------------------------------------------
 namespace {
 
-// Workspace: per (query head, cache chunk of kDecodeChunk tokens) the
-// unnormalised partial sum (f32 [B*H][n_split][D]), then its max and sum of
-// exponentials (f32 [B*H][n_split] each).
+// bf16 caches with up to 16 query heads per cached head take the streaming
+// tensor-core kernel: kDecodeStreamCtas CTAs (one per SM) over equal spans
+// of all cached tokens. Workspace: partial slots (f32 [slots][16][D], then
+// f32 [slots][16][2] max and sum), slots = kDecodeStreamCtas + B*H_kv, and
+// one int32 count per cached head.
+// The rest take one 64-token chunk per CTA. Workspace: per (query head,
+// chunk) the unnormalised partial sum (f32 [B*H][n_split][D]), then its max
+// and sum of exponentials (f32 [B*H][n_split] each).
 struct DecodePlan {
-  size_t o_part = 0, m_part = 0, l_part = 0, total = 0;
+  size_t o_part = 0, m_part = 0, l_part = 0, cnt = 0, total = 0;
   int n_split = 0, per_split = 0;
 };
 
-// bf16 caches with up to 16 query heads per cached head take the streaming
-// tensor-core kernel (cache ranges sized for about sixteen CTAs per SM over
-// the whole grid, measured best with a two-deep pipeline); the rest
-// take one 64-token chunk per CTA.
 bool decode_streams(int H, int H_kv, int dtype) { return dtype == ATTN_BF16 && H / H_kv <= 16; }
-constexpr long kDecodeStreamCtas = 16 * 148;
+constexpr int kDecodeStreamCtas = 148;
 
 DecodePlan decode_plan(int B, int H, int H_kv, int T_max, int D, int dtype) {
   DecodePlan p;
   if (decode_streams(H, H_kv, dtype)) {
-    const long stages = (T_max + kDecodePipeKeys - 1) / kDecodePipeKeys;
-    long want = (kDecodeStreamCtas + (long)B * H_kv - 1) / ((long)B * H_kv);
-    want = want < 1 ? 1 : (want > stages ? stages : want);
-    const long per = (stages + want - 1) / want;  // stages per range
-    p.per_split = (int)(per * kDecodePipeKeys);
-    p.n_split = (int)((stages + per - 1) / per);
-  } else {
-    p.per_split = kDecodeChunk;
-    p.n_split = (T_max + kDecodeChunk - 1) / kDecodeChunk;
+    const size_t slots = (size_t)kDecodeStreamCtas + (size_t)B * H_kv;
+    p.o_part = 0;
+    p.m_part = round_up(slots * 16 * D * sizeof(float));  // (max, sum) pairs
+    p.cnt = p.m_part + round_up(slots * 16 * 2 * sizeof(float));
+    p.total = p.cnt + round_up((size_t)B * H_kv * sizeof(int));
+    return p;
   }
+  p.per_split = kDecodeChunk;
+  p.n_split = (T_max + kDecodeChunk - 1) / kDecodeChunk;
   const size_t slots = (size_t)B * H * p.n_split;
   p.o_part = 0;
   p.m_part = round_up(slots * D * sizeof(float));
@@ -822,19 +822,28 @@ int decode_launch(const void* q, const void* k, const void* v, const int32_t* le
   float* lp = (float*)(ws + dp.l_part);
   const int G = H / H_kv;
   if (std::is_same<TIO, __nv_bfloat16>::value && G <= 16) {
-    // streaming tensor-core variant (up to 16 query heads per cached head)
-    static bool pipe_smem_set[64] = {};
-    if (!ensure_smem(decode_pipe_kernel<D>, DecodePipeLayout<D>::kBytes, pipe_smem_set))
+    // streaming tensor-core variant (up to 16 query heads per cached head):
+    // one launch, the heads split over CTAs merged by their last CTA
+    using SL = DecStreamLayout<D>;
+    static bool stream_smem_set[2][64] = {};
+    auto kern = G <= 8 ? decode_stream_kernel<D, 1> : decode_stream_kernel<D, 2>;
+    if (!ensure_smem(kern, SL::kAlloc, stream_smem_set[G <= 8 ? 0 : 1])) return ATTN_ECUDA;
+    CUtensorMap mk, mv;
+    if (!make_tile_map(&mk, k, false, D, T_max, B * H_kv, kDecKeys) ||
+        !make_tile_map(&mv, v, false, D, T_max, B * H_kv, kDecKeys))
       return ATTN_ECUDA;
-    ATTN_LAUNCH(KK_DECODE, st, pdl_launch(decode_pipe_kernel<D>, dim3(dp.n_split, B * H_kv), kDecodeMmaThreads,
-                                        DecodePipeLayout<D>::kBytes, st, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-                    lens, rc, rs, op, mp, lp, H, H_kv, T_max, dp.n_split, dp.per_split,
-                    scale * 1.4426950408889634f));
-  } else {
-    ATTN_LAUNCH(KK_DECODE, st, pdl_launch(decode_split_kernel<TIO, D>, dim3(dp.n_split, B * H_kv), kDecodeThreads,
-                                              L::bytes(G), st, (const TIO*)q, (const TIO*)k, (const TIO*)v, lens, rc, rs, op, mp, lp, H,
-                    H_kv, T_max, dp.n_split, dp.per_split, scale * 1.4426950408889634f));
+    int* cnt = (int*)(ws + dp.cnt);
+    if (cudaMemsetAsync(cnt, 0, (size_t)B * H_kv * sizeof(int), st) != cudaSuccess)
+      return ATTN_ECUDA;
+    ATTN_LAUNCH(KK_DECODE, st, pdl_launch(kern, kDecodeStreamCtas, kDecThreads,
+                                          SL::kAlloc, st, mk, mv, (const __nv_bfloat16*)q, lens,
+                                          rc, rs, (__nv_bfloat16*)o, lse, op, mp, cnt, B, H,
+                                          H_kv, T_max, scale * 1.4426950408889634f));
+    return launch_status();
   }
+  ATTN_LAUNCH(KK_DECODE, st, pdl_launch(decode_split_kernel<TIO, D>, dim3(dp.n_split, B * H_kv), kDecodeThreads,
+                                        L::bytes(G), st, (const TIO*)q, (const TIO*)k, (const TIO*)v, lens, rc, rs, op, mp, lp, H,
+                                        H_kv, T_max, dp.n_split, dp.per_split, scale * 1.4426950408889634f));
   if (launch_status()) return ATTN_ECUDA;
   ATTN_LAUNCH(KK_DECODE_COMBINE, st, pdl_launch(decode_combine_kernel<TIO, D>, B * H, kDecodeCombineThreads,
                                               dp.n_split * sizeof(float), st, op, mp, lp, lens, (TIO*)o, lse, H, T_max, dp.n_split, dp.per_split));

@@ -196,7 +196,10 @@ int attn_bwd_saved(const void* q, const void* k, const void* v, const void* o,
  *      cache_lens[b] tokens at positions 0 .. cache_lens[b]-1, the new
  *      token's own key and value included; keys are stored already rotated
  *      by their positions (as attn_fwd rotates k); rows past cache_lens[b]
- *      are never read;
+ *      never affect the result (their values may be anything, NaN
+ *      included: a tile load may fetch some of them, and they are masked
+ *      and zeroed before use; no byte past the [B, H_kv, T_max, D] arrays is
+ *      read);
  *      cache_lens [B] int32 device array, each in [1, T_max] (a value out of
  *      range is clamped into it and the status word reports
  *      ATTN_EDEVICE_INPUT);
@@ -206,7 +209,9 @@ int attn_bwd_saved(const void* q, const void* k, const void* v, const void* o,
  *      most 64 query heads per key/value head; B * H_kv <= 65535.
  * Out: o [B, H, D] (dtype) = softmax_j(scale * q_r . k_j) v_j over the
  *      cached tokens; lse [B, H] f32, natural log.
- * Workspace: attn_decode_workspace_bytes(B, H, H_kv, T_max, D, dtype) bytes.
+ * Workspace: attn_decode_workspace_bytes(B, H, H_kv, T_max, D, dtype) bytes;
+ *      the call clears what it needs of it on `stream` (no initial contents
+ *      are assumed).
  * Alignment, ownership, asynchrony and return codes as for attn_fwd.
  */
 int attn_decode(const void* q, const void* k_cache, const void* v_cache,

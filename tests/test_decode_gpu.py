@@ -3,7 +3,11 @@ through the C ABI, against the float64 decode oracle: small cases element by
 element (both storage types and head sizes, group sizes 1 to 32, cache
 lengths 1, ragged, a multiple of the 128-token chunk and the full capacity),
 the two named decode workloads on sampled heads, cache rows past the length
-never read, and out-of-range lengths reported and clamped."""
+(set to NaN) without effect on the result, and out-of-range lengths reported
+and clamped. The streaming kernel splits the cached tokens of all heads into
+one equal span per CTA, so the small cases put each head over several CTAs
+(partials merged by the head's last CTA) and the full-size ones mix heads
+held whole with split ones."""
 
 import numpy as np
 import pytest
@@ -56,6 +60,11 @@ SMALL = [
     ("decode_237m", dict(B=2, H=2, H_kv=1, T_max=200, len_min=1, seed=37, dtype="f32")),
     # 32 query heads per cached head: bf16 beyond the tensor-core variant's 16 rows
     ("decode_8k_gqa", dict(B=2, H=32, H_kv=1, T_max=300, len_min=1, seed=41)),
+    # 12 and 16 query heads per cached head: two 8-head column tiles
+    ("decode_8k_gqa", dict(B=2, H=24, H_kv=2, T_max=700, len_min=1, seed=42)),
+    ("decode_237m", dict(B=3, H=16, H_kv=1, T_max=400, len_min=200, seed=43)),
+    # fewer cached tokens than CTAs: most spans are empty, heads split finely
+    ("decode_8k_gqa", dict(B=1, H=4, H_kv=1, T_max=64, len_min=1, seed=44)),
 ]
 
 
