@@ -101,7 +101,7 @@ WsPlan plan(int B, int H, int T, int D, int dtype, int is_bwd, int Hkv = 0) {
 // attn_bwd_saved): rotated q, k as fp16 and their inverse tile factors, in the
 // layout rope_prep writes them.
 struct SavedPlan {
-  size_t q16 = 0, k16 = 0, qfac = 0, kfac = 0, total = 0;
+  size_t q16 = 0, k16 = 0, qfac = 0, kfac = 0, docs = 0, total = 0;
 };
 
 SavedPlan saved_plan(int B, int H, int Hkv, int T, int D) {
@@ -112,6 +112,8 @@ SavedPlan saved_plan(int B, int H, int Hkv, int T, int D) {
   p.k16 = off;  off += round_up((size_t)B * Hkv * T * D * 2);
   p.qfac = off; off += round_up((size_t)B * H * nt * 4 * sizeof(float));
   p.kfac = off; off += round_up((size_t)B * Hkv * nt * sizeof(float));
+  // per-token document start and end (int32 [B*T] each), with cu_seqlens
+  p.docs = off; off += round_up((size_t)2 * B * T * sizeof(int32_t));
   p.total = off;
   return p;
 }
@@ -238,20 +240,16 @@ int bwd_simt(const void* q, const void* k, const void* v, const void* o, const v
   return launch_status();
 }
 
-// The RoPE pre-pass over q and k (see prep.cuh): one block per tile, batch and
-// group of heads, the tile's table rows staged in dynamic shared memory.
+// The RoPE pre-pass over q and k (see prep.cuh): one block per tile, batch
+// and head.
 template <int D>
 int launch_rope_prep(const void* q, const void* k, const float* rc, const float* rs,
                      const int32_t* ds, __half* qo, __half* ko, float* qf, float* kf, float* hstat,
                      int B, int H, int Hkv, int T, int nt, cudaStream_t st) {
-  static bool smem_set[64] = {};
-  constexpr int smem = rope_prep_smem_bytes<D>();
-  if (!ensure_smem(rope_prep_kernel<D>, smem, smem_set)) return ATTN_ECUDA;
-  const int group = rope_prep_group(B, H, Hkv, nt);
-  const dim3 grid(nt, B, (H + Hkv + group - 1) / group);
-  ATTN_LAUNCH(KK_ROPE_PREP, st, pdl_launch(rope_prep_kernel<D>, grid, kRopePrepThreads, smem, st,
+  const dim3 grid(nt, B, H + Hkv);
+  ATTN_LAUNCH(KK_ROPE_PREP, st, pdl_launch(rope_prep_kernel<D>, grid, kRopePrepThreads, 0, st,
                                            (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, rc, rs,
-                                           ds, qo, ko, qf, kf, hstat, B, H, Hkv, T, nt, group));
+                                           ds, qo, ko, qf, kf, hstat, B, H, Hkv, T, nt));
   return launch_status();
 }
 
@@ -551,11 +549,19 @@ int fwd_impl(const void* q, const void* k, const void* v, const float* rope_cos,
   cudaStream_t st = (cudaStream_t)stream;
   const WsPlan p = plan(B, H, T, D, dtype, 0);
   char* ws = (char*)workspace;
+  char* sv = (dtype == ATTN_BF16 && rope_cos && saved) ? (char*)saved : nullptr;
   int32_t* ds = nullptr;
   if (cu_seqlens) {
-    ds = (int32_t*)(ws + p.doc_start);
-    ATTN_LAUNCH(KK_DOC_RANGES, st, pdl_launch(doc_ranges_kernel, 1, 1024, 0, st, cu_seqlens, B, T, ds,
-                                                      (int32_t*)(ws + p.doc_end)));
+    // kept with the saved operands when there are any: the backward reuses them
+    int32_t* de;
+    if (sv) {
+      ds = (int32_t*)(sv + saved_plan(B, H, H_kv, T, D).docs);
+      de = ds + (size_t)B * T;
+    } else {
+      ds = (int32_t*)(ws + p.doc_start);
+      de = (int32_t*)(ws + p.doc_end);
+    }
+    ATTN_LAUNCH(KK_DOC_RANGES, st, pdl_launch(doc_ranges_kernel, 1, 1024, 0, st, cu_seqlens, B, T, ds, de));
     if (launch_status()) return ATTN_ECUDA;
   }
   if (dtype == ATTN_F32) {
@@ -564,7 +570,6 @@ int fwd_impl(const void* q, const void* k, const void* v, const float* rope_cos,
                    : fwd_simt<float, 128>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, H_kv, T,
                                           scale, st);
   }
-  char* sv = (rope_cos && saved) ? (char*)saved : nullptr;
   return D == 64 ? fwd_tc<64>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, H_kv, T, scale, ws,
                               p, sv, st)
                  : fwd_tc<128>(q, k, v, rope_cos, rope_sin, ds, o, lse, B, H, H_kv, T, scale, ws,
@@ -646,8 +651,13 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   cudaStream_t st = (cudaStream_t)stream;
   const WsPlan p = plan(B, H, T, D, dtype, 1, H_kv);
   char* ws = (char*)workspace;
+  const char* sv = (dtype == ATTN_BF16 && rope_cos && saved) ? (const char*)saved : nullptr;
   int32_t *ds = nullptr, *de = nullptr;
-  if (cu_seqlens) {
+  if (cu_seqlens && sv) {
+    // the forward left them with the saved operands
+    ds = (int32_t*)(sv + saved_plan(B, H, H_kv, T, D).docs);
+    de = ds + (size_t)B * T;
+  } else if (cu_seqlens) {
     ds = (int32_t*)(ws + p.doc_start);
     de = (int32_t*)(ws + p.doc_end);
     ATTN_LAUNCH(KK_DOC_RANGES, st, pdl_launch(doc_ranges_kernel, 1, 1024, 0, st, cu_seqlens, B, T, ds, de));
@@ -660,7 +670,6 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
                    : bwd_simt<float, 128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, delta,
                                           dq, dk, dv, B, H, H_kv, T, scale, st);
   }
-  const char* sv = (rope_cos && saved) ? (const char*)saved : nullptr;
   return D == 64 ? bwd_tc<64>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, dq, dk, dv, B, H,
                               H_kv, T, scale, ws, p, sv, st)
                  : bwd_tc<128>(q, k, v, o, dO, lse, rope_cos, rope_sin, ds, de, dq, dk, dv, B, H,

@@ -86,8 +86,11 @@ __global__ void __launch_bounds__(256) delta_kernel(const TIO* __restrict__ o, c
 
 // RoPE pre-pass: rotate q and k once (fp32 arithmetic, interleaved pairs at
 // the token's document position) and store every 128-row tile as fp16 times
-// its power-of-two factor (fp16_tile_factor of the tile's largest rotated
-// magnitude). qfac receives the inverse factor of each q tile as a 16-byte
+// a power-of-two factor, fp16_tile_factor of the largest pair norm
+// sqrt(x_2m^2 + x_2m+1^2) in the tile: a rotation keeps each pair's norm, so
+// that bounds every rotated value (and is at most sqrt(2) times the largest
+// of them), and it needs no table, so the factor is known before any
+// rotation. qfac receives the inverse factor of each q tile as a 16-byte
 // record (value first, so the backward's main kernel can bulk-load it with
 // the tile), kfac that of each k tile; the forward folds them into its score
 // scale and the backward's main kernel into its own, which therefore
@@ -95,18 +98,12 @@ __global__ void __launch_bounds__(256) delta_kernel(const TIO* __restrict__ o, c
 // only, else null): zeroed here (all B*H*4 slots, by the first block) for the
 // row pass that follows, which fills it with atomic maxima.
 //
-// One block per (128-row tile, batch, group of heads): the tile's cos/sin
-// rows (indexed by document position) are staged in shared memory once and
-// serve every q and k head of the group, so the tables cost one read per
-// tile and group instead of one per head; heads run one after another, each
-// thread issuing all of its loads for a head before using any. Heads are
-// numbered q heads first (0 .. H-1), then k heads (H .. H+Hkv-1).
+// One block per (128-row tile, batch, head), heads numbered q heads first
+// (0 .. H-1), then k heads (H .. H+Hkv-1): each thread loads its chunks of
+// the tile, the block reduces the largest pair norm, and each thread rotates
+// its chunks (table rows from L2) and stores them scaled. Small blocks with
+// few registers and no shared tables keep many tiles in flight per SM.
 constexpr int kRopePrepThreads = 256;
-
-template <int D>
-constexpr int rope_prep_smem_bytes() {
-  return 2 * 128 * (D / 8) * 16;  // cos and sin rows of one tile as float4
-}
 
 template <int D>
 __global__ void __launch_bounds__(kRopePrepThreads) rope_prep_kernel(
@@ -114,96 +111,65 @@ __global__ void __launch_bounds__(kRopePrepThreads) rope_prep_kernel(
     const float* __restrict__ rc, const float* __restrict__ rs,
     const int32_t* __restrict__ doc_start, __half* __restrict__ qo, __half* __restrict__ ko,
     float* __restrict__ qfac, float* __restrict__ kfac, float* __restrict__ hstat, int B, int H,
-    int Hkv, int T, int ntiles, int group) {
+    int Hkv, int T, int ntiles) {
   pdl_wait_and_trigger();
   constexpr int CH = D / 8;                        // 16-byte chunks per row
   constexpr int NT = kRopePrepThreads;
-  constexpr int PER = 128 * CH / NT;               // chunks per thread and head
-  constexpr int P4 = D / 8;                        // float4 per table row (D/2 floats)
-  extern __shared__ float4 tab[];                  // [cos | sin][128 rows][P4]
-  __shared__ float red[2][NT / 32];                // per-head maxima, double-buffered
-  const int tile = blockIdx.x, b = blockIdx.y;
-  const int HT = H + Hkv, h_first = blockIdx.z * group, h_end = min(HT, h_first + group);
+  constexpr int PER = 128 * CH / NT;               // chunks per thread
+  __shared__ float red[NT / 32];
+  const int tile = blockIdx.x, b = blockIdx.y, hh = blockIdx.z;
   const int row0 = b * T, t0 = tile * 128;
-  if (hstat && tile == 0 && b == 0 && blockIdx.z == 0)
+  if (hstat && tile == 0 && b == 0 && hh == 0)
     for (int e = threadIdx.x; e < 4 * B * H; e += NT) hstat[e] = 0.f;
-  const float4* rc4 = reinterpret_cast<const float4*>(rc);
-  const float4* rs4 = reinterpret_cast<const float4*>(rs);
-  for (int e = threadIdx.x; e < 128 * P4; e += NT) {
-    const int r = e / P4, c = e - r * P4, t = t0 + r;
-    float4 cv = make_float4(0.f, 0.f, 0.f, 0.f), sv = cv;
-    if (t < T) {
-      const int pos = t - (doc_start ? doc_start[row0 + t] - row0 : 0);
-      cv = rc4[(size_t)pos * P4 + c];
-      sv = rs4[(size_t)pos * P4 + c];
-    }
-    tab[e] = cv;
-    tab[128 * P4 + e] = sv;
+  const bool is_k = hh >= H;
+  const int bh = is_k ? b * Hkv + (hh - H) : b * H + hh;
+  const __nv_bfloat16* src = (is_k ? k : q) + (size_t)bh * T * D;
+  __half* dst = (is_k ? ko : qo) + (size_t)bh * T * D;
+  const int c8 = threadIdx.x % CH;  // this thread's chunk column, rows threadIdx.x / CH + u * NT / CH
+  uint4 raw[PER];
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int t = t0 + (threadIdx.x + u * NT) / CH;
+    raw[u] = t < T ? *reinterpret_cast<const uint4*>(src + (size_t)t * D + c8 * 8)
+                   : make_uint4(0u, 0u, 0u, 0u);  // rows past T are zeros and stay zero
   }
+  float n2 = 0.f;
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float x0 = __low2float(hv[e]), x1 = __high2float(hv[e]);
+      n2 = fmaxf(n2, fmaf(x0, x0, x1 * x1));
+    }
+  }
+  n2 = warp_max(n2);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = n2;
   __syncthreads();
-  for (int hh = h_first; hh < h_end; ++hh) {
-    const bool is_k = hh >= H;
-    const int bh = is_k ? b * Hkv + (hh - H) : b * H + hh;
-    const __nv_bfloat16* src = (is_k ? k : q) + (size_t)bh * T * D;
-    __half* dst = (is_k ? ko : qo) + (size_t)bh * T * D;
-    uint4 raw[PER];
+  n2 = red[0];
 #pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      const int idx = threadIdx.x + u * NT, r = idx / CH, c8 = idx - r * CH, t = t0 + r;
-      raw[u] = t < T ? *reinterpret_cast<const uint4*>(src + (size_t)t * D + c8 * 8)
-                     : make_uint4(0u, 0u, 0u, 0u);
-    }
-    // rotate (rows past T are zeros and stay zero), keep the largest magnitude
-    auto rotated = [&](int u, float* v) {
-      const int idx = threadIdx.x + u * NT, r = idx / CH, c8 = idx - r * CH;
-      const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = __bfloat162float(hv[e]);
-      Rope8 rt;
-      rt.c = tab[r * P4 + c8];
-      rt.s = tab[128 * P4 + r * P4 + c8];
-      rotate8(v, rt);
-    };
-    float amax = 0.f;
-#pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      float v[8];
-      rotated(u, v);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
-    }
-    amax = warp_max(amax);
-    float* rb = red[hh & 1];
-    if ((threadIdx.x & 31) == 0) rb[threadIdx.x >> 5] = amax;
-    __syncthreads();
-    amax = rb[0];
-#pragma unroll
-    for (int w = 1; w < NT / 32; ++w) amax = fmaxf(amax, rb[w]);
-    const float f = fp16_tile_factor(amax);
-    if (threadIdx.x == 0) {
-      const size_t ti = (size_t)bh * ntiles + tile;
-      if (is_k) kfac[ti] = 1.f / f;
-      else reinterpret_cast<float4*>(qfac)[ti] = make_float4(1.f / f, 0.f, 0.f, 0.f);
-    }
-    // the same rotation again (cheaper than holding every rotated value)
-#pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      const int idx = threadIdx.x + u * NT, r = idx / CH, c8 = idx - r * CH, t = t0 + r;
-      if (t >= T) continue;
-      float v[8];
-      rotated(u, v);
-      *reinterpret_cast<uint4*>(dst + (size_t)t * D + c8 * 8) = pack8_half(v, f);
-    }
+  for (int w = 1; w < NT / 32; ++w) n2 = fmaxf(n2, red[w]);
+  const float f = fp16_tile_factor(sqrtf(n2));
+  if (threadIdx.x == 0) {
+    const size_t ti = (size_t)bh * ntiles + tile;
+    if (is_k) kfac[ti] = 1.f / f;
+    else reinterpret_cast<float4*>(qfac)[ti] = make_float4(1.f / f, 0.f, 0.f, 0.f);
   }
-}
-
-// Heads per block of the RoPE pre-pass: as many as keep about 900 blocks in
-// the grid (two waves at three blocks per SM on 148 SMs; the kernel's
-// registers allow two), at least one.
-inline int rope_prep_group(int B, int H, int Hkv, int ntiles) {
-  const long units = (long)ntiles * B * (H + Hkv);
-  const long g = units / (2 * 3 * 148);
-  return (int)(g < 1 ? 1 : (g > H + Hkv ? H + Hkv : g));
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int t = t0 + (threadIdx.x + u * NT) / CH;
+    if (t >= T) continue;
+    const int pos = t - (doc_start ? doc_start[row0 + t] - row0 : 0);
+    float v[8];
+    const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[2 * e] = __low2float(hv[e]);
+      v[2 * e + 1] = __high2float(hv[e]);
+    }
+    rotate8(v, rope8_load<D>(rc, rs, pos, c8 * 8));
+    *reinterpret_cast<uint4*>(dst + (size_t)t * D + c8 * 8) = pack8_half(v, f);
+  }
 }
 
 // Eight bf16 values (16 bytes) as fp32, and back.

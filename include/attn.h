@@ -152,7 +152,9 @@ size_t attn_workspace_bytes_gqa(int B, int H, int H_kv, int T, int D, int dtype,
  * into fp16 tiles with power-of-two tile factors, and the backward recomputes
  * the scores from exactly those operands. attn_fwd_save leaves them in the
  * caller's buffer `saved`; attn_bwd_saved reads them from there instead of
- * rotating q and k again (one pass over q and k fewer per step).
+ * rotating q and k again (one pass over q and k fewer per step). With
+ * cu_seqlens the per-token document ranges are kept there too, so the
+ * backward does not rebuild them.
  *
  * attn_saved_bytes: bytes of that buffer; 0 when there is nothing to keep
  * (dtype ATTN_F32, has_rope = 0, or invalid sizes). Pure host function.

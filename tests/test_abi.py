@@ -317,7 +317,7 @@ def test_saved_operand_buffer_size_and_validation():
     B, H, Hkv, T, D = 2, 8, 2, 300, 128
     nt = (T + 127) // 128
     want = (up(B * H * T * D * 2) + up(B * Hkv * T * D * 2) + up(B * H * nt * 16)
-            + up(B * Hkv * nt * 4))
+            + up(B * Hkv * nt * 4) + up(2 * B * T * 4))  # rotated q, k, factors, document ranges
     assert A.attn_saved_bytes(B, H, Hkv, T, D, A.ATTN_BF16, 1) == want
     # nothing to keep: float32 storage, no RoPE, invalid sizes
     assert A.attn_saved_bytes(B, H, Hkv, T, D, A.ATTN_F32, 1) == 0
