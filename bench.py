@@ -43,20 +43,21 @@ FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # one ncu capture of the kernel on the workload, valid only while the kernel
 # sources still hash to what was captured (sha256, first 16 hex digits).
 MEASURED_TRAFFIC = {
-    ("dkdv", "long_context_8k"): (709.2e6, {"bwd_sm100.cuh": "aa590a5b73769d3d",
-                                            "sm100.cuh": "e7744a090cfc5a71",
+    ("dkdv", "long_context_8k"): (681.4e6, {"bwd_sm100.cuh": "c4111e40aacd37d8",
+                                            "sm100.cuh": "efe40f0294c09366",
                                             "common.cuh": "36b3720cacd61ee7"}),
-    ("dkdv", "decoder237m_layer"): (128.8e6, {"bwd_sm100.cuh": "aa590a5b73769d3d",
-                                              "sm100.cuh": "e7744a090cfc5a71",
+    ("dkdv", "decoder237m_layer"): (121.8e6, {"bwd_sm100.cuh": "c4111e40aacd37d8",
+                                              "sm100.cuh": "efe40f0294c09366",
                                               "common.cuh": "36b3720cacd61ee7"}),
-    ("fwd", "long_context_8k"): (161.1e6, {"fwd_sm100.cuh": "dc429d5deb84e30f",
-                                           "sm100.cuh": "e7744a090cfc5a71",
+    ("fwd", "long_context_8k"): (153.6e6, {"fwd_sm100.cuh": "dc429d5deb84e30f",
+                                           "sm100.cuh": "efe40f0294c09366",
                                            "common.cuh": "36b3720cacd61ee7"}),
-    ("fwd", "decoder237m_layer"): (51.9e6, {"fwd_sm100.cuh": "dc429d5deb84e30f",
-                                            "sm100.cuh": "e7744a090cfc5a71",
+    ("fwd", "decoder237m_layer"): (50.4e6, {"fwd_sm100.cuh": "dc429d5deb84e30f",
+                                            "sm100.cuh": "efe40f0294c09366",
                                             "common.cuh": "36b3720cacd61ee7"}),
-    ("decode", "decode_8k_gqa"): (201.9e6, {"decode.cuh": "a673449f05d438a0",
-                                            "common.cuh": "067de38d459c360f"}),
+    ("decode", "decode_8k_gqa"): (204.2e6, {"decode.cuh": "54d76420f3328bb9",
+                                            "sm100.cuh": "efe40f0294c09366",
+                                            "common.cuh": "36b3720cacd61ee7"}),
 }
 
 
