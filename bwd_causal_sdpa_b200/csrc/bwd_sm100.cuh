@@ -717,8 +717,13 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
         const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]),
                                                 __uint_as_float(s[2 * e + 1])),
                                     scl2, nl);
-        // about a third of the pairs go to the FMA pipe
-        float2 pv = (e % 3 == 2) ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
+        // kPolyPairs of the QC/2 pairs go to the FMA pipe (measured: at
+        // D = 128 every pair on MUFU is fastest, 2.5 % on the 8K kernel, since
+        // dS and the products' epilogue keep the FMA pipe busy; at D = 64 five
+        // pairs of sixteen)
+        constexpr int kPolyPairs = D == 128 ? 0 : 5;
+        const bool poly = (e * kPolyPairs) / (QC / 2) != ((e + 1) * kPolyPairs) / (QC / 2);
+        float2 pv = poly ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
         if (need_mask) {
           if (i_a < j || i_a >= de_j) pv.x = 0.f;
           if (i_a + 1 < j || i_a + 1 >= de_j) pv.y = 0.f;
