@@ -101,8 +101,14 @@ struct Layout {
   // reports an error instead of running misaligned.
   static constexpr int kSmemAlloc = kBytes;
   static constexpr uint32_t kTmemCols = 512;
-  // TMEM columns: S^T (dQ_{i-1} once S^T(i) has been read), dP^T, dV, dK
+  // TMEM columns: S^T (dQ_{i-1} once S^T(i) has been read), dP^T, dV, dK.
+  // kPT (D = 64 with the dQ warpgroup, where TMEM has room): P^T (bf16, two
+  // queries per column) and dQ have columns of their own instead, so dV reads
+  // P^T from TMEM and no product waits for another to free its columns.
+  static constexpr bool kPT = kDQ && D == 64;
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+  static constexpr uint32_t kColP = 256 + 2 * D, kColDQ = kColP + 64;
+  static_assert(!kPT || kColDQ + D <= kTmemCols, "P^T and dQ columns fit");
   // Four elementwise warpgroups (16 warps); each owns kQC = 32 query columns
   // of S^T / dP^T and kDC = D/4 feature columns of dK, dV.
   static constexpr int kNWG = 4;
@@ -359,7 +365,8 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
           return mbar_wait2(bar(b1), ph1 & 1, bar(b2), ph2 & 1, abort_flag);
         };
         auto group_S = [&](int i) -> bool {
-          const bool r = i == 0   ? wait1(L::bQFull, 0)
+          // kPT: S(i-1) has been read (P(i-1) formed, which dV(i-1) waited for)
+          const bool r = (i == 0 || L::kPT) ? wait1(L::bQFull + (i & 1), i >> 1)
                          : i == 1 ? wait2(L::bQFull + 1, 0, L::bSFree, 0)
                                   : wait2(L::bQFull + (i & 1), i >> 1, L::bDQFree, i - 2);
           if (!r) return false;
@@ -389,10 +396,16 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
           if (!wait1(L::bPFull, i)) return false;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tDV, smem_desc_sw128(ps + (kk >> 2) * L::kBlockBytes + (kk & 3) * 32, 16, 1024),
-                   smem_desc_sw128(obuf(i) + kk * 2048, L::kBlockBytes, 1024), id_dv,
-                   (i > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t db = smem_desc_sw128(obuf(i) + kk * 2048, L::kBlockBytes, 1024);
+            const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+            if constexpr (L::kPT)  // A = P^T from TMEM, 8 columns per K step
+              mma_ts(tDV, tmem + L::kColP + 8 * kk, db, id_dv, acc);
+            else
+              mma_ss(tDV,
+                     smem_desc_sw128(ps + (kk >> 2) * L::kBlockBytes + (kk & 3) * 32, 16, 1024),
+                     db, id_dv, acc);
+          }
           mma_commit(bar(L::bDVDone));
           mma_commit(bar(L::bDOEmpty + i % L::kDOStages));
           return true;
@@ -410,12 +423,15 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
           return true;
         };
         auto group_dQ = [&](int i) -> bool {
-          // into the S^T columns once the elementwise warps have read S(i+1)
-          if (i < n_it - 1 && !wait1(L::bSFree, i + 1)) return false;
+          // into the S^T columns once the elementwise warps have read S(i+1);
+          // kPT: into its own columns once the dQ warps have read dQ(i-1) out
+          if (L::kPT ? (i > 0 && !wait1(L::bDQFree, i - 1))
+                     : (i < n_it - 1 && !wait1(L::bSFree, i + 1)))
+            return false;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tS, smem_desc_sw128(ps + kk * 2048, L::kBlockBytes, 1024),
+            mma_ss(L::kPT ? tmem + L::kColDQ : tS, smem_desc_sw128(ps + kk * 2048, L::kBlockBytes, 1024),
                    smem_desc_sw128(sb0 + L::kK + kk * 2048, L::kBlockBytes, 1024), id_dq, kk > 0);
           mma_commit(bar(L::bDQFull));
           mma_commit(bar(L::bDSFree));  // the P/dS tile is free again (dK(i) is covered too)
@@ -510,7 +526,7 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
     // accumulator. A buffer is rewritten only after the reduce that last used
     // it (two chunks back) has read it.
     const int sub = warp & 3;
-    const uint32_t tq = tmem + ((uint32_t)(sub * 32) << 16) + L::kColS;
+    const uint32_t tq = tmem + ((uint32_t)(sub * 32) << 16) + (L::kPT ? L::kColDQ : L::kColS);
     constexpr int NCH = D / 32;
     int chunk = 0;
     bool prev_issued = false;  // did this warp reduce the previous chunk
@@ -699,9 +715,12 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
       for (int c = 0; c < QC / 32; ++c) tmem_ld32(tS + qc0 + 32 * c, s + 32 * c);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar(L::bSFree));  // the S^T columns may take the next tile
-      // asked now, answered by the time P is formed (see the wait below)
-      const bool ds_free = i == 0 || mbar_test(bar(L::bDSFree), (i - 1) & 1);
+      if constexpr (!L::kPT) mbar_arrive(bar(L::bSFree));  // the S^T columns may take the next tile
+      // asked now, answered by the time P is formed (see the wait below):
+      // kPT, dV(i-1) done reading P^T(i-1) from TMEM; else dQ(i-1) and
+      // dK(i-1) done reading dS^T(i-1) from the tile
+      const bool p_free = i == 0 || (L::kPT ? mbar_test(bar(L::bDVDone), (i - 1) & 1)
+                                            : mbar_test(bar(L::bDSFree), (i - 1) & 1));
       float scl = p.scale_log2;
       if constexpr (kF16) {
         // loaded with this tile's lse2 and Delta rows
@@ -731,13 +750,21 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
         pf[2 * e] = pv.x;
         pf[2 * e + 1] = pv.y;
       }
-      // dQ(i-1) and dK(i-1) must be done reading dS^T(i-1) from the tile
-      if (!ds_free && !mbar_wait(bar(L::bDSFree), (i - 1) & 1, abort_flag)) return false;
+      if (!p_free && !mbar_wait(bar(L::kPT ? L::bDVDone : L::bDSFree), (i - 1) & 1, abort_flag))
+        return false;
       uint32_t w[QC / 2];
 #pragma unroll
       for (int e = 0; e < QC / 2; ++e) w[e] = pack_bf16(pf[2 * e], pf[2 * e + 1]);
-      store_row(w);
-      fence_proxy_async_smem();
+      if constexpr (L::kPT) {
+        // this thread's 32 query columns as 16 packed columns of P^T
+        tc_fence_after();
+        tmem_st16(tmem + lane_base + L::kColP + (qc0 >> 1), w);
+        tmem_wait_st();
+        tc_fence_before();
+      } else {
+        store_row(w);
+        fence_proxy_async_smem();
+      }
       mbar_arrive(bar(L::bPFull));
       return true;
     };
@@ -756,7 +783,9 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
         uint32_t dpv[16];
         tmem_ld16(tDP + qc0 + 16 * h, dpv);
         tmem_wait_ld();
-        if (h == 0) dv_done = mbar_test(bar(L::bDVDone), i & 1);  // answered by the store below
+        if (h == 0)  // answered by the store below
+          dv_done = L::kPT ? (i == 0 || mbar_test(bar(L::bDSFree), (i - 1) & 1))
+                           : mbar_test(bar(L::bDVDone), i & 1);
 #pragma unroll
         for (int e2 = 0; e2 < 8; ++e2) {
           const int e = 8 * h + e2;
@@ -772,7 +801,11 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
           }
         }
       }
-      if (!dv_done && !mbar_wait(bar(L::bDVDone), i & 1, abort_flag)) return false;
+      // the tile must be free: dV(i) done reading P^T(i) from it, or (kPT, P^T
+      // in TMEM) dK(i-1) and dQ(i-1) done reading dS^T(i-1)
+      if (!dv_done && !(L::kPT ? mbar_wait(bar(L::bDSFree), (i - 1) & 1, abort_flag)
+                               : mbar_wait(bar(L::bDVDone), i & 1, abort_flag)))
+        return false;
       store_row(w);
       fence_proxy_async_smem();
       tc_fence_before();
