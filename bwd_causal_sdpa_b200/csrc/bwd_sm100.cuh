@@ -617,7 +617,9 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
         prev_issued = rows_in;
       }
     }
-    if (lane == 0) bulk_wait_group0();
+    // before the CTA leaves, the staging ring must have been read; the adds
+    // themselves complete with the grid, before any later kernel reads dq
+    if (lane == 0) bulk_wait_group_read0();
   } else {
     // ---------------- elementwise warps ----------------
     constexpr int QC = L::kQC, DC = L::kDC;
