@@ -43,13 +43,13 @@ FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # one ncu capture of the kernel on the workload, valid only while the kernel
 # sources still hash to what was captured (sha256, first 16 hex digits).
 MEASURED_TRAFFIC = {
-    ("dkdv", "long_context_8k"): (681.4e6, {"bwd_sm100.cuh": "c4111e40aacd37d8",
+    ("dkdv", "long_context_8k"): (686.8e6, {"bwd_sm100.cuh": "b5cea3328b97428c",
                                             "sm100.cuh": "efe40f0294c09366",
                                             "common.cuh": "36b3720cacd61ee7"}),
-    ("dkdv", "decoder237m_layer"): (121.8e6, {"bwd_sm100.cuh": "c4111e40aacd37d8",
+    ("dkdv", "decoder237m_layer"): (121.8e6, {"bwd_sm100.cuh": "b5cea3328b97428c",
                                               "sm100.cuh": "efe40f0294c09366",
                                               "common.cuh": "36b3720cacd61ee7"}),
-    ("fwd", "long_context_8k"): (153.6e6, {"fwd_sm100.cuh": "dc429d5deb84e30f",
+    ("fwd", "long_context_8k"): (153.1e6, {"fwd_sm100.cuh": "dc429d5deb84e30f",
                                            "sm100.cuh": "efe40f0294c09366",
                                            "common.cuh": "36b3720cacd61ee7"}),
     ("fwd", "decoder237m_layer"): (50.4e6, {"fwd_sm100.cuh": "dc429d5deb84e30f",
