@@ -773,14 +773,18 @@ int attn_profile_read(int kind, const char** name, int* launches, double* total_
 // ---------------------------------------------------------------------------
 namespace {
 
-// bf16 caches with up to 16 query heads per cached head take the streaming
-// tensor-core kernel: kDecodeStreamCtas CTAs (one per SM) over equal spans
-// of all cached tokens. Workspace: partial slots (f32 [slots][16][D], then
-// f32 [slots][16][2] max and sum), slots = kDecodeStreamCtas + B*H_kv, and
-// one int32 count per cached head.
-// The rest take one 64-token chunk per CTA. Workspace: per (query head,
-// chunk) the unnormalised partial sum (f32 [B*H][n_split][D]), then its max
-// and sum of exponentials (f32 [B*H][n_split] each).
+// bf16 caches with up to 16 query heads per cached head take a tensor-core
+// kernel: with at most kDecodeStreamCtas cached heads the persistent
+// streaming one (one CTA per SM over equal spans of all cached tokens;
+// workspace: partial slots f32 [slots][16][D], then f32 [slots][16][2] max
+// and sum, slots = kDecodeStreamCtas + B*H_kv, and one int32 count per cached
+// head); with more, each span would hold several short heads, so the split
+// one (cache ranges sized for about sixteen CTAs per SM over the grid, a
+// two-deep cp.async pipeline, then a combine launch) measured faster. The
+// split kernels (and f32 caches and larger groups: one 64-token chunk per
+// CTA) use per (query head, range) the unnormalised partial sum
+// (f32 [B*H][n_split][D]), then its max and sum of exponentials
+// (f32 [B*H][n_split] each). n_split == 0 marks the persistent kernel.
 struct DecodePlan {
   size_t o_part = 0, m_part = 0, l_part = 0, cnt = 0, total = 0;
   int n_split = 0, per_split = 0;
@@ -788,10 +792,18 @@ struct DecodePlan {
 
 bool decode_streams(int H, int H_kv, int dtype) { return dtype == ATTN_BF16 && H / H_kv <= 16; }
 constexpr int kDecodeStreamCtas = 148;
+constexpr long kDecodePipeCtas = 16 * 148;
 
 DecodePlan decode_plan(int B, int H, int H_kv, int T_max, int D, int dtype) {
   DecodePlan p;
-  if (decode_streams(H, H_kv, dtype)) {
+  if (decode_streams(H, H_kv, dtype) && (long)B * H_kv > kDecodeStreamCtas) {
+    const long stages = (T_max + kDecodePipeKeys - 1) / kDecodePipeKeys;
+    long want = (kDecodePipeCtas + (long)B * H_kv - 1) / ((long)B * H_kv);
+    want = want < 1 ? 1 : (want > stages ? stages : want);
+    const long per = (stages + want - 1) / want;  // stages per range
+    p.per_split = (int)(per * kDecodePipeKeys);
+    p.n_split = (int)((stages + per - 1) / per);
+  } else if (decode_streams(H, H_kv, dtype)) {
     const size_t slots = (size_t)kDecodeStreamCtas + (size_t)B * H_kv;
     p.o_part = 0;
     p.m_part = round_up(slots * 16 * D * sizeof(float));  // (max, sum) pairs
@@ -830,9 +842,19 @@ int decode_launch(const void* q, const void* k, const void* v, const int32_t* le
   float* mp = (float*)(ws + dp.m_part);
   float* lp = (float*)(ws + dp.l_part);
   const int G = H / H_kv;
-  if (std::is_same<TIO, __nv_bfloat16>::value && G <= 16) {
-    // streaming tensor-core variant (up to 16 query heads per cached head):
-    // one launch, the heads split over CTAs merged by their last CTA
+  if (std::is_same<TIO, __nv_bfloat16>::value && G <= 16 && dp.n_split > 0) {
+    // split tensor-core variant (many short heads), then the combine
+    static bool pipe_smem_set[64] = {};
+    if (!ensure_smem(decode_pipe_kernel<D>, DecodePipeLayout<D>::kBytes, pipe_smem_set))
+      return ATTN_ECUDA;
+    ATTN_LAUNCH(KK_DECODE, st, pdl_launch(decode_pipe_kernel<D>, dim3(dp.n_split, B * H_kv), kDecodeMmaThreads,
+                                          DecodePipeLayout<D>::kBytes, st, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                          (const __nv_bfloat16*)v, lens, rc, rs, op, mp, lp, H, H_kv, T_max,
+                                          dp.n_split, dp.per_split, scale * 1.4426950408889634f));
+  } else if (std::is_same<TIO, __nv_bfloat16>::value && G <= 16) {
+    // persistent streaming tensor-core variant (up to 16 query heads per
+    // cached head): one launch, the heads split over CTAs merged by their
+    // last CTA
     using SL = DecStreamLayout<D>;
     static bool stream_smem_set[2][64] = {};
     auto kern = G <= 8 ? decode_stream_kernel<D, 1> : decode_stream_kernel<D, 2>;
@@ -849,10 +871,11 @@ int decode_launch(const void* q, const void* k, const void* v, const int32_t* le
                                           rc, rs, (__nv_bfloat16*)o, lse, op, mp, cnt, B, H,
                                           H_kv, T_max, scale * 1.4426950408889634f));
     return launch_status();
+  } else {
+    ATTN_LAUNCH(KK_DECODE, st, pdl_launch(decode_split_kernel<TIO, D>, dim3(dp.n_split, B * H_kv), kDecodeThreads,
+                                          L::bytes(G), st, (const TIO*)q, (const TIO*)k, (const TIO*)v, lens, rc, rs, op, mp, lp, H,
+                                          H_kv, T_max, dp.n_split, dp.per_split, scale * 1.4426950408889634f));
   }
-  ATTN_LAUNCH(KK_DECODE, st, pdl_launch(decode_split_kernel<TIO, D>, dim3(dp.n_split, B * H_kv), kDecodeThreads,
-                                        L::bytes(G), st, (const TIO*)q, (const TIO*)k, (const TIO*)v, lens, rc, rs, op, mp, lp, H,
-                                        H_kv, T_max, dp.n_split, dp.per_split, scale * 1.4426950408889634f));
   if (launch_status()) return ATTN_ECUDA;
   ATTN_LAUNCH(KK_DECODE_COMBINE, st, pdl_launch(decode_combine_kernel<TIO, D>, B * H, kDecodeCombineThreads,
                                               dp.n_split * sizeof(float), st, op, mp, lp, lens, (TIO*)o, lse, H, T_max, dp.n_split, dp.per_split));

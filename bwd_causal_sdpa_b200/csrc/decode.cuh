@@ -700,6 +700,253 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(
   }
 }
 
+constexpr int kDecodeMmaThreads = 128;
+
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+
+// ---------------------------------------------------------------------------
+// Split tensor-core variant (bf16 cache, G <= 16), for many short heads
+// (more cached heads than SMs, where the persistent kernel's spans would
+// each hold several heads and pay a query setup and merge per piece): the G
+// query heads are the rows of a 16-row tile (zero rows past G), and the
+// hardware schedules many short CTAs. One CTA walks a range
+// of the cache (per_split tokens, a multiple of kDecodePipeKeys) in stages of
+// kDecodePipeKeys tokens through a kDecodePipeStages-deep cp.async pipeline,
+// so loads stay in flight while earlier stages are scored and summed. Per
+// stage: S = (Q_hi + Q_lo) K^T with each warp taking 8 keys (the scaled,
+// rotated fp32 query is split into bf16 hi = bf16(q) and lo = bf16(q - hi),
+// so the scores keep ~16 more bits than one bf16 query would, which the lse
+// bound needs; the query fragments stay in registers), the row max combined across the warps, the
+// running max / sum updated and the output accumulators (registers, warp w
+// owning D/4 columns) rescaled by exp2(m_old - m_new) before P V of the
+// stage is added.
+// ---------------------------------------------------------------------------
+constexpr int kDecodePipeKeys = 32;
+constexpr int kDecodePipeStages = 2;
+
+template <int D>
+struct DecodePipeLayout {
+  static constexpr int kRowBytes = D * 2 + 16;                 // padded bf16 rows
+  static constexpr int kStageBytes = 2 * kDecodePipeKeys * kRowBytes;  // K rows, V rows
+  static constexpr int kQhi = kDecodePipeStages * kStageBytes;
+  static constexpr int kQlo = kQhi + 16 * kRowBytes;
+  static constexpr int kPRowBytes = kDecodePipeKeys * 2 + 16;  // [16][32] bf16
+  static constexpr int kP = kQlo + 16 * kRowBytes;
+  static constexpr int kRed = kP + 16 * kPRowBytes;             // f32 [2][4 warps][16]
+  static constexpr int kStat = kRed + 2 * 4 * 16 * 4;           // f32 running max [16], sum [16]
+  static constexpr int kBytes = kStat + 2 * 16 * 4;
+};
+static_assert(DecodePipeLayout<128>::kP % 16 == 0 && DecodePipeLayout<64>::kRed % 16 == 0,
+              "ldmatrix rows need 16-byte alignment");
+
+template <int D>
+__global__ void __launch_bounds__(kDecodeMmaThreads) decode_pipe_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_cache,
+    const __nv_bfloat16* __restrict__ v_cache, const int32_t* __restrict__ cache_lens,
+    const float* __restrict__ rc, const float* __restrict__ rs, float* __restrict__ o_part,
+    float* __restrict__ m_part, float* __restrict__ l_part, int H, int Hkv, int T_max,
+    int n_split, int per_split, float scale_log2) {
+  pdl_wait_and_trigger();
+  using L = DecodePipeLayout<D>;
+  constexpr int C = kDecodePipeKeys;
+  constexpr int NS = kDecodePipeStages;
+  constexpr int NT = D / 32;  // n8 tiles of the weighted sum per warp
+  constexpr int KS = D / 16;  // k-steps of the scores
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int G = H / Hkv;
+  const int bhk = blockIdx.y, b = bhk / Hkv, hk = bhk - b * Hkv;
+  const int split = blockIdx.x;
+  int len = cache_lens[b];
+  if (len < 1 || len > T_max) {
+    if (threadIdx.x == 0 && split == 0 && hk == 0) report_status(ATTN_EDEVICE_INPUT);
+    len = len < 1 ? 1 : T_max;
+  }
+  const int t_lo = split * per_split;
+  if (t_lo >= len) return;  // uniform: this range is past the cache
+  const int t_hi = min(t_lo + per_split, len);
+  const int n_st = (t_hi - t_lo + C - 1) / C;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sb = (uint32_t)__cvta_generic_to_shared(sm);
+  const __nv_bfloat16* kb = k_cache + (size_t)bhk * T_max * D;
+  const __nv_bfloat16* vb = v_cache + (size_t)bhk * T_max * D;
+
+  // stage si's K and V rows into buffer si % NS (rows past the range
+  // zero-filled); one commit per call, so the group counts line up
+  auto issue_stage = [&](int si) {
+    if (si < n_st) {
+      const int j0 = t_lo + si * C, nk = min(C, t_hi - j0);
+      const uint32_t st = sb + (si % NS) * L::kStageBytes;
+      for (int i = tid; i < C * D / 8; i += kDecodeMmaThreads) {
+        const int r = i / (D / 8), p = i - r * (D / 8);
+        const uint32_t nb = r < nk ? 16u : 0u;
+        const size_t src = (size_t)(j0 + (r < nk ? r : 0)) * D + p * 8;  // in bounds
+        cp_async16(st + r * L::kRowBytes + p * 16, kb + src, nb);
+        cp_async16(st + (C + r) * L::kRowBytes + p * 16, vb + src, nb);
+      }
+    }
+    cp_async_commit();
+  };
+  for (int si = 0; si < NS - 1; ++si) issue_stage(si);
+
+  // the queries: rotated to position len-1, scaled by scale*log2(e), split
+  // into bf16 hi + lo; rows G..15 zero
+  for (int i = tid; i < 16 * (D / 2); i += kDecodeMmaThreads) {
+    const int g = i / (D / 2), pi = i - g * (D / 2);
+    float x[2] = {0.f, 0.f};
+    if (g < G) {
+      load_vec<2>(q + ((size_t)b * H + hk * G + g) * D + 2 * pi, x);
+      if (rc) rope_pairs<2, D>(x, rc, rs, len - 1, 2 * pi, false);
+      x[0] *= scale_log2;
+      x[1] *= scale_log2;
+    }
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(x[0], x[1]);
+    const __nv_bfloat162 lo =
+        __floats2bfloat162_rn(x[0] - __low2float(hi), x[1] - __high2float(hi));
+    *reinterpret_cast<__nv_bfloat162*>(sm + L::kQhi + g * L::kRowBytes + pi * 4) = hi;
+    *reinterpret_cast<__nv_bfloat162*>(sm + L::kQlo + g * L::kRowBytes + pi * 4) = lo;
+  }
+  float* red = reinterpret_cast<float*>(sm + L::kRed);    // [0..63] maxima, [64..127] sums
+  float* stm = reinterpret_cast<float*>(sm + L::kStat);   // running max [16]
+  float* stl = stm + 16;                                  // running sum [16]
+  if (tid < 16) {
+    stm[tid] = -INFINITY;
+    stl[tid] = 0.f;
+  }
+  __syncthreads();
+  // query fragments (hi, lo) for all k-steps, kept in registers
+  uint32_t qh[KS][4], ql[KS][4];
+  {
+    const int arow = lane & 15, acol = (lane >> 4) * 8;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      ldsm_x4(sb + L::kQhi + arow * L::kRowBytes + (ks * 16 + acol) * 2, qh[ks][0], qh[ks][1],
+              qh[ks][2], qh[ks][3]);
+      ldsm_x4(sb + L::kQlo + arow * L::kRowBytes + (ks * 16 + acol) * 2, ql[ks][0], ql[ks][1],
+              ql[ks][2], ql[ks][3]);
+    }
+  }
+  const int r0 = lane >> 2, r1 = r0 + 8;
+  float oc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) oc[t][0] = oc[t][1] = oc[t][2] = oc[t][3] = 0.f;
+
+  for (int si = 0; si < n_st; ++si) {
+    issue_stage(si + NS - 1);
+    cp_async_wait_pending<NS - 1>();
+    __syncthreads();
+    const uint32_t kst = sb + (si % NS) * L::kStageBytes;
+    const uint32_t vst = kst + C * L::kRowBytes;
+    const int nk = min(C, t_hi - (t_lo + si * C));
+    // scores of this warp's 8 keys
+    float sc[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      const int brow = lane & 7, bcol = ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t b0, b1;
+        ldsm_x2(kst + (warp * 8 + brow) * L::kRowBytes + (ks * 16 + bcol) * 2, b0, b1);
+        mma_bf16_16816(sc, qh[ks][0], qh[ks][1], qh[ks][2], qh[ks][3], b0, b1);
+        mma_bf16_16816(sc, ql[ks][0], ql[ks][1], ql[ks][2], ql[ks][3], b0, b1);
+      }
+    }
+    const int key = warp * 8 + 2 * (lane & 3);  // this thread's two keys: key, key + 1
+    if (key >= nk) sc[0] = sc[2] = -INFINITY;
+    if (key + 1 >= nk) sc[1] = sc[3] = -INFINITY;
+    float mx0 = fmaxf(sc[0], sc[1]), mx1 = fmaxf(sc[2], sc[3]);
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    if ((lane & 3) == 0) {
+      red[warp * 16 + r0] = mx0;
+      red[warp * 16 + r1] = mx1;
+    }
+    __syncthreads();
+    // new running max, rescale factor, P of this stage
+    const float mo0 = stm[r0], mo1 = stm[r1];
+    const float mn0 = fmaxf(mo0, fmaxf(fmaxf(red[r0], red[16 + r0]), fmaxf(red[32 + r0], red[48 + r0])));
+    const float mn1 = fmaxf(mo1, fmaxf(fmaxf(red[r1], red[16 + r1]), fmaxf(red[32 + r1], red[48 + r1])));
+    const float al0 = exp2f(mo0 - mn0), al1 = exp2f(mo1 - mn1);  // 0 on the first stage
+    const float p0 = exp2f(sc[0] - mn0), p1 = exp2f(sc[1] - mn0);  // masked: 0
+    const float p2 = exp2f(sc[2] - mn1), p3 = exp2f(sc[3] - mn1);
+    *reinterpret_cast<__nv_bfloat162*>(sm + L::kP + r0 * L::kPRowBytes + key * 2) =
+        __floats2bfloat162_rn(p0, p1);
+    *reinterpret_cast<__nv_bfloat162*>(sm + L::kP + r1 * L::kPRowBytes + key * 2) =
+        __floats2bfloat162_rn(p2, p3);
+    float ls0 = p0 + p1, ls1 = p2 + p3;
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      ls0 += __shfl_xor_sync(0xffffffffu, ls0, o);
+      ls1 += __shfl_xor_sync(0xffffffffu, ls1, o);
+    }
+    if ((lane & 3) == 0) {
+      red[64 + warp * 16 + r0] = ls0;
+      red[64 + warp * 16 + r1] = ls1;
+    }
+    __syncthreads();
+    if (tid < 16) {  // running statistics of row tid
+      const float mo = stm[tid];
+      const float mn = fmaxf(mo, fmaxf(fmaxf(red[tid], red[16 + tid]), fmaxf(red[32 + tid], red[48 + tid])));
+      stl[tid] = stl[tid] * exp2f(mo - mn) + (red[64 + tid] + red[80 + tid]) +
+                 (red[96 + tid] + red[112 + tid]);
+      stm[tid] = mn;
+    }
+    // O = O * alpha + P V (this warp's D/4 columns)
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      oc[t][0] *= al0;
+      oc[t][1] *= al0;
+      oc[t][2] *= al1;
+      oc[t][3] *= al1;
+    }
+    {
+      const int arow = lane & 15, acol = (lane >> 4) * 8, vrow = lane & 15;
+#pragma unroll
+      for (int ks = 0; ks < C / 16; ++ks) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(sb + L::kP + arow * L::kPRowBytes + (ks * 16 + acol) * 2, a0, a1, a2, a3);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          uint32_t b0, b1;
+          ldsm_x2_trans(vst + (ks * 16 + vrow) * L::kRowBytes + (warp * (D / 4) + t * 8) * 2, b0,
+                        b1);
+          mma_bf16_16816(oc[t], a0, a1, a2, a3, b0, b1);
+        }
+      }
+    }
+    __syncthreads();  // buffer si % NS, P and the partial maxima / sums are reused
+  }
+
+  // partials of this range, rows < G
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int col = warp * (D / 4) + t * 8 + 2 * (lane & 3);
+    if (r0 < G) {
+      const size_t slot = ((size_t)b * H + hk * G + r0) * n_split + split;
+      *reinterpret_cast<float2*>(o_part + slot * D + col) = make_float2(oc[t][0], oc[t][1]);
+    }
+    if (r1 < G) {
+      const size_t slot = ((size_t)b * H + hk * G + r1) * n_split + split;
+      *reinterpret_cast<float2*>(o_part + slot * D + col) = make_float2(oc[t][2], oc[t][3]);
+    }
+  }
+  if (tid < G) {
+    const size_t slot = ((size_t)b * H + hk * G + tid) * n_split + split;
+    m_part[slot] = stm[tid];
+    l_part[slot] = stl[tid];
+  }
+}
+
 // Merge the chunk partials of one (b, h): M = max m_s, l = sum l_s 2^(m_s-M),
 // o = sum o_s 2^(m_s-M) / l, lse = (M + log2 l) ln 2. One block of
 // kDecodeCombineThreads threads per query head: the chunks are spread over

@@ -4,10 +4,12 @@ element (both storage types and head sizes, group sizes 1 to 32, cache
 lengths 1, ragged, a multiple of the 128-token chunk and the full capacity),
 the two named decode workloads on sampled heads, cache rows past the length
 (set to NaN) without effect on the result, and out-of-range lengths reported
-and clamped. The streaming kernel splits the cached tokens of all heads into
-one equal span per CTA, so the small cases put each head over several CTAs
-(partials merged by the head's last CTA) and the full-size ones mix heads
-held whole with split ones."""
+and clamped. With up to 148 cached heads the persistent streaming kernel
+splits the cached tokens of all heads into one equal span per CTA, so the
+small cases put each head over several CTAs (partials merged by the head's
+last CTA) and decode_8k_gqa mixes heads held whole with split ones; with
+more cached heads (decode_237m, and two small cases) the split tensor-core
+kernel and its combine run."""
 
 import numpy as np
 import pytest
@@ -65,6 +67,9 @@ SMALL = [
     ("decode_237m", dict(B=3, H=16, H_kv=1, T_max=400, len_min=200, seed=43)),
     # fewer cached tokens than CTAs: most spans are empty, heads split finely
     ("decode_8k_gqa", dict(B=1, H=4, H_kv=1, T_max=64, len_min=1, seed=44)),
+    # more cached heads than SMs: the split tensor-core kernel and its combine
+    ("decode_237m", dict(B=20, H=16, H_kv=8, T_max=200, len_min=1, seed=45)),
+    ("decode_8k_gqa", dict(B=38, H=16, H_kv=4, T_max=300, len_min=1, seed=46)),
 ]
 
 
