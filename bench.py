@@ -55,7 +55,7 @@ MEASURED_TRAFFIC = {
     ("fwd", "decoder237m_layer"): (50.4e6, {"fwd_sm100.cuh": "dc429d5deb84e30f",
                                             "sm100.cuh": "efe40f0294c09366",
                                             "common.cuh": "36b3720cacd61ee7"}),
-    ("decode", "decode_8k_gqa"): (204.2e6, {"decode.cuh": "54d76420f3328bb9",
+    ("decode", "decode_8k_gqa"): (204.2e6, {"decode.cuh": "c5b2c0ceb074a366",
                                             "sm100.cuh": "efe40f0294c09366",
                                             "common.cuh": "36b3720cacd61ee7"}),
 }
