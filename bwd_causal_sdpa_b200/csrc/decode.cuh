@@ -346,8 +346,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(
   pdl_wait_and_trigger();
   using L = DecStreamLayout<D>;
   constexpr int NS = L::kStages;
-  constexpr int KS = D / 16;  // k-steps of the scores
-  constexpr int NT = D / 8;   // n8 tiles of the output
+  constexpr int KS = D / 16;  // k-steps of the scores, and 16-feature tiles of the output
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* sm = dsm_raw + ((1024 - (smem_u32(dsm_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(sm);

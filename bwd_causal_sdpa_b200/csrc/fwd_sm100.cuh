@@ -31,7 +31,8 @@
 // log2 l) ln 2 use the same reference, so the result is exact up to rounding.
 // A fixed share of the exponentials (kPolyPairs pairs of every 32) runs as a
 // polynomial on the FMA pipe, the rest on MUFU, so that neither unit alone
-// sets the pace of the softmax.
+// sets the pace of the softmax; the share was measured per head size (0, 2,
+// 4, 6, 8 pairs: 2 best at D = 128, 3 % faster than 8; 8 best at D = 64).
 //
 // Masking is per element only on blocks that cross the diagonal or the start
 // of a row's document; key blocks wholly before the document of a tile's
@@ -46,10 +47,6 @@
 #pragma once
 
 #include "sm100.cuh"
-
-#ifndef ATTN_FWD_POLY_PAIRS
-#define ATTN_FWD_POLY_PAIRS 8
-#endif
 
 namespace fwd100 {
 
@@ -87,7 +84,7 @@ struct Layout {
   static constexpr int kSoftmaxThreads = 256;
   static constexpr int kThreads = kSoftmaxThreads + 96;
   static constexpr int kProducerWarp = 8, kMmaWarp0 = 9;
-  static constexpr int kPolyPairs = ATTN_FWD_POLY_PAIRS;  // of the 32 pairs of a block row
+  static constexpr int kPolyPairs = D == 128 ? 2 : 8;  // of the 32 pairs of a block row
   static_assert(kBytes <= 232448, "shared memory");
   static_assert(kQTileBytes % 1024 == 0 && kKVBytes % 1024 == 0, "swizzle atoms stay aligned");
   static_assert(kPolyPairs >= 0 && kPolyPairs <= 32, "poly share");
