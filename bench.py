@@ -49,13 +49,13 @@ MEASURED_TRAFFIC = {
     ("dkdv", "decoder237m_layer"): (121.8e6, {"bwd_sm100.cuh": "b5cea3328b97428c",
                                               "sm100.cuh": "efe40f0294c09366",
                                               "common.cuh": "36b3720cacd61ee7"}),
-    ("fwd", "long_context_8k"): (153.1e6, {"fwd_sm100.cuh": "dc429d5deb84e30f",
+    ("fwd", "long_context_8k"): (155.6e6, {"fwd_sm100.cuh": "7b9df616ca1a18a1",
                                            "sm100.cuh": "efe40f0294c09366",
                                            "common.cuh": "36b3720cacd61ee7"}),
-    ("fwd", "decoder237m_layer"): (50.4e6, {"fwd_sm100.cuh": "dc429d5deb84e30f",
+    ("fwd", "decoder237m_layer"): (50.4e6, {"fwd_sm100.cuh": "7b9df616ca1a18a1",
                                             "sm100.cuh": "efe40f0294c09366",
                                             "common.cuh": "36b3720cacd61ee7"}),
-    ("decode", "decode_8k_gqa"): (204.2e6, {"decode.cuh": "c5b2c0ceb074a366",
+    ("decode", "decode_8k_gqa"): (204.2e6, {"decode.cuh": "778c93a2b3db4cde",
                                             "sm100.cuh": "efe40f0294c09366",
                                             "common.cuh": "36b3720cacd61ee7"}),
 }
