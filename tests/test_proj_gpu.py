@@ -66,10 +66,13 @@ def test_small_projections_match_oracle(name, rope):
     _check(w, got, rope)
 
 
-@pytest.mark.parametrize("C,H,H_kv,D", [(8, 1, 1, 64), (24, 1, 1, 128), (1000, 5, 5, 64)])
-def test_edge_shapes(C, H, H_kv, D):
-    # one 128-token tile, K below one 64-wide block or with a tail, N tails
-    w = make_proj_workload(proj_config_by_name("proj_small_d64"), B=1, T=128, C=C, H=H,
+@pytest.mark.parametrize("C,H,H_kv,D,T", [(8, 1, 1, 64, 128), (24, 1, 1, 128, 128),
+                                         (1000, 5, 5, 64, 128), (304, 3, 1, 64, 384)])
+def test_edge_shapes(C, H, H_kv, D, T):
+    # one or three 128-token tiles (256-row pair tiles with an empty or a
+    # half-empty second CTA), K below one 64-wide block, with a tail or with an
+    # odd number of blocks (a last stage of one block), N tails
+    w = make_proj_workload(proj_config_by_name("proj_small_d64"), B=1, T=T, C=C, H=H,
                            H_kv=H_kv, D=D, packed=False, seed=40 + C)
     _, got = _run(w, True)
     _check(w, got, True)
