@@ -55,7 +55,7 @@ MEASURED_TRAFFIC = {
     ("fwd", "decoder237m_layer"): (50.4e6, {"fwd_sm100.cuh": "7b9df616ca1a18a1",
                                             "sm100.cuh": "efe40f0294c09366",
                                             "common.cuh": "36b3720cacd61ee7"}),
-    ("decode", "decode_8k_gqa"): (204.2e6, {"decode.cuh": "778c93a2b3db4cde",
+    ("decode", "decode_8k_gqa"): (204.2e6, {"decode.cuh": "ed672db8f3155da3",
                                             "sm100.cuh": "efe40f0294c09366",
                                             "common.cuh": "36b3720cacd61ee7"}),
 }

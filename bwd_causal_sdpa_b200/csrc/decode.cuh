@@ -282,19 +282,21 @@ __device__ __forceinline__ void consumer_sync() {  // the eight consumer warps
 
 // ---------------------------------------------------------------------------
 // Streaming tensor-core variant (bf16 cache, G <= 8 NH query heads per cached
-// head, NH = 1 or 2). The cached tokens of all (b, cached head) pairs, laid end to end,
-// are cut into gridDim.x equal spans, one per CTA (at most one CTA per SM),
-// so every SM reads the same number of bytes whatever the length mix. A
-// CTA's span covers pieces of one or more heads. One TMA warp streams the
-// pieces in stages of 64 keys (K and V tiles, 128-byte swizzled boxes of 64
-// keys x 64 features) through a kDecStages-deep ring; eight consumer warps
-// take the stages in turn, two groups of four (even and odd stages), each
-// warp 16 keys of a stage with its own running max, sum and output for the
-// G query heads (the rows of a 16-row tile):
-//   S = (Q_hi + Q_lo) K^T      (the scaled, rotated fp32 query split into
+// head, NH = 1 or 2), for up to one cached head per SM. The cached tokens of
+// all (b, cached head) pairs, laid end to end, are cut into gridDim.x equal
+// spans, one per CTA (at most one CTA per SM), so every SM reads the same
+// number of bytes whatever the length mix. A CTA's span covers pieces of one
+// or more heads. One TMA warp streams the pieces in stages of 64 keys (K and
+// V tiles, 128-byte swizzled boxes of 64 keys x 64 features) through a
+// kDecStages-deep ring; eight consumer warps take the stages in turn, two
+// groups of four (even and odd stages), each warp 16 keys of a stage with its
+// own running max, sum and output for the G query heads, in transposed
+// products (keys as the 16 rows of a tile, the heads as NH columns of 8):
+//   S^T = K (Q_hi + Q_lo)^T    (the scaled, rotated fp32 query split into
 //                               two bf16 parts, which keeps ~16 more bits
 //                               of the scores than one bf16 query would)
-//   O = O * 2^(m_old - m_new) + P V   (P straight from the score registers)
+//   O^T = O^T * 2^(m_old - m_new) + V^T P^T   (P^T from the score registers,
+//                               moved to the operand layout by movmatrix)
 // At the end of a piece the eight warps' states merge through shared memory.
 // A head held whole by one CTA is written out at once; otherwise each CTA
 // stores its partial (o unnormalised, max, sum) in slot (CTA + head), and
