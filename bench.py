@@ -43,10 +43,10 @@ FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # one ncu capture of the kernel on the workload, valid only while the kernel
 # sources still hash to what was captured (sha256, first 16 hex digits).
 MEASURED_TRAFFIC = {
-    ("dkdv", "long_context_8k"): (686.8e6, {"bwd_sm100.cuh": "b5cea3328b97428c",
+    ("dkdv", "long_context_8k"): (672.3e6, {"bwd_sm100.cuh": "073cb8d91447bbbf",
                                             "sm100.cuh": "efe40f0294c09366",
                                             "common.cuh": "36b3720cacd61ee7"}),
-    ("dkdv", "decoder237m_layer"): (121.8e6, {"bwd_sm100.cuh": "b5cea3328b97428c",
+    ("dkdv", "decoder237m_layer"): (122.0e6, {"bwd_sm100.cuh": "073cb8d91447bbbf",
                                               "sm100.cuh": "efe40f0294c09366",
                                               "common.cuh": "36b3720cacd61ee7"}),
     ("fwd", "long_context_8k"): (155.6e6, {"fwd_sm100.cuh": "7b9df616ca1a18a1",

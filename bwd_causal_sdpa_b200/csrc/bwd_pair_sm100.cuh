@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
   const int row0 = b * T;
   // the pair walks from its first diagonal tile to the end of its last key's document
   const int jlast = min(256 * ktp + 255, T - 1);
-  const int q_end = p.doc_end ? p.doc_end[row0 + jlast] - row0 : T;
+  const int q_end = p.doc_end ? min(max(p.doc_end[row0 + jlast] - row0, jlast + 1), T) : T;
   const int qt0 = 2 * ktp;
   const int n_q = (q_end + 127) / 128 - qt0;
   const int n_it = G * n_q;
@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     const int j = j0 + r;
     const int qc0 = QC * wg, dc0 = DC * wg;
     const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
-    const int de_j = (j < T) ? (p.doc_end ? p.doc_end[row0 + j] - row0 : T) : T;
+    const int de_j = (j < T) ? (p.doc_end ? min(max(p.doc_end[row0 + j] - row0, j + 1), T) : T) : T;
     const uint32_t tS = tmem + lane_base + L::kColS;
     const uint32_t tDP = tmem + lane_base + L::kColDP;
     uint8_t* psb = sg + L::kPS;
@@ -439,7 +439,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     if (ok && W(L::bFinal, 0)) {
       tc_fence_after();
       const int jj = min(j, T - 1);
-      const int pos = jj - (p.doc_start ? p.doc_start[row0 + jj] - row0 : 0);
+      const int pos = jj - (p.doc_start ? min(max(p.doc_start[row0 + jj] - row0, 0), jj) : 0);
       const float inv_c = 1.f / cscale;
       if (p.n_split > 1) {
         float* dka = p.dk_acc + ((size_t)bhk * T + jj) * D;

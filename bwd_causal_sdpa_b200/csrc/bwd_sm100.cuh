@@ -196,7 +196,9 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
   const int j0 = kt * 128;
   const int row0 = b * T;
   const int jlast = min(j0 + 127, T - 1);
-  const int q_end = p.doc_end ? p.doc_end[row0 + jlast] - row0 : T;  // exclusive
+  // exclusive; document ranges are clamped into the row wherever they are
+  // read (they may come from the caller's saved buffer)
+  const int q_end = p.doc_end ? min(max(p.doc_end[row0 + jlast] - row0, jlast + 1), T) : T;
   const int qt0 = kt;
   const int n_q = (q_end + 127) / 128 - qt0;
   const int n_it = G * n_q;
@@ -629,7 +631,7 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
     const int qc0 = QC * wg;        // query columns of S^T / dP^T handled here
     const int dc0 = DC * wg;        // feature columns of dK / dV handled here
     const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
-    const int de_j = (j < T) ? (p.doc_end ? p.doc_end[row0 + j] - row0 : T) : T;
+    const int de_j = (j < T) ? (p.doc_end ? min(max(p.doc_end[row0 + j] - row0, j + 1), T) : T) : T;
     const uint32_t tS = tmem + lane_base + L::kColS;
     const uint32_t tDP = tmem + lane_base + L::kColDP;
     uint8_t* psb = sg + L::kPS;
@@ -831,7 +833,7 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
     if (ok && mbar_wait(bar(L::bFinal), 0, abort_flag)) {
       tc_fence_after();
       const int jj = min(j, T - 1);
-      const int pos = jj - (p.doc_start ? p.doc_start[row0 + jj] - row0 : 0);
+      const int pos = jj - (p.doc_start ? min(max(p.doc_start[row0 + jj] - row0, 0), jj) : 0);
       __nv_bfloat16* dkrow = p.dk + ((size_t)bhk * T + jj) * D;
       __nv_bfloat16* dvrow = p.dv + ((size_t)bhk * T + jj) * D;
       constexpr int CW = DC < 32 ? DC : 32;  // columns per TMEM load

@@ -136,7 +136,9 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
   const int row0 = b * T;
   // key tiles [kt_lo, qt]: from the tile holding the start of the first row's
   // document (a query tile's allowed keys form one interval) to the diagonal
-  const int kt_lo = p.doc_start ? ((p.doc_start[row0 + qt * 128] - row0) >> 7) : 0;
+  // document ranges clamped into the row (they may come from the caller's saved buffer)
+  const int kt_lo =
+      p.doc_start ? (min(max(p.doc_start[row0 + qt * 128] - row0, 0), qt * 128) >> 7) : 0;
   const int n_kv = qt - kt_lo + 1;
 
   if (threadIdx.x == 0) {
@@ -287,7 +289,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
     const uint32_t tS = tmem + lane_base + L::kColS + kc0;
     const uint32_t tDP = tmem + lane_base + L::kColDP + kc0;
-    const int ds_i = p.doc_start ? p.doc_start[row0 + min(i, T - 1)] - row0 : 0;
+    const int ds_i = p.doc_start ? min(max(p.doc_start[row0 + min(i, T - 1)] - row0, 0), min(i, T - 1)) : 0;
     uint8_t* dsb = sg + L::kDS + (kc0 >> 6) * L::kBlockBytes;
     const int ch0 = (kc0 & 63) >> 3;
     bool ok = mbar_wait(bar(L::bQ), 0, abort_flag);
@@ -366,7 +368,7 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     if (ok && mbar_wait(bar(L::bFinal), 0, abort_flag)) {
       tc_fence_after();
       const int ii = min(i, T - 1);
-      const int pos = ii - (p.doc_start ? p.doc_start[row0 + ii] - row0 : 0);
+      const int pos = ii - (p.doc_start ? min(max(p.doc_start[row0 + ii] - row0, 0), ii) : 0);
       __nv_bfloat16* dqrow = p.dq + ((size_t)bh * T + ii) * D;
       const float f = p.scale / cscale;
       constexpr int CW = DC < 32 ? DC : 32;  // columns per TMEM load

@@ -320,7 +320,8 @@ __global__ void __launch_bounds__(256) dq_finalize_kernel(
 #pragma unroll
   for (int e = 0; e < 8; ++e) v[e] *= f;
   if (rc) {
-    const int pos = t - (doc_start ? doc_start[b * T + t] - b * T : 0);
+    // clamped into the row (the ranges may come from the caller's saved buffer)
+    const int pos = t - (doc_start ? min(max(doc_start[b * T + t] - b * T, 0), t) : 0);
     rope_pairs<8, D>(v, rc, rs, pos, d0, true);
   }
   store_vec<4>(dq + e0, v);

@@ -163,7 +163,9 @@ size_t attn_workspace_bytes_gqa(int B, int H, int H_kv, int T, int D, int dtype,
  * attn_bwd_saved: attn_bwd_gqa plus `saved` (read only): it must hold what
  * attn_fwd_save wrote for the same q, k, rope tables, cu_seqlens and sizes,
  * unchanged since; results are then identical to attn_bwd_gqa's. That
- * correspondence is the caller's contract and is not checked.
+ * correspondence is the caller's contract and is not checked; the kernels
+ * clamp every document range they read from it into its own row, so a buffer
+ * that breaks the contract gives wrong results, never an out-of-range access.
  * For both: when attn_saved_bytes is 0, or saved is NULL, the call is the
  * plain attn_fwd_gqa / attn_bwd_gqa and `saved` is not touched. Misaligned
  * saved: ATTN_EALIGN; saved_bytes too small: ATTN_EWORKSPACE. The buffer
