@@ -8,7 +8,9 @@ long-context window B=1, H=16, T=8192, D=128 with RoPE), inputs resident in
 HBM: attn_fwd_save + attn_bwd_saved, the forward's rotated q, k kept for the
 backward as a training step keeps its activations (--no-save: the plain
 attn_fwd + attn_bwd, which rotate q, k in both calls). Each timed step is bracketed by CUDA events on the launching stream; L2
-is flushed (a 256 MiB write) between steps, outside the events. FLOPs follow
+is flushed (a 256 MiB write) between steps, outside the events; warm-up steps
+repeat the timed sequence (flush included) and the NVML clock sampler starts
+before them, keeping samples of the timed steps only. FLOPs follow
 the nominal convention 4*B*H*T^2*D/2 forward and 2.5x that backward
 (7*B*H*T^2*D per step; for packed documents the within-document figure is
 reported beside it). With N > 1 (torchrun, one process per GPU) every rank
@@ -190,13 +192,26 @@ class ClockSampler:
                (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"),
                (0x2, "applications_clocks_setting"), (0x1, "gpu_idle")]
 
-    def __init__(self, index: int, period_s: float = 0.02):
+    def __init__(self, index: int, period_s: float = 0.01, gated: bool = False):
+        """Samples every ``period_s`` seconds on a thread of its own. With
+        ``gated`` the thread starts (and NVML is initialised) on entry but
+        keeps samples only between ``on()`` and ``off()``: entered before the
+        warm-up, so nothing of its start-up falls into the timed steps."""
         self.index, self.period = index, period_s
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.power_w = []
         self._stop = threading.Event()
+        self._keep = threading.Event()
+        if not gated:
+            self._keep.set()
         self._thr = None
         self.error = None
+
+    def on(self):
+        self._keep.set()
+
+    def off(self):
+        self._keep.clear()
 
     def __enter__(self):
         try:
@@ -205,24 +220,32 @@ class ClockSampler:
             self._nv = pynvml
             self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._query()  # first calls resolve NVML's entry points: keep them here
             self._thr = threading.Thread(target=self._run, daemon=True)
             self._thr.start()
         except Exception as e:  # NVML missing: report no clocks rather than guess
             self.error = repr(e)
         return self
 
-    def _run(self):
+    def _query(self):
         nv = self._nv
+        mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+        watts = nv.nvmlDeviceGetPowerUsage(self._h) / 1000.0
+        mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h) \
+            if hasattr(nv, "nvmlDeviceGetCurrentClocksEventReasons") \
+            else nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+        return mhz, watts, mask
+
+    def _run(self):
         while not self._stop.is_set():
             try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                self.power_w.append(nv.nvmlDeviceGetPowerUsage(self._h) / 1000.0)
-                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h) \
-                    if hasattr(nv, "nvmlDeviceGetCurrentClocksEventReasons") \
-                    else nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
-                for bit, name in self.REASONS:
-                    if mask & bit:
-                        self.reasons.add(name)
+                mhz, watts, mask = self._query()
+                if self._keep.is_set():
+                    self.samples.append(mhz)
+                    self.power_w.append(watts)
+                    for bit, name in self.REASONS:
+                        if mask & bit:
+                            self.reasons.add(name)
             except Exception as e:
                 self.error = repr(e)
                 break
@@ -420,22 +443,27 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     flops_step = 7.0 * w.B * w.H * w.T * w.T * w.D
 
-    with torch.cuda.stream(stream):
-        for _ in range(max(args.warmup, 0)):
-            r.forward()
-            r.backward()
-    st = r.status()
-    if st != A.ATTN_OK:
-        raise SystemExit(f"device status after warm-up: {A.error_string(st)}")
+    # The clock sampler starts before the warm-up (its start-up stays out of
+    # the timed steps) and keeps samples of the timed region only; warm-up
+    # steps are the timed steps' exact sequence, flush included.
+    with ClockSampler(local, gated=True) as clocks:
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 0)):
+                flush.zero_()
+                r.forward()
+                r.backward()
+        st = r.status()
+        if st != A.ATTN_OK:
+            raise SystemExit(f"device status after warm-up: {A.error_string(st)}")
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    torch.cuda.synchronize(dev)
-    barrier()
-    torch.cuda.synchronize(dev)
-    A.check(A.attn_tile_counts()[0], "attn_tile_counts")  # reset the device counters
-    n0 = A.attn_launch_count()
-    with ClockSampler(local) as clocks:
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        torch.cuda.synchronize(dev)
+        barrier()
+        torch.cuda.synchronize(dev)
+        A.check(A.attn_tile_counts()[0], "attn_tile_counts")  # reset the device counters
+        n0 = A.attn_launch_count()
+        clocks.on()
         with torch.cuda.stream(stream):
             for i in range(args.steps):
                 flush.zero_()
@@ -444,6 +472,7 @@ def run_ours(args):
                 r.backward()
                 ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
+        clocks.off()
     barrier()
     torch.cuda.synchronize(dev)
     launches = A.attn_launch_count() - n0
@@ -688,16 +717,18 @@ def run_decode(args):
     r = DecodeRunner(w, device=dev, stream=stream)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     peaks, peak_src = load_peaks()
-    with torch.cuda.stream(stream):
-        for _ in range(max(args.warmup, 0)):
-            r.run()
-    if r.status() != A.ATTN_OK:
-        raise SystemExit("device status after warm-up is not OK")
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    torch.cuda.synchronize(dev)
-    n0 = A.attn_launch_count()
-    with ClockSampler(0) as clocks:
+    with ClockSampler(0, gated=True) as clocks:  # started before the warm-up, as above
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 0)):
+                flush.zero_()
+                r.run()
+        if r.status() != A.ATTN_OK:
+            raise SystemExit("device status after warm-up is not OK")
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        torch.cuda.synchronize(dev)
+        n0 = A.attn_launch_count()
+        clocks.on()
         with torch.cuda.stream(stream):
             for i in range(args.steps):
                 flush.zero_()
@@ -705,6 +736,7 @@ def run_decode(args):
                 r.run()
                 ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
+        clocks.off()
     launches = A.attn_launch_count() - n0
     # per-kernel times from a separate pass (events around every launch)
     A.check(A.attn_profile_enable(1), "attn_profile_enable")
@@ -768,16 +800,18 @@ def run_proj(args):
         r.out_bwd()
         r.qkv_bwd()
 
-    with torch.cuda.stream(stream):
-        for _ in range(max(args.warmup, 0)):
-            step()
-    if r.status() != A.ATTN_OK:
-        raise SystemExit("device status after warm-up is not OK")
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    torch.cuda.synchronize(dev)
-    n0 = A.attn_launch_count()
-    with ClockSampler(0) as clocks:
+    with ClockSampler(0, gated=True) as clocks:  # started before the warm-up, as above
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 0)):
+                flush.zero_()
+                step()
+        if r.status() != A.ATTN_OK:
+            raise SystemExit("device status after warm-up is not OK")
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        torch.cuda.synchronize(dev)
+        n0 = A.attn_launch_count()
+        clocks.on()
         with torch.cuda.stream(stream):
             for i in range(args.steps):
                 flush.zero_()
@@ -785,6 +819,7 @@ def run_proj(args):
                 step()
                 ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
+        clocks.off()
     launches = A.attn_launch_count() - n0
     A.check(A.attn_profile_enable(1), "attn_profile_enable")
     with torch.cuda.stream(stream):
