@@ -304,13 +304,13 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
 
 template <int D, bool kF16, bool kDQ>
 int launch_dkdv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                const CUtensorMap& mo, const CUtensorMap& mdq, const bwd100::Params& prm,
-                unsigned grid, cudaStream_t st) {
+                const CUtensorMap& mo, const CUtensorMap& mdq, const CUtensorMap& mdk,
+                const CUtensorMap& mdv, const bwd100::Params& prm, unsigned grid, cudaStream_t st) {
   using L = bwd100::Layout<D, kDQ>;
   static bool smem_set[64] = {};
   if (!ensure_smem(bwd100::dkdv_kernel<D, kF16, kDQ>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
   ATTN_LAUNCH(KK_DKDV, st, pdl_launch(bwd100::dkdv_kernel<D, kF16, kDQ>, grid, L::kThreads,
-                                       L::kSmemAlloc, st, mq, mk, mv, mo, mdq, prm));
+                                       L::kSmemAlloc, st, mq, mk, mv, mo, mdq, mdk, mdv, prm));
   return launch_status();
 }
 
@@ -418,10 +418,11 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
                                        dq_pass ? nullptr : dq_acc, dk_acc, dv_acc,
                                        (const __nv_bfloat16*)v, hstat, H, Hkv, T, Tpad, rows_pad));
   if (launch_status()) return ATTN_ECUDA;
-  CUtensorMap mq, mk, mv, mo, mdq;
+  CUtensorMap mq, mk, mv, mo, mdq, mdk, mdv;
   if (!make_tile_map(&mq, qs, f16, D, T, BH) || !make_tile_map(&mk, ks, f16, D, T, BHkv) ||
       !make_tile_map(&mv, v, false, D, T, BHkv) || !make_tile_map(&mo, dO, false, D, T, BH) ||
-      !make_acc_map(&mdq, dq_acc, D, T, BH))
+      !make_acc_map(&mdq, dq_acc, D, T, BH) || !make_tile_map(&mdk, dk, false, D, T, BHkv) ||
+      !make_tile_map(&mdv, dv, false, D, T, BHkv))
     return ATTN_ECUDA;
   bwd100::Params prm;
   prm.T = T;
@@ -454,11 +455,11 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
       rc_k = f16 ? launch_dkdv_pair<true>(qs, dO, mq, mk, mv, mo, prm, T, BH, st)
                  : launch_dkdv_pair<false>(qs, dO, mq, mk, mv, mo, prm, T, BH, st);
   } else if (dq_pass)
-    rc_k = f16 ? launch_dkdv<D, true, false>(mq, mk, mv, mo, mdq, prm, grid, st)
-               : launch_dkdv<D, false, false>(mq, mk, mv, mo, mdq, prm, grid, st);
+    rc_k = f16 ? launch_dkdv<D, true, false>(mq, mk, mv, mo, mdq, mdk, mdv, prm, grid, st)
+               : launch_dkdv<D, false, false>(mq, mk, mv, mo, mdq, mdk, mdv, prm, grid, st);
   else
-    rc_k = f16 ? launch_dkdv<D, true, true>(mq, mk, mv, mo, mdq, prm, grid, st)
-               : launch_dkdv<D, false, true>(mq, mk, mv, mo, mdq, prm, grid, st);
+    rc_k = f16 ? launch_dkdv<D, true, true>(mq, mk, mv, mo, mdq, mdk, mdv, prm, grid, st)
+               : launch_dkdv<D, false, true>(mq, mk, mv, mo, mdq, mdk, mdv, prm, grid, st);
   if (rc_k) return rc_k;
   if (split > 1) {
     // dk = R^T (scale * sum of the parts), dv = sum of the parts

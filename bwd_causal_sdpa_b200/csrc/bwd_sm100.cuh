@@ -167,7 +167,8 @@ template <int D, bool kF16, bool kDQ>
 __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                const __grid_constant__ CUtensorMap tmDQ, const Params p) {
+                const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
+                const __grid_constant__ CUtensorMap tmDV, const Params p) {
   pdl_wait_and_trigger();
   using L = Layout<D, kDQ>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -830,7 +831,8 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
     ok = ok && phase_dS(0);
     for (int it = 1; ok && it < n_it; ++it) ok = phase_P(it) && phase_dS(it);
     // ---- epilogue: dK = R^T (scale * dK_r), dV ----
-    if (ok && mbar_wait(bar(L::bFinal), 0, abort_flag)) {
+    const bool epi = ok && mbar_wait(bar(L::bFinal), 0, abort_flag);
+    if (epi) {
       tc_fence_after();
       const int jj = min(j, T - 1);
       const int pos = jj - (p.doc_start ? min(max(p.doc_start[row0 + jj] - row0, 0), jj) : 0);
@@ -867,40 +869,91 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
           }
         }
       } else {
+      // dK and dV leave as bf16 through the two Q stages (free once the last
+      // dK product has read its Q tile) and TMA stores: one 16-byte chunk per
+      // lane and key row into the maps' 128-byte swizzle, where stores to
+      // global memory from one key row per lane took 32 cache lines per
+      // instruction and, with the RoPE table loads, held up the dQ warps'
+      // last drain on the shared load/store path. The row's table entries
+      // are requested first; 16 columns per TMEM load keep them and the
+      // accumulator values within the register budget.
+      constexpr int HC = 16;
+      static_assert(DC % HC == 0, "16-column pieces");
+      float4 rcos[DC / 8], rsin[DC / 8];
+      if (p.rope_cos) {
+        const float4* c4 = reinterpret_cast<const float4*>(p.rope_cos + (size_t)pos * (D / 2) + (dc0 >> 1));
+        const float4* s4 = reinterpret_cast<const float4*>(p.rope_sin + (size_t)pos * (D / 2) + (dc0 >> 1));
 #pragma unroll
-      for (int c = 0; c < DC / CW; ++c) {
-        const int col = dc0 + CW * c;
-        uint32_t v[CW];
-        ld(tmem + lane_base + L::kColDK + col, v);
-        tmem_wait_ld();
-        float f[CW];
-#pragma unroll
-        for (int e = 0; e < CW; ++e) f[e] = __uint_as_float(v[e]) * (p.scale * inv_c);
-        if (p.rope_cos) rope_pairs<CW, D>(f, p.rope_cos, p.rope_sin, pos, col, true);
-        if (j < T) {
-#pragma unroll
-          for (int e = 0; e < CW / 8; ++e)
-            reinterpret_cast<uint4*>(dkrow + col)[e] =
-                make_uint4(pack_bf16(f[8 * e], f[8 * e + 1]), pack_bf16(f[8 * e + 2], f[8 * e + 3]),
-                           pack_bf16(f[8 * e + 4], f[8 * e + 5]), pack_bf16(f[8 * e + 6], f[8 * e + 7]));
+        for (int q = 0; q < DC / 8; ++q) {
+          rcos[q] = c4[q];
+          rsin[q] = s4[q];
         }
       }
+      uint8_t* stage_dk = sg + L::kQ;                  // 128 rows x D bf16, 64-column blocks
+      uint8_t* stage_dv = sg + L::kQ + L::kTileBytes;
 #pragma unroll
-      for (int c = 0; c < DC / CW; ++c) {
-        const int col = dc0 + CW * c;
-        uint32_t v[CW];
-        ld(tmem + lane_base + L::kColDV + col, v);
+      for (int c = 0; c < DC / HC; ++c) {
+        const int col = dc0 + HC * c;
+        uint32_t v[HC];
+        tmem_ld16(tmem + lane_base + L::kColDV + col, v);
         tmem_wait_ld();
-        if (j < T) {
+        uint8_t* blk = stage_dv + (col >> 6) * L::kBlockBytes;
 #pragma unroll
-          for (int e = 0; e < CW / 8; ++e)
-            reinterpret_cast<uint4*>(dvrow + col)[e] = make_uint4(
-                pack_bf16(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
-                pack_bf16(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
-                pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
-                pack_bf16(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
-        }
+        for (int e = 0; e < HC / 8; ++e)
+          *reinterpret_cast<uint4*>(blk + sw128(r, ((col & 63) >> 3) + e)) = make_uint4(
+              pack_bf16(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
+              pack_bf16(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
+              pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
+              pack_bf16(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
       }
+#pragma unroll
+      for (int c = 0; c < DC / HC; ++c) {
+        const int col = dc0 + HC * c;
+        uint32_t v[HC];
+        tmem_ld16(tmem + lane_base + L::kColDK + col, v);
+        tmem_wait_ld();
+        float f[HC];
+#pragma unroll
+        for (int e = 0; e < HC; ++e) f[e] = __uint_as_float(v[e]) * (p.scale * inv_c);
+        if (p.rope_cos) {
+          // inverse rotation, the same roundings as rope_pairs
+#pragma unroll
+          for (int q = 0; q < HC / 8; ++q) {
+            const float4 cq = rcos[c * (HC / 8) + q], sq = rsin[c * (HC / 8) + q];
+            const float cs[4] = {cq.x, cq.y, cq.z, cq.w};
+            const float sn[4] = {-sq.x, -sq.y, -sq.z, -sq.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float x0 = f[8 * q + 2 * e], x1 = f[8 * q + 2 * e + 1];
+              f[8 * q + 2 * e] = fmaf(x0, cs[e], -__fmul_rn(x1, sn[e]));
+              f[8 * q + 2 * e + 1] = fmaf(x0, sn[e], __fmul_rn(x1, cs[e]));
+            }
+          }
+        }
+        uint8_t* blk = stage_dk + (col >> 6) * L::kBlockBytes;
+#pragma unroll
+        for (int e = 0; e < HC / 8; ++e)
+          *reinterpret_cast<uint4*>(blk + sw128(r, ((col & 63) >> 3) + e)) =
+              make_uint4(pack_bf16(f[8 * e], f[8 * e + 1]), pack_bf16(f[8 * e + 2], f[8 * e + 3]),
+                         pack_bf16(f[8 * e + 4], f[8 * e + 5]), pack_bf16(f[8 * e + 6], f[8 * e + 7]));
+      }
+      fence_proxy_async_smem();
+      }
+    }
+    if (p.n_split <= 1) {
+      // every elementwise thread arrives (an aborted one too, so none waits
+      // for ever); the staged rows then leave in 64-column boxes, rows past
+      // T clipped by the maps. Before the CTA leaves its boxes must have
+      // been read; the writes complete with the grid.
+      asm volatile("barrier.sync 2, %0;" ::"n"(L::kEwThreads) : "memory");
+      if (warp == 0 && lane == 0 && epi) {
+#pragma unroll
+        for (int bcol = 0; bcol < D / 64; ++bcol) {
+          tma_store_3d(&tmDK, sb0 + L::kQ + bcol * L::kBlockBytes, 64 * bcol, j0, bhk);
+          tma_store_3d(&tmDV, sb0 + L::kQ + L::kTileBytes + bcol * L::kBlockBytes, 64 * bcol, j0, bhk);
+        }
+        bulk_commit_group();
+        bulk_wait_group_read0();
       }
     }
   }

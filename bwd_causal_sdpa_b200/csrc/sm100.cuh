@@ -146,6 +146,16 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32
       "r"(src), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+// Tensor store of a shared-memory box into global memory through a tensor map;
+// coordinates must be non-negative (rows past the end are clipped).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                             int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
 // Vector fp32 reduce-add of four values into global memory (16-byte aligned).
 __device__ __forceinline__ void red_add_v4(float* p, uint32_t a, uint32_t b, uint32_t c,
                                            uint32_t d) {
