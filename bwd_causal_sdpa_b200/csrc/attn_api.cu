@@ -277,9 +277,9 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
     ks = kh;
   }
   const bool f16 = rc != nullptr;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_tile_map(&mq, qs, f16, D, T, BH) || !make_tile_map(&mk, ks, f16, D, T, BHkv, L::kKV) ||
-      !make_tile_map(&mv, v, false, D, T, BHkv, L::kKV))
+      !make_tile_map(&mv, v, false, D, T, BHkv, L::kKV) || !make_tile_map(&mo, o, false, D, T, BH))
     return ATTN_ECUDA;
   static bool smem_set[64] = {};
   if (!ensure_smem(fwd100::fwd_kernel<D>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
@@ -298,7 +298,7 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
   prm.doc_start = ds;
   prm.o = (__nv_bfloat16*)o;
   prm.lse = lse;
-  ATTN_LAUNCH(KK_FWD, st, pdl_launch(fwd100::fwd_kernel<D>, (unsigned)(n_pairs * BH), L::kThreads, L::kSmemAlloc, st, mq, mk, mv, prm));
+  ATTN_LAUNCH(KK_FWD, st, pdl_launch(fwd100::fwd_kernel<D>, (unsigned)(n_pairs * BH), L::kThreads, L::kSmemAlloc, st, mq, mk, mv, mo, prm));
   return launch_status();
 }
 

@@ -90,6 +90,12 @@ struct Layout {
   static_assert(kPolyPairs >= 0 && kPolyPairs <= 32, "poly share");
 };
 
+// Byte offset of 16-byte chunk `ch` (0..7 within a 64-column block) of row r
+// in a 128-byte-swizzled tile block (the layout of the tensor maps' boxes).
+__device__ __forceinline__ uint32_t sw128(int r, int ch) {
+  return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4));
+}
+
 struct Params {
   int T, H, Hkv, BH, n_pairs, n_qtiles;  // H query heads read Hkv key/value heads
   float scale_log2;          // scale * log2(e)
@@ -106,7 +112,8 @@ struct Params {
 template <int D>
 __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const Params p) {
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+               const Params p) {
   pdl_wait_and_trigger();
   using L = Layout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -399,27 +406,44 @@ __global__ void __launch_bounds__(Layout<D>::kThreads, 1)
       if (lane == 0) mbar_arrive(bar(L::bPFull + 2 * t + (li & 1)));
       kf = kf_next;
     }
-    if (ok && mbar_wait(bar(L::bOFinal + t), 0, abort_flag)) {
+    // O / l leaves as bf16 through this tile's Q buffer (no product reads
+    // it once O is final) and TMA stores of 64-column boxes, rows past T
+    // clipped by the map: stores to global memory from one query row per
+    // lane took 32 cache lines per instruction.
+    const bool epi = ok && mbar_wait(bar(L::bOFinal + t), 0, abort_flag);
+    uint8_t* stage = sg + L::kQ + t * L::kQTileBytes;
+    if (epi) {
       tc_fence_after();
       const float inv = 1.f / l;
-      __nv_bfloat16* orow = p.o + ((size_t)bh * T + min(i, T - 1)) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
         tmem_ld32(tO + 32 * c, ov);  // warp-collective
         tmem_wait_ld();
-        if (i < T) {
-          uint32_t pk[16];
+        uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
+        uint8_t* blk = stage + ((32 * c) >> 6) * L::kQBlockBytes;
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-        }
+        for (int e = 0; e < 4; ++e)
+          *reinterpret_cast<uint4*>(blk + sw128(r, (((32 * c) & 63) >> 3) + e)) =
+              make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
       }
+      fence_proxy_async_smem();
       if (i < T) p.lse[(size_t)bh * T + i] = (m + __log2f(l)) * 0.69314718055994531f;
+    }
+    // the tile's four warps all arrive (an aborted or idle one too, so none
+    // waits for ever); before the CTA leaves the boxes must have been read,
+    // the writes complete with the grid
+    if (t == 0) asm volatile("barrier.sync 2, 128;" ::: "memory");
+    else asm volatile("barrier.sync 3, 128;" ::: "memory");
+    if ((warp & 3) == 0 && lane == 0 && epi) {
+#pragma unroll
+      for (int bcol = 0; bcol < D / 64; ++bcol)
+        tma_store_3d(&tmO, smem_u32(stage) + bcol * L::kQBlockBytes, 64 * bcol, qt * 128, bh);
+      bulk_commit_group();
+      bulk_wait_group_read0();
     }
   }
 
