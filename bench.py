@@ -45,20 +45,20 @@ FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # one ncu capture of the kernel on the workload, valid only while the kernel
 # sources still hash to what was captured (sha256, first 16 hex digits).
 MEASURED_TRAFFIC = {
-    ("dkdv", "long_context_8k"): (672.3e6, {"bwd_sm100.cuh": "073cb8d91447bbbf",
-                                            "sm100.cuh": "efe40f0294c09366",
+    ("dkdv", "long_context_8k"): (680.4e6, {"bwd_sm100.cuh": "bc038325f3265979",
+                                            "sm100.cuh": "d00797b7a9dd3426",
                                             "common.cuh": "36b3720cacd61ee7"}),
-    ("dkdv", "decoder237m_layer"): (122.0e6, {"bwd_sm100.cuh": "073cb8d91447bbbf",
-                                              "sm100.cuh": "efe40f0294c09366",
+    ("dkdv", "decoder237m_layer"): (124.0e6, {"bwd_sm100.cuh": "bc038325f3265979",
+                                              "sm100.cuh": "d00797b7a9dd3426",
                                               "common.cuh": "36b3720cacd61ee7"}),
-    ("fwd", "long_context_8k"): (155.6e6, {"fwd_sm100.cuh": "7b9df616ca1a18a1",
-                                           "sm100.cuh": "efe40f0294c09366",
+    ("fwd", "long_context_8k"): (157.7e6, {"fwd_sm100.cuh": "1342fca937c6151e",
+                                           "sm100.cuh": "d00797b7a9dd3426",
                                            "common.cuh": "36b3720cacd61ee7"}),
-    ("fwd", "decoder237m_layer"): (50.4e6, {"fwd_sm100.cuh": "7b9df616ca1a18a1",
-                                            "sm100.cuh": "efe40f0294c09366",
+    ("fwd", "decoder237m_layer"): (50.4e6, {"fwd_sm100.cuh": "1342fca937c6151e",
+                                            "sm100.cuh": "d00797b7a9dd3426",
                                             "common.cuh": "36b3720cacd61ee7"}),
-    ("decode", "decode_8k_gqa"): (204.2e6, {"decode.cuh": "ed672db8f3155da3",
-                                            "sm100.cuh": "efe40f0294c09366",
+    ("decode", "decode_8k_gqa"): (200.6e6, {"decode.cuh": "ed672db8f3155da3",
+                                            "sm100.cuh": "d00797b7a9dd3426",
                                             "common.cuh": "36b3720cacd61ee7"}),
 }
 
