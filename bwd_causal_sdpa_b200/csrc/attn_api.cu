@@ -464,9 +464,9 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
   if (split > 1) {
     // dk = R^T (scale * sum of the parts), dv = sum of the parts
     const long n8kv = (long)BHkv * T * D / 8;
-    ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)((n8kv + 255) / 256), 256, 0, st, dk_acc, rc, rs, ds, (__nv_bfloat16*)dk, Hkv, T, scale, n8kv, (const float*)nullptr, (const float*)nullptr, Hkv, nt));
+    ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)(((n8kv + 1) / 2 + 255) / 256), 256, 0, st, dk_acc, rc, rs, ds, (__nv_bfloat16*)dk, Hkv, T, scale, n8kv, (const float*)nullptr, (const float*)nullptr, Hkv, nt));
     if (launch_status()) return ATTN_ECUDA;
-    ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)((n8kv + 255) / 256), 256, 0, st, dv_acc, nullptr, nullptr, nullptr, (__nv_bfloat16*)dv, Hkv, T, 1.0f, n8kv, (const float*)nullptr, (const float*)nullptr, Hkv, nt));
+    ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)(((n8kv + 1) / 2 + 255) / 256), 256, 0, st, dv_acc, nullptr, nullptr, nullptr, (__nv_bfloat16*)dv, Hkv, T, 1.0f, n8kv, (const float*)nullptr, (const float*)nullptr, Hkv, nt));
     if (launch_status()) return ATTN_ECUDA;
   }
   if (dq_pass) {
@@ -493,7 +493,7 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
                : launch_dq<D, false>(mq, mk, mv, mo, qp, qgrid, st);
   }
   const long n8 = (long)BH * T * D / 8;
-  ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)((n8 + 255) / 256), 256, 0, st, dq_acc, rc, rs, ds, (__nv_bfloat16*)dq, H, T, scale, n8, f16 ? (const float*)qinv : nullptr, (const float*)hstat, Hkv, nt));
+  ATTN_LAUNCH(KK_DQ_FINALIZE, st, pdl_launch(dq_finalize_kernel<D>, (unsigned)(((n8 + 1) / 2 + 255) / 256), 256, 0, st, dq_acc, rc, rs, ds, (__nv_bfloat16*)dq, H, T, scale, n8, f16 ? (const float*)qinv : nullptr, (const float*)hstat, Hkv, nt));
   return launch_status();
 }
 

@@ -289,7 +289,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
   }
 }
 
-// dq = R(pos)^T (scale * dq_acc), stored as bf16; one thread per 8 values.
+// dq = R(pos)^T (scale * dq_acc), stored as bf16; one thread per two groups
+// of 8 values, half the array apart (both loads in flight at once; the grid
+// covers ceil(n8 / 2) threads).
 // With fp16 operands (qinv non-null) the accumulator holds Cg qinv_i dS K for
 // query tile i (Cg per key/value head, in the fourth statistics slot of its
 // index), which is divided out here. The same pass finishes split dk, dv
@@ -301,29 +303,40 @@ __global__ void __launch_bounds__(256) dq_finalize_kernel(
     float scale, long n8, const float* __restrict__ qinv, const float* __restrict__ hstat,
     int Hkv, int ntiles) {
   pdl_wait_and_trigger();
+  const long half = (n8 + 1) >> 1;
   const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= n8) return;
-  const long e0 = idx * 8;
-  const long row = e0 / D;  // bh*T + t
-  const int d0 = (int)(e0 - row * D);
-  const int t = (int)(row % T);
-  const int bh = (int)(row / T);
-  const int b = bh / H;
-  float f = scale;
-  if (qinv) {
-    const int bhk = b * Hkv + (bh - b * H) / (H / Hkv);
-    f /= hstat[4 * bhk + 3] * qinv[((size_t)bh * ntiles + (t >> 7)) * 4];
-  }
-  float v[8];
-  load_vec<4>(dq_acc + e0, v);
-  load_vec<4>(dq_acc + e0 + 4, v + 4);
+  if (idx >= half) return;
+  const bool two = idx + half < n8;
+  float v[2][8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) v[e] *= f;
-  if (rc) {
-    // clamped into the row (the ranges may come from the caller's saved buffer)
-    const int pos = t - (doc_start ? min(max(doc_start[b * T + t] - b * T, 0), t) : 0);
-    rope_pairs<8, D>(v, rc, rs, pos, d0, true);
+  for (int g = 0; g < 2; ++g) {
+    if (g == 1 && !two) break;
+    const long e0 = (idx + g * half) * 8;
+    load_vec<4>(dq_acc + e0, v[g]);
+    load_vec<4>(dq_acc + e0 + 4, v[g] + 4);
   }
-  store_vec<4>(dq + e0, v);
-  store_vec<4>(dq + e0 + 4, v + 4);
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    if (g == 1 && !two) break;
+    const long e0 = (idx + g * half) * 8;
+    const long row = e0 / D;  // bh*T + t
+    const int d0 = (int)(e0 - row * D);
+    const int t = (int)(row % T);
+    const int bh = (int)(row / T);
+    const int b = bh / H;
+    float f = scale;
+    if (qinv) {
+      const int bhk = b * Hkv + (bh - b * H) / (H / Hkv);
+      f /= hstat[4 * bhk + 3] * qinv[((size_t)bh * ntiles + (t >> 7)) * 4];
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[g][e] *= f;
+    if (rc) {
+      // clamped into the row (the ranges may come from the caller's saved buffer)
+      const int pos = t - (doc_start ? min(max(doc_start[b * T + t] - b * T, 0), t) : 0);
+      rope_pairs<8, D>(v[g], rc, rs, pos, d0, true);
+    }
+    store_vec<4>(dq + e0, v[g]);
+    store_vec<4>(dq + e0 + 4, v[g] + 4);
+  }
 }
