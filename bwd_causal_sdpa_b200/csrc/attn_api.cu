@@ -155,6 +155,20 @@ bool make_tile_map(CUtensorMap* m, const void* base, bool is_f16, int D, int T, 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A RoPE table ([T][D/2] fp32) seen in boxes of 128 rows x 32 floats with the
+// 128-byte swizzle; rows past T read as zeros.
+bool make_table_map(CUtensorMap* m, const float* base, int D, int T) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)(D / 2), (cuuint64_t)T, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)(D / 2) * 4, (cuuint64_t)T * (D / 2) * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // The fp32 [B*H][T][D] dq accumulator seen in boxes of 32 rows x 32 columns
 // (128-byte swizzle) for tensor reduce-add; rows past T are clipped.
 bool make_acc_map(CUtensorMap* m, float* base, int D, int T, int BH) {
@@ -305,12 +319,13 @@ int fwd_tc(const void* q, const void* k, const void* v, const float* rc, const f
 template <int D, bool kF16, bool kDQ>
 int launch_dkdv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                 const CUtensorMap& mo, const CUtensorMap& mdq, const CUtensorMap& mdk,
-                const CUtensorMap& mdv, const bwd100::Params& prm, unsigned grid, cudaStream_t st) {
+                const CUtensorMap& mdv, const CUtensorMap& mrc, const CUtensorMap& mrs,
+                const bwd100::Params& prm, unsigned grid, cudaStream_t st) {
   using L = bwd100::Layout<D, kDQ>;
   static bool smem_set[64] = {};
   if (!ensure_smem(bwd100::dkdv_kernel<D, kF16, kDQ>, L::kSmemAlloc, smem_set)) return ATTN_ECUDA;
   ATTN_LAUNCH(KK_DKDV, st, pdl_launch(bwd100::dkdv_kernel<D, kF16, kDQ>, grid, L::kThreads,
-                                       L::kSmemAlloc, st, mq, mk, mv, mo, mdq, mdk, mdv, prm));
+                                       L::kSmemAlloc, st, mq, mk, mv, mo, mdq, mdk, mdv, mrc, mrs, prm));
   return launch_status();
 }
 
@@ -424,6 +439,10 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
       !make_acc_map(&mdq, dq_acc, D, T, BH) || !make_tile_map(&mdk, dk, false, D, T, BHkv) ||
       !make_tile_map(&mdv, dv, false, D, T, BHkv))
     return ATTN_ECUDA;
+  // the RoPE tables for the key-tile epilogue (without RoPE the kernel does
+  // not read them: any valid map stands in)
+  CUtensorMap mrc = mdk, mrs = mdk;
+  if (rc && (!make_table_map(&mrc, rc, D, T) || !make_table_map(&mrs, rs, D, T))) return ATTN_ECUDA;
   bwd100::Params prm;
   prm.T = T;
   prm.H = H;
@@ -455,11 +474,11 @@ int bwd_tc(const void* q, const void* k, const void* v, const void* o, const voi
       rc_k = f16 ? launch_dkdv_pair<true>(qs, dO, mq, mk, mv, mo, prm, T, BH, st)
                  : launch_dkdv_pair<false>(qs, dO, mq, mk, mv, mo, prm, T, BH, st);
   } else if (dq_pass)
-    rc_k = f16 ? launch_dkdv<D, true, false>(mq, mk, mv, mo, mdq, mdk, mdv, prm, grid, st)
-               : launch_dkdv<D, false, false>(mq, mk, mv, mo, mdq, mdk, mdv, prm, grid, st);
+    rc_k = f16 ? launch_dkdv<D, true, false>(mq, mk, mv, mo, mdq, mdk, mdv, mrc, mrs, prm, grid, st)
+               : launch_dkdv<D, false, false>(mq, mk, mv, mo, mdq, mdk, mdv, mrc, mrs, prm, grid, st);
   else
-    rc_k = f16 ? launch_dkdv<D, true, true>(mq, mk, mv, mo, mdq, mdk, mdv, prm, grid, st)
-               : launch_dkdv<D, false, true>(mq, mk, mv, mo, mdq, mdk, mdv, prm, grid, st);
+    rc_k = f16 ? launch_dkdv<D, true, true>(mq, mk, mv, mo, mdq, mdk, mdv, mrc, mrs, prm, grid, st)
+               : launch_dkdv<D, false, true>(mq, mk, mv, mo, mdq, mdk, mdv, mrc, mrs, prm, grid, st);
   if (rc_k) return rc_k;
   if (split > 1) {
     // dk = R^T (scale * sum of the parts), dv = sum of the parts

@@ -92,8 +92,14 @@ struct Layout {
   static constexpr int bQFull = 1, bQEmpty = 3, bDOFull = 5, bDOEmpty = 7;  // 2 each
   static constexpr int bSFull = 9, bSFree = 10, bPFull = 11, bDPFull = 12, bDSFull = 13,
                        bDVDone = 14, bDQFull = 15, bDSFree = 16, bDQFree = 17, bFinal = 18,
-                       bStats = 19;
-  static constexpr int kNumBars = 20;
+                       bStats = 19, bTab = 20;
+  static constexpr int kNumBars = 21;
+  // RoPE table rows of a key tile that lies in one document, for the dK
+  // epilogue: cos into the V tile, sin into the dO stages (both unread once
+  // the last dV product is done), 128 rows x D/2 floats each in boxes of
+  // 32 floats with the 128-byte swizzle.
+  static constexpr int kTabBytes = 128 * (D / 2) * 4;
+  static_assert(kTabBytes <= kTileBytes && kTabBytes <= kDOStages * kTileBytes, "table rows fit");
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
   // The dynamic shared-memory window starts 1024-byte aligned on sm_100 (after
@@ -168,7 +174,8 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                 const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
-                const __grid_constant__ CUtensorMap tmDV, const Params p) {
+                const __grid_constant__ CUtensorMap tmDV, const __grid_constant__ CUtensorMap tmRC,
+                const __grid_constant__ CUtensorMap tmRS, const Params p) {
   pdl_wait_and_trigger();
   using L = Layout<D, kDQ>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -222,6 +229,7 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
     mbar_init(bar(L::bDSFree), 1);
     mbar_init(bar(L::bDQFree), 128);
     mbar_init(bar(L::bFinal), 1);
+    mbar_init(bar(L::bTab), 1);
     // C is made by the dQ warpgroup when there is one (it is idle until the
     // first dQ), else by the elementwise warps
     mbar_init(bar(L::bStats), kDQ ? 128 : L::kEwThreads);
@@ -832,12 +840,24 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
     for (int it = 1; ok && it < n_it; ++it) ok = phase_P(it) && phase_dS(it);
     // ---- epilogue: dK = R^T (scale * dK_r), dV ----
     const bool epi = ok && mbar_wait(bar(L::bFinal), 0, abort_flag);
+    // one document over the whole key tile (uniform across the CTA): its
+    // table rows are consecutive from pos0
+    const int jl = min(j0 + 127, T - 1);
+    const int ds0 = p.doc_start ? min(max(p.doc_start[row0 + j0] - row0, 0), j0) : 0;
+    const bool tab_tma = p.rope_cos != nullptr && p.n_split <= 1 &&
+                         (!p.doc_start || min(max(p.doc_start[row0 + jl] - row0, 0), jl) == ds0);
+    if (tab_tma && warp == 0 && lane == 0 && epi) {
+      mbar_arrive_expect_tx(bar(L::bTab), 2 * L::kTabBytes);
+#pragma unroll
+      for (int bx = 0; bx < D / 64; ++bx) {
+        tma_load_3d(sb0 + L::kV + bx * (128 * 128), &tmRC, bar(L::bTab), 32 * bx, j0 - ds0, 0);
+        tma_load_3d(sb0 + L::kDO + bx * (128 * 128), &tmRS, bar(L::bTab), 32 * bx, j0 - ds0, 0);
+      }
+    }
     if (epi) {
       tc_fence_after();
       const int jj = min(j, T - 1);
       const int pos = jj - (p.doc_start ? min(max(p.doc_start[row0 + jj] - row0, 0), jj) : 0);
-      __nv_bfloat16* dkrow = p.dk + ((size_t)bhk * T + jj) * D;
-      __nv_bfloat16* dvrow = p.dv + ((size_t)bhk * T + jj) * D;
       constexpr int CW = DC < 32 ? DC : 32;  // columns per TMEM load
       auto ld = [&](uint32_t taddr, uint32_t* v) {
         if constexpr (CW == 32) tmem_ld32(taddr, v);
@@ -874,13 +894,15 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
       // lane and key row into the maps' 128-byte swizzle, where stores to
       // global memory from one key row per lane took 32 cache lines per
       // instruction and, with the RoPE table loads, held up the dQ warps'
-      // last drain on the shared load/store path. The row's table entries
-      // are requested first; 16 columns per TMEM load keep them and the
-      // accumulator values within the register budget.
+      // last drain on the shared load/store path. A key tile in one document
+      // reads consecutive table rows: they come in by TMA while dV is staged
+      // (other tiles load this row's entries directly). 16 columns per TMEM
+      // load keep the table entries and the accumulator values within the
+      // register budget.
       constexpr int HC = 16;
       static_assert(DC % HC == 0, "16-column pieces");
       float4 rcos[DC / 8], rsin[DC / 8];
-      if (p.rope_cos) {
+      if (p.rope_cos && !tab_tma) {
         const float4* c4 = reinterpret_cast<const float4*>(p.rope_cos + (size_t)pos * (D / 2) + (dc0 >> 1));
         const float4* s4 = reinterpret_cast<const float4*>(p.rope_sin + (size_t)pos * (D / 2) + (dc0 >> 1));
 #pragma unroll
@@ -905,6 +927,19 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
               pack_bf16(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
               pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
               pack_bf16(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
+      }
+      if (tab_tma) {
+        // this row's entries from the swizzled table boxes (4 floats per
+        // 16-byte chunk, 32 per 128-byte box row); a wait that gives up has
+        // raised the abort flag, and the results are not used then
+        mbar_wait(bar(L::bTab), 0, abort_flag);
+#pragma unroll
+        for (int q = 0; q < DC / 8; ++q) {
+          const int fc = (dc0 >> 1) + 4 * q;  // first float of the chunk
+          const uint32_t off = (uint32_t)((fc >> 5) * (128 * 128)) + sw128(r, (fc & 31) >> 2);
+          rcos[q] = *reinterpret_cast<const float4*>(sg + L::kV + off);
+          rsin[q] = *reinterpret_cast<const float4*>(sg + L::kDO + off);
+        }
       }
 #pragma unroll
       for (int c = 0; c < DC / HC; ++c) {
