@@ -839,14 +839,21 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
     ok = ok && phase_dS(0);
     for (int it = 1; ok && it < n_it; ++it) ok = phase_P(it) && phase_dS(it);
     // ---- epilogue: dK = R^T (scale * dK_r), dV ----
-    const bool epi = ok && mbar_wait(bar(L::bFinal), 0, abort_flag);
+    // Once dV of the last tile is done, V, the dO stages and the Q stage that
+    // does not hold the last Q tile are unread (dK and dQ of the last tile
+    // may still run): the RoPE table rows come in and dV is staged then.
+    const bool dv_fin = ok && mbar_wait(bar(L::bDVDone), (n_it - 1) & 1, abort_flag);
+    const uint32_t off_dv = L::kQ + (n_it & 1) * L::kTileBytes;        // free from here on
+    const uint32_t off_dk = L::kQ + ((n_it - 1) & 1) * L::kTileBytes;  // free after the last dK
     // one document over the whole key tile (uniform across the CTA): its
     // table rows are consecutive from pos0
     const int jl = min(j0 + 127, T - 1);
     const int ds0 = p.doc_start ? min(max(p.doc_start[row0 + j0] - row0, 0), j0) : 0;
     const bool tab_tma = p.rope_cos != nullptr && p.n_split <= 1 &&
                          (!p.doc_start || min(max(p.doc_start[row0 + jl] - row0, 0), jl) == ds0);
-    if (tab_tma && warp == 0 && lane == 0 && epi) {
+    constexpr int HC = 16;  // columns per TMEM load in the staged epilogue
+    static_assert(DC % HC == 0, "16-column pieces");
+    if (tab_tma && warp == 0 && lane == 0 && dv_fin) {
       mbar_arrive_expect_tx(bar(L::bTab), 2 * L::kTabBytes);
 #pragma unroll
       for (int bx = 0; bx < D / 64; ++bx) {
@@ -854,6 +861,25 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
         tma_load_3d(sb0 + L::kDO + bx * (128 * 128), &tmRS, bar(L::bTab), 32 * bx, j0 - ds0, 0);
       }
     }
+    if (dv_fin && p.n_split <= 1) {
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < DC / HC; ++c) {
+        const int col = dc0 + HC * c;
+        uint32_t v[HC];
+        tmem_ld16(tmem + lane_base + L::kColDV + col, v);
+        tmem_wait_ld();
+        uint8_t* blk = sg + off_dv + (col >> 6) * L::kBlockBytes;
+#pragma unroll
+        for (int e = 0; e < HC / 8; ++e)
+          *reinterpret_cast<uint4*>(blk + sw128(r, ((col & 63) >> 3) + e)) = make_uint4(
+              pack_bf16(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
+              pack_bf16(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
+              pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
+              pack_bf16(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
+      }
+    }
+    const bool epi = dv_fin && mbar_wait(bar(L::bFinal), 0, abort_flag);
     if (epi) {
       tc_fence_after();
       const int jj = min(j, T - 1);
@@ -889,18 +915,15 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
           }
         }
       } else {
-      // dK and dV leave as bf16 through the two Q stages (free once the last
-      // dK product has read its Q tile) and TMA stores: one 16-byte chunk per
-      // lane and key row into the maps' 128-byte swizzle, where stores to
-      // global memory from one key row per lane took 32 cache lines per
-      // instruction and, with the RoPE table loads, held up the dQ warps'
-      // last drain on the shared load/store path. A key tile in one document
-      // reads consecutive table rows: they come in by TMA while dV is staged
-      // (other tiles load this row's entries directly). 16 columns per TMEM
-      // load keep the table entries and the accumulator values within the
-      // register budget.
-      constexpr int HC = 16;
-      static_assert(DC % HC == 0, "16-column pieces");
+      // dK and dV leave as bf16 through the two Q stages and TMA stores: one
+      // 16-byte chunk per lane and key row into the maps' 128-byte swizzle,
+      // where stores to global memory from one key row per lane took 32
+      // cache lines per instruction and, with the RoPE table loads, held up
+      // the dQ warps' last drain on the shared load/store path. A key tile
+      // in one document reads consecutive table rows, which came in by TMA
+      // while dV was staged (other tiles load this row's entries directly).
+      // 16 columns per TMEM load keep the table entries and the accumulator
+      // values within the register budget.
       float4 rcos[DC / 8], rsin[DC / 8];
       if (p.rope_cos && !tab_tma) {
         const float4* c4 = reinterpret_cast<const float4*>(p.rope_cos + (size_t)pos * (D / 2) + (dc0 >> 1));
@@ -910,23 +933,6 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
           rcos[q] = c4[q];
           rsin[q] = s4[q];
         }
-      }
-      uint8_t* stage_dk = sg + L::kQ;                  // 128 rows x D bf16, 64-column blocks
-      uint8_t* stage_dv = sg + L::kQ + L::kTileBytes;
-#pragma unroll
-      for (int c = 0; c < DC / HC; ++c) {
-        const int col = dc0 + HC * c;
-        uint32_t v[HC];
-        tmem_ld16(tmem + lane_base + L::kColDV + col, v);
-        tmem_wait_ld();
-        uint8_t* blk = stage_dv + (col >> 6) * L::kBlockBytes;
-#pragma unroll
-        for (int e = 0; e < HC / 8; ++e)
-          *reinterpret_cast<uint4*>(blk + sw128(r, ((col & 63) >> 3) + e)) = make_uint4(
-              pack_bf16(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
-              pack_bf16(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
-              pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
-              pack_bf16(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
       }
       if (tab_tma) {
         // this row's entries from the swizzled table boxes (4 floats per
@@ -965,7 +971,7 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
             }
           }
         }
-        uint8_t* blk = stage_dk + (col >> 6) * L::kBlockBytes;
+        uint8_t* blk = sg + off_dk + (col >> 6) * L::kBlockBytes;
 #pragma unroll
         for (int e = 0; e < HC / 8; ++e)
           *reinterpret_cast<uint4*>(blk + sw128(r, ((col & 63) >> 3) + e)) =
@@ -984,8 +990,8 @@ __global__ void __launch_bounds__(Layout<D, kDQ>::kThreads, 1)
       if (warp == 0 && lane == 0 && epi) {
 #pragma unroll
         for (int bcol = 0; bcol < D / 64; ++bcol) {
-          tma_store_3d(&tmDK, sb0 + L::kQ + bcol * L::kBlockBytes, 64 * bcol, j0, bhk);
-          tma_store_3d(&tmDV, sb0 + L::kQ + L::kTileBytes + bcol * L::kBlockBytes, 64 * bcol, j0, bhk);
+          tma_store_3d(&tmDK, sb0 + off_dk + bcol * L::kBlockBytes, 64 * bcol, j0, bhk);
+          tma_store_3d(&tmDV, sb0 + off_dv + bcol * L::kBlockBytes, 64 * bcol, j0, bhk);
         }
         bulk_commit_group();
         bulk_wait_group_read0();
