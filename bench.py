@@ -45,10 +45,10 @@ FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # one ncu capture of the kernel on the workload, valid only while the kernel
 # sources still hash to what was captured (sha256, first 16 hex digits).
 MEASURED_TRAFFIC = {
-    ("dkdv", "long_context_8k"): (680.4e6, {"bwd_sm100.cuh": "bc038325f3265979",
+    ("dkdv", "long_context_8k"): (687.5e6, {"bwd_sm100.cuh": "a35a3b88219ce0fa",
                                             "sm100.cuh": "d00797b7a9dd3426",
                                             "common.cuh": "36b3720cacd61ee7"}),
-    ("dkdv", "decoder237m_layer"): (124.0e6, {"bwd_sm100.cuh": "bc038325f3265979",
+    ("dkdv", "decoder237m_layer"): (124.5e6, {"bwd_sm100.cuh": "a35a3b88219ce0fa",
                                               "sm100.cuh": "d00797b7a9dd3426",
                                               "common.cuh": "36b3720cacd61ee7"}),
     ("fwd", "long_context_8k"): (157.7e6, {"fwd_sm100.cuh": "1342fca937c6151e",
