@@ -54,17 +54,22 @@ def _set_cu(w, cu):
 
 
 @pytest.mark.parametrize("cu_kind", ["tile_boundaries", "length_one_docs"])
-def test_document_edges(cu_kind):
+@pytest.mark.parametrize("D", [64, 128])
+def test_document_edges(cu_kind, D):
+    """Documents on 128-row tile boundaries (every key tile inside one
+    document that starts at or before it: the backward's epilogue takes the
+    RoPE table rows of such a tile in one block) and documents that cut
+    through tiles (per-row table entries), at both head sizes."""
     _cuda()
     T = 384
-    w = make_workload(config_by_name("packed_docs"), B=2, H=2, T=T, varlen=False, seed=21)
+    w = make_workload(config_by_name("packed_docs"), B=2, H=2, T=T, D=D, varlen=False, seed=21)
     if cu_kind == "tile_boundaries":
         cu = [0, 128, 256, 384, 384 + 1, 384 + 128, 384 + 255, 768]
     else:
         cu = [0, 1, 2, 3, 130, 131, 384, 385, 386, 700, 767, 768]
     _set_cu(w, cu)
     errs = compare(w, gpu_outputs(w), oracle_outputs(w))
-    print(cu_kind, errs)
+    print(cu_kind, D, errs)
 
 
 FULL = [("tiny_fp32", None), ("gpt12m_layer", [(0, 0), (15, 5)]),
