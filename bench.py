@@ -45,16 +45,16 @@ FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # one ncu capture of the kernel on the workload, valid only while the kernel
 # sources still hash to what was captured (sha256, first 16 hex digits).
 MEASURED_TRAFFIC = {
-    ("dkdv", "long_context_8k"): (687.5e6, {"bwd_sm100.cuh": "a35a3b88219ce0fa",
+    ("dkdv", "long_context_8k"): (687.5e6, {"bwd_sm100.cuh": "c69bb6094afca43f",
                                             "sm100.cuh": "d00797b7a9dd3426",
                                             "common.cuh": "36b3720cacd61ee7"}),
-    ("dkdv", "decoder237m_layer"): (124.5e6, {"bwd_sm100.cuh": "a35a3b88219ce0fa",
+    ("dkdv", "decoder237m_layer"): (124.5e6, {"bwd_sm100.cuh": "c69bb6094afca43f",
                                               "sm100.cuh": "d00797b7a9dd3426",
                                               "common.cuh": "36b3720cacd61ee7"}),
-    ("fwd", "long_context_8k"): (157.7e6, {"fwd_sm100.cuh": "1342fca937c6151e",
+    ("fwd", "long_context_8k"): (157.7e6, {"fwd_sm100.cuh": "a1c0ac515047a7cc",
                                            "sm100.cuh": "d00797b7a9dd3426",
                                            "common.cuh": "36b3720cacd61ee7"}),
-    ("fwd", "decoder237m_layer"): (50.4e6, {"fwd_sm100.cuh": "1342fca937c6151e",
+    ("fwd", "decoder237m_layer"): (50.4e6, {"fwd_sm100.cuh": "a1c0ac515047a7cc",
                                             "sm100.cuh": "d00797b7a9dd3426",
                                             "common.cuh": "36b3720cacd61ee7"}),
     ("decode", "decode_8k_gqa"): (200.6e6, {"decode.cuh": "ed672db8f3155da3",

@@ -18,19 +18,23 @@
 // Because P^T lives in shared memory rather than in the S^T columns, S^T of
 // the next query tile is issued as soon as the elementwise warps have read
 // S^T of this one into registers, so the tensor pipe computes it while they
-// form P; the MMA warp issues each product as soon as its inputs are ready
-// rather than in a fixed order. dQ_i is drained by its own warpgroup: read out of TMEM in 32-column
-// chunks, staged through a two-buffer shared ring and added to the fp32 dq
-// accumulator in global memory by TMA bulk reduce-adds, off the elementwise
-// warps' path.
+// form P. The MMA warp issues the products in one fixed order, each group
+// after one wait that has normally completed already (probing readiness
+// instead cost more than it saved). At D = 64 (kPT) TMEM has room for P^T and
+// dQ_i in columns of their own, and dV reads P^T from TMEM. dQ_i is drained
+// by its own warpgroup: read out of TMEM in 32-column chunks, staged through
+// a two-buffer shared ring and added to the fp32 dq accumulator in global
+// memory by TMA bulk reduce-adds, off the elementwise warps' path.
 //
 // Warp roles: four elementwise warpgroups; warpgroup g takes query columns [g*kQC, (g+1)*kQC) of S^T and dP^T and
 // feature columns [g*kDC, (g+1)*kDC) of dK and dV; thread t of a warpgroup
 // owns TMEM lane t (a key row). Then the dQ warpgroup (lane = query row),
 // one TMA warp (K and V once, then Q with lse2 and Delta on the same barrier,
 // and dO) and one MMA warp, which owns TMEM. dK is scaled and rotated back
-// (R^T) in the epilogue; dq is finished by a separate kernel once every key
-// tile has added its part.
+// (R^T) in the epilogue; dK and dV leave as bf16 through shared memory (the
+// Q stages) and TMA stores, and a key tile inside one document takes its
+// RoPE table rows by TMA into stages the last products no longer read. dq is
+// finished by a separate kernel once every key tile has added its part.
 //
 // Operand types. Without RoPE every product reads bf16 (q, k as given, P^T
 // and dS^T rounded to bf16). With RoPE (kF16) the scores are recomputed from

@@ -25,6 +25,9 @@
 //              a commit (or, for a block the tile does not use, an arrive) of
 //              each issuer, so the ring cannot be overrun by either.
 //
+// O / l leaves as bf16 through the tile's Q buffer (no product reads it once
+// O is final) and TMA stores; lse is written per row.
+//
 // Online softmax in log2 units with a lazy rescale: a row's reference max
 // moves (and O, l are rescaled) only when the max grows by more than 8, so P
 // stays <= 2^8 and O is rarely touched; the final O / l and lse = (m +
