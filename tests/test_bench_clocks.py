@@ -90,3 +90,22 @@ def test_missing_nvml_reports_no_clocks(monkeypatch):
     s = c.summary()
     assert s["sm_mhz"] is None and s["samples"] == 0
     assert "no NVML here" in s["error"]
+
+
+def test_traffic_figure_only_while_the_sources_match(monkeypatch):
+    """A captured DRAM-traffic figure is reported only while every source it
+    was captured on still hashes to the recorded digest."""
+    import hashlib
+    import os
+
+    import bench
+
+    path = os.path.join(bench.ROOT, "bwd_causal_sdpa_b200", "csrc", "common.cuh")
+    with open(path, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    table = {("k", "w"): (1.5e6, {"common.cuh": digest}),
+             ("k", "stale"): (2.5e6, {"common.cuh": "0" * 16})}
+    monkeypatch.setattr(bench, "MEASURED_TRAFFIC", table)
+    assert bench.measured_traffic("k", "w") == 1.5e6
+    assert bench.measured_traffic("k", "stale") is None
+    assert bench.measured_traffic("k", "unknown") is None
