@@ -2,7 +2,8 @@
 start-up queries happen on entry, a gated sampler keeps samples only between
 on() and off() (it is entered before the warm-up, so its own start-up never
 falls into the timed steps), throttle reasons are decoded from the mask, and
-a missing NVML reports no clocks rather than guessing."""
+a missing NVML reports no clocks rather than guessing. Also the traffic
+table's rule: a captured figure only while its sources are unchanged."""
 
 import sys
 import threading
