@@ -126,6 +126,11 @@ __global__ void __launch_bounds__(kRopePrepThreads) rope_prep_kernel(
   const __nv_bfloat16* src = (is_k ? k : q) + (size_t)bh * T * D;
   __half* dst = (is_k ? ko : qo) + (size_t)bh * T * D;
   const int c8 = threadIdx.x % CH;  // this thread's chunk column, rows threadIdx.x / CH + u * NT / CH
+  // At D = 64 the tile waits for its factor in shared memory, not in
+  // registers: more blocks per SM (rope_prep 0.0224 -> 0.0214 ms on the 237M
+  // layer, same box); at D = 128 the register version measured faster.
+  constexpr bool kStage = D == 64;
+  __shared__ uint4 tile_s[kStage ? 128 * CH : 1];
   uint4 raw[PER];
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
@@ -136,6 +141,7 @@ __global__ void __launch_bounds__(kRopePrepThreads) rope_prep_kernel(
   float n2 = 0.f;
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
+    if constexpr (kStage) tile_s[threadIdx.x + u * NT] = raw[u];
     const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -161,7 +167,8 @@ __global__ void __launch_bounds__(kRopePrepThreads) rope_prep_kernel(
     if (t >= T) continue;
     const int pos = t - (doc_start ? doc_start[row0 + t] - row0 : 0);
     float v[8];
-    const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+    const uint4 rw = kStage ? tile_s[threadIdx.x + u * NT] : raw[u];  // this thread's own chunk
+    const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&rw);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       v[2 * e] = __low2float(hv[e]);
