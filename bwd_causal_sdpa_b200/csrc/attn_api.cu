@@ -581,7 +581,7 @@ int fwd_impl(const void* q, const void* k, const void* v, const float* rope_cos,
       ds = (int32_t*)(ws + p.doc_start);
       de = (int32_t*)(ws + p.doc_end);
     }
-    ATTN_LAUNCH(KK_DOC_RANGES, st, pdl_launch(doc_ranges_kernel, 1, 1024, 0, st, cu_seqlens, B, T, ds, de));
+    ATTN_LAUNCH(KK_DOC_RANGES, st, pdl_launch(doc_ranges_kernel, doc_ranges_blocks(B, T), 1024, 0, st, cu_seqlens, B, T, ds, de));
     if (launch_status()) return ATTN_ECUDA;
   }
   if (dtype == ATTN_F32) {
@@ -680,7 +680,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   } else if (cu_seqlens) {
     ds = (int32_t*)(ws + p.doc_start);
     de = (int32_t*)(ws + p.doc_end);
-    ATTN_LAUNCH(KK_DOC_RANGES, st, pdl_launch(doc_ranges_kernel, 1, 1024, 0, st, cu_seqlens, B, T, ds, de));
+    ATTN_LAUNCH(KK_DOC_RANGES, st, pdl_launch(doc_ranges_kernel, doc_ranges_blocks(B, T), 1024, 0, st, cu_seqlens, B, T, ds, de));
     if (launch_status()) return ATTN_ECUDA;
   }
   float* delta = (float*)(ws + p.delta);
@@ -1054,7 +1054,7 @@ extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, con
     // doc_ranges_kernel writes every entry of both arrays.
     ds = (int32_t*)(ws + p.doc_start);
     de = (int32_t*)(ws + p.doc_end);
-    ATTN_LAUNCH(KK_DOC_RANGES, st, pdl_launch(doc_ranges_kernel, 1, 1024, 0, st, cu_seqlens, B, T, ds, de));
+    ATTN_LAUNCH(KK_DOC_RANGES, st, pdl_launch(doc_ranges_kernel, doc_ranges_blocks(B, T), 1024, 0, st, cu_seqlens, B, T, ds, de));
     if (launch_status()) return ATTN_ECUDA;
   }
   // delta_kernel writes every row of Delta before the two passes read it.

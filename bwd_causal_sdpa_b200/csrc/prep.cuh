@@ -6,15 +6,23 @@
 
 // From cu_seqlens (over the flattened B*T token axis, end marker B*T) build,
 // for every token, the flattened index where its document starts and where it
-// ends (exclusive). One block: thread 0 walks the array up to the end marker
-// (never past it), validates it and copies up to kDocRangesSmem + 1
-// boundaries into shared memory; then all threads fill the per-token arrays
-// by binary search over that copy (over the global array when it has more
-// documents). A malformed array sets ATTN_EDEVICE_INPUT and the arrays fall
-// back to "each row is one document", so later kernels stay in bounds.
+// ends (exclusive). In every block thread 0 walks the array up to the end
+// marker (never past it), validates it and copies up to kDocRangesSmem + 1
+// boundaries into shared memory (the blocks reach the same verdict); then
+// the block's threads fill their grid-stride share of the per-token arrays by
+// binary search over that copy (over the global array when it has more
+// documents). A malformed array sets ATTN_EDEVICE_INPUT (block 0) and the
+// arrays fall back to "each row is one document", so later kernels stay in
+// bounds. Any grid size is correct; doc_ranges_blocks gives the one used.
 // (Cort33x, "Preserving context in the data": documents packed into one
 // window; attention stays within a document.)
 constexpr int kDocRangesSmem = 4096;
+// one block per 2048 tokens, at most 64 (the walk is repeated per block)
+inline unsigned doc_ranges_blocks(int B, int T) {
+  const long bt = (long)B * T;
+  const long g = (bt + 2047) / 2048;
+  return (unsigned)(g < 1 ? 1 : (g > 64 ? 64 : g));
+}
 
 __global__ void __launch_bounds__(1024) doc_ranges_kernel(const int32_t* __restrict__ cu, int B, int T,
                                                           int32_t* __restrict__ doc_start,
@@ -46,7 +54,7 @@ __global__ void __launch_bounds__(1024) doc_ranges_kernel(const int32_t* __restr
   if (s_ok) {
     const int n = s_n;
     const int32_t* bounds = n <= kDocRangesSmem ? s_cu : cu;
-    for (int t = threadIdx.x; t < BT; t += blockDim.x) {
+    for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < BT; t += gridDim.x * blockDim.x) {
       int lo = 0, hi = n;  // bounds[lo] <= t < bounds[hi]
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -56,8 +64,8 @@ __global__ void __launch_bounds__(1024) doc_ranges_kernel(const int32_t* __restr
       doc_end[t] = bounds[hi];
     }
   } else {
-    if (threadIdx.x == 0) report_status(ATTN_EDEVICE_INPUT);
-    for (int t = threadIdx.x; t < BT; t += blockDim.x) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) report_status(ATTN_EDEVICE_INPUT);
+    for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < BT; t += gridDim.x * blockDim.x) {
       doc_start[t] = (t / T) * T;
       doc_end[t] = (t / T) * T + T;
     }

@@ -187,7 +187,7 @@ int doc_positions(const int32_t* cu, int B, int T, char* ws, const ProjWs& w, cu
   *ds = nullptr;
   if (!cu) return ATTN_OK;
   int32_t* s = (int32_t*)(ws + w.doc_start);
-  ATTN_LAUNCH(KK_DOC_RANGES, st, pdl_launch(doc_ranges_kernel, 1, 1024, 0, st, cu, B, T, s,
+  ATTN_LAUNCH(KK_DOC_RANGES, st, pdl_launch(doc_ranges_kernel, doc_ranges_blocks(B, T), 1024, 0, st, cu, B, T, s,
                                             (int32_t*)(ws + w.doc_end)));
   *ds = s;
   return launch_status();
